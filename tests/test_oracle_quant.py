@@ -1,0 +1,176 @@
+"""Pins for the oracle's offline quantisation, bit planes, dequant and blob
+format.  Sources: ExactMoE (W4A16 weights), D2MoE (MWQ nested planes,
+offline quantisation).  Every expected value here is either worked out by
+hand (see tests/golden/quant_worked_examples.txt), a closed form, or an
+invariant that a wrong sign, index or dropped term would break."""
+import os
+
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_groups():
+    cases = []
+    with open(os.path.join(GOLDEN, "quant_worked_examples.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            w, s, z, q = line.split("|")
+            cases.append((np.array([float(v) for v in w.split()], np.float32), float(s), float(z),
+                          np.array([int(v) for v in q.split()], np.uint8)))
+    return cases
+
+
+@pytest.mark.parametrize("case", range(len(_golden_groups())))
+def test_worked_examples(case):
+    w, s, z, q = _golden_groups()[case]
+    qq, ss, zz = O.quantize_groups(w[None, :], w.size)
+    assert ss[0, 0] == np.float32(s)
+    assert zz[0, 0] == np.float32(z)
+    np.testing.assert_array_equal(qq[0], q)
+
+
+def test_closed_form_uniform_grid():
+    # w_i = (i - z) * s with s a power of two: the codes must be exactly i.
+    rng = np.random.default_rng(1)
+    for z in range(16):
+        for e in (-9, -6, -3):
+            s = 2.0 ** e
+            w = ((np.arange(16) - z) * s).astype(np.float32)
+            perm = rng.permutation(16)
+            q, ss, zz = O.quantize_groups(w[perm][None, :], 16)
+            lo, hi = min(w.min(), 0), max(w.max(), 0)
+            if hi - lo != 15 * s:  # range extended by 0 only when z is 0 or 15
+                continue
+            assert ss[0, 0] == s and zz[0, 0] == z
+            np.testing.assert_array_equal(q[0], np.arange(16)[perm])
+
+
+def test_zero_group_and_zero_point_range():
+    q, s, z = O.quantize_groups(np.zeros((2, 64), np.float32), 64)
+    assert (s == 1).all() and (z == 0).all() and (q == 0).all()
+    rng = np.random.default_rng(2)
+    w = rng.normal(0, 0.02, (64, 256)).astype(np.float32)
+    q, s, z = O.quantize_groups(w, 64)
+    assert q.max() <= 15 and z.min() >= 0 and z.max() <= 15
+    # scale is a bf16 value
+    np.testing.assert_array_equal(O.bf16_round(s), s)
+
+
+def test_error_bound():
+    rng = np.random.default_rng(3)
+    for dist in ("normal", "uniform", "skewed"):
+        if dist == "normal":
+            w = rng.normal(0, 0.02, (128, 512))
+        elif dist == "uniform":
+            w = rng.uniform(-1, 1, (128, 512))
+        else:
+            w = rng.exponential(0.05, (128, 512))
+        w = w.astype(np.float32)
+        for g in (64, 128):
+            q, s, z = O.quantize_groups(w, g)
+            wd = O.dequant(q, s, z, g)
+            sE = np.repeat(s, g, axis=1).astype(np.float64)
+            zE = np.repeat(z, g, axis=1).astype(np.float64)
+            err = np.abs(w.astype(np.float64) - wd)
+            assert (err <= 1.1 * sE).all()
+            raw = np.rint(w / np.repeat(s, g, axis=1)) + zE
+            interior = (raw >= 0) & (raw <= 15)
+            assert interior.mean() > 0.99
+            bound = 0.5 * sE + 2.0 ** -23 * np.abs(w)
+            assert (err[interior] <= bound[interior]).all()
+
+
+def test_pack_int4_hand_values():
+    q = np.array([[1, 2, 3, 4, 5, 6, 7, 8, 15, 0, 0, 0, 0, 0, 0, 10]], np.uint8)
+    words = O.pack_int4(q)
+    assert words.tolist() == [[0x87654321, 0xA000000F]]
+    np.testing.assert_array_equal(O.unpack_int4(words, 16), q)
+
+
+def test_planes_hand_values():
+    q = np.zeros((1, 32), np.uint8)
+    Q2, D3, D4 = O.split_planes(q + 15)
+    assert Q2.tolist() == [[0xFFFFFFFF, 0xFFFFFFFF]] and D3.tolist() == [[0xFFFFFFFF]]
+    assert D4.tolist() == [[0xFFFFFFFF]]
+    q[0, 0] = 1      # only the lowest residual bit of element 0
+    q[0, 1] = 4      # base field of element 1 = 1  -> bits 2..3 of Q2 word 0
+    q[0, 31] = 8     # base field of element 31 = 2 -> bits 30..31 of Q2 word 1
+    q[0, 5] = 2      # middle residual of element 5 -> bit 5 of D3
+    Q2, D3, D4 = O.split_planes(q)
+    assert Q2.tolist() == [[0x00000004, 0x80000000]]
+    assert D3.tolist() == [[0x00000020]]
+    assert D4.tolist() == [[0x00000001]]
+
+
+def test_planes_nesting():
+    rng = np.random.default_rng(4)
+    q = rng.integers(0, 16, (8, 256)).astype(np.uint8)
+    Q2, D3, D4 = O.split_planes(q)
+    # W(4) = Q2 + D3 + D4 reproduces the 4-bit code (D2MoE, MWQ)
+    np.testing.assert_array_equal(O.join_planes(Q2, D3, D4, 256, 4), q)
+    # INT2 within INT3 within INT4: the b-bit code is the top b bits
+    np.testing.assert_array_equal(O.join_planes(Q2, D3, D4, 256, 3), q & 0b1110)
+    np.testing.assert_array_equal(O.join_planes(Q2, D3, D4, 256, 2), q & 0b1100)
+    # 4 * Q2 + 2 * D3 + D4 == q element-wise
+    b2 = O.join_planes(Q2, D3, D4, 256, 2).astype(int)
+    b3 = O.join_planes(Q2, D3, D4, 256, 3).astype(int)
+    assert ((b3 - b2) // 2 <= 1).all() and ((q.astype(int) - b3) <= 1).all()
+
+
+def test_nested_dequant_hand_values():
+    # q = 13 = 0b1101, z = 3, s = 0.5: b=2 keeps 12 -> 4.5, b=3 keeps 12 -> 4.5,
+    # b=4 keeps 13 -> 5.0
+    q = np.full((1, 64), 13, np.uint8)
+    s = np.array([[0.5]], np.float32)
+    z = np.array([[3.0]], np.float32)
+    assert O.dequant(q, s, z, 64, 2)[0, 0] == 4.5
+    assert O.dequant(q, s, z, 64, 3)[0, 0] == 4.5
+    assert O.dequant(q, s, z, 64, 4)[0, 0] == 5.0
+
+
+def test_bf16_rounding_hand_values():
+    vals = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9, -2.5, 1.0 + 2 ** -7 + 2 ** -8], np.float32)
+    # ties go to even: 1+2^-8 -> 1.0 ; 1+3*2^-9 -> 1+2^-7 ; 1+2^-7+2^-8 -> 1+2^-6
+    exp = [0x3F80, 0x3F80, 0x3F81, 0xC020, 0x3F82]
+    assert O.f32_to_bf16_bits(vals).tolist() == exp
+
+
+def test_blob_layout_sizes_and_roundtrip():
+    # olmoe-shaped expert, INT4 g128: 3*F*d/2 code bytes + 3 * F*d/128 * 4 sz bytes
+    assert O.blob_layout(2048, 1024, 128, "int4")["bytes"] == 3342336
+    # nested shape at b=4 reads the same bytes as INT4
+    assert O.blob_layout(4096, 1024, 128, "planes")["bytes"] == O.blob_layout(4096, 1024, 128, "int4")["bytes"]
+    rng = np.random.default_rng(5)
+    d, F, g = 256, 384, 64
+    wg, wu = rng.normal(0, .02, (2, F, d)).astype(np.float32)
+    wd = rng.normal(0, .02, (d, F)).astype(np.float32)
+    for layout in ("int4", "planes"):
+        off = O.blob_layout(d, F, g, layout)
+        blob = O.build_blob(wg, wu, wd, g, layout)
+        assert blob.size == off["bytes"]
+        for m, w in (("gate", wg), ("up", wu), ("down", wd)):
+            N, K = w.shape
+            q, s, z = O.quantize_groups(w, g)
+            if layout == "int4":
+                o = off[m + ".codes"]
+                words = blob[o:o + N * K // 2].view(np.uint32).reshape(N, K // 8)
+                np.testing.assert_array_equal(O.unpack_int4(words, K), q)
+            else:
+                Q2 = blob[off[m + ".q2"]:off[m + ".q2"] + N * K // 4].view(np.uint32).reshape(N, K // 16)
+                D3 = blob[off[m + ".d3"]:off[m + ".d3"] + N * K // 8].view(np.uint32).reshape(N, K // 32)
+                D4 = blob[off[m + ".d4"]:off[m + ".d4"] + N * K // 8].view(np.uint32).reshape(N, K // 32)
+                np.testing.assert_array_equal(O.join_planes(Q2, D3, D4, K), q)
+            o = off[m + ".sz"]
+            sz = blob[o:o + N * (K // g) * 4].view(np.uint32)
+            G = K // g
+            for n in (0, 1, 127, 128, N - 1):
+                for c in range(G):
+                    word = int(sz[((n // 128) * G + c) * 128 + n % 128])
+                    assert O.bf16_bits_to_f32(np.array([word & 0xFFFF]))[0] == s[n, c]
+                    assert O.bf16_bits_to_f32(np.array([word >> 16]))[0] == z[n, c]
