@@ -1,0 +1,383 @@
+"""Benchmark: MoE-layer tokens/s of the W4A16 quantised MoE layer on B200.
+
+One step = one pass of the whole hot path over one batch: moe_route_topk ->
+moe_permute (histogram, scan, permutation, gather) -> moe_grouped_ffn_wq
+(dequant-fused gate/up + SwiGLU, then down) -> moe_unpermute_combine.
+Default workload: the OLMoE-shaped layer (d=2048, E=64, top-8, d_ff=1024,
+INT4 g128, Zipf-skewed router bias) at T=4096 tokens.  Synthetic seeded
+inputs and random weights; R distinct layer instances are rotated so the
+expert weights streamed per step are not L2-resident.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs an
+independent replica on its own token batch (the layer has no exchange step
+in this data-parallel form); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s (W4A16)"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="olmoe")
+    p.add_argument("--tokens", type=int, default=4096)
+    p.add_argument("--instances", type=int, default=4, help="distinct layer instances rotated per step")
+    p.add_argument("--sweep", default="1,16,256", help="extra token counts timed for context ('' = none)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-tokens", type=int, default=0)
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ util --
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], tc=p["bf16_tflops"], tc_sust=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    src="measured")
+    return dict(hbm=6650.0, tc=1590.0, tc_sust=1400.0, src="fallback")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# -------------------------------------------------------------- workload --
+
+def make_instances(shape, T, R, seed, device):
+    """R layer instances with weights drawn and packed on the device."""
+    import torch
+    from quantized_moe_expert_histogram_b200 import inputs as I
+    from quantized_moe_expert_histogram_b200.layer import QuantMoELayer
+    layers = []
+    for r in range(R):
+        L = I.make_layer(shape, T, seed=seed + 1000 * r, device=device)
+        layer = QuantMoELayer.from_weights(shape, L["w_router"], L["bias"], L["w_gate"], L["w_up"],
+                                           L["w_down"], max_tokens=T)
+        del L["w_gate"], L["w_up"], L["w_down"]
+        torch.cuda.empty_cache()
+        layers.append((layer, L["x"], L.get("bits")))
+    return layers
+
+
+def algorithmic(shape, T, layer, bits_present):
+    """Algorithmic bytes and flops of one layer pass from the routing taken."""
+    from quantized_moe_expert_histogram_b200 import moeq
+    counts = layer.views(T)["counts"].cpu().tolist()
+    d, F, g = shape.d, shape.F, shape.group
+    code_full = 3 * d * F // 2
+    sz = 3 * d * F // g * 4
+    bytes_w = 0
+    if not bits_present:
+        bytes_w = sum(1 for c in counts if c > 0) * (code_full + sz)
+    else:
+        for e in range(shape.E):
+            bs = [2 + j for j in range(3) if counts[3 * e + j] > 0]
+            if bs:
+                bytes_w += code_full * max(bs) // 4 + sz
+    act = 2 * T * d * 2  # x in, y out (bf16)
+    flops = 6 * d * F * T * shape.k
+    return bytes_w + act, flops
+
+
+def time_steps(layers, steps, warmup, stream, ffn_events=True):
+    """Run warmup + timed steps; returns (total ms, mean FFN ms per step)."""
+    import torch
+    R = len(layers)
+    for i in range(warmup):
+        layer, x, bits = layers[i % R]
+        layer.forward(x, bits=bits, stream=stream)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    fs = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    fe = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    from quantized_moe_expert_histogram_b200 import moeq
+    start.record(stream)
+    for i in range(steps):
+        layer, x, bits = layers[i % R]
+        T = x.shape[0]
+        v = layer.views(T)
+        moeq.moe_route_topk(x, layer.w_router, layer.bias, layer.k, topk_idx=v["topk_idx"],
+                            topk_w=v["topk_w"], stream=stream)
+        moeq.moe_permute(v["topk_idx"], layer.E, bits=bits, x=x, out=v, status=v["status"], stream=stream)
+        fs[i].record(stream)
+        moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, T, layer.E, layer.d, layer.F,
+                                layer.group, layer.layout, workspace=v["workspace"], y_perm=v["y_perm"],
+                                status=v["status"], stream=stream)
+        fe[i].record(stream)
+        moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], y=v["y"], stream=stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    total = start.elapsed_time(end)
+    ffn = sum(a.elapsed_time(b) for a, b in zip(fs, fe)) / steps
+    return total, ffn
+
+
+def time_e2e(layers, steps, stream):
+    """Same steps through the public layer call with pinned host buffers:
+    H2D of x and D2H of y inside the timed region."""
+    import torch
+    R = len(layers)
+    T, d = layers[0][1].shape
+    hx = [layers[r][1].cpu().pin_memory() for r in range(R)]
+    hy = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    hb = [layers[r][2].cpu().pin_memory() if layers[r][2] is not None else None for r in range(R)]
+    db = torch.empty_like(layers[0][2]) if layers[0][2] is not None else None
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    h2d = T * d * 2 + (hb[0].numel() if hb[0] is not None else 0)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(steps):
+            layer = layers[i % R][0]
+            dx.copy_(hx[i % R], non_blocking=True)
+            if db is not None:
+                db.copy_(hb[i % R], non_blocking=True)
+            y = layer.forward(dx, bits=db, stream=stream)
+            hy.copy_(y, non_blocking=True)
+        end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end), h2d, T * d * 2
+
+
+def cpu_baseline(shape, T, seed, sample_tokens, budget_s=20.0):
+    """The oracle as it stands, on the host cores, on a bounded token sample."""
+    import numpy as np
+    import torch
+    from oracle import moe_oracle as O
+    from quantized_moe_expert_histogram_b200 import inputs as I
+    L = I.make_layer(shape, T, seed=seed, device="cpu")
+    x = L["x"].float().numpy()
+    bias = L["bias"].numpy() if L["bias"] is not None else None
+    bits = L["bits"].numpy() if "bits" in L else None
+    ex = O.QuantExperts(L["w_gate"].numpy(), L["w_up"].numpy(), L["w_down"].numpy(), shape.group)
+    n = sample_tokens or min(T, 64)
+    sub = np.arange(n)
+    # offline quantisation of the experts the sample needs is not part of a step
+    out = O.moe_layer(x, L["w_router"].numpy(), bias, shape.k, ex, bits=bits, token_subset=sub[:1])
+    need = set(out["sel"][:n].reshape(-1).tolist())
+    for e in need:
+        ex.quant(int(e))
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        O.moe_layer(x[:n], L["w_router"].numpy(), bias, shape.k, ex,
+                    bits=None if bits is None else bits[:n])
+        reps += 1
+        if time.perf_counter() - t0 > budget_s or reps >= 3:
+            break
+    dt = time.perf_counter() - t0
+    cores = os.cpu_count()
+    return {"value": n * reps / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of the {T} tokens (route, permute, FFN, combine of the sample), x{reps}, "
+                      f"fp64 numpy oracle; expert quantisation done beforehand"}
+
+
+# ------------------------------------------------------------------ main --
+
+def run_reference(args):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    from quantized_moe_expert_histogram_b200 import inputs as I
+    shape = I.SHAPES[args.workload]
+    T = args.tokens
+    per_step = []
+    cb = None
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(shape, T, 0, args.cpu_sample_tokens or 32, budget_s=0.0)
+        if i >= args.warmup:
+            per_step.append(cb["value"])
+    v = statistics.mean(per_step)
+    cb["value"] = v
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{shape.name} MoE layer d={shape.d} E={shape.E} top-{shape.k} "
+                                   f"d_ff={shape.F} INT4 g{shape.group}", "tokens": T},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    from quantized_moe_expert_histogram_b200 import build as B
+    from quantized_moe_expert_histogram_b200 import inputs as I
+    from quantized_moe_expert_histogram_b200 import moeq
+    B.build()
+    world, rank, local = dist_setup(args)
+    moeq.load()
+    shape = I.SHAPES[args.workload]
+    T = args.tokens
+    peaks = load_peaks()
+    stream = torch.cuda.Stream()
+    layers = make_instances(shape, T, args.instances, seed=rank * 7919, device="cuda")
+    torch.cuda.synchronize()
+
+    barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    torch.cuda.synchronize()
+    total_ms, ffn_ms = time_steps(layers, args.steps, args.warmup, stream)
+    clk = clocks.stop()
+    barrier(world)
+    total_ms = max_over_ranks(world, total_ms)
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+
+    bytes_alg, flops = algorithmic(shape, T, layers[(args.steps - 1) % len(layers)][0],
+                                   layers[0][2] is not None)
+    t_ffn = ffn_ms / 1e3
+    tc_bound = flops / (peaks["tc"] * 1e12) > bytes_alg / (peaks["hbm"] * 1e9)
+    if tc_bound:
+        peak = peaks["tc_sust"] if total_ms > 1000 else peaks["tc"]
+        ach = flops / t_ffn / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak}
+    else:
+        ach = bytes_alg / t_ffn / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s", "frac": ach / peaks["hbm"]}
+    roof.update({"traffic": None, "kernel": "moe_grouped_ffn_wq (gate/up + down launches)",
+                 "peak_source": peaks["src"], "ffn_ms": ffn_ms,
+                 "per_launch_units": f"{T * shape.k} assignments"})
+
+    e2e_ms, h2d, d2h = time_e2e(layers, args.steps, stream)
+    e2e_ms = max_over_ranks(world, e2e_ms)
+    e2e = {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    sweep = {}
+    for tok in [int(s) for s in args.sweep.split(",") if s.strip()]:
+        ls = make_instances(shape, tok, 16, seed=rank * 7919 + 17, device="cuda")
+        tot, fm = time_steps(ls, max(args.steps, 50), args.warmup, stream)
+        b, fl = algorithmic(shape, tok, ls[-1][0], ls[0][2] is not None)
+        sweep[str(tok)] = {"tokens_per_s": tok * max(args.steps, 50) / (tot / 1e3),
+                           "ms_per_step": tot / max(args.steps, 50), "ffn_ms": fm,
+                           "ffn_hbm_frac": b / (fm / 1e3) / 1e9 / peaks["hbm"],
+                           "ffn_tc_frac": fl / (fm / 1e3) / 1e12 / peaks["tc"]}
+        del ls
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(shape, T, 0, args.cpu_sample_tokens)
+
+    launches_per_step = 6
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+            "config": {"workload": f"{shape.name} MoE layer d={shape.d} E={shape.E} top-{shape.k} "
+                                   f"d_ff={shape.F} INT4 g{shape.group}", "tokens": T,
+                       "global_batch": T * world, "parallelism": f"replicas x{world}",
+                       "l2": f"{args.instances} layer instances rotated ({shape.E} experts x "
+                             f"{moeq.moe_blob_bytes(shape.d, shape.F, shape.group, 0)} B each), inputs > L2"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk, "sweep": sweep}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,243 @@
+/*
+ * moeq.h -- C ABI of a B200 (sm_100a) library for one token-routed
+ * mixture-of-experts FFN layer whose expert weights are stored low-bit.
+ *
+ * The layer, in the order the calls below run it:
+ *   route (softmax top-k)  ->  per-expert histogram, prefix sum and
+ *   permutation  ->  per-expert SwiGLU FFN with the dequantisation fused in
+ *   (gate/up, then down)  ->  weighted unpermute-combine,
+ * plus an offline packer and an offload mode with a GPU slot cache.
+ *
+ * Sources (page title, section):
+ *   [ExactMoE] "Every Expert Counts: ExactMoE for Memory-Efficient W4A16
+ *              Inference": four-bit expert weights with 16-bit activations;
+ *              the router's decisions are executed exactly and every chosen
+ *              expert runs; compressed experts live in host memory and are
+ *              moved into a GPU-resident slot cache; grouped execution.
+ *   [D2MoE]    "D2MoE: Dual Routing and Dynamic Scheduling for Efficient
+ *              On-Device MoE-based LLM Serving": Dual Routing (expert gate,
+ *              bit gate), MWQ nested weights W(2)=Q2, W(3)=Q2+D3,
+ *              W(4)=Q2+D3+D4, quantisation done offline, the pipeline
+ *              "I/O -> dequant -> FP16 -> GEMM" and "Load E2 || Compute E1".
+ *   [EdgeMoE]  "EdgeMoE" article: expert weights kept outside device memory
+ *              and loaded on activation into an expert buffer.
+ *   [Read-ME]  "Innovativer Ansatz zur Optimierung der Inferenz von
+ *              Mixture-of-Experts-Modellen": expert-aware batching.
+ *
+ * Conventions for every call:
+ *   - Plain C.  Every pointer is a DEVICE pointer unless its name ends in
+ *     _host.  The caller allocates and owns every buffer; the library keeps
+ *     no pointer after a call returns (except the slot cache object).
+ *   - Streams are passed as `moe_stream_t` (a cudaStream_t; NULL = legacy
+ *     default stream).  Every call is asynchronous on its stream and
+ *     returns after launch-time validation; nothing here synchronises the
+ *     device except where a call says so.
+ *   - Errors: a call returns a moe_status_t; MOE_OK means the work was
+ *     queued.  moe_last_error() gives a message for the calling thread.
+ *     Problems that can only be seen on the device (an expert id out of
+ *     range, an activation outside fp16 range, a bounded wait that ran
+ *     out) are OR-ed into the caller's device word `status` as MOE_DEV_*
+ *     bits; the caller reads it after synchronising.  No call aborts,
+ *     traps or prints.
+ *   - Outputs are fully overwritten and must not alias inputs.
+ *   - bf16 / fp16 buffers are passed as void* and hold IEEE binary16 /
+ *     bfloat16 bit patterns.
+ */
+#ifndef MOEQ_H
+#define MOEQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef void* moe_stream_t; /* cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,       /* null pointer, negative size, k > E ... */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2, /* a size the kernels do not handle      */
+  MOE_ERR_CUDA = 3,              /* a CUDA runtime call failed            */
+  MOE_ERR_OOM = 4,               /* host or device allocation failed      */
+  MOE_ERR_TIMEOUT = 5,           /* reserved for host-side waits          */
+  MOE_ERR_WORKSPACE = 6,         /* workspace smaller than required       */
+  MOE_ERR_FAULT_INJECTED = 7     /* host-side fault injection fired       */
+} moe_status_t;
+
+/* Bits OR-ed into the caller's device status word. */
+#define MOE_DEV_BAD_INDEX 1u   /* expert id or bit-width out of range (clamped) */
+#define MOE_DEV_RANGE 2u       /* activation outside fp16 range             */
+#define MOE_DEV_TIMEOUT 4u     /* a bounded on-device wait gave up          */
+
+typedef enum {
+  MOE_LAYOUT_INT4 = 0,   /* 4-bit codes, 8 per uint32                      */
+  MOE_LAYOUT_PLANES = 1  /* MWQ bit planes Q2 (2 bit) + D3 + D4 (1 bit)    */
+} moe_layout_t;
+
+/* Thread-local message describing the last failure (never NULL). */
+MOE_API const char* moe_last_error(void);
+
+/* ---------------------------------------------------------------------
+ * Weight format ("blob"): one contiguous byte block per expert, so one
+ * copy moves one expert ([ExactMoE] slot cache; [EdgeMoE] expert buffer).
+ * For hidden size d, expert width F (d_ff) and group size g:
+ *   INT4  : gate codes [F][d/8] u32 | up codes [F][d/8] | down codes
+ *           [d][F/8] | gate sz | up sz | down sz
+ *   PLANES: gate Q2 [F][d/16] | gate D3 [F][d/32] | gate D4 [F][d/32] |
+ *           up Q2 | up D3 | up D4 | down Q2 [d][F/16] | down D3 | down D4 |
+ *           gate sz | up sz | down sz
+ * Code word packing: nibble i of a codes word = element 8w+i (low nibble
+ * first); Q2 word bits 2i..2i+1 = element 16w+i; D3/D4 word bit i =
+ * element 32w+i.  sz of an N x K matrix is N*K/g uint32 words, word =
+ * bf16(scale) | bf16(zero) << 16, ordered [N/128][K/g][128] (row tile of
+ * 128, then group, then row inside the tile).  Dequantised weight of a
+ * b-bit read: w = ((code >> (4-b) << (4-b)) - zero) * scale.
+ * Supported: d, F multiples of 128; g in {64, 128}; d % g == F % g == 0.
+ * Returns the blob size in bytes, or 0 for an unsupported shape.
+ * ------------------------------------------------------------------ */
+MOE_API size_t moe_blob_bytes(int d, int F, int group, int layout);
+
+/* moe_quant_pack -- offline quantisation ([D2MoE] quantisation is done
+ * offline; [ExactMoE] W4A16).  w_gate, w_up: fp32 [E][F][d]; w_down: fp32
+ * [E][d][F] (row-major, K contiguous).  Per (row, group of g consecutive
+ * K): mn = min(min w, 0), mx = max(max w, 0), s = bf16((mx-mn)/15) (1 if
+ * 0), z = clamp(rint(-mn/s), 0, 15), code = clamp(rint(w/s)+z, 0, 15), all
+ * IEEE fp32 with round-half-even.  Writes E blobs of moe_blob_bytes()
+ * each into `blobs` (16-byte aligned).  Not on the timed path. */
+MOE_API moe_status_t moe_quant_pack(const float* w_gate, const float* w_up, const float* w_down, int E,
+                            int d, int F, int group, int layout, void* blobs,
+                            moe_stream_t stream);
+
+/* moe_route_topk -- softmax top-k router ([D2MoE] Dual Routing, expert
+ * gate; [ExactMoE] the router decides, nothing is pruned).
+ *   x        bf16 [T][d];  w_router fp32 [E][d];  bias fp32 [E] or NULL
+ *   logits   l[t][e] = sum_i x[t][i] * w_router[e][i] + bias[e], evaluated
+ *            in fp64 (bf16 x fp32 products are exact in fp64)
+ *   topk_idx int32 [T][k]: the k largest logits, ordered by descending
+ *            logit; equal logits go to the lower expert index
+ *   topk_w   fp32 [T][k]: softmax over the k selected logits (the full
+ *            softmax renormalised over the selection)
+ *   forced_idx int32 [T][k] or NULL: when given, the selection is taken
+ *            from it as is (an external trace) and only topk_w is
+ *            computed for it; topk_idx receives a copy.
+ * Requires 1 <= k <= E <= 256, k <= 16, d % 8 == 0. */
+MOE_API moe_status_t moe_route_topk(const void* x, const float* w_router, const float* bias,
+                            const int32_t* forced_idx, int T, int d, int E, int k,
+                            int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
+/* moe_permute -- per-expert histogram, exclusive prefix sum and stable
+ * permutation of the T*k assignments a = t*k + j ([Read-ME] expert-aware
+ * batching; [ExactMoE] grouped execution).  No atomics: per-warp
+ * histograms, one block scan, and a rank-by-warp-match scatter.
+ *   bits uint8 [T][k] or NULL.  NULL: bin of a = topk_idx[a] (nbins = E).
+ *        Given ([D2MoE] bit gate): bin = 3*topk_idx[a] + (bits[a]-2),
+ *        nbins = 3E, bits in {2,3,4}.
+ *   counts  int32 [nbins]; offsets int32 [nbins+1] (offsets[nbins] = T*k)
+ *   perm    int32 [T*k]: perm[p] = a, bins contiguous, ascending a inside
+ *   inv_perm int32 [T*k]: inv_perm[perm[p]] = p
+ *   x (bf16 [T][d]) and x_perm (fp16 [T*k][d]) may both be NULL; when
+ *   given, x_perm[p] = fp16(x[perm[p]/k]) (the activation rows in expert
+ *   order, converted for the fp16 tensor-core operands).
+ * Out-of-range ids/bits are clamped into range and flag MOE_DEV_BAD_INDEX;
+ * |x| > 65504 flags MOE_DEV_RANGE.  Requires T*k <= 2^24, nbins <= 768. */
+MOE_API moe_status_t moe_permute(const int32_t* topk_idx, const uint8_t* bits, const void* x, int T,
+                         int d, int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
+                         int32_t* inv_perm, void* x_perm, int32_t* status, moe_stream_t stream);
+
+/* Workspace bytes moe_grouped_ffn_wq needs for `total_rows` = T*k rows. */
+MOE_API size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int layout);
+
+/* moe_grouped_ffn_wq -- the grouped expert FFN with dequantisation fused
+ * into both GEMMs ([D2MoE] pipeline I/O -> dequant -> FP16 -> GEMM;
+ * [ExactMoE] W4A16, grouped execution).  For every bin (expert e, width b)
+ * and each of its rows p in [offsets[bin], offsets[bin+1]):
+ *     h[p]      = silu(Wg_e,b . x_perm[p]) * (Wu_e,b . x_perm[p])
+ *     y_perm[p] = Wd_e,b . h[p]
+ * with W_e,b the b-bit dequantised weights of the blob format above (b = 4
+ * for MOE_LAYOUT_INT4, b = 2 + bin % 3 for MOE_LAYOUT_PLANES).
+ *   x_perm   fp16 [total_rows][d] (from moe_permute)
+ *   offsets  int32 [nbins+1] (device; never read by the host)
+ *   blobs    device pool of expert blobs, blob i at blobs + i*blob_bytes
+ *   slot_of  int32 [E] or NULL.  NULL: expert e is blob e.  Given: expert
+ *            e is blob slot_of[e]; experts with slot_of[e] < 0 are skipped
+ *            (their y_perm rows are left untouched).
+ *   T        token count (no bin holds more than T rows; selects the
+ *            decode GEMV regime for small T)
+ *   workspace >= moe_ffn_workspace_bytes() bytes of device scratch
+ *   y_perm   fp32 [total_rows][d]
+ * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16. */
+MOE_API moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, const void* blobs,
+                                const int32_t* slot_of, int total_rows, int T, int E, int d,
+                                int F, int group, int layout, void* workspace,
+                                size_t workspace_bytes, float* y_perm, int32_t* status,
+                                moe_stream_t stream);
+
+/* moe_unpermute_combine -- weighted combine ([ExactMoE]: every chosen
+ * expert's output is used as the router weighted it).
+ *   y[t] = bf16( residual[t] + sum_{j<k} topk_w[t][j] * y_perm[inv_perm[t*k+j]] )
+ * summed in fp32 in ascending j; residual bf16 [T][d] or NULL (0).
+ *   y bf16 [T][d]; requires d % 4 == 0. */
+MOE_API moe_status_t moe_unpermute_combine(const float* y_perm, const int32_t* inv_perm,
+                                   const float* topk_w, const void* residual, int T, int k, int d,
+                                   void* y, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------
+ * Offload mode ([ExactMoE] compressed experts in host memory, GPU slot
+ * cache; [EdgeMoE] expert buffer; [D2MoE] "Load E2 || Compute E1").
+ * One cache object per layer: `slots` device slots of one blob each.
+ * ------------------------------------------------------------------ */
+typedef struct moe_slot_cache moe_slot_cache;
+
+/* Create a cache for one layer.  host_blobs: E blobs in PINNED host memory
+ * (cudaHostAlloc / registered), blob e at host_blobs + e*blob_bytes.
+ * device_pool: caller-allocated device memory of slots*blob_bytes bytes.
+ * The cache allocates host bookkeeping, CUDA events and a small device
+ * table; it starts empty.  Requires 2 <= slots and E <= 256. */
+MOE_API moe_status_t moe_slot_cache_create(int E, int slots, size_t blob_bytes, const void* host_blobs,
+                                   void* device_pool, moe_slot_cache** out);
+
+/* Plan one layer-step: ids_host (n_ids expert ids, host memory, repeats
+ * allowed) are the experts the router chose.  Resident experts are hits;
+ * the others are misses, loaded least-recently-used-victim first.  The
+ * distinct experts are split into waves of at most slots/2 (hits first,
+ * then misses by descending row count) so that copies of wave w+1 run on
+ * copy_stream while wave w computes on compute_stream.  Issues the copies
+ * of the first two waves.  *n_waves receives the wave count; stats_host
+ * (may be NULL) receives {hits, misses, bytes_copied}. */
+MOE_API moe_status_t moe_slot_stage(moe_slot_cache* cache, const int32_t* ids_host, int n_ids,
+                            moe_stream_t copy_stream, moe_stream_t compute_stream,
+                            int32_t* n_waves, int64_t* stats_host);
+
+/* Run the staged layer-step: for each wave, compute_stream waits for the
+ * wave's copies, the grouped FFN (same arguments as moe_grouped_ffn_wq)
+ * runs on the wave's experts through the device slot table, and the next
+ * copies that reuse the wave's slots are issued after it.  Every routed
+ * expert is executed; results equal the all-resident call bit for bit. */
+MOE_API moe_status_t moe_slot_ffn(moe_slot_cache* cache, const void* x_perm, const int32_t* offsets,
+                          int total_rows, int T, int d, int F, int group, int layout,
+                          void* workspace, size_t workspace_bytes, float* y_perm,
+                          int32_t* status, moe_stream_t copy_stream, moe_stream_t compute_stream);
+
+/* Free the cache's host bookkeeping, events and device table (not the
+ * caller's pool or host blobs).  Synchronises the events it owns. */
+MOE_API void moe_slot_cache_destroy(moe_slot_cache* cache);
+
+/* Host-side fault injection for tests: the next `count` calls of
+ * moe_slot_stage fail with MOE_ERR_FAULT_INJECTED before queuing any work
+ * (what = 1), or the cache's next copy reports a failed copy (what = 2).
+ * what = 0 clears it. */
+MOE_API void moe_debug_inject_fault(int what, int count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEQ_H */

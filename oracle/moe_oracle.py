@@ -88,7 +88,8 @@ def quantize_groups(w: np.ndarray, group: int):
     mx = np.maximum(wg.max(axis=2), np.float32(0))
     s = bf16_round((mx - mn) / np.float32(15.0))
     s = np.where(s == 0, np.float32(1.0), s).astype(np.float32)
-    z = np.clip(np.rint(-mn / s), 0, 15).astype(np.float32)
+    # + 0 turns a -0 zero-point (from mn = -0) into +0: an integer has no sign
+    z = np.clip(np.rint(-mn / s), 0, 15).astype(np.float32) + np.float32(0.0)
     q = np.rint(wg / s[:, :, None]) + z[:, :, None]
     q = np.clip(q, 0, 15).astype(np.uint8).reshape(N, K)
     return q, s, z

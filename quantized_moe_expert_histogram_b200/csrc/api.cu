@@ -1,0 +1,235 @@
+// C ABI entry points: argument validation, regime dispatch, error strings.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace moeq {
+
+namespace {
+thread_local char g_err[512] = "no error";
+}
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+moe_status_t cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return MOE_OK;
+  set_error("%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+  return MOE_ERR_CUDA;
+}
+
+BlobLayout blob_layout(int d, int F, int group, int layout) {
+  BlobLayout L{};
+  L.valid = 0;
+  if (d <= 0 || F <= 0 || d % 128 || F % 128) return L;
+  if (group != 64 && group != 128) return L;
+  if (d % group || F % group) return L;
+  if (layout != MOE_LAYOUT_INT4 && layout != MOE_LAYOUT_PLANES) return L;
+  const size_t N[3] = {(size_t)F, (size_t)F, (size_t)d};
+  const size_t K[3] = {(size_t)d, (size_t)d, (size_t)F};
+  size_t pos = 0;
+  for (int m = 0; m < 3; ++m) {
+    if (layout == MOE_LAYOUT_INT4) {
+      L.codes[m] = pos;
+      pos += N[m] * K[m] / 2;
+    } else {
+      L.q2[m] = pos;
+      pos += N[m] * K[m] / 4;
+      L.d3[m] = pos;
+      pos += N[m] * K[m] / 8;
+      L.d4[m] = pos;
+      pos += N[m] * K[m] / 8;
+    }
+  }
+  for (int m = 0; m < 3; ++m) {
+    L.sz[m] = pos;
+    pos += N[m] * (K[m] / group) * 4;
+  }
+  L.bytes = pos;
+  L.valid = 1;
+  return L;
+}
+
+}  // namespace moeq
+
+using namespace moeq;
+
+namespace {
+
+inline cudaStream_t S(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Regime: the decode GEMV streams each weight row once per (at most 8)
+// rows of a bin; bins never hold more than T rows, so it is exact-fit for
+// T <= 8.  Larger T goes to the tensor-core grouped GEMM.
+constexpr int kGemvMaxT = 8;
+
+size_t workspace_for(int total_rows, int F) {
+  size_t h = static_cast<size_t>(total_rows) * F * sizeof(__half);
+  return (h + 255) & ~static_cast<size_t>(255);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_err; }
+
+size_t moe_blob_bytes(int d, int F, int group, int layout) {
+  const BlobLayout L = blob_layout(d, F, group, layout);
+  return L.valid ? L.bytes : 0;
+}
+
+moe_status_t moe_quant_pack(const float* w_gate, const float* w_up, const float* w_down, int E,
+                            int d, int F, int group, int layout, void* blobs,
+                            moe_stream_t stream) {
+  if (!w_gate || !w_up || !w_down || !blobs || E <= 0) {
+    set_error("moe_quant_pack: null pointer or E <= 0");
+    return MOE_ERR_INVALID_ARG;
+  }
+  const BlobLayout L = blob_layout(d, F, group, layout);
+  if (!L.valid) {
+    set_error("moe_quant_pack: unsupported shape d=%d F=%d group=%d layout=%d", d, F, group, layout);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (!aligned16(blobs)) {
+    set_error("moe_quant_pack: blobs must be 16-byte aligned");
+    return MOE_ERR_INVALID_ARG;
+  }
+  return launch_pack(w_gate, w_up, w_down, E, d, F, group, layout, blobs, S(stream));
+}
+
+moe_status_t moe_route_topk(const void* x, const float* w_router, const float* bias,
+                            const int32_t* forced_idx, int T, int d, int E, int k,
+                            int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0) {
+    set_error("moe_route_topk: bad sizes T=%d d=%d E=%d k=%d", T, d, E, k);
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (T > 0 && (!x || !w_router || !topk_idx || !topk_w)) {
+    set_error("moe_route_topk: null pointer");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (k > E || k > 16 || E > 256) {
+    set_error("moe_route_topk: need k <= E, k <= 16, E <= 256 (k=%d E=%d)", k, E);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (d % 32) {
+    set_error("moe_route_topk: d=%d must be a multiple of 32", d);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  return launch_route(x, w_router, bias, forced_idx, T, d, E, k, topk_idx, topk_w, S(stream));
+}
+
+moe_status_t moe_permute(const int32_t* topk_idx, const uint8_t* bits, const void* x, int T,
+                         int d, int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
+                         int32_t* inv_perm, void* x_perm, int32_t* status, moe_stream_t stream) {
+  if (T < 0 || E <= 0 || k <= 0 || k > E) {
+    set_error("moe_permute: bad sizes T=%d E=%d k=%d", T, E, k);
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (!counts || !offsets || (T > 0 && (!topk_idx || !perm || !inv_perm))) {
+    set_error("moe_permute: null pointer");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (static_cast<long>(T) * k > (1L << 24)) {
+    set_error("moe_permute: T*k = %ld exceeds 2^24", static_cast<long>(T) * k);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if ((x == nullptr) != (x_perm == nullptr)) {
+    set_error("moe_permute: x and x_perm must both be given or both be NULL");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (x_perm && (d <= 0 || d % 8 || !aligned16(x) || !aligned16(x_perm))) {
+    set_error("moe_permute: gather needs d %% 8 == 0 and 16-byte aligned x / x_perm");
+    return MOE_ERR_INVALID_ARG;
+  }
+  return launch_permute(topk_idx, bits, x, T, d, E, k, counts, offsets, perm, inv_perm, x_perm,
+                        status, S(stream));
+}
+
+size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int layout) {
+  (void)E;
+  (void)d;
+  (void)layout;
+  if (total_rows < 0 || F <= 0) return 0;
+  return workspace_for(total_rows, F);
+}
+
+moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, const void* blobs,
+                                const int32_t* slot_of, int total_rows, int T, int E, int d,
+                                int F, int group, int layout, void* workspace,
+                                size_t workspace_bytes, float* y_perm, int32_t* status,
+                                moe_stream_t stream) {
+  if (total_rows < 0 || T < 0 || E <= 0) {
+    set_error("moe_grouped_ffn_wq: bad sizes");
+    return MOE_ERR_INVALID_ARG;
+  }
+  const BlobLayout L = blob_layout(d, F, group, layout);
+  if (!L.valid) {
+    set_error("moe_grouped_ffn_wq: unsupported shape d=%d F=%d group=%d layout=%d", d, F, group,
+              layout);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (total_rows == 0) return MOE_OK;
+  if (!x_perm || !offsets || !blobs || !workspace || !y_perm) {
+    set_error("moe_grouped_ffn_wq: null pointer");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x_perm) || !aligned16(blobs) || !aligned16(workspace) || !aligned16(y_perm)) {
+    set_error("moe_grouped_ffn_wq: buffers must be 16-byte aligned");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (workspace_bytes < workspace_for(total_rows, F)) {
+    set_error("moe_grouped_ffn_wq: workspace %zu < %zu bytes", workspace_bytes,
+              workspace_for(total_rows, F));
+    return MOE_ERR_WORKSPACE;
+  }
+  if (E * (layout == MOE_LAYOUT_PLANES ? 3 : 1) > 768) {
+    set_error("moe_grouped_ffn_wq: too many bins");
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  FfnArgs a{};
+  a.x_perm = static_cast<const __half*>(x_perm);
+  a.offsets = offsets;
+  a.blobs = static_cast<const uint8_t*>(blobs);
+  a.slot_of = slot_of;
+  a.total_rows = total_rows;
+  a.T = T;
+  a.E = E;
+  a.d = d;
+  a.F = F;
+  a.group = group;
+  a.layout = layout;
+  a.blob_bytes = L.bytes;
+  a.lay = L;
+  a.h = static_cast<__half*>(workspace);
+  a.y_perm = y_perm;
+  a.status = status;
+  if (T <= kGemvMaxT || !tc_supported(a)) return launch_ffn_gemv(a, S(stream));
+  return launch_ffn_tc(a, S(stream));
+}
+
+moe_status_t moe_unpermute_combine(const float* y_perm, const int32_t* inv_perm,
+                                   const float* topk_w, const void* residual, int T, int k, int d,
+                                   void* y, moe_stream_t stream) {
+  if (T < 0 || k <= 0 || d <= 0 || d % 4) {
+    set_error("moe_unpermute_combine: bad sizes T=%d k=%d d=%d", T, k, d);
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (T > 0 && (!y_perm || !inv_perm || !topk_w || !y)) {
+    set_error("moe_unpermute_combine: null pointer");
+    return MOE_ERR_INVALID_ARG;
+  }
+  return launch_combine(y_perm, inv_perm, topk_w, residual, T, k, d, y, S(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// Shared device/host helpers of the moeq library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moeq.h"
+
+namespace moeq {
+
+// Thread-local error message (set by the API layer).
+void set_error(const char* fmt, ...);
+moe_status_t cuda_check(cudaError_t e, const char* what);
+
+// Byte offsets of each section inside one expert blob (format documented
+// in moeq.h).
+struct BlobLayout {
+  size_t codes[3];   // INT4 codes of gate, up, down
+  size_t q2[3];      // PLANES: Q2 of gate, up, down
+  size_t d3[3];
+  size_t d4[3];
+  size_t sz[3];      // (scale, zero) words of gate, up, down
+  size_t bytes;
+  int valid;
+};
+BlobLayout blob_layout(int d, int F, int group, int layout);
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ void flag_status(int32_t* status, unsigned bits) {
+  if (status) atomicOr(reinterpret_cast<unsigned*>(status), bits);
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
+  uint32_t r;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+
+// SiLU in fp32: v / (1 + exp(-v)).
+__device__ __forceinline__ float silu_f(float v) { return v / (1.0f + __expf(-v)); }
+
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Launchers (each returns MOE_OK or an error already recorded).
+moe_status_t launch_pack(const float* w_gate, const float* w_up, const float* w_down, int E, int d,
+                         int F, int group, int layout, void* blobs, cudaStream_t s);
+moe_status_t launch_route(const void* x, const float* w_router, const float* bias,
+                          const int32_t* forced, int T, int d, int E, int k, int32_t* idx,
+                          float* w, cudaStream_t s);
+moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void* x, int T, int d,
+                            int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
+                            int32_t* inv_perm, void* x_perm, int32_t* status, cudaStream_t s);
+moe_status_t launch_combine(const float* y_perm, const int32_t* inv_perm, const float* w,
+                            const void* residual, int T, int k, int d, void* y, cudaStream_t s);
+
+struct FfnArgs {
+  const __half* x_perm;
+  const int32_t* offsets;
+  const uint8_t* blobs;
+  const int32_t* slot_of;
+  int total_rows, T, E, d, F, group, layout;
+  size_t blob_bytes;
+  BlobLayout lay;
+  __half* h;          // workspace: fp16 [total_rows][F]
+  float* y_perm;
+  int32_t* status;
+};
+moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);
+moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s);
+bool tc_supported(const FfnArgs& a);
+
+}  // namespace moeq

@@ -1,0 +1,315 @@
+// Decode-regime grouped expert FFN: a warp per group of weight rows.
+//
+// Used when no bin can hold more than a few rows (T <= 8): the layer is
+// then bound by the bytes of the routed experts' codes, so each weight row
+// is streamed once with 16-byte loads and dotted against the bin's (at
+// most MAXR) activation rows, which stay in L1.  Dequantisation happens in
+// registers: a 4-bit code q becomes the fp32 value 1 + q/16 by OR-ing it
+// into the mantissa of 1.0f, so the row dot product needs no int->float
+// conversion; per 8 elements the exact  sum (q - z) * s * x  is recovered as
+//   s * (16 * (sum (1 + q/16) x - sum x) - z * sum x).
+// Accumulation is fp32.  blockIdx.y enumerates the non-empty (and, in slot
+// mode, resident) bins; blockIdx.x a block of 8 warps x RW output rows.
+//
+//   gate/up pass:  h[p][f]      = silu(Wg[f] . x_p) * (Wu[f] . x_p)   (fp16)
+//   down pass:     y_perm[p][n] = Wd[n] . h_p                          (fp32)
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace moeq {
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+constexpr int kChunkSteps = 4;  // 32-element steps whose loads are issued together
+
+struct GemvParams {
+  const __half* act;        // x_perm [rows][K] or h [rows][K]
+  const int32_t* offsets;   // [nbins+1]
+  const uint8_t* blobs;
+  const int32_t* slot_of;
+  size_t blob_bytes;
+  size_t code_off[2];       // INT4 codes (or Q2) of the 1-2 matrices
+  size_t d3_off[2];
+  size_t d4_off[2];
+  size_t sz_off[2];
+  int K, N, nbins, planes_mult;  // planes_mult: 1 for INT4 bins, 3 for (e,b) bins
+  int group;
+  __half* h_out;            // gate/up pass output [rows][N]
+  float* y_out;             // down pass output [rows][N]
+};
+
+// 8 two-bit fields (bits 2i..2i+1) -> bits 4i..4i+1.
+__device__ __forceinline__ uint32_t spread2(uint32_t x) {
+  x &= 0xFFFFu;
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  x = (x | (x << 2)) & 0x33333333u;
+  return x;
+}
+// 8 one-bit fields (bit i) -> bit 4i.
+__device__ __forceinline__ uint32_t spread1(uint32_t x) {
+  x &= 0xFFu;
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  x = (x | (x << 3)) & 0x11111111u;
+  return x;
+}
+
+// Nibble i of `w` as the float 1 + q/16.
+template <int I>
+__device__ __forceinline__ float nib_as_float(uint32_t w) {
+  constexpr int sh = 19 - 4 * I;
+  const uint32_t m = sh >= 0 ? (w << sh) : (w >> (-sh));
+  return __uint_as_float((m & 0x00780000u) | 0x3F800000u);
+}
+
+// Locate the blockIdx.y-th non-empty, resident bin.  Returns false when
+// there is none (the block has no work).
+__device__ __forceinline__ bool find_bin(const GemvParams& P, int ordinal, int& bin, int& row0,
+                                         int& nrows, int& blob_index, int& bits) {
+  const int lane = threadIdx.x & 31;
+  int seen = 0;
+  for (int b0 = 0; b0 < P.nbins; b0 += 32) {
+    const int b = b0 + lane;
+    bool ok = false;
+    int slot = 0;
+    if (b < P.nbins) {
+      const int n = P.offsets[b + 1] - P.offsets[b];
+      const int e = b / P.planes_mult;
+      slot = P.slot_of ? P.slot_of[e] : e;
+      ok = n > 0 && slot >= 0;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, ok);
+    const int cnt = __popc(m);
+    if (ordinal < seen + cnt) {
+      // the (ordinal-seen)-th set bit of m
+      int want = ordinal - seen;
+      unsigned mm = m;
+      for (int i = 0; i < want; ++i) mm &= mm - 1;
+      const int src = __ffs(mm) - 1;
+      bin = b0 + src;
+      slot = __shfl_sync(0xffffffffu, slot, src);
+      row0 = P.offsets[bin];
+      nrows = P.offsets[bin + 1] - row0;
+      blob_index = slot;
+      bits = P.planes_mult == 3 ? 2 + bin % 3 : 4;
+      return true;
+    }
+    seen += cnt;
+  }
+  return false;
+}
+
+// Load the 32 codes (as 4 nibble words) of row `r` at element offset k0.
+template <bool PLANES>
+__device__ __forceinline__ uint4 load_codes(const GemvParams& P, const uint8_t* blob, int m,
+                                            int row, int k0, int bits) {
+  if (!PLANES) {
+    const uint32_t* c = reinterpret_cast<const uint32_t*>(blob + P.code_off[m]) +
+                        static_cast<size_t>(row) * (P.K / 8) + k0 / 8;
+    return ldg_nc_v4(c);
+  } else {
+    const uint32_t* q2 = reinterpret_cast<const uint32_t*>(blob + P.code_off[m]) +
+                         static_cast<size_t>(row) * (P.K / 16) + k0 / 16;
+    uint2 base;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(base.x), "=r"(base.y)
+                 : "l"(q2));
+    uint32_t r3 = 0, r4 = 0;
+    if (bits >= 3)
+      r3 = ldg_nc_u32(reinterpret_cast<const uint32_t*>(blob + P.d3_off[m]) +
+                      static_cast<size_t>(row) * (P.K / 32) + k0 / 32);
+    if (bits >= 4)
+      r4 = ldg_nc_u32(reinterpret_cast<const uint32_t*>(blob + P.d4_off[m]) +
+                      static_cast<size_t>(row) * (P.K / 32) + k0 / 32);
+    uint4 out;
+    out.x = (spread2(base.x) << 2) | (spread1(r3) << 1) | spread1(r4);
+    out.y = (spread2(base.x >> 16) << 2) | (spread1(r3 >> 8) << 1) | spread1(r4 >> 8);
+    out.z = (spread2(base.y) << 2) | (spread1(r3 >> 16) << 1) | spread1(r4 >> 16);
+    out.w = (spread2(base.y >> 16) << 2) | (spread1(r3 >> 24) << 1) | spread1(r4 >> 24);
+    return out;
+  }
+}
+
+// RW output rows per warp; NM matrices (2 = gate+up, 1 = down).
+template <int MAXR, int NM, int RW, bool PLANES>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_gemv(const GemvParams P) {
+  constexpr int ROWS = NM * RW;  // weight rows per warp
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int bin, row0, nrows, blob_index, bits;
+  if (!find_bin(P, blockIdx.y, bin, row0, nrows, blob_index, bits)) return;
+  const uint8_t* blob = P.blobs + static_cast<size_t>(blob_index) * P.blob_bytes;
+  const int n0 = (blockIdx.x * kWarpsPerBlock + warp) * RW;  // first output row of this warp
+  if (n0 >= P.N) return;
+
+  // Bins with more than MAXR rows (only when this regime is used beyond its
+  // intended T) are processed MAXR rows at a time.
+  const int bin_row0 = row0, bin_rows = nrows;
+  for (int rc = 0; rc < bin_rows; rc += MAXR) {
+  row0 = bin_row0 + rc;
+  nrows = min(MAXR, bin_rows - rc);
+  float acc[ROWS][MAXR];
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r)
+#pragma unroll
+    for (int t = 0; t < MAXR; ++t) acc[r][t] = 0.0f;
+
+  const int G = P.K / P.group;
+  for (int kc = 0; kc < P.K; kc += kChunkSteps * 1024) {
+    uint4 codes[kChunkSteps][ROWS];
+    uint32_t sz[kChunkSteps][ROWS];
+#pragma unroll
+    for (int s = 0; s < kChunkSteps; ++s) {
+      const int k0 = kc + s * 1024 + lane * 32;
+      if (k0 < P.K) {
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+          const int m = r % NM, row = n0 + r / NM;
+          codes[s][r] = load_codes<PLANES>(P, blob, m, row, k0, bits);
+          const uint32_t* szp = reinterpret_cast<const uint32_t*>(blob + P.sz_off[m]);
+          sz[s][r] = ldg_nc_u32(szp + (static_cast<size_t>(row >> 7) * G + k0 / P.group) * 128 + (row & 127));
+        }
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < kChunkSteps; ++s) {
+      const int k0 = kc + s * 1024 + lane * 32;
+      if (k0 >= P.K) continue;
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi) {  // 8 elements per word
+        float xv[MAXR][8], px[MAXR];
+#pragma unroll
+        for (int t = 0; t < MAXR; ++t) {
+          px[t] = 0.0f;
+          if (t < nrows) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(P.act + static_cast<size_t>(row0 + t) * P.K + k0 + wi * 8);
+            const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 f = __half22float2(h2[j]);
+              xv[t][2 * j] = f.x;
+              xv[t][2 * j + 1] = f.y;
+              px[t] += f.x + f.y;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) xv[t][j] = 0.0f;
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+          const uint32_t w = wi == 0 ? codes[s][r].x : wi == 1 ? codes[s][r].y : wi == 2 ? codes[s][r].z : codes[s][r].w;
+          const float f0 = nib_as_float<0>(w), f1 = nib_as_float<1>(w), f2 = nib_as_float<2>(w),
+                      f3 = nib_as_float<3>(w), f4 = nib_as_float<4>(w), f5 = nib_as_float<5>(w),
+                      f6 = nib_as_float<6>(w), f7 = nib_as_float<7>(w);
+          const float sc = __uint_as_float(sz[s][r] << 16);
+          const float zp = __uint_as_float(sz[s][r] & 0xFFFF0000u);
+#pragma unroll
+          for (int t = 0; t < MAXR; ++t) {
+            float p = f0 * xv[t][0];
+            p = fmaf(f1, xv[t][1], p);
+            p = fmaf(f2, xv[t][2], p);
+            p = fmaf(f3, xv[t][3], p);
+            p = fmaf(f4, xv[t][4], p);
+            p = fmaf(f5, xv[t][5], p);
+            p = fmaf(f6, xv[t][6], p);
+            p = fmaf(f7, xv[t][7], p);
+            // sum (q - z) x = 16 (p - px) - z px
+            const float qx = 16.0f * (p - px[t]);
+            acc[r][t] = fmaf(sc, fmaf(-zp, px[t], qx), acc[r][t]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r)
+#pragma unroll
+    for (int t = 0; t < MAXR; ++t) {
+      float v = acc[r][t];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      acc[r][t] = v;
+    }
+  if (lane == 0) {
+#pragma unroll
+    for (int t = 0; t < MAXR; ++t) {
+      if (t >= nrows) break;
+      const size_t p = static_cast<size_t>(row0 + t);
+#pragma unroll
+      for (int j = 0; j < RW; ++j) {
+        if (NM == 2) {
+          const float g = acc[2 * j][t], u = acc[2 * j + 1][t];
+          P.h_out[p * P.N + n0 + j] = __float2half_rn(silu_f(g) * u);
+        } else {
+          P.y_out[p * P.N + n0 + j] = acc[j][t];
+        }
+      }
+    }
+  }
+  }
+}
+
+template <int MAXR, bool PLANES>
+moe_status_t run_pair(GemvParams gu, GemvParams dn, int max_bins, cudaStream_t s) {
+  constexpr int RW_GU = 2, RW_DN = 4;
+  dim3 g1(ceil_div(gu.N, kWarpsPerBlock * RW_GU), max_bins);
+  k_gemv<MAXR, 2, RW_GU, PLANES><<<g1, kWarpsPerBlock * 32, 0, s>>>(gu);
+  moe_status_t st = cuda_check(cudaGetLastError(), "ffn gemv gate/up launch");
+  if (st != MOE_OK) return st;
+  dim3 g2(ceil_div(dn.N, kWarpsPerBlock * RW_DN), max_bins);
+  k_gemv<MAXR, 1, RW_DN, PLANES><<<g2, kWarpsPerBlock * 32, 0, s>>>(dn);
+  return cuda_check(cudaGetLastError(), "ffn gemv down launch");
+}
+
+}  // namespace
+
+moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s) {
+  const bool planes = a.layout == MOE_LAYOUT_PLANES;
+  const int mult = planes ? 3 : 1;
+  const int nbins = a.E * mult;
+  GemvParams gu{};
+  gu.act = a.x_perm;
+  gu.offsets = a.offsets;
+  gu.blobs = a.blobs;
+  gu.slot_of = a.slot_of;
+  gu.blob_bytes = a.blob_bytes;
+  gu.K = a.d;
+  gu.N = a.F;
+  gu.nbins = nbins;
+  gu.planes_mult = mult;
+  gu.group = a.group;
+  gu.h_out = a.h;
+  for (int m = 0; m < 2; ++m) {
+    gu.code_off[m] = planes ? a.lay.q2[m] : a.lay.codes[m];
+    gu.d3_off[m] = a.lay.d3[m];
+    gu.d4_off[m] = a.lay.d4[m];
+    gu.sz_off[m] = a.lay.sz[m];
+  }
+  GemvParams dn = gu;
+  dn.act = a.h;
+  dn.K = a.F;
+  dn.N = a.d;
+  dn.h_out = nullptr;
+  dn.y_out = a.y_perm;
+  dn.code_off[0] = planes ? a.lay.q2[2] : a.lay.codes[2];
+  dn.d3_off[0] = a.lay.d3[2];
+  dn.d4_off[0] = a.lay.d4[2];
+  dn.sz_off[0] = a.lay.sz[2];
+  const int max_bins = std::min(nbins, a.total_rows);
+  if (max_bins == 0) return MOE_OK;
+  const int T = a.T;
+  if (planes) {
+    if (T <= 1) return run_pair<1, true>(gu, dn, max_bins, s);
+    if (T <= 2) return run_pair<2, true>(gu, dn, max_bins, s);
+    if (T <= 4) return run_pair<4, true>(gu, dn, max_bins, s);
+    return run_pair<8, true>(gu, dn, max_bins, s);
+  }
+  if (T <= 1) return run_pair<1, false>(gu, dn, max_bins, s);
+  if (T <= 2) return run_pair<2, false>(gu, dn, max_bins, s);
+  if (T <= 4) return run_pair<4, false>(gu, dn, max_bins, s);
+  return run_pair<8, false>(gu, dn, max_bins, s);
+}
+
+}  // namespace moeq

@@ -1,0 +1,356 @@
+// Offload mode: a per-layer GPU slot cache of expert blobs fed from pinned
+// host memory with cudaMemcpyAsync on a copy stream, overlapped with the
+// grouped FFN on the compute stream.
+//
+// A layer-step's distinct experts are ordered hits first, then misses by
+// descending row count (the hottest expert is loaded first), and cut into
+// waves of at most slots/2 experts.  Waves alternate between slot sets in
+// LRU order and never into a slot of the previous wave, so the copies of
+// wave w+1 overlap the compute of wave w (load E2 while computing E1).  A slot is overwritten only after the compute
+// that last read it has finished (per-slot event), and a wave computes only
+// after its copies have landed (per-wave event).  The FFN of a wave sees a
+// device table slot_of[E] listing just that wave's experts.
+#include <algorithm>
+#include <atomic>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+
+using namespace moeq;
+
+namespace {
+std::atomic<int> g_fault_what{0};
+std::atomic<int> g_fault_count{0};
+
+bool take_fault(int what) {
+  if (g_fault_what.load() != what) return false;
+  int c = g_fault_count.load();
+  while (c > 0) {
+    if (g_fault_count.compare_exchange_weak(c, c - 1)) return true;
+  }
+  return false;
+}
+
+inline cudaStream_t S(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
+}  // namespace
+
+struct moe_slot_cache {
+  int E = 0, S = 0, max_waves = 0;
+  size_t blob_bytes = 0;
+  const uint8_t* host = nullptr;
+  uint8_t* pool = nullptr;
+  std::vector<int> slot_of;        // expert -> slot, -1 when not resident
+  std::vector<int> expert_in;      // slot -> expert, -1 when empty
+  std::vector<uint64_t> last_use;  // slot -> logical time of last use
+  uint64_t clock = 1;
+  std::vector<cudaEvent_t> slot_free;  // recorded after the last compute reading the slot
+  std::vector<char> slot_free_valid;
+  std::vector<cudaEvent_t> copy_done;  // per wave
+  std::vector<char> copy_pending;      // per wave: wave has copies to wait for
+  cudaEvent_t tables_done = nullptr;
+  bool tables_done_valid = false;
+  int32_t* d_tables = nullptr;  // device [max_waves][E]
+  int32_t* h_tables = nullptr;  // pinned host [max_waves][E]
+  // plan of the current step
+  std::vector<std::vector<int>> waves;           // experts per wave
+  std::vector<std::vector<int>> wave_misses;     // experts that must be copied, per wave
+  std::vector<std::vector<int>> wave_slots;      // slot of each expert of the wave
+  int copies_issued = 0;                         // waves whose copies were issued
+  int64_t stats[3] = {0, 0, 0};
+};
+
+namespace {
+
+// After a failed copy: experts planned into waves >= w are not resident
+// (their slots hold stale bytes), and the plan is dropped.
+void invalidate_from(moe_slot_cache* c, int w) {
+  for (size_t v = static_cast<size_t>(w); v < c->waves.size(); ++v)
+    for (int e : c->wave_misses[v]) {
+      const int s = c->slot_of[e];
+      if (s >= 0) c->expert_in[s] = -1;
+      c->slot_of[e] = -1;
+    }
+  c->waves.clear();
+  c->wave_misses.clear();
+  c->wave_slots.clear();
+}
+
+moe_status_t issue_copies(moe_slot_cache* c, int w, cudaStream_t copy) {
+  const auto& slots = c->wave_slots[w];
+  const auto& exps = c->waves[w];
+  bool any = false;
+  for (size_t i = 0; i < exps.size(); ++i) {
+    const int e = exps[i];
+    if (std::find(c->wave_misses[w].begin(), c->wave_misses[w].end(), e) == c->wave_misses[w].end())
+      continue;
+    const int s = slots[i];
+    if (take_fault(2)) {
+      set_error("moe_slot_stage: injected copy failure (expert %d)", e);
+      return MOE_ERR_FAULT_INJECTED;
+    }
+    if (c->slot_free_valid[s]) {
+      moe_status_t st = cuda_check(cudaStreamWaitEvent(copy, c->slot_free[s], 0), "slot wait free");
+      if (st != MOE_OK) return st;
+    }
+    moe_status_t st = cuda_check(
+        cudaMemcpyAsync(c->pool + static_cast<size_t>(s) * c->blob_bytes,
+                        c->host + static_cast<size_t>(e) * c->blob_bytes, c->blob_bytes,
+                        cudaMemcpyHostToDevice, copy),
+        "slot H2D copy");
+    if (st != MOE_OK) return st;
+    any = true;
+  }
+  c->copy_pending[w] = any;
+  if (any) return cuda_check(cudaEventRecord(c->copy_done[w], copy), "slot copy event");
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void moe_debug_inject_fault(int what, int count) {
+  g_fault_what.store(what);
+  g_fault_count.store(what ? count : 0);
+}
+
+moe_status_t moe_slot_cache_create(int E, int slots, size_t blob_bytes, const void* host_blobs,
+                                   void* device_pool, moe_slot_cache** out) {
+  if (!out || !host_blobs || !device_pool || E <= 0 || E > 256 || slots < 2 || blob_bytes == 0) {
+    set_error("moe_slot_cache_create: bad arguments");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (blob_bytes % 16) {
+    set_error("moe_slot_cache_create: blob_bytes must be a multiple of 16");
+    return MOE_ERR_INVALID_ARG;
+  }
+  *out = nullptr;
+  moe_slot_cache* c = new (std::nothrow) moe_slot_cache();
+  if (!c) {
+    set_error("moe_slot_cache_create: out of host memory");
+    return MOE_ERR_OOM;
+  }
+  c->E = E;
+  c->S = slots;
+  c->blob_bytes = blob_bytes;
+  c->host = static_cast<const uint8_t*>(host_blobs);
+  c->pool = static_cast<uint8_t*>(device_pool);
+  c->slot_of.assign(E, -1);
+  c->expert_in.assign(slots, -1);
+  c->last_use.assign(slots, 0);
+  c->slot_free.assign(slots, nullptr);
+  c->slot_free_valid.assign(slots, 0);
+  // at most E distinct experts, at least 1 per wave
+  c->max_waves = E;
+  c->copy_done.assign(c->max_waves, nullptr);
+  c->copy_pending.assign(c->max_waves, 0);
+  moe_status_t st = MOE_OK;
+  for (int s = 0; s < slots && st == MOE_OK; ++s)
+    st = cuda_check(cudaEventCreateWithFlags(&c->slot_free[s], cudaEventDisableTiming), "event");
+  for (int w = 0; w < c->max_waves && st == MOE_OK; ++w)
+    st = cuda_check(cudaEventCreateWithFlags(&c->copy_done[w], cudaEventDisableTiming), "event");
+  if (st == MOE_OK)
+    st = cuda_check(cudaEventCreateWithFlags(&c->tables_done, cudaEventDisableTiming), "event");
+  if (st == MOE_OK)
+    st = cuda_check(cudaMalloc(&c->d_tables, sizeof(int32_t) * c->max_waves * E), "table alloc");
+  if (st == MOE_OK)
+    st = cuda_check(cudaHostAlloc(&c->h_tables, sizeof(int32_t) * c->max_waves * E,
+                                  cudaHostAllocDefault),
+                    "table host alloc");
+  if (st != MOE_OK) {
+    moe_slot_cache_destroy(c);
+    return st;
+  }
+  *out = c;
+  return MOE_OK;
+}
+
+void moe_slot_cache_destroy(moe_slot_cache* c) {
+  if (!c) return;
+  for (auto e : c->slot_free)
+    if (e) {
+      cudaEventSynchronize(e);
+      cudaEventDestroy(e);
+    }
+  for (auto e : c->copy_done)
+    if (e) {
+      cudaEventSynchronize(e);
+      cudaEventDestroy(e);
+    }
+  if (c->tables_done) {
+    cudaEventSynchronize(c->tables_done);
+    cudaEventDestroy(c->tables_done);
+  }
+  if (c->d_tables) cudaFree(c->d_tables);
+  if (c->h_tables) cudaFreeHost(c->h_tables);
+  delete c;
+}
+
+moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_ids,
+                            moe_stream_t copy_stream, moe_stream_t compute_stream,
+                            int32_t* n_waves, int64_t* stats_host) {
+  (void)compute_stream;
+  if (!c || !n_waves || n_ids < 0 || (n_ids > 0 && !ids_host)) {
+    set_error("moe_slot_stage: bad arguments");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (take_fault(1)) {
+    set_error("moe_slot_stage: injected fault before any work");
+    return MOE_ERR_FAULT_INJECTED;
+  }
+  std::vector<int> cnt(c->E, 0);
+  for (int i = 0; i < n_ids; ++i) {
+    const int e = ids_host[i];
+    if (e < 0 || e >= c->E) {
+      set_error("moe_slot_stage: expert id %d out of range [0,%d)", e, c->E);
+      return MOE_ERR_INVALID_ARG;
+    }
+    ++cnt[e];
+  }
+  std::vector<int> hits, misses;
+  for (int e = 0; e < c->E; ++e) {
+    if (!cnt[e]) continue;
+    (c->slot_of[e] >= 0 ? hits : misses).push_back(e);
+  }
+  std::stable_sort(misses.begin(), misses.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
+  std::vector<int> order(hits);
+  order.insert(order.end(), misses.begin(), misses.end());
+  const int W = std::max(1, c->S / 2);
+  const int nw = static_cast<int>((order.size() + W - 1) / W);
+  c->waves.assign(nw, {});
+  c->wave_misses.assign(nw, {});
+  c->wave_slots.assign(nw, {});
+  for (size_t i = 0; i < order.size(); ++i) c->waves[i / W].push_back(order[i]);
+
+  // Assign slots wave by wave.  Hits keep their slot; a miss takes the least
+  // recently used slot that holds nothing needed by this wave or later ones.
+  std::vector<int> slot_of = c->slot_of, expert_in = c->expert_in;
+  std::vector<uint64_t> last_use = c->last_use;
+  uint64_t clock = c->clock;
+  std::vector<char> needed_later(c->E, 0);
+  for (int e : order) needed_later[e] = 1;
+  int64_t n_hits = 0, n_miss = 0;
+  std::vector<int> prev_slots;  // slots of wave w-1: its compute may still be unqueued
+  for (int w = 0; w < nw; ++w) {
+    const uint64_t t = ++clock;
+    std::vector<char> pinned(c->S, 0);
+    for (int s : prev_slots) pinned[s] = 1;
+    for (int e : c->waves[w])
+      if (slot_of[e] >= 0) pinned[slot_of[e]] = 1;
+    for (int s = 0; s < c->S; ++s)
+      if (expert_in[s] >= 0 && needed_later[expert_in[s]]) pinned[s] = 1;
+    for (int e : c->waves[w]) {
+      int s = slot_of[e];
+      if (s >= 0) {
+        ++n_hits;
+      } else {
+        int best = -1;
+        for (int cand = 0; cand < c->S; ++cand) {
+          if (pinned[cand]) continue;
+          if (best < 0 || last_use[cand] < last_use[best]) best = cand;
+        }
+        if (best < 0) {
+          set_error("moe_slot_stage: no free slot (slots=%d)", c->S);
+          return MOE_ERR_INVALID_ARG;
+        }
+        s = best;
+        if (expert_in[s] >= 0) slot_of[expert_in[s]] = -1;
+        expert_in[s] = e;
+        slot_of[e] = s;
+        pinned[s] = 1;
+        c->wave_misses[w].push_back(e);
+        ++n_miss;
+      }
+      last_use[s] = t;
+      c->wave_slots[w].push_back(s);
+    }
+    for (int e : c->waves[w]) needed_later[e] = 0;
+    prev_slots = c->wave_slots[w];
+  }
+  c->slot_of.swap(slot_of);
+  c->expert_in.swap(expert_in);
+  c->last_use.swap(last_use);
+  c->clock = clock;
+  // Device tables of this step: the previous step's uploads must have run
+  // before the pinned staging rows are rewritten.
+  if (c->tables_done_valid) {
+    moe_status_t st = cuda_check(cudaEventSynchronize(c->tables_done), "slot table reuse");
+    if (st != MOE_OK) return st;
+  }
+  for (int w = 0; w < nw; ++w) {
+    int32_t* row = c->h_tables + static_cast<size_t>(w) * c->E;
+    for (int e = 0; e < c->E; ++e) row[e] = -1;
+    for (size_t i = 0; i < c->waves[w].size(); ++i) row[c->waves[w][i]] = c->wave_slots[w][i];
+  }
+  c->copies_issued = 0;
+  for (int w = 0; w < std::min(nw, 2); ++w) {
+    moe_status_t st = issue_copies(c, w, S(copy_stream));
+    if (st != MOE_OK) {
+      invalidate_from(c, w);
+      return st;
+    }
+    c->copies_issued = w + 1;
+  }
+  *n_waves = nw;
+  c->stats[0] = n_hits;
+  c->stats[1] = n_miss;
+  c->stats[2] = n_miss * static_cast<int64_t>(c->blob_bytes);
+  if (stats_host) {
+    stats_host[0] = c->stats[0];
+    stats_host[1] = c->stats[1];
+    stats_host[2] = c->stats[2];
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_slot_ffn(moe_slot_cache* c, const void* x_perm, const int32_t* offsets,
+                          int total_rows, int T, int d, int F, int group, int layout,
+                          void* workspace, size_t workspace_bytes, float* y_perm,
+                          int32_t* status, moe_stream_t copy_stream,
+                          moe_stream_t compute_stream) {
+  if (!c) {
+    set_error("moe_slot_ffn: null cache");
+    return MOE_ERR_INVALID_ARG;
+  }
+  const int nw = static_cast<int>(c->waves.size());
+  const size_t table_bytes = sizeof(int32_t) * c->E;
+  for (int w = 0; w < nw; ++w) {
+    if (c->copy_pending[w]) {
+      moe_status_t st = cuda_check(cudaStreamWaitEvent(S(compute_stream), c->copy_done[w], 0),
+                                   "slot wait copies");
+      if (st != MOE_OK) return st;
+    }
+    int32_t* dt = c->d_tables + static_cast<size_t>(w) * c->E;
+    moe_status_t st = cuda_check(cudaMemcpyAsync(dt, c->h_tables + static_cast<size_t>(w) * c->E,
+                                                 table_bytes, cudaMemcpyHostToDevice,
+                                                 S(compute_stream)),
+                                 "slot table upload");
+    if (st != MOE_OK) return st;
+    if (w == nw - 1) {
+      st = cuda_check(cudaEventRecord(c->tables_done, S(compute_stream)), "table event");
+      if (st != MOE_OK) return st;
+      c->tables_done_valid = true;
+    }
+    st = moe_grouped_ffn_wq(x_perm, offsets, c->pool, dt, total_rows, T, c->E, d, F, group, layout,
+                            workspace, workspace_bytes, y_perm, status, compute_stream);
+    if (st != MOE_OK) return st;
+    for (int s : c->wave_slots[w]) {
+      st = cuda_check(cudaEventRecord(c->slot_free[s], S(compute_stream)), "slot free event");
+      if (st != MOE_OK) return st;
+      c->slot_free_valid[s] = 1;
+    }
+    const int nxt = w + 2;
+    if (nxt < nw && nxt >= c->copies_issued) {
+      st = issue_copies(c, nxt, S(copy_stream));
+      if (st != MOE_OK) {
+        invalidate_from(c, nxt);
+        return st;
+      }
+      c->copies_issued = nxt + 1;
+    }
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,253 @@
+"""Thin ctypes binding of libmoeq.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does
+nothing but check tensor dtypes/devices, pass raw pointers and sizes, and
+turn a non-zero status into an exception.  All arithmetic runs in the CUDA
+kernels of the library; there is no CPU fallback: ``load()`` raises when
+the library is missing or no CUDA device is present.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoeq.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "moeq.h")
+
+LAYOUT_INT4 = 0
+LAYOUT_PLANES = 1
+DEV_BAD_INDEX = 1
+DEV_RANGE = 2
+DEV_TIMEOUT = 4
+
+_c_p = ctypes.c_void_p
+_c_i = ctypes.c_int
+_c_sz = ctypes.c_size_t
+
+_SIGS = {
+    "moe_last_error": (ctypes.c_char_p, []),
+    "moe_blob_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
+    "moe_quant_pack": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p]),
+    "moe_route_topk": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]),
+    "moe_permute": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_p,
+                           _c_p, _c_p]),
+    "moe_ffn_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
+    "moe_grouped_ffn_wq": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
+                                  _c_p, _c_sz, _c_p, _c_p, _c_p]),
+    "moe_unpermute_combine": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_p, _c_p]),
+    "moe_slot_cache_create": (_c_i, [_c_i, _c_i, _c_sz, _c_p, _c_p, ctypes.POINTER(_c_p)]),
+    "moe_slot_stage": (_c_i, [_c_p, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p]),
+    "moe_slot_ffn": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p,
+                            _c_p, _c_p, _c_p]),
+    "moe_slot_cache_destroy": (None, [_c_p]),
+    "moe_debug_inject_fault": (None, [_c_i, _c_i]),
+}
+
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn, code, msg):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+def header_symbols() -> list:
+    """Names of the functions declared in include/moeq.h."""
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
+
+
+def open_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """dlopen the library and attach signatures (needs no GPU)."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built; run quantized_moe_expert_histogram_b200.build.build()")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+def load():
+    """The library, for compute calls; raises without a CUDA device."""
+    global _lib
+    if not torch.cuda.is_available():
+        raise RuntimeError("moeq needs a CUDA device (B200, sm_100a); no CPU fallback exists")
+    if _lib is None:
+        _lib = open_library()
+    return _lib
+
+
+def _check(fn, code):
+    if code != 0:
+        raise MoeError(fn, code, _lib.moe_last_error().decode())
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def moe_blob_bytes(d, F, group, layout):
+    return int(load().moe_blob_bytes(d, F, group, layout))
+
+
+def moe_ffn_workspace_bytes(total_rows, E, d, F, layout):
+    return int(load().moe_ffn_workspace_bytes(total_rows, E, d, F, layout))
+
+
+def moe_quant_pack(w_gate, w_up, w_down, group, layout, blobs=None, stream=None):
+    lib = load()
+    E, F, d = w_gate.shape
+    nb = lib.moe_blob_bytes(d, F, group, layout)
+    if blobs is None:
+        blobs = torch.empty(E, nb, dtype=torch.uint8, device=w_gate.device)
+    _check("moe_quant_pack", lib.moe_quant_pack(
+        _ptr(w_gate, torch.float32, "w_gate"), _ptr(w_up, torch.float32, "w_up"),
+        _ptr(w_down, torch.float32, "w_down"), E, d, F, group, layout,
+        _ptr(blobs, torch.uint8, "blobs"), _stream(stream)))
+    return blobs
+
+
+def moe_route_topk(x, w_router, bias, k, forced_idx=None, topk_idx=None, topk_w=None, stream=None):
+    lib = load()
+    T, d = x.shape
+    E = w_router.shape[0]
+    if topk_idx is None:
+        topk_idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    _check("moe_route_topk", lib.moe_route_topk(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_router, torch.float32, "w_router"),
+        _ptr(bias, torch.float32, "bias"), _ptr(forced_idx, torch.int32, "forced_idx"), T, d, E, k,
+        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
+        _stream(stream)))
+    return topk_idx, topk_w
+
+
+def moe_permute(topk_idx, E, bits=None, x=None, out=None, status=None, stream=None):
+    """Returns dict(counts, offsets, perm, inv_perm, x_perm)."""
+    lib = load()
+    T, k = topk_idx.shape
+    nb = 3 * E if bits is not None else E
+    dev = topk_idx.device
+    d = x.shape[1] if x is not None else 0
+    if out is None:
+        out = dict(counts=torch.empty(nb, dtype=torch.int32, device=dev),
+                   offsets=torch.empty(nb + 1, dtype=torch.int32, device=dev),
+                   perm=torch.empty(T * k, dtype=torch.int32, device=dev),
+                   inv_perm=torch.empty(T * k, dtype=torch.int32, device=dev),
+                   x_perm=torch.empty(T * k, d, dtype=torch.float16, device=dev) if x is not None else None)
+    _check("moe_permute", lib.moe_permute(
+        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(bits, torch.uint8, "bits"),
+        _ptr(x, torch.bfloat16, "x"), T, d, E, k, _ptr(out["counts"], torch.int32),
+        _ptr(out["offsets"], torch.int32), _ptr(out["perm"], torch.int32),
+        _ptr(out["inv_perm"], torch.int32), _ptr(out["x_perm"], torch.float16),
+        _ptr(status, torch.int32, "status"), _stream(stream)))
+    return out
+
+
+def moe_grouped_ffn_wq(x_perm, offsets, blobs, T, E, d, F, group, layout, slot_of=None,
+                       workspace=None, y_perm=None, status=None, stream=None):
+    lib = load()
+    rows = x_perm.shape[0]
+    if workspace is None:
+        workspace = torch.empty(lib.moe_ffn_workspace_bytes(rows, E, d, F, layout), dtype=torch.uint8,
+                                device=x_perm.device)
+    if y_perm is None:
+        y_perm = torch.empty(rows, d, dtype=torch.float32, device=x_perm.device)
+    _check("moe_grouped_ffn_wq", lib.moe_grouped_ffn_wq(
+        _ptr(x_perm, torch.float16, "x_perm"), _ptr(offsets, torch.int32, "offsets"), _ptr(blobs),
+        _ptr(slot_of, torch.int32, "slot_of"), rows, T, E, d, F, group, layout, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(y_perm, torch.float32, "y_perm"),
+        _ptr(status, torch.int32, "status"), _stream(stream)))
+    return y_perm
+
+
+def moe_unpermute_combine(y_perm, inv_perm, topk_w, residual=None, y=None, stream=None):
+    lib = load()
+    T, k = topk_w.shape
+    d = y_perm.shape[1]
+    if y is None:
+        y = torch.empty(T, d, dtype=torch.bfloat16, device=y_perm.device)
+    _check("moe_unpermute_combine", lib.moe_unpermute_combine(
+        _ptr(y_perm, torch.float32, "y_perm"), _ptr(inv_perm, torch.int32, "inv_perm"),
+        _ptr(topk_w, torch.float32, "topk_w"), _ptr(residual, torch.bfloat16, "residual"), T, k, d,
+        _ptr(y, torch.bfloat16, "y"), _stream(stream)))
+    return y
+
+
+class SlotCache:
+    """One layer's GPU slot cache (moe_slot_cache_create / _destroy)."""
+
+    def __init__(self, E, slots, blob_bytes, host_blobs, device_pool):
+        lib = load()
+        if not host_blobs.is_pinned():
+            raise ValueError("host_blobs must be pinned host memory")
+        self._host = host_blobs
+        self._pool = device_pool
+        h = _c_p()
+        _check("moe_slot_cache_create", lib.moe_slot_cache_create(
+            E, slots, blob_bytes, host_blobs.data_ptr(), _ptr(device_pool), ctypes.byref(h)))
+        self.handle = h
+        self.E = E
+        self._ids = None
+
+    def stage(self, ids_host, copy_stream, compute_stream):
+        """moe_slot_stage; returns (n_waves, [hits, misses, bytes])."""
+        lib = load()
+        ids = ids_host.to(torch.int32).contiguous()
+        self._ids = ids
+        nw = ctypes.c_int32(0)
+        stats = (ctypes.c_int64 * 3)()
+        _check("moe_slot_stage", lib.moe_slot_stage(
+            self.handle, ids.data_ptr(), ids.numel(), copy_stream.cuda_stream,
+            compute_stream.cuda_stream, ctypes.byref(nw), stats))
+        return nw.value, list(stats)
+
+    def ffn(self, x_perm, offsets, T, d, F, group, layout, workspace, y_perm, status, copy_stream,
+            compute_stream):
+        lib = load()
+        _check("moe_slot_ffn", lib.moe_slot_ffn(
+            self.handle, _ptr(x_perm, torch.float16), _ptr(offsets, torch.int32), x_perm.shape[0], T,
+            d, F, group, layout, _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _ptr(y_perm, torch.float32), _ptr(status, torch.int32), copy_stream.cuda_stream,
+            compute_stream.cuda_stream))
+
+    def close(self):
+        if self.handle is not None and self.handle.value:
+            load().moe_slot_cache_destroy(self.handle)
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def moe_debug_inject_fault(what, count):
+    load().moe_debug_inject_fault(what, count)
+
+
+def moe_last_error():
+    return load().moe_last_error().decode()

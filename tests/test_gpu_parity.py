@@ -1,0 +1,185 @@
+"""GPU parity: every call of the C ABI against the oracle on the same seeded
+inputs.  Integer and index outputs (codes, expert ids, counts, offsets,
+permutations) must match bit for bit; floating outputs must satisfy
+|y - y_ref| <= 1e-2 + 1e-2 |y_ref| against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from quantized_moe_expert_histogram_b200 import build
+from quantized_moe_expert_histogram_b200 import inputs as I
+from quantized_moe_expert_histogram_b200 import moeq
+
+from gpu_helpers import gpu_layer, layer_inputs, oracle_layer, run_gpu_layer, within_tol
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+    moeq.load()
+
+
+# ---------------------------------------------------------------- pack ----
+
+@pytest.mark.parametrize("d,F,g,layout,E", [(256, 512, 64, "int4", 3), (256, 384, 64, "planes", 2),
+                                            (2048, 1024, 128, "int4", 2), (4096, 1024, 128, "planes", 1)])
+def test_pack_bitexact(d, F, g, layout, E):
+    shape = I.custom_shape(d=d, E=E, k=1, F=F, group=g, layout=layout)
+    L = I.make_layer(shape, 1, seed=11)
+    # a few special groups: all zero, all positive, all negative, constant
+    L["w_gate"][0, 0, :g] = 0
+    L["w_gate"][0, 1, :g] = L["w_gate"][0, 1, :g].abs()
+    L["w_up"][0, 2, :g] = -L["w_up"][0, 2, :g].abs()
+    L["w_down"][0, 3, :g] = 0.37
+    lay = moeq.LAYOUT_PLANES if layout == "planes" else moeq.LAYOUT_INT4
+    blobs = moeq.moe_quant_pack(L["w_gate"].cuda(), L["w_up"].cuda(), L["w_down"].cuda(), g, lay)
+    torch.cuda.synchronize()
+    got = blobs.cpu().numpy()
+    for e in range(E):
+        ref = O.build_blob(L["w_gate"][e].numpy(), L["w_up"][e].numpy(), L["w_down"][e].numpy(), g, layout)
+        assert got[e].size == ref.size
+        diff = np.nonzero(got[e] != ref)[0]
+        assert diff.size == 0, f"expert {e}: {diff.size} bytes differ, first at {diff[:5]}"
+
+
+# --------------------------------------------------------------- route ----
+
+@pytest.mark.parametrize("name,T,dup", [("tiny", 64, False), ("olmoe", 256, False), ("olmoe", 1, False),
+                                        ("mixtral", 32, False), ("tiny", 100, True),
+                                        ("nested", 77, False)])
+def test_route_bitexact(name, T, dup):
+    shape = I.SHAPES[name]
+    L = I.make_layer(shape, T, seed=3, weights=False)
+    if dup:  # exact ties: identical router rows must resolve to the lower index
+        L["w_router"][5] = L["w_router"][2]
+        L["w_router"][7] = L["w_router"][0]
+    bias = L["bias"].cuda() if L["bias"] is not None else None
+    idx, w = moeq.moe_route_topk(L["x"].cuda(), L["w_router"].cuda(), bias, shape.k)
+    torch.cuda.synchronize()
+    sel, gates, logits = O.route(L["x"].float().numpy(), L["w_router"].numpy(),
+                                 None if L["bias"] is None else L["bias"].numpy(), shape.k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), sel)
+    np.testing.assert_allclose(w.cpu().numpy(), gates, rtol=2e-6, atol=1e-7)
+
+
+def test_route_k_equals_E_and_forced():
+    shape = I.custom_shape(d=256, E=8, k=8, F=512, group=64)
+    L = I.make_layer(shape, 40, seed=4, weights=False)
+    idx, w = moeq.moe_route_topk(L["x"].cuda(), L["w_router"].cuda(), None, 8)
+    sel, gates, logits = O.route(L["x"].float().numpy(), L["w_router"].numpy(), None, 8)
+    np.testing.assert_array_equal(idx.cpu().numpy(), sel)
+    forced = torch.tensor(np.stack([np.random.default_rng(t).permutation(8)[:3] for t in range(40)]),
+                          dtype=torch.int32)
+    idx3, w3 = moeq.moe_route_topk(L["x"].cuda(), L["w_router"].cuda(), None, 3, forced_idx=forced.cuda())
+    np.testing.assert_array_equal(idx3.cpu().numpy(), forced.numpy())
+    np.testing.assert_allclose(w3.cpu().numpy(), O.gates_for(logits, forced.numpy()), rtol=2e-6, atol=1e-7)
+
+
+# ------------------------------------------------------------- permute ----
+
+@pytest.mark.parametrize("T,k,E,nested,skew", [(1, 2, 8, False, False), (33, 2, 8, False, True),
+                                                (4096, 8, 64, False, True), (777, 4, 16, True, False),
+                                                (100, 3, 256, True, True), (5, 8, 8, False, False)])
+def test_permute_bitexact(T, k, E, nested, skew):
+    rng = np.random.default_rng(T * 7 + E)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    if skew:
+        idx[: T // 2, 0] = 0
+    bits = rng.choice([2, 3, 4], size=(T, k), p=[.3, .4, .3]).astype(np.uint8) if nested else None
+    d = 64
+    x = torch.randn(T, d).to(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moeq.moe_permute(torch.from_numpy(idx).cuda(), E,
+                           bits=None if bits is None else torch.from_numpy(bits).cuda(), x=x.cuda(),
+                           status=status)
+    torch.cuda.synchronize()
+    keys, mult = O.assignment_keys(idx, bits)
+    counts, offsets, perm, inv = O.permute(keys, E * (mult or 1))
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), counts)
+    np.testing.assert_array_equal(out["offsets"].cpu().numpy(), offsets)
+    np.testing.assert_array_equal(out["perm"].cpu().numpy(), perm)
+    np.testing.assert_array_equal(out["inv_perm"].cpu().numpy(), inv)
+    xp = out["x_perm"].cpu()
+    np.testing.assert_array_equal(xp.numpy(), x[torch.from_numpy(perm // k).long()].to(torch.float16).numpy())
+    assert int(status.item()) == 0
+
+
+def test_permute_flags_bad_ids_and_range():
+    idx = torch.tensor([[0, 9], [3, -1]], dtype=torch.int32).cuda()
+    x = torch.tensor([[1.0] * 8, [1e5] * 8]).to(torch.bfloat16).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moeq.moe_permute(idx, 4, x=x, status=status)
+    torch.cuda.synchronize()
+    st = int(status.item())
+    assert st & moeq.DEV_BAD_INDEX and st & moeq.DEV_RANGE
+    # clamped ids still give a valid permutation
+    assert sorted(out["perm"].cpu().tolist()) == [0, 1, 2, 3]
+
+
+# --------------------------------------------------------------- layer ----
+
+def _check_layer(shape, T, seed=0, token_subset=None):
+    L = layer_inputs(shape, T, seed=seed)
+    layer = gpu_layer(shape, L, T)
+    bits = L.get("bits")
+    v, y = run_gpu_layer(layer, L, T, bits=bits)
+    ref, _ = oracle_layer(shape, L, bits=bits, token_subset=token_subset)
+    np.testing.assert_array_equal(v["topk_idx"].cpu().numpy(), ref["sel"])
+    np.testing.assert_array_equal(v["perm"].cpu().numpy(), ref["perm"])
+    np.testing.assert_array_equal(v["offsets"].cpu().numpy(), ref["offsets"])
+    toks = ref["tokens"]
+    ok, worst = within_tol(y[toks], ref["y"][toks])
+    assert ok, f"worst err/tol = {worst:.3f}"
+    # per-assignment expert outputs (before the combine)
+    yp = v["y_perm"].cpu().numpy()
+    rows = np.array([a for t in toks for a in range(t * shape.k, (t + 1) * shape.k)])
+    ok2, worst2 = within_tol(yp[ref["inv_perm"][rows]], ref["y_assign"][rows])
+    assert ok2, f"y_perm worst err/tol = {worst2:.3f}"
+    assert int(v["status"].item()) == 0
+    return worst, worst2
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 64), ("olmoe", 1), ("olmoe", 16), ("nested", 1),
+                                    ("nested", 64)])
+def test_layer_parity(name, T):
+    _check_layer(I.SHAPES[name], T)
+
+
+@pytest.mark.parametrize("d,E,k,F,g,layout,T", [(384, 5, 3, 640, 64, "int4", 7),
+                                                (128, 4, 4, 128, 64, "int4", 3),
+                                                (256, 6, 2, 384, 128, "planes", 13),
+                                                (1152, 12, 2, 256, 128, "int4", 2)])
+def test_layer_ragged_shapes(d, E, k, F, g, layout, T):
+    _check_layer(I.custom_shape(d=d, E=E, k=k, F=F, group=g, layout=layout), T, seed=5)
+
+
+def test_layer_deterministic():
+    shape = I.SHAPES["tiny"]
+    L = layer_inputs(shape, 64)
+    layer = gpu_layer(shape, L, 64)
+    _, y1 = run_gpu_layer(layer, L, 64)
+    _, y2 = run_gpu_layer(layer, L, 64)
+    np.testing.assert_array_equal(y1, y2)
+
+
+# ---------------------------------------------------------- api errors ----
+
+def test_api_rejects_bad_arguments():
+    x = torch.randn(4, 256).to(torch.bfloat16).cuda()
+    wr = torch.randn(8, 256).cuda()
+    with pytest.raises(moeq.MoeError) as ei:
+        moeq.moe_route_topk(x, wr, None, 9)
+    assert ei.value.code in (1, 2)
+    xp = torch.zeros(8, 256, dtype=torch.float16, device="cuda")
+    off = torch.zeros(9, dtype=torch.int32, device="cuda")
+    blobs = torch.zeros(8, moeq.moe_blob_bytes(256, 512, 64, 0), dtype=torch.uint8, device="cuda")
+    with pytest.raises(moeq.MoeError) as ei:
+        moeq.moe_grouped_ffn_wq(xp, off, blobs, 4, 8, 256, 512, 64, 0,
+                                workspace=torch.zeros(16, dtype=torch.uint8, device="cuda"))
+    assert ei.value.code == 6
+    with pytest.raises(moeq.MoeError) as ei:
+        moeq.moe_grouped_ffn_wq(xp, off, blobs, 4, 8, 256, 500, 64, 0)
+    assert ei.value.code == 2
