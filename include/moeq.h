@@ -128,7 +128,7 @@ MOE_API moe_status_t moe_quant_pack(const float* w_gate, const float* w_up, cons
  *   forced_idx int32 [T][k] or NULL: when given, the selection is taken
  *            from it as is (an external trace) and only topk_w is
  *            computed for it; topk_idx receives a copy.
- * Requires 1 <= k <= E <= 256, k <= 16, d % 8 == 0. */
+ * Requires 1 <= k <= E <= 256, k <= 16, d % 32 == 0. */
 MOE_API moe_status_t moe_route_topk(const void* x, const float* w_router, const float* bias,
                             const int32_t* forced_idx, int T, int d, int E, int k,
                             int32_t* topk_idx, float* topk_w, moe_stream_t stream);
@@ -235,6 +235,11 @@ MOE_API void moe_slot_cache_destroy(moe_slot_cache* cache);
  * (what = 1), or the cache's next copy reports a failed copy (what = 2).
  * what = 0 clears it. */
 MOE_API void moe_debug_inject_fault(int what, int count);
+
+/* Test hook: 0 = choose the FFN kernel by T (decode GEMV for T <= 8,
+ * tensor-core grouped GEMM above), 1 = always the decode GEMV, 2 = the
+ * tensor-core kernel whenever the shape allows it.  Process-wide. */
+MOE_API void moe_debug_force_regime(int regime);
 
 #ifdef __cplusplus
 }

@@ -72,6 +72,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // T <= 8.  Larger T goes to the tensor-core grouped GEMM.
 constexpr int kGemvMaxT = 8;
 
+// 0: pick by T; 1: always the decode GEMV; 2: tensor cores whenever possible.
+int g_force_regime = 0;
+
 size_t workspace_for(int total_rows, int F) {
   size_t h = static_cast<size_t>(total_rows) * F * sizeof(__half);
   return (h + 255) & ~static_cast<size_t>(255);
@@ -82,6 +85,8 @@ size_t workspace_for(int total_rows, int F) {
 extern "C" {
 
 const char* moe_last_error(void) { return g_err; }
+
+void moe_debug_force_regime(int regime) { g_force_regime = (regime >= 0 && regime <= 2) ? regime : 0; }
 
 size_t moe_blob_bytes(int d, int F, int group, int layout) {
   const BlobLayout L = blob_layout(d, F, group, layout);
@@ -214,8 +219,9 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   a.h = static_cast<__half*>(workspace);
   a.y_perm = y_perm;
   a.status = status;
-  if (T <= kGemvMaxT || !tc_supported(a)) return launch_ffn_gemv(a, S(stream));
-  return launch_ffn_tc(a, S(stream));
+  const bool tc_ok = total_rows >= 16 && tc_supported(a);
+  const bool use_tc = g_force_regime == 2 ? tc_ok : (g_force_regime == 1 ? false : (T > kGemvMaxT && tc_ok));
+  return use_tc ? launch_ffn_tc(a, S(stream)) : launch_ffn_gemv(a, S(stream));
 }
 
 moe_status_t moe_unpermute_combine(const float* y_perm, const int32_t* inv_perm,

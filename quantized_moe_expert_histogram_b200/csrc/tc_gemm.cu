@@ -1,18 +1,726 @@
-// Prefill-regime grouped expert FFN on the tcgen05 tensor cores.
+// Prefill-regime grouped expert FFN on the 5th-generation tensor cores.
+//
+// One persistent CTA per SM walks a tile list built on the device from the
+// bin offsets (no host sync).  A tile is (bin, token block, 128-row weight
+// block).  The MMA is issued "swap-AB": the 128 dequantised weight rows are
+// the M side (operand A, built in shared memory) and the bin's tokens are
+// the N side (operand B, fp16 activation rows loaded by TMA), so a bin of
+// any size is covered with at most 15 padded token columns, and
+// D[weight row][token] accumulates in TMEM (fp32).
+//
+// Warp roles (12 warps):
+//   warp 0      codes producer: packed codes (3-D tensor map over the blob
+//               pool, one box per 128 K) and their scale/zero words (1-D
+//               bulk copy)
+//   warp 3      activation producer: fp16 rows of the bin (16-row TMA
+//               boxes, 128B swizzle)
+//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=tokens,
+//               K=16) and tcgen05.commit
+//   warp 2      TMEM allocator (512 columns: two accumulator buffers)
+//   warps 4-7   dequantisers: thread i turns weight row i of a staged codes
+//               block into fp16 ((code - zero) * scale, one rounding) and
+//               writes it in the UMMA K-major 128B-swizzled layout
+//   warps 8-11  epilogue: tcgen05.ld of its TMEM lane quadrant; gate/up
+//               pass writes h = silu(gate) * up (fp16), down pass y_perm
+//               (fp32)
+// Pipelines: codes (4 stages of 128 K) -> dequant -> A/B (3 stages of 64 K)
+// -> MMA -> TMEM (2 buffers) -> epilogue.  Every wait is bounded; on a
+// timeout the CTA raises MOE_DEV_TIMEOUT, drains its copies and MMAs,
+// frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moeq {
+namespace {
+
+// ------------------------------------------------------------ PTX utils --
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: only reached when something is broken
+
+// Bounded wait.  Returns false when the CTA is aborting (flag set here on
+// timeout, or by another role).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        flag_status(status, MOE_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4}], [%5];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// UMMA shared-memory descriptor: K-major, 128B swizzle, 8-row atoms 1024 B
+// apart (SBO), version 1.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp16 A and B (K-major), fp32 D,
+// M = 128, N = n.
+__device__ __forceinline__ uint32_t umma_idesc_f16(int n) {
+  return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
+      "[%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------ config ----
+
+constexpr int kThreads = 384;
+constexpr int kMaxBins = 768;
+
+template <int NMAT, int NT_MAX>
+struct Cfg {
+  static constexpr int STAGES = 3;    // A/B stages of 64 K
+  static constexpr int CSTAGES = 4;   // codes stages of 128 K
+  static constexpr int A_BYTES = 128 * 128;      // 128 rows x 64 fp16
+  static constexpr int B_BYTES = NT_MAX * 128;   // NT rows x 64 fp16
+  static constexpr int C_BYTES = 8192;           // 128 rows x 128 K codes (either layout)
+  static constexpr int SZ_BYTES = 1024;          // 128 rows x up to 2 groups x 4 B
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * NMAT * A_BYTES;
+  static constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_SZ = OFF_C + CSTAGES * NMAT * C_BYTES;
+  static constexpr int OFF_TILE = OFF_SZ + CSTAGES * NMAT * SZ_BYTES;  // int tile_start[769], off[769]
+  static constexpr int OFF_BAR = OFF_TILE + 2 * (kMaxBins + 1) * 4 + 8;
+  static constexpr int N_BARS = 2 * CSTAGES + 3 * STAGES + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + alignment slack
+  static constexpr int TMEM_COLS = 512;
+  static_assert(2 * NMAT * NT_MAX <= TMEM_COLS, "TMEM budget");
+};
+
+struct TcParams {
+  CUtensorMap act;       // fp16 [rows][K], box 64 x 16, 128B swizzle
+  CUtensorMap codes[2];  // INT4: u32 [nblob][N][K/8];   PLANES: Q2 u32 [nblob][N][K/16]
+  CUtensorMap d3[2];     // PLANES only: u32 [nblob][N][K/32]
+  CUtensorMap d4[2];
+  const int32_t* offsets;
+  const int32_t* slot_of;
+  const uint8_t* blobs;
+  size_t blob_bytes;
+  size_t sz_off[2];
+  int K, N, nbins, planes_mult, group;
+  __half* h_out;
+  float* y_out;
+  int32_t* status;
+};
+
+struct Tile {
+  int bin, slot, bits, row0, nrows, nt, mb;
+};
+
+template <int NT_MAX>
+__device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const int* off, int nbins,
+                                            int MB, int planes_mult, const int32_t* slot_of) {
+  int lo = 0, hi = nbins;  // largest b with tile_start[b] <= t (tile_start[nbins] = total)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_start[mid] <= t) lo = mid; else hi = mid;
+  }
+  Tile T;
+  T.bin = lo;
+  const int local = t - tile_start[lo];
+  const int tb = local / MB;
+  T.mb = local - tb * MB;
+  const int n = off[lo + 1] - off[lo];
+  const int nb = (n + NT_MAX - 1) / NT_MAX;
+  const int per = (((n + nb - 1) / nb) + 15) & ~15;
+  T.row0 = off[lo] + tb * per;
+  T.nrows = min(per, n - tb * per);
+  T.nt = (T.nrows + 15) & ~15;
+  const int e = lo / planes_mult;
+  T.slot = slot_of ? slot_of[e] : e;
+  T.bits = planes_mult == 3 ? 2 + lo % 3 : 4;
+  return T;
+}
+
+// 8 two-bit fields -> bits 4i..4i+1 ; 8 one-bit fields -> bit 4i.
+__device__ __forceinline__ uint32_t spread2(uint32_t x) {
+  x &= 0xFFFFu;
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  x = (x | (x << 2)) & 0x33333333u;
+  return x;
+}
+__device__ __forceinline__ uint32_t spread1(uint32_t x) {
+  x &= 0xFFu;
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  x = (x | (x << 3)) & 0x11111111u;
+  return x;
+}
+
+// Eight 4-bit codes (nibble i = element i) -> four half2 (e0,e1)..(e6,e7)
+// holding (code - z) * s rounded once to fp16.
+__device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 zoff, __half2 s2) {
+  uint32_t v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t raw = ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;  // (1024+q_j, 1024+q_{j+4})
+    __half2 h = *reinterpret_cast<const __half2*>(&raw);
+    h = __hmul2(__hsub2(h, zoff), s2);
+    v[j] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  uint4 o;
+  o.x = __byte_perm(v[0], v[1], 0x5410);
+  o.y = __byte_perm(v[2], v[3], 0x5410);
+  o.z = __byte_perm(v[0], v[1], 0x7632);
+  o.w = __byte_perm(v[2], v[3], 0x7632);
+  return o;
+}
+
+template <int NMAT, int NT_MAX, bool PLANES>
+__global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ TcParams P) {
+  using C = Cfg<NMAT, NT_MAX>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int* tile_start = reinterpret_cast<int*>(smem + C::OFF_TILE);
+  int* off_s = tile_start + (kMaxBins + 1);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const uint32_t bar0 = smem_u32(bars);
+  auto codes_full = [&](int i) { return bar0 + 8u * i; };
+  auto codes_empty = [&](int i) { return bar0 + 8u * (C::CSTAGES + i); };
+  auto a_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + i); };
+  auto b_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + C::STAGES + i); };
+  auto ab_empty = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 2 * C::STAGES + i); };
+  auto acc_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + i); };
+  auto acc_empty = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 2 + i); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nbins = P.nbins;
+  const int MB = P.N / 128;
+  const int KC = P.K / 128;
+
+  // ---- set-up: barriers, TMEM, tile table --------------------------------
+  if (tid == 0) {
+    for (int i = 0; i < C::CSTAGES; ++i) {
+      mbar_init(codes_full(i), 1);
+      mbar_init(codes_empty(i), 4);
+    }
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(a_full(i), 4);
+      mbar_init(b_full(i), 1);
+      mbar_init(ab_empty(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full(i), 1);
+      mbar_init(acc_empty(i), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  for (int b = tid; b <= nbins; b += kThreads) off_s[b] = P.offsets[b];
+  __syncthreads();
+  if (warp == 0) {
+    // tiles per bin -> exclusive scan (lane owns a contiguous run of bins)
+    const int per_lane = (nbins + 31) / 32;
+    const int b0 = lane * per_lane;
+    int run = 0;
+    for (int i = 0; i < per_lane; ++i) {
+      const int b = b0 + i;
+      if (b < nbins) {
+        int n = off_s[b + 1] - off_s[b];
+        if (P.slot_of && P.slot_of[b / P.planes_mult] < 0) n = 0;
+        const int tiles = ((n + NT_MAX - 1) / NT_MAX) * MB;
+        tile_start[b] = run;  // lane-local exclusive prefix for now
+        run += tiles;
+      }
+    }
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int base = incl - run;
+    for (int i = 0; i < per_lane; ++i) {
+      const int b = b0 + i;
+      if (b < nbins) tile_start[b] += base;
+    }
+    if (lane == 31) tile_start[nbins] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = tile_start[nbins];
+
+  // ---- producers: codes (warp 0) and activations (warp 3) ----------------
+  if (warp == 0 || warp == 3) {
+    if (lane == 0) {
+      const bool codes_role = warp == 0;
+      int cs = 0, cph = 0, s = 0, sph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const Tile T = decode_tile<NT_MAX>(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
+        if (codes_role) {
+          const uint8_t* blob = P.blobs + static_cast<size_t>(T.slot) * P.blob_bytes;
+          const int gpc = 128 / P.group;  // groups per codes stage
+          const uint32_t sz_bytes = gpc * 512;
+          uint32_t code_bytes = 8192;
+          if (PLANES) code_bytes = 4096 + (T.bits >= 3 ? 2048 : 0) + (T.bits >= 4 ? 2048 : 0);
+          for (int kc = 0; kc < KC && ok; ++kc) {
+            ok = mbar_wait(codes_empty(cs), cph ^ 1, abort_flag, P.status);
+            if (!ok) break;
+            mbar_expect_tx(codes_full(cs), NMAT * (code_bytes + sz_bytes));
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+              const uint32_t cdst = smem_u32(smem + C::OFF_C + (cs * NMAT + m) * C::C_BYTES);
+              if (!PLANES) {
+                tma_load_3d(cdst, &P.codes[m], kc * 16, T.mb * 128, T.slot, codes_full(cs));
+              } else {
+                tma_load_3d(cdst, &P.codes[m], kc * 8, T.mb * 128, T.slot, codes_full(cs));
+                if (T.bits >= 3) tma_load_3d(cdst + 4096, &P.d3[m], kc * 4, T.mb * 128, T.slot, codes_full(cs));
+                if (T.bits >= 4) tma_load_3d(cdst + 6144, &P.d4[m], kc * 4, T.mb * 128, T.slot, codes_full(cs));
+              }
+              const uint8_t* szsrc = blob + P.sz_off[m] +
+                                     (static_cast<size_t>(T.mb) * (P.K / P.group) + kc * gpc) * 512;
+              bulk_load(smem_u32(smem + C::OFF_SZ + (cs * NMAT + m) * C::SZ_BYTES), szsrc, sz_bytes,
+                        codes_full(cs));
+            }
+            if (++cs == C::CSTAGES) { cs = 0; cph ^= 1; }
+          }
+        } else {
+          for (int kb = 0; kb < 2 * KC && ok; ++kb) {
+            ok = mbar_wait(ab_empty(s), sph ^ 1, abort_flag, P.status);
+            if (!ok) break;
+            mbar_expect_tx(b_full(s), T.nt * 128);
+            const uint32_t bdst = smem_u32(smem + C::OFF_B + s * C::B_BYTES);
+            for (int i = 0; i < T.nt / 16; ++i) tma_load_2d(bdst + i * 2048, &P.act, kb * 64, T.row0 + 16 * i, b_full(s));
+            if (++s == C::STAGES) { s = 0; sph ^= 1; }
+          }
+        }
+      }
+      if (!ok) {
+        // drain: the most recent arming of every stage must land before exit
+        const uint64_t t0 = global_ns();
+        if (codes_role) {
+          for (int idx = 0; idx < C::CSTAGES; ++idx) {
+            const int ph = (idx < cs) ? cph : cph ^ 1;
+            while (!mbar_try(codes_full(idx), ph) && global_ns() - t0 < kWaitLimitNs) {}
+          }
+        } else {
+          for (int idx = 0; idx < C::STAGES; ++idx) {
+            const int ph = (idx < s) ? sph : sph ^ 1;
+            while (!mbar_try(b_full(idx), ph) && global_ns() - t0 < kWaitLimitNs) {}
+          }
+        }
+      }
+    }
+  }
+  // ---- MMA issuer --------------------------------------------------------
+  else if (warp == 1) {
+    if (lane == 0) {
+      int s = 0, sph = 0, acc = 0, aph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const Tile T = decode_tile<NT_MAX>(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
+        const uint32_t idesc = umma_idesc_f16(T.nt);
+        ok = mbar_wait(acc_empty(acc), aph ^ 1, abort_flag, P.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t dcol = tmem_base + acc * (NMAT * NT_MAX);
+        for (int kb = 0; kb < 2 * KC && ok; ++kb) {
+          ok = mbar_wait(a_full(s), sph, abort_flag, P.status) && mbar_wait(b_full(s), sph, abort_flag, P.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::OFF_B + s * C::B_BYTES));
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) {
+            const uint64_t adesc = umma_desc_sw128(smem_u32(smem + C::OFF_A + (s * NMAT + m) * C::A_BYTES));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f16(dcol + m * NT_MAX, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          }
+          umma_commit(ab_empty(s));
+          if (++s == C::STAGES) { s = 0; sph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(acc_full(acc));
+        if (++acc == 2) { acc = 0; aph ^= 1; }
+      }
+      // all MMAs issued by this thread complete before TMEM is released
+      umma_commit(drain_bar);
+      const uint64_t t0 = global_ns();
+      while (!mbar_try(drain_bar, 0) && global_ns() - t0 < kWaitLimitNs) {}
+    }
+  }
+  // ---- dequantisers ------------------------------------------------------
+  else if (warp >= 4 && warp < 8) {
+    const int i = tid - 128;  // weight row inside the 128-row block
+    int cs = 0, cph = 0, s = 0, sph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      const Tile T = decode_tile<NT_MAX>(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
+      for (int kc = 0; kc < KC && ok; ++kc) {
+        ok = mbar_wait(codes_full(cs), cph, abort_flag, P.status);
+        if (!ok) break;
+        uint32_t w[NMAT][16];
+        uint32_t sz[NMAT][2];
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+          const uint8_t* cb = smem + C::OFF_C + (cs * NMAT + m) * C::C_BYTES;
+          if (!PLANES) {
+            // row i: 64 B = 4 chunks, 64B swizzle: chunk j at j ^ ((i >> 1) & 3)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 v = *reinterpret_cast<const uint4*>(cb + i * 64 + ((j ^ ((i >> 1) & 3)) << 4));
+              w[m][4 * j] = v.x; w[m][4 * j + 1] = v.y; w[m][4 * j + 2] = v.z; w[m][4 * j + 3] = v.w;
+            }
+          } else {
+            // Q2 row i: 32 B = 2 chunks, 32B swizzle: chunk j at j ^ ((i >> 2) & 1)
+            uint32_t q2[8];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const uint4 v = *reinterpret_cast<const uint4*>(cb + i * 32 + ((j ^ ((i >> 2) & 1)) << 4));
+              q2[4 * j] = v.x; q2[4 * j + 1] = v.y; q2[4 * j + 2] = v.z; q2[4 * j + 3] = v.w;
+            }
+            uint4 r3 = make_uint4(0, 0, 0, 0), r4 = make_uint4(0, 0, 0, 0);
+            if (T.bits >= 3) r3 = *reinterpret_cast<const uint4*>(cb + 4096 + i * 16);
+            if (T.bits >= 4) r4 = *reinterpret_cast<const uint4*>(cb + 6144 + i * 16);
+            const uint32_t d3w[4] = {r3.x, r3.y, r3.z, r3.w};
+            const uint32_t d4w[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+            for (int wd = 0; wd < 16; ++wd) {  // word wd = elements 8wd..8wd+7
+              const uint32_t base = q2[wd >> 1] >> (16 * (wd & 1));
+              const uint32_t b3 = d3w[wd >> 2] >> (8 * (wd & 3));
+              const uint32_t b4 = d4w[wd >> 2] >> (8 * (wd & 3));
+              w[m][wd] = (spread2(base) << 2) | (spread1(b3) << 1) | spread1(b4);
+            }
+          }
+          const uint32_t* szb = reinterpret_cast<const uint32_t*>(smem + C::OFF_SZ + (cs * NMAT + m) * C::SZ_BYTES);
+          sz[m][0] = szb[i];
+          sz[m][1] = (P.group == 64) ? szb[128 + i] : sz[m][0];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(codes_empty(cs));
+        if (++cs == C::CSTAGES) { cs = 0; cph ^= 1; }
+        for (int h = 0; h < 2 && ok; ++h) {
+          ok = mbar_wait(ab_empty(s), sph ^ 1, abort_flag, P.status);
+          if (!ok) break;
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) {
+            // the 64 elements of half h lie in group (h * 64) / group of the stage
+            const uint32_t word = sz[m][h];
+            const __half sc = __float2half_rn(__uint_as_float(word << 16));
+            const float zf = __uint_as_float(word & 0xFFFF0000u);
+            const __half2 s2 = __half2half2(sc);
+            const __half2 z2 = __half2half2(__float2half_rn(1024.0f + zf));
+            uint8_t* arow = smem + C::OFF_A + (s * NMAT + m) * C::A_BYTES + i * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = elements 8j..8j+7 of the half
+              const uint4 o = dequant8(w[m][8 * h + j], z2, s2);
+              *reinterpret_cast<uint4*>(arow + ((j ^ (i & 7)) << 4)) = o;
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(a_full(s));
+          if (++s == C::STAGES) { s = 0; sph ^= 1; }
+        }
+      }
+    }
+  }
+  // ---- epilogue ----------------------------------------------------------
+  else if (warp >= 8) {
+    const int q = warp & 3;  // TMEM lane quadrant
+    int acc = 0, aph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      const Tile T = decode_tile<NT_MAX>(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
+      ok = mbar_wait(acc_full(acc), aph, abort_flag, P.status);
+      if (!ok) break;
+      tc_fence_after();
+      const int row = T.mb * 128 + 32 * q + lane;  // output feature of this thread
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * (NMAT * NT_MAX);
+      for (int j0 = 0; j0 < T.nrows; j0 += 16) {
+        uint32_t g[16];
+        tmem_ld16(tbase + j0, g);
+        if (NMAT == 2) {
+          uint32_t u[16];
+          tmem_ld16(tbase + NT_MAX + j0, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (j0 + j < T.nrows) {
+              const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
+              P.h_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + row] = __float2half_rn(silu_f(gv) * uv);
+            }
+          }
+        } else {
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j0 + j < T.nrows)
+              P.y_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + row] = __uint_as_float(g[j]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty(acc));
+      if (++acc == 2) { acc = 0; aph ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------ host side --
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+            const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// act: fp16 [rows][K]; weight matrices m of the pass (N x K each).
+moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int rows, int K, int N,
+                         const int* mats, int nmat, int n_blobs) {
+  const bool planes = a.layout == MOE_LAYOUT_PLANES;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t str[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {64, 16};
+    if (!encode(&P.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, act, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) {
+      set_error("tensor map (activations) could not be encoded");
+      return MOE_ERR_CUDA;
+    }
+  }
+  for (int i = 0; i < nmat; ++i) {
+    const int m = mats[i];
+    if (!planes) {
+      cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 8), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_blobs)};
+      cuuint64_t str[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(a.blob_bytes)};
+      cuuint32_t box[3] = {16, 128, 1};
+      if (!encode(&P.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.codes[m], dims, str, box,
+                  CU_TENSOR_MAP_SWIZZLE_64B)) {
+        set_error("tensor map (codes) could not be encoded");
+        return MOE_ERR_CUDA;
+      }
+    } else {
+      cuuint64_t dq[3] = {static_cast<cuuint64_t>(K / 16), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_blobs)};
+      cuuint64_t sq[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(a.blob_bytes)};
+      cuuint32_t bq[3] = {8, 128, 1};
+      cuuint64_t dr[3] = {static_cast<cuuint64_t>(K / 32), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_blobs)};
+      cuuint64_t sr[2] = {static_cast<cuuint64_t>(K / 8), static_cast<cuuint64_t>(a.blob_bytes)};
+      cuuint32_t br[3] = {4, 128, 1};
+      if (!encode(&P.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.q2[m], dq, sq, bq,
+                  CU_TENSOR_MAP_SWIZZLE_32B) ||
+          !encode(&P.d3[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.d3[m], dr, sr, br,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+          !encode(&P.d4[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.d4[m], dr, sr, br,
+                  CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        set_error("tensor map (bit planes) could not be encoded");
+        return MOE_ERR_CUDA;
+      }
+    }
+    P.sz_off[i] = a.lay.sz[m];
+  }
+  P.offsets = a.offsets;
+  P.slot_of = a.slot_of;
+  P.blobs = a.blobs;
+  P.blob_bytes = a.blob_bytes;
+  P.K = K;
+  P.N = N;
+  P.planes_mult = planes ? 3 : 1;
+  P.nbins = a.E * P.planes_mult;
+  P.group = a.group;
+  P.status = a.status;
+  return MOE_OK;
+}
+
+template <int NMAT, int NT_MAX, bool PLANES>
+moe_status_t launch_one(const TcParams& P, cudaStream_t s) {
+  using C = Cfg<NMAT, NT_MAX>;
+  auto kern = k_ffn_tc<NMAT, NT_MAX, PLANES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return cuda_check(e, "tc ffn smem attribute");
+  kern<<<sm_count(), kThreads, C::SMEM, s>>>(P);
+  return cuda_check(cudaGetLastError(), "tc ffn launch");
+}
+
+}  // namespace
 
 bool tc_supported(const FfnArgs& a) {
-  (void)a;
-  return false;
+  return get_encode() != nullptr && a.d % 128 == 0 && a.F % 128 == 0 && a.E * (a.layout == MOE_LAYOUT_PLANES ? 3 : 1) <= kMaxBins;
 }
 
 moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s) {
-  (void)a;
-  (void)s;
-  set_error("tensor-core FFN path not available for this shape");
-  return MOE_ERR_UNSUPPORTED_SHAPE;
+  const int n_blobs = a.slot_of ? 65536 : a.E;
+  const bool planes = a.layout == MOE_LAYOUT_PLANES;
+  TcParams gu{};
+  const int m_gu[2] = {0, 1};
+  moe_status_t st = make_params(gu, a, a.x_perm, a.total_rows, a.d, a.F, m_gu, 2, n_blobs);
+  if (st != MOE_OK) return st;
+  gu.h_out = a.h;
+  gu.y_out = nullptr;
+  st = planes ? launch_one<2, 128, true>(gu, s) : launch_one<2, 128, false>(gu, s);
+  if (st != MOE_OK) return st;
+  TcParams dn{};
+  const int m_dn[1] = {2};
+  st = make_params(dn, a, a.h, a.total_rows, a.F, a.d, m_dn, 1, n_blobs);
+  if (st != MOE_OK) return st;
+  dn.h_out = nullptr;
+  dn.y_out = a.y_perm;
+  return planes ? launch_one<1, 256, true>(dn, s) : launch_one<1, 256, false>(dn, s);
 }
 
 }  // namespace moeq

@@ -45,6 +45,7 @@ _SIGS = {
                             _c_p, _c_p, _c_p]),
     "moe_slot_cache_destroy": (None, [_c_p]),
     "moe_debug_inject_fault": (None, [_c_i, _c_i]),
+    "moe_debug_force_regime": (None, [_c_i]),
 }
 
 _lib = None
@@ -251,3 +252,8 @@ def moe_debug_inject_fault(what, count):
 
 def moe_last_error():
     return load().moe_last_error().decode()
+
+
+def moe_debug_force_regime(regime):
+    """0 = by T, 1 = decode GEMV, 2 = tensor cores (test hook)."""
+    load().moe_debug_force_regime(regime)
