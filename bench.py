@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--sweep", default="1,16,256", help="extra token counts timed for context ('' = none)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=0)
+    p.add_argument("--profile", action="store_true",
+                   help="profiling driver: one instance, warmup + steps of the eager step, no JSON")
     return p.parse_args()
 
 
@@ -172,38 +174,50 @@ def algorithmic(shape, T, layer, bits_present):
     return bytes_w + act, flops
 
 
-def time_steps(layers, steps, warmup, stream, ffn_events=True):
-    """Run warmup + timed steps; returns (total ms, mean FFN ms per step)."""
+def _step_calls(layer, x, bits, stream, part):
+    """The ABI calls of one step: part 'all', or 'ffn' (the FFN call only)."""
+    from quantized_moe_expert_histogram_b200 import moeq
+    T = x.shape[0]
+    v = layer.views(T)
+    if part == "all":
+        moeq.moe_route_topk(x, layer.w_router, layer.bias, layer.k, topk_idx=v["topk_idx"],
+                            topk_w=v["topk_w"], workspace=v["route_ws"], stream=stream)
+        moeq.moe_permute(v["topk_idx"], layer.E, bits=bits, x=x, out=v, status=v["status"], stream=stream)
+    moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, T, layer.E, layer.d, layer.F,
+                            layer.group, layer.layout, workspace=v["workspace"], y_perm=v["y_perm"],
+                            status=v["status"], stream=stream)
+    if part == "all":
+        moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], y=v["y"], stream=stream)
+
+
+def capture(layers, stream, part):
+    """One CUDA graph running the steps of all R instances back to back."""
     import torch
-    R = len(layers)
-    for i in range(warmup):
-        layer, x, bits = layers[i % R]
-        layer.forward(x, bits=bits, stream=stream)
+    for layer, x, bits in layers:  # eager pass first (sets kernel attributes, routing for 'ffn')
+        _step_calls(layer, x, bits, stream, "all")
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for layer, x, bits in layers:
+            _step_calls(layer, x, bits, stream, part)
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(g, replays, warmup, stream):
+    import torch
+    for _ in range(warmup):
+        g.replay()
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    fs = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    fe = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    from quantized_moe_expert_histogram_b200 import moeq
-    start.record(stream)
-    for i in range(steps):
-        layer, x, bits = layers[i % R]
-        T = x.shape[0]
-        v = layer.views(T)
-        moeq.moe_route_topk(x, layer.w_router, layer.bias, layer.k, topk_idx=v["topk_idx"],
-                            topk_w=v["topk_w"], stream=stream)
-        moeq.moe_permute(v["topk_idx"], layer.E, bits=bits, x=x, out=v, status=v["status"], stream=stream)
-        fs[i].record(stream)
-        moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, T, layer.E, layer.d, layer.F,
-                                layer.group, layer.layout, workspace=v["workspace"], y_perm=v["y_perm"],
-                                status=v["status"], stream=stream)
-        fe[i].record(stream)
-        moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], y=v["y"], stream=stream)
-    end.record(stream)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(replays):
+            g.replay()
+        end.record(stream)
     torch.cuda.synchronize()
-    total = start.elapsed_time(end)
-    ffn = sum(a.elapsed_time(b) for a, b in zip(fs, fe)) / steps
-    return total, ffn
+    return start.elapsed_time(end)
 
 
 def time_e2e(layers, steps, stream):
@@ -311,22 +325,36 @@ def main():
     T = args.tokens
     peaks = load_peaks()
     stream = torch.cuda.Stream()
+    if args.profile:
+        layers = make_instances(shape, T, 1, seed=0, device="cuda")
+        for _ in range(args.warmup + args.steps):
+            _step_calls(*layers[0], stream, "all")
+        torch.cuda.synchronize()
+        print(f"profile run done: {shape.name} T={T} steps={args.warmup + args.steps}")
+        return
     layers = make_instances(shape, T, args.instances, seed=rank * 7919, device="cuda")
     torch.cuda.synchronize()
 
+    R = len(layers)
+    replays = max(1, (args.steps + R - 1) // R)
+    steps = replays * R
+    g_all = capture(layers, stream, "all")
+    g_ffn = capture(layers, stream, "ffn")
     barrier(world)
     clocks = ClockSampler(local)
     clocks.start()
     torch.cuda.synchronize()
-    total_ms, ffn_ms = time_steps(layers, args.steps, args.warmup, stream)
+    total_ms = time_graph(g_all, replays, max(1, args.warmup // R + 1), stream)
     clk = clocks.stop()
+    ffn_total = time_graph(g_ffn, replays, 1, stream)
+    ffn_ms = ffn_total / steps
     barrier(world)
     total_ms = max_over_ranks(world, total_ms)
-    ms_per_step = total_ms / args.steps
-    value = world * T * args.steps / (total_ms / 1e3)
+    ms_per_step = total_ms / steps
+    value = world * T * steps / (total_ms / 1e3)
+    del g_all, g_ffn
 
-    bytes_alg, flops = algorithmic(shape, T, layers[(args.steps - 1) % len(layers)][0],
-                                   layers[0][2] is not None)
+    bytes_alg, flops = algorithmic(shape, T, layers[-1][0], layers[0][2] is not None)
     t_ffn = ffn_ms / 1e3
     tc_bound = flops / (peaks["tc"] * 1e12) > bytes_alg / (peaks["hbm"] * 1e9)
     if tc_bound:
@@ -337,24 +365,27 @@ def main():
         ach = bytes_alg / t_ffn / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s", "frac": ach / peaks["hbm"]}
     roof.update({"traffic": None, "kernel": "moe_grouped_ffn_wq (gate/up + down launches)",
+                 "timing": "FFN-only CUDA graph over the same rotated instances, events around the replays",
                  "peak_source": peaks["src"], "ffn_ms": ffn_ms,
                  "per_launch_units": f"{T * shape.k} assignments"})
 
-    e2e_ms, h2d, d2h = time_e2e(layers, args.steps, stream)
+    e2e_ms, h2d, d2h = time_e2e(layers, steps, stream)
     e2e_ms = max_over_ranks(world, e2e_ms)
-    e2e = {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+    e2e = {"value": world * T * steps / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     sweep = {}
-    for tok in [int(s) for s in args.sweep.split(",") if s.strip()]:
+    for tok in [int(x) for x in args.sweep.split(",") if x.strip()]:
         ls = make_instances(shape, tok, 16, seed=rank * 7919 + 17, device="cuda")
-        tot, fm = time_steps(ls, max(args.steps, 50), args.warmup, stream)
+        ga, gf = capture(ls, stream, "all"), capture(ls, stream, "ffn")
+        rep = max(4, 64 // len(ls))
+        tot = time_graph(ga, rep, 2, stream) / (rep * len(ls))
+        fm = time_graph(gf, rep, 1, stream) / (rep * len(ls))
         b, fl = algorithmic(shape, tok, ls[-1][0], ls[0][2] is not None)
-        sweep[str(tok)] = {"tokens_per_s": tok * max(args.steps, 50) / (tot / 1e3),
-                           "ms_per_step": tot / max(args.steps, 50), "ffn_ms": fm,
+        sweep[str(tok)] = {"tokens_per_s": tok / (tot / 1e3), "ms_per_step": tot, "ffn_ms": fm,
                            "ffn_hbm_frac": b / (fm / 1e3) / 1e9 / peaks["hbm"],
                            "ffn_tc_frac": fl / (fm / 1e3) / 1e12 / peaks["tc"]}
-        del ls
+        del ls, ga, gf
         torch.cuda.empty_cache()
 
     cpu = None
@@ -362,7 +393,7 @@ def main():
         cpu = cpu_baseline(shape, T, 0, args.cpu_sample_tokens)
 
     launches_per_step = 6
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
             "config": {"workload": f"{shape.name} MoE layer d={shape.d} E={shape.E} top-{shape.k} "
@@ -370,7 +401,7 @@ def main():
                        "global_batch": T * world, "parallelism": f"replicas x{world}",
                        "l2": f"{args.instances} layer instances rotated ({shape.E} experts x "
                              f"{moeq.moe_blob_bytes(shape.d, shape.F, shape.group, 0)} B each), inputs > L2"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * steps,
             "clocks": clk, "sweep": sweep}
     if rank == 0:
         print(json.dumps(line))

@@ -128,10 +128,16 @@ MOE_API moe_status_t moe_quant_pack(const float* w_gate, const float* w_up, cons
  *   forced_idx int32 [T][k] or NULL: when given, the selection is taken
  *            from it as is (an external trace) and only topk_w is
  *            computed for it; topk_idx receives a copy.
+ *   workspace >= moe_route_workspace_bytes(T, d, E) bytes of device
+ *            scratch, 16-byte aligned (x and w_router too).
  * Requires 1 <= k <= E <= 256, k <= 16, d % 32 == 0. */
 MOE_API moe_status_t moe_route_topk(const void* x, const float* w_router, const float* bias,
                             const int32_t* forced_idx, int T, int d, int E, int k,
-                            int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+                            int32_t* topk_idx, float* topk_w, void* workspace,
+                            size_t workspace_bytes, moe_stream_t stream);
+
+/* Device scratch moe_route_topk needs (per-slice fp64 partial logits). */
+MOE_API size_t moe_route_workspace_bytes(int T, int d, int E);
 
 /* moe_permute -- per-expert histogram, exclusive prefix sum and stable
  * permutation of the T*k assignments a = t*k + j ([Read-ME] expert-aware

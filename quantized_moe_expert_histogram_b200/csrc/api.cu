@@ -112,9 +112,12 @@ moe_status_t moe_quant_pack(const float* w_gate, const float* w_up, const float*
   return launch_pack(w_gate, w_up, w_down, E, d, F, group, layout, blobs, S(stream));
 }
 
+size_t moe_route_workspace_bytes(int T, int d, int E) { return route_workspace_bytes(T, d, E); }
+
 moe_status_t moe_route_topk(const void* x, const float* w_router, const float* bias,
                             const int32_t* forced_idx, int T, int d, int E, int k,
-                            int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+                            int32_t* topk_idx, float* topk_w, void* workspace,
+                            size_t workspace_bytes, moe_stream_t stream) {
   if (T < 0 || d <= 0 || E <= 0 || k <= 0) {
     set_error("moe_route_topk: bad sizes T=%d d=%d E=%d k=%d", T, d, E, k);
     return MOE_ERR_INVALID_ARG;
@@ -131,7 +134,17 @@ moe_status_t moe_route_topk(const void* x, const float* w_router, const float* b
     set_error("moe_route_topk: d=%d must be a multiple of 32", d);
     return MOE_ERR_UNSUPPORTED_SHAPE;
   }
-  return launch_route(x, w_router, bias, forced_idx, T, d, E, k, topk_idx, topk_w, S(stream));
+  if (T > 0 && (!workspace || workspace_bytes < route_workspace_bytes(T, d, E))) {
+    set_error("moe_route_topk: workspace %zu < %zu bytes", workspace_bytes,
+              route_workspace_bytes(T, d, E));
+    return MOE_ERR_WORKSPACE;
+  }
+  if (T > 0 && (!aligned16(x) || !aligned16(w_router) || !aligned16(workspace))) {
+    set_error("moe_route_topk: x, w_router and workspace must be 16-byte aligned");
+    return MOE_ERR_INVALID_ARG;
+  }
+  return launch_route(x, w_router, bias, forced_idx, T, d, E, k, topk_idx, topk_w, workspace,
+                      S(stream));
 }
 
 moe_status_t moe_permute(const int32_t* topk_idx, const uint8_t* bits, const void* x, int T,

@@ -59,7 +59,8 @@ moe_status_t launch_pack(const float* w_gate, const float* w_up, const float* w_
                          int F, int group, int layout, void* blobs, cudaStream_t s);
 moe_status_t launch_route(const void* x, const float* w_router, const float* bias,
                           const int32_t* forced, int T, int d, int E, int k, int32_t* idx,
-                          float* w, cudaStream_t s);
+                          float* w, void* workspace, cudaStream_t s);
+size_t route_workspace_bytes(int T, int d, int E);
 moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void* x, int T, int d,
                             int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
                             int32_t* inv_perm, void* x_perm, int32_t* status, cudaStream_t s);

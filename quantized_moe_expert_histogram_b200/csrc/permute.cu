@@ -45,8 +45,9 @@ __global__ void __launch_bounds__(kWarps * 32) k_permute(const int32_t* __restri
                                                           int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ perm,
                                                           int32_t* __restrict__ inv_perm,
-                                                          int32_t* status) {
-  extern __shared__ int32_t hist[];  // [kWarps][nbins]
+                                                          int32_t* status, int stage_perm) {
+  extern __shared__ int32_t hist[];  // [kWarps][nbins], then perm staging [n] when stage_perm
+  int32_t* perm_s = hist + kWarps * nbins;
   __shared__ int32_t scan_buf[kWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const unsigned lt_mask = (1u << lane) - 1u;
@@ -113,39 +114,52 @@ __global__ void __launch_bounds__(kWarps * 32) k_permute(const int32_t* __restri
     const unsigned peers = __match_any_sync(0xffffffffu, key);
     if (valid) {
       const int p = my[key] + __popc(peers & lt_mask);
-      perm[p] = a;
+      if (stage_perm) perm_s[p] = a; else perm[p] = a;
       inv_perm[a] = p;
     }
     __syncwarp();
     if (valid && (peers & lt_mask) == 0) my[key] += __popc(peers);
     __syncwarp();
   }
+  if (stage_perm) {  // scattered positions land in shared memory; write out coalesced
+    __syncthreads();
+    for (int i = tid; i < n; i += blockDim.x) perm[i] = perm_s[i];
+  }
 }
 
-// x_perm[p] = fp16(x[perm[p] / k]); one thread moves 8 elements (16 bytes).
+// x_perm[p] = fp16(x[perm[p] / k]); a warp moves one row, 16 bytes per lane
+// per step with up to four independent loads in flight.
 __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict__ x,
                                                  const int32_t* __restrict__ perm, int rows, int k,
                                                  int d, __half* __restrict__ x_perm,
                                                  int32_t* status) {
-  const int vec_per_row = d / 8;
-  const long total = static_cast<long>(rows) * vec_per_row;
+  const int lane = threadIdx.x & 31;
+  const int vec = d / 8;
   bool bad = false;
-  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<long>(gridDim.x) * blockDim.x) {
-    const int p = static_cast<int>(i / vec_per_row);
-    const int c = static_cast<int>(i % vec_per_row);
+  for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < rows; p += (gridDim.x * blockDim.x) >> 5) {
     const int t = perm[p] / k;
-    const uint4 v = *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d + c * 8);
-    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-    uint4 o;
-    __half2* h2 = reinterpret_cast<__half2*>(&o);
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(p) * d);
+    for (int c0 = lane; c0 < vec; c0 += 128) {
+      uint4 v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __bfloat1622float2(b2[j]);
-      bad |= fabsf(f.x) > 65504.0f || fabsf(f.y) > 65504.0f;
-      h2[j] = __floats2half2_rn(f.x, f.y);
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 32 * u < vec) v[u] = src[c0 + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (c0 + 32 * u >= vec) break;
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+        uint4 o;
+        __half2* h2 = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(b2[j]);
+          bad |= fabsf(f.x) > 65504.0f || fabsf(f.y) > 65504.0f;
+          h2[j] = __floats2half2_rn(f.x, f.y);
+        }
+        dst[c0 + 32 * u] = o;
+      }
     }
-    *reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(p) * d + c * 8) = o;
   }
   if (bad) flag_status(status, MOE_DEV_RANGE);
 }
@@ -161,16 +175,25 @@ moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void*
     set_error("moe_permute: %d bins exceed %d", nbins, kMaxBins);
     return MOE_ERR_UNSUPPORTED_SHAPE;
   }
-  const size_t smem = sizeof(int32_t) * kWarps * nbins;
-  cudaError_t e = cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return cuda_check(e, "moe_permute smem attribute");
+  // Shared memory: per-warp histograms, plus the permutation itself when it
+  // fits, so that its scattered positions are written to shared memory and
+  // leave the SM as coalesced rows.
+  constexpr size_t kSmemCap = 226 * 1024;  // 227 KB per block, less the static scan buffer
+  const size_t hist_bytes = sizeof(int32_t) * kWarps * nbins;
+  const int stage = hist_bytes + sizeof(int32_t) * static_cast<size_t>(n) <= kSmemCap;
+  const size_t smem = hist_bytes + (stage ? sizeof(int32_t) * static_cast<size_t>(n) : 0);
+  static bool attr_set = false;  // once per process, to the cap
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemCap));
+    if (e != cudaSuccess) return cuda_check(e, "moe_permute smem attribute");
+    attr_set = true;
+  }
   k_permute<<<1, kWarps * 32, smem, s>>>(idx, bits, n, E, nbins, counts, offsets, perm, inv_perm,
-                                         status);
+                                         status, stage);
   moe_status_t st = cuda_check(cudaGetLastError(), "moe_permute launch");
   if (st != MOE_OK || !x_perm || n == 0) return st;
-  const long vecs = static_cast<long>(n) * (d / 8);
-  const int blocks = static_cast<int>(std::min<long>((vecs + 255) / 256, 148L * 16));
+  const int blocks = static_cast<int>(std::min<long>((static_cast<long>(n) + 7) / 8, 148L * 8));
   k_gather<<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), perm, n, k, d,
                                   static_cast<__half*>(x_perm), status);
   return cuda_check(cudaGetLastError(), "moe_permute gather launch");

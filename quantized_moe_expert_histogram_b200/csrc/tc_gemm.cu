@@ -691,8 +691,13 @@ template <int NMAT, int NT_MAX, bool PLANES>
 moe_status_t launch_one(const TcParams& P, cudaStream_t s) {
   using C = Cfg<NMAT, NT_MAX>;
   auto kern = k_ffn_tc<NMAT, NT_MAX, PLANES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return cuda_check(e, "tc ffn smem attribute");
+  // Set once per process (the first call must precede any stream capture).
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return cuda_check(e, "tc ffn smem attribute");
+    attr_set = true;
+  }
   kern<<<sm_count(), kThreads, C::SMEM, s>>>(P);
   return cuda_check(cudaGetLastError(), "tc ffn launch");
 }

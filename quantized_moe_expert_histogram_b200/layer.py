@@ -46,6 +46,8 @@ class QuantMoELayer:
                                   dtype=torch.uint8, device=dev),
             y=torch.empty(T, d, dtype=torch.bfloat16, device=dev),
             status=torch.zeros(1, dtype=torch.int32, device=dev),
+            route_ws=torch.empty(max(256, moeq.moe_route_workspace_bytes(T, d, self.E)), dtype=torch.uint8,
+                                 device=dev),
         )
 
     def views(self, T):
@@ -54,7 +56,7 @@ class QuantMoELayer:
         return dict(topk_idx=b["topk_idx"][:T], topk_w=b["topk_w"][:T], counts=b["counts"],
                     offsets=b["offsets"], perm=b["perm"][:rows], inv_perm=b["inv_perm"][:rows],
                     x_perm=b["x_perm"][:rows], y_perm=b["y_perm"][:rows], workspace=b["workspace"],
-                    y=b["y"][:T], status=b["status"])
+                    y=b["y"][:T], status=b["status"], route_ws=b["route_ws"])
 
     def forward(self, x, bits=None, forced_idx=None, residual=None, stream=None):
         T = x.shape[0]
@@ -62,7 +64,8 @@ class QuantMoELayer:
             raise ValueError(f"T={T} exceeds max_tokens={self.max_tokens}")
         v = self.views(T)
         moeq.moe_route_topk(x, self.w_router, self.bias, self.k, forced_idx=forced_idx,
-                            topk_idx=v["topk_idx"], topk_w=v["topk_w"], stream=stream)
+                            topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"],
+                            stream=stream)
         moeq.moe_permute(v["topk_idx"], self.E, bits=bits, x=x, out=v, status=v["status"], stream=stream)
         moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], self.blobs, T, self.E, self.d, self.F,
                                 self.group, self.layout, workspace=v["workspace"], y_perm=v["y_perm"],

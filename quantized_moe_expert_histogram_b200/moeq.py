@@ -32,7 +32,9 @@ _SIGS = {
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_blob_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
     "moe_quant_pack": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p]),
-    "moe_route_topk": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]),
+    "moe_route_topk": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p, _c_sz,
+                              _c_p]),
+    "moe_route_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
     "moe_permute": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_p,
                            _c_p, _c_p]),
     "moe_ffn_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
@@ -129,7 +131,12 @@ def moe_quant_pack(w_gate, w_up, w_down, group, layout, blobs=None, stream=None)
     return blobs
 
 
-def moe_route_topk(x, w_router, bias, k, forced_idx=None, topk_idx=None, topk_w=None, stream=None):
+def moe_route_workspace_bytes(T, d, E):
+    return int(load().moe_route_workspace_bytes(T, d, E))
+
+
+def moe_route_topk(x, w_router, bias, k, forced_idx=None, topk_idx=None, topk_w=None, workspace=None,
+                   stream=None):
     lib = load()
     T, d = x.shape
     E = w_router.shape[0]
@@ -137,11 +144,13 @@ def moe_route_topk(x, w_router, bias, k, forced_idx=None, topk_idx=None, topk_w=
         topk_idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(lib.moe_route_workspace_bytes(T, d, E), dtype=torch.uint8, device=x.device)
     _check("moe_route_topk", lib.moe_route_topk(
         _ptr(x, torch.bfloat16, "x"), _ptr(w_router, torch.float32, "w_router"),
         _ptr(bias, torch.float32, "bias"), _ptr(forced_idx, torch.int32, "forced_idx"), T, d, E, k,
         _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
-        _stream(stream)))
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return topk_idx, topk_w
 
 
