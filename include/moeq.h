@@ -247,6 +247,13 @@ MOE_API void moe_debug_inject_fault(int what, int count);
  * tensor-core kernel whenever the shape allows it.  Process-wide. */
 MOE_API void moe_debug_force_regime(int regime);
 
+/* Test hook: when non-NULL, the tensor-core FFN kernels record each warp
+ * role's progress into this pinned, device-mapped host buffer of
+ * 2 * gridDim * 16 ints (slot = (wait site << 24) | (tile << 12) | k-block),
+ * so that a stalled launch can be read from the host while it runs.
+ * NULL (the default) disables it. */
+MOE_API void moe_debug_set_trace(void* host_mapped_ints);
+
 #ifdef __cplusplus
 }
 #endif

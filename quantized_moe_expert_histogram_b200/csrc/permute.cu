@@ -21,6 +21,7 @@ namespace {
 
 constexpr int kWarps = 32;
 constexpr int kMaxBins = 768;
+constexpr int kBatch = 16;  // 32-assignment slices whose keys are loaded together
 
 __device__ __forceinline__ int load_key(const int32_t* idx, const uint8_t* bits, int a, int E,
                                         int32_t* status) {
@@ -60,13 +61,21 @@ __global__ void __launch_bounds__(kWarps * 32) k_permute(const int32_t* __restri
   const int end = min(n, begin + chunk);
   int32_t* my = hist + warp * nbins;
 
-  for (int base = begin; base < end; base += 32) {
-    const int a = base + lane;
-    const bool valid = a < end;
-    const int key = valid ? load_key(idx, bits, a, E, status) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    if (valid && (peers & lt_mask) == 0) my[key] += __popc(peers);
-    __syncwarp();
+  // Keys are fetched kBatch slices at a time (independent loads in flight),
+  // then consumed slice by slice.
+  for (int base = begin; base < end; base += 32 * kBatch) {
+    int keys[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int a = base + 32 * u + lane;
+      keys[u] = a < end ? load_key(idx, bits, a, E, status) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const unsigned peers = __match_any_sync(0xffffffffu, keys[u]);
+      if (keys[u] >= 0 && (peers & lt_mask) == 0) my[keys[u]] += __popc(peers);
+      __syncwarp();
+    }
   }
   __syncthreads();
 
@@ -107,19 +116,27 @@ __global__ void __launch_bounds__(kWarps * 32) k_permute(const int32_t* __restri
   if (tid == 0) offsets[nbins] = n;
   __syncthreads();
 
-  for (int base = begin; base < end; base += 32) {
-    const int a = base + lane;
-    const bool valid = a < end;
-    const int key = valid ? load_key(idx, bits, a, E, nullptr) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    if (valid) {
-      const int p = my[key] + __popc(peers & lt_mask);
-      if (stage_perm) perm_s[p] = a; else perm[p] = a;
-      inv_perm[a] = p;
+  for (int base = begin; base < end; base += 32 * kBatch) {
+    int keys[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int a = base + 32 * u + lane;
+      keys[u] = a < end ? load_key(idx, bits, a, E, nullptr) : -1;
     }
-    __syncwarp();
-    if (valid && (peers & lt_mask) == 0) my[key] += __popc(peers);
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int a = base + 32 * u + lane;
+      const int key = keys[u];
+      const unsigned peers = __match_any_sync(0xffffffffu, key);
+      if (key >= 0) {
+        const int p = my[key] + __popc(peers & lt_mask);
+        if (stage_perm) perm_s[p] = a; else perm[p] = a;
+        inv_perm[a] = p;
+      }
+      __syncwarp();
+      if (key >= 0 && (peers & lt_mask) == 0) my[key] += __popc(peers);
+      __syncwarp();
+    }
   }
   if (stage_perm) {  // scattered positions land in shared memory; write out coalesced
     __syncthreads();

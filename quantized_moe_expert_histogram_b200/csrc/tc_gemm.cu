@@ -97,6 +97,27 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Bounded wait by a whole warp: every lane observes the barrier, then the
+// warp reconverges and agrees on the outcome, so the warp-aligned
+// instructions that follow (tcgen05.ld, barriers) run converged.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status);
+  __syncwarp();
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Optional progress record (a test hook): slot `role` of this CTA holds
+// (site << 24) | (tile & 0xfff) << 12 | (kb & 0xfff), written through to
+// host-visible memory so that a stalled launch can be inspected.
+__device__ __forceinline__ void trace_put(int* trace, int role, int site, int tile, int kb) {
+  if (trace) {
+    reinterpret_cast<volatile int*>(trace)[blockIdx.x * 16 + role] =
+        (site << 24) | ((tile & 0xfff) << 12) | (kb & 0xfff);
+    __threadfence_system();
+  }
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -178,29 +199,31 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 // ------------------------------------------------------------ config ----
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;  // 16 warps
 constexpr int kMaxBins = 768;
+constexpr int kNT = 256;       // largest token block (MMA N)
 
-template <int NMAT, int NT_MAX>
 struct Cfg {
   static constexpr int STAGES = 3;    // A/B stages of 64 K
   static constexpr int CSTAGES = 4;   // codes stages of 128 K
-  static constexpr int A_BYTES = 128 * 128;      // 128 rows x 64 fp16
-  static constexpr int B_BYTES = NT_MAX * 128;   // NT rows x 64 fp16
-  static constexpr int C_BYTES = 8192;           // 128 rows x 128 K codes (either layout)
-  static constexpr int SZ_BYTES = 1024;          // 128 rows x up to 2 groups x 4 B
+  static constexpr int A_BYTES = 128 * 128;     // 128 weight rows x 64 fp16
+  static constexpr int B_BYTES = kNT * 128;     // 256 token rows x 64 fp16
+  static constexpr int C_BYTES = 8192;          // 128 rows x 128 K of codes (either layout)
+  static constexpr int SZ_BYTES = 1024;         // 128 rows x up to 2 groups x 4 B
+  static constexpr int X_BYTES = 2 * 16 * 64 * 4;  // gate/up exchange, double buffered
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * NMAT * A_BYTES;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_SZ = OFF_C + CSTAGES * NMAT * C_BYTES;
-  static constexpr int OFF_TILE = OFF_SZ + CSTAGES * NMAT * SZ_BYTES;  // int tile_start[769], off[769]
+  static constexpr int OFF_SZ = OFF_C + CSTAGES * C_BYTES;
+  static constexpr int OFF_X = OFF_SZ + CSTAGES * SZ_BYTES;
+  static constexpr int OFF_TILE = OFF_X + X_BYTES;  // int tile_start[769], off[769]
   static constexpr int OFF_BAR = OFF_TILE + 2 * (kMaxBins + 1) * 4 + 8;
-  static constexpr int N_BARS = 2 * CSTAGES + 3 * STAGES + 4 + 1;
+  static constexpr int N_BARS = 2 * CSTAGES + 3 * STAGES + 4 + 1 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag
   static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + alignment slack
-  static constexpr int TMEM_COLS = 512;
-  static_assert(2 * NMAT * NT_MAX <= TMEM_COLS, "TMEM budget");
+  static constexpr int TMEM_COLS = 512;                  // two accumulators of kNT columns
 };
+static_assert(Cfg::SMEM <= 232448, "shared memory budget");
 
 struct TcParams {
   CUtensorMap act;       // fp16 [rows][K], box 64 x 16, 128B swizzle
@@ -216,13 +239,13 @@ struct TcParams {
   __half* h_out;
   float* y_out;
   int32_t* status;
+  int* trace;  // optional progress record (null in normal use)
 };
 
 struct Tile {
   int bin, slot, bits, row0, nrows, nt, mb;
 };
 
-template <int NT_MAX>
 __device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const int* off, int nbins,
                                             int MB, int planes_mult, const int32_t* slot_of) {
   int lo = 0, hi = nbins;  // largest b with tile_start[b] <= t (tile_start[nbins] = total)
@@ -236,7 +259,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const 
   const int tb = local / MB;
   T.mb = local - tb * MB;
   const int n = off[lo + 1] - off[lo];
-  const int nb = (n + NT_MAX - 1) / NT_MAX;
+  const int nb = (n + kNT - 1) / kNT;
   const int per = (((n + nb - 1) / nb) + 15) & ~15;
   T.row0 = off[lo] + tb * per;
   T.nrows = min(per, n - tb * per);
@@ -263,28 +286,32 @@ __device__ __forceinline__ uint32_t spread1(uint32_t x) {
   return x;
 }
 
-// Eight 4-bit codes (nibble i = element i) -> four half2 (e0,e1)..(e6,e7)
-// holding (code - z) * s rounded once to fp16.
+// Eight 4-bit codes (nibble i = element i) -> (code - z) * s as fp16,
+// elements in order.  Byte j holds the pair (e_2j, e_2j+1); replicated
+// into both halves and masked, it reads as the half2 (1024 + e_2j,
+// 64 + e_2j+1) (the high nibble lands at mantissa bits 4..7, whose unit at
+// exponent 64 is 1/16).  Subtracting (1024 + z, 64 + z) is exact, and one
+// multiply by s rounds each product once.
 __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 zoff, __half2 s2) {
   uint32_t v[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t raw = ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;  // (1024+q_j, 1024+q_{j+4})
+    const uint32_t rep = __byte_perm(w, 0u, 0x1111u * j);
+    uint32_t raw;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(raw) : "r"(rep), "r"(0x00F0000Fu), "r"(0x54006400u));
     __half2 h = *reinterpret_cast<const __half2*>(&raw);
     h = __hmul2(__hsub2(h, zoff), s2);
     v[j] = *reinterpret_cast<uint32_t*>(&h);
   }
-  uint4 o;
-  o.x = __byte_perm(v[0], v[1], 0x5410);
-  o.y = __byte_perm(v[2], v[3], 0x5410);
-  o.z = __byte_perm(v[0], v[1], 0x7632);
-  o.w = __byte_perm(v[2], v[3], 0x7632);
-  return o;
+  return make_uint4(v[0], v[1], v[2], v[3]);
 }
 
-template <int NMAT, int NT_MAX, bool PLANES>
+// GATEUP: a tile's 128 weight rows are 64 gate rows then the 64 up rows of
+// the same features, so one MMA covers both and the epilogue pairs TMEM
+// lane i with lane i + 64.  DOWN: 128 rows of W_down.
+template <bool GATEUP, bool PLANES>
 __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ TcParams P) {
-  using C = Cfg<NMAT, NT_MAX>;
+  using C = Cfg;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   int* tile_start = reinterpret_cast<int*>(smem + C::OFF_TILE);
@@ -302,17 +329,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
   auto acc_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + i); };
   auto acc_empty = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 2 + i); };
   const uint32_t drain_bar = bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 4);
+  auto x_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 5 + i); };
+  auto x_empty = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 7 + i); };
+  const uint32_t exit_bar = bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 9);
+  int* trace = P.trace ? P.trace + (GATEUP ? 0 : gridDim.x * 16) : nullptr;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbins = P.nbins;
-  const int MB = P.N / 128;
+  const int rows_per_mat = GATEUP ? 64 : 128;  // weight rows of each matrix in a tile
+  const int MB = P.N / rows_per_mat;
   const int KC = P.K / 128;
 
   // ---- set-up: barriers, TMEM, tile table --------------------------------
   if (tid == 0) {
     for (int i = 0; i < C::CSTAGES; ++i) {
       mbar_init(codes_full(i), 1);
-      mbar_init(codes_empty(i), 4);
+      mbar_init(codes_empty(i), 8);
     }
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(a_full(i), 4);
@@ -324,6 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       mbar_init(acc_empty(i), 4);
     }
     mbar_init(drain_bar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(x_full(i), 2);
+      mbar_init(x_empty(i), 2);
+    }
+    mbar_init(exit_bar, kThreads / 32);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -334,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   for (int b = tid; b <= nbins; b += kThreads) off_s[b] = P.offsets[b];
+  __syncwarp();
   __syncthreads();
   if (warp == 0) {
     // tiles per bin -> exclusive scan (lane owns a contiguous run of bins)
@@ -345,8 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       if (b < nbins) {
         int n = off_s[b + 1] - off_s[b];
         if (P.slot_of && P.slot_of[b / P.planes_mult] < 0) n = 0;
-        const int tiles = ((n + NT_MAX - 1) / NT_MAX) * MB;
-        tile_start[b] = run;  // lane-local exclusive prefix for now
+        const int tiles = ((n + kNT - 1) / kNT) * MB;
+        tile_start[b] = run;
         run += tiles;
       }
     }
@@ -363,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
     }
     if (lane == 31) tile_start[nbins] = incl;
   }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -376,36 +415,44 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       int cs = 0, cph = 0, s = 0, sph = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile T = decode_tile<NT_MAX>(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
+        const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
         if (codes_role) {
           const uint8_t* blob = P.blobs + static_cast<size_t>(T.slot) * P.blob_bytes;
           const int gpc = 128 / P.group;  // groups per codes stage
-          const uint32_t sz_bytes = gpc * 512;
+          const int G = P.K / P.group;
           uint32_t code_bytes = 8192;
           if (PLANES) code_bytes = 4096 + (T.bits >= 3 ? 2048 : 0) + (T.bits >= 4 ? 2048 : 0);
+          const int r0 = T.mb * rows_per_mat;  // first weight row of each matrix
           for (int kc = 0; kc < KC && ok; ++kc) {
+            trace_put(trace, 0, 1, t, kc);
             ok = mbar_wait(codes_empty(cs), cph ^ 1, abort_flag, P.status);
             if (!ok) break;
-            mbar_expect_tx(codes_full(cs), NMAT * (code_bytes + sz_bytes));
+            mbar_expect_tx(codes_full(cs), code_bytes + gpc * 512);
+            const uint32_t cdst = smem_u32(smem + C::OFF_C + cs * C::C_BYTES);
+            const uint32_t szdst = smem_u32(smem + C::OFF_SZ + cs * C::SZ_BYTES);
 #pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
-              const uint32_t cdst = smem_u32(smem + C::OFF_C + (cs * NMAT + m) * C::C_BYTES);
+            for (int m = 0; m < (GATEUP ? 2 : 1); ++m) {
+              // INT4 rows are 64 B, Q2 rows 32 B, residual rows 16 B
               if (!PLANES) {
-                tma_load_3d(cdst, &P.codes[m], kc * 16, T.mb * 128, T.slot, codes_full(cs));
+                tma_load_3d(cdst + m * 4096, &P.codes[m], kc * 16, r0, T.slot, codes_full(cs));
               } else {
-                tma_load_3d(cdst, &P.codes[m], kc * 8, T.mb * 128, T.slot, codes_full(cs));
-                if (T.bits >= 3) tma_load_3d(cdst + 4096, &P.d3[m], kc * 4, T.mb * 128, T.slot, codes_full(cs));
-                if (T.bits >= 4) tma_load_3d(cdst + 6144, &P.d4[m], kc * 4, T.mb * 128, T.slot, codes_full(cs));
+                tma_load_3d(cdst + m * 2048, &P.codes[m], kc * 8, r0, T.slot, codes_full(cs));
+                if (T.bits >= 3)
+                  tma_load_3d(cdst + 4096 + m * 1024, &P.d3[m], kc * 4, r0, T.slot, codes_full(cs));
+                if (T.bits >= 4)
+                  tma_load_3d(cdst + 6144 + m * 1024, &P.d4[m], kc * 4, r0, T.slot, codes_full(cs));
               }
-              const uint8_t* szsrc = blob + P.sz_off[m] +
-                                     (static_cast<size_t>(T.mb) * (P.K / P.group) + kc * gpc) * 512;
-              bulk_load(smem_u32(smem + C::OFF_SZ + (cs * NMAT + m) * C::SZ_BYTES), szsrc, sz_bytes,
-                        codes_full(cs));
+              for (int c = 0; c < gpc; ++c) {
+                const uint8_t* src = blob + P.sz_off[m] +
+                                     ((static_cast<size_t>(r0 >> 7) * G + kc * gpc + c) * 128 + (r0 & 127)) * 4;
+                bulk_load(szdst + c * 512 + m * 256, src, rows_per_mat * 4, codes_full(cs));
+              }
             }
             if (++cs == C::CSTAGES) { cs = 0; cph ^= 1; }
           }
         } else {
           for (int kb = 0; kb < 2 * KC && ok; ++kb) {
+            trace_put(trace, 2, 2, t, kb);
             ok = mbar_wait(ab_empty(s), sph ^ 1, abort_flag, P.status);
             if (!ok) break;
             mbar_expect_tx(b_full(s), T.nt * 128);
@@ -415,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
           }
         }
       }
+      trace_put(trace, codes_role ? 0 : 2, ok ? 12 : 13, 0, 0);
       if (!ok) {
         // drain: the most recent arming of every stage must land before exit
         const uint64_t t0 = global_ns();
@@ -438,24 +486,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       int s = 0, sph = 0, acc = 0, aph = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile T = decode_tile<NT_MAX>(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
+        const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
         const uint32_t idesc = umma_idesc_f16(T.nt);
+        trace_put(trace, 1, 3, t, 0);
         ok = mbar_wait(acc_empty(acc), aph ^ 1, abort_flag, P.status);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t dcol = tmem_base + acc * (NMAT * NT_MAX);
+        const uint32_t dcol = tmem_base + acc * kNT;
         for (int kb = 0; kb < 2 * KC && ok; ++kb) {
-          ok = mbar_wait(a_full(s), sph, abort_flag, P.status) && mbar_wait(b_full(s), sph, abort_flag, P.status);
+          trace_put(trace, 1, 4, t, kb);
+          ok = mbar_wait(a_full(s), sph, abort_flag, P.status);
+          if (!ok) break;
+          trace_put(trace, 1, 5, t, kb);
+          ok = mbar_wait(b_full(s), sph, abort_flag, P.status);
           if (!ok) break;
           tc_fence_after();
           const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::OFF_B + s * C::B_BYTES));
+          const uint64_t adesc = umma_desc_sw128(smem_u32(smem + C::OFF_A + s * C::A_BYTES));
 #pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            const uint64_t adesc = umma_desc_sw128(smem_u32(smem + C::OFF_A + (s * NMAT + m) * C::A_BYTES));
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_f16(dcol + m * NT_MAX, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
-          }
+          for (int kk = 0; kk < 4; ++kk) umma_f16(dcol, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
           umma_commit(ab_empty(s));
           if (++s == C::STAGES) { s = 0; sph ^= 1; }
         }
@@ -463,122 +512,136 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         umma_commit(acc_full(acc));
         if (++acc == 2) { acc = 0; aph ^= 1; }
       }
+      trace_put(trace, 1, ok ? 12 : 13, 0, 0);
       // all MMAs issued by this thread complete before TMEM is released
       umma_commit(drain_bar);
       const uint64_t t0 = global_ns();
       while (!mbar_try(drain_bar, 0) && global_ns() - t0 < kWaitLimitNs) {}
     }
   }
-  // ---- dequantisers ------------------------------------------------------
-  else if (warp >= 4 && warp < 8) {
-    const int i = tid - 128;  // weight row inside the 128-row block
-    int cs = 0, cph = 0, s = 0, sph = 0;
+  // ---- dequantisers: warps 4-7 take K half 0, warps 8-11 half 1 ----------
+  else if (warp >= 4 && warp < 12) {
+    const int h = (warp - 4) >> 2;       // which 64-K half of a codes stage
+    const int i = tid - 128 - 128 * h;   // weight row inside the tile
+    int cs = 0, cph = 0;
+    int kbc = h;  // running k-block counter of this half (stage = kbc % STAGES)
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-      const Tile T = decode_tile<NT_MAX>(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
+      const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
       for (int kc = 0; kc < KC && ok; ++kc) {
-        ok = mbar_wait(codes_full(cs), cph, abort_flag, P.status);
+        if (lane == 0) trace_put(trace, 3 + h, 6, t, kc);
+        ok = warp_wait(codes_full(cs), cph, abort_flag, P.status);
         if (!ok) break;
-        uint32_t w[NMAT][16];
-        uint32_t sz[NMAT][2];
+        const uint8_t* cb = smem + C::OFF_C + cs * C::C_BYTES;
+        uint32_t w[8];
+        if (!PLANES) {
+          // row i: 64 B, 64B swizzle (chunk j at j ^ ((i >> 1) & 3)); this half = chunks 2h, 2h+1
 #pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-          const uint8_t* cb = smem + C::OFF_C + (cs * NMAT + m) * C::C_BYTES;
-          if (!PLANES) {
-            // row i: 64 B = 4 chunks, 64B swizzle: chunk j at j ^ ((i >> 1) & 3)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint4 v = *reinterpret_cast<const uint4*>(cb + i * 64 + ((j ^ ((i >> 1) & 3)) << 4));
-              w[m][4 * j] = v.x; w[m][4 * j + 1] = v.y; w[m][4 * j + 2] = v.z; w[m][4 * j + 3] = v.w;
-            }
-          } else {
-            // Q2 row i: 32 B = 2 chunks, 32B swizzle: chunk j at j ^ ((i >> 2) & 1)
-            uint32_t q2[8];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const uint4 v = *reinterpret_cast<const uint4*>(cb + i * 32 + ((j ^ ((i >> 2) & 1)) << 4));
-              q2[4 * j] = v.x; q2[4 * j + 1] = v.y; q2[4 * j + 2] = v.z; q2[4 * j + 3] = v.w;
-            }
-            uint4 r3 = make_uint4(0, 0, 0, 0), r4 = make_uint4(0, 0, 0, 0);
-            if (T.bits >= 3) r3 = *reinterpret_cast<const uint4*>(cb + 4096 + i * 16);
-            if (T.bits >= 4) r4 = *reinterpret_cast<const uint4*>(cb + 6144 + i * 16);
-            const uint32_t d3w[4] = {r3.x, r3.y, r3.z, r3.w};
-            const uint32_t d4w[4] = {r4.x, r4.y, r4.z, r4.w};
-#pragma unroll
-            for (int wd = 0; wd < 16; ++wd) {  // word wd = elements 8wd..8wd+7
-              const uint32_t base = q2[wd >> 1] >> (16 * (wd & 1));
-              const uint32_t b3 = d3w[wd >> 2] >> (8 * (wd & 3));
-              const uint32_t b4 = d4w[wd >> 2] >> (8 * (wd & 3));
-              w[m][wd] = (spread2(base) << 2) | (spread1(b3) << 1) | spread1(b4);
-            }
+          for (int jj = 0; jj < 2; ++jj) {
+            const int j = 2 * h + jj;
+            const uint4 v = *reinterpret_cast<const uint4*>(cb + i * 64 + ((j ^ ((i >> 1) & 3)) << 4));
+            w[4 * jj] = v.x; w[4 * jj + 1] = v.y; w[4 * jj + 2] = v.z; w[4 * jj + 3] = v.w;
           }
-          const uint32_t* szb = reinterpret_cast<const uint32_t*>(smem + C::OFF_SZ + (cs * NMAT + m) * C::SZ_BYTES);
-          sz[m][0] = szb[i];
-          sz[m][1] = (P.group == 64) ? szb[128 + i] : sz[m][0];
+        } else {
+          // Q2 row i: 32 B, 32B swizzle (chunk j at j ^ ((i >> 2) & 1)); this half = chunk h
+          const uint4 q2 = *reinterpret_cast<const uint4*>(cb + i * 32 + ((h ^ ((i >> 2) & 1)) << 4));
+          uint2 r3 = make_uint2(0, 0), r4 = make_uint2(0, 0);
+          if (T.bits >= 3) r3 = *reinterpret_cast<const uint2*>(cb + 4096 + i * 16 + 8 * h);
+          if (T.bits >= 4) r4 = *reinterpret_cast<const uint2*>(cb + 6144 + i * 16 + 8 * h);
+          const uint32_t qw[4] = {q2.x, q2.y, q2.z, q2.w};
+          const uint32_t d3w[2] = {r3.x, r3.y};
+          const uint32_t d4w[2] = {r4.x, r4.y};
+#pragma unroll
+          for (int wd = 0; wd < 8; ++wd) {  // word wd = elements 8wd..8wd+7 of the half
+            const uint32_t base = qw[wd >> 1] >> (16 * (wd & 1));
+            const uint32_t b3 = d3w[wd >> 2] >> (8 * (wd & 3));
+            const uint32_t b4 = d4w[wd >> 2] >> (8 * (wd & 3));
+            w[wd] = (spread2(base) << 2) | (spread1(b3) << 1) | spread1(b4);
+          }
         }
+        const uint32_t* szb = reinterpret_cast<const uint32_t*>(smem + C::OFF_SZ + cs * C::SZ_BYTES);
+        const uint32_t word = szb[(P.group == 64 ? h : 0) * 128 + i];
         __syncwarp();
         if (lane == 0) mbar_arrive(codes_empty(cs));
         if (++cs == C::CSTAGES) { cs = 0; cph ^= 1; }
-        for (int h = 0; h < 2 && ok; ++h) {
-          ok = mbar_wait(ab_empty(s), sph ^ 1, abort_flag, P.status);
-          if (!ok) break;
+
+        const int s = kbc % C::STAGES;
+        const int sph = (kbc / C::STAGES) & 1;
+        kbc += 2;
+        if (lane == 0) trace_put(trace, 3 + h, 7, t, kbc - 2);
+        ok = warp_wait(ab_empty(s), sph ^ 1, abort_flag, P.status);
+        if (!ok) break;
+        const __half sc = __float2half_rn(__uint_as_float(word << 16));
+        const float zf = __uint_as_float(word & 0xFFFF0000u);
+        const __half2 s2 = __half2half2(sc);
+        const __half2 z2 = __halves2half2(__float2half_rn(1024.0f + zf), __float2half_rn(64.0f + zf));
+        uint8_t* arow = smem + C::OFF_A + s * C::A_BYTES + i * 128;
 #pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            // the 64 elements of half h lie in group (h * 64) / group of the stage
-            const uint32_t word = sz[m][h];
-            const __half sc = __float2half_rn(__uint_as_float(word << 16));
-            const float zf = __uint_as_float(word & 0xFFFF0000u);
-            const __half2 s2 = __half2half2(sc);
-            const __half2 z2 = __half2half2(__float2half_rn(1024.0f + zf));
-            uint8_t* arow = smem + C::OFF_A + (s * NMAT + m) * C::A_BYTES + i * 128;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = elements 8j..8j+7 of the half
-              const uint4 o = dequant8(w[m][8 * h + j], z2, s2);
-              *reinterpret_cast<uint4*>(arow + ((j ^ (i & 7)) << 4)) = o;
-            }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(a_full(s));
-          if (++s == C::STAGES) { s = 0; sph ^= 1; }
+        for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = elements 8j..8j+7 of the half
+          const uint4 o = dequant8(w[j], z2, s2);
+          *reinterpret_cast<uint4*>(arow + ((j ^ (i & 7)) << 4)) = o;
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(a_full(s));
       }
     }
   }
-  // ---- epilogue ----------------------------------------------------------
-  else if (warp >= 8) {
-    const int q = warp & 3;  // TMEM lane quadrant
-    int acc = 0, aph = 0;
+  // ---- epilogue: warps 12-15, TMEM lane quadrant = warp % 4 ---------------
+  else {
+    const int q = warp & 3;
+    float* xch = reinterpret_cast<float*>(smem + C::OFF_X);  // [2][16][64]: up values by column
+    int acc = 0, aph = 0, xuse = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-      const Tile T = decode_tile<NT_MAX>(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
-      ok = mbar_wait(acc_full(acc), aph, abort_flag, P.status);
+      const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
+      if (lane == 0) trace_put(trace, 5 + (q >> 1), 8, t, 0);
+      ok = warp_wait(acc_full(acc), aph, abort_flag, P.status);
       if (!ok) break;
       tc_fence_after();
-      const int row = T.mb * 128 + 32 * q + lane;  // output feature of this thread
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * (NMAT * NT_MAX);
-      for (int j0 = 0; j0 < T.nrows; j0 += 16) {
-        uint32_t g[16];
-        tmem_ld16(tbase + j0, g);
-        if (NMAT == 2) {
-          uint32_t u[16];
-          tmem_ld16(tbase + NT_MAX + j0, u);
-          tmem_ld_wait();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * kNT;
+      for (int j0 = 0; j0 < T.nrows && ok; j0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tbase + j0, v);
+        tmem_ld_wait();
+        if (GATEUP) {
+          // up rows (quadrants 2, 3) hand their values to the gate rows of
+          // the same features (quadrants 0, 1) through a two-slot buffer
+          const int xb = xuse & 1, xph = (xuse >> 1) & 1;
+          ++xuse;
+          float* xbuf = xch + xb * (16 * 64);
+          if (q >= 2) {
+            if (lane == 0) trace_put(trace, 6, 9, t, j0);
+            ok = warp_wait(x_empty(xb), xph ^ 1, abort_flag, P.status);
+            if (!ok) break;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (j0 + j < T.nrows) {
-              const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
-              P.h_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + row] = __float2half_rn(silu_f(gv) * uv);
+            for (int j = 0; j < 16; ++j) xbuf[j * 64 + (q - 2) * 32 + lane] = __uint_as_float(v[j]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(x_full(xb));
+          } else {
+            if (lane == 0) trace_put(trace, 5, 10, t, j0);
+            ok = warp_wait(x_full(xb), xph, abort_flag, P.status);
+            if (!ok) break;
+            const int f = T.mb * 64 + 32 * q + lane;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (j0 + j < T.nrows) {
+                const float gv = __uint_as_float(v[j]), uv = xbuf[j * 64 + q * 32 + lane];
+                P.h_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + f] = __float2half_rn(silu_f(gv) * uv);
+              }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(x_empty(xb));
           }
         } else {
-          tmem_ld_wait();
+          const int n = T.mb * 128 + 32 * q + lane;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (j0 + j < T.nrows)
-              P.y_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + row] = __uint_as_float(g[j]);
+              P.y_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + n] = __uint_as_float(v[j]);
         }
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(acc));
@@ -586,12 +649,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
     }
   }
 
+  // Exit: every warp reconverges (single-lane roles included) and reports;
+  // the allocator warp frees TMEM once all have left their loops.
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  if (lane == 0) mbar_arrive(exit_bar);
   if (warp == 2) {
+    if (lane == 0) trace_put(trace, 7, 14, 0, 0);
+    warp_wait(exit_bar, 0, abort_flag, P.status);
+    tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
                  : "memory");
+    if (lane == 0) trace_put(trace, 7, 15, 0, 0);
   }
 }
 
@@ -620,6 +689,8 @@ bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, 
   return r == CUDA_SUCCESS;
 }
 
+int* g_trace = nullptr;  // test hook: host-mapped progress record
+
 int sm_count() {
   static int n = 0;
   if (!n) {
@@ -631,9 +702,10 @@ int sm_count() {
   return n;
 }
 
-// act: fp16 [rows][K]; weight matrices m of the pass (N x K each).
+// act: fp16 [rows][K]; weight matrices `mats` of the pass (N x K each),
+// `box_rows` weight rows per matrix per tile.
 moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int rows, int K, int N,
-                         const int* mats, int nmat, int n_blobs) {
+                         const int* mats, int nmat, int box_rows, int n_blobs) {
   const bool planes = a.layout == MOE_LAYOUT_PLANES;
   {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
@@ -644,12 +716,13 @@ moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int r
       return MOE_ERR_CUDA;
     }
   }
+  const cuuint32_t br = static_cast<cuuint32_t>(box_rows);
   for (int i = 0; i < nmat; ++i) {
     const int m = mats[i];
     if (!planes) {
       cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 8), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_blobs)};
       cuuint64_t str[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(a.blob_bytes)};
-      cuuint32_t box[3] = {16, 128, 1};
+      cuuint32_t box[3] = {16, br, 1};
       if (!encode(&P.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.codes[m], dims, str, box,
                   CU_TENSOR_MAP_SWIZZLE_64B)) {
         set_error("tensor map (codes) could not be encoded");
@@ -658,15 +731,15 @@ moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int r
     } else {
       cuuint64_t dq[3] = {static_cast<cuuint64_t>(K / 16), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_blobs)};
       cuuint64_t sq[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(a.blob_bytes)};
-      cuuint32_t bq[3] = {8, 128, 1};
+      cuuint32_t bq[3] = {8, br, 1};
       cuuint64_t dr[3] = {static_cast<cuuint64_t>(K / 32), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_blobs)};
       cuuint64_t sr[2] = {static_cast<cuuint64_t>(K / 8), static_cast<cuuint64_t>(a.blob_bytes)};
-      cuuint32_t br[3] = {4, 128, 1};
+      cuuint32_t bb[3] = {4, br, 1};
       if (!encode(&P.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.q2[m], dq, sq, bq,
                   CU_TENSOR_MAP_SWIZZLE_32B) ||
-          !encode(&P.d3[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.d3[m], dr, sr, br,
+          !encode(&P.d3[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.d3[m], dr, sr, bb,
                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-          !encode(&P.d4[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.d4[m], dr, sr, br,
+          !encode(&P.d4[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.d4[m], dr, sr, bb,
                   CU_TENSOR_MAP_SWIZZLE_NONE)) {
         set_error("tensor map (bit planes) could not be encoded");
         return MOE_ERR_CUDA;
@@ -684,28 +757,29 @@ moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int r
   P.nbins = a.E * P.planes_mult;
   P.group = a.group;
   P.status = a.status;
+  P.trace = g_trace;
   return MOE_OK;
 }
 
-template <int NMAT, int NT_MAX, bool PLANES>
+template <bool GATEUP, bool PLANES>
 moe_status_t launch_one(const TcParams& P, cudaStream_t s) {
-  using C = Cfg<NMAT, NT_MAX>;
-  auto kern = k_ffn_tc<NMAT, NT_MAX, PLANES>;
+  auto kern = k_ffn_tc<GATEUP, PLANES>;
   // Set once per process (the first call must precede any stream capture).
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return cuda_check(e, "tc ffn smem attribute");
     attr_set = true;
   }
-  kern<<<sm_count(), kThreads, C::SMEM, s>>>(P);
+  kern<<<sm_count(), kThreads, Cfg::SMEM, s>>>(P);
   return cuda_check(cudaGetLastError(), "tc ffn launch");
 }
 
 }  // namespace
 
 bool tc_supported(const FfnArgs& a) {
-  return get_encode() != nullptr && a.d % 128 == 0 && a.F % 128 == 0 && a.E * (a.layout == MOE_LAYOUT_PLANES ? 3 : 1) <= kMaxBins;
+  return get_encode() != nullptr && a.d % 128 == 0 && a.F % 128 == 0 &&
+         a.E * (a.layout == MOE_LAYOUT_PLANES ? 3 : 1) <= kMaxBins;
 }
 
 moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s) {
@@ -713,19 +787,23 @@ moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s) {
   const bool planes = a.layout == MOE_LAYOUT_PLANES;
   TcParams gu{};
   const int m_gu[2] = {0, 1};
-  moe_status_t st = make_params(gu, a, a.x_perm, a.total_rows, a.d, a.F, m_gu, 2, n_blobs);
+  moe_status_t st = make_params(gu, a, a.x_perm, a.total_rows, a.d, a.F, m_gu, 2, 64, n_blobs);
   if (st != MOE_OK) return st;
   gu.h_out = a.h;
   gu.y_out = nullptr;
-  st = planes ? launch_one<2, 128, true>(gu, s) : launch_one<2, 128, false>(gu, s);
+  st = planes ? launch_one<true, true>(gu, s) : launch_one<true, false>(gu, s);
   if (st != MOE_OK) return st;
   TcParams dn{};
   const int m_dn[1] = {2};
-  st = make_params(dn, a, a.h, a.total_rows, a.F, a.d, m_dn, 1, n_blobs);
+  st = make_params(dn, a, a.h, a.total_rows, a.F, a.d, m_dn, 1, 128, n_blobs);
   if (st != MOE_OK) return st;
   dn.h_out = nullptr;
   dn.y_out = a.y_perm;
-  return planes ? launch_one<1, 256, true>(dn, s) : launch_one<1, 256, false>(dn, s);
+  return planes ? launch_one<false, true>(dn, s) : launch_one<false, false>(dn, s);
 }
 
 }  // namespace moeq
+
+extern "C" void moe_debug_set_trace(void* host_mapped_ints) {
+  moeq::g_trace = static_cast<int*>(host_mapped_ints);
+}

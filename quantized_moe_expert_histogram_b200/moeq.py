@@ -48,6 +48,7 @@ _SIGS = {
     "moe_slot_cache_destroy": (None, [_c_p]),
     "moe_debug_inject_fault": (None, [_c_i, _c_i]),
     "moe_debug_force_regime": (None, [_c_i]),
+    "moe_debug_set_trace": (None, [_c_p]),
 }
 
 _lib = None
@@ -266,3 +267,8 @@ def moe_last_error():
 def moe_debug_force_regime(regime):
     """0 = by T, 1 = decode GEMV, 2 = tensor cores (test hook)."""
     load().moe_debug_force_regime(regime)
+
+
+def moe_debug_set_trace(pinned_int32=None):
+    """Progress record of the tensor-core FFN kernels (test hook)."""
+    load().moe_debug_set_trace(None if pinned_int32 is None else pinned_int32.data_ptr())
