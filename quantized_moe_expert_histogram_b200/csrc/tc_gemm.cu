@@ -1,32 +1,40 @@
 // Prefill-regime grouped expert FFN on the 5th-generation tensor cores.
 //
 // One persistent CTA per SM walks a tile list built on the device from the
-// bin offsets (no host sync).  A tile is (bin, token block, 128-row weight
-// block).  The MMA is issued "swap-AB": the 128 dequantised weight rows are
-// the M side (operand A, built in shared memory) and the bin's tokens are
-// the N side (operand B, fp16 activation rows loaded by TMA), so a bin of
-// any size is covered with at most 15 padded token columns, and
+// bin offsets (no host sync).  A tile is (bin, token block of up to 128
+// rows, weight block).  The MMA is issued "swap-AB": dequantised weight
+// rows are the M side (operand A, built in shared memory) and the bin's
+// tokens the N side (operand B, fp16 activation rows loaded by TMA), so a
+// bin of any size is covered with at most 15 padded token columns;
 // D[weight row][token] accumulates in TMEM (fp32).
 //
-// Warp roles (12 warps):
+// Each k-block issues two M=128 MMAs that share one B tile: the gate and
+// up rows of the same 128 features (first GEMM), or two adjacent 128-row
+// blocks of W_down (second GEMM).  Sharing B halves the activation bytes
+// per MAC, and in the first GEMM lane i of both accumulators belongs to
+// feature i, so the SwiGLU epilogue needs no exchange.
+//
+// Warp roles (16 warps):
 //   warp 0      codes producer: packed codes (3-D tensor map over the blob
-//               pool, one box per 128 K) and their scale/zero words (1-D
-//               bulk copy)
+//               pool, one 128-row box per 128 K per matrix) and their
+//               scale/zero words (1-D bulk copies)
 //   warp 3      activation producer: fp16 rows of the bin (16-row TMA
 //               boxes, 128B swizzle)
 //   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=tokens,
 //               K=16) and tcgen05.commit
-//   warp 2      TMEM allocator (512 columns: two accumulator buffers)
-//   warps 4-7   dequantisers: thread i turns weight row i of a staged codes
-//               block into fp16 ((code - zero) * scale, one rounding) and
-//               writes it in the UMMA K-major 128B-swizzled layout
-//   warps 8-11  epilogue: tcgen05.ld of its TMEM lane quadrant; gate/up
+//   warp 2      TMEM allocator (512 columns: two buffers of two accumulators)
+//   warps 4-7   dequantisers of matrix 0, warps 8-11 of matrix 1: thread i
+//               turns weight row i of a staged codes block into fp16
+//               ((code - zero) * scale, one rounding) and writes it in the
+//               UMMA K-major 128B-swizzled layout
+//   warps 12-15 epilogue: tcgen05.ld of its TMEM lane quadrant; gate/up
 //               pass writes h = silu(gate) * up (fp16), down pass y_perm
 //               (fp32)
-// Pipelines: codes (4 stages of 128 K) -> dequant -> A/B (3 stages of 64 K)
+// Pipelines: codes (3 stages of 128 K) -> dequant -> A/B (3 stages of 64 K)
 // -> MMA -> TMEM (2 buffers) -> epilogue.  Every wait is bounded; on a
 // timeout the CTA raises MOE_DEV_TIMEOUT, drains its copies and MMAs,
-// frees TMEM and returns.
+// frees TMEM and returns.  Warps reconverge after every wait, before any
+// warp-aligned instruction.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -80,8 +88,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: only reached when some
 
 // Bounded wait.  Returns false when the CTA is aborting (flag set here on
 // timeout, or by another role).
+// Where the first timeout of a CTA happened (test hook, see trace_put).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status) {
+                                          int32_t* status, int* trace = nullptr, uint32_t bar0 = 0) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
@@ -91,6 +100,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       if (global_ns() - t0 > kWaitLimitNs) {
         *abort_flag = 1;
         flag_status(status, MOE_DEV_TIMEOUT);
+        if (trace) {  // slot 8: barrier index and parity of the wait that gave up
+          reinterpret_cast<volatile int*>(trace)[blockIdx.x * 16 + 8] =
+              (0x7F << 24) | (static_cast<int>((bar - bar0) / 8) << 4) | static_cast<int>(parity);
+          __threadfence_system();
+        }
         return false;
       }
     }
@@ -101,8 +115,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // warp reconverges and agrees on the outcome, so the warp-aligned
 // instructions that follow (tcgen05.ld, barriers) run converged.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, status);
+                                          int32_t* status, int* trace = nullptr, uint32_t bar0 = 0) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status, trace, bar0);
   __syncwarp();
   return __all_sync(0xffffffffu, ok);
 }
@@ -201,27 +215,25 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 constexpr int kThreads = 512;  // 16 warps
 constexpr int kMaxBins = 768;
-constexpr int kNT = 256;       // largest token block (MMA N)
+constexpr int kNT = 128;       // largest token block (MMA N)
 
 struct Cfg {
   static constexpr int STAGES = 3;    // A/B stages of 64 K
-  static constexpr int CSTAGES = 4;   // codes stages of 128 K
-  static constexpr int A_BYTES = 128 * 128;     // 128 weight rows x 64 fp16
-  static constexpr int B_BYTES = kNT * 128;     // 256 token rows x 64 fp16
-  static constexpr int C_BYTES = 8192;          // 128 rows x 128 K of codes (either layout)
-  static constexpr int SZ_BYTES = 1024;         // 128 rows x up to 2 groups x 4 B
-  static constexpr int X_BYTES = 2 * 16 * 64 * 4;  // gate/up exchange, double buffered
+  static constexpr int CSTAGES = 3;   // codes stages of 128 K
+  static constexpr int A_BYTES = 128 * 128;     // 128 weight rows x 64 fp16, per matrix
+  static constexpr int B_BYTES = kNT * 128;     // 128 token rows x 64 fp16
+  static constexpr int C_BYTES = 8192;          // per matrix: 128 rows x 128 K of codes
+  static constexpr int SZ_BYTES = 1024;         // per matrix: 128 rows x up to 2 groups x 4 B
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_B = OFF_A + STAGES * 2 * A_BYTES;
   static constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_SZ = OFF_C + CSTAGES * C_BYTES;
-  static constexpr int OFF_X = OFF_SZ + CSTAGES * SZ_BYTES;
-  static constexpr int OFF_TILE = OFF_X + X_BYTES;  // int tile_start[769], off[769]
+  static constexpr int OFF_SZ = OFF_C + CSTAGES * 2 * C_BYTES;
+  static constexpr int OFF_TILE = OFF_SZ + CSTAGES * 2 * SZ_BYTES;  // int tile_start[769], off[769]
   static constexpr int OFF_BAR = OFF_TILE + 2 * (kMaxBins + 1) * 4 + 8;
-  static constexpr int N_BARS = 2 * CSTAGES + 3 * STAGES + 4 + 1 + 4 + 1;
+  static constexpr int N_BARS = 2 * CSTAGES + 3 * STAGES + 4 + 1 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag
   static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + alignment slack
-  static constexpr int TMEM_COLS = 512;                  // two accumulators of kNT columns
+  static constexpr int TMEM_COLS = 512;                  // 2 buffers x 2 accumulators x kNT
 };
 static_assert(Cfg::SMEM <= 232448, "shared memory budget");
 
@@ -306,9 +318,13 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 zoff, __half2 s2) 
   return make_uint4(v[0], v[1], v[2], v[3]);
 }
 
-// GATEUP: a tile's 128 weight rows are 64 gate rows then the 64 up rows of
-// the same features, so one MMA covers both and the epilogue pairs TMEM
-// lane i with lane i + 64.  DOWN: 128 rows of W_down.
+// silu(v) = v / (1 + exp(-v)), with the exponential and reciprocal at fp32
+// hardware precision (the result is rounded to fp16 afterwards).
+__device__ __forceinline__ float silu_fast(float v) { return v * __frcp_rn(1.0f + __expf(-v)); }
+
+// GATEUP: matrix 0 = gate rows, matrix 1 = up rows of features
+// [128 mb, 128 mb + 128).  DOWN: matrix 0 = W_down rows [256 mb, +128),
+// matrix 1 = rows [256 mb + 128, +128) when they exist (d % 256 may be 128).
 template <bool GATEUP, bool PLANES>
 __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ TcParams P) {
   using C = Cfg;
@@ -329,16 +345,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
   auto acc_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + i); };
   auto acc_empty = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 2 + i); };
   const uint32_t drain_bar = bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 4);
-  auto x_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 5 + i); };
-  auto x_empty = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 7 + i); };
-  const uint32_t exit_bar = bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 9);
+  const uint32_t exit_bar = bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 5);
   int* trace = P.trace ? P.trace + (GATEUP ? 0 : gridDim.x * 16) : nullptr;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbins = P.nbins;
-  const int rows_per_mat = GATEUP ? 64 : 128;  // weight rows of each matrix in a tile
-  const int MB = P.N / rows_per_mat;
+  const int rows_per_block = GATEUP ? 128 : 256;      // weight rows of one matrix pair
+  const int MB = (P.N + rows_per_block - 1) / rows_per_block;
   const int KC = P.K / 128;
+  auto has_m1 = [&](int mb) { return GATEUP || mb * 256 + 128 < P.N; };
+  auto row_base = [&](int mb, int m) { return GATEUP ? mb * 128 : mb * 256 + 128 * m; };
 
   // ---- set-up: barriers, TMEM, tile table --------------------------------
   if (tid == 0) {
@@ -347,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       mbar_init(codes_empty(i), 8);
     }
     for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(a_full(i), 4);
+      mbar_init(a_full(i), 8);
       mbar_init(b_full(i), 1);
       mbar_init(ab_empty(i), 1);
     }
@@ -356,10 +372,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       mbar_init(acc_empty(i), 4);
     }
     mbar_init(drain_bar, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(x_full(i), 2);
-      mbar_init(x_empty(i), 2);
-    }
     mbar_init(exit_bar, kThreads / 32);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -420,40 +432,38 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
           const uint8_t* blob = P.blobs + static_cast<size_t>(T.slot) * P.blob_bytes;
           const int gpc = 128 / P.group;  // groups per codes stage
           const int G = P.K / P.group;
+          const int nm = has_m1(T.mb) ? 2 : 1;
           uint32_t code_bytes = 8192;
           if (PLANES) code_bytes = 4096 + (T.bits >= 3 ? 2048 : 0) + (T.bits >= 4 ? 2048 : 0);
-          const int r0 = T.mb * rows_per_mat;  // first weight row of each matrix
           for (int kc = 0; kc < KC && ok; ++kc) {
             trace_put(trace, 0, 1, t, kc);
-            ok = mbar_wait(codes_empty(cs), cph ^ 1, abort_flag, P.status);
+            ok = mbar_wait(codes_empty(cs), cph ^ 1, abort_flag, P.status, trace, bar0);
             if (!ok) break;
-            mbar_expect_tx(codes_full(cs), code_bytes + gpc * 512);
-            const uint32_t cdst = smem_u32(smem + C::OFF_C + cs * C::C_BYTES);
-            const uint32_t szdst = smem_u32(smem + C::OFF_SZ + cs * C::SZ_BYTES);
-#pragma unroll
-            for (int m = 0; m < (GATEUP ? 2 : 1); ++m) {
-              // INT4 rows are 64 B, Q2 rows 32 B, residual rows 16 B
+            mbar_expect_tx(codes_full(cs), nm * (code_bytes + gpc * 512));
+            for (int m = 0; m < nm; ++m) {
+              const int r0 = row_base(T.mb, m);
+              const uint32_t cdst = smem_u32(smem + C::OFF_C + (cs * 2 + m) * C::C_BYTES);
+              const CUtensorMap* cm = &P.codes[GATEUP ? m : 0];
               if (!PLANES) {
-                tma_load_3d(cdst + m * 4096, &P.codes[m], kc * 16, r0, T.slot, codes_full(cs));
+                tma_load_3d(cdst, cm, kc * 16, r0, T.slot, codes_full(cs));
               } else {
-                tma_load_3d(cdst + m * 2048, &P.codes[m], kc * 8, r0, T.slot, codes_full(cs));
+                tma_load_3d(cdst, cm, kc * 8, r0, T.slot, codes_full(cs));
                 if (T.bits >= 3)
-                  tma_load_3d(cdst + 4096 + m * 1024, &P.d3[m], kc * 4, r0, T.slot, codes_full(cs));
+                  tma_load_3d(cdst + 4096, &P.d3[GATEUP ? m : 0], kc * 4, r0, T.slot, codes_full(cs));
                 if (T.bits >= 4)
-                  tma_load_3d(cdst + 6144 + m * 1024, &P.d4[m], kc * 4, r0, T.slot, codes_full(cs));
+                  tma_load_3d(cdst + 6144, &P.d4[GATEUP ? m : 0], kc * 4, r0, T.slot, codes_full(cs));
               }
-              for (int c = 0; c < gpc; ++c) {
-                const uint8_t* src = blob + P.sz_off[m] +
-                                     ((static_cast<size_t>(r0 >> 7) * G + kc * gpc + c) * 128 + (r0 & 127)) * 4;
-                bulk_load(szdst + c * 512 + m * 256, src, rows_per_mat * 4, codes_full(cs));
-              }
+              const uint8_t* src = blob + P.sz_off[GATEUP ? m : 0] +
+                                   (static_cast<size_t>(r0 >> 7) * G + kc * gpc) * 512;
+              bulk_load(smem_u32(smem + C::OFF_SZ + (cs * 2 + m) * C::SZ_BYTES), src, gpc * 512,
+                        codes_full(cs));
             }
             if (++cs == C::CSTAGES) { cs = 0; cph ^= 1; }
           }
         } else {
           for (int kb = 0; kb < 2 * KC && ok; ++kb) {
             trace_put(trace, 2, 2, t, kb);
-            ok = mbar_wait(ab_empty(s), sph ^ 1, abort_flag, P.status);
+            ok = mbar_wait(ab_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
             if (!ok) break;
             mbar_expect_tx(b_full(s), T.nt * 128);
             const uint32_t bdst = smem_u32(smem + C::OFF_B + s * C::B_BYTES);
@@ -488,23 +498,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
         const uint32_t idesc = umma_idesc_f16(T.nt);
+        const int nm = has_m1(T.mb) ? 2 : 1;
         trace_put(trace, 1, 3, t, 0);
-        ok = mbar_wait(acc_empty(acc), aph ^ 1, abort_flag, P.status);
+        ok = mbar_wait(acc_empty(acc), aph ^ 1, abort_flag, P.status, trace, bar0);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t dcol = tmem_base + acc * kNT;
+        const uint32_t dcol = tmem_base + acc * (2 * kNT);
         for (int kb = 0; kb < 2 * KC && ok; ++kb) {
           trace_put(trace, 1, 4, t, kb);
-          ok = mbar_wait(a_full(s), sph, abort_flag, P.status);
+          ok = mbar_wait(a_full(s), sph, abort_flag, P.status, trace, bar0);
           if (!ok) break;
           trace_put(trace, 1, 5, t, kb);
-          ok = mbar_wait(b_full(s), sph, abort_flag, P.status);
+          ok = mbar_wait(b_full(s), sph, abort_flag, P.status, trace, bar0);
           if (!ok) break;
           tc_fence_after();
           const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::OFF_B + s * C::B_BYTES));
-          const uint64_t adesc = umma_desc_sw128(smem_u32(smem + C::OFF_A + s * C::A_BYTES));
+          for (int m = 0; m < nm; ++m) {
+            const uint64_t adesc = umma_desc_sw128(smem_u32(smem + C::OFF_A + (s * 2 + m) * C::A_BYTES));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) umma_f16(dcol, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f16(dcol + m * kNT, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          }
           umma_commit(ab_empty(s));
           if (++s == C::STAGES) { s = 0; sph ^= 1; }
         }
@@ -519,129 +533,120 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       while (!mbar_try(drain_bar, 0) && global_ns() - t0 < kWaitLimitNs) {}
     }
   }
-  // ---- dequantisers: warps 4-7 take K half 0, warps 8-11 half 1 ----------
+  // ---- dequantisers: warps 4-7 matrix 0, warps 8-11 matrix 1 -------------
   else if (warp >= 4 && warp < 12) {
-    const int h = (warp - 4) >> 2;       // which 64-K half of a codes stage
-    const int i = tid - 128 - 128 * h;   // weight row inside the tile
-    int cs = 0, cph = 0;
-    int kbc = h;  // running k-block counter of this half (stage = kbc % STAGES)
+    const int m = (warp - 4) >> 2;
+    const int i = tid - 128 - 128 * m;   // weight row inside the 128-row block
+    int cs = 0, cph = 0, s = 0, sph = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
       const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
+      const bool live = m == 0 || has_m1(T.mb);  // matrix 1 may be absent in the last W_down block
       for (int kc = 0; kc < KC && ok; ++kc) {
-        if (lane == 0) trace_put(trace, 3 + h, 6, t, kc);
-        ok = warp_wait(codes_full(cs), cph, abort_flag, P.status);
+        if (lane == 0) trace_put(trace, 3 + m, 6, t, kc);
+        ok = warp_wait(codes_full(cs), cph, abort_flag, P.status, trace, bar0);
         if (!ok) break;
-        const uint8_t* cb = smem + C::OFF_C + cs * C::C_BYTES;
-        uint32_t w[8];
+        const uint8_t* cb = smem + C::OFF_C + (cs * 2 + m) * C::C_BYTES;
+        uint32_t w[16];
         if (!PLANES) {
-          // row i: 64 B, 64B swizzle (chunk j at j ^ ((i >> 1) & 3)); this half = chunks 2h, 2h+1
+          // row i: 64 B, 64B swizzle (chunk j at j ^ ((i >> 1) & 3))
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const int j = 2 * h + jj;
+          for (int j = 0; j < 4; ++j) {
             const uint4 v = *reinterpret_cast<const uint4*>(cb + i * 64 + ((j ^ ((i >> 1) & 3)) << 4));
-            w[4 * jj] = v.x; w[4 * jj + 1] = v.y; w[4 * jj + 2] = v.z; w[4 * jj + 3] = v.w;
+            w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
           }
         } else {
-          // Q2 row i: 32 B, 32B swizzle (chunk j at j ^ ((i >> 2) & 1)); this half = chunk h
-          const uint4 q2 = *reinterpret_cast<const uint4*>(cb + i * 32 + ((h ^ ((i >> 2) & 1)) << 4));
-          uint2 r3 = make_uint2(0, 0), r4 = make_uint2(0, 0);
-          if (T.bits >= 3) r3 = *reinterpret_cast<const uint2*>(cb + 4096 + i * 16 + 8 * h);
-          if (T.bits >= 4) r4 = *reinterpret_cast<const uint2*>(cb + 6144 + i * 16 + 8 * h);
-          const uint32_t qw[4] = {q2.x, q2.y, q2.z, q2.w};
-          const uint32_t d3w[2] = {r3.x, r3.y};
-          const uint32_t d4w[2] = {r4.x, r4.y};
+          // Q2 row i: 32 B, 32B swizzle (chunk j at j ^ ((i >> 2) & 1)); D3, D4 rows 16 B
+          uint32_t qw[8];
 #pragma unroll
-          for (int wd = 0; wd < 8; ++wd) {  // word wd = elements 8wd..8wd+7 of the half
+          for (int j = 0; j < 2; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(cb + i * 32 + ((j ^ ((i >> 2) & 1)) << 4));
+            qw[4 * j] = v.x; qw[4 * j + 1] = v.y; qw[4 * j + 2] = v.z; qw[4 * j + 3] = v.w;
+          }
+          uint4 r3 = make_uint4(0, 0, 0, 0), r4 = make_uint4(0, 0, 0, 0);
+          if (T.bits >= 3) r3 = *reinterpret_cast<const uint4*>(cb + 4096 + i * 16);
+          if (T.bits >= 4) r4 = *reinterpret_cast<const uint4*>(cb + 6144 + i * 16);
+          const uint32_t d3w[4] = {r3.x, r3.y, r3.z, r3.w};
+          const uint32_t d4w[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+          for (int wd = 0; wd < 16; ++wd) {  // word wd = elements 8wd..8wd+7
             const uint32_t base = qw[wd >> 1] >> (16 * (wd & 1));
             const uint32_t b3 = d3w[wd >> 2] >> (8 * (wd & 3));
             const uint32_t b4 = d4w[wd >> 2] >> (8 * (wd & 3));
             w[wd] = (spread2(base) << 2) | (spread1(b3) << 1) | spread1(b4);
           }
         }
-        const uint32_t* szb = reinterpret_cast<const uint32_t*>(smem + C::OFF_SZ + cs * C::SZ_BYTES);
-        const uint32_t word = szb[(P.group == 64 ? h : 0) * 128 + i];
+        const uint32_t* szb = reinterpret_cast<const uint32_t*>(smem + C::OFF_SZ + (cs * 2 + m) * C::SZ_BYTES);
+        const uint32_t sz0 = szb[i];
+        const uint32_t sz1 = P.group == 64 ? szb[128 + i] : sz0;
         __syncwarp();
         if (lane == 0) mbar_arrive(codes_empty(cs));
         if (++cs == C::CSTAGES) { cs = 0; cph ^= 1; }
-
-        const int s = kbc % C::STAGES;
-        const int sph = (kbc / C::STAGES) & 1;
-        kbc += 2;
-        if (lane == 0) trace_put(trace, 3 + h, 7, t, kbc - 2);
-        ok = warp_wait(ab_empty(s), sph ^ 1, abort_flag, P.status);
-        if (!ok) break;
-        const __half sc = __float2half_rn(__uint_as_float(word << 16));
-        const float zf = __uint_as_float(word & 0xFFFF0000u);
-        const __half2 s2 = __half2half2(sc);
-        const __half2 z2 = __halves2half2(__float2half_rn(1024.0f + zf), __float2half_rn(64.0f + zf));
-        uint8_t* arow = smem + C::OFF_A + s * C::A_BYTES + i * 128;
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (lane == 0) trace_put(trace, 3 + m, 7, t, 2 * kc + h);
+          ok = warp_wait(ab_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
+          if (!ok) break;
+          if (live) {
+            const uint32_t word = h ? sz1 : sz0;
+            const __half sc = __float2half_rn(__uint_as_float(word << 16));
+            const float zf = __uint_as_float(word & 0xFFFF0000u);
+            const __half2 s2 = __half2half2(sc);
+            const __half2 z2 = __halves2half2(__float2half_rn(1024.0f + zf), __float2half_rn(64.0f + zf));
+            uint8_t* arow = smem + C::OFF_A + (s * 2 + m) * C::A_BYTES + i * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = elements 8j..8j+7 of the half
-          const uint4 o = dequant8(w[j], z2, s2);
-          *reinterpret_cast<uint4*>(arow + ((j ^ (i & 7)) << 4)) = o;
+            for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = elements 8j..8j+7 of the half
+              const uint4 o = dequant8(w[8 * h + j], z2, s2);
+              *reinterpret_cast<uint4*>(arow + ((j ^ (i & 7)) << 4)) = o;
+            }
+            fence_proxy_async_smem();
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(a_full(s));
+          if (++s == C::STAGES) { s = 0; sph ^= 1; }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(a_full(s));
       }
     }
   }
   // ---- epilogue: warps 12-15, TMEM lane quadrant = warp % 4 ---------------
-  else {
+  else if (warp >= 12) {
     const int q = warp & 3;
-    float* xch = reinterpret_cast<float*>(smem + C::OFF_X);  // [2][16][64]: up values by column
-    int acc = 0, aph = 0, xuse = 0;
+    int acc = 0, aph = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
       const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
-      if (lane == 0) trace_put(trace, 5 + (q >> 1), 8, t, 0);
-      ok = warp_wait(acc_full(acc), aph, abort_flag, P.status);
+      const bool m1 = has_m1(T.mb);
+      if (lane == 0) trace_put(trace, 5, 8, t, 0);
+      ok = warp_wait(acc_full(acc), aph, abort_flag, P.status, trace, bar0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * kNT;
-      for (int j0 = 0; j0 < T.nrows && ok; j0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(tbase + j0, v);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * (2 * kNT);
+      const int r = 32 * q + lane;  // row of the weight block
+      for (int j0 = 0; j0 < T.nrows; j0 += 16) {
+        uint32_t a0[16], a1[16];
+        tmem_ld16(tbase + j0, a0);
+        if (m1) tmem_ld16(tbase + kNT + j0, a1);
         tmem_ld_wait();
         if (GATEUP) {
-          // up rows (quadrants 2, 3) hand their values to the gate rows of
-          // the same features (quadrants 0, 1) through a two-slot buffer
-          const int xb = xuse & 1, xph = (xuse >> 1) & 1;
-          ++xuse;
-          float* xbuf = xch + xb * (16 * 64);
-          if (q >= 2) {
-            if (lane == 0) trace_put(trace, 6, 9, t, j0);
-            ok = warp_wait(x_empty(xb), xph ^ 1, abort_flag, P.status);
-            if (!ok) break;
+          const int f = T.mb * 128 + r;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xbuf[j * 64 + (q - 2) * 32 + lane] = __uint_as_float(v[j]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(x_full(xb));
-          } else {
-            if (lane == 0) trace_put(trace, 5, 10, t, j0);
-            ok = warp_wait(x_full(xb), xph, abort_flag, P.status);
-            if (!ok) break;
-            const int f = T.mb * 64 + 32 * q + lane;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (j0 + j < T.nrows) {
-                const float gv = __uint_as_float(v[j]), uv = xbuf[j * 64 + q * 32 + lane];
-                P.h_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + f] = __float2half_rn(silu_f(gv) * uv);
-              }
+          for (int j = 0; j < 16; ++j) {
+            if (j0 + j < T.nrows) {
+              const float gv = __uint_as_float(a0[j]), uv = __uint_as_float(a1[j]);
+              P.h_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + f] = __float2half_rn(silu_fast(gv) * uv);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(x_empty(xb));
           }
         } else {
-          const int n = T.mb * 128 + 32 * q + lane;
+          const int n0 = row_base(T.mb, 0) + r, n1 = row_base(T.mb, 1) + r;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (j0 + j < T.nrows)
-              P.y_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + n] = __uint_as_float(v[j]);
+          for (int j = 0; j < 16; ++j) {
+            if (j0 + j < T.nrows) {
+              float* yrow = P.y_out + static_cast<size_t>(T.row0 + j0 + j) * P.N;
+              yrow[n0] = __uint_as_float(a0[j]);
+              if (m1) yrow[n1] = __uint_as_float(a1[j]);
+            }
+          }
         }
       }
-      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(acc));
@@ -656,7 +661,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
   if (lane == 0) mbar_arrive(exit_bar);
   if (warp == 2) {
     if (lane == 0) trace_put(trace, 7, 14, 0, 0);
-    warp_wait(exit_bar, 0, abort_flag, P.status);
+    {  // not cut short by an abort: every warp must have left before TMEM goes
+      const uint64_t t0 = global_ns();
+      while (!mbar_try(exit_bar, 0) && global_ns() - t0 < kWaitLimitNs) {}
+      __syncwarp();
+    }
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
                  : "memory");
@@ -787,7 +796,7 @@ moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s) {
   const bool planes = a.layout == MOE_LAYOUT_PLANES;
   TcParams gu{};
   const int m_gu[2] = {0, 1};
-  moe_status_t st = make_params(gu, a, a.x_perm, a.total_rows, a.d, a.F, m_gu, 2, 64, n_blobs);
+  moe_status_t st = make_params(gu, a, a.x_perm, a.total_rows, a.d, a.F, m_gu, 2, 128, n_blobs);
   if (st != MOE_OK) return st;
   gu.h_out = a.h;
   gu.y_out = nullptr;
