@@ -178,20 +178,21 @@ MOE_API size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int 
  *   T        token count (no bin holds more than T rows; selects the
  *            decode GEMV regime for small T)
  *   workspace >= moe_ffn_workspace_bytes() bytes of device scratch
- *   y_perm   fp32 [total_rows][d]
- * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16. */
+ *   y_perm   bf16 [total_rows][d]
+ * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16 and
+ * each expert output row as bf16 (the combine sums them in fp32). */
 MOE_API moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, const void* blobs,
                                 const int32_t* slot_of, int total_rows, int T, int E, int d,
                                 int F, int group, int layout, void* workspace,
-                                size_t workspace_bytes, float* y_perm, int32_t* status,
+                                size_t workspace_bytes, void* y_perm, int32_t* status,
                                 moe_stream_t stream);
 
 /* moe_unpermute_combine -- weighted combine ([ExactMoE]: every chosen
  * expert's output is used as the router weighted it).
  *   y[t] = bf16( residual[t] + sum_{j<k} topk_w[t][j] * y_perm[inv_perm[t*k+j]] )
- * summed in fp32 in ascending j; residual bf16 [T][d] or NULL (0).
- *   y bf16 [T][d]; requires d % 4 == 0. */
-MOE_API moe_status_t moe_unpermute_combine(const float* y_perm, const int32_t* inv_perm,
+ * summed in fp32 in ascending j; y_perm bf16 [T*k][d]; residual bf16 [T][d]
+ * or NULL (0).  y bf16 [T][d]; requires d % 8 == 0 and 16-byte aligned rows. */
+MOE_API moe_status_t moe_unpermute_combine(const void* y_perm, const int32_t* inv_perm,
                                    const float* topk_w, const void* residual, int T, int k, int d,
                                    void* y, moe_stream_t stream);
 
@@ -229,7 +230,7 @@ MOE_API moe_status_t moe_slot_stage(moe_slot_cache* cache, const int32_t* ids_ho
  * expert is executed; results equal the all-resident call bit for bit. */
 MOE_API moe_status_t moe_slot_ffn(moe_slot_cache* cache, const void* x_perm, const int32_t* offsets,
                           int total_rows, int T, int d, int F, int group, int layout,
-                          void* workspace, size_t workspace_bytes, float* y_perm,
+                          void* workspace, size_t workspace_bytes, void* y_perm,
                           int32_t* status, moe_stream_t copy_stream, moe_stream_t compute_stream);
 
 /* Free the cache's host bookkeeping, events and device table (not the

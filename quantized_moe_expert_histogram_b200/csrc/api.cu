@@ -185,7 +185,7 @@ size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int layout) 
 moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, const void* blobs,
                                 const int32_t* slot_of, int total_rows, int T, int E, int d,
                                 int F, int group, int layout, void* workspace,
-                                size_t workspace_bytes, float* y_perm, int32_t* status,
+                                size_t workspace_bytes, void* y_perm, int32_t* status,
                                 moe_stream_t stream) {
   if (total_rows < 0 || T < 0 || E <= 0) {
     set_error("moe_grouped_ffn_wq: bad sizes");
@@ -230,17 +230,17 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   a.blob_bytes = L.bytes;
   a.lay = L;
   a.h = static_cast<__half*>(workspace);
-  a.y_perm = y_perm;
+  a.y_perm = static_cast<__nv_bfloat16*>(y_perm);
   a.status = status;
   const bool tc_ok = total_rows >= 16 && tc_supported(a);
   const bool use_tc = g_force_regime == 2 ? tc_ok : (g_force_regime == 1 ? false : (T > kGemvMaxT && tc_ok));
   return use_tc ? launch_ffn_tc(a, S(stream)) : launch_ffn_gemv(a, S(stream));
 }
 
-moe_status_t moe_unpermute_combine(const float* y_perm, const int32_t* inv_perm,
+moe_status_t moe_unpermute_combine(const void* y_perm, const int32_t* inv_perm,
                                    const float* topk_w, const void* residual, int T, int k, int d,
                                    void* y, moe_stream_t stream) {
-  if (T < 0 || k <= 0 || d <= 0 || d % 4) {
+  if (T < 0 || k <= 0 || d <= 0 || d % 8) {
     set_error("moe_unpermute_combine: bad sizes T=%d k=%d d=%d", T, k, d);
     return MOE_ERR_INVALID_ARG;
   }

@@ -64,7 +64,7 @@ size_t route_workspace_bytes(int T, int d, int E);
 moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void* x, int T, int d,
                             int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
                             int32_t* inv_perm, void* x_perm, int32_t* status, cudaStream_t s);
-moe_status_t launch_combine(const float* y_perm, const int32_t* inv_perm, const float* w,
+moe_status_t launch_combine(const void* y_perm, const int32_t* inv_perm, const float* w,
                             const void* residual, int T, int k, int d, void* y, cudaStream_t s);
 
 struct FfnArgs {
@@ -76,7 +76,7 @@ struct FfnArgs {
   size_t blob_bytes;
   BlobLayout lay;
   __half* h;          // workspace: fp16 [total_rows][F]
-  float* y_perm;
+  __nv_bfloat16* y_perm;  // [total_rows][d]
   int32_t* status;
 };
 moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);

@@ -306,7 +306,7 @@ moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_id
 
 moe_status_t moe_slot_ffn(moe_slot_cache* c, const void* x_perm, const int32_t* offsets,
                           int total_rows, int T, int d, int F, int group, int layout,
-                          void* workspace, size_t workspace_bytes, float* y_perm,
+                          void* workspace, size_t workspace_bytes, void* y_perm,
                           int32_t* status, moe_stream_t copy_stream,
                           moe_stream_t compute_stream) {
   if (!c) {

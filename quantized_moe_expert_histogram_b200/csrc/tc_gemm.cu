@@ -29,9 +29,10 @@
 //               UMMA K-major 128B-swizzled layout
 //   warps 12-15 epilogue: tcgen05.ld of its TMEM lane quadrant; gate/up
 //               pass writes h = silu(gate) * up (fp16), down pass y_perm
-//               (fp32)
-// Pipelines: codes (3 stages of 128 K) -> dequant -> A/B (3 stages of 64 K)
-// -> MMA -> TMEM (2 buffers) -> epilogue.  Every wait is bounded; on a
+//               (bf16)
+// Pipelines: codes (3 stages of 128 K) -> dequant -> A (2 stages of 64 K);
+// activations B (6 stages of 64 K); both -> MMA -> TMEM (2 buffers) ->
+// epilogue.  Every wait is bounded; on a
 // timeout the CTA raises MOE_DEV_TIMEOUT, drains its copies and MMAs,
 // frees TMEM and returns.  Warps reconverge after every wait, before any
 // warp-aligned instruction.
@@ -218,19 +219,20 @@ constexpr int kMaxBins = 768;
 constexpr int kNT = 128;       // largest token block (MMA N)
 
 struct Cfg {
-  static constexpr int STAGES = 3;    // A/B stages of 64 K
+  static constexpr int SA = 2;        // A (dequantised weight) stages of 64 K
+  static constexpr int SB = 6;        // B (activation) stages of 64 K: deep, to cover TMA latency
   static constexpr int CSTAGES = 3;   // codes stages of 128 K
   static constexpr int A_BYTES = 128 * 128;     // 128 weight rows x 64 fp16, per matrix
   static constexpr int B_BYTES = kNT * 128;     // 128 token rows x 64 fp16
   static constexpr int C_BYTES = 8192;          // per matrix: 128 rows x 128 K of codes
   static constexpr int SZ_BYTES = 1024;         // per matrix: 128 rows x up to 2 groups x 4 B
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * 2 * A_BYTES;
-  static constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_B = OFF_A + SA * 2 * A_BYTES;
+  static constexpr int OFF_C = OFF_B + SB * B_BYTES;
   static constexpr int OFF_SZ = OFF_C + CSTAGES * 2 * C_BYTES;
   static constexpr int OFF_TILE = OFF_SZ + CSTAGES * 2 * SZ_BYTES;  // int tile_start[769], off[769]
   static constexpr int OFF_BAR = OFF_TILE + 2 * (kMaxBins + 1) * 4 + 8;
-  static constexpr int N_BARS = 2 * CSTAGES + 3 * STAGES + 4 + 1 + 1;
+  static constexpr int N_BARS = 2 * CSTAGES + 2 * SA + 2 * SB + 4 + 1 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag
   static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + alignment slack
   static constexpr int TMEM_COLS = 512;                  // 2 buffers x 2 accumulators x kNT
@@ -249,7 +251,7 @@ struct TcParams {
   size_t sz_off[2];
   int K, N, nbins, planes_mult, group;
   __half* h_out;
-  float* y_out;
+  __nv_bfloat16* y_out;
   int32_t* status;
   int* trace;  // optional progress record (null in normal use)
 };
@@ -339,13 +341,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
   const uint32_t bar0 = smem_u32(bars);
   auto codes_full = [&](int i) { return bar0 + 8u * i; };
   auto codes_empty = [&](int i) { return bar0 + 8u * (C::CSTAGES + i); };
-  auto a_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + i); };
-  auto b_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + C::STAGES + i); };
-  auto ab_empty = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 2 * C::STAGES + i); };
-  auto acc_full = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + i); };
-  auto acc_empty = [&](int i) { return bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 2 + i); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 4);
-  const uint32_t exit_bar = bar0 + 8u * (2 * C::CSTAGES + 3 * C::STAGES + 5);
+  constexpr int kA = 2 * C::CSTAGES, kB = kA + 2 * C::SA, kR = kB + 2 * C::SB;
+  auto a_full = [&](int i) { return bar0 + 8u * (kA + i); };
+  auto a_empty = [&](int i) { return bar0 + 8u * (kA + C::SA + i); };
+  auto b_full = [&](int i) { return bar0 + 8u * (kB + i); };
+  auto b_empty = [&](int i) { return bar0 + 8u * (kB + C::SB + i); };
+  auto acc_full = [&](int i) { return bar0 + 8u * (kR + i); };
+  auto acc_empty = [&](int i) { return bar0 + 8u * (kR + 2 + i); };
+  const uint32_t drain_bar = bar0 + 8u * (kR + 4);
+  const uint32_t exit_bar = bar0 + 8u * (kR + 5);
   int* trace = P.trace ? P.trace + (GATEUP ? 0 : gridDim.x * 16) : nullptr;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -362,10 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       mbar_init(codes_full(i), 1);
       mbar_init(codes_empty(i), 8);
     }
-    for (int i = 0; i < C::STAGES; ++i) {
+    for (int i = 0; i < C::SA; ++i) {
       mbar_init(a_full(i), 8);
+      mbar_init(a_empty(i), 1);
+    }
+    for (int i = 0; i < C::SB; ++i) {
       mbar_init(b_full(i), 1);
-      mbar_init(ab_empty(i), 1);
+      mbar_init(b_empty(i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full(i), 1);
@@ -463,12 +470,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         } else {
           for (int kb = 0; kb < 2 * KC && ok; ++kb) {
             trace_put(trace, 2, 2, t, kb);
-            ok = mbar_wait(ab_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
+            ok = mbar_wait(b_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
             if (!ok) break;
             mbar_expect_tx(b_full(s), T.nt * 128);
             const uint32_t bdst = smem_u32(smem + C::OFF_B + s * C::B_BYTES);
             for (int i = 0; i < T.nt / 16; ++i) tma_load_2d(bdst + i * 2048, &P.act, kb * 64, T.row0 + 16 * i, b_full(s));
-            if (++s == C::STAGES) { s = 0; sph ^= 1; }
+            if (++s == C::SB) { s = 0; sph ^= 1; }
           }
         }
       }
@@ -482,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
             while (!mbar_try(codes_full(idx), ph) && global_ns() - t0 < kWaitLimitNs) {}
           }
         } else {
-          for (int idx = 0; idx < C::STAGES; ++idx) {
+          for (int idx = 0; idx < C::SB; ++idx) {
             const int ph = (idx < s) ? sph : sph ^ 1;
             while (!mbar_try(b_full(idx), ph) && global_ns() - t0 < kWaitLimitNs) {}
           }
@@ -493,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
   // ---- MMA issuer --------------------------------------------------------
   else if (warp == 1) {
     if (lane == 0) {
-      int s = 0, sph = 0, acc = 0, aph = 0;
+      int sa = 0, saph = 0, sb = 0, sbph = 0, acc = 0, aph = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
@@ -506,21 +513,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         const uint32_t dcol = tmem_base + acc * (2 * kNT);
         for (int kb = 0; kb < 2 * KC && ok; ++kb) {
           trace_put(trace, 1, 4, t, kb);
-          ok = mbar_wait(a_full(s), sph, abort_flag, P.status, trace, bar0);
+          ok = mbar_wait(a_full(sa), saph, abort_flag, P.status, trace, bar0);
           if (!ok) break;
           trace_put(trace, 1, 5, t, kb);
-          ok = mbar_wait(b_full(s), sph, abort_flag, P.status, trace, bar0);
+          ok = mbar_wait(b_full(sb), sbph, abort_flag, P.status, trace, bar0);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::OFF_B + s * C::B_BYTES));
+          const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::OFF_B + sb * C::B_BYTES));
           for (int m = 0; m < nm; ++m) {
-            const uint64_t adesc = umma_desc_sw128(smem_u32(smem + C::OFF_A + (s * 2 + m) * C::A_BYTES));
+            const uint64_t adesc = umma_desc_sw128(smem_u32(smem + C::OFF_A + (sa * 2 + m) * C::A_BYTES));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               umma_f16(dcol + m * kNT, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
           }
-          umma_commit(ab_empty(s));
-          if (++s == C::STAGES) { s = 0; sph ^= 1; }
+          umma_commit(a_empty(sa));
+          umma_commit(b_empty(sb));
+          if (++sa == C::SA) { sa = 0; saph ^= 1; }
+          if (++sb == C::SB) { sb = 0; sbph ^= 1; }
         }
         if (!ok) break;
         umma_commit(acc_full(acc));
@@ -584,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         if (++cs == C::CSTAGES) { cs = 0; cph ^= 1; }
         for (int h = 0; h < 2 && ok; ++h) {
           if (lane == 0) trace_put(trace, 3 + m, 7, t, 2 * kc + h);
-          ok = warp_wait(ab_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
+          ok = warp_wait(a_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
           if (!ok) break;
           if (live) {
             const uint32_t word = h ? sz1 : sz0;
@@ -602,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(a_full(s));
-          if (++s == C::STAGES) { s = 0; sph ^= 1; }
+          if (++s == C::SA) { s = 0; sph ^= 1; }
         }
       }
     }
@@ -640,9 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (j0 + j < T.nrows) {
-              float* yrow = P.y_out + static_cast<size_t>(T.row0 + j0 + j) * P.N;
-              yrow[n0] = __uint_as_float(a0[j]);
-              if (m1) yrow[n1] = __uint_as_float(a1[j]);
+              __nv_bfloat16* yrow = P.y_out + static_cast<size_t>(T.row0 + j0 + j) * P.N;
+              yrow[n0] = __float2bfloat16_rn(__uint_as_float(a0[j]));
+              if (m1) yrow[n1] = __float2bfloat16_rn(__uint_as_float(a1[j]));
             }
           }
         }

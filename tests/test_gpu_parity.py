@@ -134,7 +134,7 @@ def _check_layer(shape, T, seed=0, token_subset=None):
     ok, worst = within_tol(y[toks], ref["y"][toks])
     assert ok, f"worst err/tol = {worst:.3f}"
     # per-assignment expert outputs (before the combine)
-    yp = v["y_perm"].cpu().numpy()
+    yp = v["y_perm"].float().cpu().numpy()
     rows = np.array([a for t in toks for a in range(t * shape.k, (t + 1) * shape.k)])
     ok2, worst2 = within_tol(yp[ref["inv_perm"][rows]], ref["y_assign"][rows])
     assert ok2, f"y_perm worst err/tol = {worst2:.3f}"

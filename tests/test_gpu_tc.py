@@ -32,7 +32,7 @@ def _check(shape, T, seed=0):
     ref, _ = oracle_layer(shape, L, bits=bits)
     np.testing.assert_array_equal(v["perm"].cpu().numpy(), ref["perm"])
     assert int(v["status"].item()) == 0, f"device status {int(v['status'].item())}"
-    yp = v["y_perm"].cpu().numpy()
+    yp = v["y_perm"].float().cpu().numpy()
     ok2, worst2 = within_tol(yp[ref["inv_perm"]], ref["y_assign"])
     ok, worst = within_tol(y, ref["y"])
     assert ok2, f"y_perm worst err/tol = {worst2:.3f}"
