@@ -139,6 +139,7 @@ MOE_API moe_status_t moe_route_topk(const void* x, const float* w_router, const 
 /* Device scratch moe_route_topk needs (per-slice fp64 partial logits). */
 MOE_API size_t moe_route_workspace_bytes(int T, int d, int E);
 
+
 /* moe_permute -- per-expert histogram, exclusive prefix sum and stable
  * permutation of the T*k assignments a = t*k + j ([Read-ME] expert-aware
  * batching; [ExactMoE] grouped execution).  No atomics: per-warp
@@ -178,9 +179,8 @@ MOE_API size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int 
  *   T        token count (no bin holds more than T rows; selects the
  *            decode GEMV regime for small T)
  *   workspace >= moe_ffn_workspace_bytes() bytes of device scratch
- *   y_perm   bf16 [total_rows][d]
- * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16 and
- * each expert output row as bf16 (the combine sums them in fp32). */
+ *   y_perm   fp32 [total_rows][d]
+ * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16. */
 MOE_API moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, const void* blobs,
                                 const int32_t* slot_of, int total_rows, int T, int E, int d,
                                 int F, int group, int layout, void* workspace,
@@ -190,7 +190,7 @@ MOE_API moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offse
 /* moe_unpermute_combine -- weighted combine ([ExactMoE]: every chosen
  * expert's output is used as the router weighted it).
  *   y[t] = bf16( residual[t] + sum_{j<k} topk_w[t][j] * y_perm[inv_perm[t*k+j]] )
- * summed in fp32 in ascending j; y_perm bf16 [T*k][d]; residual bf16 [T][d]
+ * summed in fp32 in ascending j; y_perm fp32 [T*k][d]; residual bf16 [T][d]
  * or NULL (0).  y bf16 [T][d]; requires d % 8 == 0 and 16-byte aligned rows. */
 MOE_API moe_status_t moe_unpermute_combine(const void* y_perm, const int32_t* inv_perm,
                                    const float* topk_w, const void* residual, int T, int k, int d,

@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/moeq.h"
+#include "moeq.h"
 
 namespace moeq {
 
@@ -76,7 +76,7 @@ struct FfnArgs {
   size_t blob_bytes;
   BlobLayout lay;
   __half* h;          // workspace: fp16 [total_rows][F]
-  __nv_bfloat16* y_perm;  // [total_rows][d]
+  float* y_perm;  // [total_rows][d]
   int32_t* status;
 };
 moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);

@@ -12,7 +12,7 @@
 // mode, resident) bins; blockIdx.x a block of 8 warps x RW output rows.
 //
 //   gate/up pass:  h[p][f]      = silu(Wg[f] . x_p) * (Wu[f] . x_p)   (fp16)
-//   down pass:     y_perm[p][n] = Wd[n] . h_p                          (bf16)
+//   down pass:     y_perm[p][n] = Wd[n] . h_p                          (fp32)
 #include <algorithm>
 
 #include "common.cuh"
@@ -36,7 +36,7 @@ struct GemvParams {
   int K, N, nbins, planes_mult;  // planes_mult: 1 for INT4 bins, 3 for (e,b) bins
   int group;
   __half* h_out;            // gate/up pass output [rows][N]
-  __nv_bfloat16* y_out;     // down pass output [rows][N]
+  float* y_out;             // down pass output [rows][N]
 };
 
 // 8 two-bit fields (bits 2i..2i+1) -> bits 4i..4i+1.
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_gemv(const GemvParams P
           const float g = acc[2 * j][t], u = acc[2 * j + 1][t];
           P.h_out[p * P.N + n0 + j] = __float2half_rn(silu_f(g) * u);
         } else {
-          P.y_out[p * P.N + n0 + j] = __float2bfloat16_rn(acc[j][t]);
+          P.y_out[p * P.N + n0 + j] = acc[j][t];
         }
       }
     }

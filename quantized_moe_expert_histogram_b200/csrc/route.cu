@@ -222,3 +222,4 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
 }
 
 }  // namespace moeq
+

@@ -29,9 +29,9 @@
 //               UMMA K-major 128B-swizzled layout
 //   warps 12-15 epilogue: tcgen05.ld of its TMEM lane quadrant; gate/up
 //               pass writes h = silu(gate) * up (fp16), down pass y_perm
-//               (bf16)
-// Pipelines: codes (3 stages of 128 K) -> dequant -> A (2 stages of 64 K);
-// activations B (6 stages of 64 K); both -> MMA -> TMEM (2 buffers) ->
+//               (fp32)
+// Pipelines: codes (2 stages of 128 K) -> dequant -> A (4 stages of 64 K);
+// activations B (3 stages of 64 K); both -> MMA -> TMEM (2 buffers) ->
 // epilogue.  Every wait is bounded; on a
 // timeout the CTA raises MOE_DEV_TIMEOUT, drains its copies and MMAs,
 // frees TMEM and returns.  Warps reconverge after every wait, before any
@@ -79,6 +79,22 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try, but lets the hardware suspend the thread for up to
+// `hint_ns` while the phase is incomplete (it resumes as soon as the phase
+// completes), so waiting warps do not spin on the issue slots that the
+// working warps of the same SM sub-partition need.
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -95,8 +111,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try(bar, parity)) return true;
-    if ((i & 63) == 0) {
+    if (mbar_try_sleep(bar, parity, 20000u)) return true;
+    if ((i & 7) == 0) {
       if (*abort_flag) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
         *abort_flag = 1;
@@ -219,9 +235,9 @@ constexpr int kMaxBins = 768;
 constexpr int kNT = 128;       // largest token block (MMA N)
 
 struct Cfg {
-  static constexpr int SA = 2;        // A (dequantised weight) stages of 64 K
-  static constexpr int SB = 6;        // B (activation) stages of 64 K: deep, to cover TMA latency
-  static constexpr int CSTAGES = 3;   // codes stages of 128 K
+  static constexpr int SA = 4;        // A (dequantised weight) stages of 64 K
+  static constexpr int SB = 3;        // B (activation) stages of 64 K
+  static constexpr int CSTAGES = 2;   // codes stages of 128 K
   static constexpr int A_BYTES = 128 * 128;     // 128 weight rows x 64 fp16, per matrix
   static constexpr int B_BYTES = kNT * 128;     // 128 token rows x 64 fp16
   static constexpr int C_BYTES = 8192;          // per matrix: 128 rows x 128 K of codes
@@ -251,7 +267,7 @@ struct TcParams {
   size_t sz_off[2];
   int K, N, nbins, planes_mult, group;
   __half* h_out;
-  __nv_bfloat16* y_out;
+  float* y_out;
   int32_t* status;
   int* trace;  // optional progress record (null in normal use)
 };
@@ -649,9 +665,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (j0 + j < T.nrows) {
-              __nv_bfloat16* yrow = P.y_out + static_cast<size_t>(T.row0 + j0 + j) * P.N;
-              yrow[n0] = __float2bfloat16_rn(__uint_as_float(a0[j]));
-              if (m1) yrow[n1] = __float2bfloat16_rn(__uint_as_float(a1[j]));
+              float* yrow = P.y_out + static_cast<size_t>(T.row0 + j0 + j) * P.N;
+              yrow[n0] = __uint_as_float(a0[j]);
+              if (m1) yrow[n1] = __uint_as_float(a1[j]);
             }
           }
         }

@@ -1,0 +1,148 @@
+"""Offload mode: stacked layers whose experts live in pinned host memory and
+reach the GPU through a per-layer slot cache (moe_slot_cache_create,
+moe_slot_stage, moe_slot_ffn).  Sources: ExactMoE (compressed experts in
+host memory, GPU-resident slot cache; offload changes where experts are
+stored, not what is computed), EdgeMoE (expert buffer filled on
+activation), D2MoE (load the next expert while computing the current one).
+
+Checks: every layer's output equals the all-resident path bit for bit; the
+resident path matches the oracle per layer; cache statistics add up; and
+host-side fault injection fails a stage cleanly without corrupting later
+steps."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from quantized_moe_expert_histogram_b200 import build
+from quantized_moe_expert_histogram_b200 import inputs as I
+from quantized_moe_expert_histogram_b200 import moeq
+from quantized_moe_expert_histogram_b200.layer import QuantMoELayer
+
+from gpu_helpers import within_tol
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+    moeq.load()
+
+
+class Stack:
+    """Layers of one shape; each layer's experts packed on the GPU, then
+    copied to pinned host memory for its slot cache."""
+
+    def __init__(self, shape, layers, slots, batch, seed=0):
+        self.shape, self.n, self.batch = shape, layers, batch
+        self.layers, self.host, self.pools, self.caches = [], [], [], []
+        for l in range(layers):
+            w = I.make_expert_weights(shape, seed=seed + 101 * l, device="cuda")
+            r = I.make_router(shape, seed=seed + 101 * l + 1, device="cuda")
+            layer = QuantMoELayer.from_weights(shape, r["w_router"], r["bias"], w["w_gate"], w["w_up"],
+                                               w["w_down"], max_tokens=batch)
+            host = layer.blobs.cpu().pin_memory()
+            pool = torch.empty(slots, layer.blobs.shape[1], dtype=torch.uint8, device="cuda")
+            self.layers.append((layer, w))
+            self.host.append(host)
+            self.pools.append(pool)
+            self.caches.append(moeq.SlotCache(shape.E, slots, layer.blobs.shape[1], host, pool))
+        self.copy = torch.cuda.Stream()
+        self.compute = torch.cuda.current_stream()
+
+    def step(self, x, ids, offload):
+        """One decode step through all layers; returns per-layer inputs and outputs."""
+        xs, ys, stats = [x], [], []
+        for l, (layer, _) in enumerate(self.layers):
+            v = layer.views(self.batch)
+            forced = ids[l].contiguous()
+            moeq.moe_route_topk(xs[-1], layer.w_router, layer.bias, self.shape.k, forced_idx=forced,
+                                topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"])
+            moeq.moe_permute(v["topk_idx"], self.shape.E, x=xs[-1], out=v, status=v["status"])
+            if offload:
+                routed = v["topk_idx"].cpu()  # the one device->host crossing per layer
+                nw, st = self.caches[l].stage(routed.reshape(-1), self.copy, self.compute)
+                stats.append(st + [nw])
+                self.caches[l].ffn(v["x_perm"], v["offsets"], self.batch, self.shape.d, self.shape.F,
+                                   self.shape.group, layer.layout, v["workspace"], v["y_perm"], v["status"],
+                                   self.copy, self.compute)
+            else:
+                moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, self.batch, self.shape.E,
+                                        self.shape.d, self.shape.F, self.shape.group, layer.layout,
+                                        workspace=v["workspace"], y_perm=v["y_perm"], status=v["status"])
+            y = torch.empty_like(xs[-1])
+            moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], residual=xs[-1], y=y)
+            torch.cuda.synchronize()
+            assert int(v["status"].item()) == 0
+            ys.append(y)
+            xs.append(y)
+        return xs, ys, stats
+
+    def close(self):
+        for c in self.caches:
+            c.close()
+
+
+def _small_stack(slots=4):
+    shape = I.custom_shape(d=256, E=16, k=4, F=256, group=64)
+    return shape, Stack(shape, layers=3, slots=slots, batch=8, seed=5)
+
+
+def test_slot_mode_equals_resident_and_oracle():
+    shape, st = _small_stack()
+    trace = I.make_slot_trace(shape.E, shape.k, 3, steps=4, batch=8, seed=3).cuda()
+    xs_all = I.make_slot_x(shape.d, 4, 8, seed=3, device="cuda")
+    total = np.zeros(3, dtype=np.int64)
+    for s in range(4):
+        xs_r, ys_r, _ = st.step(xs_all[s], trace[s], offload=False)
+        xs_o, ys_o, stats = st.step(xs_all[s], trace[s], offload=True)
+        for l in range(3):
+            assert torch.equal(ys_o[l], ys_r[l]), f"step {s} layer {l}: offload differs from resident"
+            hits, misses, nbytes, nw = stats[l]
+            distinct = len(set(trace[s, l].reshape(-1).tolist()))
+            assert hits + misses == distinct and nbytes == misses * st.host[l].shape[1]
+            assert nw == -(-distinct // 2)  # waves of slots/2 experts
+            total += np.array([hits, misses, nbytes])
+        # the resident path against the oracle, layer by layer (inputs from the GPU chain)
+        for l, (layer, w) in enumerate(st.layers):
+            ex = O.QuantExperts(w["w_gate"].cpu().numpy(), w["w_up"].cpu().numpy(), w["w_down"].cpu().numpy(),
+                                shape.group)
+            x = xs_r[l].float().cpu().numpy()
+            ref = O.moe_layer(x, layer.w_router.cpu().numpy(), None, shape.k, ex,
+                              sel=trace[s, l].cpu().numpy())
+            ok, worst = within_tol(ys_r[l].float().cpu().numpy(), x + ref["y"])
+            assert ok, f"step {s} layer {l}: worst err/tol {worst:.3f}"
+    assert total[0] > 0 and total[1] > 0  # both hits and misses happened
+    st.close()
+
+
+def test_slot_stage_fault_injection_recovers():
+    shape, st = _small_stack()
+    trace = I.make_slot_trace(shape.E, shape.k, 3, steps=3, batch=8, seed=4).cuda()
+    xs_all = I.make_slot_x(shape.d, 3, 8, seed=4, device="cuda")
+    _, ys_ref, _ = st.step(xs_all[0], trace[0], offload=False)
+    # a stage that fails before queuing anything
+    moeq.moe_debug_inject_fault(1, 1)
+    with pytest.raises(moeq.MoeError) as ei:
+        st.step(xs_all[0], trace[0], offload=True)
+    assert ei.value.code == 7
+    # a copy that fails half way through staging
+    moeq.moe_debug_inject_fault(2, 1)
+    with pytest.raises(moeq.MoeError) as ei:
+        st.step(xs_all[0], trace[0], offload=True)
+    assert ei.value.code == 7
+    moeq.moe_debug_inject_fault(0, 0)
+    torch.cuda.synchronize()
+    # later steps are still exact
+    _, ys_o, _ = st.step(xs_all[0], trace[0], offload=True)
+    for l in range(3):
+        assert torch.equal(ys_o[l], ys_ref[l])
+    st.close()
+
+
+def test_slot_cache_rejects_bad_arguments():
+    shape, st = _small_stack()
+    with pytest.raises(moeq.MoeError):
+        st.caches[0].stage(torch.tensor([0, 99], dtype=torch.int32), st.copy, st.compute)
+    st.close()
