@@ -139,6 +139,26 @@ MOE_API moe_status_t moe_route_topk(const void* x, const float* w_router, const 
 /* Device scratch moe_route_topk needs (per-slice fp64 partial logits). */
 MOE_API size_t moe_route_workspace_bytes(int T, int d, int E);
 
+/* moe_route_topk_noalloc -- the same router with no workspace argument.
+ * (Library plumbing: the pages describe no counterpart.)  For callers that
+ * cannot allocate device memory where they route: code running during
+ * CUDA graph stream capture (no cudaMalloc allowed), plugins that receive
+ * only a stream and no allocator, and serving paths that must not risk an
+ * allocation failure or its implicit synchronisation.  The scratch lives in
+ * a fixed 8 MiB device array inside the library, which every GPU that loads
+ * the library holds until the process exits; the call allocates nothing.
+ *   - Arguments and results are those of moe_route_topk.
+ *   - Sizes whose scratch (moe_route_workspace_bytes) exceeds 8 MiB are
+ *     rejected with MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - The first call on a device resolves the array's device address for
+ *     that device (cudaGetSymbolAddress, with that device current); make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array: calls that may overlap on
+ *     the GPU (different streams without ordering) race and must not be
+ *     issued.  Nothing in the array needs clearing between calls. */
+MOE_API moe_status_t moe_route_topk_noalloc(const void* x, const float* w_router, const float* bias,
+                                            const int32_t* forced_idx, int T, int d, int E, int k,
+                                            int32_t* topk_idx, float* topk_w, moe_stream_t stream);
 
 /* moe_permute -- per-expert histogram, exclusive prefix sum and stable
  * permutation of the T*k assignments a = t*k + j ([Read-ME] expert-aware

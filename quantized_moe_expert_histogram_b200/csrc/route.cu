@@ -223,3 +223,70 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
 
 }  // namespace moeq
 
+// ---------------------------------------------------------------------------
+// Allocation-free router entry point.
+//
+// Some callers cannot allocate device memory at the point where they route:
+// code that runs while a stream is being captured into a CUDA graph (where
+// cudaMalloc is not allowed), plugins and runtimes that hand us only a
+// stream and have no allocator of their own to lend, and latency-critical
+// serving paths that must not risk an allocation failure or an implicit
+// synchronisation.  moe_route_topk_noalloc keeps the router's scratch (the
+// per-slice fp64 partial logits) in a fixed device array owned by this
+// library instead of a caller-provided workspace.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace moeq {
+namespace {
+
+constexpr size_t kRouteScratchBytes = 8u << 20;  // 8 MiB, held by every GPU that loads the library
+static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, resolved once
+// per device (with that device current).
+moe_status_t route_scratch(void** out) {
+  int dev = 0;
+  moe_status_t st = cuda_check(cudaGetDevice(&dev), "moe_route_topk_noalloc: cudaGetDevice");
+  if (st != MOE_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) {
+    set_error("moe_route_topk_noalloc: device %d beyond the supported %d", dev, kMaxDevices);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    st = cuda_check(cudaGetSymbolAddress(&p, g_route_scratch), "moe_route_topk_noalloc: cudaGetSymbolAddress");
+    if (st != MOE_OK) return st;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moeq
+
+extern "C" moe_status_t moe_route_topk_noalloc(const void* x, const float* w_router, const float* bias,
+                                                const int32_t* forced_idx, int T, int d, int E, int k,
+                                                int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+  using namespace moeq;
+  const size_t need = route_workspace_bytes(T, d, E);
+  if (T > 0 && need > kRouteScratchBytes) {
+    set_error("moe_route_topk_noalloc: T=%d d=%d E=%d needs %zu bytes of scratch, above the fixed %zu",
+              T, d, E, need, kRouteScratchBytes);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  void* scratch = nullptr;
+  if (T > 0) {
+    moe_status_t st = route_scratch(&scratch);
+    if (st != MOE_OK) return st;
+  }
+  return moe_route_topk(x, w_router, bias, forced_idx, T, d, E, k, topk_idx, topk_w, scratch,
+                        kRouteScratchBytes, stream);
+}

@@ -35,6 +35,7 @@ _SIGS = {
     "moe_route_topk": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p, _c_sz,
                               _c_p]),
     "moe_route_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
+    "moe_route_topk_noalloc": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]),
     "moe_permute": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_p,
                            _c_p, _c_p]),
     "moe_ffn_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
@@ -273,3 +274,20 @@ def moe_debug_set_trace(pinned_int32=None):
     """Progress record of the tensor-core FFN kernels (test hook)."""
     load().moe_debug_set_trace(None if pinned_int32 is None else pinned_int32.data_ptr())
 
+
+
+def moe_route_topk_noalloc(x, w_router, bias, k, forced_idx=None, topk_idx=None, topk_w=None, stream=None):
+    """The router without a workspace argument: its scratch is a fixed
+    device array inside the library (see include/moeq.h)."""
+    lib = load()
+    T, d = x.shape
+    E = w_router.shape[0]
+    if topk_idx is None:
+        topk_idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    _check("moe_route_topk_noalloc", lib.moe_route_topk_noalloc(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_router, torch.float32, "w_router"),
+        _ptr(bias, torch.float32, "bias"), _ptr(forced_idx, torch.int32, "forced_idx"), T, d, E, k,
+        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"), _stream(stream)))
+    return topk_idx, topk_w
