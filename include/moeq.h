@@ -162,8 +162,10 @@ MOE_API moe_status_t moe_route_topk_noalloc(const void* x, const float* w_router
 
 /* moe_permute -- per-expert histogram, exclusive prefix sum and stable
  * permutation of the T*k assignments a = t*k + j ([Read-ME] expert-aware
- * batching; [ExactMoE] grouped execution).  No atomics: per-warp
- * histograms, one block scan, and a rank-by-warp-match scatter.
+ * batching; [ExactMoE] grouped execution).  No atomics: per-block
+ * histograms of 1024 assignments, one scan over (bin, block), and a
+ * rank-by-warp-match scatter that also gathers the rows.
+ *   workspace >= moe_permute_workspace_bytes(T, E, k, bits != NULL) bytes.
  *   bits uint8 [T][k] or NULL.  NULL: bin of a = topk_idx[a] (nbins = E).
  *        Given ([D2MoE] bit gate): bin = 3*topk_idx[a] + (bits[a]-2),
  *        nbins = 3E, bits in {2,3,4}.
@@ -177,7 +179,12 @@ MOE_API moe_status_t moe_route_topk_noalloc(const void* x, const float* w_router
  * |x| > 65504 flags MOE_DEV_RANGE.  Requires T*k <= 2^24, nbins <= 768. */
 MOE_API moe_status_t moe_permute(const int32_t* topk_idx, const uint8_t* bits, const void* x, int T,
                          int d, int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
-                         int32_t* inv_perm, void* x_perm, int32_t* status, moe_stream_t stream);
+                         int32_t* inv_perm, void* x_perm, int32_t* status, void* workspace,
+                         size_t workspace_bytes, moe_stream_t stream);
+
+/* Device scratch moe_permute needs (per-block histograms); nested != 0 for
+ * the (expert, width) bins. */
+MOE_API size_t moe_permute_workspace_bytes(int T, int E, int k, int nested);
 
 /* Workspace bytes moe_grouped_ffn_wq needs for `total_rows` = T*k rows. */
 MOE_API size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int layout);

@@ -147,9 +147,15 @@ moe_status_t moe_route_topk(const void* x, const float* w_router, const float* b
                       S(stream));
 }
 
+size_t moe_permute_workspace_bytes(int T, int E, int k, int nested) {
+  if (T < 0 || E <= 0 || k <= 0) return 0;
+  return permute_workspace_bytes(T, k, nested ? 3 * E : E);
+}
+
 moe_status_t moe_permute(const int32_t* topk_idx, const uint8_t* bits, const void* x, int T,
                          int d, int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
-                         int32_t* inv_perm, void* x_perm, int32_t* status, moe_stream_t stream) {
+                         int32_t* inv_perm, void* x_perm, int32_t* status, void* workspace,
+                         size_t workspace_bytes, moe_stream_t stream) {
   if (T < 0 || E <= 0 || k <= 0 || k > E) {
     set_error("moe_permute: bad sizes T=%d E=%d k=%d", T, E, k);
     return MOE_ERR_INVALID_ARG;
@@ -170,8 +176,13 @@ moe_status_t moe_permute(const int32_t* topk_idx, const uint8_t* bits, const voi
     set_error("moe_permute: gather needs d %% 8 == 0 and 16-byte aligned x / x_perm");
     return MOE_ERR_INVALID_ARG;
   }
+  const size_t need = permute_workspace_bytes(T, k, bits ? 3 * E : E);
+  if (!workspace || workspace_bytes < need) {
+    set_error("moe_permute: workspace %zu < %zu bytes", workspace_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
   return launch_permute(topk_idx, bits, x, T, d, E, k, counts, offsets, perm, inv_perm, x_perm,
-                        status, S(stream));
+                        status, workspace, S(stream));
 }
 
 size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int layout) {

@@ -63,7 +63,9 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
 size_t route_workspace_bytes(int T, int d, int E);
 moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void* x, int T, int d,
                             int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
-                            int32_t* inv_perm, void* x_perm, int32_t* status, cudaStream_t s);
+                            int32_t* inv_perm, void* x_perm, int32_t* status, void* workspace,
+                            cudaStream_t s);
+size_t permute_workspace_bytes(int T, int k, int nbins);
 moe_status_t launch_combine(const void* y_perm, const int32_t* inv_perm, const float* w,
                             const void* residual, int T, int k, int d, void* y, cudaStream_t s);
 

@@ -1,27 +1,37 @@
 // Per-expert histogram, exclusive prefix sum and stable permutation of the
-// T*k assignments, then the gather of activation rows into expert order.
+// T*k assignments, plus the gather of activation rows into expert order.
 //
-// One CTA of 32 warps sorts all assignments without atomics:
-//   pass 1  warp w counts the keys of its contiguous chunk; inside a
-//           32-assignment slice the lanes with equal keys are found with
-//           __match_any_sync and the lowest of them adds the group size to
-//           the warp's private histogram row;
-//   scan    thread b turns column b of the [warps][bins] histogram into
-//           per-warp start positions and the bin total; a block scan of
-//           the totals gives offsets;
-//   pass 2  warp w re-reads its chunk; a lane's position is its warp's
-//           cursor for the key plus the number of lower lanes with the same
-//           key in the slice, so the order inside a bin is ascending a.
+// Three kernels, deterministic and atomics-free:
+//   k_perm_hist     CTA c owns assignments [c*CH, (c+1)*CH); each warp
+//                   counts its 32-wide slices: lanes with equal keys are
+//                   found with __match_any_sync and the lowest of them adds
+//                   the group size to the warp's shared histogram; the CTA
+//                   histogram (warps summed in order) goes to hist[bin][c].
+//   k_perm_scan     one CTA: thread b turns row b of hist into per-CTA start
+//                   positions inside bin b and the bin total; a block scan
+//                   of the totals gives offsets, added to every start.
+//   k_perm_scatter  CTA c recounts its warps, so that warp w starts at the
+//                   CTA's start plus the counts of warps 0..w-1; a lane's
+//                   position is its warp's cursor plus the number of lower
+//                   lanes with the same key in the slice (ascending a inside
+//                   a bin).  It writes perm and inv_perm.
+// When all assignments fit one CTA's chunk (T*k <= 1024, decode-sized
+// batches) k_perm_one does the three steps in a single launch.  The gather
+// of activation rows (bf16 -> fp16) is its own grid-wide launch: it moves
+// T*k*d*2 bytes and needs every SM, while the sort needs only T*k/1024
+// CTAs.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 
 namespace moeq {
 namespace {
 
-constexpr int kWarps = 32;
+constexpr int kWarps = 8;                   // per CTA
+constexpr int kSlices = 4;                  // 32-assignment slices per warp
+constexpr int kCH = kWarps * 32 * kSlices;  // assignments per CTA (1024)
 constexpr int kMaxBins = 768;
-constexpr int kBatch = 16;  // 32-assignment slices whose keys are loaded together
 
 __device__ __forceinline__ int load_key(const int32_t* idx, const uint8_t* bits, int a, int E,
                                         int32_t* status) {
@@ -39,57 +49,61 @@ __device__ __forceinline__ int load_key(const int32_t* idx, const uint8_t* bits,
   return 3 * e + (b - 2);
 }
 
-__global__ void __launch_bounds__(kWarps * 32) k_permute(const int32_t* __restrict__ idx,
-                                                          const uint8_t* __restrict__ bits, int n,
-                                                          int E, int nbins,
-                                                          int32_t* __restrict__ counts,
-                                                          int32_t* __restrict__ offsets,
-                                                          int32_t* __restrict__ perm,
-                                                          int32_t* __restrict__ inv_perm,
-                                                          int32_t* status, int stage_perm) {
-  extern __shared__ int32_t hist[];  // [kWarps][nbins], then perm staging [n] when stage_perm
-  int32_t* perm_s = hist + kWarps * nbins;
-  __shared__ int32_t scan_buf[kWarps];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+// Per-warp histograms of this CTA's chunk into smem [kWarps][nbins]; the
+// keys of the warp's slices are returned in `keys` (-1 past the end).
+__device__ __forceinline__ void warp_hist(const int32_t* idx, const uint8_t* bits, int n, int E,
+                                          int nbins, int32_t* hist_s, int32_t* status,
+                                          int (&keys)[kSlices]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned lt_mask = (1u << lane) - 1u;
-
-  for (int i = tid; i < kWarps * nbins; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-
-  const int chunk = ((n + kWarps - 1) / kWarps + 31) & ~31;
-  const int begin = warp * chunk;
-  const int end = min(n, begin + chunk);
-  int32_t* my = hist + warp * nbins;
-
-  // Keys are fetched kBatch slices at a time (independent loads in flight),
-  // then consumed slice by slice.
-  for (int base = begin; base < end; base += 32 * kBatch) {
-    int keys[kBatch];
+  const int base = blockIdx.x * kCH + warp * 32 * kSlices;
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int a = base + 32 * u + lane;
-      keys[u] = a < end ? load_key(idx, bits, a, E, status) : -1;
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const unsigned peers = __match_any_sync(0xffffffffu, keys[u]);
-      if (keys[u] >= 0 && (peers & lt_mask) == 0) my[keys[u]] += __popc(peers);
-      __syncwarp();
-    }
+  for (int u = 0; u < kSlices; ++u) {
+    const int a = base + 32 * u + lane;
+    keys[u] = a < n ? load_key(idx, bits, a, E, status) : -1;
   }
-  __syncthreads();
+  int32_t* my = hist_s + warp * nbins;
+#pragma unroll
+  for (int u = 0; u < kSlices; ++u) {
+    const unsigned peers = __match_any_sync(0xffffffffu, keys[u]);
+    if (keys[u] >= 0 && (peers & lt_mask) == 0) my[keys[u]] += __popc(peers);
+    __syncwarp();
+  }
+}
 
-  // Column scan over warps: start of warp w inside bin b, and bin totals.
+__global__ void __launch_bounds__(kWarps * 32) k_perm_hist(const int32_t* __restrict__ idx,
+                                                           const uint8_t* __restrict__ bits, int n,
+                                                           int E, int nbins,
+                                                           int32_t* __restrict__ hist,
+                                                           int32_t* status) {
+  extern __shared__ int32_t hist_s[];  // [kWarps][nbins]
+  for (int i = threadIdx.x; i < kWarps * nbins; i += blockDim.x) hist_s[i] = 0;
+  __syncthreads();
+  int keys[kSlices];
+  warp_hist(idx, bits, n, E, nbins, hist_s, status, keys);
+  __syncthreads();
+  for (int b = threadIdx.x; b < nbins; b += blockDim.x) {
+    int c = 0;
+    for (int w = 0; w < kWarps; ++w) c += hist_s[w * nbins + b];
+    hist[static_cast<size_t>(b) * gridDim.x + blockIdx.x] = c;
+  }
+}
+
+__global__ void __launch_bounds__(1024) k_perm_scan(int32_t* __restrict__ hist, int ctas, int nbins,
+                                                    int n, int32_t* __restrict__ counts,
+                                                    int32_t* __restrict__ offsets) {
+  __shared__ int32_t scan_buf[32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int total = 0;
   if (tid < nbins) {
-    for (int w = 0; w < kWarps; ++w) {
-      const int c = hist[w * nbins + tid];
-      hist[w * nbins + tid] = total;
-      total += c;
+    int32_t* row = hist + static_cast<size_t>(tid) * ctas;
+    for (int c = 0; c < ctas; ++c) {
+      const int v = row[c];
+      row[c] = total;
+      total += v;
     }
     counts[tid] = total;
   }
-  // Block-wide exclusive scan of the bin totals (nbins <= 1024 threads).
   int incl = total;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -105,47 +119,44 @@ __global__ void __launch_bounds__(kWarps * 32) k_permute(const int32_t* __restri
       const int u = __shfl_up_sync(0xffffffffu, v, o);
       if (lane >= o) v += u;
     }
-    scan_buf[lane] = v;  // inclusive over warps
+    scan_buf[lane] = v;
   }
   __syncthreads();
   const int excl = incl - total + (warp > 0 ? scan_buf[warp - 1] : 0);
   if (tid < nbins) {
     offsets[tid] = excl;
-    for (int w = 0; w < kWarps; ++w) hist[w * nbins + tid] += excl;
+    int32_t* row = hist + static_cast<size_t>(tid) * ctas;
+    for (int c = 0; c < ctas; ++c) row[c] += excl;
   }
   if (tid == 0) offsets[nbins] = n;
-  __syncthreads();
+}
 
-  for (int base = begin; base < end; base += 32 * kBatch) {
-    int keys[kBatch];
+// Scatter of this CTA's assignments once hist_s[w][b] holds the first
+// position of warp w's keys in bin b.
+__device__ __forceinline__ void scatter(const int (&keys)[kSlices], int32_t* hist_s, int nbins,
+                                        int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  int32_t* my = hist_s + warp * nbins;
+  const int base = blockIdx.x * kCH + warp * 32 * kSlices;
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int a = base + 32 * u + lane;
-      keys[u] = a < end ? load_key(idx, bits, a, E, nullptr) : -1;
+  for (int u = 0; u < kSlices; ++u) {
+    const int a = base + 32 * u + lane;
+    const int key = keys[u];
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (key >= 0) {
+      const int p = my[key] + __popc(peers & lt_mask);
+      perm[p] = a;
+      inv_perm[a] = p;
     }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int a = base + 32 * u + lane;
-      const int key = keys[u];
-      const unsigned peers = __match_any_sync(0xffffffffu, key);
-      if (key >= 0) {
-        const int p = my[key] + __popc(peers & lt_mask);
-        if (stage_perm) perm_s[p] = a; else perm[p] = a;
-        inv_perm[a] = p;
-      }
-      __syncwarp();
-      if (key >= 0 && (peers & lt_mask) == 0) my[key] += __popc(peers);
-      __syncwarp();
-    }
-  }
-  if (stage_perm) {  // scattered positions land in shared memory; write out coalesced
-    __syncthreads();
-    for (int i = tid; i < n; i += blockDim.x) perm[i] = perm_s[i];
+    __syncwarp();
+    if (key >= 0 && (peers & lt_mask) == 0) my[key] += __popc(peers);
+    __syncwarp();
   }
 }
 
-// x_perm[p] = fp16(x[perm[p] / k]); a warp moves one row, 16 bytes per lane
-// per step with up to four independent loads in flight.
+// x_perm[p] = fp16(x[perm[p] / k]): a warp per destination row, 16-byte
+// loads, four in flight per lane; grid-stride over rows.
 __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict__ x,
                                                  const int32_t* __restrict__ perm, int rows, int k,
                                                  int d, __half* __restrict__ x_perm,
@@ -160,12 +171,12 @@ __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict_
     for (int c0 = lane; c0 < vec; c0 += 128) {
       uint4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (c0 + 32 * u < vec) v[u] = src[c0 + 32 * u];
+      for (int q = 0; q < 4; ++q)
+        if (c0 + 32 * q < vec) v[q] = src[c0 + 32 * q];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (c0 + 32 * u >= vec) break;
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+      for (int q = 0; q < 4; ++q) {
+        if (c0 + 32 * q >= vec) break;
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v[q]);
         uint4 o;
         __half2* h2 = reinterpret_cast<__half2*>(&o);
 #pragma unroll
@@ -174,43 +185,152 @@ __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict_
           bad |= fabsf(f.x) > 65504.0f || fabsf(f.y) > 65504.0f;
           h2[j] = __floats2half2_rn(f.x, f.y);
         }
-        dst[c0 + 32 * u] = o;
+        dst[c0 + 32 * q] = o;
       }
     }
   }
   if (bad) flag_status(status, MOE_DEV_RANGE);
 }
 
+__global__ void __launch_bounds__(kWarps * 32) k_perm_scatter(
+    const int32_t* __restrict__ idx, const uint8_t* __restrict__ bits, int n, int E, int nbins, int k,
+    const int32_t* __restrict__ hist, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
+  extern __shared__ int32_t hist_s[];  // [kWarps][nbins] -> per-warp start positions
+  for (int i = threadIdx.x; i < kWarps * nbins; i += blockDim.x) hist_s[i] = 0;
+  __syncthreads();
+  int keys[kSlices];
+  warp_hist(idx, bits, n, E, nbins, hist_s, nullptr, keys);
+  __syncthreads();
+  for (int b = threadIdx.x; b < nbins; b += blockDim.x) {
+    int start = hist[static_cast<size_t>(b) * gridDim.x + blockIdx.x];
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = hist_s[w * nbins + b];
+      hist_s[w * nbins + b] = start;
+      start += c;
+    }
+  }
+  __syncthreads();
+  scatter(keys, hist_s, nbins, perm, inv_perm);
+}
+
+// All of it in one CTA when the assignments fit one chunk (n <= 1024): the
+// bin totals are scanned in the block, so no workspace round trip and one
+// launch instead of three.
+__global__ void __launch_bounds__(kWarps * 32) k_perm_one(
+    const int32_t* __restrict__ idx, const uint8_t* __restrict__ bits, int n, int E, int nbins, int k,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv_perm, int32_t* status) {
+  extern __shared__ int32_t hist_s[];  // [kWarps][nbins]
+  __shared__ int32_t warp_sum[kWarps];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < kWarps * nbins; i += blockDim.x) hist_s[i] = 0;
+  __syncthreads();
+  int keys[kSlices];
+  warp_hist(idx, bits, n, E, nbins, hist_s, status, keys);
+  __syncthreads();
+  // thread t owns bins [t * per, t * per + per): total, then a block scan
+  const int per = (nbins + blockDim.x - 1) / blockDim.x;
+  const int b0 = tid * per;
+  int own = 0;
+  for (int i = 0; i < per; ++i) {
+    const int b = b0 + i;
+    if (b < nbins) {
+      int c = 0;
+      for (int w = 0; w < kWarps; ++w) c += hist_s[w * nbins + b];
+      counts[b] = c;
+      own += c;
+    }
+  }
+  int incl = own;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += warp_sum[w];
+  int start = before + incl - own;
+  for (int i = 0; i < per; ++i) {
+    const int b = b0 + i;
+    if (b < nbins) {
+      offsets[b] = start;
+      for (int w = 0; w < kWarps; ++w) {
+        const int c = hist_s[w * nbins + b];
+        hist_s[w * nbins + b] = start;
+        start += c;
+      }
+    }
+  }
+  if (tid == 0) offsets[nbins] = n;
+  __syncthreads();
+  scatter(keys, hist_s, nbins, perm, inv_perm);
+}
+
+int sm_count_permute() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 }  // namespace
+
+size_t permute_workspace_bytes(int T, int k, int nbins) {
+  const long n = static_cast<long>(T) * k;
+  const long ctas = std::max<long>(1, (n + kCH - 1) / kCH);
+  return static_cast<size_t>(std::max<long>(256, ctas * nbins * 4));
+}
 
 moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void* x, int T, int d,
                             int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
-                            int32_t* inv_perm, void* x_perm, int32_t* status, cudaStream_t s) {
+                            int32_t* inv_perm, void* x_perm, int32_t* status, void* workspace,
+                            cudaStream_t s) {
   const int n = T * k;
   const int nbins = bits ? 3 * E : E;
   if (nbins > kMaxBins) {
     set_error("moe_permute: %d bins exceed %d", nbins, kMaxBins);
     return MOE_ERR_UNSUPPORTED_SHAPE;
   }
-  // Shared memory: per-warp histograms, plus the permutation itself when it
-  // fits, so that its scattered positions are written to shared memory and
-  // leave the SM as coalesced rows.
-  constexpr size_t kSmemCap = 226 * 1024;  // 227 KB per block, less the static scan buffer
-  const size_t hist_bytes = sizeof(int32_t) * kWarps * nbins;
-  const int stage = hist_bytes + sizeof(int32_t) * static_cast<size_t>(n) <= kSmemCap;
-  const size_t smem = hist_bytes + (stage ? sizeof(int32_t) * static_cast<size_t>(n) : 0);
-  static bool attr_set = false;  // once per process, to the cap
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemCap));
+  const int ctas = std::max(1, (n + kCH - 1) / kCH);
+  int32_t* hist = static_cast<int32_t*>(workspace);
+  const size_t smem = sizeof(int32_t) * kWarps * nbins;
+  // The shared-memory opt-in is a per-device function attribute: set it once
+  // per device, to the largest bin count.
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_check(e, "moe_permute cudaGetDevice");
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (!bit || !(attr_set.load() & bit)) {
+    const int cap = static_cast<int>(sizeof(int32_t) * kWarps * kMaxBins);
+    e = cudaFuncSetAttribute(k_perm_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_perm_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_perm_one, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
     if (e != cudaSuccess) return cuda_check(e, "moe_permute smem attribute");
-    attr_set = true;
+    attr_set.fetch_or(bit);
   }
-  k_permute<<<1, kWarps * 32, smem, s>>>(idx, bits, n, E, nbins, counts, offsets, perm, inv_perm,
-                                         status, stage);
-  moe_status_t st = cuda_check(cudaGetLastError(), "moe_permute launch");
+  moe_status_t st;
+  if (ctas == 1) {
+    k_perm_one<<<1, kWarps * 32, smem, s>>>(idx, bits, n, E, nbins, k, counts, offsets, perm, inv_perm,
+                                            status);
+    st = cuda_check(cudaGetLastError(), "moe_permute launch");
+  } else {
+    k_perm_hist<<<ctas, kWarps * 32, smem, s>>>(idx, bits, n, E, nbins, hist, status);
+    st = cuda_check(cudaGetLastError(), "moe_permute histogram launch");
+    if (st != MOE_OK) return st;
+    k_perm_scan<<<1, 1024, 0, s>>>(hist, ctas, nbins, n, counts, offsets);
+    st = cuda_check(cudaGetLastError(), "moe_permute scan launch");
+    if (st != MOE_OK) return st;
+    k_perm_scatter<<<ctas, kWarps * 32, smem, s>>>(idx, bits, n, E, nbins, k, hist, perm, inv_perm);
+    st = cuda_check(cudaGetLastError(), "moe_permute scatter launch");
+  }
   if (st != MOE_OK || !x_perm || n == 0) return st;
-  const int blocks = static_cast<int>(std::min<long>((static_cast<long>(n) + 7) / 8, 148L * 8));
+  // a warp per row: up to 8 rows per block, at most 8 blocks per SM
+  const int blocks = std::max(1, std::min((n + 7) / 8, 8 * sm_count_permute()));
   k_gather<<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), perm, n, k, d,
                                   static_cast<__half*>(x_perm), status);
   return cuda_check(cudaGetLastError(), "moe_permute gather launch");

@@ -48,6 +48,8 @@ class QuantMoELayer:
             status=torch.zeros(1, dtype=torch.int32, device=dev),
             route_ws=torch.empty(max(256, moeq.moe_route_workspace_bytes(T, d, self.E)), dtype=torch.uint8,
                                  device=dev),
+            perm_ws=torch.empty(moeq.moe_permute_workspace_bytes(T, self.E, k, self.layout == moeq.LAYOUT_PLANES),
+                                dtype=torch.uint8, device=dev),
         )
 
     def views(self, T):
@@ -56,7 +58,7 @@ class QuantMoELayer:
         return dict(topk_idx=b["topk_idx"][:T], topk_w=b["topk_w"][:T], counts=b["counts"],
                     offsets=b["offsets"], perm=b["perm"][:rows], inv_perm=b["inv_perm"][:rows],
                     x_perm=b["x_perm"][:rows], y_perm=b["y_perm"][:rows], workspace=b["workspace"],
-                    y=b["y"][:T], status=b["status"], route_ws=b["route_ws"])
+                    y=b["y"][:T], status=b["status"], route_ws=b["route_ws"], perm_ws=b["perm_ws"])
 
     def forward(self, x, bits=None, forced_idx=None, residual=None, stream=None):
         T = x.shape[0]

@@ -37,7 +37,8 @@ _SIGS = {
     "moe_route_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
     "moe_route_topk_noalloc": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]),
     "moe_permute": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_p,
-                           _c_p, _c_p]),
+                           _c_p, _c_p, _c_sz, _c_p]),
+    "moe_permute_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
     "moe_ffn_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
     "moe_grouped_ffn_wq": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                   _c_p, _c_sz, _c_p, _c_p, _c_p]),
@@ -156,7 +157,11 @@ def moe_route_topk(x, w_router, bias, k, forced_idx=None, topk_idx=None, topk_w=
     return topk_idx, topk_w
 
 
-def moe_permute(topk_idx, E, bits=None, x=None, out=None, status=None, stream=None):
+def moe_permute_workspace_bytes(T, E, k, nested):
+    return int(load().moe_permute_workspace_bytes(T, E, k, int(bool(nested))))
+
+
+def moe_permute(topk_idx, E, bits=None, x=None, out=None, status=None, workspace=None, stream=None):
     """Returns dict(counts, offsets, perm, inv_perm, x_perm)."""
     lib = load()
     T, k = topk_idx.shape
@@ -169,12 +174,18 @@ def moe_permute(topk_idx, E, bits=None, x=None, out=None, status=None, stream=No
                    perm=torch.empty(T * k, dtype=torch.int32, device=dev),
                    inv_perm=torch.empty(T * k, dtype=torch.int32, device=dev),
                    x_perm=torch.empty(T * k, d, dtype=torch.float16, device=dev) if x is not None else None)
+    if workspace is None:
+        workspace = out.get("perm_ws")
+    if workspace is None:
+        workspace = torch.empty(lib.moe_permute_workspace_bytes(T, E, k, int(bits is not None)),
+                                dtype=torch.uint8, device=dev)
     _check("moe_permute", lib.moe_permute(
         _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(bits, torch.uint8, "bits"),
         _ptr(x, torch.bfloat16, "x"), T, d, E, k, _ptr(out["counts"], torch.int32),
         _ptr(out["offsets"], torch.int32), _ptr(out["perm"], torch.int32),
         _ptr(out["inv_perm"], torch.int32), _ptr(out["x_perm"], torch.float16),
-        _ptr(status, torch.int32, "status"), _stream(stream)))
+        _ptr(status, torch.int32, "status"), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
     return out
 
 

@@ -80,16 +80,21 @@ def test_route_k_equals_E_and_forced():
 
 # ------------------------------------------------------------- permute ----
 
-@pytest.mark.parametrize("T,k,E,nested,skew", [(1, 2, 8, False, False), (33, 2, 8, False, True),
-                                                (4096, 8, 64, False, True), (777, 4, 16, True, False),
-                                                (100, 3, 256, True, True), (5, 8, 8, False, False)])
-def test_permute_bitexact(T, k, E, nested, skew):
+@pytest.mark.parametrize("T,k,E,nested,skew,d", [(1, 2, 8, False, False, 64), (33, 2, 8, False, True, 64),
+                                                  (4096, 8, 64, False, True, 64), (777, 4, 16, True, False, 64),
+                                                  (100, 3, 256, True, True, 64), (5, 8, 8, False, False, 64),
+                                                  # many 1024-assignment blocks, ragged last block, wide rows
+                                                  (2049, 8, 64, False, True, 2056),
+                                                  # the largest bin count (3 * 256) over several blocks
+                                                  (3001, 4, 256, True, True, 8),
+                                                  # exactly one full block (single-launch path), one past it
+                                                  (128, 8, 64, False, True, 64), (129, 8, 64, False, True, 64)])
+def test_permute_bitexact(T, k, E, nested, skew, d):
     rng = np.random.default_rng(T * 7 + E)
     idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
     if skew:
         idx[: T // 2, 0] = 0
     bits = rng.choice([2, 3, 4], size=(T, k), p=[.3, .4, .3]).astype(np.uint8) if nested else None
-    d = 64
     x = torch.randn(T, d).to(torch.bfloat16)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = moeq.moe_permute(torch.from_numpy(idx).cuda(), E,
