@@ -119,12 +119,16 @@ MOE_API moe_status_t moe_quant_pack(const float* w_gate, const float* w_up, cons
 /* moe_route_topk -- softmax top-k router ([D2MoE] Dual Routing, expert
  * gate; [ExactMoE] the router decides, nothing is pruned).
  *   x        bf16 [T][d];  w_router fp32 [E][d];  bias fp32 [E] or NULL
- *   logits   l[t][e] = sum_i x[t][i] * w_router[e][i] + bias[e], evaluated
- *            in fp64 (bf16 x fp32 products are exact in fp64)
+ *   logits   l[t][e] = sum_i x[t][i] * w_router[e][i] + bias[e]
  *   topk_idx int32 [T][k]: the k largest logits, ordered by descending
- *            logit; equal logits go to the lower expert index
+ *            logit; equal logits go to the lower expert index.  The choice
+ *            is that of the exact logits: they are evaluated in fp32 with
+ *            a proven error bound, and a token whose choice the bound does
+ *            not settle (near ties, non-finite values) is re-evaluated and
+ *            selected in fp64, where every bf16 x fp32 product is exact.
  *   topk_w   fp32 [T][k]: softmax over the k selected logits (the full
- *            softmax renormalised over the selection)
+ *            softmax renormalised over the selection), from the fp32
+ *            logits (fp64 ones for re-evaluated tokens)
  *   forced_idx int32 [T][k] or NULL: when given, the selection is taken
  *            from it as is (an external trace) and only topk_w is
  *            computed for it; topk_idx receives a copy.
@@ -136,7 +140,8 @@ MOE_API moe_status_t moe_route_topk(const void* x, const float* w_router, const 
                             int32_t* topk_idx, float* topk_w, void* workspace,
                             size_t workspace_bytes, moe_stream_t stream);
 
-/* Device scratch moe_route_topk needs (per-slice fp64 partial logits). */
+/* Device scratch moe_route_topk needs (per-slice fp32 partial logits and
+ * squared norms). */
 MOE_API size_t moe_route_workspace_bytes(int T, int d, int E);
 
 /* moe_route_topk_noalloc -- the same router with no workspace argument.

@@ -1,208 +1,498 @@
 // Softmax top-k router.
 //
-// Logits l[t][e] = x[t] . W_r[e] (+ bias[e]) are accumulated in fp64: a
-// bf16 x fp32 product is exact in fp64, and fp64 leaves no practical room
-// for a summation-order difference to flip a top-k decision, so the expert
-// choice equals a plain fp64 evaluation of the definition.
+// The expert choice must equal the top k of the exact logits
+//   l[t][e] = x[t] . W_r[e] + bias[e]
+// (ties -> lower index), i.e. what a plain fp64 evaluation gives.  Doing all
+// T*E*d products in fp64 runs at the fp64 rate; instead:
 //
-// Two kernels:
-//   k_route_partial  grid (token tiles, expert tiles, K splits): a 64 x 64
-//                    (token x expert) tile over one slice of d, 4 x 4 fp64
-//                    register tile per thread, 32-wide d chunks staged in
-//                    shared memory as fp64; writes partial[split][t][e].
-//   k_route_select   one warp per token: sums the splits in split order
-//                    (the same order for every expert, so identical router
-//                    rows give identical logits), adds the bias, takes the
-//                    top k by a warp argmax repeated k times (ties -> lower
-//                    index) and the softmax over the k picks.
-// The split count is chosen so that small T still spreads the read of W_r
-// over many SMs and large T keeps every SM busy.
+//   k_route_logits  fp32 logits with blocked accumulation: a thread sums 32
+//                   products with FMA into a fresh chunk sum, then adds the
+//                   chunk sum to its running total; slices of d (splits)
+//                   are summed later in split order.  The same CTAs also
+//                   produce the sums of squares of x rows and W_r rows.
+//   k_route_select  warp per token: the split sums and the bias give the
+//                   fp32 logit L[e]; with the error bound
+//                     |L[e] - l[e]| <= D[e]
+//                       = 2 (g(32 + d/32) |x| |W_e| (1 + 2^-8) + u (|L| + |b|))
+//                   (u = 2^-24, g(m) = m u / (1 - m u); Cauchy-Schwarz for
+//                   sum |x_i W_ei|; the factor 2 is margin), the top k of L,
+//                   in order, is that of l whenever consecutive picks are
+//                   separated by more than their bounds and the last pick
+//                   beats every other expert:
+//                     L[k-th pick] - D  >  max over the rest (L + D).
+//                   Tokens where that fails (near ties, non-finite values)
+//                   are recomputed by the whole CTA in fp64 (each product of
+//                   a bf16 and an fp32 is exact in fp64) and selected on the
+//                   fp64 logits.  Gates are the softmax over the k picked
+//                   logits, in fp64 arithmetic on those values.
+//
+// Error bound of the fp32 sum: an FMA chain over m products errs by at most
+// g(m) times the sum of their magnitudes; a chunk (32 products) and then the
+// d/32 chunk sums in any order give g(32) + g(d/32)(1 + g(32)) <= g(32 + d/32).
+// The squared norms are fp32 sums too (relative error below 2^-8 for
+// d < 2^15) and the bias addition rounds once more (the u term).
 #include "common.cuh"
 
 namespace moeq {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTT = 64;   // tokens per tile
-constexpr int kEC = 64;   // experts per tile
-constexpr int kDC = 32;   // d chunk
-constexpr int kMT = 4, kME = 4;
-constexpr int kTX = kEC / kME;  // 16 threads along experts
-constexpr int kTY = kTT / kMT;  // 16 threads along tokens
+constexpr int kDC = 32;  // d chunk: fp32 accumulation block and shared-memory stage
+constexpr int kMT = 4;   // tokens per thread
+constexpr int kLT = 128; // threads of a logits CTA (4 warps)
 
-__global__ void __launch_bounds__(kThreads) k_route_partial(const __nv_bfloat16* __restrict__ x,
-                                                             const float* __restrict__ wr, int T,
-                                                             int d, int E, int dk,
-                                                             double* __restrict__ partial) {
-  __shared__ double xs[kDC][kTT + 1];
-  __shared__ double ws[kDC][kEC + 1];
-  const int tid = threadIdx.x;
-  const int tx = tid % kTX, ty = tid / kTX;
-  const int t0 = blockIdx.x * kTT, e0 = blockIdx.y * kEC, split = blockIdx.z;
-  const int kbeg = split * dk;
+// EC experts per CTA tile (64, or 16 for E <= 16): ME per thread, TX threads
+// along experts, TYW thread rows per warp; a CTA covers TT tokens.
+template <int EC>
+struct Tile {
+  static constexpr int ME = EC == 64 ? 8 : 4;
+  static constexpr int TX = EC / ME;
+  static constexpr int TYW = 32 / TX;
+  static constexpr int TT = (kLT / 32) * TYW * kMT;
+  static constexpr int XP = kDC + 1;   // x stage row pitch (floats): conflict-free
+  static constexpr int XS = TT * XP;   // floats per x stage ([token][k])
+  static constexpr int WS = kDC * EC;  // floats per W stage ([k][expert])
+  static constexpr size_t SMEM = 2 * (XS + WS) * sizeof(float);
+  static constexpr int XL = TT * 4 / kLT;   // 16-byte x loads per thread per chunk
+  static constexpr int WL = EC * 8 / kLT;   // 16-byte W loads per thread per chunk
+};
 
-  double acc[kMT][kME];
+// Workspace: partial[S][T][E] fp32, xsq[S][T], wsq[S][E].
+struct RouteWs {
+  float* partial;
+  float* xsq;
+  float* wsq;
+};
+
+__host__ __device__ inline RouteWs route_ws(void* base, int S, int T, int E) {
+  float* p = static_cast<float*>(base);
+  return {p, p + static_cast<size_t>(S) * T * E, p + static_cast<size_t>(S) * T * E + static_cast<size_t>(S) * T};
+}
+
+template <int EC>
+__global__ void __launch_bounds__(kLT) k_route_logits(const __nv_bfloat16* __restrict__ x,
+                                                       const float* __restrict__ wr, int T, int d, int E,
+                                                       int dk, RouteWs ws) {
+  using G = Tile<EC>;
+  extern __shared__ __align__(16) float sm[];
+  float* xs = sm;               // [2][TT][XP]
+  float* wsm = sm + 2 * G::XS;  // [2][kDC][EC]
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int tx = lane % G::TX;
+  const int ty = (tid >> 5) * G::TYW + lane / G::TX;
+  const int t0 = blockIdx.x * G::TT, e0 = blockIdx.y * EC, split = blockIdx.z;
+  const int kbeg = split * dk, nch = dk / kDC;
+  const bool do_x = blockIdx.y == 0, do_w = blockIdx.x == 0;
+
+  // loaders: x load q covers token row (tid + kLT q) / 4, columns ((tid + kLT q) % 4) * 8 .. +8;
+  // W load q covers expert (tid + kLT q) % EC, columns ((tid + kLT q) / EC) * 4 .. +4
+  uint4 xr[G::XL];
+  float4 wv4[G::WL];
+  float xsq[G::XL], wsq[G::WL];
+#pragma unroll
+  for (int q = 0; q < G::XL; ++q) xsq[q] = 0.f;
+#pragma unroll
+  for (int q = 0; q < G::WL; ++q) wsq[q] = 0.f;
+
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < G::XL; ++q) {
+      const int i = tid + kLT * q, t = t0 + (i >> 2);
+      xr[q] = t < T ? *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d + k0 + (i & 3) * 8)
+                    : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int q = 0; q < G::WL; ++q) {
+      const int i = tid + kLT * q, e = e0 + i % EC;
+      wv4[q] = e < E ? *reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * d + k0 + (i / EC) * 4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto stash = [&](int b) {
+    float* xb = xs + b * G::XS;
+#pragma unroll
+    for (int q = 0; q < G::XL; ++q) {
+      const int i = tid + kLT * q, r = i >> 2, c = (i & 3) * 8;
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xr[q]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(b2[j]);
+        xb[r * G::XP + c + 2 * j] = f.x;
+        xb[r * G::XP + c + 2 * j + 1] = f.y;
+        if (do_x) xsq[q] = fmaf(f.x, f.x, fmaf(f.y, f.y, xsq[q]));
+      }
+    }
+    float* wb = wsm + b * G::WS;
+#pragma unroll
+    for (int q = 0; q < G::WL; ++q) {
+      const int i = tid + kLT * q, e = i % EC, c = (i / EC) * 4;
+      const float v[4] = {wv4[q].x, wv4[q].y, wv4[q].z, wv4[q].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        wb[(c + j) * EC + e] = v[j];
+        if (do_w) wsq[q] = fmaf(v[j], v[j], wsq[q]);
+      }
+    }
+  };
+
+  float acc[kMT][G::ME];
 #pragma unroll
   for (int i = 0; i < kMT; ++i)
 #pragma unroll
-    for (int j = 0; j < kME; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < G::ME; ++j) acc[i][j] = 0.f;
 
-  for (int k0 = kbeg; k0 < kbeg + dk; k0 += kDC) {
-    __syncthreads();
-    // x chunk: 64 tokens x 32 -> 2048 values, 8 per thread (one 16-byte load)
-    {
-      const int r = tid / 4, c = (tid % 4) * 8;
-      const int t = t0 + r;
-      if (t < T) {
-        const uint4 v = *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d + k0 + c);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+  fetch(kbeg);
+  stash(0);
+  __syncthreads();
+  for (int c = 0; c < nch; ++c) {
+    const int b = c & 1;
+    if (c + 1 < nch) fetch(kbeg + (c + 1) * kDC);
+    const float* xb = xs + b * G::XS + ty * kMT * G::XP;
+    const float* wb = wsm + b * G::WS + tx * G::ME;
+    float cs[kMT][G::ME];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = __bfloat1622float2(b2[j]);
-          xs[c + 2 * j][r] = f.x;
-          xs[c + 2 * j + 1][r] = f.y;
-        }
-      } else {
+    for (int i = 0; i < kMT; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) xs[c + j][r] = 0.0;
-      }
-    }
-    // W chunk: 64 experts x 32 -> 2048 values, 8 per thread (two 16-byte loads)
-    {
-      const int r = tid / 4, c = (tid % 4) * 8;
-      const int e = e0 + r;
-      if (e < E) {
-        const float4 a = *reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * d + k0 + c);
-        const float4 b = *reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * d + k0 + c + 4);
-        ws[c + 0][r] = a.x; ws[c + 1][r] = a.y; ws[c + 2][r] = a.z; ws[c + 3][r] = a.w;
-        ws[c + 4][r] = b.x; ws[c + 5][r] = b.y; ws[c + 6][r] = b.z; ws[c + 7][r] = b.w;
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) ws[c + j][r] = 0.0;
-      }
-    }
-    __syncthreads();
+      for (int j = 0; j < G::ME; ++j) cs[i][j] = 0.f;
 #pragma unroll 8
-    for (int c = 0; c < kDC; ++c) {
-      double xv[kMT], wv[kME];
+    for (int kk = 0; kk < kDC; ++kk) {
+      float xa[kMT], wv[G::ME];
 #pragma unroll
-      for (int i = 0; i < kMT; ++i) xv[i] = xs[c][i * kTY + ty];
+      for (int i = 0; i < kMT; ++i) xa[i] = xb[i * G::XP + kk];
 #pragma unroll
-      for (int j = 0; j < kME; ++j) wv[j] = ws[c][j * kTX + tx];
+      for (int j = 0; j < G::ME; j += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(wb + kk * EC + j);
+        wv[j] = w4.x; wv[j + 1] = w4.y; wv[j + 2] = w4.z; wv[j + 3] = w4.w;
+      }
 #pragma unroll
       for (int i = 0; i < kMT; ++i)
 #pragma unroll
-        for (int j = 0; j < kME; ++j) acc[i][j] = fma(xv[i], wv[j], acc[i][j]);
+        for (int j = 0; j < G::ME; ++j) cs[i][j] = fmaf(xa[i], wv[j], cs[i][j]);
     }
+#pragma unroll
+    for (int i = 0; i < kMT; ++i)
+#pragma unroll
+      for (int j = 0; j < G::ME; ++j) acc[i][j] += cs[i][j];
+    if (c + 1 < nch) stash(b ^ 1);
+    __syncthreads();
   }
-  double* out = partial + static_cast<size_t>(split) * T * E;
+
+  float* out = ws.partial + static_cast<size_t>(split) * T * E;
 #pragma unroll
   for (int i = 0; i < kMT; ++i) {
-    const int t = t0 + i * kTY + ty;
+    const int t = t0 + ty * kMT + i;
     if (t >= T) continue;
 #pragma unroll
-    for (int j = 0; j < kME; ++j) {
-      const int e = e0 + j * kTX + tx;
+    for (int j = 0; j < G::ME; ++j) {
+      const int e = e0 + tx * G::ME + j;
       if (e < E) out[static_cast<size_t>(t) * E + e] = acc[i][j];
     }
   }
+  // squared norms: the 4 x-loader lanes of a row are adjacent; a W row's
+  // loaders are the threads i with i % EC equal, reduced through shared memory
+  if (do_x) {
+#pragma unroll
+    for (int q = 0; q < G::XL; ++q) {
+      float v = xsq[q];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      const int i = tid + kLT * q, t = t0 + (i >> 2);
+      if ((i & 3) == 0 && t < T) ws.xsq[static_cast<size_t>(split) * T + t] = v;
+    }
+  }
+  if (do_w) {
+    float* red = sm;  // reuse the stages (the loop ended with a barrier)
+#pragma unroll
+    for (int q = 0; q < G::WL; ++q) red[tid + kLT * q] = wsq[q];
+    __syncthreads();
+    if (tid < EC) {
+      float v = 0.f;
+      for (int i = tid; i < EC * 8; i += EC) v += red[i];
+      const int e = e0 + tid;
+      if (e < E) ws.wsq[static_cast<size_t>(split) * E + e] = v;
+    }
+  }
 }
 
-__global__ void __launch_bounds__(kThreads) k_route_select(const double* __restrict__ partial,
-                                                            int splits, const float* __restrict__ bias,
-                                                            const int32_t* __restrict__ forced, int T,
-                                                            int E, int k, int32_t* __restrict__ out_idx,
-                                                            float* __restrict__ out_w) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int t = warp;
-  if (t >= T) return;
-  constexpr int kPer = 8;  // E <= 256 -> at most 8 experts per lane
-  double l[kPer];
+constexpr int kPer = 8;  // E <= 256: at most 8 experts per lane (e = lane + 32 m)
+
+// True on every lane of a warp when any lane lists a contender.
+__device__ __forceinline__ bool contender_any(uint32_t c) { return __any_sync(0xffffffffu, c != 0); }
+
+// fp64 dot product x[t] . W_r[e] by one warp: lanes over 8-element pieces
+// of d, four pieces' loads issued before their FMAs, then a shuffle tree.
+__device__ __forceinline__ double dot64(const __nv_bfloat16* x, const float* w, int d, int lane) {
+  double a = 0.0;
+  for (int i0 = lane * 8; i0 < d; i0 += 4 * 256) {
+    uint4 xv[4];
+    float4 w0[4], w1[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * 256;
+      if (i < d) {
+        xv[u] = *reinterpret_cast<const uint4*>(x + i);
+        w0[u] = *reinterpret_cast<const float4*>(w + i);
+        w1[u] = *reinterpret_cast<const float4*>(w + i + 4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (i0 + u * 256 >= d) break;
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xv[u]);
+      const float wv[8] = {w0[u].x, w0[u].y, w0[u].z, w0[u].w, w1[u].x, w1[u].y, w1[u].z, w1[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(b2[j]);
+        a = fma(static_cast<double>(f.x), static_cast<double>(wv[2 * j]), a);
+        a = fma(static_cast<double>(f.y), static_cast<double>(wv[2 * j + 1]), a);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+  return a;
+}
+
+// Top k of the lane-distributed values v[m] (expert lane + 32 m; experts
+// with ok[m] false take no part), ties to the lower index; returns the picks
+// in order and the lane's taken mask.
+template <typename V>
+__device__ __forceinline__ uint32_t warp_topk(const V (&v)[kPer], uint32_t allowed, int E, int k, int lane,
+                                              int (&sel)[16]) {
+  uint32_t taken = 0;
+  for (int j = 0; j < k; ++j) {
+    V best = -INFINITY;
+    int best_e = 0x7fffffff;
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) {
+      const int e = lane + 32 * m;
+      if (e < E && (allowed & (1u << m)) && !(taken & (1u << m)) &&
+          (v[m] > best || (v[m] == best && e < best_e))) {
+        best = v[m];
+        best_e = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const V ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, best_e, o);
+      if (ov > best || (ov == best && oe < best_e)) {
+        best = ov;
+        best_e = oe;
+      }
+    }
+    if (best_e >= E) best_e = 0;  // only when fewer than k values are comparable (NaN)
+    sel[j] = best_e;
+    if ((best_e & 31) == lane) taken |= 1u << (best_e >> 5);
+  }
+  return taken;
+}
+
+// Value of expert e from the lane-distributed array.
+template <typename V>
+__device__ __forceinline__ V lane_value(const V (&v)[kPer], int e) {
+  V r = 0;
 #pragma unroll
   for (int m = 0; m < kPer; ++m) {
-    const int e = lane + 32 * m;
-    double v = -INFINITY;
-    if (e < E) {
-      v = 0.0;
-      for (int s = 0; s < splits; ++s) v += partial[(static_cast<size_t>(s) * T + t) * E + e];
-      if (bias) v += static_cast<double>(bias[e]);
-    }
-    l[m] = v;
+    const V o = __shfl_sync(0xffffffffu, v[m], e & 31);
+    if ((e >> 5) == m) r = o;
   }
-  int sel_e[16];
-  double sel_l[16];
-  if (forced) {
-    for (int j = 0; j < k; ++j) {
-      int e = forced[static_cast<size_t>(t) * k + j];
-      e = e < 0 ? 0 : (e >= E ? E - 1 : e);
-      double v = 0.0;
-#pragma unroll
-      for (int m = 0; m < kPer; ++m) {
-        const double o = __shfl_sync(0xffffffffu, l[m], e & 31);
-        if ((e >> 5) == m) v = o;
-      }
-      sel_e[j] = e;
-      sel_l[j] = v;
-    }
-  } else {
-    uint32_t taken = 0;
-    for (int j = 0; j < k; ++j) {
-      double best = -INFINITY;
-      int best_e = 0x7fffffff;
-#pragma unroll
-      for (int m = 0; m < kPer; ++m) {
-        const int e = lane + 32 * m;
-        if (e < E && !(taken & (1u << m))) {
-          if (l[m] > best || (l[m] == best && e < best_e)) {
-            best = l[m];
-            best_e = e;
-          }
-        }
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const double ov = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, best_e, o);
-        if (ov > best || (ov == best && oe < best_e)) {
-          best = ov;
-          best_e = oe;
-        }
-      }
-      sel_e[j] = best_e;
-      sel_l[j] = best;
-      if ((best_e & 31) == lane) taken |= 1u << (best_e >> 5);
-    }
-  }
-  double mx = sel_l[0];
-  for (int j = 1; j < k; ++j) mx = fmax(mx, sel_l[j]);
-  double sum = 0.0;
-  double ex[16];
-  for (int j = 0; j < k; ++j) {
-    ex[j] = exp(sel_l[j] - mx);
-    sum += ex[j];
-  }
-  for (int j = 0; j < k; ++j)
-    if (j == lane) {
-      out_idx[static_cast<size_t>(t) * k + j] = sel_e[j];
-      out_w[static_cast<size_t>(t) * k + j] = static_cast<float>(ex[j] / sum);
-    }
+  return r;
 }
 
-}  // namespace
+// Softmax over the k picks: lane j < k owns pick j; maximum and sum are
+// fixed-order shuffle trees (picks given by the caller need not be sorted).
+template <typename V>
+__device__ __forceinline__ void write_gates(const V (&v)[kPer], const int (&sel)[16], int k, int t,
+                                            int lane, int32_t* out_idx, float* out_w) {
+  int mine = 0;
+  for (int j = 0; j < k; ++j)
+    if (j == lane) mine = sel[j];
+  const double lv = static_cast<double>(lane_value(v, mine));
+  double mx = lane < k ? lv : -INFINITY;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const double ex = lane < k ? exp(lv - mx) : 0.0;
+  double sum = ex;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < k) {
+    out_idx[static_cast<size_t>(t) * k + lane] = mine;
+    out_w[static_cast<size_t>(t) * k + lane] = static_cast<float>(ex / sum);
+  }
+}
+
+constexpr int kSelThreads = 256;
+constexpr int kSelWarps = kSelThreads / 32;
+
+// Warp per token.  A token the fp32 bounds do not settle lists its
+// contenders -- every expert whose upper bound reaches the lowest lower
+// bound among the picks (all others are certainly out) -- and the CTA's
+// warps recompute those logits in fp64; the token's warp then selects among
+// them on the fp64 values.
+__global__ void __launch_bounds__(kSelThreads) k_route_select(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, RouteWs ws, int splits,
+    const float* __restrict__ bias, const int32_t* __restrict__ forced, int T, int d, int E, int k,
+    float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w) {
+  __shared__ int n_cand[kSelWarps];
+  __shared__ uint8_t cand[kSelWarps][256];
+  __shared__ double l64[kSelWarps][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kSelWarps + warp;
+  if (lane == 0) n_cand[warp] = 0;
+  uint32_t contender = 0;  // lane's experts listed for fp64
+  if (t < T) {
+    float L[kPer], D[kPer];
+    // split sums in split order, loads of a batch of 16 splits issued together
+    float xq = 0.f;
+    for (int s0 = 0; s0 < splits; s0 += 16) {
+      float q[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) q[u] = s0 + u < splits ? ws.xsq[static_cast<size_t>(s0 + u) * T + t] : 0.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) xq += q[u];
+    }
+    const float xn = sqrtf(xq);
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) {
+      const int e = lane + 32 * m;
+      L[m] = -INFINITY;
+      D[m] = 0.f;
+      if (e < E) {
+        float v = 0.f, wq = 0.f;
+        for (int s0 = 0; s0 < splits; s0 += 16) {
+          float pv[16], qv[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const bool in = s0 + u < splits;
+            pv[u] = in ? ws.partial[(static_cast<size_t>(s0 + u) * T + t) * E + e] : 0.f;
+            qv[u] = in ? ws.wsq[static_cast<size_t>(s0 + u) * E + e] : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            v += pv[u];
+            wq += qv[u];
+          }
+        }
+        const float b = bias ? bias[e] : 0.f;
+        v += b;
+        L[m] = v;
+        D[m] = 2.0f * (gamma * xn * sqrtf(wq) * (1.0f + 0.00390625f) +
+                       5.9604645e-8f * (fabsf(v) + fabsf(b))) + 1e-30f;
+      }
+    }
+    int sel[16];
+    if (forced) {
+      for (int j = 0; j < k; ++j) {
+        const int e = forced[static_cast<size_t>(t) * k + j];
+        sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
+      }
+      write_gates(L, sel, k, t, lane, out_idx, out_w);
+    } else {
+      const uint32_t taken = warp_topk(L, 0xffu, E, k, lane, sel);
+      float hi = -INFINITY;
+#pragma unroll
+      for (int m = 0; m < kPer; ++m)
+        if (lane + 32 * m < E && !(taken & (1u << m))) hi = fmaxf(hi, L[m] + D[m]);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      // Certified when the order of the picks and the cut after the k-th are
+      // both wider than the bounds: pick j beats pick j+1, and the last pick
+      // beats every other expert (comparisons with NaN are false, so
+      // non-finite values fall through to fp64).
+      bool sure = true;
+      float prev_lo = INFINITY, lo_min = INFINITY;
+      for (int j = 0; j < k; ++j) {
+        const float lj = lane_value(L, sel[j]), dj = lane_value(D, sel[j]);
+        sure = sure && (j == 0 || prev_lo > lj + dj);
+        prev_lo = lj - dj;
+        lo_min = fminf(lo_min, prev_lo);
+      }
+      if (k < E) sure = sure && prev_lo > hi;
+      else sure = sure && prev_lo == prev_lo;
+      if (sure) {
+        write_gates(L, sel, k, t, lane, out_idx, out_w);
+      } else {
+        // contenders: picks, and every other expert whose upper bound reaches
+        // the lowest pick's lower bound (all of them when a value is not finite)
+        const bool finite = lo_min == lo_min && fabsf(lo_min) <= 3.0e38f;
+#pragma unroll
+        for (int m = 0; m < kPer; ++m) {
+          const int e = lane + 32 * m;
+          if (e < E && (!finite || (taken & (1u << m)) || !(L[m] + D[m] < lo_min))) contender |= 1u << m;
+        }
+        int base = 0;
+#pragma unroll
+        for (int m = 0; m < kPer; ++m) {
+          const unsigned bal = __ballot_sync(0xffffffffu, (contender >> m) & 1u);
+          if ((contender >> m) & 1u) cand[warp][base + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * m;
+          base += __popc(bal);
+        }
+        if (lane == 0) n_cand[warp] = base;
+      }
+    }
+  }
+  __syncthreads();
+  // fp64 logits of all listed (token, expert) pairs of this CTA, spread over its warps
+  int total = 0;
+  for (int w = 0; w < kSelWarps; ++w) total += n_cand[w];
+  if (total == 0) return;  // CTA-uniform
+  for (int item = warp; item < total; item += kSelWarps) {
+    int w = 0, r = item;
+    while (r >= n_cand[w]) r -= n_cand[w++];
+    const int tu = blockIdx.x * kSelWarps + w, e = cand[w][r];
+    const double v = dot64(x + static_cast<size_t>(tu) * d, wr + static_cast<size_t>(e) * d, d, lane);
+    if (lane == 0) l64[w][e] = v + (bias ? static_cast<double>(bias[e]) : 0.0);
+  }
+  __syncthreads();
+  if (contender_any(contender)) {
+    double v[kPer];
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) v[m] = ((contender >> m) & 1u) ? l64[warp][lane + 32 * m] : -INFINITY;
+    int sel[16];
+    warp_topk(v, contender, E, k, lane, sel);
+    write_gates(v, sel, k, t, lane, out_idx, out_w);
+  }
+}
 
 int route_splits(int T, int d, int E) {
-  const int tiles = ceil_div(T, kTT) * ceil_div(E, kEC);
+  const int ec = E <= 16 ? 16 : 64;
+  const int tt = ec == 64 ? Tile<64>::TT : Tile<16>::TT;
+  const int tiles = ceil_div(T, tt) * ceil_div(E, ec);
   const int chunks = d / kDC;
-  const int target = ceil_div(2 * 148, tiles);
+  const int target = ceil_div(4 * 148, tiles);  // about four CTAs per SM
   int s = 1;
   while (s * 2 <= target && chunks % (s * 2) == 0 && s * 2 <= 64) s *= 2;
   return s;
 }
 
+float route_gamma(int d) {
+  const double u = std::ldexp(1.0, -24);
+  const double m = kDC + d / kDC;
+  return static_cast<float>(m * u / (1.0 - m * u));
+}
+
+template <int EC>
+moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d, int E, int splits,
+                           RouteWs ws, cudaStream_t s) {
+  using G = Tile<EC>;
+  static bool attr_set = false;  // once per process (the first call precedes any capture)
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_route_logits<EC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(G::SMEM));
+    if (e != cudaSuccess) return cuda_check(e, "moe_route_topk smem attribute");
+    attr_set = true;
+  }
+  dim3 grid(ceil_div(T, G::TT), ceil_div(E, EC), splits);
+  k_route_logits<EC><<<grid, kLT, G::SMEM, s>>>(x, wr, T, d, E, d / splits, ws);
+  return cuda_check(cudaGetLastError(), "moe_route_topk logits launch");
+}
+
+}  // namespace
+
 size_t route_workspace_bytes(int T, int d, int E) {
   if (T <= 0 || d <= 0 || E <= 0) return 256;
-  return static_cast<size_t>(route_splits(T, d, E)) * T * E * sizeof(double);
+  const size_t S = static_cast<size_t>(route_splits(T, d, E));
+  return std::max<size_t>(256, S * (static_cast<size_t>(T) * E + T + E) * sizeof(float));
 }
 
 moe_status_t launch_route(const void* x, const float* w_router, const float* bias,
@@ -210,14 +500,13 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
                           float* w, void* workspace, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   const int splits = route_splits(T, d, E);
-  double* partial = static_cast<double*>(workspace);
-  dim3 grid(ceil_div(T, kTT), ceil_div(E, kEC), splits);
-  k_route_partial<<<grid, kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), w_router, T, d, E,
-                                            d / splits, partial);
-  moe_status_t st = cuda_check(cudaGetLastError(), "moe_route_topk partial launch");
+  const RouteWs ws = route_ws(workspace, splits, T, E);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, splits, ws, s)
+                            : launch_logits<64>(xb, w_router, T, d, E, splits, ws, s);
   if (st != MOE_OK) return st;
-  k_route_select<<<ceil_div(T * 32, kThreads), kThreads, 0, s>>>(partial, splits, bias, forced, T, E,
-                                                                  k, idx, w);
+  k_route_select<<<ceil_div(T, kSelWarps), kSelThreads, 0, s>>>(xb, w_router, ws, splits, bias, forced, T,
+                                                                  d, E, k, route_gamma(d), idx, w);
   return cuda_check(cudaGetLastError(), "moe_route_topk select launch");
 }
 

@@ -11,6 +11,13 @@ from quantized_moe_expert_histogram_b200.layer import QuantMoELayer
 RTOL = 1e-2  # |y - y_ref| <= ATOL + RTOL * |y_ref|  (the layer's stated bar)
 ATOL = 1e-2
 
+# Gates come from fp32 logits (fp64 only for tokens whose top-k the fp32
+# error bound leaves open).  Their typical logit error is ~1e-7; the proven
+# bound is a few 1e-4 at d = 4096, which moves a gate by at most that
+# fraction and the layer output far less than its 1e-2 bar.
+GATE_RTOL = 1e-4
+GATE_ATOL = 1e-6
+
 
 def within_tol(y, y_ref, atol=ATOL, rtol=RTOL):
     y = np.asarray(y, dtype=np.float64)

@@ -13,7 +13,7 @@ from quantized_moe_expert_histogram_b200 import inputs as I
 from quantized_moe_expert_histogram_b200 import moeq
 from quantized_moe_expert_histogram_b200.layer import QuantMoELayer
 
-from gpu_helpers import within_tol
+from gpu_helpers import within_tol, GATE_RTOL, GATE_ATOL
 
 pytestmark = pytest.mark.gpu
 
@@ -40,7 +40,7 @@ def test_full_size_sampled(name, T, n_sample):
     bias = L["bias"].cpu().numpy() if L["bias"] is not None else None
     sel, gates, _ = O.route(x, L["w_router"].cpu().numpy(), bias, shape.k)
     np.testing.assert_array_equal(v["topk_idx"].cpu().numpy(), sel)
-    np.testing.assert_allclose(v["topk_w"].cpu().numpy(), gates, rtol=2e-6, atol=1e-7)
+    np.testing.assert_allclose(v["topk_w"].cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
     keys, mult = O.assignment_keys(sel, None if bits is None else bits.cpu().numpy())
     counts, offsets, perm, inv = O.permute(keys, shape.E * (mult or 1))
     np.testing.assert_array_equal(v["counts"].cpu().numpy(), counts)

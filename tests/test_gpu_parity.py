@@ -11,7 +11,7 @@ from quantized_moe_expert_histogram_b200 import build
 from quantized_moe_expert_histogram_b200 import inputs as I
 from quantized_moe_expert_histogram_b200 import moeq
 
-from gpu_helpers import gpu_layer, layer_inputs, oracle_layer, run_gpu_layer, within_tol
+from gpu_helpers import gpu_layer, layer_inputs, oracle_layer, run_gpu_layer, within_tol, GATE_RTOL, GATE_ATOL
 
 pytestmark = pytest.mark.gpu
 
@@ -62,7 +62,32 @@ def test_route_bitexact(name, T, dup):
     sel, gates, logits = O.route(L["x"].float().numpy(), L["w_router"].numpy(),
                                  None if L["bias"] is None else L["bias"].numpy(), shape.k)
     np.testing.assert_array_equal(idx.cpu().numpy(), sel)
-    np.testing.assert_allclose(w.cpu().numpy(), gates, rtol=2e-6, atol=1e-7)
+    np.testing.assert_allclose(w.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
+
+
+@pytest.mark.parametrize("scale", [0.0, 1e-9, 1e-7, 1e-5])
+def test_route_near_ties_resolved_exactly(scale):
+    """Router rows that are copies of others plus a perturbation of the given
+    size: the logits of the pairs differ by about scale * |x| (exact ties at
+    0), below what fp32 logits can order, so these tokens must take the fp64
+    re-evaluation and still match the oracle's choice and order exactly."""
+    shape = I.SHAPES["olmoe"]
+    T = 300
+    L = I.make_layer(shape, T, seed=9, weights=False)
+    w = L["w_router"].clone()
+    b = L["bias"].clone()
+    rng = np.random.default_rng(1)
+    for a, src in ((1, 0), (9, 4), (33, 17), (63, 62), (2, 0)):
+        w[a] = w[src] + torch.from_numpy((rng.standard_normal(shape.d) * scale).astype(np.float32))
+        b[a] = b[src]
+    idx, gw = moeq.moe_route_topk(L["x"].cuda(), w.cuda(), b.cuda(), shape.k)
+    torch.cuda.synchronize()
+    sel, gates, _ = O.route(L["x"].float().numpy(), w.numpy(), b.numpy(), shape.k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), sel)
+    np.testing.assert_allclose(gw.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
+    # the pairs really are near-tied inside many tokens' picks
+    both = sum(int((s == 0).any() and (s == 1).any()) for s in sel)
+    assert both > 10
 
 
 def test_route_k_equals_E_and_forced():
@@ -75,7 +100,7 @@ def test_route_k_equals_E_and_forced():
                           dtype=torch.int32)
     idx3, w3 = moeq.moe_route_topk(L["x"].cuda(), L["w_router"].cuda(), None, 3, forced_idx=forced.cuda())
     np.testing.assert_array_equal(idx3.cpu().numpy(), forced.numpy())
-    np.testing.assert_allclose(w3.cpu().numpy(), O.gates_for(logits, forced.numpy()), rtol=2e-6, atol=1e-7)
+    np.testing.assert_allclose(w3.cpu().numpy(), O.gates_for(logits, forced.numpy()), rtol=GATE_RTOL, atol=GATE_ATOL)
 
 
 # ------------------------------------------------------------- permute ----
