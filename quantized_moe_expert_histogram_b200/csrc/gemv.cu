@@ -11,6 +11,14 @@
 // Accumulation is fp32.  blockIdx.y enumerates the non-empty (and, in slot
 // mode, resident) bins; blockIdx.x a block of 8 warps x RW output rows.
 //
+// The down pass is a programmatic dependent launch of the gate/up pass: its
+// blocks start while the gate/up pass runs, locate their bin and issue the
+// loads of their weight codes (which do not depend on h), and only then
+// wait (griddepcontrol.wait) for the gate/up grid before reading h.  The
+// gate/up pass allows that early start as soon as it begins; everything the
+// down pass reads before its wait (offsets, slot table, weights) was
+// complete before the gate/up pass was launched.
+//
 //   gate/up pass:  h[p][f]      = silu(Wg[f] . x_p) * (Wu[f] . x_p)   (fp16)
 //   down pass:     y_perm[p][n] = Wd[n] . h_p                          (fp32)
 #include <algorithm>
@@ -137,6 +145,10 @@ template <int MAXR, int NM, int RW, bool PLANES>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_gemv(const GemvParams P) {
   constexpr int ROWS = NM * RW;  // weight rows per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // gate/up: let the down pass launch now; down: activations (h) are read
+  // only after griddepcontrol.wait below
+  if (NM == 2) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  bool dep_waited = NM == 2;
   int bin, row0, nrows, blob_index, bits;
   if (!find_bin(P, blockIdx.y, bin, row0, nrows, blob_index, bits)) return;
   const uint8_t* blob = P.blobs + static_cast<size_t>(blob_index) * P.blob_bytes;
@@ -171,6 +183,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_gemv(const GemvParams P
           sz[s][r] = ldg_nc_u32(szp + (static_cast<size_t>(row >> 7) * G + k0 / P.group) * 128 + (row & 127));
         }
       }
+    }
+    if (!dep_waited) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      dep_waited = true;
     }
 #pragma unroll
     for (int s = 0; s < kChunkSteps; ++s) {
@@ -258,9 +274,18 @@ moe_status_t run_pair(GemvParams gu, GemvParams dn, int max_bins, cudaStream_t s
   k_gemv<MAXR, 2, RW_GU, PLANES><<<g1, kWarpsPerBlock * 32, 0, s>>>(gu);
   moe_status_t st = cuda_check(cudaGetLastError(), "ffn gemv gate/up launch");
   if (st != MOE_OK) return st;
-  dim3 g2(ceil_div(dn.N, kWarpsPerBlock * RW_DN), max_bins);
-  k_gemv<MAXR, 1, RW_DN, PLANES><<<g2, kWarpsPerBlock * 32, 0, s>>>(dn);
-  return cuda_check(cudaGetLastError(), "ffn gemv down launch");
+  // programmatic dependent launch (see the note at the top of the file)
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(ceil_div(dn.N, kWarpsPerBlock * RW_DN), max_bins);
+  cfg.blockDim = dim3(kWarpsPerBlock * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, k_gemv<MAXR, 1, RW_DN, PLANES>, dn), "ffn gemv down launch");
 }
 
 }  // namespace

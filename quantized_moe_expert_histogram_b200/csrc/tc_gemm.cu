@@ -3,39 +3,58 @@
 // One persistent CTA per SM walks a tile list built on the device from the
 // bin offsets (no host sync).  A tile is (bin, token block of up to 128
 // rows, weight block).  The MMA is issued "swap-AB": dequantised weight
-// rows are the M side (operand A, built in shared memory) and the bin's
-// tokens the N side (operand B, fp16 activation rows loaded by TMA), so a
-// bin of any size is covered with at most 15 padded token columns;
-// D[weight row][token] accumulates in TMEM (fp32).
+// rows are the M side (operand A) and the bin's tokens the N side (operand
+// B, fp16 activation rows loaded by TMA), so a bin of any size is covered
+// with at most 15 padded token columns; D[weight row][token] accumulates in
+// TMEM (fp32).
+//
+// Operand A lives in tensor memory, not shared memory: a dequantiser thread
+// owns one weight row, which is one TMEM lane, and stores its fp16 values
+// there with tcgen05.st (two per 32-bit column, K ascending).  The MMA
+// reads A from TMEM and only B from shared memory.  At N = 128 a 128-row
+// MMA that took both operands from shared memory would already use the
+// whole shared-memory bandwidth of the SM (A + B slices every 64 cycles),
+// and building A there as well (dequantiser stores) would double that.
 //
 // Each k-block issues two M=128 MMAs that share one B tile: the gate and
 // up rows of the same 128 features (first GEMM), or two adjacent 128-row
 // blocks of W_down (second GEMM).  Sharing B halves the activation bytes
 // per MAC, and in the first GEMM lane i of both accumulators belongs to
-// feature i, so the SwiGLU epilogue needs no exchange.
+// feature i, so the SwiGLU epilogue needs no exchange.  The MMA warp issues
+// the eight MMAs of a k-block back to back from fixed descriptor bases plus
+// constant offsets: address arithmetic between tcgen05.mma instructions
+// (descriptors rebuilt per MMA) was measured to cost 3-6x the MMA time.
+//
+// TMEM (512 columns) holds the two accumulators (2 x 128 columns) and four
+// A stages (4 x 2 matrices x 32 columns), so there is one accumulator
+// buffer.  To keep the MMA waiting as little as possible for the
+// epilogue, the epilogue only moves the accumulators through registers
+// into a shared-memory staging buffer (h as fp16, double-buffered; y_perm
+// as fp32), releases them, and then writes the staged rows out with
+// 16-byte stores while the next tile's MMAs run.
 //
 // Warp roles (16 warps):
 //   warp 0      codes producer: packed codes (3-D tensor map over the blob
 //               pool, one 128-row box per 128 K per matrix) and their
 //               scale/zero words (1-D bulk copies)
-//   warp 3      activation producer: fp16 rows of the bin (16-row TMA
-//               boxes, 128B swizzle)
-//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=tokens,
-//               K=16) and tcgen05.commit
-//   warp 2      TMEM allocator (512 columns: two buffers of two accumulators)
+//   warp 3      activation producer: one 128-row TMA box (128B swizzle)
+//               per 64 K of the tile's fp16 activation rows
+//   warp 1      MMA issuer: the whole warp waits, one elected lane issues
+//               tcgen05.mma (M=128, N=tokens, K=16) and tcgen05.commit
+//   warp 2      TMEM allocator
 //   warps 4-7   dequantisers of matrix 0, warps 8-11 of matrix 1: thread i
 //               turns weight row i of a staged codes block into fp16
-//               ((code - zero) * scale, one rounding) and writes it in the
-//               UMMA K-major 128B-swizzled layout
+//               ((code - zero) * scale, one rounding) and stores it to TMEM
+//               lane i (the warp's lane quadrant is warp % 4)
 //   warps 12-15 epilogue: tcgen05.ld of its TMEM lane quadrant; gate/up
-//               pass writes h = silu(gate) * up (fp16), down pass y_perm
-//               (fp32)
-// Pipelines: codes (2 stages of 128 K) -> dequant -> A (4 stages of 64 K);
-// activations B (3 stages of 64 K); both -> MMA -> TMEM (2 buffers) ->
-// epilogue.  Every wait is bounded; on a
-// timeout the CTA raises MOE_DEV_TIMEOUT, drains its copies and MMAs,
-// frees TMEM and returns.  Warps reconverge after every wait, before any
-// warp-aligned instruction.
+//               pass stages h = silu(gate) * up (fp16), down pass y_perm
+//               (fp32); then the four warps copy the staged rows out
+// Pipelines: codes (3 / 2 stages of 128 K) -> dequant -> A in TMEM (4
+// stages of 64 K); activations B (6 / 3 stages of 64 K, first / second
+// GEMM); both -> MMA -> accumulators -> epilogue staging -> global.  Every
+// wait is bounded; on a timeout the CTA raises MOE_DEV_TIMEOUT, drains its
+// copies and MMAs, frees TMEM and returns.  Warps reconverge after every
+// wait, before any warp-aligned instruction.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -149,10 +168,6 @@ __device__ __forceinline__ void trace_put(int* trace, int role, int site, int ti
   }
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             uint32_t bar) {
   asm volatile(
@@ -199,19 +214,40 @@ __device__ __forceinline__ uint32_t umma_idesc_f16(int n) {
   return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t accumulate) {
+
+// 32 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+
+
+__device__ __forceinline__ void umma_commit_elect(uint32_t bar) {
+  asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+               "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
                : "memory");
+}
+
+__device__ __forceinline__ void umma_f16_ts_elect(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -234,26 +270,37 @@ constexpr int kThreads = 512;  // 16 warps
 constexpr int kMaxBins = 768;
 constexpr int kNT = 128;       // largest token block (MMA N)
 
+// The epilogue stages a tile's outputs in shared memory (h fp16, 32 KB,
+// double-buffered; y fp32, 128 KB), releases the accumulators, and then
+// writes them out with 16-byte stores while the next tile's MMAs run.
+template <bool GATEUP>
 struct Cfg {
-  static constexpr int SA = 4;        // A (dequantised weight) stages of 64 K
-  static constexpr int SB = 3;        // B (activation) stages of 64 K
-  static constexpr int CSTAGES = 2;   // codes stages of 128 K
-  static constexpr int A_BYTES = 128 * 128;     // 128 weight rows x 64 fp16, per matrix
+  static constexpr int AK = 64;       // K of one A stage (TMEM)
+  static constexpr int SA = 4;        // A stages
+  static constexpr int ACC = 1;       // accumulator buffers (each: 2 matrices x kNT columns)
+  static constexpr int SB = GATEUP ? 6 : 3;        // B (activation) stages of 64 K
+  static constexpr int CSTAGES = GATEUP ? 3 : 2;   // codes stages of 128 K
+  static constexpr int OUT_BYTES = GATEUP ? kNT * 128 * 2 : kNT * 256 * 4;  // one staging buffer
+  static constexpr int OUT_BUFS = GATEUP ? 2 : 1;
   static constexpr int B_BYTES = kNT * 128;     // 128 token rows x 64 fp16
   static constexpr int C_BYTES = 8192;          // per matrix: 128 rows x 128 K of codes
   static constexpr int SZ_BYTES = 1024;         // per matrix: 128 rows x up to 2 groups x 4 B
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + SA * 2 * A_BYTES;
+  static constexpr int OFF_B = 0;
   static constexpr int OFF_C = OFF_B + SB * B_BYTES;
   static constexpr int OFF_SZ = OFF_C + CSTAGES * 2 * C_BYTES;
-  static constexpr int OFF_TILE = OFF_SZ + CSTAGES * 2 * SZ_BYTES;  // int tile_start[769], off[769]
+  static constexpr int OFF_OUT = OFF_SZ + CSTAGES * 2 * SZ_BYTES;
+  static constexpr int OFF_TILE = OFF_OUT + OUT_BUFS * OUT_BYTES;  // int tile_start[769], off[769]
   static constexpr int OFF_BAR = OFF_TILE + 2 * (kMaxBins + 1) * 4 + 8;
-  static constexpr int N_BARS = 2 * CSTAGES + 2 * SA + 2 * SB + 4 + 1 + 1;
+  static constexpr int N_BARS = 2 * CSTAGES + 2 * SA + 2 * SB + 2 * ACC + 1 + 1 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag
   static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + alignment slack
-  static constexpr int TMEM_COLS = 512;                  // 2 buffers x 2 accumulators x kNT
+  static constexpr int A_COLS = AK / 2;                  // TMEM columns of one matrix's A stage
+  static constexpr int ACOL = ACC * 2 * kNT;             // first A column
+  static constexpr int TMEM_COLS = 512;
 };
-static_assert(Cfg::SMEM <= 232448, "shared memory budget");
+static_assert(Cfg<true>::SMEM <= 232448 && Cfg<false>::SMEM <= 232448, "shared memory budget");
+static_assert(Cfg<true>::ACOL + Cfg<true>::SA * 2 * Cfg<true>::A_COLS <= Cfg<true>::TMEM_COLS, "TMEM budget");
+static_assert(Cfg<true>::AK == 64, "one A stage per B stage of 64 K");
 
 struct TcParams {
   CUtensorMap act;       // fp16 [rows][K], box 64 x 16, 128B swizzle
@@ -345,7 +392,7 @@ __device__ __forceinline__ float silu_fast(float v) { return v * __frcp_rn(1.0f 
 // matrix 1 = rows [256 mb + 128, +128) when they exist (d % 256 may be 128).
 template <bool GATEUP, bool PLANES>
 __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ TcParams P) {
-  using C = Cfg;
+  using C = Cfg<GATEUP>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   int* tile_start = reinterpret_cast<int*>(smem + C::OFF_TILE);
@@ -357,15 +404,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
   const uint32_t bar0 = smem_u32(bars);
   auto codes_full = [&](int i) { return bar0 + 8u * i; };
   auto codes_empty = [&](int i) { return bar0 + 8u * (C::CSTAGES + i); };
-  constexpr int kA = 2 * C::CSTAGES, kB = kA + 2 * C::SA, kR = kB + 2 * C::SB;
+  constexpr int kA = 2 * C::CSTAGES, kB = kA + 2 * C::SA, kR = kB + 2 * C::SB, kE = kR + 2 * C::ACC;
   auto a_full = [&](int i) { return bar0 + 8u * (kA + i); };
   auto a_empty = [&](int i) { return bar0 + 8u * (kA + C::SA + i); };
   auto b_full = [&](int i) { return bar0 + 8u * (kB + i); };
   auto b_empty = [&](int i) { return bar0 + 8u * (kB + C::SB + i); };
   auto acc_full = [&](int i) { return bar0 + 8u * (kR + i); };
-  auto acc_empty = [&](int i) { return bar0 + 8u * (kR + 2 + i); };
-  const uint32_t drain_bar = bar0 + 8u * (kR + 4);
-  const uint32_t exit_bar = bar0 + 8u * (kR + 5);
+  auto acc_empty = [&](int i) { return bar0 + 8u * (kR + C::ACC + i); };
+  const uint32_t drain_bar = bar0 + 8u * kE;
+  const uint32_t exit_bar = bar0 + 8u * (kE + 1);
+  const uint32_t epi_bar = bar0 + 8u * (kE + 2);  // the 4 epilogue warps, once per tile
   int* trace = P.trace ? P.trace + (GATEUP ? 0 : gridDim.x * 16) : nullptr;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -390,12 +438,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       mbar_init(b_full(i), 1);
       mbar_init(b_empty(i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::ACC; ++i) {
       mbar_init(acc_full(i), 1);
       mbar_init(acc_empty(i), 4);
     }
     mbar_init(drain_bar, 1);
     mbar_init(exit_bar, kThreads / 32);
+    mbar_init(epi_bar, 4);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -488,9 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
             trace_put(trace, 2, 2, t, kb);
             ok = mbar_wait(b_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
             if (!ok) break;
-            mbar_expect_tx(b_full(s), T.nt * 128);
-            const uint32_t bdst = smem_u32(smem + C::OFF_B + s * C::B_BYTES);
-            for (int i = 0; i < T.nt / 16; ++i) tma_load_2d(bdst + i * 2048, &P.act, kb * 64, T.row0 + 16 * i, b_full(s));
+            // one 128-row box: rows past this tile's are loaded but not read
+            // by the MMA (N = nt); rows past the tensor are zero-filled
+            mbar_expect_tx(b_full(s), C::B_BYTES);
+            tma_load_2d(smem_u32(smem + C::OFF_B + s * C::B_BYTES), &P.act, kb * 64, T.row0, b_full(s));
             if (++s == C::SB) { s = 0; sph ^= 1; }
           }
         }
@@ -515,53 +565,65 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
   }
   // ---- MMA issuer --------------------------------------------------------
   else if (warp == 1) {
-    if (lane == 0) {
+    {
       int sa = 0, saph = 0, sb = 0, sbph = 0, acc = 0, aph = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
         const uint32_t idesc = umma_idesc_f16(T.nt);
         const int nm = has_m1(T.mb) ? 2 : 1;
-        trace_put(trace, 1, 3, t, 0);
-        ok = mbar_wait(acc_empty(acc), aph ^ 1, abort_flag, P.status, trace, bar0);
+        if (lane == 0) trace_put(trace, 1, 3, t, 0);
+        ok = warp_wait(acc_empty(acc), aph ^ 1, abort_flag, P.status, trace, bar0);
         if (!ok) break;
         tc_fence_after();
         const uint32_t dcol = tmem_base + acc * (2 * kNT);
+        // operand addresses: fixed bases plus stage offsets, so that the
+        // MMAs of a k-block issue back to back
+        const uint64_t bdesc0 = umma_desc_sw128(smem_u32(smem + C::OFF_B));
+        const uint32_t acol0 = tmem_base + C::ACOL;
         for (int kb = 0; kb < 2 * KC && ok; ++kb) {
-          trace_put(trace, 1, 4, t, kb);
-          ok = mbar_wait(a_full(sa), saph, abort_flag, P.status, trace, bar0);
+          if (lane == 0) trace_put(trace, 1, 4, t, kb);
+          ok = warp_wait(a_full(sa), saph, abort_flag, P.status, trace, bar0);
           if (!ok) break;
-          trace_put(trace, 1, 5, t, kb);
-          ok = mbar_wait(b_full(sb), sbph, abort_flag, P.status, trace, bar0);
+          if (lane == 0) trace_put(trace, 1, 5, t, kb);
+          ok = warp_wait(b_full(sb), sbph, abort_flag, P.status, trace, bar0);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::OFF_B + sb * C::B_BYTES));
-          for (int m = 0; m < nm; ++m) {
-            const uint64_t adesc = umma_desc_sw128(smem_u32(smem + C::OFF_A + (sa * 2 + m) * C::A_BYTES));
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_f16(dcol + m * kNT, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(sb * (C::B_BYTES >> 4));
+          const uint32_t acol = acol0 + sa * (2 * C::A_COLS);
+          const uint32_t first = kb != 0;
+          umma_f16_ts_elect(dcol, acol, bdesc, idesc, first);
+          umma_f16_ts_elect(dcol, acol + 8, bdesc + 2, idesc, 1u);
+          umma_f16_ts_elect(dcol, acol + 16, bdesc + 4, idesc, 1u);
+          umma_f16_ts_elect(dcol, acol + 24, bdesc + 6, idesc, 1u);
+          if (nm == 2) {
+            umma_f16_ts_elect(dcol + kNT, acol + C::A_COLS, bdesc, idesc, first);
+            umma_f16_ts_elect(dcol + kNT, acol + C::A_COLS + 8, bdesc + 2, idesc, 1u);
+            umma_f16_ts_elect(dcol + kNT, acol + C::A_COLS + 16, bdesc + 4, idesc, 1u);
+            umma_f16_ts_elect(dcol + kNT, acol + C::A_COLS + 24, bdesc + 6, idesc, 1u);
           }
-          umma_commit(a_empty(sa));
-          umma_commit(b_empty(sb));
+          umma_commit_elect(a_empty(sa));
+          umma_commit_elect(b_empty(sb));
           if (++sa == C::SA) { sa = 0; saph ^= 1; }
           if (++sb == C::SB) { sb = 0; sbph ^= 1; }
         }
         if (!ok) break;
-        umma_commit(acc_full(acc));
-        if (++acc == 2) { acc = 0; aph ^= 1; }
+        umma_commit_elect(acc_full(acc));
+        if (++acc == C::ACC) { acc = 0; aph ^= 1; }
       }
-      trace_put(trace, 1, ok ? 12 : 13, 0, 0);
+      if (lane == 0) trace_put(trace, 1, ok ? 12 : 13, 0, 0);
       // all MMAs issued by this thread complete before TMEM is released
-      umma_commit(drain_bar);
+      umma_commit_elect(drain_bar);
       const uint64_t t0 = global_ns();
       while (!mbar_try(drain_bar, 0) && global_ns() - t0 < kWaitLimitNs) {}
+      __syncwarp();
     }
   }
   // ---- dequantisers: warps 4-7 matrix 0, warps 8-11 matrix 1 -------------
   else if (warp >= 4 && warp < 12) {
     const int m = (warp - 4) >> 2;
-    const int i = tid - 128 - 128 * m;   // weight row inside the 128-row block
+    const int i = tid - 128 - 128 * m;   // weight row inside the 128-row block = TMEM lane
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
     int cs = 0, cph = 0, s = 0, sph = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
@@ -611,20 +673,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
           if (lane == 0) trace_put(trace, 3 + m, 7, t, 2 * kc + h);
           ok = warp_wait(a_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
           if (!ok) break;
+          tc_fence_after();  // the MMAs that read this stage have completed
           if (live) {
             const uint32_t word = h ? sz1 : sz0;
             const __half sc = __float2half_rn(__uint_as_float(word << 16));
             const float zf = __uint_as_float(word & 0xFFFF0000u);
             const __half2 s2 = __half2half2(sc);
             const __half2 z2 = __halves2half2(__float2half_rn(1024.0f + zf), __float2half_rn(64.0f + zf));
-            uint8_t* arow = smem + C::OFF_A + (s * 2 + m) * C::A_BYTES + i * 128;
+            uint32_t v[32];  // column c = elements (2c, 2c + 1) of this 64-K slice of row i
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = elements 8j..8j+7 of the half
+            for (int j = 0; j < 8; ++j) {
               const uint4 o = dequant8(w[8 * h + j], z2, s2);
-              *reinterpret_cast<uint4*>(arow + ((j ^ (i & 7)) << 4)) = o;
+              v[4 * j] = o.x; v[4 * j + 1] = o.y; v[4 * j + 2] = o.z; v[4 * j + 3] = o.w;
             }
-            fence_proxy_async_smem();
+            tmem_st32(lane_base + C::ACOL + (s * 2 + m) * C::A_COLS, v);
+            tmem_st_wait();
           }
+          tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(a_full(s));
           if (++s == C::SA) { s = 0; sph ^= 1; }
@@ -635,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
   // ---- epilogue: warps 12-15, TMEM lane quadrant = warp % 4 ---------------
   else if (warp >= 12) {
     const int q = warp & 3;
-    int acc = 0, aph = 0;
+    int acc = 0, aph = 0, ep_tile = 0, ep_ph = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
       const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
@@ -646,36 +711,83 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * (2 * kNT);
       const int r = 32 * q + lane;  // row of the weight block
-      for (int j0 = 0; j0 < T.nrows; j0 += 16) {
-        uint32_t a0[16], a1[16];
-        tmem_ld16(tbase + j0, a0);
-        if (m1) tmem_ld16(tbase + kNT + j0, a1);
-        tmem_ld_wait();
+      // 16-token chunks; the TMEM loads of chunk c + 1 are in flight while
+      // chunk c is converted and written to the staging buffer
+      uint8_t* stage = smem + C::OFF_OUT + (C::OUT_BUFS == 2 ? (ep_tile & 1) : 0) * C::OUT_BYTES;
+      auto emit = [&](const uint32_t (&a0)[16], const uint32_t (&a1)[16], int j0) {
         if (GATEUP) {
-          const int f = T.mb * 128 + r;
+          __half* hs = reinterpret_cast<__half*>(stage);  // [token][128 features]
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            if (j0 + j < T.nrows) {
-              const float gv = __uint_as_float(a0[j]), uv = __uint_as_float(a1[j]);
-              P.h_out[static_cast<size_t>(T.row0 + j0 + j) * P.N + f] = __float2half_rn(silu_fast(gv) * uv);
-            }
+            const float gv = __uint_as_float(a0[j]), uv = __uint_as_float(a1[j]);
+            hs[(j0 + j) * 128 + r] = __float2half_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
           }
         } else {
-          const int n0 = row_base(T.mb, 0) + r, n1 = row_base(T.mb, 1) + r;
+          float* ys = reinterpret_cast<float*>(stage);  // [token][256 outputs]
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            if (j0 + j < T.nrows) {
-              float* yrow = P.y_out + static_cast<size_t>(T.row0 + j0 + j) * P.N;
-              yrow[n0] = __uint_as_float(a0[j]);
-              if (m1) yrow[n1] = __uint_as_float(a1[j]);
-            }
+            ys[(j0 + j) * 256 + r] = __uint_as_float(a0[j]);
+            ys[(j0 + j) * 256 + 128 + r] = __uint_as_float(a1[j]);
           }
         }
+      };
+      uint32_t g0[16], u0[16], g1[16], u1[16];
+      tmem_ld16(tbase, g0);
+      if (m1) tmem_ld16(tbase + kNT, u0);
+      tmem_ld_wait();
+      for (int j0 = 0; j0 < T.nrows; j0 += 32) {
+        const bool more1 = j0 + 16 < T.nrows;
+        if (more1) {
+          tmem_ld16(tbase + j0 + 16, g1);
+          if (m1) tmem_ld16(tbase + kNT + j0 + 16, u1);
+        }
+        emit(g0, u0, j0);
+        tmem_ld_wait();
+        if (more1) {
+          const bool more2 = j0 + 32 < T.nrows;
+          if (more2) {
+            tmem_ld16(tbase + j0 + 32, g0);
+            if (m1) tmem_ld16(tbase + kNT + j0 + 32, u0);
+          }
+          emit(g1, u1, j0 + 16);
+          tmem_ld_wait();
+        }
       }
+      // accumulators read: the MMA may start the next tile
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(acc));
-      if (++acc == 2) { acc = 0; aph ^= 1; }
+      if (++acc == C::ACC) { acc = 0; aph ^= 1; }
+      // all four warps have staged their rows
+      if (lane == 0) mbar_arrive(epi_bar);
+      ok = warp_wait(epi_bar, ep_ph, abort_flag, P.status, trace, bar0);
+      ep_ph ^= 1;
+      if (!ok) break;
+      // 16-byte stores of the staged rows (tokens) that belong to this tile
+      const int et = tid - 12 * 32;  // 0..127
+      if (GATEUP) {
+        const uint4* src = reinterpret_cast<const uint4*>(stage);
+        const size_t f0 = static_cast<size_t>(T.mb) * 128;
+        for (int c = et; c < T.nrows * 16; c += 128) {
+          const int row = c >> 4, col = c & 15;
+          *reinterpret_cast<uint4*>(P.h_out + static_cast<size_t>(T.row0 + row) * P.N + f0 + col * 8) = src[c];
+        }
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(stage);
+        const int n0 = row_base(T.mb, 0);
+        const int per_row = m1 ? 64 : 32;  // 16-byte pieces of a row's 256 (or 128) outputs
+        for (int c = et; c < T.nrows * 64; c += 128) {
+          const int row = c >> 6, col = c & 63;
+          if (col < per_row)
+            *reinterpret_cast<uint4*>(P.y_out + static_cast<size_t>(T.row0 + row) * P.N + n0 + col * 4) = src[c];
+        }
+        // the single buffer is rewritten by the next tile: wait for every warp's copy
+        if (lane == 0) mbar_arrive(epi_bar);
+        ok = warp_wait(epi_bar, ep_ph, abort_flag, P.status, trace, bar0);
+        ep_ph ^= 1;
+        if (!ok) break;
+      }
+      ++ep_tile;
     }
   }
 
@@ -744,7 +856,7 @@ moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int r
   {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
     cuuint64_t str[1] = {static_cast<cuuint64_t>(K) * 2};
-    cuuint32_t box[2] = {64, 16};
+    cuuint32_t box[2] = {64, 128};
     if (!encode(&P.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, act, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) {
       set_error("tensor map (activations) could not be encoded");
       return MOE_ERR_CUDA;
@@ -801,11 +913,11 @@ moe_status_t launch_one(const TcParams& P, cudaStream_t s) {
   // Set once per process (the first call must precede any stream capture).
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<GATEUP>::SMEM);
     if (e != cudaSuccess) return cuda_check(e, "tc ffn smem attribute");
     attr_set = true;
   }
-  kern<<<sm_count(), kThreads, Cfg::SMEM, s>>>(P);
+  kern<<<sm_count(), kThreads, Cfg<GATEUP>::SMEM, s>>>(P);
   return cuda_check(cudaGetLastError(), "tc ffn launch");
 }
 
