@@ -206,6 +206,27 @@ def make_instances(shape, T, R, seed, device):
     return layers
 
 
+def profiled_traffic(workload, T):
+    """DRAM bytes (read + write) of one FFN call (gate/up + down launches) from
+    the committed ncu summary, if it covers this workload and the kernel
+    source is unchanged since the counters were taken; else None."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", f"k_ffn_tc_{workload}_t{T}.md")
+    src = os.path.join(ROOT, "quantized_moe_expert_histogram_b200", "csrc", "tc_gemm.cu")
+    if not os.path.exists(path):
+        return None, None
+    text = open(path).read()
+    m_hash = re.search(r"source_sha1: ([0-9a-f]{40})", text)
+    m_bytes = re.search(r"dram_bytes_per_step: (\d+)", text)
+    if not m_hash or not m_bytes:
+        return None, None
+    with open(src, "rb") as f:
+        if hashlib.sha1(f.read()).hexdigest() != m_hash.group(1):
+            return None, "kernel changed since the ncu capture"
+    return int(m_bytes.group(1)), os.path.relpath(path, ROOT)
+
+
 def algorithmic(shape, T, layer, bits_present):
     """Algorithmic bytes and flops of one layer pass from the routing taken."""
     from quantized_moe_expert_histogram_b200 import moeq
@@ -416,7 +437,9 @@ def main():
     else:
         ach = bytes_alg / t_ffn / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s", "frac": ach / peaks["hbm"]}
-    roof.update({"traffic": None, "kernel": "moe_grouped_ffn_wq (gate/up + down launches)",
+    traffic, traffic_src = profiled_traffic(shape.name, T)
+    roof.update({"traffic": traffic, "traffic_source": traffic_src,
+                 "kernel": "moe_grouped_ffn_wq (gate/up + down launches)",
                  "timing": "FFN-only CUDA graph over the same rotated instances, events around the replays",
                  "peak_source": peaks["src"], "ffn_ms": ffn_ms,
                  "per_launch_units": f"{T * shape.k} assignments"})
