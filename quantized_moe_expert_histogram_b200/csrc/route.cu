@@ -69,7 +69,7 @@ __host__ __device__ inline RouteWs route_ws(void* base, int S, int T, int E) {
 }
 
 template <int EC>
-__global__ void __launch_bounds__(kLT) k_route_logits(const __nv_bfloat16* __restrict__ x,
+__global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __restrict__ x,
                                                        const float* __restrict__ wr, int T, int d, int E,
                                                        int dk, RouteWs ws) {
   using G = Tile<EC>;
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kLT) k_route_logits(const __nv_bfloat16* __res
     const int b = c & 1;
     if (c + 1 < nch) fetch(kbeg + (c + 1) * kDC);
     const float* xb = xs + b * G::XS + ty * kMT * G::XP;
-    const float* wb = wsm + b * G::WS + tx * G::ME;
+    const float* wb = wsm + b * G::WS + tx * 4;
     float cs[kMT][G::ME];
 #pragma unroll
     for (int i = 0; i < kMT; ++i)
@@ -159,8 +159,8 @@ __global__ void __launch_bounds__(kLT) k_route_logits(const __nv_bfloat16* __res
 #pragma unroll
       for (int i = 0; i < kMT; ++i) xa[i] = xb[i * G::XP + kk];
 #pragma unroll
-      for (int j = 0; j < G::ME; j += 4) {
-        const float4 w4 = *reinterpret_cast<const float4*>(wb + kk * EC + j);
+      for (int j = 0; j < G::ME; j += 4) {  // experts tx*4 + (0..3) [+ EC/2]
+        const float4 w4 = *reinterpret_cast<const float4*>(wb + kk * EC + (j / 4) * (EC / 2));
         wv[j] = w4.x; wv[j + 1] = w4.y; wv[j + 2] = w4.z; wv[j + 3] = w4.w;
       }
 #pragma unroll
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kLT) k_route_logits(const __nv_bfloat16* __res
     if (t >= T) continue;
 #pragma unroll
     for (int j = 0; j < G::ME; ++j) {
-      const int e = e0 + tx * G::ME + j;
+      const int e = e0 + tx * 4 + (j & 3) + (j / 4) * (EC / 2);
       if (e < E) out[static_cast<size_t>(t) * E + e] = acc[i][j];
     }
   }

@@ -582,10 +582,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         const uint64_t bdesc0 = umma_desc_sw128(smem_u32(smem + C::OFF_B));
         const uint32_t acol0 = tmem_base + C::ACOL;
         for (int kb = 0; kb < 2 * KC && ok; ++kb) {
-          if (lane == 0) trace_put(trace, 1, 4, t, kb);
           ok = warp_wait(a_full(sa), saph, abort_flag, P.status, trace, bar0);
           if (!ok) break;
-          if (lane == 0) trace_put(trace, 1, 5, t, kb);
           ok = warp_wait(b_full(sb), sbph, abort_flag, P.status, trace, bar0);
           if (!ok) break;
           tc_fence_after();
