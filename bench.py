@@ -43,6 +43,8 @@ def parse():
     p.add_argument("--sweep", default="1,16,256", help="extra token counts timed for context ('' = none)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=0)
+    p.add_argument("--offload-steps", type=int, default=24,
+                   help="decode steps of the offload (slot-cache) workload reported under 'offload' (0 = skip)")
     p.add_argument("--profile", action="store_true",
                    help="profiling driver: one instance, warmup + steps of the eager step, no JSON")
     return p.parse_args()
@@ -322,6 +324,58 @@ def time_e2e(layers, steps, stream):
     return start.elapsed_time(end), h2d, T * d * 2
 
 
+def h2d_peak_gbs(nbytes=256 << 20, reps=5):
+    """Pinned host -> device copy bandwidth (one large cudaMemcpyAsync)."""
+    import torch
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dv = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        dv.copy_(h, non_blocking=True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(reps):
+            dv.copy_(h, non_blocking=True)
+        b.record(s)
+    torch.cuda.synchronize()
+    return nbytes * reps / (a.elapsed_time(b) / 1e3) / 1e9
+
+
+def run_offload(steps, layers=16, slots=16, batch=8, seed=0):
+    """The offload workload: stacked OLMoE-shaped layers with experts in pinned
+    host memory and a slot cache per layer, decode steps at a fixed batch on a
+    Zipf + successor-correlated routing trace.  Wall time around whole steps
+    (each layer's step synchronises once for the routed ids)."""
+    import torch
+    from quantized_moe_expert_histogram_b200 import inputs as I
+    from quantized_moe_expert_histogram_b200.offload import OffloadStack
+    shape = I.SHAPES["olmoe"]
+    stack = OffloadStack(shape, layers, slots, batch, seed=seed)
+    warm = 2
+    trace = I.make_slot_trace(shape.E, shape.k, layers, steps + warm, batch, seed=seed + 1).cuda()
+    xs = I.make_slot_x(shape.d, steps + warm, batch, seed=seed + 1, device="cuda")
+    for s in range(warm):
+        stack.step(xs[s], trace[s])
+    torch.cuda.synchronize()
+    peak = h2d_peak_gbs()
+    hits = misses = nbytes = 0
+    t0 = time.perf_counter()
+    for s in range(warm, warm + steps):
+        _, st = stack.step(xs[s], trace[s])
+        for h, m, b, _w in st:
+            hits, misses, nbytes = hits + h, misses + m, nbytes + b
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    stack.close()
+    h2d = nbytes / wall / 1e9
+    return {"workload": f"{layers} OLMoE-shaped layers (d=2048, E=64, top-8, d_ff=1024, INT4 g128), "
+                        f"{slots} GPU slots per layer, batch {batch}, Zipf routing with 70% successor correlation",
+            "steps": steps, "tokens_per_s": batch * steps / wall, "ms_per_step": wall / steps * 1e3,
+            "h2d_bytes_per_step": nbytes / steps, "h2d_gbs": h2d, "h2d_peak_gbs": peak,
+            "h2d_frac": h2d / peak, "hit_rate": hits / max(1, hits + misses),
+            "timing": "host wall clock around whole steps (one routed-id sync per layer)"}
+
+
 def cpu_baseline(shape, T, seed, sample_tokens, budget_s=20.0):
     """The oracle as it stands, on the host cores, on a bounded token sample."""
     import numpy as np
@@ -463,11 +517,19 @@ def main():
         del ls, ga, gf
         torch.cuda.empty_cache()
 
+    offload = None
+    if world == 1 and args.offload_steps > 0:
+        del layers
+        torch.cuda.empty_cache()
+        offload = run_offload(args.offload_steps)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(shape, T, 0, args.cpu_sample_tokens)
 
-    launches_per_step = 6
+    # our kernels per step: router 2, permutation 1 + gather (<= 1024 assignments) or
+    # 3 + gather, FFN 2, combine 1
+    launches_per_step = 2 + (2 if T * shape.k <= 1024 else 4) + 2 + 1
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
@@ -477,7 +539,7 @@ def main():
                        "l2": f"{args.instances} layer instances rotated ({shape.E} experts x "
                              f"{moeq.moe_blob_bytes(shape.d, shape.F, shape.group, 0)} B each), inputs > L2"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * steps,
-            "clocks": clk, "sweep": sweep}
+            "clocks": clk, "sweep": sweep, "offload": offload}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

@@ -13,6 +13,8 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y_per
                                                   const float* __restrict__ gw,
                                                   const __nv_bfloat16* __restrict__ residual, int T,
                                                   int k, int d, __nv_bfloat16* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int vec = d / 8;
   const long total = static_cast<long>(T) * vec;
   for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
@@ -62,10 +64,10 @@ moe_status_t launch_combine(const void* y_perm, const int32_t* inv_perm, const f
   if (T == 0) return MOE_OK;
   const long vecs = static_cast<long>(T) * (d / 8);
   const int blocks = static_cast<int>(std::min<long>((vecs + 255) / 256, 148L * 16));
-  k_combine<<<blocks, 256, 0, s>>>(static_cast<const float*>(y_perm), inv_perm, w,
+  const cudaError_t e = launch_pdl(pdl_for(static_cast<long>(T) * k), k_combine, dim3(blocks), dim3(256), 0, s, static_cast<const float*>(y_perm), inv_perm, w,
                                    static_cast<const __nv_bfloat16*>(residual), T, k, d,
                                    static_cast<__nv_bfloat16*>(y));
-  return cuda_check(cudaGetLastError(), "moe_unpermute_combine launch");
+  return cuda_check(e, "moe_unpermute_combine launch");
 }
 
 }  // namespace moeq

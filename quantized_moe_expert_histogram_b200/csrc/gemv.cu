@@ -11,13 +11,12 @@
 // Accumulation is fp32.  blockIdx.y enumerates the non-empty (and, in slot
 // mode, resident) bins; blockIdx.x a block of 8 warps x RW output rows.
 //
-// The down pass is a programmatic dependent launch of the gate/up pass: its
-// blocks start while the gate/up pass runs, locate their bin and issue the
-// loads of their weight codes (which do not depend on h), and only then
-// wait (griddepcontrol.wait) for the gate/up grid before reading h.  The
-// gate/up pass allows that early start as soon as it begins; everything the
-// down pass reads before its wait (offsets, slot table, weights) was
-// complete before the gate/up pass was launched.
+// Both passes are programmatic dependent launches (launch_pdl).  The down
+// pass starts while the gate/up pass runs, locates its bin and issues the
+// loads of its weight codes (which do not depend on h), and only then waits
+// for the gate/up grid before reading h.  The gate/up pass triggers after
+// its own wait, so everything the down pass reads before its wait
+// (offsets, slot table, weights) is complete by then.
 //
 //   gate/up pass:  h[p][f]      = silu(Wg[f] . x_p) * (Wu[f] . x_p)   (fp16)
 //   down pass:     y_perm[p][n] = Wd[n] . h_p                          (fp32)
@@ -29,7 +28,7 @@ namespace moeq {
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
-constexpr int kChunkSteps = 4;  // 32-element steps whose loads are issued together
+constexpr int kChunkSteps = 2;  // 32-element steps whose loads are issued together
 
 struct GemvParams {
   const __half* act;        // x_perm [rows][K] or h [rows][K]
@@ -142,12 +141,15 @@ __device__ __forceinline__ uint4 load_codes(const GemvParams& P, const uint8_t* 
 
 // RW output rows per warp; NM matrices (2 = gate+up, 1 = down).
 template <int MAXR, int NM, int RW, bool PLANES>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_gemv(const GemvParams P) {
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, MAXR <= 2 ? 3 : 1) k_gemv(const GemvParams P) {
   constexpr int ROWS = NM * RW;  // weight rows per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // gate/up: let the down pass launch now; down: activations (h) are read
-  // only after griddepcontrol.wait below
-  if (NM == 2) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // gate/up: wait for the earlier kernels, then let the down pass launch;
+  // down: h is read only after the wait below (the weight codes before it)
+  if (NM == 2) {
+    pdl_wait();
+    pdl_trigger();
+  }
   bool dep_waited = NM == 2;
   int bin, row0, nrows, blob_index, bits;
   if (!find_bin(P, blockIdx.y, bin, row0, nrows, blob_index, bits)) return;
@@ -185,7 +187,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_gemv(const GemvParams P
       }
     }
     if (!dep_waited) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");
+      pdl_wait();
+      pdl_trigger();
       dep_waited = true;
     }
 #pragma unroll
@@ -271,21 +274,12 @@ template <int MAXR, bool PLANES>
 moe_status_t run_pair(GemvParams gu, GemvParams dn, int max_bins, cudaStream_t s) {
   constexpr int RW_GU = 2, RW_DN = 4;
   dim3 g1(ceil_div(gu.N, kWarpsPerBlock * RW_GU), max_bins);
-  k_gemv<MAXR, 2, RW_GU, PLANES><<<g1, kWarpsPerBlock * 32, 0, s>>>(gu);
-  moe_status_t st = cuda_check(cudaGetLastError(), "ffn gemv gate/up launch");
+  moe_status_t st = cuda_check(launch_pdl(true, k_gemv<MAXR, 2, RW_GU, PLANES>, g1, dim3(kWarpsPerBlock * 32), 0, s, gu),
+                               "ffn gemv gate/up launch");
   if (st != MOE_OK) return st;
-  // programmatic dependent launch (see the note at the top of the file)
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(ceil_div(dn.N, kWarpsPerBlock * RW_DN), max_bins);
-  cfg.blockDim = dim3(kWarpsPerBlock * 32);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, k_gemv<MAXR, 1, RW_DN, PLANES>, dn), "ffn gemv down launch");
+  dim3 g2(ceil_div(dn.N, kWarpsPerBlock * RW_DN), max_bins);
+  return cuda_check(launch_pdl(true, k_gemv<MAXR, 1, RW_DN, PLANES>, g2, dim3(kWarpsPerBlock * 32), 0, s, dn),
+                    "ffn gemv down launch");
 }
 
 }  // namespace

@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_perm_hist(const int32_t* __rest
                                                            int E, int nbins,
                                                            int32_t* __restrict__ hist,
                                                            int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t hist_s[];  // [kWarps][nbins]
   for (int i = threadIdx.x; i < kWarps * nbins; i += blockDim.x) hist_s[i] = 0;
   __syncthreads();
@@ -92,6 +94,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_perm_hist(const int32_t* __rest
 __global__ void __launch_bounds__(1024) k_perm_scan(int32_t* __restrict__ hist, int ctas, int nbins,
                                                     int n, int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int32_t scan_buf[32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int total = 0;
@@ -161,6 +165,8 @@ __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict_
                                                  const int32_t* __restrict__ perm, int rows, int k,
                                                  int d, __half* __restrict__ x_perm,
                                                  int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int vec = d / 8;
   bool bad = false;
@@ -195,6 +201,8 @@ __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict_
 __global__ void __launch_bounds__(kWarps * 32) k_perm_scatter(
     const int32_t* __restrict__ idx, const uint8_t* __restrict__ bits, int n, int E, int nbins, int k,
     const int32_t* __restrict__ hist, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t hist_s[];  // [kWarps][nbins] -> per-warp start positions
   for (int i = threadIdx.x; i < kWarps * nbins; i += blockDim.x) hist_s[i] = 0;
   __syncthreads();
@@ -220,6 +228,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_perm_one(
     const int32_t* __restrict__ idx, const uint8_t* __restrict__ bits, int n, int E, int nbins, int k,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
     int32_t* __restrict__ inv_perm, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t hist_s[];  // [kWarps][nbins]
   __shared__ int32_t warp_sum[kWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -315,25 +325,26 @@ moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void*
   }
   moe_status_t st;
   if (ctas == 1) {
-    k_perm_one<<<1, kWarps * 32, smem, s>>>(idx, bits, n, E, nbins, k, counts, offsets, perm, inv_perm,
-                                            status);
-    st = cuda_check(cudaGetLastError(), "moe_permute launch");
+    st = cuda_check(launch_pdl(pdl_for(n), k_perm_one, dim3(1), dim3(kWarps * 32), smem, s, idx, bits, n, E, nbins, k, counts,
+                               offsets, perm, inv_perm, status),
+                    "moe_permute launch");
   } else {
-    k_perm_hist<<<ctas, kWarps * 32, smem, s>>>(idx, bits, n, E, nbins, hist, status);
-    st = cuda_check(cudaGetLastError(), "moe_permute histogram launch");
+    st = cuda_check(launch_pdl(pdl_for(n), k_perm_hist, dim3(ctas), dim3(kWarps * 32), smem, s, idx, bits, n, E, nbins, hist, status),
+                    "moe_permute histogram launch");
     if (st != MOE_OK) return st;
-    k_perm_scan<<<1, 1024, 0, s>>>(hist, ctas, nbins, n, counts, offsets);
-    st = cuda_check(cudaGetLastError(), "moe_permute scan launch");
+    st = cuda_check(launch_pdl(pdl_for(n), k_perm_scan, dim3(1), dim3(1024), 0, s, hist, ctas, nbins, n, counts, offsets),
+                    "moe_permute scan launch");
     if (st != MOE_OK) return st;
-    k_perm_scatter<<<ctas, kWarps * 32, smem, s>>>(idx, bits, n, E, nbins, k, hist, perm, inv_perm);
-    st = cuda_check(cudaGetLastError(), "moe_permute scatter launch");
+    st = cuda_check(launch_pdl(pdl_for(n), k_perm_scatter, dim3(ctas), dim3(kWarps * 32), smem, s, idx, bits, n, E, nbins, k,
+                               static_cast<const int32_t*>(hist), perm, inv_perm),
+                    "moe_permute scatter launch");
   }
   if (st != MOE_OK || !x_perm || n == 0) return st;
   // a warp per row: up to 8 rows per block, at most 8 blocks per SM
   const int blocks = std::max(1, std::min((n + 7) / 8, 8 * sm_count_permute()));
-  k_gather<<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), perm, n, k, d,
-                                  static_cast<__half*>(x_perm), status);
-  return cuda_check(cudaGetLastError(), "moe_permute gather launch");
+  return cuda_check(launch_pdl(pdl_for(n), k_gather, dim3(blocks), dim3(256), 0, s, static_cast<const __nv_bfloat16*>(x),
+                                static_cast<const int32_t*>(perm), n, k, d, static_cast<__half*>(x_perm), status),
+                    "moe_permute gather launch");
 }
 
 }  // namespace moeq

@@ -72,6 +72,8 @@ template <int EC>
 __global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __restrict__ x,
                                                        const float* __restrict__ wr, int T, int d, int E,
                                                        int dk, RouteWs ws) {
+  pdl_wait();
+  pdl_trigger();
   using G = Tile<EC>;
   extern __shared__ __align__(16) float sm[];
   float* xs = sm;               // [2][TT][XP]
@@ -333,6 +335,8 @@ __global__ void __launch_bounds__(kSelThreads) k_route_select(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, RouteWs ws, int splits,
     const float* __restrict__ bias, const int32_t* __restrict__ forced, int T, int d, int E, int k,
     float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int n_cand[kSelWarps];
   __shared__ uint8_t cand[kSelWarps][256];
   __shared__ double l64[kSelWarps][256];
@@ -472,7 +476,7 @@ float route_gamma(int d) {
 }
 
 template <int EC>
-moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d, int E, int splits,
+moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d, int E, int k_route, int splits,
                            RouteWs ws, cudaStream_t s) {
   using G = Tile<EC>;
   static bool attr_set = false;  // once per process (the first call precedes any capture)
@@ -483,8 +487,8 @@ moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d
     attr_set = true;
   }
   dim3 grid(ceil_div(T, G::TT), ceil_div(E, EC), splits);
-  k_route_logits<EC><<<grid, kLT, G::SMEM, s>>>(x, wr, T, d, E, d / splits, ws);
-  return cuda_check(cudaGetLastError(), "moe_route_topk logits launch");
+  return cuda_check(launch_pdl(pdl_for(static_cast<long>(T) * k_route), k_route_logits<EC>, grid, dim3(kLT), G::SMEM, s, x, wr, T, d, E, d / splits, ws),
+                    "moe_route_topk logits launch");
 }
 
 }  // namespace
@@ -502,12 +506,12 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
   const int splits = route_splits(T, d, E);
   const RouteWs ws = route_ws(workspace, splits, T, E);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, splits, ws, s)
-                            : launch_logits<64>(xb, w_router, T, d, E, splits, ws, s);
+  moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, k, splits, ws, s)
+                            : launch_logits<64>(xb, w_router, T, d, E, k, splits, ws, s);
   if (st != MOE_OK) return st;
-  k_route_select<<<ceil_div(T, kSelWarps), kSelThreads, 0, s>>>(xb, w_router, ws, splits, bias, forced, T,
-                                                                  d, E, k, route_gamma(d), idx, w);
-  return cuda_check(cudaGetLastError(), "moe_route_topk select launch");
+  return cuda_check(launch_pdl(pdl_for(static_cast<long>(T) * k), k_route_select, dim3(ceil_div(T, kSelWarps)), dim3(kSelThreads), 0, s, xb, w_router, ws,
+                               splits, bias, forced, T, d, E, k, route_gamma(d), idx, w),
+                    "moe_route_topk select launch");
 }
 
 }  // namespace moeq

@@ -454,6 +454,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  // barrier set-up and the TMEM allocation may overlap the previous kernel;
+  // everything below reads what earlier kernels wrote
+  pdl_wait();
+  pdl_trigger();
   for (int b = tid; b <= nbins; b += kThreads) off_s[b] = P.offsets[b];
   __syncwarp();
   __syncthreads();
@@ -906,7 +910,7 @@ moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int r
 }
 
 template <bool GATEUP, bool PLANES>
-moe_status_t launch_one(const TcParams& P, cudaStream_t s) {
+moe_status_t launch_one(const TcParams& P, bool pdl, cudaStream_t s) {
   auto kern = k_ffn_tc<GATEUP, PLANES>;
   // Set once per process (the first call must precede any stream capture).
   static bool attr_set = false;
@@ -915,8 +919,7 @@ moe_status_t launch_one(const TcParams& P, cudaStream_t s) {
     if (e != cudaSuccess) return cuda_check(e, "tc ffn smem attribute");
     attr_set = true;
   }
-  kern<<<sm_count(), kThreads, Cfg<GATEUP>::SMEM, s>>>(P);
-  return cuda_check(cudaGetLastError(), "tc ffn launch");
+  return cuda_check(launch_pdl(pdl, kern, dim3(sm_count()), dim3(kThreads), Cfg<GATEUP>::SMEM, s, P), "tc ffn launch");
 }
 
 }  // namespace
@@ -927,6 +930,7 @@ bool tc_supported(const FfnArgs& a) {
 }
 
 moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s) {
+  const bool pdl = pdl_for(a.total_rows);
   const int n_blobs = a.slot_of ? 65536 : a.E;
   const bool planes = a.layout == MOE_LAYOUT_PLANES;
   TcParams gu{};
@@ -935,7 +939,7 @@ moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s) {
   if (st != MOE_OK) return st;
   gu.h_out = a.h;
   gu.y_out = nullptr;
-  st = planes ? launch_one<true, true>(gu, s) : launch_one<true, false>(gu, s);
+  st = planes ? launch_one<true, true>(gu, pdl, s) : launch_one<true, false>(gu, pdl, s);
   if (st != MOE_OK) return st;
   TcParams dn{};
   const int m_dn[1] = {2};
@@ -943,7 +947,7 @@ moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s) {
   if (st != MOE_OK) return st;
   dn.h_out = nullptr;
   dn.y_out = a.y_perm;
-  return planes ? launch_one<false, true>(dn, s) : launch_one<false, false>(dn, s);
+  return planes ? launch_one<false, true>(dn, pdl, s) : launch_one<false, false>(dn, pdl, s);
 }
 
 }  // namespace moeq

@@ -1,0 +1,75 @@
+"""Offload mode: stacked MoE layers whose experts live in pinned host memory.
+
+Each layer keeps all of its packed experts in pinned host memory and a GPU
+slot pool of a few experts; ``moe_slot_stage`` brings the experts a layer
+step routes to into the pool on a copy stream (hits first, then misses by
+token count, in waves of half the slots) and ``moe_slot_ffn`` runs the
+grouped FFN wave by wave as the copies land.  Pages: ExactMoE (compressed
+experts in host memory, GPU-resident slot cache, every routed expert
+executed), EdgeMoE (expert buffer filled on activation), D2MoE (loading the
+next expert while computing the current one).
+
+``OffloadStack.step`` runs one decode step through all layers: route (the
+expert ids may be forced from a trace), the one device-to-host copy of the
+routed ids per layer, stage, permute, slot FFN, combine with the residual.
+This module only orchestrates calls of the C ABI; torch supplies device
+memory, pinned host memory and streams.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import inputs as I
+from . import moeq
+from .layer import QuantMoELayer
+
+
+class OffloadStack:
+    def __init__(self, shape, layers: int, slots: int, batch: int, seed: int = 0, device="cuda"):
+        self.shape, self.n_layers, self.slots, self.batch = shape, layers, slots, batch
+        self.layers, self.host, self.pools, self.caches = [], [], [], []
+        for l in range(layers):
+            w = I.make_expert_weights(shape, seed=seed + 101 * l, device=device)
+            r = I.make_router(shape, seed=seed + 101 * l + 1, device=device)
+            layer = QuantMoELayer.from_weights(shape, r["w_router"], r["bias"], w["w_gate"], w["w_up"],
+                                               w["w_down"], max_tokens=batch)
+            del w
+            host = layer.blobs.cpu().pin_memory()
+            pool = torch.empty(slots, layer.blobs.shape[1], dtype=torch.uint8, device=device)
+            layer.blobs = None  # the experts now live in host memory only
+            self.layers.append(layer)
+            self.host.append(host)
+            self.pools.append(pool)
+            self.caches.append(moeq.SlotCache(shape.E, slots, host.shape[1], host, pool))
+        self.blob_bytes = self.host[0].shape[1]
+        self.copy = torch.cuda.Stream()
+        self.compute = torch.cuda.current_stream()
+        self.ids_host = [torch.empty(batch, shape.k, dtype=torch.int32).pin_memory() for _ in range(layers)]
+
+    def step(self, x, forced_ids=None):
+        """One decode step of the batch x (bf16 [batch][d]) through all layers.
+        forced_ids: int32 [layers][batch][k] on the device, or None (the
+        routers decide).  Returns (y, per-layer [hits, misses, bytes, waves])."""
+        sh, stats = self.shape, []
+        for l, layer in enumerate(self.layers):
+            v = layer.views(self.batch)
+            moeq.moe_route_topk(x, layer.w_router, layer.bias, sh.k,
+                                forced_idx=None if forced_ids is None else forced_ids[l].contiguous(),
+                                topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"])
+            moeq.moe_permute(v["topk_idx"], sh.E, x=x, out=v, status=v["status"])
+            # the one device -> host crossing per layer: the routed ids
+            self.ids_host[l].copy_(v["topk_idx"], non_blocking=True)
+            self.compute.synchronize()
+            n_waves, st = self.caches[l].stage(self.ids_host[l].reshape(-1), self.copy, self.compute)
+            self.caches[l].ffn(v["x_perm"], v["offsets"], self.batch, sh.d, sh.F, sh.group, layer.layout,
+                               v["workspace"], v["y_perm"], v["status"], self.copy, self.compute)
+            y = torch.empty_like(x)
+            moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], residual=x, y=y)
+            stats.append(st + [n_waves])
+            x = y
+        return x, stats
+
+    def close(self):
+        for c in self.caches:
+            c.close()
+        self.caches = []

@@ -18,6 +18,7 @@ from quantized_moe_expert_histogram_b200 import build
 from quantized_moe_expert_histogram_b200 import inputs as I
 from quantized_moe_expert_histogram_b200 import moeq
 from quantized_moe_expert_histogram_b200.layer import QuantMoELayer
+from quantized_moe_expert_histogram_b200.offload import OffloadStack
 
 from gpu_helpers import within_tol
 
@@ -146,3 +147,25 @@ def test_slot_cache_rejects_bad_arguments():
     with pytest.raises(moeq.MoeError):
         st.caches[0].stage(torch.tensor([0, 99], dtype=torch.int32), st.copy, st.compute)
     st.close()
+
+
+def test_offload_stack_equals_resident():
+    """The packaged offload driver (experts only in pinned host memory, the
+    device copies of the blobs dropped) gives the resident path's outputs bit
+    for bit, layer after layer."""
+    shape = I.custom_shape(d=256, E=16, k=4, F=256, group=64)
+    ref = Stack(shape, layers=3, slots=4, batch=8, seed=5)
+    off = OffloadStack(shape, layers=3, slots=4, batch=8, seed=5)
+    trace = I.make_slot_trace(shape.E, shape.k, 3, steps=3, batch=8, seed=6).cuda()
+    xs_all = I.make_slot_x(shape.d, 3, 8, seed=6, device="cuda")
+    for s in range(3):
+        _, ys_r, _ = ref.step(xs_all[s], trace[s], offload=False)
+        y_o, stats = off.step(xs_all[s], trace[s])
+        torch.cuda.synchronize()
+        assert torch.equal(y_o, ys_r[-1]), f"step {s}"
+        for l in range(3):
+            hits, misses, nbytes, nw = stats[l]
+            assert hits + misses == len(set(trace[s, l].reshape(-1).tolist()))
+            assert nbytes == misses * off.blob_bytes
+    ref.close()
+    off.close()
