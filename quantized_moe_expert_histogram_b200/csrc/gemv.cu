@@ -141,7 +141,7 @@ __device__ __forceinline__ uint4 load_codes(const GemvParams& P, const uint8_t* 
 
 // RW output rows per warp; NM matrices (2 = gate+up, 1 = down).
 template <int MAXR, int NM, int RW, bool PLANES>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32, MAXR <= 2 ? 3 : 1) k_gemv(const GemvParams P) {
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, MAXR == 1 ? 2 : (MAXR == 2 ? 3 : 1)) k_gemv(const GemvParams P) {
   constexpr int ROWS = NM * RW;  // weight rows per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // gate/up: wait for the earlier kernels, then let the down pass launch;
@@ -272,7 +272,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, MAXR <= 2 ? 3 : 1) k_gemv
 
 template <int MAXR, bool PLANES>
 moe_status_t run_pair(GemvParams gu, GemvParams dn, int max_bins, cudaStream_t s) {
-  constexpr int RW_GU = 2, RW_DN = 4;
+  // one token per bin: twice the rows per warp, so that the grid (8 warps
+  // per block) fits the resident blocks of one wave
+  constexpr int RW_GU = MAXR == 1 ? 4 : 2, RW_DN = MAXR == 1 ? 8 : 4;
   dim3 g1(ceil_div(gu.N, kWarpsPerBlock * RW_GU), max_bins);
   moe_status_t st = cuda_check(launch_pdl(true, k_gemv<MAXR, 2, RW_GU, PLANES>, g1, dim3(kWarpsPerBlock * 32), 0, s, gu),
                                "ffn gemv gate/up launch");
