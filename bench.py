@@ -43,6 +43,8 @@ def parse():
     p.add_argument("--sweep", default="1,16,256", help="extra token counts timed for context ('' = none)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=0)
+    p.add_argument("--workloads", default="mixtral:8192,mixtral:1,nested:2048,nested:1,tiny:64",
+                   help="other configured workloads reported for context (name:tokens,...; '' = none)")
     p.add_argument("--offload-steps", type=int, default=24,
                    help="decode steps of the offload (slot-cache) workload reported under 'offload' (0 = skip)")
     p.add_argument("--profile", action="store_true",
@@ -324,6 +326,28 @@ def time_e2e(layers, steps, stream):
     return start.elapsed_time(end), h2d, T * d * 2
 
 
+def measure_workload(name, T, R, peaks, stream, reps=8):
+    """Step time and FFN roofline fraction of another configured workload
+    (CUDA graphs over R rotated instances, as for the default workload)."""
+    import torch
+    from quantized_moe_expert_histogram_b200 import inputs as I
+    shape = I.SHAPES[name]
+    ls = make_instances(shape, T, R, seed=31, device="cuda")
+    ga, gf = capture(ls, stream, "all"), capture(ls, stream, "ffn")
+    tot = time_graph(ga, reps, 2, stream) / (reps * R)
+    fm = time_graph(gf, reps, 1, stream) / (reps * R)
+    b, fl = algorithmic(shape, T, ls[-1][0], ls[0][2] is not None)
+    tc_bound = fl / (peaks["tc"] * 1e12) > b / (peaks["hbm"] * 1e9)
+    out = {"workload": f"{name}: d={shape.d} E={shape.E} top-{shape.k} d_ff={shape.F} "
+                       f"{'nested 2/3/4-bit planes' if shape.layout == 'planes' else 'INT4'} g{shape.group}",
+           "tokens": T, "tokens_per_s": T / (tot / 1e3), "ms_per_step": tot, "ffn_ms": fm,
+           "ffn_bound": "tensor" if tc_bound else "hbm",
+           "ffn_frac": (fl / (fm / 1e3) / 1e12 / peaks["tc"]) if tc_bound else (b / (fm / 1e3) / 1e9 / peaks["hbm"])}
+    del ls, ga, gf
+    torch.cuda.empty_cache()
+    return out
+
+
 def h2d_peak_gbs(nbytes=256 << 20, reps=5):
     """Pinned host -> device copy bandwidth (one large cudaMemcpyAsync)."""
     import torch
@@ -341,7 +365,7 @@ def h2d_peak_gbs(nbytes=256 << 20, reps=5):
     return nbytes * reps / (a.elapsed_time(b) / 1e3) / 1e9
 
 
-def run_offload(steps, layers=16, slots=16, batch=8, seed=0):
+def run_offload(steps, layers=16, slots=16, batch=8, seed=0, prefetch=False):
     """The offload workload: stacked OLMoE-shaped layers with experts in pinned
     host memory and a slot cache per layer, decode steps at a fixed batch on a
     Zipf + successor-correlated routing trace.  Wall time around whole steps
@@ -350,7 +374,7 @@ def run_offload(steps, layers=16, slots=16, batch=8, seed=0):
     from quantized_moe_expert_histogram_b200 import inputs as I
     from quantized_moe_expert_histogram_b200.offload import OffloadStack
     shape = I.SHAPES["olmoe"]
-    stack = OffloadStack(shape, layers, slots, batch, seed=seed)
+    stack = OffloadStack(shape, layers, slots, batch, seed=seed, prefetch=prefetch)
     warm = 2
     trace = I.make_slot_trace(shape.E, shape.k, layers, steps + warm, batch, seed=seed + 1).cuda()
     xs = I.make_slot_x(shape.d, steps + warm, batch, seed=seed + 1, device="cuda")
@@ -373,6 +397,7 @@ def run_offload(steps, layers=16, slots=16, batch=8, seed=0):
             "steps": steps, "tokens_per_s": batch * steps / wall, "ms_per_step": wall / steps * 1e3,
             "h2d_bytes_per_step": nbytes / steps, "h2d_gbs": h2d, "h2d_peak_gbs": peak,
             "h2d_frac": h2d / peak, "hit_rate": hits / max(1, hits + misses),
+            "prefetch": prefetch, "prefetch_copies_per_step": stack.prefetched / (steps + warm),
             "timing": "host wall clock around whole steps (one routed-id sync per layer)"}
 
 
@@ -517,11 +542,18 @@ def main():
         del ls, ga, gf
         torch.cuda.empty_cache()
 
+    workloads = []
+    if args.workloads:
+        for item in args.workloads.split(","):
+            name, tok = item.split(":")
+            workloads.append(measure_workload(name, int(tok), 2, peaks, stream))
+
     offload = None
     if world == 1 and args.offload_steps > 0:
         del layers
         torch.cuda.empty_cache()
         offload = run_offload(args.offload_steps)
+        offload["with_prefetch"] = run_offload(args.offload_steps, prefetch=True)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -539,7 +571,7 @@ def main():
                        "l2": f"{args.instances} layer instances rotated ({shape.E} experts x "
                              f"{moeq.moe_blob_bytes(shape.d, shape.F, shape.group, 0)} B each), inputs > L2"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * steps,
-            "clocks": clk, "sweep": sweep, "offload": offload}
+            "clocks": clk, "sweep": sweep, "workloads": workloads, "offload": offload}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

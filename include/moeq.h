@@ -219,6 +219,17 @@ MOE_API moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offse
                                 size_t workspace_bytes, void* y_perm, int32_t* status,
                                 moe_stream_t stream);
 
+/* moe_static_bits -- per-expert static bit widths ([EdgeMoE] expert-wise
+ * bit-width adaptation, the fixed-width case of [D2MoE] nested weights):
+ *   bits[t][j] = width_of[topk_idx[t][j]]
+ *   topk_idx int32 [T][k]; width_of uint8 [E] (device), each in {2, 3, 4};
+ *   bits uint8 [T][k] (device), the input moe_permute takes for the (expert,
+ *   width) bins of the nested-plane layout.
+ * Ids outside [0, E) or widths outside {2, 3, 4} are clamped and flag
+ * MOE_DEV_BAD_INDEX in `status` (may be NULL). */
+MOE_API moe_status_t moe_static_bits(const int32_t* topk_idx, const uint8_t* width_of, int T, int k, int E,
+                                     uint8_t* bits, int32_t* status, moe_stream_t stream);
+
 /* moe_unpermute_combine -- weighted combine ([ExactMoE]: every chosen
  * expert's output is used as the router weighted it).
  *   y[t] = bf16( residual[t] + sum_{j<k} topk_w[t][j] * y_perm[inv_perm[t*k+j]] )
@@ -264,6 +275,36 @@ MOE_API moe_status_t moe_slot_ffn(moe_slot_cache* cache, const void* x_perm, con
                           int total_rows, int T, int d, int F, int group, int layout,
                           void* workspace, size_t workspace_bytes, void* y_perm,
                           int32_t* status, moe_stream_t copy_stream, moe_stream_t compute_stream);
+
+/* Stage experts ahead of their layer-step ([EdgeMoE] expert preloading;
+ * [D2MoE] load the next experts while the current ones compute): copies up
+ * to `max_copies` of the listed experts that are not resident into the
+ * least recently used slots, in list order, on copy_stream.  Each copy waits
+ * for the compute that last read its slot; the next moe_slot_ffn of this
+ * cache waits for these copies, and the next moe_slot_stage counts them as
+ * hits.  Use the copy stream of this cache's moe_slot_stage calls: a later
+ * stage may reuse a prefetched slot, and stream order keeps the two copies
+ * apart.  n_copied (may be NULL) receives the number of copies issued.
+ * Prefetching changes only where experts are when they are needed, never
+ * the result. */
+MOE_API moe_status_t moe_slot_prefetch(moe_slot_cache* cache, const int32_t* ids_host, int n_ids, int max_copies,
+                                       moe_stream_t copy_stream, int32_t* n_copied);
+
+/* Next-layer expert predictor (host-only): counts of (expert at layer l-1,
+ * expert at layer l) pairs at the same token and choice position, learned
+ * online with moe_predictor_observe; moe_predictor_predict scores experts
+ * of `layer` from the routed ids of layer-1 (sum of the conditional
+ * frequencies: the expected number of assignments to each expert) and
+ * writes up to max_out ids, best first (ties: lower id), only experts whose
+ * score is nonzero and at least min_score.  ids are host int32 [T][k]. */
+typedef struct moe_route_predictor moe_route_predictor;
+MOE_API moe_status_t moe_predictor_create(int layers, int E, moe_route_predictor** out);
+MOE_API void moe_predictor_destroy(moe_route_predictor* p);
+MOE_API moe_status_t moe_predictor_observe(moe_route_predictor* p, int layer, const int32_t* prev_ids,
+                                           const int32_t* cur_ids, int T, int k);
+MOE_API moe_status_t moe_predictor_predict(const moe_route_predictor* p, int layer, const int32_t* prev_ids,
+                                           int T, int k, int max_out, double min_score, int32_t* out_ids,
+                                           int32_t* n_out);
 
 /* Free the cache's host bookkeeping, events and device table (not the
  * caller's pool or host blobs).  Synchronises the events it owns. */

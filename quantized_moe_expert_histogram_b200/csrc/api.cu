@@ -248,6 +248,24 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   return use_tc ? launch_ffn_tc(a, S(stream)) : launch_ffn_gemv(a, S(stream));
 }
 
+moe_status_t moe_static_bits(const int32_t* topk_idx, const uint8_t* width_of, int T, int k, int E,
+                             uint8_t* bits, int32_t* status, moe_stream_t stream) {
+  if (T < 0 || k <= 0 || E <= 0) {
+    set_error("moe_static_bits: bad sizes T=%d k=%d E=%d", T, k, E);
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (static_cast<long>(T) * k > (1L << 24)) {
+    set_error("moe_static_bits: T*k exceeds 2^24");
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (T == 0) return MOE_OK;
+  if (!topk_idx || !width_of || !bits) {
+    set_error("moe_static_bits: null pointer");
+    return MOE_ERR_INVALID_ARG;
+  }
+  return launch_static_bits(topk_idx, width_of, T * k, E, bits, status, S(stream));
+}
+
 moe_status_t moe_unpermute_combine(const void* y_perm, const int32_t* inv_perm,
                                    const float* topk_w, const void* residual, int T, int k, int d,
                                    void* y, moe_stream_t stream) {

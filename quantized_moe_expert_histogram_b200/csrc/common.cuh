@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <algorithm>
 #include <utility>
 #include <stdint.h>
 
@@ -92,6 +93,8 @@ struct FfnArgs {
   int32_t* status;
 };
 moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);
+moe_status_t launch_static_bits(const int32_t* idx, const uint8_t* width_of, int n, int E, uint8_t* bits,
+                                int32_t* status, cudaStream_t s);
 moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s);
 bool tc_supported(const FfnArgs& a);
 

@@ -7,9 +7,10 @@
 //                   found with __match_any_sync and the lowest of them adds
 //                   the group size to the warp's shared histogram; the CTA
 //                   histogram (warps summed in order) goes to hist[bin][c].
-//   k_perm_scan     one CTA: thread b turns row b of hist into per-CTA start
-//                   positions inside bin b and the bin total; a block scan
-//                   of the totals gives offsets, added to every start.
+//   k_perm_scan     one CTA: a warp per bin scans its row of hist into
+//                   per-CTA start positions inside the bin and the bin
+//                   total; a block scan of the totals gives offsets, which
+//                   the warps then add to every start.
 //   k_perm_scatter  CTA c recounts its warps, so that warp w starts at the
 //                   CTA's start plus the counts of warps 0..w-1; a lane's
 //                   position is its warp's cursor plus the number of lower
@@ -96,18 +97,34 @@ __global__ void __launch_bounds__(1024) k_perm_scan(int32_t* __restrict__ hist, 
                                                     int32_t* __restrict__ offsets) {
   pdl_wait();
   pdl_trigger();
+  __shared__ int32_t total_s[kMaxBins];
   __shared__ int32_t scan_buf[32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int total = 0;
-  if (tid < nbins) {
-    int32_t* row = hist + static_cast<size_t>(tid) * ctas;
-    for (int c = 0; c < ctas; ++c) {
-      const int v = row[c];
-      row[c] = total;
-      total += v;
+  // 1. a warp per bin: exclusive scan of the bin's per-CTA counts (32 CTAs
+  //    per step, shuffle scan, running carry), and the bin total
+  for (int bin = warp; bin < nbins; bin += 32) {
+    int32_t* row = hist + static_cast<size_t>(bin) * ctas;
+    int carry = 0;
+    for (int c0 = 0; c0 < ctas; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < ctas ? row[c] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (c < ctas) row[c] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    counts[tid] = total;
+    if (lane == 0) {
+      total_s[bin] = carry;
+      counts[bin] = carry;
+    }
   }
+  __syncthreads();
+  // 2. block scan of the bin totals (thread = bin) -> offsets
+  const int total = tid < nbins ? total_s[tid] : 0;
   int incl = total;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -129,10 +146,16 @@ __global__ void __launch_bounds__(1024) k_perm_scan(int32_t* __restrict__ hist, 
   const int excl = incl - total + (warp > 0 ? scan_buf[warp - 1] : 0);
   if (tid < nbins) {
     offsets[tid] = excl;
-    int32_t* row = hist + static_cast<size_t>(tid) * ctas;
-    for (int c = 0; c < ctas; ++c) row[c] += excl;
+    total_s[tid] = excl;
   }
   if (tid == 0) offsets[nbins] = n;
+  __syncthreads();
+  // 3. a warp per bin: add the bin's offset to its per-CTA starts
+  for (int bin = warp; bin < nbins; bin += 32) {
+    int32_t* row = hist + static_cast<size_t>(bin) * ctas;
+    const int off = total_s[bin];
+    for (int c = lane; c < ctas; c += 32) row[c] += off;
+  }
 }
 
 // Scatter of this CTA's assignments once hist_s[w][b] holds the first

@@ -150,30 +150,37 @@ __global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __
     if (c + 1 < nch) fetch(kbeg + (c + 1) * kDC);
     const float* xb = xs + b * G::XS + ty * kMT * G::XP;
     const float* wb = wsm + b * G::WS + tx * 4;
-    float cs[kMT][G::ME];
+    // chunk sums, two experts per packed fp32 FMA (each lane of the pair is
+    // an ordinary round-to-nearest FMA, so the error bound is unchanged)
+    float2 cs[kMT][G::ME / 2];
 #pragma unroll
     for (int i = 0; i < kMT; ++i)
 #pragma unroll
-      for (int j = 0; j < G::ME; ++j) cs[i][j] = 0.f;
+      for (int j = 0; j < G::ME / 2; ++j) cs[i][j] = make_float2(0.f, 0.f);
 #pragma unroll 8
     for (int kk = 0; kk < kDC; ++kk) {
-      float xa[kMT], wv[G::ME];
-#pragma unroll
-      for (int i = 0; i < kMT; ++i) xa[i] = xb[i * G::XP + kk];
+      float2 wv[G::ME / 2];
 #pragma unroll
       for (int j = 0; j < G::ME; j += 4) {  // experts tx*4 + (0..3) [+ EC/2]
         const float4 w4 = *reinterpret_cast<const float4*>(wb + kk * EC + (j / 4) * (EC / 2));
-        wv[j] = w4.x; wv[j + 1] = w4.y; wv[j + 2] = w4.z; wv[j + 3] = w4.w;
+        wv[j / 2] = make_float2(w4.x, w4.y);
+        wv[j / 2 + 1] = make_float2(w4.z, w4.w);
       }
 #pragma unroll
-      for (int i = 0; i < kMT; ++i)
+      for (int i = 0; i < kMT; ++i) {
+        const float xv = xb[i * G::XP + kk];
+        const float2 x2 = make_float2(xv, xv);
 #pragma unroll
-        for (int j = 0; j < G::ME; ++j) cs[i][j] = fmaf(xa[i], wv[j], cs[i][j]);
+        for (int j = 0; j < G::ME / 2; ++j) cs[i][j] = __ffma2_rn(x2, wv[j], cs[i][j]);
+      }
     }
 #pragma unroll
     for (int i = 0; i < kMT; ++i)
 #pragma unroll
-      for (int j = 0; j < G::ME; ++j) acc[i][j] += cs[i][j];
+      for (int j = 0; j < G::ME / 2; ++j) {
+        acc[i][2 * j] += cs[i][j].x;
+        acc[i][2 * j + 1] += cs[i][j].y;
+      }
     if (c + 1 < nch) stash(b ^ 1);
     __syncthreads();
   }
@@ -465,7 +472,7 @@ int route_splits(int T, int d, int E) {
   const int chunks = d / kDC;
   const int target = ceil_div(4 * 148, tiles);  // about four CTAs per SM
   int s = 1;
-  while (s * 2 <= target && chunks % (s * 2) == 0 && s * 2 <= 64) s *= 2;
+  while (s * 2 <= target && chunks % (s * 2) == 0 && s * 2 <= 16) s *= 2;
   return s;
 }
 

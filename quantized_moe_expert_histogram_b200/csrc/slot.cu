@@ -48,6 +48,8 @@ struct moe_slot_cache {
   std::vector<char> slot_free_valid;
   std::vector<cudaEvent_t> copy_done;  // per wave
   std::vector<char> copy_pending;      // per wave: wave has copies to wait for
+  cudaEvent_t prefetch_done = nullptr;  // after the last moe_slot_prefetch copies
+  bool prefetch_pending = false;        // the next moe_slot_ffn waits for them
   cudaEvent_t tables_done = nullptr;
   bool tables_done_valid = false;
   int32_t* d_tables = nullptr;  // device [max_waves][E]
@@ -153,6 +155,8 @@ moe_status_t moe_slot_cache_create(int E, int slots, size_t blob_bytes, const vo
   if (st == MOE_OK)
     st = cuda_check(cudaEventCreateWithFlags(&c->tables_done, cudaEventDisableTiming), "event");
   if (st == MOE_OK)
+    st = cuda_check(cudaEventCreateWithFlags(&c->prefetch_done, cudaEventDisableTiming), "event");
+  if (st == MOE_OK)
     st = cuda_check(cudaMalloc(&c->d_tables, sizeof(int32_t) * c->max_waves * E), "table alloc");
   if (st == MOE_OK)
     st = cuda_check(cudaHostAlloc(&c->h_tables, sizeof(int32_t) * c->max_waves * E,
@@ -181,6 +185,10 @@ void moe_slot_cache_destroy(moe_slot_cache* c) {
   if (c->tables_done) {
     cudaEventSynchronize(c->tables_done);
     cudaEventDestroy(c->tables_done);
+  }
+  if (c->prefetch_done) {
+    cudaEventSynchronize(c->prefetch_done);
+    cudaEventDestroy(c->prefetch_done);
   }
   if (c->d_tables) cudaFree(c->d_tables);
   if (c->h_tables) cudaFreeHost(c->h_tables);
@@ -304,6 +312,61 @@ moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_id
   return MOE_OK;
 }
 
+moe_status_t moe_slot_prefetch(moe_slot_cache* c, const int32_t* ids_host, int n_ids, int max_copies,
+                               moe_stream_t copy_stream, int32_t* n_copied) {
+  if (!c || n_ids < 0 || max_copies < 0 || (n_ids > 0 && !ids_host)) {
+    set_error("moe_slot_prefetch: bad arguments");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (n_copied) *n_copied = 0;
+  // Victims: least recently used slots, never one filled by this call; each
+  // copy waits for the compute that last read its slot (a step of this layer
+  // whose FFN may still run).
+  std::vector<char> pinned(c->S, 0);
+  int copied = 0;
+  for (int i = 0; i < n_ids && copied < max_copies; ++i) {
+    const int e = ids_host[i];
+    if (e < 0 || e >= c->E) {
+      set_error("moe_slot_prefetch: expert id %d out of range [0,%d)", e, c->E);
+      return MOE_ERR_INVALID_ARG;
+    }
+    if (c->slot_of[e] >= 0) continue;
+    int best = -1;
+    for (int cand = 0; cand < c->S; ++cand) {
+      if (pinned[cand]) continue;
+      if (best < 0 || c->last_use[cand] < c->last_use[best]) best = cand;
+    }
+    if (best < 0) break;
+    if (take_fault(2)) {
+      set_error("moe_slot_prefetch: injected copy failure (expert %d)", e);
+      return MOE_ERR_FAULT_INJECTED;
+    }
+    if (c->slot_free_valid[best]) {
+      moe_status_t st = cuda_check(cudaStreamWaitEvent(S(copy_stream), c->slot_free[best], 0), "slot wait free");
+      if (st != MOE_OK) return st;
+    }
+    moe_status_t st = cuda_check(
+        cudaMemcpyAsync(c->pool + static_cast<size_t>(best) * c->blob_bytes,
+                        c->host + static_cast<size_t>(e) * c->blob_bytes, c->blob_bytes, cudaMemcpyHostToDevice,
+                        S(copy_stream)),
+        "slot prefetch H2D copy");
+    if (st != MOE_OK) return st;
+    if (c->expert_in[best] >= 0) c->slot_of[c->expert_in[best]] = -1;
+    c->expert_in[best] = e;
+    c->slot_of[e] = best;
+    c->last_use[best] = ++c->clock;
+    pinned[best] = 1;
+    ++copied;
+  }
+  if (copied) {
+    moe_status_t st = cuda_check(cudaEventRecord(c->prefetch_done, S(copy_stream)), "slot prefetch event");
+    if (st != MOE_OK) return st;
+    c->prefetch_pending = true;
+  }
+  if (n_copied) *n_copied = copied;
+  return MOE_OK;
+}
+
 moe_status_t moe_slot_ffn(moe_slot_cache* c, const void* x_perm, const int32_t* offsets,
                           int total_rows, int T, int d, int F, int group, int layout,
                           void* workspace, size_t workspace_bytes, void* y_perm,
@@ -315,6 +378,12 @@ moe_status_t moe_slot_ffn(moe_slot_cache* c, const void* x_perm, const int32_t* 
   }
   const int nw = static_cast<int>(c->waves.size());
   const size_t table_bytes = sizeof(int32_t) * c->E;
+  if (c->prefetch_pending) {  // experts staged ahead by moe_slot_prefetch count as hits
+    moe_status_t st = cuda_check(cudaStreamWaitEvent(S(compute_stream), c->prefetch_done, 0),
+                                 "slot wait prefetch");
+    if (st != MOE_OK) return st;
+    c->prefetch_pending = false;
+  }
   for (int w = 0; w < nw; ++w) {
     if (c->copy_pending[w]) {
       moe_status_t st = cuda_check(cudaStreamWaitEvent(S(compute_stream), c->copy_done[w], 0),

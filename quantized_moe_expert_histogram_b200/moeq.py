@@ -39,6 +39,7 @@ _SIGS = {
     "moe_permute": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_p,
                            _c_p, _c_p, _c_sz, _c_p]),
     "moe_permute_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
+    "moe_static_bits": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]),
     "moe_ffn_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
     "moe_grouped_ffn_wq": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                   _c_p, _c_sz, _c_p, _c_p, _c_p]),
@@ -48,6 +49,11 @@ _SIGS = {
     "moe_slot_ffn": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p,
                             _c_p, _c_p, _c_p]),
     "moe_slot_cache_destroy": (None, [_c_p]),
+    "moe_slot_prefetch": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_p, _c_p]),
+    "moe_predictor_create": (_c_i, [_c_i, _c_i, ctypes.POINTER(_c_p)]),
+    "moe_predictor_destroy": (None, [_c_p]),
+    "moe_predictor_observe": (_c_i, [_c_p, _c_i, _c_p, _c_p, _c_i, _c_i]),
+    "moe_predictor_predict": (_c_i, [_c_p, _c_i, _c_p, _c_i, _c_i, _c_i, ctypes.c_double, _c_p, _c_p]),
     "moe_debug_inject_fault": (None, [_c_i, _c_i]),
     "moe_debug_force_regime": (None, [_c_i]),
     "moe_debug_set_trace": (None, [_c_p]),
@@ -189,6 +195,18 @@ def moe_permute(topk_idx, E, bits=None, x=None, out=None, status=None, workspace
     return out
 
 
+def moe_static_bits(topk_idx, width_of, E, bits=None, status=None, stream=None):
+    """bits[t][j] = width_of[topk_idx[t][j]] (uint8 [T][k])."""
+    lib = load()
+    T, k = topk_idx.shape
+    if bits is None:
+        bits = torch.empty(T, k, dtype=torch.uint8, device=topk_idx.device)
+    _check("moe_static_bits", lib.moe_static_bits(
+        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(width_of, torch.uint8, "width_of"), T, k, E,
+        _ptr(bits, torch.uint8, "bits"), _ptr(status, torch.int32, "status"), _stream(stream)))
+    return bits
+
+
 def moe_grouped_ffn_wq(x_perm, offsets, blobs, T, E, d, F, group, layout, slot_of=None,
                        workspace=None, y_perm=None, status=None, stream=None):
     lib = load()
@@ -256,9 +274,74 @@ class SlotCache:
             _ptr(y_perm, torch.float32), _ptr(status, torch.int32), copy_stream.cuda_stream,
             compute_stream.cuda_stream))
 
+    def prefetch(self, ids_host, max_copies, copy_stream):
+        """moe_slot_prefetch: stage up to max_copies of the listed experts
+        ahead of their layer-step; returns the number of copies issued."""
+        return moe_slot_prefetch(self.handle, ids_host, max_copies, copy_stream)
+
     def close(self):
         if self.handle is not None and self.handle.value:
             load().moe_slot_cache_destroy(self.handle)
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def moe_slot_prefetch(handle, ids_host, max_copies, copy_stream):
+    ids = ids_host.to(torch.int32).contiguous()
+    n = ctypes.c_int32(0)
+    _check("moe_slot_prefetch", load().moe_slot_prefetch(handle, ids.data_ptr(), ids.numel(), int(max_copies),
+                                                          copy_stream.cuda_stream, ctypes.byref(n)))
+    return n.value
+
+
+def moe_predictor_create(layers, E):
+    h = _c_p()
+    _check("moe_predictor_create", load().moe_predictor_create(layers, E, ctypes.byref(h)))
+    return h
+
+
+def moe_predictor_destroy(handle):
+    load().moe_predictor_destroy(handle)
+
+
+def moe_predictor_observe(handle, layer, prev_ids, cur_ids):
+    prev = prev_ids.to(torch.int32).contiguous().cpu()
+    cur = cur_ids.to(torch.int32).contiguous().cpu()
+    T, k = prev.shape
+    _check("moe_predictor_observe", load().moe_predictor_observe(handle, layer, prev.data_ptr(), cur.data_ptr(),
+                                                                  T, k))
+
+
+def moe_predictor_predict(handle, layer, prev_ids, max_out, min_score=0.0):
+    prev = prev_ids.to(torch.int32).contiguous().cpu()
+    T, k = prev.shape
+    out = torch.empty(max(1, max_out), dtype=torch.int32)
+    n = ctypes.c_int32(0)
+    _check("moe_predictor_predict", load().moe_predictor_predict(handle, layer, prev.data_ptr(), T, k, max_out,
+                                                                  float(min_score), out.data_ptr(), ctypes.byref(n)))
+    return out[:n.value]
+
+
+class RoutePredictor:
+    """Next-layer expert predictor (moe_predictor_*), host-side."""
+
+    def __init__(self, layers, E):
+        self.handle = moe_predictor_create(layers, E)
+
+    def observe(self, layer, prev_ids, cur_ids):
+        moe_predictor_observe(self.handle, layer, prev_ids, cur_ids)
+
+    def predict(self, layer, prev_ids, max_out, min_score=0.0):
+        return moe_predictor_predict(self.handle, layer, prev_ids, max_out, min_score)
+
+    def close(self):
+        if self.handle is not None and self.handle.value:
+            moe_predictor_destroy(self.handle)
         self.handle = None
 
     def __del__(self):

@@ -12,6 +12,13 @@ next expert while computing the current one).
 ``OffloadStack.step`` runs one decode step through all layers: route (the
 expert ids may be forced from a trace), the one device-to-host copy of the
 routed ids per layer, stage, permute, slot FFN, combine with the residual.
+With ``prefetch`` (EdgeMoE's expert preloading), once layer l's ids are
+known a host predictor (moe_predictor_*, counts of consecutive-layer expert
+pairs learned online) names layer l+1's likely experts and
+``moe_slot_prefetch`` copies the confident ones (expected to receive at
+least one assignment; at most a quarter of a cache) into layer l+1's
+slots on the copy stream, behind layer l's own copies, so that they land
+while layer l computes.
 This module only orchestrates calls of the C ABI; torch supplies device
 memory, pinned host memory and streams.
 """
@@ -25,8 +32,12 @@ from .layer import QuantMoELayer
 
 
 class OffloadStack:
-    def __init__(self, shape, layers: int, slots: int, batch: int, seed: int = 0, device="cuda"):
+    def __init__(self, shape, layers: int, slots: int, batch: int, seed: int = 0, device="cuda",
+                 prefetch: bool = False):
         self.shape, self.n_layers, self.slots, self.batch = shape, layers, slots, batch
+        self.prefetch = prefetch
+        self.predictor = moeq.RoutePredictor(layers, shape.E) if prefetch else None
+        self.prefetched = 0
         self.layers, self.host, self.pools, self.caches = [], [], [], []
         for l in range(layers):
             w = I.make_expert_weights(shape, seed=seed + 101 * l, device=device)
@@ -63,6 +74,15 @@ class OffloadStack:
             n_waves, st = self.caches[l].stage(self.ids_host[l].reshape(-1), self.copy, self.compute)
             self.caches[l].ffn(v["x_perm"], v["offsets"], self.batch, sh.d, sh.F, sh.group, layer.layout,
                                v["workspace"], v["y_perm"], v["status"], self.copy, self.compute)
+            if self.predictor is not None:
+                if l > 0:
+                    self.predictor.observe(l, self.ids_host[l - 1], self.ids_host[l])
+                if l + 1 < self.n_layers:
+                    # confident predictions only: the link is the bottleneck, and a
+                    # wrong copy costs a slot and bandwidth
+                    pred = self.predictor.predict(l + 1, self.ids_host[l], self.slots // 4, min_score=1.0)
+                    if pred.numel():
+                        self.prefetched += self.caches[l + 1].prefetch(pred, self.slots // 4, self.copy)
             y = torch.empty_like(x)
             moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], residual=x, y=y)
             stats.append(st + [n_waves])
@@ -73,3 +93,6 @@ class OffloadStack:
         for c in self.caches:
             c.close()
         self.caches = []
+        if self.predictor is not None:
+            self.predictor.close()
+            self.predictor = None

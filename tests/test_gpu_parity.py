@@ -186,6 +186,46 @@ def test_layer_ragged_shapes(d, E, k, F, g, layout, T):
     _check_layer(I.custom_shape(d=d, E=E, k=k, F=F, group=g, layout=layout), T, seed=5)
 
 
+@pytest.mark.parametrize("T", [5, 300])
+def test_static_per_expert_widths(T):
+    """Static per-expert widths: bits come from moe_static_bits (width_of[e]
+    for every assignment of expert e), the layer then runs the nested-plane
+    path; bits bit-exact, outputs against the oracle at those widths."""
+    shape = I.custom_shape(d=512, E=12, k=3, F=256, group=128, layout="planes")
+    L = layer_inputs(shape, T, seed=8)
+    layer = gpu_layer(shape, L, T)
+    width_of = torch.tensor(np.random.default_rng(8).choice([2, 3, 4], size=shape.E).astype(np.uint8))
+    x = L["x"].cuda()
+    v = layer.views(T)
+    moeq.moe_route_topk(x, layer.w_router, layer.bias, shape.k, topk_idx=v["topk_idx"], topk_w=v["topk_w"],
+                        workspace=v["route_ws"])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bits = moeq.moe_static_bits(v["topk_idx"], width_of.cuda(), shape.E, status=status)
+    torch.cuda.synchronize()
+    sel = v["topk_idx"].cpu().numpy()
+    np.testing.assert_array_equal(bits.cpu().numpy(), width_of.numpy()[sel])
+    assert int(status.item()) == 0
+    _, y = run_gpu_layer(layer, L, T, bits=bits.cpu())
+    ref, _ = oracle_layer(shape, L, bits=bits.cpu())
+    np.testing.assert_array_equal(ref["sel"], sel)
+    ok, worst = within_tol(y, ref["y"])
+    assert ok, f"worst err/tol = {worst:.3f}"
+    # each expert occupies exactly one (expert, width) bin: its own width
+    counts = layer.views(T)["counts"].cpu().numpy().reshape(shape.E, 3)
+    for e in range(shape.E):
+        assert (counts[e][np.arange(3) != width_of[e].item() - 2] == 0).all()
+
+
+def test_static_bits_flags_bad_widths():
+    idx = torch.tensor([[0, 1], [2, 7]], dtype=torch.int32, device="cuda")
+    width_of = torch.tensor([2, 5, 4, 3], dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bits = moeq.moe_static_bits(idx, width_of, 4, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & moeq.DEV_BAD_INDEX
+    assert bits.cpu().tolist() == [[2, 4], [4, 3]]  # width 5 clamped to 4; id 7 clamped to 3
+
+
 def test_layer_deterministic():
     shape = I.SHAPES["tiny"]
     L = layer_inputs(shape, 64)

@@ -149,16 +149,19 @@ def test_slot_cache_rejects_bad_arguments():
     st.close()
 
 
-def test_offload_stack_equals_resident():
+@pytest.mark.parametrize("prefetch", [False, True])
+def test_offload_stack_equals_resident(prefetch):
     """The packaged offload driver (experts only in pinned host memory, the
-    device copies of the blobs dropped) gives the resident path's outputs bit
-    for bit, layer after layer."""
+    device copies of the blobs dropped), with and without predictive
+    prefetching of the next layer's experts, gives the resident path's
+    outputs bit for bit, layer after layer."""
     shape = I.custom_shape(d=256, E=16, k=4, F=256, group=64)
-    ref = Stack(shape, layers=3, slots=4, batch=8, seed=5)
-    off = OffloadStack(shape, layers=3, slots=4, batch=8, seed=5)
-    trace = I.make_slot_trace(shape.E, shape.k, 3, steps=3, batch=8, seed=6).cuda()
-    xs_all = I.make_slot_x(shape.d, 3, 8, seed=6, device="cuda")
-    for s in range(3):
+    ref = Stack(shape, layers=3, slots=8, batch=8, seed=5)
+    off = OffloadStack(shape, layers=3, slots=8, batch=8, seed=5, prefetch=prefetch)
+    steps = 6
+    trace = I.make_slot_trace(shape.E, shape.k, 3, steps=steps, batch=8, seed=6).cuda()
+    xs_all = I.make_slot_x(shape.d, steps, 8, seed=6, device="cuda")
+    for s in range(steps):
         _, ys_r, _ = ref.step(xs_all[s], trace[s], offload=False)
         y_o, stats = off.step(xs_all[s], trace[s])
         torch.cuda.synchronize()
@@ -167,5 +170,7 @@ def test_offload_stack_equals_resident():
             hits, misses, nbytes, nw = stats[l]
             assert hits + misses == len(set(trace[s, l].reshape(-1).tolist()))
             assert nbytes == misses * off.blob_bytes
+    if prefetch:
+        assert off.prefetched > 0
     ref.close()
     off.close()
