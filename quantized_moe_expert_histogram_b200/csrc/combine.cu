@@ -37,7 +37,8 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y_per
     }
     for (int j = 0; j < k; ++j) {
       const float g = gw[static_cast<size_t>(t) * k + j];
-      const int p = inv_perm[static_cast<size_t>(t) * k + j];
+      // clamped: an inconsistent inv_perm gives wrong rows, never an out-of-range read
+      const int p = min(max(inv_perm[static_cast<size_t>(t) * k + j], 0), T * k - 1);
       const float4* row = reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(p) * d + c);
       const float4 a = row[0], b = row[1];
       acc[0] = fmaf(g, a.x, acc[0]);

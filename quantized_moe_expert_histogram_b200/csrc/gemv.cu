@@ -41,6 +41,7 @@ struct GemvParams {
   size_t d4_off[2];
   size_t sz_off[2];
   int K, N, nbins, planes_mult;  // planes_mult: 1 for INT4 bins, 3 for (e,b) bins
+  int rows;                 // activation rows: bin ranges are clamped into [0, rows]
   int group;
   __half* h_out;            // gate/up pass output [rows][N]
   float* y_out;             // down pass output [rows][N]
@@ -82,7 +83,7 @@ __device__ __forceinline__ bool find_bin(const GemvParams& P, int ordinal, int& 
     bool ok = false;
     int slot = 0;
     if (b < P.nbins) {
-      const int n = P.offsets[b + 1] - P.offsets[b];
+      const int n = min(max(P.offsets[b + 1], 0), P.rows) - min(max(P.offsets[b], 0), P.rows);
       const int e = b / P.planes_mult;
       slot = P.slot_of ? P.slot_of[e] : e;
       ok = n > 0 && slot >= 0;
@@ -97,8 +98,8 @@ __device__ __forceinline__ bool find_bin(const GemvParams& P, int ordinal, int& 
       const int src = __ffs(mm) - 1;
       bin = b0 + src;
       slot = __shfl_sync(0xffffffffu, slot, src);
-      row0 = P.offsets[bin];
-      nrows = P.offsets[bin + 1] - row0;
+      row0 = min(max(P.offsets[bin], 0), P.rows);
+      nrows = max(0, min(max(P.offsets[bin + 1], 0), P.rows) - row0);
       blob_index = slot;
       bits = P.planes_mult == 3 ? 2 + bin % 3 : 4;
       return true;
@@ -131,10 +132,22 @@ __device__ __forceinline__ uint4 load_codes(const GemvParams& P, const uint8_t* 
       r4 = ldg_nc_u32(reinterpret_cast<const uint32_t*>(blob + P.d4_off[m]) +
                       static_cast<size_t>(row) * (P.K / 32) + k0 / 32);
     uint4 out;
-    out.x = (spread2(base.x) << 2) | (spread1(r3) << 1) | spread1(r4);
-    out.y = (spread2(base.x >> 16) << 2) | (spread1(r3 >> 8) << 1) | spread1(r4 >> 8);
-    out.z = (spread2(base.y) << 2) | (spread1(r3 >> 16) << 1) | spread1(r4 >> 16);
-    out.w = (spread2(base.y >> 16) << 2) | (spread1(r3 >> 24) << 1) | spread1(r4 >> 24);
+    out.x = spread2(base.x) << 2;
+    out.y = spread2(base.x >> 16) << 2;
+    out.z = spread2(base.y) << 2;
+    out.w = spread2(base.y >> 16) << 2;
+    if (bits >= 3) {
+      out.x |= spread1(r3) << 1;
+      out.y |= spread1(r3 >> 8) << 1;
+      out.z |= spread1(r3 >> 16) << 1;
+      out.w |= spread1(r3 >> 24) << 1;
+    }
+    if (bits >= 4) {
+      out.x |= spread1(r4);
+      out.y |= spread1(r4 >> 8);
+      out.z |= spread1(r4 >> 16);
+      out.w |= spread1(r4 >> 24);
+    }
     return out;
   }
 }
@@ -204,13 +217,15 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, MAXR == 1 ? 2 : (MAXR == 
           if (t < nrows) {
             const uint4 raw = *reinterpret_cast<const uint4*>(P.act + static_cast<size_t>(row0 + t) * P.K + k0 + wi * 8);
             const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+            float2 s2 = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const float2 f = __half22float2(h2[j]);
               xv[t][2 * j] = f.x;
               xv[t][2 * j + 1] = f.y;
-              px[t] += f.x + f.y;
+              s2 = __fadd2_rn(s2, f);
             }
+            px[t] = s2.x + s2.y;
           } else {
 #pragma unroll
             for (int j = 0; j < 8; ++j) xv[t][j] = 0.0f;
@@ -226,14 +241,12 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, MAXR == 1 ? 2 : (MAXR == 
           const float zp = __uint_as_float(sz[s][r] & 0xFFFF0000u);
 #pragma unroll
           for (int t = 0; t < MAXR; ++t) {
-            float p = f0 * xv[t][0];
-            p = fmaf(f1, xv[t][1], p);
-            p = fmaf(f2, xv[t][2], p);
-            p = fmaf(f3, xv[t][3], p);
-            p = fmaf(f4, xv[t][4], p);
-            p = fmaf(f5, xv[t][5], p);
-            p = fmaf(f6, xv[t][6], p);
-            p = fmaf(f7, xv[t][7], p);
+            // even and odd elements as the two lanes of packed fp32 FMAs
+            float2 p2 = __fmul2_rn(make_float2(f0, f1), make_float2(xv[t][0], xv[t][1]));
+            p2 = __ffma2_rn(make_float2(f2, f3), make_float2(xv[t][2], xv[t][3]), p2);
+            p2 = __ffma2_rn(make_float2(f4, f5), make_float2(xv[t][4], xv[t][5]), p2);
+            p2 = __ffma2_rn(make_float2(f6, f7), make_float2(xv[t][6], xv[t][7]), p2);
+            const float p = p2.x + p2.y;
             // sum (q - z) x = 16 (p - px) - z px
             const float qx = 16.0f * (p - px[t]);
             acc[r][t] = fmaf(sc, fmaf(-zp, px[t], qx), acc[r][t]);
@@ -302,6 +315,7 @@ moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s) {
   gu.planes_mult = mult;
   gu.group = a.group;
   gu.h_out = a.h;
+  gu.rows = a.total_rows;
   for (int m = 0; m < 2; ++m) {
     gu.code_off[m] = planes ? a.lay.q2[m] : a.lay.codes[m];
     gu.d3_off[m] = a.lay.d3[m];

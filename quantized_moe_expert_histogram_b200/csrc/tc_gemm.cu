@@ -313,6 +313,7 @@ struct TcParams {
   size_t blob_bytes;
   size_t sz_off[2];
   int K, N, nbins, planes_mult, group;
+  int rows;  // activation rows (= total_rows): every bin range is clamped into [0, rows]
   __half* h_out;
   float* y_out;
   int32_t* status;
@@ -335,7 +336,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const 
   const int local = t - tile_start[lo];
   const int tb = local / MB;
   T.mb = local - tb * MB;
-  const int n = off[lo + 1] - off[lo];
+  const int n = max(0, off[lo + 1] - off[lo]);
   const int nb = (n + kNT - 1) / kNT;
   const int per = (((n + nb - 1) / nb) + 15) & ~15;
   T.row0 = off[lo] + tb * per;
@@ -458,7 +459,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
   // everything below reads what earlier kernels wrote
   pdl_wait();
   pdl_trigger();
-  for (int b = tid; b <= nbins; b += kThreads) off_s[b] = P.offsets[b];
+  // offsets come from the caller: clamp them into [0, rows] so that no
+  // inconsistent table (e.g. one built for another bin layout) can send a
+  // tile outside the activation rows; such a table is flagged
+  for (int b = tid; b <= nbins; b += kThreads) {
+    const int v = P.offsets[b];
+    const int c = min(max(v, 0), P.rows);
+    if (c != v || (b == nbins && v != P.rows)) flag_status(P.status, MOE_DEV_BAD_INDEX);
+    off_s[b] = c;
+  }
   __syncwarp();
   __syncthreads();
   if (warp == 0) {
@@ -469,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
     for (int i = 0; i < per_lane; ++i) {
       const int b = b0 + i;
       if (b < nbins) {
-        int n = off_s[b + 1] - off_s[b];
+        int n = max(0, off_s[b + 1] - off_s[b]);
         if (P.slot_of && P.slot_of[b / P.planes_mult] < 0) n = 0;
         const int tiles = ((n + kNT - 1) / kNT) * MB;
         tile_start[b] = run;
@@ -657,12 +666,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
           if (T.bits >= 4) r4 = *reinterpret_cast<const uint4*>(cb + 6144 + i * 16);
           const uint32_t d3w[4] = {r3.x, r3.y, r3.z, r3.w};
           const uint32_t d4w[4] = {r4.x, r4.y, r4.z, r4.w};
+          // word wd = elements 8wd..8wd+7; residual planes only up to the
+          // bin's width (the tile's width is uniform across the warp)
 #pragma unroll
-          for (int wd = 0; wd < 16; ++wd) {  // word wd = elements 8wd..8wd+7
-            const uint32_t base = qw[wd >> 1] >> (16 * (wd & 1));
-            const uint32_t b3 = d3w[wd >> 2] >> (8 * (wd & 3));
-            const uint32_t b4 = d4w[wd >> 2] >> (8 * (wd & 3));
-            w[wd] = (spread2(base) << 2) | (spread1(b3) << 1) | spread1(b4);
+          for (int wd = 0; wd < 16; ++wd) w[wd] = spread2(qw[wd >> 1] >> (16 * (wd & 1))) << 2;
+          if (T.bits >= 3) {
+#pragma unroll
+            for (int wd = 0; wd < 16; ++wd) w[wd] |= spread1(d3w[wd >> 2] >> (8 * (wd & 3))) << 1;
+          }
+          if (T.bits >= 4) {
+#pragma unroll
+            for (int wd = 0; wd < 16; ++wd) w[wd] |= spread1(d4w[wd >> 2] >> (8 * (wd & 3)));
           }
         }
         const uint32_t* szb = reinterpret_cast<const uint32_t*>(smem + C::OFF_SZ + (cs * 2 + m) * C::SZ_BYTES);
@@ -900,6 +914,7 @@ moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int r
   P.blobs = a.blobs;
   P.blob_bytes = a.blob_bytes;
   P.K = K;
+  P.rows = rows;
   P.N = N;
   P.planes_mult = planes ? 3 : 1;
   P.nbins = a.E * P.planes_mult;
