@@ -94,9 +94,13 @@ MOE_API const char* moe_last_error(void);
  *   PLANES: gate Q2 [F][d/16] | gate D3 [F][d/32] | gate D4 [F][d/32] |
  *           up Q2 | up D3 | up D4 | down Q2 [d][F/16] | down D3 | down D4 |
  *           gate sz | up sz | down sz
- * Code word packing: nibble i of a codes word = element 8w+i (low nibble
- * first); Q2 word bits 2i..2i+1 = element 16w+i; D3/D4 word bit i =
- * element 32w+i.  sz of an N x K matrix is N*K/g uint32 words, word =
+ * Code word packing: nibble i of an INT4 codes word = element 8w+i (low
+ * nibble first).  Planes use the plane order, n(i) = (i >> 1) + 4 (i & 1)
+ * for element i of a run of 8 (even elements in nibbles 0..3, odd ones in
+ * 4..7): Q2 word w holds element 16w + 8h + i in bits 2h + 4 n(i) .. +1;
+ * D3/D4 word w holds element 32w + 8g + i in bit g + 4 n(i), so a 4-bit
+ * code word of 8 elements is (Q2 parts) << 2 | D3 part << 1 | D4 part
+ * with one shift and mask per plane.  sz of an N x K matrix is N*K/g uint32 words, word =
  * bf16(scale) | bf16(zero) << 16, ordered [N/128][K/g][128] (row tile of
  * 128, then group, then row inside the tile).  Dequantised weight of a
  * b-bit read: w = ((code >> (4-b) << (4-b)) - zero) * scale.

@@ -114,10 +114,21 @@ def unpack_int4(words: np.ndarray, K: int) -> np.ndarray:
     return out.reshape(N, K)
 
 
+def plane_nibble(i: int) -> int:
+    """Nibble that element i (0..7) of an 8-element run occupies in the
+    planes' storage order: even elements in nibbles 0..3, odd ones in 4..7
+    (element 2j -> nibble j, element 2j+1 -> nibble 4+j)."""
+    return (i >> 1) + 4 * (i & 1)
+
+
 def split_planes(q: np.ndarray):
-    """MWQ bit planes of a 4-bit code (D2MoE, MWQ):
-    Q2 = q >> 2 (2-bit base, 16 per uint32, element 16w+i in bits 2i..2i+1),
-    D3 = (q >> 1) & 1 and D4 = q & 1 (32 per uint32, element 32w+i in bit i).
+    """MWQ bit planes of a 4-bit code (D2MoE, MWQ): base = q >> 2 (2 bits),
+    D3 = (q >> 1) & 1, D4 = q & 1, stored in the library's plane order:
+      Q2 word v (elements 16v..16v+15): element 16v + 8h + i in bits
+         2h + 4*plane_nibble(i) .. +1;
+      D3, D4 word u (elements 32u..32u+31): element 32u + 8g + i in bit
+         g + 4*plane_nibble(i).
+    (The method fixes the planes, not their bit order in a storage word.)
     """
     N, K = q.shape
     q = q.astype(np.uint32)
@@ -125,28 +136,33 @@ def split_planes(q: np.ndarray):
     d3 = ((q >> 1) & 1).reshape(N, K // 32, 32)
     d4 = (q & 1).reshape(N, K // 32, 32)
     Q2 = np.zeros((N, K // 16), dtype=np.uint32)
-    for i in range(16):
-        Q2 |= base[:, :, i] << np.uint32(2 * i)
+    for o in range(16):
+        h, i = o // 8, o % 8
+        Q2 |= base[:, :, o] << np.uint32(2 * h + 4 * plane_nibble(i))
     D3 = np.zeros((N, K // 32), dtype=np.uint32)
     D4 = np.zeros((N, K // 32), dtype=np.uint32)
-    for i in range(32):
-        D3 |= d3[:, :, i] << np.uint32(i)
-        D4 |= d4[:, :, i] << np.uint32(i)
+    for o in range(32):
+        g, i = o // 8, o % 8
+        D3 |= d3[:, :, o] << np.uint32(g + 4 * plane_nibble(i))
+        D4 |= d4[:, :, o] << np.uint32(g + 4 * plane_nibble(i))
     return Q2, D3, D4
 
 
 def join_planes(Q2, D3, D4, K: int, b: int = 4) -> np.ndarray:
     """Nested code of width b: W(2) = Q2, W(3) = Q2 + D3, W(4) = Q2 + D3 + D4,
-    written as the top b bits of the 4-bit code with the low 4-b bits zero."""
+    written as the top b bits of the 4-bit code with the low 4-b bits zero
+    (plane order as in split_planes)."""
     N = Q2.shape[0]
     base = np.empty((N, K // 16, 16), dtype=np.uint32)
-    for i in range(16):
-        base[:, :, i] = (Q2 >> np.uint32(2 * i)) & np.uint32(3)
+    for o in range(16):
+        h, i = o // 8, o % 8
+        base[:, :, o] = (Q2 >> np.uint32(2 * h + 4 * plane_nibble(i))) & np.uint32(3)
     r3 = np.empty((N, K // 32, 32), dtype=np.uint32)
     r4 = np.empty((N, K // 32, 32), dtype=np.uint32)
-    for i in range(32):
-        r3[:, :, i] = (D3 >> np.uint32(i)) & np.uint32(1)
-        r4[:, :, i] = (D4 >> np.uint32(i)) & np.uint32(1)
+    for o in range(32):
+        g, i = o // 8, o % 8
+        r3[:, :, o] = (D3 >> np.uint32(g + 4 * plane_nibble(i))) & np.uint32(1)
+        r4[:, :, o] = (D4 >> np.uint32(g + 4 * plane_nibble(i))) & np.uint32(1)
     code = base.reshape(N, K) << np.uint32(2)
     if b >= 3:
         code = code + (r3.reshape(N, K) << np.uint32(1))
@@ -178,7 +194,7 @@ def blob_layout(d: int, F: int, group: int, layout: str) -> dict:
            gate sz | up sz | down sz]
     planes: [gate Q2 F x d/16 u32 | gate D3 F x d/32 | gate D4 | up Q2 | up D3
              | up D4 | down Q2 d x F/16 | down D3 | down D4 | gate sz | up sz
-             | down sz]
+             | down sz]  (bit order inside the words: split_planes)
     sz of an N x K matrix: (scale, zero) bf16 pairs ordered
       [N/128][K/group][128], i.e. pair index ((n//128)*(K/group) + c)*128 + n%128.
     """

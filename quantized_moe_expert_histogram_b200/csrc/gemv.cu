@@ -47,23 +47,6 @@ struct GemvParams {
   float* y_out;             // down pass output [rows][N]
 };
 
-// 8 two-bit fields (bits 2i..2i+1) -> bits 4i..4i+1.
-__device__ __forceinline__ uint32_t spread2(uint32_t x) {
-  x &= 0xFFFFu;
-  x = (x | (x << 8)) & 0x00FF00FFu;
-  x = (x | (x << 4)) & 0x0F0F0F0Fu;
-  x = (x | (x << 2)) & 0x33333333u;
-  return x;
-}
-// 8 one-bit fields (bit i) -> bit 4i.
-__device__ __forceinline__ uint32_t spread1(uint32_t x) {
-  x &= 0xFFu;
-  x = (x | (x << 12)) & 0x000F000Fu;
-  x = (x | (x << 6)) & 0x03030303u;
-  x = (x | (x << 3)) & 0x11111111u;
-  return x;
-}
-
 // Nibble i of `w` as the float 1 + q/16.
 template <int I>
 __device__ __forceinline__ float nib_as_float(uint32_t w) {
@@ -109,7 +92,8 @@ __device__ __forceinline__ bool find_bin(const GemvParams& P, int ordinal, int& 
   return false;
 }
 
-// Load the 32 codes (as 4 nibble words) of row `r` at element offset k0.
+// Load the 32 codes of row `r` at element offset k0 as 4 code words (INT4:
+// nibble i = element i; planes: element 2j in nibble j, 2j+1 in nibble 4+j).
 template <bool PLANES>
 __device__ __forceinline__ uint4 load_codes(const GemvParams& P, const uint8_t* blob, int m,
                                             int row, int k0, int bits) {
@@ -131,22 +115,25 @@ __device__ __forceinline__ uint4 load_codes(const GemvParams& P, const uint8_t* 
     if (bits >= 4)
       r4 = ldg_nc_u32(reinterpret_cast<const uint32_t*>(blob + P.d4_off[m]) +
                       static_cast<size_t>(row) * (P.K / 32) + k0 / 32);
+    // plane-order code words (element 2j in nibble j, 2j+1 in nibble 4+j):
+    // word wd takes the base from bits 2(wd & 1) of each nibble of Q2 word
+    // wd >> 1 and the residuals from bit wd of the D3/D4 word
     uint4 out;
-    out.x = spread2(base.x) << 2;
-    out.y = spread2(base.x >> 16) << 2;
-    out.z = spread2(base.y) << 2;
-    out.w = spread2(base.y >> 16) << 2;
+    out.x = (base.x << 2) & 0xCCCCCCCCu;
+    out.y = base.x & 0xCCCCCCCCu;
+    out.z = (base.y << 2) & 0xCCCCCCCCu;
+    out.w = base.y & 0xCCCCCCCCu;
     if (bits >= 3) {
-      out.x |= spread1(r3) << 1;
-      out.y |= spread1(r3 >> 8) << 1;
-      out.z |= spread1(r3 >> 16) << 1;
-      out.w |= spread1(r3 >> 24) << 1;
+      out.x |= (r3 << 1) & 0x22222222u;
+      out.y |= r3 & 0x22222222u;
+      out.z |= (r3 >> 1) & 0x22222222u;
+      out.w |= (r3 >> 2) & 0x22222222u;
     }
     if (bits >= 4) {
-      out.x |= spread1(r4);
-      out.y |= spread1(r4 >> 8);
-      out.z |= spread1(r4 >> 16);
-      out.w |= spread1(r4 >> 24);
+      out.x |= r4 & 0x11111111u;
+      out.y |= (r4 >> 1) & 0x11111111u;
+      out.z |= (r4 >> 2) & 0x11111111u;
+      out.w |= (r4 >> 3) & 0x11111111u;
     }
     return out;
   }
@@ -234,9 +221,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, MAXR == 1 ? 2 : (MAXR == 
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
           const uint32_t w = wi == 0 ? codes[s][r].x : wi == 1 ? codes[s][r].y : wi == 2 ? codes[s][r].z : codes[s][r].w;
-          const float f0 = nib_as_float<0>(w), f1 = nib_as_float<1>(w), f2 = nib_as_float<2>(w),
-                      f3 = nib_as_float<3>(w), f4 = nib_as_float<4>(w), f5 = nib_as_float<5>(w),
-                      f6 = nib_as_float<6>(w), f7 = nib_as_float<7>(w);
+          // element e of the word: nibble e (INT4) or nibble (e >> 1) + 4 (e & 1) (planes)
+          const float f0 = nib_as_float<0>(w), f1 = nib_as_float<PLANES ? 4 : 1>(w),
+                      f2 = nib_as_float<PLANES ? 1 : 2>(w), f3 = nib_as_float<PLANES ? 5 : 3>(w),
+                      f4 = nib_as_float<PLANES ? 2 : 4>(w), f5 = nib_as_float<PLANES ? 6 : 5>(w),
+                      f6 = nib_as_float<PLANES ? 3 : 6>(w), f7 = nib_as_float<7>(w);
           const float sc = __uint_as_float(sz[s][r] << 16);
           const float zp = __uint_as_float(sz[s][r] & 0xFFFF0000u);
 #pragma unroll

@@ -2,10 +2,10 @@
 //
 // One warp quantises one (row, group): lane l holds elements l, l+32, ...
 // of the group, so the min/max is a warp reduction and each packed word is
-// an OR-reduction over the lanes that own its elements (nibbles) or a
-// ballot (1-bit residual planes).  The arithmetic is the asymmetric 4-bit
-// rule of moe_quant_pack, in IEEE fp32 with round-half-even, so the codes
-// are bit-identical to any other IEEE implementation of the same rule.
+// an OR-reduction over the lanes that own its elements.  The arithmetic is
+// the asymmetric 4-bit rule of moe_quant_pack, in IEEE fp32 with
+// round-half-even, so the codes are bit-identical to any other IEEE
+// implementation of the same rule.
 #include "common.cuh"
 
 namespace moeq {
@@ -73,17 +73,27 @@ __global__ void __launch_bounds__(256) k_pack(const float* __restrict__ w, int r
     uint32_t* q2 = reinterpret_cast<uint32_t*>(blob + off_q2) + static_cast<size_t>(n) * (K / 16);
     uint32_t* d3 = reinterpret_cast<uint32_t*>(blob + off_d3) + static_cast<size_t>(n) * (K / 32);
     uint32_t* d4 = reinterpret_cast<uint32_t*>(blob + off_d4) + static_cast<size_t>(n) * (K / 32);
+    // plane order: element i of a run of 8 in nibble (i >> 1) + 4 (i & 1);
+    // Q2 shifts the second run of its 16 by 2 bits, D3/D4 run g of 32 by g
+    const int nib = 4 * (((lane & 7) >> 1) + 4 * (lane & 1));
+    const int sh2 = 2 * ((lane >> 3) & 1) + nib;
+    const int sh1 = (lane >> 3) + nib;
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) {
-      uint32_t part = (q[i] >> 2) << (2 * (lane & 15));
+      uint32_t part = (q[i] >> 2) << sh2;
+      uint32_t p3 = ((q[i] >> 1) & 1u) << sh1;
+      uint32_t p4 = (q[i] & 1u) << sh1;
 #pragma unroll
       for (int o = 1; o < 16; o <<= 1) part |= __shfl_xor_sync(0xffffffffu, part, o);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        p3 |= __shfl_xor_sync(0xffffffffu, p3, o);
+        p4 |= __shfl_xor_sync(0xffffffffu, p4, o);
+      }
       if ((lane & 15) == 0) q2[(c * G + 32 * i + lane) / 16] = part;
-      const uint32_t b3 = __ballot_sync(0xffffffffu, (q[i] >> 1) & 1u);
-      const uint32_t b4 = __ballot_sync(0xffffffffu, q[i] & 1u);
       if (lane == 0) {
-        d3[(c * G + 32 * i) / 32] = b3;
-        d4[(c * G + 32 * i) / 32] = b4;
+        d3[(c * G + 32 * i) / 32] = p3;
+        d4[(c * G + 32 * i) / 32] = p4;
       }
     }
   }

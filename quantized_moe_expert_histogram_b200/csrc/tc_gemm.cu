@@ -348,20 +348,11 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const 
   return T;
 }
 
-// 8 two-bit fields -> bits 4i..4i+1 ; 8 one-bit fields -> bit 4i.
-__device__ __forceinline__ uint32_t spread2(uint32_t x) {
-  x &= 0xFFFFu;
-  x = (x | (x << 8)) & 0x00FF00FFu;
-  x = (x | (x << 4)) & 0x0F0F0F0Fu;
-  x = (x | (x << 2)) & 0x33333333u;
-  return x;
-}
-__device__ __forceinline__ uint32_t spread1(uint32_t x) {
-  x &= 0xFFu;
-  x = (x | (x << 12)) & 0x000F000Fu;
-  x = (x | (x << 6)) & 0x03030303u;
-  x = (x | (x << 3)) & 0x11111111u;
-  return x;
+// (a & m) | c in one instruction.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t c) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(m), "r"(c));
+  return r;
 }
 
 // Eight 4-bit codes (nibble i = element i) -> (code - z) * s as fp16,
@@ -379,6 +370,26 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 zoff, __half2 s2) 
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(raw) : "r"(rep), "r"(0x00F0000Fu), "r"(0x54006400u));
     __half2 h = *reinterpret_cast<const __half2*>(&raw);
     h = __hmul2(__hsub2(h, zoff), s2);
+    v[j] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(v[0], v[1], v[2], v[3]);
+}
+
+// Eight 4-bit codes in plane order (element 2j in nibble j, element 2j+1
+// in nibble 4+j) -> (code - z) * s as fp16, elements in order.  Masking
+// nibbles (j, 4+j) into 0x6400 gives the half2 (1024 + e_2j, 1024 + e_2j+1);
+// nibbles at bits 4..7 of each half, masked into 0x5400, read as (64 + e,
+// 64 + e) (their unit at exponent 64 is 1/16).  Subtracting (1024 + z) or
+// (64 + z) is exact; one multiply by s rounds each product once.
+__device__ __forceinline__ uint4 dequant8_planes(uint32_t w, __half2 z_lo, __half2 z_hi, __half2 s2) {
+  const uint32_t w8 = w >> 8;
+  const uint32_t r[4] = {and_or(w, 0x000F000Fu, 0x64006400u), and_or(w, 0x00F000F0u, 0x54005400u),
+                         and_or(w8, 0x000F000Fu, 0x64006400u), and_or(w8, 0x00F000F0u, 0x54005400u)};
+  uint32_t v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    __half2 h = *reinterpret_cast<const __half2*>(&r[j]);
+    h = __hmul2(__hsub2(h, (j & 1) ? z_hi : z_lo), s2);
     v[j] = *reinterpret_cast<uint32_t*>(&h);
   }
   return make_uint4(v[0], v[1], v[2], v[3]);
@@ -666,17 +677,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
           if (T.bits >= 4) r4 = *reinterpret_cast<const uint4*>(cb + 6144 + i * 16);
           const uint32_t d3w[4] = {r3.x, r3.y, r3.z, r3.w};
           const uint32_t d4w[4] = {r4.x, r4.y, r4.z, r4.w};
-          // word wd = elements 8wd..8wd+7; residual planes only up to the
-          // bin's width (the tile's width is uniform across the warp)
+          // word wd = elements 8wd..8wd+7 as a plane-order code word: the
+          // base sits at bits 2wd' (wd' = wd & 1) of each nibble of Q2 word
+          // wd >> 1, the residuals at bit wd & 3 of D3/D4 word wd >> 2;
+          // residual planes only up to the bin's width (uniform across the
+          // warp)
 #pragma unroll
-          for (int wd = 0; wd < 16; ++wd) w[wd] = spread2(qw[wd >> 1] >> (16 * (wd & 1))) << 2;
+          for (int wd = 0; wd < 16; ++wd) w[wd] = (qw[wd >> 1] << (2 - 2 * (wd & 1))) & 0xCCCCCCCCu;
           if (T.bits >= 3) {
 #pragma unroll
-            for (int wd = 0; wd < 16; ++wd) w[wd] |= spread1(d3w[wd >> 2] >> (8 * (wd & 3))) << 1;
+            for (int wd = 0; wd < 16; ++wd) {
+              const int sh = 1 - (wd & 3);
+              w[wd] = and_or(sh >= 0 ? d3w[wd >> 2] << sh : d3w[wd >> 2] >> -sh, 0x22222222u, w[wd]);
+            }
           }
           if (T.bits >= 4) {
 #pragma unroll
-            for (int wd = 0; wd < 16; ++wd) w[wd] |= spread1(d4w[wd >> 2] >> (8 * (wd & 3)));
+            for (int wd = 0; wd < 16; ++wd) w[wd] = and_or(d4w[wd >> 2] >> (wd & 3), 0x11111111u, w[wd]);
           }
         }
         const uint32_t* szb = reinterpret_cast<const uint32_t*>(smem + C::OFF_SZ + (cs * 2 + m) * C::SZ_BYTES);
@@ -695,11 +712,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
             const __half sc = __float2half_rn(__uint_as_float(word << 16));
             const float zf = __uint_as_float(word & 0xFFFF0000u);
             const __half2 s2 = __half2half2(sc);
-            const __half2 z2 = __halves2half2(__float2half_rn(1024.0f + zf), __float2half_rn(64.0f + zf));
+            const __half z1024 = __float2half_rn(1024.0f + zf), z64 = __float2half_rn(64.0f + zf);
             uint32_t v[32];  // column c = elements (2c, 2c + 1) of this 64-K slice of row i
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const uint4 o = dequant8(w[8 * h + j], z2, s2);
+              const uint4 o = PLANES ? dequant8_planes(w[8 * h + j], __half2half2(z1024), __half2half2(z64), s2)
+                                     : dequant8(w[8 * h + j], __halves2half2(z1024, z64), s2);
               v[4 * j] = o.x; v[4 * j + 1] = o.y; v[4 * j + 2] = o.z; v[4 * j + 3] = o.w;
             }
             tmem_st32(lane_base + C::ACOL + (s * 2 + m) * C::A_COLS, v);

@@ -98,14 +98,23 @@ def test_planes_hand_values():
     Q2, D3, D4 = O.split_planes(q + 15)
     assert Q2.tolist() == [[0xFFFFFFFF, 0xFFFFFFFF]] and D3.tolist() == [[0xFFFFFFFF]]
     assert D4.tolist() == [[0xFFFFFFFF]]
-    q[0, 0] = 1      # only the lowest residual bit of element 0
-    q[0, 1] = 4      # base field of element 1 = 1  -> bits 2..3 of Q2 word 0
-    q[0, 31] = 8     # base field of element 31 = 2 -> bits 30..31 of Q2 word 1
-    q[0, 5] = 2      # middle residual of element 5 -> bit 5 of D3
+    # plane order: in a run of 8 elements, element 2j sits in nibble j and
+    # element 2j+1 in nibble 4+j; Q2 puts the second run of its 16 at +2
+    # bits, D3/D4 put run g of their 32 at +g bits
+    q[0, 0] = 1      # D4 of element 0 (run 0, nibble 0)        -> D4 bit 0
+    q[0, 8] = 1      # D4 of element 8 (run 1, nibble 0)        -> D4 bit 1
+    q[0, 1] = 4      # base 1 of element 1 (run 0, nibble 4)    -> Q2 word 0 bits 16..17
+    q[0, 10] = 12    # base 3 of element 10 (run 1, nibble 1)   -> Q2 word 0 bits 6..7
+    q[0, 31] = 8     # base 2 of element 31 (run 1, nibble 7)   -> Q2 word 1 bits 30..31
+    q[0, 5] = 2      # D3 of element 5 (run 0, nibble 6)        -> D3 bit 24
+    q[0, 9] = 2      # D3 of element 9 (run 1, nibble 4)        -> D3 bit 17
+    q[0, 30] = 2     # D3 of element 30 (run 3, nibble 3)       -> D3 bit 15
     Q2, D3, D4 = O.split_planes(q)
-    assert Q2.tolist() == [[0x00000004, 0x80000000]]
-    assert D3.tolist() == [[0x00000020]]
-    assert D4.tolist() == [[0x00000001]]
+    assert Q2.tolist() == [[0x000100C0, 0x80000000]]
+    assert D3.tolist() == [[0x01028000]]
+    assert D4.tolist() == [[0x00000003]]
+    np.testing.assert_array_equal(O.join_planes(Q2, D3, D4, 32), q)
+    assert [O.plane_nibble(i) for i in range(8)] == [0, 4, 1, 5, 2, 6, 3, 7]
 
 
 def test_planes_nesting():
