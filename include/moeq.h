@@ -74,7 +74,7 @@ typedef enum {
 
 /* Bits OR-ed into the caller's device status word. */
 #define MOE_DEV_BAD_INDEX 1u   /* expert id or bit-width out of range (clamped) */
-#define MOE_DEV_RANGE 2u       /* activation outside fp16 range             */
+#define MOE_DEV_RANGE 2u       /* activation or expert output outside fp16 range */
 #define MOE_DEV_TIMEOUT 4u     /* a bounded on-device wait gave up          */
 
 typedef enum {
@@ -215,8 +215,10 @@ MOE_API size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int 
  *   T        token count (no bin holds more than T rows; selects the
  *            decode GEMV regime for small T)
  *   workspace >= moe_ffn_workspace_bytes() bytes of device scratch
- *   y_perm   fp32 [total_rows][d]
- * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16. */
+ *   y_perm   fp16 [total_rows][d]
+ * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16 and
+ * y_perm rounded once to fp16; an output beyond the fp16 range (|y| >
+ * 65504, or NaN) flags MOE_DEV_RANGE in `status`. */
 MOE_API moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, const void* blobs,
                                 const int32_t* slot_of, int total_rows, int T, int E, int d,
                                 int F, int group, int layout, void* workspace,
@@ -237,7 +239,7 @@ MOE_API moe_status_t moe_static_bits(const int32_t* topk_idx, const uint8_t* wid
 /* moe_unpermute_combine -- weighted combine ([ExactMoE]: every chosen
  * expert's output is used as the router weighted it).
  *   y[t] = bf16( residual[t] + sum_{j<k} topk_w[t][j] * y_perm[inv_perm[t*k+j]] )
- * summed in fp32 in ascending j; y_perm fp32 [T*k][d]; residual bf16 [T][d]
+ * summed in fp32 in ascending j; y_perm fp16 [T*k][d]; residual bf16 [T][d]
  * or NULL (0).  y bf16 [T][d]; requires d % 8 == 0 and 16-byte aligned rows. */
 MOE_API moe_status_t moe_unpermute_combine(const void* y_perm, const int32_t* inv_perm,
                                    const float* topk_w, const void* residual, int T, int k, int d,

@@ -241,7 +241,7 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   a.blob_bytes = L.bytes;
   a.lay = L;
   a.h = static_cast<__half*>(workspace);
-  a.y_perm = static_cast<float*>(y_perm);
+  a.y_perm = static_cast<__half*>(y_perm);
   a.status = status;
   const bool tc_ok = total_rows >= 16 && tc_supported(a);
   const bool use_tc = g_force_regime == 2 ? tc_ok : (g_force_regime == 1 ? false : (T > kGemvMaxT && tc_ok));

@@ -1,6 +1,6 @@
 // Weighted unpermute-combine: y[t] = bf16(res[t] + sum_j g[t][j] * y_perm[inv_perm[t*k+j]]).
-// One thread produces 8 consecutive outputs of one token (two 16-byte loads
-// per permuted fp32 row), summing in fp32 in ascending j.
+// One thread produces 8 consecutive outputs of one token (one 16-byte load
+// per permuted fp16 row), summing in fp32 in ascending j.
 #include <algorithm>
 
 #include "common.cuh"
@@ -8,7 +8,7 @@
 namespace moeq {
 namespace {
 
-__global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y_perm,
+__global__ void __launch_bounds__(256) k_combine(const __half* __restrict__ y_perm,
                                                   const int32_t* __restrict__ inv_perm,
                                                   const float* __restrict__ gw,
                                                   const __nv_bfloat16* __restrict__ residual, int T,
@@ -39,16 +39,14 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y_per
       const float g = gw[static_cast<size_t>(t) * k + j];
       // clamped: an inconsistent inv_perm gives wrong rows, never an out-of-range read
       const int p = min(max(inv_perm[static_cast<size_t>(t) * k + j], 0), T * k - 1);
-      const float4* row = reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(p) * d + c);
-      const float4 a = row[0], b = row[1];
-      acc[0] = fmaf(g, a.x, acc[0]);
-      acc[1] = fmaf(g, a.y, acc[1]);
-      acc[2] = fmaf(g, a.z, acc[2]);
-      acc[3] = fmaf(g, a.w, acc[3]);
-      acc[4] = fmaf(g, b.x, acc[4]);
-      acc[5] = fmaf(g, b.y, acc[5]);
-      acc[6] = fmaf(g, b.z, acc[6]);
-      acc[7] = fmaf(g, b.w, acc[7]);
+      const uint4 raw = *reinterpret_cast<const uint4*>(y_perm + static_cast<size_t>(p) * d + c);
+      const __half2* v2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 f = __half22float2(v2[u]);
+        acc[2 * u] = fmaf(g, f.x, acc[2 * u]);
+        acc[2 * u + 1] = fmaf(g, f.y, acc[2 * u + 1]);
+      }
     }
     uint4 o;
     __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
@@ -65,7 +63,7 @@ moe_status_t launch_combine(const void* y_perm, const int32_t* inv_perm, const f
   if (T == 0) return MOE_OK;
   const long vecs = static_cast<long>(T) * (d / 8);
   const int blocks = static_cast<int>(std::min<long>((vecs + 255) / 256, 148L * 16));
-  const cudaError_t e = launch_pdl(pdl_for(static_cast<long>(T) * k), k_combine, dim3(blocks), dim3(256), 0, s, static_cast<const float*>(y_perm), inv_perm, w,
+  const cudaError_t e = launch_pdl(pdl_for(static_cast<long>(T) * k), k_combine, dim3(blocks), dim3(256), 0, s, static_cast<const __half*>(y_perm), inv_perm, w,
                                    static_cast<const __nv_bfloat16*>(residual), T, k, d,
                                    static_cast<__nv_bfloat16*>(y));
   return cuda_check(e, "moe_unpermute_combine launch");

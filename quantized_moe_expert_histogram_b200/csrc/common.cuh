@@ -89,7 +89,7 @@ struct FfnArgs {
   size_t blob_bytes;
   BlobLayout lay;
   __half* h;          // workspace: fp16 [total_rows][F]
-  float* y_perm;  // [total_rows][d]
+  __half* y_perm;  // [total_rows][d]
   int32_t* status;
 };
 moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);

@@ -19,7 +19,7 @@
 // (offsets, slot table, weights) is complete by then.
 //
 //   gate/up pass:  h[p][f]      = silu(Wg[f] . x_p) * (Wu[f] . x_p)   (fp16)
-//   down pass:     y_perm[p][n] = Wd[n] . h_p                          (fp32)
+//   down pass:     y_perm[p][n] = Wd[n] . h_p                          (fp16)
 #include <algorithm>
 
 #include "common.cuh"
@@ -44,7 +44,8 @@ struct GemvParams {
   int rows;                 // activation rows: bin ranges are clamped into [0, rows]
   int group;
   __half* h_out;            // gate/up pass output [rows][N]
-  float* y_out;             // down pass output [rows][N]
+  __half* y_out;            // down pass output [rows][N]
+  int32_t* status;
 };
 
 // Nibble i of `w` as the float 1 + q/16.
@@ -264,7 +265,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, MAXR == 1 ? 2 : (MAXR == 
           const float g = acc[2 * j][t], u = acc[2 * j + 1][t];
           P.h_out[p * P.N + n0 + j] = __float2half_rn(silu_f(g) * u);
         } else {
-          P.y_out[p * P.N + n0 + j] = acc[j][t];
+          if (!(fabsf(acc[j][t]) <= 65504.0f)) flag_status(P.status, MOE_DEV_RANGE);
+          P.y_out[p * P.N + n0 + j] = __float2half_rn(acc[j][t]);
         }
       }
     }
@@ -305,6 +307,7 @@ moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s) {
   gu.group = a.group;
   gu.h_out = a.h;
   gu.rows = a.total_rows;
+  gu.status = a.status;
   for (int m = 0; m < 2; ++m) {
     gu.code_off[m] = planes ? a.lay.q2[m] : a.lay.codes[m];
     gu.d3_off[m] = a.lay.d3[m];

@@ -29,8 +29,8 @@
 // A stages (4 x 2 matrices x 32 columns), so there is one accumulator
 // buffer.  To keep the MMA waiting as little as possible for the
 // epilogue, the epilogue only moves the accumulators through registers
-// into a shared-memory staging buffer (h as fp16, double-buffered; y_perm
-// as fp32), releases them, and then writes the staged rows out with
+// into a shared-memory staging buffer (h and y_perm as fp16, both
+// double-buffered), releases them, and then writes the staged rows out with
 // 16-byte stores while the next tile's MMAs run.
 //
 // Warp roles (16 warps):
@@ -48,7 +48,7 @@
 //               lane i (the warp's lane quadrant is warp % 4)
 //   warps 12-15 epilogue: tcgen05.ld of its TMEM lane quadrant; gate/up
 //               pass stages h = silu(gate) * up (fp16), down pass y_perm
-//               (fp32); then the four warps copy the staged rows out
+//               (fp16); then the four warps copy the staged rows out
 // Pipelines: codes (3 / 2 stages of 128 K) -> dequant -> A in TMEM (4
 // stages of 64 K); activations B (6 / 3 stages of 64 K, first / second
 // GEMM); both -> MMA -> accumulators -> epilogue staging -> global.  Every
@@ -270,8 +270,8 @@ constexpr int kThreads = 512;  // 16 warps
 constexpr int kMaxBins = 768;
 constexpr int kNT = 128;       // largest token block (MMA N)
 
-// The epilogue stages a tile's outputs in shared memory (h fp16, 32 KB,
-// double-buffered; y fp32, 128 KB), releases the accumulators, and then
+// The epilogue stages a tile's outputs in shared memory (h fp16, 32 KB; y
+// fp16, 64 KB; both double-buffered), releases the accumulators, and then
 // writes them out with 16-byte stores while the next tile's MMAs run.
 template <bool GATEUP>
 struct Cfg {
@@ -280,8 +280,8 @@ struct Cfg {
   static constexpr int ACC = 1;       // accumulator buffers (each: 2 matrices x kNT columns)
   static constexpr int SB = GATEUP ? 6 : 3;        // B (activation) stages of 64 K
   static constexpr int CSTAGES = GATEUP ? 3 : 2;   // codes stages of 128 K
-  static constexpr int OUT_BYTES = GATEUP ? kNT * 128 * 2 : kNT * 256 * 4;  // one staging buffer
-  static constexpr int OUT_BUFS = GATEUP ? 2 : 1;
+  static constexpr int OUT_BYTES = GATEUP ? kNT * 128 * 2 : kNT * 256 * 2;  // one staging buffer
+  static constexpr int OUT_BUFS = 2;
   static constexpr int B_BYTES = kNT * 128;     // 128 token rows x 64 fp16
   static constexpr int C_BYTES = 8192;          // per matrix: 128 rows x 128 K of codes
   static constexpr int SZ_BYTES = 1024;         // per matrix: 128 rows x up to 2 groups x 4 B
@@ -315,7 +315,7 @@ struct TcParams {
   int K, N, nbins, planes_mult, group;
   int rows;  // activation rows (= total_rows): every bin range is clamped into [0, rows]
   __half* h_out;
-  float* y_out;
+  __half* y_out;
   int32_t* status;
   int* trace;  // optional progress record (null in normal use)
 };
@@ -748,20 +748,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       // 16-token chunks; the TMEM loads of chunk c + 1 are in flight while
       // chunk c is converted and written to the staging buffer
       uint8_t* stage = smem + C::OFF_OUT + (C::OUT_BUFS == 2 ? (ep_tile & 1) : 0) * C::OUT_BYTES;
+      float ymax = 0.0f;  // largest |y_perm| of this tile's rows (fp16 range check)
       auto emit = [&](const uint32_t (&a0)[16], const uint32_t (&a1)[16], int j0) {
         if (GATEUP) {
-          __half* hs = reinterpret_cast<__half*>(stage);  // [token][128 features]
+          // [token pair][128 features] words of fp16 (token 2p, token 2p + 1)
+          uint32_t* hs = reinterpret_cast<uint32_t*>(stage);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float gv = __uint_as_float(a0[j]), uv = __uint_as_float(a1[j]);
-            hs[(j0 + j) * 128 + r] = __float2half_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
+          for (int j = 0; j < 16; j += 2) {
+            const float g0 = __uint_as_float(a0[j]), u0 = __uint_as_float(a1[j]);
+            const float g1 = __uint_as_float(a0[j + 1]), u1 = __uint_as_float(a1[j + 1]);
+            const __half2 hv = __floats2half2_rn(__fdividef(g0, 1.0f + __expf(-g0)) * u0,
+                                                 __fdividef(g1, 1.0f + __expf(-g1)) * u1);
+            hs[((j0 + j) >> 1) * 128 + r] = *reinterpret_cast<const uint32_t*>(&hv);
           }
         } else {
-          float* ys = reinterpret_cast<float*>(stage);  // [token][256 outputs]
+          // [token pair][256 outputs] words of fp16 (token 2p, token 2p + 1)
+          uint32_t* ys = reinterpret_cast<uint32_t*>(stage);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            ys[(j0 + j) * 256 + r] = __uint_as_float(a0[j]);
-            ys[(j0 + j) * 256 + 128 + r] = __uint_as_float(a1[j]);
+          for (int j = 0; j < 16; j += 2) {
+            const int pr = (j0 + j) >> 1;
+            const float y00 = __uint_as_float(a0[j]), y01 = __uint_as_float(a0[j + 1]);
+            const float y10 = __uint_as_float(a1[j]), y11 = __uint_as_float(a1[j + 1]);
+            // rows past the tile's (padding up to a multiple of 16) do not count;
+            // matrix 1 is absent in a last 128-row W_down block
+            const float m0 = fmaxf(j0 + j < T.nrows ? fabsf(y00) : 0.0f, j0 + j + 1 < T.nrows ? fabsf(y01) : 0.0f);
+            const float m1v = fmaxf(j0 + j < T.nrows ? fabsf(y10) : 0.0f, j0 + j + 1 < T.nrows ? fabsf(y11) : 0.0f);
+            ymax = fmaxf(ymax, m1 ? fmaxf(m0, m1v) : m0);
+            const __half2 v0 = __floats2half2_rn(y00, y01), v1 = __floats2half2_rn(y10, y11);
+            ys[pr * 256 + r] = *reinterpret_cast<const uint32_t*>(&v0);
+            ys[pr * 256 + 128 + r] = *reinterpret_cast<const uint32_t*>(&v1);
           }
         }
       };
@@ -787,6 +802,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
           tmem_ld_wait();
         }
       }
+      // NaN compares false: flagged too
+      if (!GATEUP && !(ymax <= 65504.0f)) flag_status(P.status, MOE_DEV_RANGE);
       // accumulators read: the MMA may start the next tile
       tc_fence_before();
       __syncwarp();
@@ -799,23 +816,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       if (!ok) break;
       // 16-byte stores of the staged rows (tokens) that belong to this tile
       const int et = tid - 12 * 32;  // 0..127
+      // features / outputs 8 col .. 8 col + 7 of a token are the low (even
+      // token) or high (odd token) halves of 8 staged words
+      auto unpair = [](const uint32_t* wds, int row) {
+        const uint4 lo = reinterpret_cast<const uint4*>(wds)[0], hi = reinterpret_cast<const uint4*>(wds)[1];
+        const uint32_t sel = (row & 1) ? 0x7632u : 0x5410u;
+        return make_uint4(__byte_perm(lo.x, lo.y, sel), __byte_perm(lo.z, lo.w, sel),
+                          __byte_perm(hi.x, hi.y, sel), __byte_perm(hi.z, hi.w, sel));
+      };
       if (GATEUP) {
-        const uint4* src = reinterpret_cast<const uint4*>(stage);
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(stage);
         const size_t f0 = static_cast<size_t>(T.mb) * 128;
         for (int c = et; c < T.nrows * 16; c += 128) {
           const int row = c >> 4, col = c & 15;
-          *reinterpret_cast<uint4*>(P.h_out + static_cast<size_t>(T.row0 + row) * P.N + f0 + col * 8) = src[c];
+          *reinterpret_cast<uint4*>(P.h_out + static_cast<size_t>(T.row0 + row) * P.N + f0 + col * 8) =
+              unpair(src + (row >> 1) * 128 + col * 8, row);
         }
       } else {
-        const uint4* src = reinterpret_cast<const uint4*>(stage);
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(stage);
         const int n0 = row_base(T.mb, 0);
-        const int per_row = m1 ? 64 : 32;  // 16-byte pieces of a row's 256 (or 128) outputs
-        for (int c = et; c < T.nrows * 64; c += 128) {
-          const int row = c >> 6, col = c & 63;
+        const int per_row = m1 ? 32 : 16;  // 16-byte pieces (8 outputs) of a row's 256 (or 128)
+        for (int c = et; c < T.nrows * 32; c += 128) {
+          const int row = c >> 5, col = c & 31;
           if (col < per_row)
-            *reinterpret_cast<uint4*>(P.y_out + static_cast<size_t>(T.row0 + row) * P.N + n0 + col * 4) = src[c];
+            *reinterpret_cast<uint4*>(P.y_out + static_cast<size_t>(T.row0 + row) * P.N + n0 + col * 8) =
+                unpair(src + (row >> 1) * 256 + col * 8, row);
         }
-        // the single buffer is rewritten by the next tile: wait for every warp's copy
+      }
+      if (C::OUT_BUFS == 1) {
+        // a single buffer is rewritten by the next tile: wait for every warp's copy
         if (lane == 0) mbar_arrive(epi_bar);
         ok = warp_wait(epi_bar, ep_ph, abort_flag, P.status, trace, bar0);
         ep_ph ^= 1;

@@ -41,7 +41,7 @@ class QuantMoELayer:
             perm=torch.empty(rows, dtype=torch.int32, device=dev),
             inv_perm=torch.empty(rows, dtype=torch.int32, device=dev),
             x_perm=torch.empty(rows, d, dtype=torch.float16, device=dev),
-            y_perm=torch.empty(rows, d, dtype=torch.float32, device=dev),
+            y_perm=torch.empty(rows, d, dtype=torch.float16, device=dev),
             workspace=torch.empty(max(16, moeq.moe_ffn_workspace_bytes(rows, self.E, d, self.F, self.layout)),
                                   dtype=torch.uint8, device=dev),
             y=torch.empty(T, d, dtype=torch.bfloat16, device=dev),

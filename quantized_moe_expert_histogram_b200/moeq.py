@@ -215,11 +215,11 @@ def moe_grouped_ffn_wq(x_perm, offsets, blobs, T, E, d, F, group, layout, slot_o
         workspace = torch.empty(lib.moe_ffn_workspace_bytes(rows, E, d, F, layout), dtype=torch.uint8,
                                 device=x_perm.device)
     if y_perm is None:
-        y_perm = torch.empty(rows, d, dtype=torch.float32, device=x_perm.device)
+        y_perm = torch.empty(rows, d, dtype=torch.float16, device=x_perm.device)
     _check("moe_grouped_ffn_wq", lib.moe_grouped_ffn_wq(
         _ptr(x_perm, torch.float16, "x_perm"), _ptr(offsets, torch.int32, "offsets"), _ptr(blobs),
         _ptr(slot_of, torch.int32, "slot_of"), rows, T, E, d, F, group, layout, _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _ptr(y_perm, torch.float32, "y_perm"),
+        workspace.numel() * workspace.element_size(), _ptr(y_perm, torch.float16, "y_perm"),
         _ptr(status, torch.int32, "status"), _stream(stream)))
     return y_perm
 
@@ -231,7 +231,7 @@ def moe_unpermute_combine(y_perm, inv_perm, topk_w, residual=None, y=None, strea
     if y is None:
         y = torch.empty(T, d, dtype=torch.bfloat16, device=y_perm.device)
     _check("moe_unpermute_combine", lib.moe_unpermute_combine(
-        _ptr(y_perm, torch.float32, "y_perm"), _ptr(inv_perm, torch.int32, "inv_perm"),
+        _ptr(y_perm, torch.float16, "y_perm"), _ptr(inv_perm, torch.int32, "inv_perm"),
         _ptr(topk_w, torch.float32, "topk_w"), _ptr(residual, torch.bfloat16, "residual"), T, k, d,
         _ptr(y, torch.bfloat16, "y"), _stream(stream)))
     return y
@@ -271,7 +271,7 @@ class SlotCache:
         _check("moe_slot_ffn", lib.moe_slot_ffn(
             self.handle, _ptr(x_perm, torch.float16), _ptr(offsets, torch.int32), x_perm.shape[0], T,
             d, F, group, layout, _ptr(workspace), workspace.numel() * workspace.element_size(),
-            _ptr(y_perm, torch.float32), _ptr(status, torch.int32), copy_stream.cuda_stream,
+            _ptr(y_perm, torch.float16), _ptr(status, torch.int32), copy_stream.cuda_stream,
             compute_stream.cuda_stream))
 
     def prefetch(self, ids_host, max_copies, copy_stream):
