@@ -338,7 +338,7 @@ constexpr int kSelWarps = kSelThreads / 32;
 // bound among the picks (all others are certainly out) -- and the CTA's
 // warps recompute those logits in fp64; the token's warp then selects among
 // them on the fp64 values.
-__global__ void __launch_bounds__(kSelThreads) k_route_select(
+__global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, RouteWs ws, int splits,
     const float* __restrict__ bias, const int32_t* __restrict__ forced, int T, int d, int E, int k,
     float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w) {
