@@ -322,9 +322,10 @@ MOE_API void moe_slot_cache_destroy(moe_slot_cache* cache);
  * what = 0 clears it. */
 MOE_API void moe_debug_inject_fault(int what, int count);
 
-/* Test hook: 0 = choose the FFN kernel by T (decode GEMV for T <= 8,
- * tensor-core grouped GEMM above), 1 = always the decode GEMV, 2 = the
- * tensor-core kernel whenever the shape allows it.  Process-wide. */
+/* Test hook: 0 = choose the FFN kernel by T (decode GEMV for T = 1, the
+ * small-batch mma.sync kernel for 2 <= T <= 8, tensor-core grouped GEMM
+ * above), 1 = always the decode GEMV, 2 = the tensor-core kernel whenever
+ * the shape allows it, 3 = always the small-batch kernel.  Process-wide. */
 MOE_API void moe_debug_force_regime(int regime);
 
 /* Test hook: when non-NULL, the tensor-core FFN kernels record each warp

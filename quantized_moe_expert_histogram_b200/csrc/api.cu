@@ -67,12 +67,16 @@ inline cudaStream_t S(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Regime: the decode GEMV streams each weight row once per (at most 8)
-// rows of a bin; bins never hold more than T rows, so it is exact-fit for
-// T <= 8.  Larger T goes to the tensor-core grouped GEMM.
-constexpr int kGemvMaxT = 8;
+// Regime by T (bins never hold more than T rows): one token -> the decode
+// GEMV (CUDA-core dot products, one weight pass); up to kMmaMaxT tokens ->
+// the small-batch kernel (mma.sync dot products, cost per weight flat up to
+// 16 rows per pass); above -> the tensor-core grouped GEMM (128-row tiles).
+// Measured on the OLMoE-shaped layer: 2-8 tokens fastest on the small-batch
+// kernel, 16 and more on the tensor-core kernel.
+constexpr int kMmaMaxT = 8;
 
-// 0: pick by T; 1: always the decode GEMV; 2: tensor cores whenever possible.
+// 0: pick by T; 1: always the decode GEMV; 2: tensor cores whenever
+// possible; 3: always the small-batch kernel.
 int g_force_regime = 0;
 
 size_t workspace_for(int total_rows, int F) {
@@ -86,7 +90,7 @@ extern "C" {
 
 const char* moe_last_error(void) { return g_err; }
 
-void moe_debug_force_regime(int regime) { g_force_regime = (regime >= 0 && regime <= 2) ? regime : 0; }
+void moe_debug_force_regime(int regime) { g_force_regime = (regime >= 0 && regime <= 3) ? regime : 0; }
 
 size_t moe_blob_bytes(int d, int F, int group, int layout) {
   const BlobLayout L = blob_layout(d, F, group, layout);
@@ -244,8 +248,11 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   a.y_perm = static_cast<__half*>(y_perm);
   a.status = status;
   const bool tc_ok = total_rows >= 16 && tc_supported(a);
-  const bool use_tc = g_force_regime == 2 ? tc_ok : (g_force_regime == 1 ? false : (T > kGemvMaxT && tc_ok));
-  return use_tc ? launch_ffn_tc(a, S(stream)) : launch_ffn_gemv(a, S(stream));
+  int regime = g_force_regime;
+  if (regime == 0) regime = T <= 1 ? 1 : (T <= kMmaMaxT || !tc_ok ? 3 : 2);
+  if (regime == 2 && !tc_ok) regime = 3;
+  if (regime == 2) return launch_ffn_tc(a, S(stream));
+  return regime == 1 ? launch_ffn_gemv(a, S(stream)) : launch_ffn_gemv_mma(a, S(stream));
 }
 
 moe_status_t moe_static_bits(const int32_t* topk_idx, const uint8_t* width_of, int T, int k, int E,

@@ -93,6 +93,7 @@ struct FfnArgs {
   int32_t* status;
 };
 moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);
+moe_status_t launch_ffn_gemv_mma(const FfnArgs& a, cudaStream_t s);
 moe_status_t launch_static_bits(const int32_t* idx, const uint8_t* width_of, int n, int E, uint8_t* bits,
                                 int32_t* status, cudaStream_t s);
 moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s);

@@ -186,6 +186,17 @@ def test_layer_ragged_shapes(d, E, k, F, g, layout, T):
     _check_layer(I.custom_shape(d=d, E=E, k=k, F=F, group=g, layout=layout), T, seed=5)
 
 
+@pytest.mark.parametrize("layout", ["int4", "planes"])
+def test_small_batch_kernel_multi_pass(layout):
+    # bins of ~27 rows: the small-batch kernel runs two 16-row passes per bin
+    shape = I.custom_shape(d=384, E=3, k=2, F=256, group=64, layout=layout)
+    moeq.moe_debug_force_regime(3)
+    try:
+        _check_layer(shape, 40, seed=7)
+    finally:
+        moeq.moe_debug_force_regime(0)
+
+
 @pytest.mark.parametrize("T", [5, 300])
 def test_static_per_expert_widths(T):
     """Static per-expert widths: bits come from moe_static_bits (width_of[e]
