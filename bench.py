@@ -445,14 +445,17 @@ def run_reference(args):
     T = args.tokens
     per_step = []
     cb = None
+    n = args.cpu_sample_tokens or 32
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(shape, T, 0, args.cpu_sample_tokens or 32, budget_s=0.0)
+        cb = cpu_baseline(shape, T, 0, n, budget_s=0.0)  # one pass over the sample per step
         if i >= args.warmup:
             per_step.append(cb["value"])
     v = statistics.mean(per_step)
     cb["value"] = v
+    ms = statistics.mean(1000.0 * n / x for x in per_step)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{shape.name} MoE layer d={shape.d} E={shape.E} top-{shape.k} "
                                    f"d_ff={shape.F} INT4 g{shape.group}", "tokens": T},
