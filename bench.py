@@ -76,13 +76,20 @@ def barrier(world):
 
 
 def max_over_ranks(world, value):
+    """The largest of the ranks' values (every rank gets it)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, units_per_step, steps, max_ms):
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_step * steps / (max_ms / 1e3)
 
 
 def load_peaks():
@@ -506,7 +513,7 @@ def main():
     barrier(world)
     total_ms = max_over_ranks(world, total_ms)
     ms_per_step = total_ms / steps
-    value = world * T * steps / (total_ms / 1e3)
+    value = job_throughput(world, T, steps, total_ms)
     del g_all, g_ffn
 
     bytes_alg, flops = algorithmic(shape, T, layers[-1][0], layers[0][2] is not None)
@@ -528,7 +535,7 @@ def main():
 
     e2e_ms, h2d, d2h = time_e2e(layers, steps, stream)
     e2e_ms = max_over_ranks(world, e2e_ms)
-    e2e = {"value": world * T * steps / (e2e_ms / 1e3), "unit": "tokens/s",
+    e2e = {"value": job_throughput(world, T, steps, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     sweep = {}
