@@ -213,7 +213,8 @@ MOE_API size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int 
  *            e is blob slot_of[e]; experts with slot_of[e] < 0 are skipped
  *            (their y_perm rows are left untouched).
  *   T        token count (no bin holds more than T rows; selects the
- *            decode GEMV regime for small T)
+ *            kernel: one-token GEMV for T = 1, the small-batch mma.sync
+ *            kernel for T <= 8, the tensor-core grouped GEMM above)
  *   workspace >= moe_ffn_workspace_bytes() bytes of device scratch
  *   y_perm   fp16 [total_rows][d]
  * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16 and

@@ -75,7 +75,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // kernel, 16 and more on the tensor-core kernel.
 constexpr int kMmaMaxT = 8;
 
-// 0: pick by T; 1: always the decode GEMV; 2: tensor cores whenever
+// 0: pick by T; 1: always the one-token GEMV; 2: tensor cores whenever
 // possible; 3: always the small-batch kernel.
 int g_force_regime = 0;
 

@@ -1,9 +1,9 @@
 // Decode-regime grouped expert FFN: a warp per group of weight rows.
 //
-// Used when no bin can hold more than a few rows (T <= 8): the layer is
-// then bound by the bytes of the routed experts' codes, so each weight row
-// is streamed once with 16-byte loads and dotted against the bin's (at
-// most MAXR) activation rows, which stay in L1.  Dequantisation happens in
+// Used for one token (bins of one row; any T when the regime is forced):
+// the layer is then bound by the bytes of the routed experts' codes, so
+// each weight row is streamed once with 16-byte loads and dotted against
+// the bin's (at most MAXR) activation rows, which stay in L1.  Dequantisation happens in
 // registers: a 4-bit code q becomes the fp32 value 1 + q/16 by OR-ing it
 // into the mantissa of 1.0f, so the row dot product needs no int->float
 // conversion; per 8 elements the exact  sum (q - z) * s * x  is recovered as

@@ -360,7 +360,7 @@ def moe_last_error():
 
 
 def moe_debug_force_regime(regime):
-    """0 = by T, 1 = decode GEMV, 2 = tensor cores (test hook)."""
+    """0 = by T, 1 = one-token GEMV, 2 = tensor cores, 3 = small-batch mma.sync kernel (test hook)."""
     load().moe_debug_force_regime(regime)
 
 
