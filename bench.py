@@ -40,7 +40,7 @@ def parse():
     p.add_argument("--workload", default="olmoe")
     p.add_argument("--tokens", type=int, default=4096)
     p.add_argument("--instances", type=int, default=4, help="distinct layer instances rotated per step")
-    p.add_argument("--sweep", default="1,16,256", help="extra token counts timed for context ('' = none)")
+    p.add_argument("--sweep", default="1,8,16,256", help="extra token counts timed for context ('' = none)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=0)
     p.add_argument("--workloads", default="mixtral:8192,mixtral:1,nested:2048,nested:1,tiny:64",
