@@ -31,7 +31,8 @@ notes): the group range is widened to include 0; the zero-point is an
 integer 0..15 stored as bf16; an all-zero group has s=1, z=0; the nested
 b-bit weight keeps the top b bits of the 4-bit code with the same s and z;
 top-k ties go to the lower expert index and the k outputs are ordered by
-descending logit; nested permutation bins are ordered key = 3*e + (b-2).
+descending logit; nested permutation bins are ordered key = 3*e + (b-2);
+the bit gate is a linear score per width, ties to the narrower width.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 (closed forms, brute force on tiny inputs, invariants, textbook routines).
@@ -287,6 +288,38 @@ def route(x, w_router, bias, k):
     l = router_logits(x, w_router, bias)
     sel = topk_select(l, k)
     return sel, gates_for(l, sel), l
+
+
+# ---------------------------------------------------------------------------
+# Bit-width router (D2MoE, Design / Dual Routing: x -> Bit Gate -> b_i next
+# to x -> Expert Gate -> E_i; Token-Adaptive Bit-Width Selection)
+# ---------------------------------------------------------------------------
+
+BIT_WIDTHS = (2, 3, 4)
+
+
+def bit_gate(x: np.ndarray, w_bit: np.ndarray, bias_bit, sel: np.ndarray) -> np.ndarray:
+    """Width b[t,j] in {2, 3, 4} of the j-th selected expert e = sel[t,j] of
+    token t: the width whose score  x[t] . W_bit[e,c] (+ bias_bit[e,c])  is
+    the largest, c = 0, 1, 2 for b = 2, 3, 4, scores in fp64; equal scores
+    go to the narrower width.  W_bit fp32 [E, 3, d], bias_bit fp32 [E, 3]
+    or None.  (The page places the bit gate per token next to the expert
+    gate and ties the width to the expert's importance for the token, but
+    gives no form; a linear score per width, read like the expert gate's
+    logits, is the plain reading.)"""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_bit, dtype=np.float64)
+    b = None if bias_bit is None else np.asarray(bias_bit, dtype=np.float64)
+    T, k = sel.shape
+    out = np.empty((T, k), dtype=np.uint8)
+    for t in range(T):
+        for j in range(k):
+            e = int(sel[t, j])
+            scores = w[e] @ x[t]
+            if b is not None:
+                scores = scores + b[e]
+            out[t, j] = BIT_WIDTHS[int(np.argmax(scores))]  # first maximum: the narrower width
+    return out
 
 
 # ---------------------------------------------------------------------------
