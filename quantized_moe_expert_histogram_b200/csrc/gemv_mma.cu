@@ -176,9 +176,10 @@ __device__ __forceinline__ bool piece_src(const GemvParams& P, const uint8_t* bl
 
 // NM matrices (2 = gate+up of the same 8 features, 1 = down); RG 8-row
 // groups per matrix; NM * RG = 2 fragments (16 rows) per warp.  HI: bins
-// may hold more than 8 rows (token rows 8..15 of the MMA are used; only
-// when the regime is forced beyond its T); without it the activations of
-// stage i + 1 are loaded while stage i is computed.
+// may hold more than 8 rows (T > 8: the tensor-core kernel does not take
+// the shape, or the regime is forced), and token rows 8..15 of the MMA are
+// used; without it the activations of stage i + 1 are loaded while stage i
+// is computed.
 template <int NM, int RG, bool PLANES, bool HI, int S>
 __global__ void __launch_bounds__(kWarps * 32) k_gemv(const GemvParams P) {
   static_assert(NM * RG == 2, "two 8-row fragments per warp");
