@@ -156,9 +156,12 @@ MOE_API size_t moe_route_workspace_bytes(int T, int d, int E);
  * allocation failure or its implicit synchronisation.  The scratch lives in
  * a fixed 8 MiB device array inside the library, which every GPU that loads
  * the library holds until the process exits; the call allocates nothing.
- *   - Arguments and results are those of moe_route_topk.
- *   - Sizes whose scratch (moe_route_workspace_bytes) exceeds 8 MiB are
- *     rejected with MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - Arguments and results are those of moe_route_topk (expert ids equal
+ *     bit for bit; gates may differ in the last bits where this call sums
+ *     the logits over fewer slices of d).
+ *   - The number of d slices is lowered until the scratch fits the array;
+ *     sizes whose one-slice scratch, (T*E + T + E) fp32 words, exceeds
+ *     8 MiB are rejected with MOE_ERR_UNSUPPORTED_SHAPE.
  *   - The first call on a device resolves the array's device address for
  *     that device (cudaGetSymbolAddress, with that device current); make
  *     that first call before any stream capture.
@@ -226,6 +229,25 @@ MOE_API moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offse
                                 size_t workspace_bytes, void* y_perm, int32_t* status,
                                 moe_stream_t stream);
 
+/* moe_bit_gate -- bit-width router ([D2MoE] Dual Routing: x -> Bit Gate ->
+ * b beside x -> Expert Gate -> E; Token-Adaptive Bit-Width Selection): the
+ * width at which each selected expert runs for each token.  For the j-th
+ * selected expert e = topk_idx[t][j] of token t:
+ *   score[c]   = x[t] . w_bit[e][c] + bias_bit[e][c],   c = 0, 1, 2
+ *   bits[t][j] = 2 + the c of the largest score (equal scores -> the lower
+ *                c, i.e. the narrower width)
+ * The decision is that of the exact scores: they are evaluated in fp32 with
+ * a proven error bound, and an assignment whose winner the bound does not
+ * settle is re-evaluated in fp64, where every bf16 x fp32 product is exact.
+ *   x bf16 [T][d]; w_bit fp32 [E][3][d]; bias_bit fp32 [E][3] or NULL;
+ *   topk_idx int32 [T][k] (from moe_route_topk); bits uint8 [T][k], the
+ *   input moe_permute takes for the (expert, width) bins.
+ * Ids outside [0, E) are clamped and flag MOE_DEV_BAD_INDEX in `status`
+ * (may be NULL).  Requires d % 8 == 0 and 16-byte aligned x and w_bit. */
+MOE_API moe_status_t moe_bit_gate(const void* x, const float* w_bit, const float* bias_bit,
+                                  const int32_t* topk_idx, int T, int d, int E, int k, uint8_t* bits,
+                                  int32_t* status, moe_stream_t stream);
+
 /* moe_static_bits -- per-expert static bit widths ([EdgeMoE] expert-wise
  * bit-width adaptation, the fixed-width case of [D2MoE] nested weights):
  *   bits[t][j] = width_of[topk_idx[t][j]]
@@ -292,8 +314,11 @@ MOE_API moe_status_t moe_slot_ffn(moe_slot_cache* cache, const void* x_perm, con
  * hits.  Use the copy stream of this cache's moe_slot_stage calls: a later
  * stage may reuse a prefetched slot, and stream order keeps the two copies
  * apart.  n_copied (may be NULL) receives the number of copies issued.
- * Prefetching changes only where experts are when they are needed, never
- * the result. */
+ * Allowed order per cache: ... moe_slot_ffn -> moe_slot_prefetch ->
+ * moe_slot_stage -> moe_slot_ffn ...; a call between moe_slot_stage and
+ * its moe_slot_ffn is rejected with MOE_ERR_INVALID_ARG (it could evict an
+ * expert the staged plan relies on).  Prefetching changes only where
+ * experts are when they are needed, never the result. */
 MOE_API moe_status_t moe_slot_prefetch(moe_slot_cache* cache, const int32_t* ids_host, int n_ids, int max_copies,
                                        moe_stream_t copy_stream, int32_t* n_copied);
 

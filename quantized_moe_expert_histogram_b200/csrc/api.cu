@@ -10,6 +10,35 @@ namespace moeq {
 
 namespace {
 thread_local char g_err[512] = "no error";
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+}
+
+// Argument checks shared by the router entry points (everything except
+// the scratch, which each entry point provides its own way).
+moe_status_t route_check_args(const void* x, const float* w_router, int T, int d, int E, int k,
+                              const int32_t* topk_idx, const float* topk_w, const char* fn) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0) {
+    set_error("%s: bad sizes T=%d d=%d E=%d k=%d", fn, T, d, E, k);
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (T > 0 && (!x || !w_router || !topk_idx || !topk_w)) {
+    set_error("%s: null pointer", fn);
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (k > E || k > 16 || E > 256) {
+    set_error("%s: need k <= E, k <= 16, E <= 256 (k=%d E=%d)", fn, k, E);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (d % 32) {
+    set_error("%s: d=%d must be a multiple of 32", fn, d);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (T > 0 && (!aligned16(x) || !aligned16(w_router))) {
+    set_error("%s: x and w_router must be 16-byte aligned", fn);
+    return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
 }
 
 void set_error(const char* fmt, ...) {
@@ -64,8 +93,6 @@ using namespace moeq;
 namespace {
 
 inline cudaStream_t S(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Regime by T (bins never hold more than T rows): one token -> the decode
 // GEMV (CUDA-core dot products, one weight pass); up to kMmaMaxT tokens ->
@@ -122,33 +149,19 @@ moe_status_t moe_route_topk(const void* x, const float* w_router, const float* b
                             const int32_t* forced_idx, int T, int d, int E, int k,
                             int32_t* topk_idx, float* topk_w, void* workspace,
                             size_t workspace_bytes, moe_stream_t stream) {
-  if (T < 0 || d <= 0 || E <= 0 || k <= 0) {
-    set_error("moe_route_topk: bad sizes T=%d d=%d E=%d k=%d", T, d, E, k);
-    return MOE_ERR_INVALID_ARG;
-  }
-  if (T > 0 && (!x || !w_router || !topk_idx || !topk_w)) {
-    set_error("moe_route_topk: null pointer");
-    return MOE_ERR_INVALID_ARG;
-  }
-  if (k > E || k > 16 || E > 256) {
-    set_error("moe_route_topk: need k <= E, k <= 16, E <= 256 (k=%d E=%d)", k, E);
-    return MOE_ERR_UNSUPPORTED_SHAPE;
-  }
-  if (d % 32) {
-    set_error("moe_route_topk: d=%d must be a multiple of 32", d);
-    return MOE_ERR_UNSUPPORTED_SHAPE;
-  }
+  moe_status_t st = route_check_args(x, w_router, T, d, E, k, topk_idx, topk_w, "moe_route_topk");
+  if (st != MOE_OK) return st;
   if (T > 0 && (!workspace || workspace_bytes < route_workspace_bytes(T, d, E))) {
     set_error("moe_route_topk: workspace %zu < %zu bytes", workspace_bytes,
               route_workspace_bytes(T, d, E));
     return MOE_ERR_WORKSPACE;
   }
-  if (T > 0 && (!aligned16(x) || !aligned16(w_router) || !aligned16(workspace))) {
-    set_error("moe_route_topk: x, w_router and workspace must be 16-byte aligned");
+  if (T > 0 && !aligned16(workspace)) {
+    set_error("moe_route_topk: workspace must be 16-byte aligned");
     return MOE_ERR_INVALID_ARG;
   }
   return launch_route(x, w_router, bias, forced_idx, T, d, E, k, topk_idx, topk_w, workspace,
-                      S(stream));
+                      workspace_bytes, S(stream));
 }
 
 size_t moe_permute_workspace_bytes(int T, int E, int k, int nested) {
@@ -253,6 +266,32 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   if (regime == 2 && !tc_ok) regime = 3;
   if (regime == 2) return launch_ffn_tc(a, S(stream));
   return regime == 1 ? launch_ffn_gemv(a, S(stream)) : launch_ffn_gemv_mma(a, S(stream));
+}
+
+moe_status_t moe_bit_gate(const void* x, const float* w_bit, const float* bias_bit, const int32_t* topk_idx,
+                          int T, int d, int E, int k, uint8_t* bits, int32_t* status, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E) {
+    set_error("moe_bit_gate: bad sizes T=%d d=%d E=%d k=%d", T, d, E, k);
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (d % 8) {
+    set_error("moe_bit_gate: d=%d must be a multiple of 8", d);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (static_cast<long>(T) * k > (1L << 24)) {
+    set_error("moe_bit_gate: T*k exceeds 2^24");
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (T == 0) return MOE_OK;
+  if (!x || !w_bit || !topk_idx || !bits) {
+    set_error("moe_bit_gate: null pointer");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x) || !aligned16(w_bit)) {
+    set_error("moe_bit_gate: x and w_bit must be 16-byte aligned");
+    return MOE_ERR_INVALID_ARG;
+  }
+  return launch_bit_gate(x, w_bit, bias_bit, topk_idx, T, d, E, k, bits, status, S(stream));
 }
 
 moe_status_t moe_static_bits(const int32_t* topk_idx, const uint8_t* width_of, int T, int k, int E,

@@ -1,0 +1,126 @@
+// Bit-width router: the "bit gate" that D2MoE places beside the expert gate
+// (Design, Dual Routing; Token-Adaptive Bit-Width Selection).  For the j-th
+// selected expert e of token t it scores the three widths
+//   l[c] = x[t] . W_bit[e][c] + b_bit[e][c],   c = 0, 1, 2  (b = 2, 3, 4)
+// and picks the first maximum (equal scores -> the narrower width).
+//
+// The decision must equal the one the exact scores give.  As in the expert
+// router, the scores are evaluated in fp32 with a proven error bound and
+// only undecided assignments are re-evaluated in fp64 (every bf16 x fp32
+// product is exact there):
+//   a lane sums its d/32 products with an FMA chain, the warp adds the 32
+//   lane sums in a shuffle tree (5 levels), so |S - s| <= g(m) sum |x_i W_i|
+//   with m = (products per lane) + 5 and g(m) = m u / (1 - m u), u = 2^-24.
+//   The sum of magnitudes A is accumulated alongside (it errs by the same
+//   relative g(m), covered by the factor 1 + 2^-8), and adding the bias
+//   rounds once more:
+//     |L[c] - l[c]| <= D[c] = 2 (g(m) A[c] (1 + 2^-8) + u (|L[c]| + |b[c]|))
+//   (factor 2: margin).  The fp32 winner c* is certain when it beats every
+//   other width by more than both bounds, L[c*] - D[c*] > L[c] + D[c].
+//
+// A warp per token: x[t] is read once per selected expert (it stays in L1),
+// W_bit rows (3 x d fp32 per expert) come through L2.
+#include <cmath>
+
+#include "common.cuh"
+
+namespace moeq {
+namespace {
+
+constexpr int kWarps = 8;
+
+__global__ void __launch_bounds__(kWarps * 32) k_bit_gate(const __nv_bfloat16* __restrict__ x,
+                                                         const float* __restrict__ wb,
+                                                         const float* __restrict__ bb,
+                                                         const int32_t* __restrict__ idx, int T, int d, int E,
+                                                         int k, float gamma, uint8_t* __restrict__ bits,
+                                                         int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kWarps + warp;
+  if (t >= T) return;  // warp-uniform
+  const __nv_bfloat16* xr = x + static_cast<size_t>(t) * d;
+  for (int j = 0; j < k; ++j) {
+    int e = idx[static_cast<size_t>(t) * k + j];
+    if (e < 0 || e >= E) {
+      if (lane == 0) flag_status(status, MOE_DEV_BAD_INDEX);
+      e = e < 0 ? 0 : E - 1;
+    }
+    const float* w0 = wb + static_cast<size_t>(e) * 3 * d;
+    float s[3] = {0.f, 0.f, 0.f}, a[3] = {0.f, 0.f, 0.f};
+    for (int i = lane * 8; i < d; i += 256) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(xr + i);
+      float4 wv[3][2];
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        wv[c][0] = *reinterpret_cast<const float4*>(w0 + static_cast<size_t>(c) * d + i);
+        wv[c][1] = *reinterpret_cast<const float4*>(w0 + static_cast<size_t>(c) * d + i + 4);
+      }
+      const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        const float w[8] = {wv[c][0].x, wv[c][0].y, wv[c][0].z, wv[c][0].w,
+                            wv[c][1].x, wv[c][1].y, wv[c][1].z, wv[c][1].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(x2[q]);
+          s[c] = fmaf(f.x, w[2 * q], s[c]);
+          a[c] = fmaf(fabsf(f.x), fabsf(w[2 * q]), a[c]);
+          s[c] = fmaf(f.y, w[2 * q + 1], s[c]);
+          a[c] = fmaf(fabsf(f.y), fabsf(w[2 * q + 1]), a[c]);
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 3; ++c)
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        s[c] += __shfl_xor_sync(0xffffffffu, s[c], o);
+        a[c] += __shfl_xor_sync(0xffffffffu, a[c], o);
+      }
+    float L[3], D[3];
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      const float b = bb ? bb[static_cast<size_t>(e) * 3 + c] : 0.f;
+      L[c] = s[c] + b;
+      D[c] = 2.0f * (gamma * a[c] * (1.0f + 0.00390625f) + 5.9604645e-8f * (fabsf(L[c]) + fabsf(b))) + 1e-30f;
+    }
+    int best = 0;
+    if (L[1] > L[best]) best = 1;
+    if (L[2] > L[best]) best = 2;
+    // certain when the winner's lower bound clears every other upper bound
+    // (comparisons with NaN are false: non-finite scores go to fp64)
+    bool sure = true;
+#pragma unroll
+    for (int c = 0; c < 3; ++c)
+      if (c != best) sure = sure && (L[best] - D[best] > L[c] + D[c]);
+    if (!sure) {  // warp-uniform: every lane holds the reduced sums
+      double v[3];
+#pragma unroll
+      for (int c = 0; c < 3; ++c)
+        v[c] = dot_bf16_f32_fp64(xr, w0 + static_cast<size_t>(c) * d, d, lane) +
+               (bb ? static_cast<double>(bb[static_cast<size_t>(e) * 3 + c]) : 0.0);
+      best = 0;
+      if (v[1] > v[best]) best = 1;
+      if (v[2] > v[best]) best = 2;
+    }
+    if (lane == 0) bits[static_cast<size_t>(t) * k + j] = static_cast<uint8_t>(2 + best);
+  }
+}
+
+}  // namespace
+
+moe_status_t launch_bit_gate(const void* x, const float* w_bit, const float* bias_bit, const int32_t* idx,
+                             int T, int d, int E, int k, uint8_t* bits, int32_t* status, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const double u = std::ldexp(1.0, -24);
+  const double m = ceil_div(d, 256) * 8 + 5;
+  const float gamma = static_cast<float>(m * u / (1.0 - m * u));
+  return cuda_check(launch_pdl(pdl_for(static_cast<long>(T) * k), k_bit_gate, dim3(ceil_div(T, kWarps)),
+                               dim3(kWarps * 32), 0, s, static_cast<const __nv_bfloat16*>(x), w_bit, bias_bit,
+                               idx, T, d, E, k, gamma, bits, status),
+                    "moe_bit_gate launch");
+}
+
+}  // namespace moeq

@@ -65,13 +65,51 @@ __device__ __forceinline__ float silu_f(float v) { return v / (1.0f + __expf(-v)
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// fp64 dot product of a bf16 row and an fp32 row (d % 8 == 0) by one warp: lanes over 8-element pieces
+// of d, four pieces' loads issued before their FMAs, then a shuffle tree.
+__device__ __forceinline__ double dot_bf16_f32_fp64(const __nv_bfloat16* x, const float* w, int d, int lane) {
+  double a = 0.0;
+  for (int i0 = lane * 8; i0 < d; i0 += 4 * 256) {
+    uint4 xv[4];
+    float4 w0[4], w1[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * 256;
+      if (i < d) {
+        xv[u] = *reinterpret_cast<const uint4*>(x + i);
+        w0[u] = *reinterpret_cast<const float4*>(w + i);
+        w1[u] = *reinterpret_cast<const float4*>(w + i + 4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (i0 + u * 256 >= d) break;
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xv[u]);
+      const float wv[8] = {w0[u].x, w0[u].y, w0[u].z, w0[u].w, w1[u].x, w1[u].y, w1[u].z, w1[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(b2[j]);
+        a = fma(static_cast<double>(f.x), static_cast<double>(wv[2 * j]), a);
+        a = fma(static_cast<double>(f.y), static_cast<double>(wv[2 * j + 1]), a);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+  return a;
+}
+
+
 // Launchers (each returns MOE_OK or an error already recorded).
 moe_status_t launch_pack(const float* w_gate, const float* w_up, const float* w_down, int E, int d,
                          int F, int group, int layout, void* blobs, cudaStream_t s);
 moe_status_t launch_route(const void* x, const float* w_router, const float* bias,
                           const int32_t* forced, int T, int d, int E, int k, int32_t* idx,
-                          float* w, void* workspace, cudaStream_t s);
+                          float* w, void* workspace, size_t workspace_bytes, cudaStream_t s);
 size_t route_workspace_bytes(int T, int d, int E);
+size_t route_min_workspace_bytes(int T, int d, int E);
+moe_status_t route_check_args(const void* x, const float* w_router, int T, int d, int E, int k,
+                              const int32_t* topk_idx, const float* topk_w, const char* fn);
 moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void* x, int T, int d,
                             int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
                             int32_t* inv_perm, void* x_perm, int32_t* status, void* workspace,
@@ -94,6 +132,8 @@ struct FfnArgs {
 };
 moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);
 moe_status_t launch_ffn_gemv_mma(const FfnArgs& a, cudaStream_t s);
+moe_status_t launch_bit_gate(const void* x, const float* w_bit, const float* bias_bit, const int32_t* idx,
+                             int T, int d, int E, int k, uint8_t* bits, int32_t* status, cudaStream_t s);
 moe_status_t launch_static_bits(const int32_t* idx, const uint8_t* width_of, int n, int E, uint8_t* bits,
                                 int32_t* status, cudaStream_t s);
 moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s);

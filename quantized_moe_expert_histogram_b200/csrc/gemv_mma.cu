@@ -372,11 +372,11 @@ moe_status_t run_one(const GemvParams& p, int max_bins, cudaStream_t s, const ch
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
+  if (dev >= 64 || !attr_set[dev]) {
     const cudaError_t e = cudaFuncSetAttribute(k_gemv<NM, RG, PLANES, HI, S>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_check(e, what);
-    attr_set[dev] = true;
+    if (dev < 64) attr_set[dev] = true;
   }
   const dim3 grid(ceil_div(p.N, kWarps * 8 * RG), max_bins);
   return cuda_check(launch_pdl(true, k_gemv<NM, RG, PLANES, HI, S>, grid, dim3(kWarps * 32), smem, s, p), what);

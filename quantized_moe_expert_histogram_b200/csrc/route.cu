@@ -31,6 +31,8 @@
 // d/32 chunk sums in any order give g(32) + g(d/32)(1 + g(32)) <= g(32 + d/32).
 // The squared norms are fp32 sums too (relative error below 2^-8 for
 // d < 2^15) and the bias addition rounds once more (the u term).
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moeq {
@@ -227,40 +229,6 @@ constexpr int kPer = 8;  // E <= 256: at most 8 experts per lane (e = lane + 32 
 // True on every lane of a warp when any lane lists a contender.
 __device__ __forceinline__ bool contender_any(uint32_t c) { return __any_sync(0xffffffffu, c != 0); }
 
-// fp64 dot product x[t] . W_r[e] by one warp: lanes over 8-element pieces
-// of d, four pieces' loads issued before their FMAs, then a shuffle tree.
-__device__ __forceinline__ double dot64(const __nv_bfloat16* x, const float* w, int d, int lane) {
-  double a = 0.0;
-  for (int i0 = lane * 8; i0 < d; i0 += 4 * 256) {
-    uint4 xv[4];
-    float4 w0[4], w1[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0 + u * 256;
-      if (i < d) {
-        xv[u] = *reinterpret_cast<const uint4*>(x + i);
-        w0[u] = *reinterpret_cast<const float4*>(w + i);
-        w1[u] = *reinterpret_cast<const float4*>(w + i + 4);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (i0 + u * 256 >= d) break;
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xv[u]);
-      const float wv[8] = {w0[u].x, w0[u].y, w0[u].z, w0[u].w, w1[u].x, w1[u].y, w1[u].z, w1[u].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(b2[j]);
-        a = fma(static_cast<double>(f.x), static_cast<double>(wv[2 * j]), a);
-        a = fma(static_cast<double>(f.y), static_cast<double>(wv[2 * j + 1]), a);
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-  return a;
-}
-
 // Top k of the lane-distributed values v[m] (expert lane + 32 m; experts
 // with ok[m] false take no part), ties to the lower index; returns the picks
 // in order and the lane's taken mask.
@@ -451,7 +419,7 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
     int w = 0, r = item;
     while (r >= n_cand[w]) r -= n_cand[w++];
     const int tu = blockIdx.x * kSelWarps + w, e = cand[w][r];
-    const double v = dot64(x + static_cast<size_t>(tu) * d, wr + static_cast<size_t>(e) * d, d, lane);
+    const double v = dot_bf16_f32_fp64(x + static_cast<size_t>(tu) * d, wr + static_cast<size_t>(e) * d, d, lane);
     if (lane == 0) l64[w][e] = v + (bias ? static_cast<double>(bias[e]) : 0.0);
   }
   __syncthreads();
@@ -465,7 +433,16 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
   }
 }
 
-int route_splits(int T, int d, int E) {
+// Scratch bytes of a route with S slices of d.
+size_t route_ws_for(size_t S, int T, int E) {
+  return std::max<size_t>(256, S * (static_cast<size_t>(T) * E + T + E) * sizeof(float));
+}
+
+// Slices of d: enough CTAs for about four per SM, halved while the scratch
+// they need exceeds `cap` bytes (one slice always remains; the error bound
+// of the logits holds for any slicing, since slices are sums of 32-product
+// chunk sums).
+int route_splits(int T, int d, int E, size_t cap = static_cast<size_t>(-1)) {
   const int ec = E <= 16 ? 16 : 64;
   const int tt = ec == 64 ? Tile<64>::TT : Tile<16>::TT;
   const int tiles = ceil_div(T, tt) * ceil_div(E, ec);
@@ -473,6 +450,7 @@ int route_splits(int T, int d, int E) {
   const int target = ceil_div(4 * 148, tiles);  // about four CTAs per SM
   int s = 1;
   while (s * 2 <= target && chunks % (s * 2) == 0 && s * 2 <= 16) s *= 2;
+  while (s > 1 && route_ws_for(s, T, E) > cap) s /= 2;
   return s;
 }
 
@@ -486,12 +464,18 @@ template <int EC>
 moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d, int E, int k_route, int splits,
                            RouteWs ws, cudaStream_t s) {
   using G = Tile<EC>;
-  static bool attr_set = false;  // once per process (the first call precedes any capture)
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_route_logits<EC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(G::SMEM));
+  // the shared-memory opt-in is a per-device attribute: set once per device
+  // (the first call on a device precedes any stream capture)
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_check(e, "moe_route_topk cudaGetDevice");
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (!bit || !(attr_set.load() & bit)) {
+    e = cudaFuncSetAttribute(k_route_logits<EC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(G::SMEM));
     if (e != cudaSuccess) return cuda_check(e, "moe_route_topk smem attribute");
-    attr_set = true;
+    attr_set.fetch_or(bit);
   }
   dim3 grid(ceil_div(T, G::TT), ceil_div(E, EC), splits);
   return cuda_check(launch_pdl(pdl_for(static_cast<long>(T) * k_route), k_route_logits<EC>, grid, dim3(kLT), G::SMEM, s, x, wr, T, d, E, d / splits, ws),
@@ -502,15 +486,19 @@ moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d
 
 size_t route_workspace_bytes(int T, int d, int E) {
   if (T <= 0 || d <= 0 || E <= 0) return 256;
-  const size_t S = static_cast<size_t>(route_splits(T, d, E));
-  return std::max<size_t>(256, S * (static_cast<size_t>(T) * E + T + E) * sizeof(float));
+  return route_ws_for(static_cast<size_t>(route_splits(T, d, E)), T, E);
+}
+
+size_t route_min_workspace_bytes(int T, int d, int E) {
+  if (T <= 0 || d <= 0 || E <= 0) return 256;
+  return route_ws_for(1, T, E);
 }
 
 moe_status_t launch_route(const void* x, const float* w_router, const float* bias,
                           const int32_t* forced, int T, int d, int E, int k, int32_t* idx,
-                          float* w, void* workspace, cudaStream_t s) {
+                          float* w, void* workspace, size_t workspace_bytes, cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  const int splits = route_splits(T, d, E);
+  const int splits = route_splits(T, d, E, workspace_bytes);
   const RouteWs ws = route_ws(workspace, splits, T, E);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, k, splits, ws, s)
@@ -532,8 +520,9 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
 // stream and have no allocator of their own to lend, and latency-critical
 // serving paths that must not risk an allocation failure or an implicit
 // synchronisation.  moe_route_topk_noalloc keeps the router's scratch (the
-// per-slice fp64 partial logits) in a fixed device array owned by this
-// library instead of a caller-provided workspace.
+// per-slice fp32 partial logits and squared norms) in a fixed device array
+// owned by this library instead of a caller-provided workspace; the number
+// of d slices is capped so that the scratch fits the array.
 // ---------------------------------------------------------------------------
 
 #include <mutex>
@@ -576,17 +565,18 @@ extern "C" moe_status_t moe_route_topk_noalloc(const void* x, const float* w_rou
                                                 const int32_t* forced_idx, int T, int d, int E, int k,
                                                 int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
   using namespace moeq;
-  const size_t need = route_workspace_bytes(T, d, E);
+  moe_status_t st = route_check_args(x, w_router, T, d, E, k, topk_idx, topk_w, "moe_route_topk_noalloc");
+  if (st != MOE_OK) return st;
+  const size_t need = route_min_workspace_bytes(T, d, E);
   if (T > 0 && need > kRouteScratchBytes) {
     set_error("moe_route_topk_noalloc: T=%d d=%d E=%d needs %zu bytes of scratch, above the fixed %zu",
               T, d, E, need, kRouteScratchBytes);
     return MOE_ERR_UNSUPPORTED_SHAPE;
   }
+  if (T == 0) return MOE_OK;
   void* scratch = nullptr;
-  if (T > 0) {
-    moe_status_t st = route_scratch(&scratch);
-    if (st != MOE_OK) return st;
-  }
-  return moe_route_topk(x, w_router, bias, forced_idx, T, d, E, k, topk_idx, topk_w, scratch,
-                        kRouteScratchBytes, stream);
+  st = route_scratch(&scratch);
+  if (st != MOE_OK) return st;
+  return launch_route(x, w_router, bias, forced_idx, T, d, E, k, topk_idx, topk_w, scratch,
+                      kRouteScratchBytes, static_cast<cudaStream_t>(stream));
 }

@@ -59,6 +59,7 @@ struct moe_slot_cache {
   std::vector<std::vector<int>> wave_misses;     // experts that must be copied, per wave
   std::vector<std::vector<int>> wave_slots;      // slot of each expert of the wave
   int copies_issued = 0;                         // waves whose copies were issued
+  bool staged = false;  // a plan is staged and its moe_slot_ffn has not run yet
   int64_t stats[3] = {0, 0, 0};
 };
 
@@ -76,6 +77,7 @@ void invalidate_from(moe_slot_cache* c, int w) {
   c->waves.clear();
   c->wave_misses.clear();
   c->wave_slots.clear();
+  c->staged = false;
 }
 
 moe_status_t issue_copies(moe_slot_cache* c, int w, cudaStream_t copy) {
@@ -301,6 +303,7 @@ moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_id
     c->copies_issued = w + 1;
   }
   *n_waves = nw;
+  c->staged = true;
   c->stats[0] = n_hits;
   c->stats[1] = n_miss;
   c->stats[2] = n_miss * static_cast<int64_t>(c->blob_bytes);
@@ -319,6 +322,12 @@ moe_status_t moe_slot_prefetch(moe_slot_cache* c, const int32_t* ids_host, int n
     return MOE_ERR_INVALID_ARG;
   }
   if (n_copied) *n_copied = 0;
+  if (c->staged) {
+    // the staged plan's slots (hits, and misses of waves whose copies are
+    // issued later) must keep their experts until its moe_slot_ffn has run
+    set_error("moe_slot_prefetch: called between moe_slot_stage and moe_slot_ffn of the same cache");
+    return MOE_ERR_INVALID_ARG;
+  }
   // Victims: least recently used slots, never one filled by this call; each
   // copy waits for the compute that last read its slot (a step of this layer
   // whose FFN may still run).
@@ -419,6 +428,7 @@ moe_status_t moe_slot_ffn(moe_slot_cache* c, const void* x_perm, const int32_t* 
       c->copies_issued = nxt + 1;
     }
   }
+  c->staged = false;
   return MOE_OK;
 }
 

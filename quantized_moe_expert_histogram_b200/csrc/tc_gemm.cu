@@ -59,6 +59,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -900,14 +901,16 @@ bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, 
 
 int* g_trace = nullptr;  // test hook: host-mapped progress record
 
+// SM count of the current device (cached per device).
 int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
+  static std::atomic<int> cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev].load() > 0) return cached[dev].load();
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cached[dev].store(n);
   return n;
 }
 
@@ -974,12 +977,17 @@ moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int r
 template <bool GATEUP, bool PLANES>
 moe_status_t launch_one(const TcParams& P, bool pdl, cudaStream_t s) {
   auto kern = k_ffn_tc<GATEUP, PLANES>;
-  // Set once per process (the first call must precede any stream capture).
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<GATEUP>::SMEM);
+  // The shared-memory opt-in is a per-device attribute: set once per device
+  // (the first call on a device must precede any stream capture).
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_check(e, "tc ffn cudaGetDevice");
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (!bit || !(attr_set.load() & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<GATEUP>::SMEM);
     if (e != cudaSuccess) return cuda_check(e, "tc ffn smem attribute");
-    attr_set = true;
+    attr_set.fetch_or(bit);
   }
   return cuda_check(launch_pdl(pdl, kern, dim3(sm_count()), dim3(kThreads), Cfg<GATEUP>::SMEM, s, P), "tc ffn launch");
 }

@@ -110,6 +110,16 @@ def make_layer(shape: LayerShape, T: int, seed: int = 0, device="cpu", weights=T
     return out
 
 
+def make_bit_gate(shape: LayerShape, seed: int, device="cpu", bias: bool = False) -> dict:
+    """Synthetic weights of a bit-width gate (one linear score per width and
+    expert): ``w_bit`` fp32 [E,3,d] ~ N(0, 0.02^2) and, when ``bias``,
+    ``bias_bit`` fp32 [E,3] ~ N(0, 0.1^2) (else None)."""
+    gen = _gen(seed, device)
+    out = {"w_bit": torch.randn(shape.E, 3, shape.d, generator=gen, device=device) * ROUTER_STD}
+    out["bias_bit"] = torch.randn(shape.E, 3, generator=gen, device=device) * 0.1 if bias else None
+    return out
+
+
 def make_expert_weights(shape: LayerShape, seed: int, device="cpu") -> dict:
     """Expert weights alone (used for the stacked offload layers)."""
     gen = _gen(seed, device)

@@ -12,11 +12,15 @@ from . import moeq
 
 
 class QuantMoELayer:
-    def __init__(self, d, E, k, F, group, layout, w_router, bias, blobs, max_tokens, device="cuda"):
+    def __init__(self, d, E, k, F, group, layout, w_router, bias, blobs, max_tokens, device="cuda",
+                 w_bit=None, bias_bit=None):
         self.d, self.E, self.k, self.F, self.group = d, E, k, F, group
         self.layout = layout
         self.w_router = w_router
         self.bias = bias
+        # optional bit-width gate (nested-plane layout): widths chosen per
+        # (token, selected expert) on the device by moe_bit_gate
+        self.w_bit, self.bias_bit = w_bit, bias_bit
         self.blobs = blobs
         self.device = torch.device(device)
         self.max_tokens = max_tokens
@@ -45,6 +49,7 @@ class QuantMoELayer:
             workspace=torch.empty(max(16, moeq.moe_ffn_workspace_bytes(rows, self.E, d, self.F, self.layout)),
                                   dtype=torch.uint8, device=dev),
             y=torch.empty(T, d, dtype=torch.bfloat16, device=dev),
+            bits=torch.empty(T, k, dtype=torch.uint8, device=dev),
             status=torch.zeros(1, dtype=torch.int32, device=dev),
             route_ws=torch.empty(max(256, moeq.moe_route_workspace_bytes(T, d, self.E)), dtype=torch.uint8,
                                  device=dev),
@@ -58,9 +63,13 @@ class QuantMoELayer:
         return dict(topk_idx=b["topk_idx"][:T], topk_w=b["topk_w"][:T], counts=b["counts"],
                     offsets=b["offsets"], perm=b["perm"][:rows], inv_perm=b["inv_perm"][:rows],
                     x_perm=b["x_perm"][:rows], y_perm=b["y_perm"][:rows], workspace=b["workspace"],
-                    y=b["y"][:T], status=b["status"], route_ws=b["route_ws"], perm_ws=b["perm_ws"])
+                    y=b["y"][:T], status=b["status"], route_ws=b["route_ws"], perm_ws=b["perm_ws"],
+                    bits=b["bits"][:T])
 
     def forward(self, x, bits=None, forced_idx=None, residual=None, stream=None):
+        """One layer pass.  ``bits`` (uint8 [T,k], nested layout) fixes the
+        widths; when it is None and the layer has a bit gate, the widths come
+        from moe_bit_gate on the device."""
         T = x.shape[0]
         if T > self.max_tokens:
             raise ValueError(f"T={T} exceeds max_tokens={self.max_tokens}")
@@ -68,6 +77,9 @@ class QuantMoELayer:
         moeq.moe_route_topk(x, self.w_router, self.bias, self.k, forced_idx=forced_idx,
                             topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"],
                             stream=stream)
+        if bits is None and self.w_bit is not None:
+            bits = moeq.moe_bit_gate(x, self.w_bit, self.bias_bit, v["topk_idx"], bits=v["bits"],
+                                     status=v["status"], stream=stream)
         moeq.moe_permute(v["topk_idx"], self.E, bits=bits, x=x, out=v, status=v["status"], stream=stream)
         moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], self.blobs, T, self.E, self.d, self.F,
                                 self.group, self.layout, workspace=v["workspace"], y_perm=v["y_perm"],

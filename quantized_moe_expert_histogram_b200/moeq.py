@@ -40,6 +40,7 @@ _SIGS = {
                            _c_p, _c_p, _c_sz, _c_p]),
     "moe_permute_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
     "moe_static_bits": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]),
+    "moe_bit_gate": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]),
     "moe_ffn_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
     "moe_grouped_ffn_wq": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                   _c_p, _c_sz, _c_p, _c_p, _c_p]),
@@ -203,6 +204,22 @@ def moe_static_bits(topk_idx, width_of, E, bits=None, status=None, stream=None):
         bits = torch.empty(T, k, dtype=torch.uint8, device=topk_idx.device)
     _check("moe_static_bits", lib.moe_static_bits(
         _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(width_of, torch.uint8, "width_of"), T, k, E,
+        _ptr(bits, torch.uint8, "bits"), _ptr(status, torch.int32, "status"), _stream(stream)))
+    return bits
+
+
+def moe_bit_gate(x, w_bit, bias_bit, topk_idx, bits=None, status=None, stream=None):
+    """bits[t][j] = 2 + argmax_c (x[t] . w_bit[e][c] + bias_bit[e][c]) for
+    e = topk_idx[t][j] (uint8 [T][k])."""
+    lib = load()
+    T, d = x.shape
+    E = w_bit.shape[0]
+    k = topk_idx.shape[1]
+    if bits is None:
+        bits = torch.empty(T, k, dtype=torch.uint8, device=x.device)
+    _check("moe_bit_gate", lib.moe_bit_gate(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_bit, torch.float32, "w_bit"),
+        _ptr(bias_bit, torch.float32, "bias_bit"), _ptr(topk_idx, torch.int32, "topk_idx"), T, d, E, k,
         _ptr(bits, torch.uint8, "bits"), _ptr(status, torch.int32, "status"), _stream(stream)))
     return bits
 

@@ -197,6 +197,25 @@ def test_small_batch_kernel_multi_pass(layout):
         moeq.moe_debug_force_regime(0)
 
 
+@pytest.mark.parametrize("regime", [1, 3])
+@pytest.mark.parametrize("d,E,k,F,g,layout,T", [
+    (4096, 4, 2, 512, 128, "int4", 8),     # gate/up rows of K = 4096: more stages than one ring
+    (4096, 4, 2, 512, 128, "planes", 8),
+    (256, 2, 1, 14336, 128, "int4", 6),    # down rows of K = 14336
+    (256, 3, 2, 14336, 64, "planes", 5),
+    (4096, 3, 2, 256, 64, "int4", 40),     # bins above 16 rows: several passes per bin
+])
+def test_decode_kernels_long_rows(regime, d, E, k, F, g, layout, T):
+    """The decode-regime kernels forced on (1: the one-token kernel, 3: the
+    small-batch kernel) at the row lengths of the d = 4096 and d_ff = 14336
+    workloads, where a row spans many shared-memory stages."""
+    moeq.moe_debug_force_regime(regime)
+    try:
+        _check_layer(I.custom_shape(d=d, E=E, k=k, F=F, group=g, layout=layout), T, seed=13)
+    finally:
+        moeq.moe_debug_force_regime(0)
+
+
 @pytest.mark.parametrize("T", [5, 300])
 def test_static_per_expert_widths(T):
     """Static per-expert widths: bits come from moe_static_bits (width_of[e]

@@ -174,3 +174,59 @@ def test_offload_stack_equals_resident(prefetch):
         assert off.prefetched > 0
     ref.close()
     off.close()
+
+
+@pytest.mark.parametrize("prefetch", [False, True])
+def test_offload_olmoe_shaped_stack_equals_resident(prefetch):
+    """The offload driver on the layer shape the benchmark times (OLMoE-shaped:
+    d 2048, 64 experts, top-8, d_ff 1024, 16 slots, batch 8; two layers, four
+    steps) gives the resident path's outputs bit for bit."""
+    shape = I.SHAPES["olmoe"]
+    ref = Stack(shape, layers=2, slots=16, batch=8, seed=7)
+    off = OffloadStack(shape, layers=2, slots=16, batch=8, seed=7, prefetch=prefetch)
+    steps = 4
+    trace = I.make_slot_trace(shape.E, shape.k, 2, steps=steps, batch=8, seed=8).cuda()
+    xs_all = I.make_slot_x(shape.d, steps, 8, seed=8, device="cuda")
+    for s in range(steps):
+        _, ys_r, _ = ref.step(xs_all[s], trace[s], offload=False)
+        y_o, stats = off.step(xs_all[s], trace[s])
+        torch.cuda.synchronize()
+        assert torch.equal(y_o, ys_r[-1]), f"step {s}"
+        for l in range(2):
+            hits, misses, nbytes, nw = stats[l]
+            assert hits + misses == len(set(trace[s, l].reshape(-1).tolist()))
+            assert nbytes == misses * off.blob_bytes
+    ref.close()
+    off.close()
+
+
+def test_prefetch_between_stage_and_ffn_is_rejected():
+    """moe_slot_prefetch may not run between a cache's moe_slot_stage and its
+    moe_slot_ffn (it could evict an expert the staged plan relies on); after
+    the FFN it is allowed again and the results stay exact."""
+    shape, st = _small_stack(slots=4)
+    trace = I.make_slot_trace(shape.E, shape.k, 3, steps=2, batch=8, seed=9).cuda()
+    xs_all = I.make_slot_x(shape.d, 2, 8, seed=9, device="cuda")
+    _, ys_ref, _ = st.step(xs_all[0], trace[0], offload=False)
+    layer = st.layers[0][0]
+    v = layer.views(8)
+    moeq.moe_route_topk(xs_all[0], layer.w_router, layer.bias, shape.k, forced_idx=trace[0, 0].contiguous(),
+                        topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"])
+    moeq.moe_permute(v["topk_idx"], shape.E, x=xs_all[0], out=v, status=v["status"])
+    routed = v["topk_idx"].cpu().reshape(-1)
+    st.caches[0].stage(routed, st.copy, st.compute)
+    others = torch.tensor([e for e in range(shape.E) if e not in set(routed.tolist())][:4], dtype=torch.int32)
+    with pytest.raises(moeq.MoeError) as ei:
+        st.caches[0].prefetch(others, 4, st.copy)
+    assert ei.value.code == 1
+    st.caches[0].ffn(v["x_perm"], v["offsets"], 8, shape.d, shape.F, shape.group, layer.layout, v["workspace"],
+                     v["y_perm"], v["status"], st.copy, st.compute)
+    y = torch.empty_like(xs_all[0])
+    moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], residual=xs_all[0], y=y)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ys_ref[0])
+    assert st.caches[0].prefetch(others, 4, st.copy) > 0  # allowed again after the FFN
+    _, ys_o, _ = st.step(xs_all[0], trace[0], offload=True)
+    for l in range(3):
+        assert torch.equal(ys_o[l], ys_ref[l])
+    st.close()

@@ -38,6 +38,28 @@ def test_noalloc_router_matches_workspace_router(name, T, seed):
         np.testing.assert_allclose(w_b.cpu().numpy(), w_a.cpu().numpy(), rtol=2e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("T", [2048, 4096])
+def test_noalloc_router_at_large_batches(T):
+    """Batches whose preferred d-slicing needs more scratch than the fixed
+    array: the call lowers the slice count instead of refusing.  Expert ids
+    equal the workspace router's bit for bit; gates (summed over fewer
+    slices) agree with the fp64 oracle as the workspace router's do."""
+    from oracle import moe_oracle as O
+    from gpu_helpers import GATE_RTOL, GATE_ATOL
+    shape = I.SHAPES["olmoe"]
+    assert moeq.moe_route_workspace_bytes(T, shape.d, shape.E) > (8 << 20)
+    for call in range(2):
+        L = I.make_layer(shape, T, seed=40 + call, weights=False)
+        x, wr, bias = L["x"].cuda(), L["w_router"].cuda(), L["bias"].cuda()
+        idx_a, _ = moeq.moe_route_topk(x, wr, bias, shape.k)
+        idx_b, w_b = moeq.moe_route_topk_noalloc(x, wr, bias, shape.k)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(idx_b.cpu().numpy(), idx_a.cpu().numpy())
+        sel, gates, _ = O.route(L["x"].float().numpy(), L["w_router"].numpy(), L["bias"].numpy(), shape.k)
+        np.testing.assert_array_equal(idx_b.cpu().numpy(), sel)
+        np.testing.assert_allclose(w_b.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
+
+
 def test_noalloc_router_rejects_oversized_scratch():
     shape = I.SHAPES["olmoe"]
     T = 1 << 16  # needs more than the fixed 8 MiB of partial logits
