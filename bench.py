@@ -45,8 +45,9 @@ def parse():
     p.add_argument("--cpu-sample-tokens", type=int, default=0)
     p.add_argument("--workloads", default="mixtral:8192,mixtral:1,nested:2048,nested:1,tiny:64",
                    help="other configured workloads reported for context (name:tokens,...; '' = none)")
-    p.add_argument("--offload-steps", type=int, default=24,
-                   help="decode steps of the offload (slot-cache) workload reported under 'offload' (0 = skip)")
+    p.add_argument("--offload-steps", type=int, default=512,
+                   help="decode steps of the offload (slot-cache) workload reported under 'offload', after "
+                        "16 warm-up steps, per schedule (0 = skip)")
     p.add_argument("--profile", action="store_true",
                    help="profiling driver: one instance, warmup + steps of the eager step, no JSON")
     return p.parse_args()
@@ -372,40 +373,58 @@ def h2d_peak_gbs(nbytes=256 << 20, reps=5):
     return nbytes * reps / (a.elapsed_time(b) / 1e3) / 1e9
 
 
-def run_offload(steps, layers=16, slots=16, batch=8, seed=0, prefetch=False):
+def run_offload(steps, layers=16, slots=16, batch=8, seed=0, warm=16):
     """The offload workload: stacked OLMoE-shaped layers with experts in pinned
     host memory and a slot cache per layer, decode steps at a fixed batch on a
-    Zipf + successor-correlated routing trace.  Wall time around whole steps
-    (each layer's step synchronises once for the routed ids)."""
+    Zipf + successor-correlated routing trace, in three schedules on the same
+    stack: a routed-id sync per layer ("sync"), that plus predictive
+    prefetching of the next layer's experts ("prefetch"), and lookahead
+    (every layer's ids known at the start of the step, one id copy per step,
+    no per-layer sync).  Wall clock around whole steps; busy times of the
+    copies and of the compute from CUDA events that exclude each stream's
+    waits for the other, giving
+        overlap = (copy + compute - wall) / min(copy, compute)
+    (1 = the shorter of the two is hidden entirely, 0 = none of it)."""
     import torch
     from quantized_moe_expert_histogram_b200 import inputs as I
     from quantized_moe_expert_histogram_b200.offload import OffloadStack
     shape = I.SHAPES["olmoe"]
-    stack = OffloadStack(shape, layers, slots, batch, seed=seed, prefetch=prefetch)
-    warm = 2
-    trace = I.make_slot_trace(shape.E, shape.k, layers, steps + warm, batch, seed=seed + 1).cuda()
-    xs = I.make_slot_x(shape.d, steps + warm, batch, seed=seed + 1, device="cuda")
-    for s in range(warm):
-        stack.step(xs[s], trace[s])
-    torch.cuda.synchronize()
+    stack = OffloadStack(shape, layers, slots, batch, seed=seed, prefetch=True)
+    n = steps + warm
+    trace = I.make_slot_trace(shape.E, shape.k, layers, n, batch, seed=seed + 1).cuda()
+    xs = I.make_slot_x(shape.d, n, batch, seed=seed + 1, device="cuda")
     peak = h2d_peak_gbs()
-    hits = misses = nbytes = 0
-    t0 = time.perf_counter()
-    for s in range(warm, warm + steps):
-        _, st = stack.step(xs[s], trace[s])
-        for h, m, b, _w in st:
-            hits, misses, nbytes = hits + h, misses + m, nbytes + b
-    torch.cuda.synchronize()
-    wall = time.perf_counter() - t0
+    out = {"workload": f"{layers} OLMoE-shaped layers (d=2048, E=64, top-8, d_ff=1024, INT4 g128), "
+                       f"{slots} GPU slots per layer, batch {batch}, Zipf routing with 70% successor correlation",
+           "steps": steps, "warmup_steps": warm, "h2d_peak_gbs": peak,
+           "timing": "host wall clock around whole steps; copy/compute busy time from CUDA events"}
+    for mode in ("sync", "prefetch", "lookahead"):
+        stack.prefetch, stack.lookahead = mode == "prefetch", mode == "lookahead"
+        stack.prefetched = 0
+        for s in range(warm):
+            stack.step(xs[s], trace[s])
+        torch.cuda.synchronize()
+        stack.timing(True)
+        hits = misses = nbytes = 0
+        t0 = time.perf_counter()
+        for s in range(warm, n):
+            _, st = stack.step(xs[s], trace[s])
+            for h, m, b, _w in st:
+                hits, misses, nbytes = hits + h, misses + m, nbytes + b
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+        copy_ms, comp_ms = stack.timing_read()
+        stack.timing(False)
+        wall_ms = wall * 1e3
+        h2d = nbytes / wall / 1e9
+        out[mode] = {"tokens_per_s": batch * steps / wall, "ms_per_step": wall_ms / steps,
+                     "h2d_bytes_per_step": nbytes / steps, "h2d_gbs": h2d, "h2d_frac": h2d / peak,
+                     "hit_rate": hits / max(1, hits + misses),
+                     "copy_busy_ms_per_step": copy_ms / steps, "compute_busy_ms_per_step": comp_ms / steps,
+                     "overlap": (copy_ms + comp_ms - wall_ms) / max(1e-9, min(copy_ms, comp_ms)),
+                     "prefetch_copies_per_step": stack.prefetched / n}
     stack.close()
-    h2d = nbytes / wall / 1e9
-    return {"workload": f"{layers} OLMoE-shaped layers (d=2048, E=64, top-8, d_ff=1024, INT4 g128), "
-                        f"{slots} GPU slots per layer, batch {batch}, Zipf routing with 70% successor correlation",
-            "steps": steps, "tokens_per_s": batch * steps / wall, "ms_per_step": wall / steps * 1e3,
-            "h2d_bytes_per_step": nbytes / steps, "h2d_gbs": h2d, "h2d_peak_gbs": peak,
-            "h2d_frac": h2d / peak, "hit_rate": hits / max(1, hits + misses),
-            "prefetch": prefetch, "prefetch_copies_per_step": stack.prefetched / (steps + warm),
-            "timing": "host wall clock around whole steps (one routed-id sync per layer)"}
+    return out
 
 
 def cpu_baseline(shape, T, seed, sample_tokens, budget_s=20.0):
@@ -563,7 +582,6 @@ def main():
         del layers
         torch.cuda.empty_cache()
         offload = run_offload(args.offload_steps)
-        offload["with_prefetch"] = run_offload(args.offload_steps, prefetch=True)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -322,6 +322,17 @@ MOE_API moe_status_t moe_slot_ffn(moe_slot_cache* cache, const void* x_perm, con
 MOE_API moe_status_t moe_slot_prefetch(moe_slot_cache* cache, const int32_t* ids_host, int n_ids, int max_copies,
                                        moe_stream_t copy_stream, int32_t* n_copied);
 
+/* Busy-time measurement of the offload pipeline (the load/compute overlap
+ * figure): with enable != 0 the cache records CUDA timing events around each
+ * wave's copies (after the copy stream's waits for free slots) and around
+ * each wave's FFN (after the compute stream's wait for those copies), so the
+ * sums count only the time each stream works, not the time it waits for the
+ * other.  moe_slot_timing_read waits for the recorded events (a host
+ * synchronisation), returns the copy and FFN milliseconds since the last
+ * read or enable, and starts new sums.  Off by default. */
+MOE_API moe_status_t moe_slot_timing(moe_slot_cache* cache, int enable);
+MOE_API moe_status_t moe_slot_timing_read(moe_slot_cache* cache, double* copy_ms, double* ffn_ms);
+
 /* Next-layer expert predictor (host-only): counts of (expert at layer l-1,
  * expert at layer l) pairs at the same token and choice position, learned
  * online with moe_predictor_observe; moe_predictor_predict scores experts
@@ -360,6 +371,21 @@ MOE_API void moe_debug_force_regime(int regime);
  * so that a stalled launch can be read from the host while it runs.
  * NULL (the default) disables it. */
 MOE_API void moe_debug_set_trace(void* host_mapped_ints);
+
+/* Test hook: 1 (the default) lets moe_route_topk run decode-sized batches
+ * (up to 64 tokens, E <= 64) as one launch of a thread-block cluster; 0
+ * forces the two-launch router (same arithmetic).  Process-wide. */
+MOE_API void moe_debug_route_fused(int enable);
+
+/* Test hook of the on-device failure path: while enabled, the tensor-core
+ * FFN kernels give every bounded wait a 20 ms limit (instead of 2 s), and in
+ * the gate/up kernel the epilogue of CTA 0 withholds the release of its
+ * first tile's accumulators -- an arrive with no copy behind it -- so that
+ * the MMA warp's wait for its next tile runs out whenever CTA 0 has more than
+ * one tile.  The CTA then sets MOE_DEV_TIMEOUT in `status`, drains its
+ * copies and MMAs, frees its tensor memory and returns; that call's outputs
+ * are undefined.  0 (the default) disables it.  Process-wide. */
+MOE_API void moe_debug_ffn_timeout(int enable);
 
 #ifdef __cplusplus
 }

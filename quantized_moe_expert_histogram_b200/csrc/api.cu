@@ -94,16 +94,16 @@ namespace {
 
 inline cudaStream_t S(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 
-// Regime by T (bins never hold more than T rows): one token -> the decode
-// GEMV (CUDA-core dot products, one weight pass); up to kMmaMaxT tokens ->
-// the small-batch kernel (mma.sync dot products, cost per weight flat up to
-// 16 rows per pass); above -> the tensor-core grouped GEMM (128-row tiles).
-// Measured on the OLMoE-shaped layer: 2-8 tokens fastest on the small-batch
-// kernel, 16 and more on the tensor-core kernel.
-constexpr int kMmaMaxT = 8;
+// Regime by T (bins never hold more than T rows): up to kDecMaxT tokens ->
+// the decode kernel (weight-streaming, split-K over warps, mma.sync with one
+// or two 8-token blocks); above -> the tensor-core grouped GEMM (128-row
+// weight tiles, tcgen05).
+constexpr int kDecMaxT = 16;
 
-// 0: pick by T; 1: always the one-token GEMV; 2: tensor cores whenever
-// possible; 3: always the small-batch kernel.
+// 0: pick by T; 1: the decode kernel with one 8-token block per pass; 2:
+// tensor cores whenever possible; 3: the decode kernel with two 8-token
+// blocks; 4, 5: the earlier CUDA-core GEMV and the earlier small-batch
+// kernel (comparison only).
 int g_force_regime = 0;
 
 size_t workspace_for(int total_rows, int F) {
@@ -117,7 +117,7 @@ extern "C" {
 
 const char* moe_last_error(void) { return g_err; }
 
-void moe_debug_force_regime(int regime) { g_force_regime = (regime >= 0 && regime <= 3) ? regime : 0; }
+void moe_debug_force_regime(int regime) { g_force_regime = (regime >= 0 && regime <= 5) ? regime : 0; }
 
 size_t moe_blob_bytes(int d, int F, int group, int layout) {
   const BlobLayout L = blob_layout(d, F, group, layout);
@@ -262,10 +262,12 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   a.status = status;
   const bool tc_ok = total_rows >= 16 && tc_supported(a);
   int regime = g_force_regime;
-  if (regime == 0) regime = T <= 1 ? 1 : (T <= kMmaMaxT || !tc_ok ? 3 : 2);
+  if (regime == 0) regime = T <= kDecMaxT || !tc_ok ? (T <= 8 ? 1 : 3) : 2;
   if (regime == 2 && !tc_ok) regime = 3;
   if (regime == 2) return launch_ffn_tc(a, S(stream));
-  return regime == 1 ? launch_ffn_gemv(a, S(stream)) : launch_ffn_gemv_mma(a, S(stream));
+  if (regime == 4) return launch_ffn_gemv(a, S(stream));
+  if (regime == 5) return launch_ffn_gemv_mma(a, S(stream));
+  return launch_ffn_decode(a, regime == 1 ? 1 : 2, S(stream));
 }
 
 moe_status_t moe_bit_gate(const void* x, const float* w_bit, const float* bias_bit, const int32_t* topk_idx,

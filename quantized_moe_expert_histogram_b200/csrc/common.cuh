@@ -107,6 +107,7 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
                           const int32_t* forced, int T, int d, int E, int k, int32_t* idx,
                           float* w, void* workspace, size_t workspace_bytes, cudaStream_t s);
 size_t route_workspace_bytes(int T, int d, int E);
+extern int g_route_fused;  // test hook: 0 = always the two-launch router
 size_t route_min_workspace_bytes(int T, int d, int E);
 moe_status_t route_check_args(const void* x, const float* w_router, int T, int d, int E, int k,
                               const int32_t* topk_idx, const float* topk_w, const char* fn);
@@ -132,6 +133,7 @@ struct FfnArgs {
 };
 moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);
 moe_status_t launch_ffn_gemv_mma(const FfnArgs& a, cudaStream_t s);
+moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t s);
 moe_status_t launch_bit_gate(const void* x, const float* w_bit, const float* bias_bit, const int32_t* idx,
                              int T, int d, int E, int k, uint8_t* bits, int32_t* status, cudaStream_t s);
 moe_status_t launch_static_bits(const int32_t* idx, const uint8_t* width_of, int n, int E, uint8_t* bits,

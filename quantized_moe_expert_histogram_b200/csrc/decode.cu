@@ -1,0 +1,493 @@
+// Decode-regime grouped expert FFN: small bins (up to 16 token rows), where
+// the layer is bound by the bytes of the routed experts' weights.
+//
+// Swap-AB tensor-core dot products (mma.sync m16n8k16, fp32 accumulate):
+// dequantised weight rows are operand A (16 rows x 16 K per instruction)
+// and the bin's token rows operand B (N = 8 tokens), so one instruction
+// consumes 256 weights whatever the number of tokens up to 8 (two per A
+// fragment for 9-16 tokens).  A holds (code - zero) in fp16, which is exact;
+// the scale of a 128-wide group is applied to the fp32 partial sum of that
+// group, acc += s * sum_k (q_k - z) x_k (for groups of 64, where one lane's
+// K run spans two groups, A holds (q - z) * s rounded once to fp16, as in
+// the 128-row kernel).
+//
+// Work split: a CTA (8 warps) owns one item = (bin, block of weight rows):
+// 16 features x {gate, up} in the first GEMM, 16 or 32 rows of W_down in
+// the second, and its warps split K: warp w takes the 128-K stages w, w+8,
+// w+16, ... of every row of the item (so a 14336-long row is eight warps'
+// work, and at any time the CTA reads a contiguous K window of each row).
+// Each warp streams its stages with cp.async into a 4-deep shared-memory
+// ring (the bytes in flight take no registers).  The warps' partial sums
+// are added in shared memory in a fixed order (deterministic), and the
+// epilogue writes h = silu(gate) * up or y_perm (fp16).
+//
+// Register layout of one MMA, lane = (g, c) = (lane / 4, lane % 4): A rows g
+// and g + 8, K slots {2c, 2c+1, 2c+8, 2c+9}; B token g at the same slots;
+// D rows g, g + 8 x tokens 2c, 2c + 1.  The sum runs over K, so each lane
+// feeds its K slots from its own run of 32 consecutive elements of the
+// stage: a code word (8 elements) gives four fp16 pairs by masking nibble
+// pairs into the mantissa of 1024 (low nibbles) or 64 (high nibbles), and
+// the activations are paired the same way -- elements (j, j + 4) for INT4
+// words, (2j, 2j + 1) for plane-order words.
+//
+// Both passes are programmatic dependent launches (launch_pdl).  The down
+// pass locates its bin and issues the copies of its first weight stages
+// (which do not depend on h) before it waits for the gate/up grid.
+//
+//   gate/up pass:  h[p][f]      = silu(Wg[f] . x_p) * (Wu[f] . x_p)   (fp16)
+//   down pass:     y_perm[p][n] = Wd[n] . h_p                          (fp16)
+#include <algorithm>
+#include <atomic>
+
+#include "common.cuh"
+
+namespace moeq {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kStageK = 128;       // K per stage (one group of 128, two of 64)
+constexpr int kFragBytes = 1024;   // one stage of one 16-row fragment: 16 rows x 64 B
+constexpr int kSzBytes = 128;      // its scale/zero words: 16 rows x up to 2 groups
+constexpr int kRing = 4;           // stages in flight per warp
+
+struct DecParams {
+  const __half* act;        // x_perm or h: fp16 [rows][K]
+  const int32_t* offsets;   // [nbins + 1]
+  const uint8_t* blobs;
+  const int32_t* slot_of;
+  size_t blob_bytes;
+  size_t code_off[2];       // INT4 codes (or Q2) of matrix 0 / 1
+  size_t d3_off[2];
+  size_t d4_off[2];
+  size_t sz_off[2];
+  int K, N, nbins, planes_mult;
+  int rows;                 // activation rows: bin ranges are clamped into [0, rows]
+  int group;
+  int row_blocks;           // items per bin (weight-row blocks)
+  __half* out;              // h (gate/up) or y_perm (down): fp16 [rows][N]
+  int32_t* status;
+};
+
+// Locate the ordinal-th non-empty, resident bin (ballot over 32 bins at a
+// time).  Returns false when there is none.
+__device__ __forceinline__ bool find_bin(const DecParams& P, int ordinal, int& bin, int& row0, int& nrows,
+                                         int& slot, int& bits) {
+  const int lane = threadIdx.x & 31;
+  int seen = 0;
+  for (int b0 = 0; b0 < P.nbins; b0 += 32) {
+    const int b = b0 + lane;
+    bool ok = false;
+    int sl = 0;
+    if (b < P.nbins) {
+      const int n = min(max(P.offsets[b + 1], 0), P.rows) - min(max(P.offsets[b], 0), P.rows);
+      const int e = b / P.planes_mult;
+      sl = P.slot_of ? P.slot_of[e] : e;
+      ok = n > 0 && sl >= 0;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, ok);
+    const int cnt = __popc(m);
+    if (ordinal < seen + cnt) {
+      unsigned mm = m;
+      for (int i = 0; i < ordinal - seen; ++i) mm &= mm - 1;
+      const int src = __ffs(mm) - 1;
+      bin = b0 + src;
+      slot = __shfl_sync(0xffffffffu, sl, src);
+      row0 = min(max(P.offsets[bin], 0), P.rows);
+      nrows = max(0, min(max(P.offsets[bin + 1], 0), P.rows) - row0);
+      bits = P.planes_mult == 3 ? 2 + bin % 3 : 4;
+      return true;
+    }
+    seen += cnt;
+  }
+  return false;
+}
+
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t c) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(m), "r"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// The four fp16 pairs of a code word: nibbles (0,4), (1,5), (2,6), (3,7)
+// minus the zero-point.  Nibbles masked into 0x6400 read as 1024 + n, those
+// at bits 4..7 of a half masked into 0x5400 as 64 + n (unit 1/16 at 64);
+// z_lo = 1024 + z, z_hi = 64 + z (both exact), so each pair is exactly
+// (n - z).  For an INT4 word these are elements (j, j + 4); for a
+// plane-order word elements (2j, 2j + 1).
+__device__ __forceinline__ void pairs(uint32_t w, __half2 z_lo, __half2 z_hi, uint32_t (&p)[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = h2u(__hsub2(u2h(and_or(w, 0x000F000Fu, 0x64006400u)), z_lo));
+  p[1] = h2u(__hsub2(u2h(and_or(w, 0x00F000F0u, 0x54005400u)), z_hi));
+  p[2] = h2u(__hsub2(u2h(and_or(w8, 0x000F000Fu, 0x64006400u)), z_lo));
+  p[3] = h2u(__hsub2(u2h(and_or(w8, 0x00F000F0u, 0x54005400u)), z_hi));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ldg_act(const __half* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// GU: first GEMM (fragment 0 = gate rows, 1 = up rows of 16 features);
+// else the second GEMM (FW fragments of 16 consecutive W_down rows).  NB
+// token blocks of 8 per pass over K (bins with more rows take more passes).
+template <bool GU, bool PLANES, bool G64, int FW, int NB>
+__global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
+  static_assert(!GU || FW == 2, "gate and up fragments");
+  constexpr int kSlot = FW * (kFragBytes + kSzBytes);  // one ring stage of a warp
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  if (GU) {  // x_perm comes from the previous launch
+    pdl_wait();
+    pdl_trigger();
+  }
+  int bin, row0, nrows, slot, bits;
+  const int ordinal = blockIdx.x / P.row_blocks;
+  if (!find_bin(P, ordinal, bin, row0, nrows, slot, bits)) {
+    if (!GU) pdl_wait();  // CTA-uniform; keeps the wait/trigger order of every CTA
+    return;
+  }
+  const int rb = blockIdx.x - ordinal * P.row_blocks;
+  const int n0 = rb * (GU ? 16 : 16 * FW);  // first output row (feature) of this item
+  const uint8_t* blob = P.blobs + static_cast<size_t>(slot) * P.blob_bytes;
+  const int n_stages = P.K / kStageK;
+  const int G = P.K / P.group;
+  uint8_t* ring = smem + warp * (kRing * kSlot);
+  const uint32_t ring_u = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
+  // weight row of fragment f: matrix mat(f), row frow(f) + 0..15
+  auto mat = [](int f) { return GU ? f : 0; };
+  auto frow = [&](int f) { return GU ? n0 : n0 + 16 * f; };
+
+  // copies of this warp's i-th stage (global stage warp + 8 i) into ring
+  // slot i % kRing: per fragment 64 pieces of 16 B of codes, plus the
+  // fragment's scale/zero words (16 rows x 1 or 2 groups, contiguous)
+  auto issue = [&](int i) {
+    const int s = warp + kWarps * i;
+    if (s < n_stages) {
+      const uint32_t dst0 = ring_u + (i % kRing) * kSlot;
+#pragma unroll
+      for (int f = 0; f < FW; ++f) {
+        const int m = mat(f);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int q = lane + 32 * u;  // piece 0..63 of this fragment
+          const uint8_t* src = nullptr;
+          uint32_t dst = dst0 + f * kFragBytes;
+          if (!PLANES) {
+            const int rr = q >> 2, cc = q & 3;
+            src = blob + P.code_off[m] + static_cast<size_t>(frow(f) + rr) * (P.K / 2) + s * 64 + cc * 16;
+            dst += rr * 64 + cc * 16;
+          } else if (q < 32) {  // Q2: 16 rows x 32 B
+            const int rr = q >> 1, hh = q & 1;
+            src = blob + P.code_off[m] + static_cast<size_t>(frow(f) + rr) * (P.K / 4) + s * 32 + hh * 16;
+            dst += rr * 32 + hh * 16;
+          } else if (q < 48) {  // D3: 16 rows x 16 B
+            const int rr = q - 32;
+            if (bits >= 3) src = blob + P.d3_off[m] + static_cast<size_t>(frow(f) + rr) * (P.K / 8) + s * 16;
+            dst += 512 + rr * 16;
+          } else {  // D4
+            const int rr = q - 48;
+            if (bits >= 4) src = blob + P.d4_off[m] + static_cast<size_t>(frow(f) + rr) * (P.K / 8) + s * 16;
+            dst += 768 + rr * 16;
+          }
+          if (src) cp_async16(dst, src);
+        }
+        // scale/zero: rows frow(f)..+15 of group gi: 64 contiguous bytes
+        const int npieces = G64 ? 8 : 4;
+        if (lane < npieces) {
+          const int gi = lane >> 2, pc = lane & 3;
+          const int row = frow(f);
+          const int grp = s * kStageK / P.group + gi;
+          const uint8_t* src = blob + P.sz_off[m] +
+                               ((static_cast<size_t>(row >> 7) * G + grp) * 128 + (row & 127)) * 4 + pc * 16;
+          cp_async16(dst0 + FW * kFragBytes + f * kSzBytes + gi * 64 + pc * 16, src);
+        }
+      }
+    }
+    cp_async_commit();  // an empty group past the end keeps the count uniform
+  };
+
+  const int my_stages = n_stages > warp ? (n_stages - warp + kWarps - 1) / kWarps : 0;
+  bool waited = GU;
+  float acc[FW][NB][4];
+  float* red = reinterpret_cast<float*>(smem);  // reused after the ring drains
+  constexpr int kVals = FW * NB * 4;
+
+  for (int t0 = 0; t0 < nrows; t0 += 8 * NB) {  // one pass over K per 8 NB tokens
+#pragma unroll
+    for (int f = 0; f < FW; ++f)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[f][nb][j] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kRing; ++i) issue(i);
+    if (!waited) {  // down pass: h is read only from here on
+      pdl_wait();
+      pdl_trigger();
+      waited = true;
+    }
+    // token rows of this lane's B fragments
+    bool tok_in[NB];
+    const __half* xrow[NB];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const int tk = t0 + 8 * nb + g;
+      tok_in[nb] = tk < nrows;
+      xrow[nb] = P.act + static_cast<size_t>(row0 + (tok_in[nb] ? tk : 0)) * P.K;
+    }
+    for (int i = 0; i < my_stages; ++i) {
+      const int s = warp + kWarps * i;
+      const int kl = s * kStageK + 32 * c;  // this lane's K run
+      // activations (4 x 8 elements per token block), loaded before the wait
+      uint4 xv[NB][4];
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd)
+          xv[nb][wd] = tok_in[nb] ? ldg_act(xrow[nb] + kl + 8 * wd) : make_uint4(0, 0, 0, 0);
+      cp_async_wait<kRing - 1>();
+      __syncwarp();
+      const uint8_t* sb = ring + (i % kRing) * kSlot;
+#pragma unroll
+      for (int f = 0; f < FW; ++f) {
+        const uint8_t* fb = sb + f * kFragBytes;
+        const uint32_t* szw = reinterpret_cast<const uint32_t*>(sb + FW * kFragBytes + f * kSzBytes);
+        const int gsel = G64 ? (c >> 1) * 16 : 0;  // this lane's group inside the stage
+        const uint32_t wlo = szw[gsel + g], whi = szw[gsel + g + 8];
+        const float zlo_f = __uint_as_float(wlo & 0xFFFF0000u), zhi_f = __uint_as_float(whi & 0xFFFF0000u);
+        const float slo = __uint_as_float(wlo << 16), shi = __uint_as_float(whi << 16);
+        const __half2 za_lo = __half2half2(__float2half_rn(1024.0f + zlo_f));
+        const __half2 za_hi = __half2half2(__float2half_rn(64.0f + zlo_f));
+        const __half2 zb_lo = __half2half2(__float2half_rn(1024.0f + zhi_f));
+        const __half2 zb_hi = __half2half2(__float2half_rn(64.0f + zhi_f));
+        // this lane's 32 elements of rows g and g + 8 as four code words each
+        uint32_t ca[4], cb[4];
+        if (!PLANES) {
+          const uint4 va = *reinterpret_cast<const uint4*>(fb + g * 64 + c * 16);
+          const uint4 vb = *reinterpret_cast<const uint4*>(fb + (g + 8) * 64 + c * 16);
+          ca[0] = va.x; ca[1] = va.y; ca[2] = va.z; ca[3] = va.w;
+          cb[0] = vb.x; cb[1] = vb.y; cb[2] = vb.z; cb[3] = vb.w;
+        } else {
+          // plane-order words: base from bits 2 (wd & 1) of each nibble of Q2
+          // word wd >> 1, residuals from bit wd of the D3 / D4 word
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int r = g + 8 * half;
+            const uint2 q2 = *reinterpret_cast<const uint2*>(fb + r * 32 + c * 8);
+            const uint32_t d3 = bits >= 3 ? *reinterpret_cast<const uint32_t*>(fb + 512 + r * 16 + c * 4) : 0u;
+            const uint32_t d4 = bits >= 4 ? *reinterpret_cast<const uint32_t*>(fb + 768 + r * 16 + c * 4) : 0u;
+            uint32_t* cw = half ? cb : ca;
+            const uint32_t qw[2] = {q2.x, q2.y};
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+              uint32_t v = (qw[wd >> 1] << (2 - 2 * (wd & 1))) & 0xCCCCCCCCu;
+              const int sh = 1 - wd;
+              v = and_or(sh >= 0 ? d3 << sh : d3 >> -sh, 0x22222222u, v);
+              v = and_or(d4 >> wd, 0x11111111u, v);
+              cw[wd] = v;
+            }
+          }
+        }
+        float dsum[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dsum[nb][j] = 0.0f;
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          uint32_t pa[4], pb[4];
+          pairs(ca[wd], za_lo, za_hi, pa);
+          pairs(cb[wd], zb_lo, zb_hi, pb);
+          if (G64) {  // groups of 64: the scale goes into A (one fp16 rounding)
+            const __half2 sa = __half2half2(__float2half_rn(slo)), sb2 = __half2half2(__float2half_rn(shi));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              pa[j] = h2u(__hmul2(u2h(pa[j]), sa));
+              pb[j] = h2u(__hmul2(u2h(pb[j]), sb2));
+            }
+          }
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+              const uint4 x = xv[nb][wd];
+              uint32_t b0, b1;
+              if (PLANES) {
+                b0 = hh ? x.z : x.x;
+                b1 = hh ? x.w : x.y;
+              } else {  // (x_j, x_j+4) pairs
+                b0 = hh ? __byte_perm(x.y, x.w, 0x5410) : __byte_perm(x.x, x.z, 0x5410);
+                b1 = hh ? __byte_perm(x.y, x.w, 0x7632) : __byte_perm(x.x, x.z, 0x7632);
+              }
+              if (G64)
+                mma16816(acc[f][nb], pa[2 * hh], pb[2 * hh], pa[2 * hh + 1], pb[2 * hh + 1], b0, b1);
+              else
+                mma16816(dsum[nb], pa[2 * hh], pb[2 * hh], pa[2 * hh + 1], pb[2 * hh + 1], b0, b1);
+            }
+          }
+        }
+        if (!G64) {
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            acc[f][nb][0] = fmaf(slo, dsum[nb][0], acc[f][nb][0]);
+            acc[f][nb][1] = fmaf(slo, dsum[nb][1], acc[f][nb][1]);
+            acc[f][nb][2] = fmaf(shi, dsum[nb][2], acc[f][nb][2]);
+            acc[f][nb][3] = fmaf(shi, dsum[nb][3], acc[f][nb][3]);
+          }
+        }
+      }
+      __syncwarp();  // every lane is done with ring slot i % kRing
+      issue(i + kRing);
+    }
+    cp_async_wait<0>();
+    __syncthreads();  // every warp's ring is drained: the space becomes the reduction buffer
+#pragma unroll
+    for (int f = 0; f < FW; ++f)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[(warp * kVals + (f * NB + nb) * 4 + j) * 32 + lane] = acc[f][nb][j];
+    __syncthreads();
+    // thread -> (lane', nb, j): sum over warps in order, then the epilogue
+    for (int v = threadIdx.x; v < 32 * NB * 4; v += kWarps * 32) {
+      const int ln = v & 31, nb = (v >> 5) / 4, j = (v >> 5) & 3;
+      const int gg = ln >> 2, cc = ln & 3;
+      const int row = gg + 8 * (j >> 1);           // weight row inside the fragment
+      const int tk = t0 + 8 * nb + 2 * cc + (j & 1);  // token row inside the bin
+      float sum[FW];
+#pragma unroll
+      for (int f = 0; f < FW; ++f) {
+        float a = 0.0f;
+        for (int w = 0; w < kWarps; ++w) a += red[(w * kVals + (f * NB + nb) * 4 + j) * 32 + ln];
+        sum[f] = a;
+      }
+      if (tk < nrows) {
+        const size_t p = static_cast<size_t>(row0 + tk);
+        if (GU) {
+          P.out[p * P.N + n0 + row] = __float2half_rn(silu_f(sum[0]) * sum[1]);
+        } else {
+#pragma unroll
+          for (int f = 0; f < FW; ++f) {
+            if (!(fabsf(sum[f]) <= 65504.0f)) flag_status(P.status, MOE_DEV_RANGE);
+            P.out[p * P.N + n0 + 16 * f + row] = __float2half_rn(sum[f]);
+          }
+        }
+      }
+    }
+    __syncthreads();  // the reduction buffer is the next pass's ring
+  }
+}
+
+template <bool GU, bool PLANES, bool G64, int FW, int NB>
+moe_status_t run_dec(const DecParams& p, int grid, cudaStream_t s, const char* what) {
+  constexpr int smem = kWarps * kRing * FW * (kFragBytes + kSzBytes);
+  static_assert(smem >= kWarps * FW * NB * 4 * 32 * 4, "reduction buffer fits the ring");
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_check(e, what);
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (!bit || !(attr_set.load() & bit)) {
+    e = cudaFuncSetAttribute(k_dec<GU, PLANES, G64, FW, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_check(e, what);
+    attr_set.fetch_or(bit);
+  }
+  return cuda_check(launch_pdl(true, k_dec<GU, PLANES, G64, FW, NB>, dim3(grid), dim3(kWarps * 32), smem, s, p),
+                    what);
+}
+
+template <bool GU, bool PLANES, bool G64, int FW>
+moe_status_t run_nb(const DecParams& p, int nb, int grid, cudaStream_t s, const char* what) {
+  return nb == 1 ? run_dec<GU, PLANES, G64, FW, 1>(p, grid, s, what) : run_dec<GU, PLANES, G64, FW, 2>(p, grid, s, what);
+}
+
+template <bool PLANES, bool G64>
+moe_status_t run_pair(DecParams gu, DecParams dn, int max_bins, int nb, int sms, cudaStream_t s) {
+  gu.row_blocks = gu.N / 16;
+  moe_status_t st = run_nb<true, PLANES, G64, 2>(gu, nb, max_bins * gu.row_blocks, s, "ffn decode gate/up launch");
+  if (st != MOE_OK) return st;
+  // 32-row items unless that leaves fewer than two CTAs per SM
+  const bool wide = static_cast<long>(max_bins) * (dn.N / 32) >= 2L * sms && dn.N % 32 == 0;
+  dn.row_blocks = dn.N / (wide ? 32 : 16);
+  const int grid = max_bins * dn.row_blocks;
+  return wide ? run_nb<false, PLANES, G64, 2>(dn, nb, grid, s, "ffn decode down launch")
+              : run_nb<false, PLANES, G64, 1>(dn, nb, grid, s, "ffn decode down launch");
+}
+
+int sm_count_dec() {
+  static std::atomic<int> cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev].load() > 0) return cached[dev].load();
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cached[dev].store(n);
+  return n;
+}
+
+}  // namespace
+
+moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t s) {
+  const bool planes = a.layout == MOE_LAYOUT_PLANES;
+  const int mult = planes ? 3 : 1;
+  DecParams gu{};
+  gu.act = a.x_perm;
+  gu.offsets = a.offsets;
+  gu.blobs = a.blobs;
+  gu.slot_of = a.slot_of;
+  gu.blob_bytes = a.blob_bytes;
+  gu.K = a.d;
+  gu.N = a.F;
+  gu.nbins = a.E * mult;
+  gu.planes_mult = mult;
+  gu.rows = a.total_rows;
+  gu.group = a.group;
+  gu.out = a.h;
+  gu.status = a.status;
+  for (int m = 0; m < 2; ++m) {
+    gu.code_off[m] = planes ? a.lay.q2[m] : a.lay.codes[m];
+    gu.d3_off[m] = a.lay.d3[m];
+    gu.d4_off[m] = a.lay.d4[m];
+    gu.sz_off[m] = a.lay.sz[m];
+  }
+  DecParams dn = gu;
+  dn.act = a.h;
+  dn.K = a.F;
+  dn.N = a.d;
+  dn.out = a.y_perm;
+  dn.code_off[0] = planes ? a.lay.q2[2] : a.lay.codes[2];
+  dn.d3_off[0] = a.lay.d3[2];
+  dn.d4_off[0] = a.lay.d4[2];
+  dn.sz_off[0] = a.lay.sz[2];
+  const int max_bins = std::min(gu.nbins, a.total_rows);
+  if (max_bins == 0) return MOE_OK;
+  const int nb = token_blocks <= 1 ? 1 : 2;
+  const int sms = sm_count_dec();
+  const bool g64 = a.group == 64;
+  if (planes) return g64 ? run_pair<true, true>(gu, dn, max_bins, nb, sms, s) : run_pair<true, false>(gu, dn, max_bins, nb, sms, s);
+  return g64 ? run_pair<false, true>(gu, dn, max_bins, nb, sms, s) : run_pair<false, false>(gu, dn, max_bins, nb, sms, s);
+}
+
+}  // namespace moeq

@@ -17,8 +17,9 @@
 //                   lanes with the same key in the slice (ascending a inside
 //                   a bin).  It writes perm and inv_perm.
 // When all assignments fit one CTA's chunk (T*k <= 1024, decode-sized
-// batches) k_perm_one does the three steps in a single launch.  The gather
-// of activation rows (bf16 -> fp16) is its own grid-wide launch: it moves
+// batches) k_perm_one does the three steps in a single launch, and for up
+// to 64 K gathered elements the gather of activation rows too.  Otherwise
+// the gather (bf16 -> fp16) is its own grid-wide launch: it moves
 // T*k*d*2 bytes and needs every SM, while the sort needs only T*k/1024
 // CTAs.
 #include <algorithm>
@@ -182,18 +183,15 @@ __device__ __forceinline__ void scatter(const int (&keys)[kSlices], int32_t* his
   }
 }
 
-// x_perm[p] = fp16(x[perm[p] / k]): a warp per destination row, 16-byte
-// loads, four in flight per lane; grid-stride over rows.
-__global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict__ x,
-                                                 const int32_t* __restrict__ perm, int rows, int k,
-                                                 int d, __half* __restrict__ x_perm,
-                                                 int32_t* status) {
-  pdl_wait();
-  pdl_trigger();
+// x_perm[p] = fp16(x[perm[p] / k]) for rows p = first, first + stride, ...:
+// a warp per destination row, 16-byte loads, four in flight per lane.
+// Returns whether any value was outside the fp16 range.
+__device__ __forceinline__ bool gather_rows(const __nv_bfloat16* __restrict__ x, const int32_t* perm, int rows,
+                                            int k, int d, __half* __restrict__ x_perm, int first, int stride) {
   const int lane = threadIdx.x & 31;
   const int vec = d / 8;
   bool bad = false;
-  for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < rows; p += (gridDim.x * blockDim.x) >> 5) {
+  for (int p = first; p < rows; p += stride) {
     const int t = perm[p] / k;
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
     uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(p) * d);
@@ -218,7 +216,19 @@ __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict_
       }
     }
   }
-  if (bad) flag_status(status, MOE_DEV_RANGE);
+  return bad;
+}
+
+// The gather as its own grid-wide launch (large batches).
+__global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict__ x,
+                                                 const int32_t* __restrict__ perm, int rows, int k,
+                                                 int d, __half* __restrict__ x_perm,
+                                                 int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  const int first = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int stride = (gridDim.x * blockDim.x) >> 5;
+  if (gather_rows(x, perm, rows, k, d, x_perm, first, stride)) flag_status(status, MOE_DEV_RANGE);
 }
 
 __global__ void __launch_bounds__(kWarps * 32) k_perm_scatter(
@@ -250,7 +260,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_perm_scatter(
 __global__ void __launch_bounds__(kWarps * 32) k_perm_one(
     const int32_t* __restrict__ idx, const uint8_t* __restrict__ bits, int n, int E, int nbins, int k,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
-    int32_t* __restrict__ inv_perm, int32_t* status) {
+    int32_t* __restrict__ inv_perm, int32_t* status, const __nv_bfloat16* __restrict__ x, int d,
+    __half* __restrict__ x_perm) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int32_t hist_s[];  // [kWarps][nbins]
@@ -299,6 +310,10 @@ __global__ void __launch_bounds__(kWarps * 32) k_perm_one(
   if (tid == 0) offsets[nbins] = n;
   __syncthreads();
   scatter(keys, hist_s, nbins, perm, inv_perm);
+  if (x_perm) {  // small batches: the gather too (perm is visible to the block after the barrier)
+    __syncthreads();
+    if (gather_rows(x, perm, n, k, d, x_perm, warp, kWarps)) flag_status(status, MOE_DEV_RANGE);
+  }
 }
 
 int sm_count_permute() {
@@ -347,9 +362,13 @@ moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void*
     attr_set.fetch_or(bit);
   }
   moe_status_t st;
+  // one CTA gathers the rows itself when they are few (up to 64 K elements:
+  // decode-sized batches), which saves the gather launch
+  const bool fused_gather = ctas == 1 && x_perm && static_cast<long>(n) * d <= (64L << 10);
   if (ctas == 1) {
     st = cuda_check(launch_pdl(pdl_for(n), k_perm_one, dim3(1), dim3(kWarps * 32), smem, s, idx, bits, n, E, nbins, k, counts,
-                               offsets, perm, inv_perm, status),
+                               offsets, perm, inv_perm, status, static_cast<const __nv_bfloat16*>(x), d,
+                               fused_gather ? static_cast<__half*>(x_perm) : static_cast<__half*>(nullptr)),
                     "moe_permute launch");
   } else {
     st = cuda_check(launch_pdl(pdl_for(n), k_perm_hist, dim3(ctas), dim3(kWarps * 32), smem, s, idx, bits, n, E, nbins, hist, status),
@@ -362,7 +381,7 @@ moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void*
                                static_cast<const int32_t*>(hist), perm, inv_perm),
                     "moe_permute scatter launch");
   }
-  if (st != MOE_OK || !x_perm || n == 0) return st;
+  if (st != MOE_OK || !x_perm || n == 0 || fused_gather) return st;
   // a warp per row: up to 8 rows per block, at most 8 blocks per SM
   const int blocks = std::max(1, std::min((n + 7) / 8, 8 * sm_count_permute()));
   return cuda_check(launch_pdl(pdl_for(n), k_gather, dim3(blocks), dim3(256), 0, s, static_cast<const __nv_bfloat16*>(x),

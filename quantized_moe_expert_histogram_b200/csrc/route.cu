@@ -70,22 +70,25 @@ __host__ __device__ inline RouteWs route_ws(void* base, int S, int T, int E) {
   return {p, p + static_cast<size_t>(S) * T * E, p + static_cast<size_t>(S) * T * E + static_cast<size_t>(S) * T};
 }
 
+// The kLT threads of a logits tile synchronise on named barrier 1 (so that
+// a kernel with more threads can run the tile on its first kLT threads).
+__device__ __forceinline__ void tile_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kLT) : "memory"); }
+
+// Partial logits of token tile bt, expert tile be, slice `split` of d (dk
+// wide) into the workspace, by threads 0..kLT-1.
 template <int EC>
-__global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __restrict__ x,
-                                                       const float* __restrict__ wr, int T, int d, int E,
-                                                       int dk, RouteWs ws) {
-  pdl_wait();
-  pdl_trigger();
+__device__ __forceinline__ void logits_tile(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr,
+                                            int T, int d, int E, int dk, RouteWs ws, int bt, int be, int split,
+                                            float* sm) {
   using G = Tile<EC>;
-  extern __shared__ __align__(16) float sm[];
   float* xs = sm;               // [2][TT][XP]
   float* wsm = sm + 2 * G::XS;  // [2][kDC][EC]
   const int tid = threadIdx.x, lane = tid & 31;
   const int tx = lane % G::TX;
   const int ty = (tid >> 5) * G::TYW + lane / G::TX;
-  const int t0 = blockIdx.x * G::TT, e0 = blockIdx.y * EC, split = blockIdx.z;
+  const int t0 = bt * G::TT, e0 = be * EC;
   const int kbeg = split * dk, nch = dk / kDC;
-  const bool do_x = blockIdx.y == 0, do_w = blockIdx.x == 0;
+  const bool do_x = be == 0, do_w = bt == 0;
 
   // loaders: x load q covers token row (tid + kLT q) / 4, columns ((tid + kLT q) % 4) * 8 .. +8;
   // W load q covers expert (tid + kLT q) % EC, columns ((tid + kLT q) / EC) * 4 .. +4
@@ -146,7 +149,7 @@ __global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __
 
   fetch(kbeg);
   stash(0);
-  __syncthreads();
+  tile_sync();
   for (int c = 0; c < nch; ++c) {
     const int b = c & 1;
     if (c + 1 < nch) fetch(kbeg + (c + 1) * kDC);
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __
         acc[i][2 * j + 1] += cs[i][j].y;
       }
     if (c + 1 < nch) stash(b ^ 1);
-    __syncthreads();
+    tile_sync();
   }
 
   float* out = ws.partial + static_cast<size_t>(split) * T * E;
@@ -214,7 +217,7 @@ __global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __
     float* red = sm;  // reuse the stages (the loop ended with a barrier)
 #pragma unroll
     for (int q = 0; q < G::WL; ++q) red[tid + kLT * q] = wsq[q];
-    __syncthreads();
+    tile_sync();
     if (tid < EC) {
       float v = 0.f;
       for (int i = tid; i < EC * 8; i += EC) v += red[i];
@@ -222,6 +225,16 @@ __global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __
       if (e < E) ws.wsq[static_cast<size_t>(split) * E + e] = v;
     }
   }
+}
+
+template <int EC>
+__global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __restrict__ x,
+                                                       const float* __restrict__ wr, int T, int d, int E,
+                                                       int dk, RouteWs ws) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) float sm[];
+  logits_tile<EC>(x, wr, T, d, E, dk, ws, blockIdx.x, blockIdx.y, blockIdx.z, sm);
 }
 
 constexpr int kPer = 8;  // E <= 256: at most 8 experts per lane (e = lane + 32 m)
@@ -306,17 +319,16 @@ constexpr int kSelWarps = kSelThreads / 32;
 // bound among the picks (all others are certainly out) -- and the CTA's
 // warps recompute those logits in fp64; the token's warp then selects among
 // them on the fp64 values.
-__global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
+// Tokens block * kSelWarps .. + kSelWarps - 1, by all kSelThreads threads.
+__device__ __forceinline__ void select_block(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, RouteWs ws, int splits,
     const float* __restrict__ bias, const int32_t* __restrict__ forced, int T, int d, int E, int k,
-    float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w) {
-  pdl_wait();
-  pdl_trigger();
+    float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w, int block) {
   __shared__ int n_cand[kSelWarps];
   __shared__ uint8_t cand[kSelWarps][256];
   __shared__ double l64[kSelWarps][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kSelWarps + warp;
+  const int t = block * kSelWarps + warp;
   if (lane == 0) n_cand[warp] = 0;
   uint32_t contender = 0;  // lane's experts listed for fp64
   if (t < T) {
@@ -418,7 +430,7 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
   for (int item = warp; item < total; item += kSelWarps) {
     int w = 0, r = item;
     while (r >= n_cand[w]) r -= n_cand[w++];
-    const int tu = blockIdx.x * kSelWarps + w, e = cand[w][r];
+    const int tu = block * kSelWarps + w, e = cand[w][r];
     const double v = dot_bf16_f32_fp64(x + static_cast<size_t>(tu) * d, wr + static_cast<size_t>(e) * d, d, lane);
     if (lane == 0) l64[w][e] = v + (bias ? static_cast<double>(bias[e]) : 0.0);
   }
@@ -442,6 +454,37 @@ size_t route_ws_for(size_t S, int T, int E) {
 // they need exceeds `cap` bytes (one slice always remains; the error bound
 // of the logits holds for any slicing, since slices are sums of 32-product
 // chunk sums).
+
+__global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, RouteWs ws, int splits,
+    const float* __restrict__ bias, const int32_t* __restrict__ forced, int T, int d, int E, int k,
+    float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w) {
+  pdl_wait();
+  pdl_trigger();
+  select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, blockIdx.x);
+}
+
+// Both steps in one launch for decode-sized batches (one token tile, one
+// expert tile): the CTAs of one thread-block cluster take one slice of d
+// each (threads 0..kLT-1 write the slice's partial logits and norms to the
+// workspace), a cluster barrier with release/acquire semantics makes them
+// visible to the whole cluster, and the first ceil(T / kSelWarps) CTAs run
+// the selection.  Same arithmetic and order as the two-launch path.
+template <int EC>
+__global__ void __launch_bounds__(kSelThreads) k_route_small(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, RouteWs ws, int splits, int dk,
+    const float* __restrict__ bias, const int32_t* __restrict__ forced, int T, int d, int E, int k,
+    float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) float sm[];
+  const int rank = blockIdx.x;  // the grid is one cluster
+  if (threadIdx.x < kLT) logits_tile<EC>(x, wr, T, d, E, dk, ws, 0, 0, rank, sm);
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  if (rank * kSelWarps < T)
+    select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, rank);
+}
+
 int route_splits(int T, int d, int E, size_t cap = static_cast<size_t>(-1)) {
   const int ec = E <= 16 ? 16 : 64;
   const int tt = ec == 64 ? Tile<64>::TT : Tile<16>::TT;
@@ -484,6 +527,8 @@ moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d
 
 }  // namespace
 
+int g_route_fused = 1;
+
 size_t route_workspace_bytes(int T, int d, int E) {
   if (T <= 0 || d <= 0 || E <= 0) return 256;
   return route_ws_for(static_cast<size_t>(route_splits(T, d, E)), T, E);
@@ -494,6 +539,42 @@ size_t route_min_workspace_bytes(int T, int d, int E) {
   return route_ws_for(1, T, E);
 }
 
+// One-launch route for decode-sized batches: a cluster of `splits` CTAs.
+template <int EC>
+moe_status_t launch_small(const __nv_bfloat16* x, const float* wr, const float* bias, const int32_t* forced,
+                          int T, int d, int E, int k, int splits, RouteWs ws, int32_t* idx, float* w,
+                          cudaStream_t s) {
+  using G = Tile<EC>;
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_check(e, "moe_route_topk cudaGetDevice");
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (!bit || !(attr_set.load() & bit)) {
+    e = cudaFuncSetAttribute(k_route_small<EC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(G::SMEM));
+    if (e != cudaSuccess) return cuda_check(e, "moe_route_topk smem attribute");
+    attr_set.fetch_or(bit);
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(splits);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = G::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cuda_check(cudaLaunchKernelEx(&cfg, k_route_small<EC>, x, wr, ws, splits, d / splits, bias, forced, T, d, E,
+                                       k, route_gamma(d), idx, w),
+                    "moe_route_topk fused launch");
+}
+
 moe_status_t launch_route(const void* x, const float* w_router, const float* bias,
                           const int32_t* forced, int T, int d, int E, int k, int32_t* idx,
                           float* w, void* workspace, size_t workspace_bytes, cudaStream_t s) {
@@ -501,6 +582,14 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
   const int splits = route_splits(T, d, E, workspace_bytes);
   const RouteWs ws = route_ws(workspace, splits, T, E);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  // decode-sized batches: one token tile and one expert tile, a cluster of
+  // up to 8 CTAs over d, selection in the same launch
+  const int fused_splits = std::min(splits, 8);
+  if (T <= kSelWarps * fused_splits && E <= 64 && fused_splits >= 2 && g_route_fused) {
+    const RouteWs wsf = route_ws(workspace, fused_splits, T, E);
+    return E <= 16 ? launch_small<16>(xb, w_router, bias, forced, T, d, E, k, fused_splits, wsf, idx, w, s)
+                   : launch_small<64>(xb, w_router, bias, forced, T, d, E, k, fused_splits, wsf, idx, w, s);
+  }
   moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, k, splits, ws, s)
                             : launch_logits<64>(xb, w_router, T, d, E, k, splits, ws, s);
   if (st != MOE_OK) return st;
@@ -560,6 +649,8 @@ moe_status_t route_scratch(void** out) {
 
 }  // namespace
 }  // namespace moeq
+
+extern "C" void moe_debug_route_fused(int enable) { moeq::g_route_fused = enable ? 1 : 0; }
 
 extern "C" moe_status_t moe_route_topk_noalloc(const void* x, const float* w_router, const float* bias,
                                                 const int32_t* forced_idx, int T, int d, int E, int k,

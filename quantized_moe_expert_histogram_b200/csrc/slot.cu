@@ -60,6 +60,11 @@ struct moe_slot_cache {
   std::vector<std::vector<int>> wave_slots;      // slot of each expert of the wave
   int copies_issued = 0;                         // waves whose copies were issued
   bool staged = false;  // a plan is staged and its moe_slot_ffn has not run yet
+  // busy-time measurement (moe_slot_timing): event pairs around each wave's
+  // copies and each wave's FFN, recorded after the waits on the other stream
+  bool timing = false;
+  std::vector<cudaEvent_t> tev[2];  // [0] copies, [1] FFN: start, end, start, end, ...
+  size_t tev_used[2] = {0, 0};
   int64_t stats[3] = {0, 0, 0};
 };
 
@@ -80,10 +85,25 @@ void invalidate_from(moe_slot_cache* c, int w) {
   c->staged = false;
 }
 
+// Record the next timing event of kind k (0 copies, 1 FFN) on stream s.
+moe_status_t timing_mark(moe_slot_cache* c, int k, cudaStream_t s) {
+  if (!c->timing) return MOE_OK;
+  auto& v = c->tev[k];
+  if (c->tev_used[k] == v.size()) {
+    cudaEvent_t e = nullptr;
+    moe_status_t st = cuda_check(cudaEventCreate(&e), "timing event");
+    if (st != MOE_OK) return st;
+    v.push_back(e);
+  }
+  return cuda_check(cudaEventRecord(v[c->tev_used[k]++], s), "timing event record");
+}
+
 moe_status_t issue_copies(moe_slot_cache* c, int w, cudaStream_t copy) {
   const auto& slots = c->wave_slots[w];
   const auto& exps = c->waves[w];
-  bool any = false;
+  // the wave's copies: first every wait for a slot to be free, then the
+  // copies back to back (so that their busy time can be measured alone)
+  std::vector<std::pair<int, int>> todo;  // (expert, slot)
   for (size_t i = 0; i < exps.size(); ++i) {
     const int e = exps[i];
     if (std::find(c->wave_misses[w].begin(), c->wave_misses[w].end(), e) == c->wave_misses[w].end())
@@ -97,17 +117,22 @@ moe_status_t issue_copies(moe_slot_cache* c, int w, cudaStream_t copy) {
       moe_status_t st = cuda_check(cudaStreamWaitEvent(copy, c->slot_free[s], 0), "slot wait free");
       if (st != MOE_OK) return st;
     }
-    moe_status_t st = cuda_check(
-        cudaMemcpyAsync(c->pool + static_cast<size_t>(s) * c->blob_bytes,
-                        c->host + static_cast<size_t>(e) * c->blob_bytes, c->blob_bytes,
-                        cudaMemcpyHostToDevice, copy),
-        "slot H2D copy");
-    if (st != MOE_OK) return st;
-    any = true;
+    todo.emplace_back(e, s);
   }
-  c->copy_pending[w] = any;
-  if (any) return cuda_check(cudaEventRecord(c->copy_done[w], copy), "slot copy event");
-  return MOE_OK;
+  c->copy_pending[w] = !todo.empty();
+  if (todo.empty()) return MOE_OK;
+  moe_status_t st = timing_mark(c, 0, copy);
+  if (st != MOE_OK) return st;
+  for (const auto& es : todo) {
+    st = cuda_check(cudaMemcpyAsync(c->pool + static_cast<size_t>(es.second) * c->blob_bytes,
+                                    c->host + static_cast<size_t>(es.first) * c->blob_bytes, c->blob_bytes,
+                                    cudaMemcpyHostToDevice, copy),
+                    "slot H2D copy");
+    if (st != MOE_OK) return st;
+  }
+  st = timing_mark(c, 0, copy);
+  if (st != MOE_OK) return st;
+  return cuda_check(cudaEventRecord(c->copy_done[w], copy), "slot copy event");
 }
 
 }  // namespace
@@ -192,9 +217,46 @@ void moe_slot_cache_destroy(moe_slot_cache* c) {
     cudaEventSynchronize(c->prefetch_done);
     cudaEventDestroy(c->prefetch_done);
   }
+  for (int k = 0; k < 2; ++k)
+    for (auto e : c->tev[k]) {
+      cudaEventSynchronize(e);
+      cudaEventDestroy(e);
+    }
   if (c->d_tables) cudaFree(c->d_tables);
   if (c->h_tables) cudaFreeHost(c->h_tables);
   delete c;
+}
+
+moe_status_t moe_slot_timing(moe_slot_cache* c, int enable) {
+  if (!c) {
+    set_error("moe_slot_timing: null cache");
+    return MOE_ERR_INVALID_ARG;
+  }
+  c->timing = enable != 0;
+  c->tev_used[0] = c->tev_used[1] = 0;
+  return MOE_OK;
+}
+
+moe_status_t moe_slot_timing_read(moe_slot_cache* c, double* copy_ms, double* ffn_ms) {
+  if (!c || !copy_ms || !ffn_ms) {
+    set_error("moe_slot_timing_read: bad arguments");
+    return MOE_ERR_INVALID_ARG;
+  }
+  double sum[2] = {0.0, 0.0};
+  for (int k = 0; k < 2; ++k) {
+    for (size_t i = 0; i + 1 < c->tev_used[k]; i += 2) {
+      moe_status_t st = cuda_check(cudaEventSynchronize(c->tev[k][i + 1]), "timing event wait");
+      if (st != MOE_OK) return st;
+      float ms = 0.f;
+      st = cuda_check(cudaEventElapsedTime(&ms, c->tev[k][i], c->tev[k][i + 1]), "timing elapsed");
+      if (st != MOE_OK) return st;
+      sum[k] += ms;
+    }
+    c->tev_used[k] = 0;
+  }
+  *copy_ms = sum[0];
+  *ffn_ms = sum[1];
+  return MOE_OK;
 }
 
 moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_ids,
@@ -410,8 +472,12 @@ moe_status_t moe_slot_ffn(moe_slot_cache* c, const void* x_perm, const int32_t* 
       if (st != MOE_OK) return st;
       c->tables_done_valid = true;
     }
+    st = timing_mark(c, 1, S(compute_stream));
+    if (st != MOE_OK) return st;
     st = moe_grouped_ffn_wq(x_perm, offsets, c->pool, dt, total_rows, T, c->E, d, F, group, layout,
                             workspace, workspace_bytes, y_perm, status, compute_stream);
+    if (st != MOE_OK) return st;
+    st = timing_mark(c, 1, S(compute_stream));
     if (st != MOE_OK) return st;
     for (int s : c->wave_slots[w]) {
       st = cuda_check(cudaEventRecord(c->slot_free[s], S(compute_stream)), "slot free event");

@@ -127,14 +127,15 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: only reached when some
 // timeout, or by another role).
 // Where the first timeout of a CTA happened (test hook, see trace_put).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status, int* trace = nullptr, uint32_t bar0 = 0) {
+                                          int32_t* status, int* trace = nullptr, uint32_t bar0 = 0,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_sleep(bar, parity, 20000u)) return true;
     if ((i & 7) == 0) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         flag_status(status, MOE_DEV_TIMEOUT);
         if (trace) {  // slot 8: barrier index and parity of the wait that gave up
@@ -152,8 +153,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // warp reconverges and agrees on the outcome, so the warp-aligned
 // instructions that follow (tcgen05.ld, barriers) run converged.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status, int* trace = nullptr, uint32_t bar0 = 0) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, status, trace, bar0);
+                                          int32_t* status, int* trace = nullptr, uint32_t bar0 = 0,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status, trace, bar0, limit_ns);
   __syncwarp();
   return __all_sync(0xffffffffu, ok);
 }
@@ -319,6 +321,8 @@ struct TcParams {
   __half* y_out;
   int32_t* status;
   int* trace;  // optional progress record (null in normal use)
+  uint64_t wait_ns;  // limit of every wait (2 s; shorter under the timeout test hook)
+  int debug_stall;   // test hook: CTA 0's epilogue withholds its first accumulator release
 };
 
 struct Tile {
@@ -534,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
           if (PLANES) code_bytes = 4096 + (T.bits >= 3 ? 2048 : 0) + (T.bits >= 4 ? 2048 : 0);
           for (int kc = 0; kc < KC && ok; ++kc) {
             trace_put(trace, 0, 1, t, kc);
-            ok = mbar_wait(codes_empty(cs), cph ^ 1, abort_flag, P.status, trace, bar0);
+            ok = mbar_wait(codes_empty(cs), cph ^ 1, abort_flag, P.status, trace, bar0, P.wait_ns);
             if (!ok) break;
             mbar_expect_tx(codes_full(cs), nm * (code_bytes + gpc * 512));
             for (int m = 0; m < nm; ++m) {
@@ -560,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         } else {
           for (int kb = 0; kb < 2 * KC && ok; ++kb) {
             trace_put(trace, 2, 2, t, kb);
-            ok = mbar_wait(b_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
+            ok = mbar_wait(b_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0, P.wait_ns);
             if (!ok) break;
             // one 128-row box: rows past this tile's are loaded but not read
             // by the MMA (N = nt); rows past the tensor are zero-filled
@@ -577,12 +581,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         if (codes_role) {
           for (int idx = 0; idx < C::CSTAGES; ++idx) {
             const int ph = (idx < cs) ? cph : cph ^ 1;
-            while (!mbar_try(codes_full(idx), ph) && global_ns() - t0 < kWaitLimitNs) {}
+            while (!mbar_try(codes_full(idx), ph) && global_ns() - t0 < P.wait_ns) {}
           }
         } else {
           for (int idx = 0; idx < C::SB; ++idx) {
             const int ph = (idx < s) ? sph : sph ^ 1;
-            while (!mbar_try(b_full(idx), ph) && global_ns() - t0 < kWaitLimitNs) {}
+            while (!mbar_try(b_full(idx), ph) && global_ns() - t0 < P.wait_ns) {}
           }
         }
       }
@@ -598,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         const uint32_t idesc = umma_idesc_f16(T.nt);
         const int nm = has_m1(T.mb) ? 2 : 1;
         if (lane == 0) trace_put(trace, 1, 3, t, 0);
-        ok = warp_wait(acc_empty(acc), aph ^ 1, abort_flag, P.status, trace, bar0);
+        ok = warp_wait(acc_empty(acc), aph ^ 1, abort_flag, P.status, trace, bar0, P.wait_ns);
         if (!ok) break;
         tc_fence_after();
         const uint32_t dcol = tmem_base + acc * (2 * kNT);
@@ -607,9 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         const uint64_t bdesc0 = umma_desc_sw128(smem_u32(smem + C::OFF_B));
         const uint32_t acol0 = tmem_base + C::ACOL;
         for (int kb = 0; kb < 2 * KC && ok; ++kb) {
-          ok = warp_wait(a_full(sa), saph, abort_flag, P.status, trace, bar0);
+          ok = warp_wait(a_full(sa), saph, abort_flag, P.status, trace, bar0, P.wait_ns);
           if (!ok) break;
-          ok = warp_wait(b_full(sb), sbph, abort_flag, P.status, trace, bar0);
+          ok = warp_wait(b_full(sb), sbph, abort_flag, P.status, trace, bar0, P.wait_ns);
           if (!ok) break;
           tc_fence_after();
           const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(sb * (C::B_BYTES >> 4));
@@ -638,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       // all MMAs issued by this thread complete before TMEM is released
       umma_commit_elect(drain_bar);
       const uint64_t t0 = global_ns();
-      while (!mbar_try(drain_bar, 0) && global_ns() - t0 < kWaitLimitNs) {}
+      while (!mbar_try(drain_bar, 0) && global_ns() - t0 < P.wait_ns) {}
       __syncwarp();
     }
   }
@@ -654,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       const bool live = m == 0 || has_m1(T.mb);  // matrix 1 may be absent in the last W_down block
       for (int kc = 0; kc < KC && ok; ++kc) {
         if (lane == 0) trace_put(trace, 3 + m, 6, t, kc);
-        ok = warp_wait(codes_full(cs), cph, abort_flag, P.status, trace, bar0);
+        ok = warp_wait(codes_full(cs), cph, abort_flag, P.status, trace, bar0, P.wait_ns);
         if (!ok) break;
         const uint8_t* cb = smem + C::OFF_C + (cs * 2 + m) * C::C_BYTES;
         uint32_t w[16];
@@ -705,7 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
         if (++cs == C::CSTAGES) { cs = 0; cph ^= 1; }
         for (int h = 0; h < 2 && ok; ++h) {
           if (lane == 0) trace_put(trace, 3 + m, 7, t, 2 * kc + h);
-          ok = warp_wait(a_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0);
+          ok = warp_wait(a_empty(s), sph ^ 1, abort_flag, P.status, trace, bar0, P.wait_ns);
           if (!ok) break;
           tc_fence_after();  // the MMAs that read this stage have completed
           if (live) {
@@ -741,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       const Tile T = decode_tile(t, tile_start, off_s, nbins, MB, P.planes_mult, P.slot_of);
       const bool m1 = has_m1(T.mb);
       if (lane == 0) trace_put(trace, 5, 8, t, 0);
-      ok = warp_wait(acc_full(acc), aph, abort_flag, P.status, trace, bar0);
+      ok = warp_wait(acc_full(acc), aph, abort_flag, P.status, trace, bar0, P.wait_ns);
       if (!ok) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * (2 * kNT);
@@ -808,11 +812,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       // accumulators read: the MMA may start the next tile
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty(acc));
+      // (test hook: withheld once, so that the MMA warp's wait for the next
+      // tile's accumulators runs out -- the arrive has no copy behind it)
+      const bool withhold = GATEUP && P.debug_stall && blockIdx.x == 0 && t == static_cast<int>(blockIdx.x);
+      if (lane == 0 && !withhold) mbar_arrive(acc_empty(acc));
       if (++acc == C::ACC) { acc = 0; aph ^= 1; }
       // all four warps have staged their rows
       if (lane == 0) mbar_arrive(epi_bar);
-      ok = warp_wait(epi_bar, ep_ph, abort_flag, P.status, trace, bar0);
+      ok = warp_wait(epi_bar, ep_ph, abort_flag, P.status, trace, bar0, P.wait_ns);
       ep_ph ^= 1;
       if (!ok) break;
       // 16-byte stores of the staged rows (tokens) that belong to this tile
@@ -847,7 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
       if (C::OUT_BUFS == 1) {
         // a single buffer is rewritten by the next tile: wait for every warp's copy
         if (lane == 0) mbar_arrive(epi_bar);
-        ok = warp_wait(epi_bar, ep_ph, abort_flag, P.status, trace, bar0);
+        ok = warp_wait(epi_bar, ep_ph, abort_flag, P.status, trace, bar0, P.wait_ns);
         ep_ph ^= 1;
         if (!ok) break;
       }
@@ -864,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
     if (lane == 0) trace_put(trace, 7, 14, 0, 0);
     {  // not cut short by an abort: every warp must have left before TMEM goes
       const uint64_t t0 = global_ns();
-      while (!mbar_try(exit_bar, 0) && global_ns() - t0 < kWaitLimitNs) {}
+      while (!mbar_try(exit_bar, 0) && global_ns() - t0 < P.wait_ns) {}
       __syncwarp();
     }
     tc_fence_after();
@@ -900,6 +907,7 @@ bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, 
 }
 
 int* g_trace = nullptr;  // test hook: host-mapped progress record
+int g_debug_stall = 0;   // test hook: a withheld arrive and a 20 ms wait limit
 
 // SM count of the current device (cached per device).
 int sm_count() {
@@ -971,6 +979,8 @@ moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int r
   P.group = a.group;
   P.status = a.status;
   P.trace = g_trace;
+  P.wait_ns = g_debug_stall ? 20000000ull : kWaitLimitNs;
+  P.debug_stall = g_debug_stall;
   return MOE_OK;
 }
 
@@ -1025,3 +1035,5 @@ moe_status_t launch_ffn_tc(const FfnArgs& a, cudaStream_t s) {
 extern "C" void moe_debug_set_trace(void* host_mapped_ints) {
   moeq::g_trace = static_cast<int*>(host_mapped_ints);
 }
+
+extern "C" void moe_debug_ffn_timeout(int enable) { moeq::g_debug_stall = enable ? 1 : 0; }

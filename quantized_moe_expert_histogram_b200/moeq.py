@@ -51,6 +51,8 @@ _SIGS = {
                             _c_p, _c_p, _c_p]),
     "moe_slot_cache_destroy": (None, [_c_p]),
     "moe_slot_prefetch": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_p, _c_p]),
+    "moe_slot_timing": (_c_i, [_c_p, _c_i]),
+    "moe_slot_timing_read": (_c_i, [_c_p, _c_p, _c_p]),
     "moe_predictor_create": (_c_i, [_c_i, _c_i, ctypes.POINTER(_c_p)]),
     "moe_predictor_destroy": (None, [_c_p]),
     "moe_predictor_observe": (_c_i, [_c_p, _c_i, _c_p, _c_p, _c_i, _c_i]),
@@ -58,6 +60,8 @@ _SIGS = {
     "moe_debug_inject_fault": (None, [_c_i, _c_i]),
     "moe_debug_force_regime": (None, [_c_i]),
     "moe_debug_set_trace": (None, [_c_p]),
+    "moe_debug_ffn_timeout": (None, [_c_i]),
+    "moe_debug_route_fused": (None, [_c_i]),
 }
 
 _lib = None
@@ -296,6 +300,14 @@ class SlotCache:
         ahead of their layer-step; returns the number of copies issued."""
         return moe_slot_prefetch(self.handle, ids_host, max_copies, copy_stream)
 
+    def timing(self, enable):
+        """moe_slot_timing: record copy and FFN busy time from now on."""
+        moe_slot_timing(self.handle, enable)
+
+    def timing_read(self):
+        """moe_slot_timing_read: (copy_ms, ffn_ms) since the last read."""
+        return moe_slot_timing_read(self.handle)
+
     def close(self):
         if self.handle is not None and self.handle.value:
             load().moe_slot_cache_destroy(self.handle)
@@ -314,6 +326,16 @@ def moe_slot_prefetch(handle, ids_host, max_copies, copy_stream):
     _check("moe_slot_prefetch", load().moe_slot_prefetch(handle, ids.data_ptr(), ids.numel(), int(max_copies),
                                                           copy_stream.cuda_stream, ctypes.byref(n)))
     return n.value
+
+
+def moe_slot_timing(handle, enable):
+    _check("moe_slot_timing", load().moe_slot_timing(handle, int(bool(enable))))
+
+
+def moe_slot_timing_read(handle):
+    cm, fm = ctypes.c_double(0), ctypes.c_double(0)
+    _check("moe_slot_timing_read", load().moe_slot_timing_read(handle, ctypes.addressof(cm), ctypes.addressof(fm)))
+    return cm.value, fm.value
 
 
 def moe_predictor_create(layers, E):
@@ -379,6 +401,16 @@ def moe_last_error():
 def moe_debug_force_regime(regime):
     """0 = by T, 1 = one-token GEMV, 2 = tensor cores, 3 = small-batch mma.sync kernel (test hook)."""
     load().moe_debug_force_regime(regime)
+
+
+def moe_debug_route_fused(enable):
+    """Test hook: 0 forces the two-launch router for small batches."""
+    load().moe_debug_route_fused(int(bool(enable)))
+
+
+def moe_debug_ffn_timeout(enable):
+    """Test hook: a withheld arrive and a 20 ms wait limit in the tensor-core FFN."""
+    load().moe_debug_ffn_timeout(int(bool(enable)))
 
 
 def moe_debug_set_trace(pinned_int32=None):

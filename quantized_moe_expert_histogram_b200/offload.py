@@ -7,18 +7,32 @@ token count, in waves of half the slots) and ``moe_slot_ffn`` runs the
 grouped FFN wave by wave as the copies land.  Pages: ExactMoE (compressed
 experts in host memory, GPU-resident slot cache, every routed expert
 executed), EdgeMoE (expert buffer filled on activation), D2MoE (loading the
-next expert while computing the current one).
+next expert while computing the current one), Read-ME (a pre-gating router
+decoupled from the backbone decides every layer's experts before the layers
+compute, which allows lookahead scheduling of expert loads).
 
-``OffloadStack.step`` runs one decode step through all layers: route (the
-expert ids may be forced from a trace), the one device-to-host copy of the
-routed ids per layer, stage, permute, slot FFN, combine with the residual.
-With ``prefetch`` (EdgeMoE's expert preloading), once layer l's ids are
-known a host predictor (moe_predictor_*, counts of consecutive-layer expert
-pairs learned online) names layer l+1's likely experts and
-``moe_slot_prefetch`` copies the confident ones (expected to receive at
-least one assignment; at most a quarter of a cache) into layer l+1's
-slots on the copy stream, behind layer l's own copies, so that they land
-while layer l computes.
+``OffloadStack.step`` runs one decode step through all layers in one of
+two schedules:
+
+* per-layer routing (``lookahead=False``): route layer l (the expert ids may
+  be forced from a trace), one device-to-host copy of the routed ids and a
+  host wait per layer, stage, permute, slot FFN, combine with the residual.
+  With ``prefetch`` (EdgeMoE's expert preloading), once layer l's ids are
+  known a host predictor (moe_predictor_*) names layer l+1's likely experts
+  and ``moe_slot_prefetch`` copies the confident ones (expected to receive
+  at least one assignment; at most a quarter of a cache) into layer l+1's
+  slots behind layer l's own copies.
+* lookahead (``lookahead=True``, Read-ME's pre-gating): every layer's
+  expert ids for the step are known before the first layer computes -- the
+  forced trace, or, without one, each layer's router applied to the step's
+  input -- and reach the host in one copy per step.  The host then plans
+  and enqueues every layer's staging and FFN back to back with no further
+  wait, so layer l+1's copies are queued while layer l computes; layers
+  alternate between two copy streams so that one layer's later waves (which
+  wait for its own compute to free slots) do not hold back the next layer's
+  first copies.  Gates still come from each layer's router logits at the
+  given ids (the layer's own input), so the results equal the resident path
+  fed the same ids.
 This module only orchestrates calls of the C ABI; torch supplies device
 memory, pinned host memory and streams.
 """
@@ -33,9 +47,9 @@ from .layer import QuantMoELayer
 
 class OffloadStack:
     def __init__(self, shape, layers: int, slots: int, batch: int, seed: int = 0, device="cuda",
-                 prefetch: bool = False):
+                 prefetch: bool = False, lookahead: bool = False):
         self.shape, self.n_layers, self.slots, self.batch = shape, layers, slots, batch
-        self.prefetch = prefetch
+        self.prefetch, self.lookahead = prefetch, lookahead
         self.predictor = moeq.RoutePredictor(layers, shape.E) if prefetch else None
         self.prefetched = 0
         self.layers, self.host, self.pools, self.caches = [], [], [], []
@@ -54,27 +68,68 @@ class OffloadStack:
             self.caches.append(moeq.SlotCache(shape.E, slots, host.shape[1], host, pool))
         self.blob_bytes = self.host[0].shape[1]
         self.copy = torch.cuda.Stream()
+        self.copy2 = torch.cuda.Stream()  # lookahead: odd layers' copies
+        self.side = torch.cuda.Stream()   # lookahead: the per-step id copy
         self.compute = torch.cuda.current_stream()
         self.ids_host = [torch.empty(batch, shape.k, dtype=torch.int32).pin_memory() for _ in range(layers)]
+        self.ids_all_host = torch.empty(layers, batch, shape.k, dtype=torch.int32).pin_memory()
+        self.ids_pregated = torch.empty(layers, batch, shape.k, dtype=torch.int32, device=device)
+        self._marks = None  # busy-time events of the compute stream's own segments
+
+    def timing(self, enable: bool):
+        """Record busy time from now on: each cache's copies and FFN waves
+        (moe_slot_timing) and, on the compute stream, the route + permute and
+        combine segments (wait-free, so event pairs measure their work)."""
+        for c in self.caches:
+            c.timing(enable)
+        self._marks = [] if enable else None
+
+    def timing_read(self):
+        """(copy_ms, compute_ms) since timing(True) or the last read."""
+        copy_ms = ffn_ms = 0.0
+        for c in self.caches:
+            cm, fm = c.timing_read()
+            copy_ms, ffn_ms = copy_ms + cm, ffn_ms + fm
+        seg = 0.0
+        if self._marks:
+            self._marks[-1][1].synchronize()
+            seg = sum(a.elapsed_time(b) for a, b in self._marks)
+            self._marks = []
+        return copy_ms, ffn_ms + seg
+
+    def _mark(self):
+        if self._marks is None:
+            return None
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(self.compute)
+        return ev
+
+    def _segment(self, start):
+        if start is not None:
+            self._marks.append((start, self._mark()))
 
     def step(self, x, forced_ids=None):
         """One decode step of the batch x (bf16 [batch][d]) through all layers.
         forced_ids: int32 [layers][batch][k] on the device, or None (the
         routers decide).  Returns (y, per-layer [hits, misses, bytes, waves])."""
+        if self.lookahead:
+            return self._step_lookahead(x, forced_ids)
         sh, stats = self.shape, []
         for l, layer in enumerate(self.layers):
             v = layer.views(self.batch)
+            t0 = self._mark()
             moeq.moe_route_topk(x, layer.w_router, layer.bias, sh.k,
                                 forced_idx=None if forced_ids is None else forced_ids[l].contiguous(),
                                 topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"])
             moeq.moe_permute(v["topk_idx"], sh.E, x=x, out=v, status=v["status"])
+            self._segment(t0)
             # the one device -> host crossing per layer: the routed ids
             self.ids_host[l].copy_(v["topk_idx"], non_blocking=True)
             self.compute.synchronize()
             n_waves, st = self.caches[l].stage(self.ids_host[l].reshape(-1), self.copy, self.compute)
             self.caches[l].ffn(v["x_perm"], v["offsets"], self.batch, sh.d, sh.F, sh.group, layer.layout,
                                v["workspace"], v["y_perm"], v["status"], self.copy, self.compute)
-            if self.predictor is not None:
+            if self.prefetch and self.predictor is not None:
                 if l > 0:
                     self.predictor.observe(l, self.ids_host[l - 1], self.ids_host[l])
                 if l + 1 < self.n_layers:
@@ -84,7 +139,47 @@ class OffloadStack:
                     if pred.numel():
                         self.prefetched += self.caches[l + 1].prefetch(pred, self.slots // 4, self.copy)
             y = torch.empty_like(x)
+            t0 = self._mark()
             moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], residual=x, y=y)
+            self._segment(t0)
+            stats.append(st + [n_waves])
+            x = y
+        return x, stats
+
+    def pregate(self, x):
+        """Every layer's expert ids for the step from the step's input (each
+        layer's router applied to x): int32 [layers][batch][k] on the device."""
+        for l, layer in enumerate(self.layers):
+            v = layer.views(self.batch)
+            moeq.moe_route_topk(x, layer.w_router, layer.bias, self.shape.k, topk_idx=self.ids_pregated[l],
+                                topk_w=v["topk_w"], workspace=v["route_ws"])
+        return self.ids_pregated
+
+    def _step_lookahead(self, x, forced_ids):
+        sh, stats = self.shape, []
+        ids = self.pregate(x) if forced_ids is None else forced_ids
+        # the one device -> host crossing per step: all layers' ids
+        ev = torch.cuda.Event()
+        ev.record(self.compute)
+        self.side.wait_event(ev)
+        with torch.cuda.stream(self.side):
+            self.ids_all_host.copy_(ids, non_blocking=True)
+        self.side.synchronize()
+        for l, layer in enumerate(self.layers):
+            copy = self.copy if l % 2 == 0 else self.copy2
+            v = layer.views(self.batch)
+            t0 = self._mark()
+            moeq.moe_route_topk(x, layer.w_router, layer.bias, sh.k, forced_idx=ids[l].contiguous(),
+                                topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"])
+            moeq.moe_permute(v["topk_idx"], sh.E, x=x, out=v, status=v["status"])
+            self._segment(t0)
+            n_waves, st = self.caches[l].stage(self.ids_all_host[l].reshape(-1), copy, self.compute)
+            self.caches[l].ffn(v["x_perm"], v["offsets"], self.batch, sh.d, sh.F, sh.group, layer.layout,
+                               v["workspace"], v["y_perm"], v["status"], copy, self.compute)
+            y = torch.empty_like(x)
+            t0 = self._mark()
+            moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], residual=x, y=y)
+            self._segment(t0)
             stats.append(st + [n_waves])
             x = y
         return x, stats

@@ -65,6 +65,30 @@ def test_route_bitexact(name, T, dup):
     np.testing.assert_allclose(w.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
 
 
+@pytest.mark.parametrize("name,T", [("olmoe", 1), ("olmoe", 8), ("olmoe", 33), ("olmoe", 64), ("nested", 1),
+                                    ("nested", 17), ("mixtral", 1), ("tiny", 64)])
+def test_route_fused_small_batches(name, T):
+    """Decode-sized batches run the router as one cluster launch; its expert
+    ids equal the two-launch router's and the oracle's bit for bit, its gates
+    match the oracle's."""
+    shape = I.SHAPES[name]
+    L = I.make_layer(shape, T, seed=17, weights=False)
+    bias = L["bias"].cuda() if L["bias"] is not None else None
+    x, wr = L["x"].cuda(), L["w_router"].cuda()
+    idx_f, w_f = moeq.moe_route_topk(x, wr, bias, shape.k)
+    moeq.moe_debug_route_fused(0)
+    try:
+        idx_2, _ = moeq.moe_route_topk(x, wr, bias, shape.k)
+    finally:
+        moeq.moe_debug_route_fused(1)
+    torch.cuda.synchronize()
+    sel, gates, _ = O.route(L["x"].float().numpy(), L["w_router"].numpy(),
+                            None if L["bias"] is None else L["bias"].numpy(), shape.k)
+    np.testing.assert_array_equal(idx_f.cpu().numpy(), sel)
+    np.testing.assert_array_equal(idx_2.cpu().numpy(), sel)
+    np.testing.assert_allclose(w_f.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
+
+
 @pytest.mark.parametrize("scale", [0.0, 1e-9, 1e-7, 1e-5])
 def test_route_near_ties_resolved_exactly(scale):
     """Router rows that are copies of others plus a perturbation of the given

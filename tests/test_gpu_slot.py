@@ -149,15 +149,18 @@ def test_slot_cache_rejects_bad_arguments():
     st.close()
 
 
-@pytest.mark.parametrize("prefetch", [False, True])
-def test_offload_stack_equals_resident(prefetch):
+@pytest.mark.parametrize("mode", ["sync", "prefetch", "lookahead"])
+def test_offload_stack_equals_resident(mode):
     """The packaged offload driver (experts only in pinned host memory, the
-    device copies of the blobs dropped), with and without predictive
-    prefetching of the next layer's experts, gives the resident path's
-    outputs bit for bit, layer after layer."""
+    device copies of the blobs dropped) in each schedule -- a routed-id sync
+    per layer, that plus predictive prefetching of the next layer's experts,
+    and lookahead (all layers' ids known up front, no per-layer sync) --
+    gives the resident path's outputs bit for bit, layer after layer."""
+    prefetch = mode == "prefetch"
     shape = I.custom_shape(d=256, E=16, k=4, F=256, group=64)
     ref = Stack(shape, layers=3, slots=8, batch=8, seed=5)
-    off = OffloadStack(shape, layers=3, slots=8, batch=8, seed=5, prefetch=prefetch)
+    off = OffloadStack(shape, layers=3, slots=8, batch=8, seed=5, prefetch=prefetch,
+                       lookahead=mode == "lookahead")
     steps = 6
     trace = I.make_slot_trace(shape.E, shape.k, 3, steps=steps, batch=8, seed=6).cuda()
     xs_all = I.make_slot_x(shape.d, steps, 8, seed=6, device="cuda")
@@ -176,14 +179,15 @@ def test_offload_stack_equals_resident(prefetch):
     off.close()
 
 
-@pytest.mark.parametrize("prefetch", [False, True])
-def test_offload_olmoe_shaped_stack_equals_resident(prefetch):
+@pytest.mark.parametrize("mode", ["sync", "prefetch", "lookahead"])
+def test_offload_olmoe_shaped_stack_equals_resident(mode):
     """The offload driver on the layer shape the benchmark times (OLMoE-shaped:
     d 2048, 64 experts, top-8, d_ff 1024, 16 slots, batch 8; two layers, four
     steps) gives the resident path's outputs bit for bit."""
     shape = I.SHAPES["olmoe"]
     ref = Stack(shape, layers=2, slots=16, batch=8, seed=7)
-    off = OffloadStack(shape, layers=2, slots=16, batch=8, seed=7, prefetch=prefetch)
+    off = OffloadStack(shape, layers=2, slots=16, batch=8, seed=7, prefetch=mode == "prefetch",
+                       lookahead=mode == "lookahead")
     steps = 4
     trace = I.make_slot_trace(shape.E, shape.k, 2, steps=steps, batch=8, seed=8).cuda()
     xs_all = I.make_slot_x(shape.d, steps, 8, seed=8, device="cuda")
@@ -230,3 +234,25 @@ def test_prefetch_between_stage_and_ffn_is_rejected():
     for l in range(3):
         assert torch.equal(ys_o[l], ys_ref[l])
     st.close()
+
+
+def test_lookahead_pregated_ids_equal_resident():
+    """Lookahead without a trace: every layer's ids come from its router
+    applied to the step's input (pre-gating), fetched to the host once per
+    step; the stack's outputs equal the resident path fed those ids, and each
+    layer's ids are the top-k of its router on the step input."""
+    shape = I.custom_shape(d=256, E=16, k=4, F=256, group=64)
+    ref = Stack(shape, layers=3, slots=8, batch=8, seed=5)
+    off = OffloadStack(shape, layers=3, slots=8, batch=8, seed=5, lookahead=True)
+    xs_all = I.make_slot_x(shape.d, 3, 8, seed=11, device="cuda")
+    for s in range(3):
+        y_o, _ = off.step(xs_all[s], None)
+        torch.cuda.synchronize()
+        ids = off.ids_pregated.clone()
+        for l, (layer, _) in enumerate(ref.layers):
+            sel, _, _ = O.route(xs_all[s].float().cpu().numpy(), layer.w_router.cpu().numpy(), None, shape.k)
+            np.testing.assert_array_equal(ids[l].cpu().numpy(), sel)
+        _, ys_r, _ = ref.step(xs_all[s], ids, offload=False)
+        assert torch.equal(y_o, ys_r[-1]), f"step {s}"
+    ref.close()
+    off.close()
