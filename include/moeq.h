@@ -333,21 +333,28 @@ MOE_API moe_status_t moe_slot_prefetch(moe_slot_cache* cache, const int32_t* ids
 MOE_API moe_status_t moe_slot_timing(moe_slot_cache* cache, int enable);
 MOE_API moe_status_t moe_slot_timing_read(moe_slot_cache* cache, double* copy_ms, double* ffn_ms);
 
-/* Next-layer expert predictor (host-only): counts of (expert at layer l-1,
- * expert at layer l) pairs at the same token and choice position, learned
- * online with moe_predictor_observe; moe_predictor_predict scores experts
- * of `layer` from the routed ids of layer-1 (sum of the conditional
- * frequencies: the expected number of assignments to each expert) and
- * writes up to max_out ids, best first (ties: lower id), only experts whose
- * score is nonzero and at least min_score.  ids are host int32 [T][k]. */
+/* Next-layer expert predictor (host-only; [EdgeMoE] expert preloading: a
+ * statistical profile keyed by the experts activated at the two preceding
+ * layers, experts preloaded in order of their estimated probability).
+ * Learned online with moe_predictor_observe from the routed ids of earlier
+ * steps, per token and choice position j: counts of (expert at layer-1 ->
+ * expert at layer) and, when prev2_ids is given and E <= 64, of
+ * ((expert at layer-2, expert at layer-1) -> expert at layer).
+ * moe_predictor_predict scores the experts of `layer` by the summed
+ * conditional frequencies (the expected number of assignments to each
+ * expert), using the pair key for a pair seen at least twice and the
+ * one-layer key otherwise, and writes up to max_out ids, best first (ties:
+ * lower id), only experts whose score is nonzero and at least min_score.
+ * ids are host int32 [T][k]; prev2_ids may be NULL (one-layer key only) and
+ * needs layer >= 2. */
 typedef struct moe_route_predictor moe_route_predictor;
 MOE_API moe_status_t moe_predictor_create(int layers, int E, moe_route_predictor** out);
 MOE_API void moe_predictor_destroy(moe_route_predictor* p);
-MOE_API moe_status_t moe_predictor_observe(moe_route_predictor* p, int layer, const int32_t* prev_ids,
-                                           const int32_t* cur_ids, int T, int k);
-MOE_API moe_status_t moe_predictor_predict(const moe_route_predictor* p, int layer, const int32_t* prev_ids,
-                                           int T, int k, int max_out, double min_score, int32_t* out_ids,
-                                           int32_t* n_out);
+MOE_API moe_status_t moe_predictor_observe(moe_route_predictor* p, int layer, const int32_t* prev2_ids,
+                                           const int32_t* prev_ids, const int32_t* cur_ids, int T, int k);
+MOE_API moe_status_t moe_predictor_predict(const moe_route_predictor* p, int layer, const int32_t* prev2_ids,
+                                           const int32_t* prev_ids, int T, int k, int max_out, double min_score,
+                                           int32_t* out_ids, int32_t* n_out);
 
 /* Free the cache's host bookkeeping, events and device table (not the
  * caller's pool or host blobs).  Synchronises the events it owns. */

@@ -55,8 +55,8 @@ _SIGS = {
     "moe_slot_timing_read": (_c_i, [_c_p, _c_p, _c_p]),
     "moe_predictor_create": (_c_i, [_c_i, _c_i, ctypes.POINTER(_c_p)]),
     "moe_predictor_destroy": (None, [_c_p]),
-    "moe_predictor_observe": (_c_i, [_c_p, _c_i, _c_p, _c_p, _c_i, _c_i]),
-    "moe_predictor_predict": (_c_i, [_c_p, _c_i, _c_p, _c_i, _c_i, _c_i, ctypes.c_double, _c_p, _c_p]),
+    "moe_predictor_observe": (_c_i, [_c_p, _c_i, _c_p, _c_p, _c_p, _c_i, _c_i]),
+    "moe_predictor_predict": (_c_i, [_c_p, _c_i, _c_p, _c_p, _c_i, _c_i, _c_i, ctypes.c_double, _c_p, _c_p]),
     "moe_debug_inject_fault": (None, [_c_i, _c_i]),
     "moe_debug_force_regime": (None, [_c_i]),
     "moe_debug_set_trace": (None, [_c_p]),
@@ -348,21 +348,25 @@ def moe_predictor_destroy(handle):
     load().moe_predictor_destroy(handle)
 
 
-def moe_predictor_observe(handle, layer, prev_ids, cur_ids):
-    prev = prev_ids.to(torch.int32).contiguous().cpu()
-    cur = cur_ids.to(torch.int32).contiguous().cpu()
+def _host_ids(ids):
+    return None if ids is None else ids.to(torch.int32).contiguous().cpu()
+
+
+def moe_predictor_observe(handle, layer, prev_ids, cur_ids, prev2_ids=None):
+    prev, cur, prev2 = _host_ids(prev_ids), _host_ids(cur_ids), _host_ids(prev2_ids)
     T, k = prev.shape
-    _check("moe_predictor_observe", load().moe_predictor_observe(handle, layer, prev.data_ptr(), cur.data_ptr(),
-                                                                  T, k))
+    _check("moe_predictor_observe", load().moe_predictor_observe(
+        handle, layer, None if prev2 is None else prev2.data_ptr(), prev.data_ptr(), cur.data_ptr(), T, k))
 
 
-def moe_predictor_predict(handle, layer, prev_ids, max_out, min_score=0.0):
-    prev = prev_ids.to(torch.int32).contiguous().cpu()
+def moe_predictor_predict(handle, layer, prev_ids, max_out, min_score=0.0, prev2_ids=None):
+    prev, prev2 = _host_ids(prev_ids), _host_ids(prev2_ids)
     T, k = prev.shape
     out = torch.empty(max(1, max_out), dtype=torch.int32)
     n = ctypes.c_int32(0)
-    _check("moe_predictor_predict", load().moe_predictor_predict(handle, layer, prev.data_ptr(), T, k, max_out,
-                                                                  float(min_score), out.data_ptr(), ctypes.byref(n)))
+    _check("moe_predictor_predict", load().moe_predictor_predict(
+        handle, layer, None if prev2 is None else prev2.data_ptr(), prev.data_ptr(), T, k, max_out,
+        float(min_score), out.data_ptr(), ctypes.byref(n)))
     return out[:n.value]
 
 
@@ -372,11 +376,11 @@ class RoutePredictor:
     def __init__(self, layers, E):
         self.handle = moe_predictor_create(layers, E)
 
-    def observe(self, layer, prev_ids, cur_ids):
-        moe_predictor_observe(self.handle, layer, prev_ids, cur_ids)
+    def observe(self, layer, prev_ids, cur_ids, prev2_ids=None):
+        moe_predictor_observe(self.handle, layer, prev_ids, cur_ids, prev2_ids)
 
-    def predict(self, layer, prev_ids, max_out, min_score=0.0):
-        return moe_predictor_predict(self.handle, layer, prev_ids, max_out, min_score)
+    def predict(self, layer, prev_ids, max_out, min_score=0.0, prev2_ids=None):
+        return moe_predictor_predict(self.handle, layer, prev_ids, max_out, min_score, prev2_ids)
 
     def close(self):
         if self.handle is not None and self.handle.value:

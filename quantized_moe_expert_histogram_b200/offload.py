@@ -131,11 +131,14 @@ class OffloadStack:
                                v["workspace"], v["y_perm"], v["status"], self.copy, self.compute)
             if self.prefetch and self.predictor is not None:
                 if l > 0:
-                    self.predictor.observe(l, self.ids_host[l - 1], self.ids_host[l])
+                    self.predictor.observe(l, self.ids_host[l - 1], self.ids_host[l],
+                                           prev2_ids=self.ids_host[l - 2] if l >= 2 else None)
                 if l + 1 < self.n_layers:
                     # confident predictions only: the link is the bottleneck, and a
-                    # wrong copy costs a slot and bandwidth
-                    pred = self.predictor.predict(l + 1, self.ids_host[l], self.slots // 4, min_score=1.0)
+                    # wrong copy costs a slot and bandwidth; keyed by the experts of
+                    # this layer and the one before it (EdgeMoE's profile key)
+                    pred = self.predictor.predict(l + 1, self.ids_host[l], self.slots // 4, min_score=1.0,
+                                                  prev2_ids=self.ids_host[l - 1] if l >= 1 else None)
                     if pred.numel():
                         self.prefetched += self.caches[l + 1].prefetch(pred, self.slots // 4, self.copy)
             y = torch.empty_like(x)
