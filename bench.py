@@ -43,7 +43,8 @@ def parse():
     p.add_argument("--sweep", default="1,8,16,256", help="extra token counts timed for context ('' = none)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=0)
-    p.add_argument("--workloads", default="mixtral:8192,mixtral:1,nested:2048,nested:1,tiny:64",
+    p.add_argument("--workloads", default="mixtral:8192,mixtral:512,mixtral:32,mixtral:1,nested:2048,nested:64,"
+                                          "nested:1,nested_gate:2048,nested_gate:1,tiny:64",
                    help="other configured workloads reported for context (name:tokens,...; '' = none)")
     p.add_argument("--offload-steps", type=int, default=512,
                    help="decode steps of the offload (slot-cache) workload reported under 'offload', after "
@@ -202,8 +203,11 @@ class ClockSampler:
 
 # -------------------------------------------------------------- workload --
 
-def make_instances(shape, T, R, seed, device):
-    """R layer instances with weights drawn and packed on the device."""
+def make_instances(shape, T, R, seed, device, bit_gate=False):
+    """R layer instances with weights drawn and packed on the device.  With
+    bit_gate (nested-plane layout), each instance gets a bit-width gate and
+    its widths are chosen on the device every step (moe_bit_gate) instead of
+    being drawn from the seed."""
     import torch
     from quantized_moe_expert_histogram_b200 import inputs as I
     from quantized_moe_expert_histogram_b200.layer import QuantMoELayer
@@ -214,8 +218,33 @@ def make_instances(shape, T, R, seed, device):
                                            L["w_down"], max_tokens=T)
         del L["w_gate"], L["w_up"], L["w_down"]
         torch.cuda.empty_cache()
-        layers.append((layer, L["x"], L.get("bits")))
+        bits = L.get("bits")
+        if bit_gate:
+            G = I.make_bit_gate(shape, seed=seed + 1000 * r + 1, device=device, bias=True)
+            layer.w_bit, layer.bias_bit = G["w_bit"], G["bias_bit"]
+            bits = None
+        layers.append((layer, L["x"], bits))
     return layers
+
+
+def kernel_launches(shape, T, bit_gate=False):
+    """Kernels of this library launched by one layer step, following the
+    library's own choices: router 1 (one cluster launch for decode-sized
+    batches) or 2, bit gate 1 when used, permutation 1 (single CTA, with the
+    gather when it is small) or 1 + gather, or 3 + gather, FFN 2, combine 1."""
+    n = T * shape.k
+    nbins = shape.E * (3 if shape.layout == "planes" else 1)
+    d32 = shape.d // 32
+    splits = 1
+    while splits * 2 <= 8 and d32 % (splits * 2) == 0:
+        splits *= 2
+    route = 1 if (T <= 8 * splits and shape.E <= 64 and splits >= 2) else 2
+    if n <= 1024:
+        perm = 1 if n * shape.d <= 64 * 1024 else 2
+    else:
+        perm = 4
+    del nbins
+    return route + (1 if bit_gate else 0) + perm + 2 + 1
 
 
 def profiled_traffic(workload, T):
@@ -267,6 +296,9 @@ def _step_calls(layer, x, bits, stream, part):
     if part == "all":
         moeq.moe_route_topk(x, layer.w_router, layer.bias, layer.k, topk_idx=v["topk_idx"],
                             topk_w=v["topk_w"], workspace=v["route_ws"], stream=stream)
+        if bits is None and layer.w_bit is not None:
+            bits = moeq.moe_bit_gate(x, layer.w_bit, layer.bias_bit, v["topk_idx"], bits=v["bits"],
+                                     status=v["status"], stream=stream)
         moeq.moe_permute(v["topk_idx"], layer.E, bits=bits, x=x, out=v, status=v["status"], stream=stream)
     moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, T, layer.E, layer.d, layer.F,
                             layer.group, layer.layout, workspace=v["workspace"], y_perm=v["y_perm"],
@@ -334,23 +366,37 @@ def time_e2e(layers, steps, stream):
     return start.elapsed_time(end), h2d, T * d * 2
 
 
-def measure_workload(name, T, R, peaks, stream, reps=8):
+def instances_for(shape, min_bytes=3 * 126 * 2 ** 20):
+    """Layer instances to rotate so that the expert weights of one pass over
+    all of them exceed three times the 126 MB L2 (at least 2)."""
+    from quantized_moe_expert_histogram_b200 import moeq
+    per = shape.E * moeq.moe_blob_bytes(shape.d, shape.F, shape.group, 1 if shape.layout == "planes" else 0)
+    return max(2, -(-min_bytes // per))
+
+
+def measure_workload(name, T, peaks, stream, reps=8):
     """Step time and FFN roofline fraction of another configured workload
-    (CUDA graphs over R rotated instances, as for the default workload)."""
+    (CUDA graphs over rotated instances, as for the default workload).
+    'nested_gate' is the nested-plane layer with its widths chosen on the
+    device by the bit-width gate (moe_bit_gate inside the step)."""
     import torch
     from quantized_moe_expert_histogram_b200 import inputs as I
-    shape = I.SHAPES[name]
-    ls = make_instances(shape, T, R, seed=31, device="cuda")
+    gate = name == "nested_gate"
+    shape = I.SHAPES["nested" if gate else name]
+    R = instances_for(shape)
+    ls = make_instances(shape, T, R, seed=31, device="cuda", bit_gate=gate)
     ga, gf = capture(ls, stream, "all"), capture(ls, stream, "ffn")
     tot = time_graph(ga, reps, 2, stream) / (reps * R)
     fm = time_graph(gf, reps, 1, stream) / (reps * R)
-    b, fl = algorithmic(shape, T, ls[-1][0], ls[0][2] is not None)
+    b, fl = algorithmic(shape, T, ls[-1][0], shape.layout == "planes")
     tc_bound = fl / (peaks["tc"] * 1e12) > b / (peaks["hbm"] * 1e9)
     out = {"workload": f"{name}: d={shape.d} E={shape.E} top-{shape.k} d_ff={shape.F} "
-                       f"{'nested 2/3/4-bit planes' if shape.layout == 'planes' else 'INT4'} g{shape.group}",
-           "tokens": T, "tokens_per_s": T / (tot / 1e3), "ms_per_step": tot, "ffn_ms": fm,
+                       f"{'nested 2/3/4-bit planes' if shape.layout == 'planes' else 'INT4'} g{shape.group}"
+                       + (", widths from the bit-width gate" if gate else ""),
+           "tokens": T, "instances": R, "tokens_per_s": T / (tot / 1e3), "ms_per_step": tot, "ffn_ms": fm,
            "ffn_bound": "tensor" if tc_bound else "hbm",
-           "ffn_frac": (fl / (fm / 1e3) / 1e12 / peaks["tc"]) if tc_bound else (b / (fm / 1e3) / 1e9 / peaks["hbm"])}
+           "ffn_frac": (fl / (fm / 1e3) / 1e12 / peaks["tc"]) if tc_bound else (b / (fm / 1e3) / 1e9 / peaks["hbm"]),
+           "ffn_alg_bytes": b, "ffn_flops": fl, "launches_per_step": kernel_launches(shape, T, gate)}
     del ls, ga, gf
     torch.cuda.empty_cache()
     return out
@@ -575,7 +621,7 @@ def main():
     if args.workloads:
         for item in args.workloads.split(","):
             name, tok = item.split(":")
-            workloads.append(measure_workload(name, int(tok), 2, peaks, stream))
+            workloads.append(measure_workload(name, int(tok), peaks, stream))
 
     offload = None
     if world == 1 and args.offload_steps > 0:
@@ -589,7 +635,7 @@ def main():
 
     # our kernels per step: router 2, permutation 1 + gather (<= 1024 assignments) or
     # 3 + gather, FFN 2, combine 1
-    launches_per_step = 2 + (2 if T * shape.k <= 1024 else 4) + 2 + 1
+    launches_per_step = kernel_launches(shape, T)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16", "data": "synthetic",

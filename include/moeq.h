@@ -283,17 +283,35 @@ typedef struct moe_slot_cache moe_slot_cache;
 MOE_API moe_status_t moe_slot_cache_create(int E, int slots, size_t blob_bytes, const void* host_blobs,
                                    void* device_pool, moe_slot_cache** out);
 
+/* The same for nested-plane blobs (MOE_LAYOUT_PLANES of shape d, F, group;
+ * blob_bytes = moe_blob_bytes(d, F, group, MOE_LAYOUT_PLANES)), in plane
+ * mode ([D2MoE] MWQ: W(2) needs only Q2, W(3) adds D3, W(4) adds D4): a
+ * slot holds an expert's planes up to some width, a step copies an expert
+ * only up to the widest width its assignments use (the Q2 planes and the
+ * scales for width 2, plus D3 for 3, plus D4 for 4), a resident expert that
+ * is later needed wider receives only its missing planes, and inside a wave
+ * the copies go plane by plane -- every Q2 + scales first, then every D3,
+ * then every D4 ([D2MoE] Hottest-Expert-Bit-First: hottest experts first,
+ * in bit order). */
+MOE_API moe_status_t moe_slot_cache_create_planes(int E, int slots, int d, int F, int group,
+                                                  const void* host_blobs, void* device_pool,
+                                                  moe_slot_cache** out);
+
 /* Plan one layer-step: ids_host (n_ids expert ids, host memory, repeats
- * allowed) are the experts the router chose.  Resident experts are hits;
- * the others are misses, loaded least-recently-used-victim first.  The
- * distinct experts are split into waves of at most slots/2 (hits first,
- * then misses by descending row count) so that copies of wave w+1 run on
- * copy_stream while wave w computes on compute_stream.  Issues the copies
- * of the first two waves.  *n_waves receives the wave count; stats_host
- * (may be NULL) receives {hits, misses, bytes_copied}. */
-MOE_API moe_status_t moe_slot_stage(moe_slot_cache* cache, const int32_t* ids_host, int n_ids,
-                            moe_stream_t copy_stream, moe_stream_t compute_stream,
-                            int32_t* n_waves, int64_t* stats_host);
+ * allowed) are the experts the router chose; bits_host (n_ids widths in
+ * {2, 3, 4}, host memory) their widths in plane mode, or NULL (every expert
+ * at width 4; ignored outside plane mode).  Resident experts holding every
+ * plane the step needs are hits; the others need copies (a fresh load into
+ * the least-recently-used free slot, or the missing planes of a resident
+ * expert).  The distinct experts are split into waves of at most slots/2
+ * (hits first, then the experts with copies by descending row count) so
+ * that copies of wave w+1 run on copy_stream while wave w computes on
+ * compute_stream.  Issues the copies of the first two waves.  *n_waves
+ * receives the wave count; stats_host (may be NULL) receives {hits,
+ * experts copied, bytes copied}. */
+MOE_API moe_status_t moe_slot_stage(moe_slot_cache* cache, const int32_t* ids_host, const uint8_t* bits_host,
+                                    int n_ids, moe_stream_t copy_stream, moe_stream_t compute_stream,
+                                    int32_t* n_waves, int64_t* stats_host);
 
 /* Run the staged layer-step: for each wave, compute_stream waits for the
  * wave's copies, the grouped FFN (same arguments as moe_grouped_ffn_wq)

@@ -2,14 +2,23 @@
 // host memory with cudaMemcpyAsync on a copy stream, overlapped with the
 // grouped FFN on the compute stream.
 //
-// A layer-step's distinct experts are ordered hits first, then misses by
-// descending row count (the hottest expert is loaded first), and cut into
-// waves of at most slots/2 experts.  Waves alternate between slot sets in
-// LRU order and never into a slot of the previous wave, so the copies of
-// wave w+1 overlap the compute of wave w (load E2 while computing E1).  A slot is overwritten only after the compute
-// that last read it has finished (per-slot event), and a wave computes only
-// after its copies have landed (per-wave event).  The FFN of a wave sees a
-// device table slot_of[E] listing just that wave's experts.
+// A layer-step's distinct experts are ordered hits first, then the experts
+// that need copies by descending row count (the hottest expert is loaded
+// first), and cut into waves of at most slots/2 experts.  Waves alternate
+// between slot sets in LRU order and never into a slot of the previous wave,
+// so the copies of wave w+1 overlap the compute of wave w (load E2 while
+// computing E1).  A slot is overwritten only after the compute that last
+// read it has finished (per-slot event), and a wave computes only after its
+// copies have landed (per-wave event).  The FFN of a wave sees a device
+// table slot_of[E] listing just that wave's experts.
+//
+// Plane mode (nested-width blobs): a slot records the widest width whose bit
+// planes it holds.  An expert is copied only up to the widest width its
+// assignments of the step use -- the Q2 planes and the scales for width 2,
+// plus D3 for 3, plus D4 for 4 -- and a resident expert needed wider later
+// receives only the missing planes.  Inside a wave the copies go plane by
+// plane (every Q2 + scales first, then every D3, then every D4): the bit
+// order of D2MoE's Hottest-Expert-Bit-First schedule.
 #include <algorithm>
 #include <atomic>
 #include <new>
@@ -33,6 +42,12 @@ bool take_fault(int what) {
 }
 
 inline cudaStream_t S(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
+
+// One planned copy: expert e into slot s, planes of widths (from, to]
+// (from = 0: a fresh load, including the scales).
+struct SlotCopy {
+  int e, s, from, to;
+};
 }  // namespace
 
 struct moe_slot_cache {
@@ -40,8 +55,13 @@ struct moe_slot_cache {
   size_t blob_bytes = 0;
   const uint8_t* host = nullptr;
   uint8_t* pool = nullptr;
+  // plane mode: byte ranges of the blob format (gate, up, down)
+  bool planes = false;
+  size_t q2_off[3] = {}, q2_len[3] = {}, d3_off[3] = {}, d3_len[3] = {}, d4_off[3] = {}, d4_len[3] = {};
+  size_t sz_off = 0, sz_len = 0;
   std::vector<int> slot_of;        // expert -> slot, -1 when not resident
   std::vector<int> expert_in;      // slot -> expert, -1 when empty
+  std::vector<int> width_in;       // slot -> widest width whose planes it holds (4 in blob mode)
   std::vector<uint64_t> last_use;  // slot -> logical time of last use
   uint64_t clock = 1;
   std::vector<cudaEvent_t> slot_free;  // recorded after the last compute reading the slot
@@ -55,10 +75,10 @@ struct moe_slot_cache {
   int32_t* d_tables = nullptr;  // device [max_waves][E]
   int32_t* h_tables = nullptr;  // pinned host [max_waves][E]
   // plan of the current step
-  std::vector<std::vector<int>> waves;           // experts per wave
-  std::vector<std::vector<int>> wave_misses;     // experts that must be copied, per wave
-  std::vector<std::vector<int>> wave_slots;      // slot of each expert of the wave
-  int copies_issued = 0;                         // waves whose copies were issued
+  std::vector<std::vector<int>> waves;             // experts per wave
+  std::vector<std::vector<SlotCopy>> wave_copies;  // copies per wave
+  std::vector<std::vector<int>> wave_slots;        // slot of each expert of the wave
+  int copies_issued = 0;                           // waves whose copies were issued
   bool staged = false;  // a plan is staged and its moe_slot_ffn has not run yet
   // busy-time measurement (moe_slot_timing): event pairs around each wave's
   // copies and each wave's FFN, recorded after the waits on the other stream
@@ -70,17 +90,30 @@ struct moe_slot_cache {
 
 namespace {
 
-// After a failed copy: experts planned into waves >= w are not resident
-// (their slots hold stale bytes), and the plan is dropped.
+// Bytes a copy of widths (from, to] moves.
+size_t copy_bytes(const moe_slot_cache* c, const SlotCopy& k) {
+  if (!c->planes) return c->blob_bytes;
+  size_t n = 0;
+  for (int m = 0; m < 3; ++m) {
+    if (k.from < 2) n += c->q2_len[m];
+    if (k.from < 3 && k.to >= 3) n += c->d3_len[m];
+    if (k.from < 4 && k.to >= 4) n += c->d4_len[m];
+  }
+  if (k.from < 2) n += c->sz_len;
+  return n;
+}
+
+// After a failed copy: the slots of waves >= w that were to receive copies
+// hold stale bytes, so their experts are dropped, and the plan is dropped.
 void invalidate_from(moe_slot_cache* c, int w) {
   for (size_t v = static_cast<size_t>(w); v < c->waves.size(); ++v)
-    for (int e : c->wave_misses[v]) {
-      const int s = c->slot_of[e];
-      if (s >= 0) c->expert_in[s] = -1;
-      c->slot_of[e] = -1;
+    for (const SlotCopy& k : c->wave_copies[v]) {
+      if (c->expert_in[k.s] == k.e) c->expert_in[k.s] = -1;
+      c->width_in[k.s] = 0;
+      c->slot_of[k.e] = -1;
     }
   c->waves.clear();
-  c->wave_misses.clear();
+  c->wave_copies.clear();
   c->wave_slots.clear();
   c->staged = false;
 }
@@ -98,54 +131,65 @@ moe_status_t timing_mark(moe_slot_cache* c, int k, cudaStream_t s) {
   return cuda_check(cudaEventRecord(v[c->tev_used[k]++], s), "timing event record");
 }
 
-moe_status_t issue_copies(moe_slot_cache* c, int w, cudaStream_t copy) {
-  const auto& slots = c->wave_slots[w];
-  const auto& exps = c->waves[w];
-  // the wave's copies: first every wait for a slot to be free, then the
-  // copies back to back (so that their busy time can be measured alone)
-  std::vector<std::pair<int, int>> todo;  // (expert, slot)
-  for (size_t i = 0; i < exps.size(); ++i) {
-    const int e = exps[i];
-    if (std::find(c->wave_misses[w].begin(), c->wave_misses[w].end(), e) == c->wave_misses[w].end())
-      continue;
-    const int s = slots[i];
-    if (take_fault(2)) {
-      set_error("moe_slot_stage: injected copy failure (expert %d)", e);
-      return MOE_ERR_FAULT_INJECTED;
-    }
-    if (c->slot_free_valid[s]) {
-      moe_status_t st = cuda_check(cudaStreamWaitEvent(copy, c->slot_free[s], 0), "slot wait free");
-      if (st != MOE_OK) return st;
-    }
-    todo.emplace_back(e, s);
-  }
-  c->copy_pending[w] = !todo.empty();
-  if (todo.empty()) return MOE_OK;
-  moe_status_t st = timing_mark(c, 0, copy);
-  if (st != MOE_OK) return st;
-  for (const auto& es : todo) {
-    st = cuda_check(cudaMemcpyAsync(c->pool + static_cast<size_t>(es.second) * c->blob_bytes,
-                                    c->host + static_cast<size_t>(es.first) * c->blob_bytes, c->blob_bytes,
+moe_status_t h2d(moe_slot_cache* c, int s, int e, size_t off, size_t len, cudaStream_t copy) {
+  return cuda_check(cudaMemcpyAsync(c->pool + static_cast<size_t>(s) * c->blob_bytes + off,
+                                    c->host + static_cast<size_t>(e) * c->blob_bytes + off, len,
                                     cudaMemcpyHostToDevice, copy),
                     "slot H2D copy");
-    if (st != MOE_OK) return st;
+}
+
+// Issue the copies `todo` on `copy` after their slots are free: blob mode
+// one copy per expert; plane mode plane by plane (all Q2 + scales, then all
+// D3, then all D4).
+moe_status_t issue(moe_slot_cache* c, const std::vector<SlotCopy>& todo, cudaStream_t copy) {
+  for (const SlotCopy& k : todo) {
+    if (c->slot_free_valid[k.s]) {
+      moe_status_t st = cuda_check(cudaStreamWaitEvent(copy, c->slot_free[k.s], 0), "slot wait free");
+      if (st != MOE_OK) return st;
+    }
   }
-  st = timing_mark(c, 0, copy);
+  moe_status_t st = timing_mark(c, 0, copy);
+  if (st != MOE_OK) return st;
+  if (!c->planes) {
+    for (const SlotCopy& k : todo)
+      if ((st = h2d(c, k.s, k.e, 0, c->blob_bytes, copy)) != MOE_OK) return st;
+  } else {
+    for (const SlotCopy& k : todo) {
+      if (k.from >= 2) continue;
+      for (int m = 0; m < 3; ++m)
+        if ((st = h2d(c, k.s, k.e, c->q2_off[m], c->q2_len[m], copy)) != MOE_OK) return st;
+      if ((st = h2d(c, k.s, k.e, c->sz_off, c->sz_len, copy)) != MOE_OK) return st;
+    }
+    for (const SlotCopy& k : todo) {
+      if (k.from >= 3 || k.to < 3) continue;
+      for (int m = 0; m < 3; ++m)
+        if ((st = h2d(c, k.s, k.e, c->d3_off[m], c->d3_len[m], copy)) != MOE_OK) return st;
+    }
+    for (const SlotCopy& k : todo) {
+      if (k.to < 4) continue;
+      for (int m = 0; m < 3; ++m)
+        if ((st = h2d(c, k.s, k.e, c->d4_off[m], c->d4_len[m], copy)) != MOE_OK) return st;
+    }
+  }
+  return timing_mark(c, 0, copy);
+}
+
+moe_status_t issue_copies(moe_slot_cache* c, int w, cudaStream_t copy) {
+  const auto& todo = c->wave_copies[w];
+  for (size_t i = 0; i < todo.size(); ++i)
+    if (take_fault(2)) {
+      set_error("moe_slot_stage: injected copy failure (expert %d)", todo[i].e);
+      return MOE_ERR_FAULT_INJECTED;
+    }
+  c->copy_pending[w] = !todo.empty();
+  if (todo.empty()) return MOE_OK;
+  moe_status_t st = issue(c, todo, copy);
   if (st != MOE_OK) return st;
   return cuda_check(cudaEventRecord(c->copy_done[w], copy), "slot copy event");
 }
 
-}  // namespace
-
-extern "C" {
-
-void moe_debug_inject_fault(int what, int count) {
-  g_fault_what.store(what);
-  g_fault_count.store(what ? count : 0);
-}
-
-moe_status_t moe_slot_cache_create(int E, int slots, size_t blob_bytes, const void* host_blobs,
-                                   void* device_pool, moe_slot_cache** out) {
+moe_status_t create(int E, int slots, size_t blob_bytes, const void* host_blobs, void* device_pool,
+                    const BlobLayout* planes, moe_slot_cache** out) {
   if (!out || !host_blobs || !device_pool || E <= 0 || E > 256 || slots < 2 || blob_bytes == 0) {
     set_error("moe_slot_cache_create: bad arguments");
     return MOE_ERR_INVALID_ARG;
@@ -165,8 +209,22 @@ moe_status_t moe_slot_cache_create(int E, int slots, size_t blob_bytes, const vo
   c->blob_bytes = blob_bytes;
   c->host = static_cast<const uint8_t*>(host_blobs);
   c->pool = static_cast<uint8_t*>(device_pool);
+  if (planes) {
+    c->planes = true;
+    for (int m = 0; m < 3; ++m) {
+      c->q2_off[m] = planes->q2[m];
+      c->q2_len[m] = planes->d3[m] - planes->q2[m];
+      c->d3_off[m] = planes->d3[m];
+      c->d3_len[m] = planes->d4[m] - planes->d3[m];
+      c->d4_off[m] = planes->d4[m];
+      c->d4_len[m] = (m < 2 ? planes->q2[m + 1] : planes->sz[0]) - planes->d4[m];
+    }
+    c->sz_off = planes->sz[0];
+    c->sz_len = planes->bytes - planes->sz[0];
+  }
   c->slot_of.assign(E, -1);
   c->expert_in.assign(slots, -1);
+  c->width_in.assign(slots, 0);
   c->last_use.assign(slots, 0);
   c->slot_free.assign(slots, nullptr);
   c->slot_free_valid.assign(slots, 0);
@@ -195,6 +253,30 @@ moe_status_t moe_slot_cache_create(int E, int slots, size_t blob_bytes, const vo
   }
   *out = c;
   return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void moe_debug_inject_fault(int what, int count) {
+  g_fault_what.store(what);
+  g_fault_count.store(what ? count : 0);
+}
+
+moe_status_t moe_slot_cache_create(int E, int slots, size_t blob_bytes, const void* host_blobs,
+                                   void* device_pool, moe_slot_cache** out) {
+  return create(E, slots, blob_bytes, host_blobs, device_pool, nullptr, out);
+}
+
+moe_status_t moe_slot_cache_create_planes(int E, int slots, int d, int F, int group, const void* host_blobs,
+                                          void* device_pool, moe_slot_cache** out) {
+  const BlobLayout L = blob_layout(d, F, group, MOE_LAYOUT_PLANES);
+  if (!L.valid) {
+    set_error("moe_slot_cache_create_planes: unsupported shape d=%d F=%d group=%d", d, F, group);
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  return create(E, slots, L.bytes, host_blobs, device_pool, &L, out);
 }
 
 void moe_slot_cache_destroy(moe_slot_cache* c) {
@@ -259,7 +341,7 @@ moe_status_t moe_slot_timing_read(moe_slot_cache* c, double* copy_ms, double* ff
   return MOE_OK;
 }
 
-moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_ids,
+moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, const uint8_t* bits_host, int n_ids,
                             moe_stream_t copy_stream, moe_stream_t compute_stream,
                             int32_t* n_waves, int64_t* stats_host) {
   (void)compute_stream;
@@ -271,38 +353,51 @@ moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_id
     set_error("moe_slot_stage: injected fault before any work");
     return MOE_ERR_FAULT_INJECTED;
   }
-  std::vector<int> cnt(c->E, 0);
+  std::vector<int> cnt(c->E, 0), need(c->E, 0);
   for (int i = 0; i < n_ids; ++i) {
     const int e = ids_host[i];
     if (e < 0 || e >= c->E) {
       set_error("moe_slot_stage: expert id %d out of range [0,%d)", e, c->E);
       return MOE_ERR_INVALID_ARG;
     }
+    int b = 4;
+    if (c->planes && bits_host) {
+      b = bits_host[i];
+      if (b < 2 || b > 4) {
+        set_error("moe_slot_stage: bit width %d not in {2, 3, 4}", b);
+        return MOE_ERR_INVALID_ARG;
+      }
+    }
     ++cnt[e];
+    need[e] = std::max(need[e], b);
   }
-  std::vector<int> hits, misses;
+  // hits: resident with every plane the step needs; the others need copies
+  // (a fresh load, or in plane mode the missing planes of a resident expert)
+  std::vector<int> hits, copies;
   for (int e = 0; e < c->E; ++e) {
     if (!cnt[e]) continue;
-    (c->slot_of[e] >= 0 ? hits : misses).push_back(e);
+    const int s = c->slot_of[e];
+    (s >= 0 && c->width_in[s] >= need[e] ? hits : copies).push_back(e);
   }
-  std::stable_sort(misses.begin(), misses.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
+  std::stable_sort(copies.begin(), copies.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
   std::vector<int> order(hits);
-  order.insert(order.end(), misses.begin(), misses.end());
+  order.insert(order.end(), copies.begin(), copies.end());
   const int W = std::max(1, c->S / 2);
   const int nw = static_cast<int>((order.size() + W - 1) / W);
   c->waves.assign(nw, {});
-  c->wave_misses.assign(nw, {});
+  c->wave_copies.assign(nw, {});
   c->wave_slots.assign(nw, {});
   for (size_t i = 0; i < order.size(); ++i) c->waves[i / W].push_back(order[i]);
 
-  // Assign slots wave by wave.  Hits keep their slot; a miss takes the least
-  // recently used slot that holds nothing needed by this wave or later ones.
-  std::vector<int> slot_of = c->slot_of, expert_in = c->expert_in;
+  // Assign slots wave by wave.  Resident experts keep their slot; a fresh
+  // load takes the least recently used slot that holds nothing needed by
+  // this wave or later ones.
+  std::vector<int> slot_of = c->slot_of, expert_in = c->expert_in, width_in = c->width_in;
   std::vector<uint64_t> last_use = c->last_use;
   uint64_t clock = c->clock;
   std::vector<char> needed_later(c->E, 0);
   for (int e : order) needed_later[e] = 1;
-  int64_t n_hits = 0, n_miss = 0;
+  int64_t n_hits = 0, n_copy = 0, bytes = 0;
   std::vector<int> prev_slots;  // slots of wave w-1: its compute may still be unqueued
   for (int w = 0; w < nw; ++w) {
     const uint64_t t = ++clock;
@@ -314,25 +409,34 @@ moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_id
       if (expert_in[s] >= 0 && needed_later[expert_in[s]]) pinned[s] = 1;
     for (int e : c->waves[w]) {
       int s = slot_of[e];
-      if (s >= 0) {
+      if (s >= 0 && width_in[s] >= need[e]) {
         ++n_hits;
       } else {
-        int best = -1;
-        for (int cand = 0; cand < c->S; ++cand) {
-          if (pinned[cand]) continue;
-          if (best < 0 || last_use[cand] < last_use[best]) best = cand;
+        SlotCopy k{e, s, 0, need[e]};
+        if (s >= 0) {
+          k.from = width_in[s];  // plane mode: only the missing planes
+        } else {
+          int best = -1;
+          for (int cand = 0; cand < c->S; ++cand) {
+            if (pinned[cand]) continue;
+            if (best < 0 || last_use[cand] < last_use[best]) best = cand;
+          }
+          if (best < 0) {
+            set_error("moe_slot_stage: no free slot (slots=%d)", c->S);
+            return MOE_ERR_INVALID_ARG;
+          }
+          s = best;
+          if (expert_in[s] >= 0) slot_of[expert_in[s]] = -1;
+          expert_in[s] = e;
+          slot_of[e] = s;
+          pinned[s] = 1;
+          k.s = s;
         }
-        if (best < 0) {
-          set_error("moe_slot_stage: no free slot (slots=%d)", c->S);
-          return MOE_ERR_INVALID_ARG;
-        }
-        s = best;
-        if (expert_in[s] >= 0) slot_of[expert_in[s]] = -1;
-        expert_in[s] = e;
-        slot_of[e] = s;
-        pinned[s] = 1;
-        c->wave_misses[w].push_back(e);
-        ++n_miss;
+        width_in[s] = c->planes ? need[e] : 4;
+        if (!c->planes) k.to = 4;
+        c->wave_copies[w].push_back(k);
+        bytes += static_cast<int64_t>(copy_bytes(c, k));
+        ++n_copy;
       }
       last_use[s] = t;
       c->wave_slots[w].push_back(s);
@@ -342,6 +446,7 @@ moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_id
   }
   c->slot_of.swap(slot_of);
   c->expert_in.swap(expert_in);
+  c->width_in.swap(width_in);
   c->last_use.swap(last_use);
   c->clock = clock;
   // Device tables of this step: the previous step's uploads must have run
@@ -367,8 +472,8 @@ moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, int n_id
   *n_waves = nw;
   c->staged = true;
   c->stats[0] = n_hits;
-  c->stats[1] = n_miss;
-  c->stats[2] = n_miss * static_cast<int64_t>(c->blob_bytes);
+  c->stats[1] = n_copy;
+  c->stats[2] = bytes;
   if (stats_host) {
     stats_host[0] = c->stats[0];
     stats_host[1] = c->stats[1];
@@ -385,17 +490,17 @@ moe_status_t moe_slot_prefetch(moe_slot_cache* c, const int32_t* ids_host, int n
   }
   if (n_copied) *n_copied = 0;
   if (c->staged) {
-    // the staged plan's slots (hits, and misses of waves whose copies are
-    // issued later) must keep their experts until its moe_slot_ffn has run
+    // the staged plan's slots (hits, and copies of waves issued later) must
+    // keep their experts until its moe_slot_ffn has run
     set_error("moe_slot_prefetch: called between moe_slot_stage and moe_slot_ffn of the same cache");
     return MOE_ERR_INVALID_ARG;
   }
   // Victims: least recently used slots, never one filled by this call; each
-  // copy waits for the compute that last read its slot (a step of this layer
-  // whose FFN may still run).
+  // copy (every plane) waits for the compute that last read its slot (a step
+  // of this layer whose FFN may still run).
   std::vector<char> pinned(c->S, 0);
-  int copied = 0;
-  for (int i = 0; i < n_ids && copied < max_copies; ++i) {
+  std::vector<SlotCopy> todo;
+  for (int i = 0; i < n_ids && static_cast<int>(todo.size()) < max_copies; ++i) {
     const int e = ids_host[i];
     if (e < 0 || e >= c->E) {
       set_error("moe_slot_prefetch: expert id %d out of range [0,%d)", e, c->E);
@@ -412,29 +517,22 @@ moe_status_t moe_slot_prefetch(moe_slot_cache* c, const int32_t* ids_host, int n
       set_error("moe_slot_prefetch: injected copy failure (expert %d)", e);
       return MOE_ERR_FAULT_INJECTED;
     }
-    if (c->slot_free_valid[best]) {
-      moe_status_t st = cuda_check(cudaStreamWaitEvent(S(copy_stream), c->slot_free[best], 0), "slot wait free");
-      if (st != MOE_OK) return st;
-    }
-    moe_status_t st = cuda_check(
-        cudaMemcpyAsync(c->pool + static_cast<size_t>(best) * c->blob_bytes,
-                        c->host + static_cast<size_t>(e) * c->blob_bytes, c->blob_bytes, cudaMemcpyHostToDevice,
-                        S(copy_stream)),
-        "slot prefetch H2D copy");
-    if (st != MOE_OK) return st;
     if (c->expert_in[best] >= 0) c->slot_of[c->expert_in[best]] = -1;
     c->expert_in[best] = e;
     c->slot_of[e] = best;
+    c->width_in[best] = 4;
     c->last_use[best] = ++c->clock;
     pinned[best] = 1;
-    ++copied;
+    todo.push_back(SlotCopy{e, best, 0, 4});
   }
-  if (copied) {
-    moe_status_t st = cuda_check(cudaEventRecord(c->prefetch_done, S(copy_stream)), "slot prefetch event");
+  if (!todo.empty()) {
+    moe_status_t st = issue(c, todo, S(copy_stream));
+    if (st != MOE_OK) return st;
+    st = cuda_check(cudaEventRecord(c->prefetch_done, S(copy_stream)), "slot prefetch event");
     if (st != MOE_OK) return st;
     c->prefetch_pending = true;
   }
-  if (n_copied) *n_copied = copied;
+  if (n_copied) *n_copied = static_cast<int32_t>(todo.size());
   return MOE_OK;
 }
 
@@ -445,6 +543,10 @@ moe_status_t moe_slot_ffn(moe_slot_cache* c, const void* x_perm, const int32_t* 
                           moe_stream_t compute_stream) {
   if (!c) {
     set_error("moe_slot_ffn: null cache");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (c->planes && layout != MOE_LAYOUT_PLANES) {
+    set_error("moe_slot_ffn: a plane-mode cache holds nested-plane blobs (layout %d given)", layout);
     return MOE_ERR_INVALID_ARG;
   }
   const int nw = static_cast<int>(c->waves.size());

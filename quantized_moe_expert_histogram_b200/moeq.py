@@ -46,7 +46,8 @@ _SIGS = {
                                   _c_p, _c_sz, _c_p, _c_p, _c_p]),
     "moe_unpermute_combine": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_p, _c_p]),
     "moe_slot_cache_create": (_c_i, [_c_i, _c_i, _c_sz, _c_p, _c_p, ctypes.POINTER(_c_p)]),
-    "moe_slot_stage": (_c_i, [_c_p, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p]),
+    "moe_slot_cache_create_planes": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, ctypes.POINTER(_c_p)]),
+    "moe_slot_stage": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p]),
     "moe_slot_ffn": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p,
                             _c_p, _c_p, _c_p]),
     "moe_slot_cache_destroy": (None, [_c_p]),
@@ -259,31 +260,38 @@ def moe_unpermute_combine(y_perm, inv_perm, topk_w, residual=None, y=None, strea
 
 
 class SlotCache:
-    """One layer's GPU slot cache (moe_slot_cache_create / _destroy)."""
+    """One layer's GPU slot cache (moe_slot_cache_create / _destroy); with
+    planes=(d, F, group) a plane-mode cache of nested-plane blobs
+    (moe_slot_cache_create_planes)."""
 
-    def __init__(self, E, slots, blob_bytes, host_blobs, device_pool):
+    def __init__(self, E, slots, blob_bytes, host_blobs, device_pool, planes=None):
         lib = load()
         if not host_blobs.is_pinned():
             raise ValueError("host_blobs must be pinned host memory")
         self._host = host_blobs
         self._pool = device_pool
         h = _c_p()
-        _check("moe_slot_cache_create", lib.moe_slot_cache_create(
-            E, slots, blob_bytes, host_blobs.data_ptr(), _ptr(device_pool), ctypes.byref(h)))
+        if planes is None:
+            _check("moe_slot_cache_create", lib.moe_slot_cache_create(
+                E, slots, blob_bytes, host_blobs.data_ptr(), _ptr(device_pool), ctypes.byref(h)))
+        else:
+            d, F, group = planes
+            moe_slot_cache_create_planes(E, slots, d, F, group, host_blobs, device_pool, h)
         self.handle = h
         self.E = E
         self._ids = None
 
-    def stage(self, ids_host, copy_stream, compute_stream):
-        """moe_slot_stage; returns (n_waves, [hits, misses, bytes])."""
+    def stage(self, ids_host, copy_stream, compute_stream, bits_host=None):
+        """moe_slot_stage; returns (n_waves, [hits, experts copied, bytes])."""
         lib = load()
         ids = ids_host.to(torch.int32).contiguous()
-        self._ids = ids
+        bits = None if bits_host is None else bits_host.to(torch.uint8).contiguous().cpu()
+        self._ids, self._bits = ids, bits
         nw = ctypes.c_int32(0)
         stats = (ctypes.c_int64 * 3)()
         _check("moe_slot_stage", lib.moe_slot_stage(
-            self.handle, ids.data_ptr(), ids.numel(), copy_stream.cuda_stream,
-            compute_stream.cuda_stream, ctypes.byref(nw), stats))
+            self.handle, ids.data_ptr(), None if bits is None else bits.data_ptr(), ids.numel(),
+            copy_stream.cuda_stream, compute_stream.cuda_stream, ctypes.byref(nw), stats))
         return nw.value, list(stats)
 
     def ffn(self, x_perm, offsets, T, d, F, group, layout, workspace, y_perm, status, copy_stream,
@@ -326,6 +334,12 @@ def moe_slot_prefetch(handle, ids_host, max_copies, copy_stream):
     _check("moe_slot_prefetch", load().moe_slot_prefetch(handle, ids.data_ptr(), ids.numel(), int(max_copies),
                                                           copy_stream.cuda_stream, ctypes.byref(n)))
     return n.value
+
+
+def moe_slot_cache_create_planes(E, slots, d, F, group, host_blobs, device_pool, handle):
+    _check("moe_slot_cache_create_planes", load().moe_slot_cache_create_planes(
+        E, slots, d, F, group, host_blobs.data_ptr(), _ptr(device_pool), ctypes.byref(handle)))
+    return handle
 
 
 def moe_slot_timing(handle, enable):

@@ -256,3 +256,105 @@ def test_lookahead_pregated_ids_equal_resident():
         assert torch.equal(y_o, ys_r[-1]), f"step {s}"
     ref.close()
     off.close()
+
+
+def _plane_bytes(shape):
+    """Bytes of each plane set of a nested-plane blob: (Q2 of the three
+    matrices + scales, D3 of the three, D4 of the three)."""
+    d, F, g = shape.d, shape.F, shape.group
+    elems = 3 * d * F
+    return elems // 4 + 3 * d * F // g * 4, elems // 8, elems // 8
+
+
+def test_plane_mode_copies_only_the_needed_planes():
+    """Plane-mode slot cache (nested widths): an expert used only at width 2
+    moves its Q2 planes and scales; needed at width 4 later it receives only
+    D3 and D4; at width 3 after that it is a hit.  The FFN through the cache
+    equals the resident FFN bit for bit at every step."""
+    shape = I.custom_shape(d=256, E=16, k=2, F=256, group=64, layout="planes")
+    T = 2
+    w = I.make_expert_weights(shape, seed=31, device="cuda")
+    r = I.make_router(shape, seed=32, device="cuda")
+    layer = QuantMoELayer.from_weights(shape, r["w_router"], r["bias"], w["w_gate"], w["w_up"], w["w_down"],
+                                       max_tokens=T)
+    blob = layer.blobs.shape[1]
+    host = layer.blobs.cpu().pin_memory()
+    pool = torch.empty(8, blob, dtype=torch.uint8, device="cuda")
+    cache = moeq.SlotCache(shape.E, 8, blob, host, pool, planes=(shape.d, shape.F, shape.group))
+    copy, compute = torch.cuda.Stream(), torch.cuda.current_stream()
+    q2sz, d3, d4 = _plane_bytes(shape)
+    assert q2sz + d3 + d4 == blob
+    ids = torch.tensor([[1, 2], [3, 4]], dtype=torch.int32, device="cuda")
+    x = I.make_slot_x(shape.d, 1, T, seed=5, device="cuda")[0]
+    v = layer.views(T)
+    expect = [(0, 4, 4 * q2sz), (0, 4, 4 * (d3 + d4)), (4, 0, 0)]
+    for step, b in enumerate((2, 4, 3)):
+        bits = torch.full((T, shape.k), b, dtype=torch.uint8, device="cuda")
+        moeq.moe_route_topk(x, layer.w_router, layer.bias, shape.k, forced_idx=ids, topk_idx=v["topk_idx"],
+                            topk_w=v["topk_w"], workspace=v["route_ws"])
+        moeq.moe_permute(v["topk_idx"], shape.E, bits=bits, x=x, out=v, status=v["status"])
+        y_ref = moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, T, shape.E, shape.d, shape.F,
+                                        shape.group, layer.layout, workspace=v["workspace"],
+                                        status=v["status"]).clone()
+        nw, st = cache.stage(ids.cpu().reshape(-1), copy, compute, bits_host=bits.cpu().reshape(-1))
+        assert tuple(st) == expect[step], (step, st)
+        y_off = torch.empty_like(y_ref)
+        cache.ffn(v["x_perm"], v["offsets"], T, shape.d, shape.F, shape.group, layer.layout, v["workspace"],
+                  y_off, v["status"], copy, compute)
+        torch.cuda.synchronize()
+        assert torch.equal(y_off, y_ref), f"step {step} (width {b})"
+        assert int(v["status"].item()) == 0
+    cache.close()
+
+
+def test_plane_mode_offload_equals_resident_on_mixed_widths():
+    """Plane-mode offload of a nested-plane stack with widths drawn per
+    assignment ({0.3, 0.4, 0.3} over 2/3/4) on the Zipf/successor trace: every
+    layer equals the resident path bit for bit, and the bytes moved are
+    below what whole-blob staging of the same experts would move."""
+    shape = I.custom_shape(d=256, E=16, k=4, F=256, group=64, layout="planes")
+    layers, slots, batch, steps = 2, 8, 8, 5
+    trace = I.make_slot_trace(shape.E, shape.k, layers, steps, batch, seed=12).cuda()
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(13)
+    bits_all = I.draw_bits(steps * layers * batch, shape.k, gen, "cpu").reshape(steps, layers, batch, shape.k)
+    built = []
+    for l in range(layers):
+        w = I.make_expert_weights(shape, seed=40 + l, device="cuda")
+        r = I.make_router(shape, seed=50 + l, device="cuda")
+        layer = QuantMoELayer.from_weights(shape, r["w_router"], r["bias"], w["w_gate"], w["w_up"], w["w_down"],
+                                           max_tokens=batch)
+        blob = layer.blobs.shape[1]
+        host = layer.blobs.cpu().pin_memory()
+        pool = torch.empty(slots, blob, dtype=torch.uint8, device="cuda")
+        built.append((layer, moeq.SlotCache(shape.E, slots, blob, host, pool,
+                                            planes=(shape.d, shape.F, shape.group)), blob))
+    copy, compute = torch.cuda.Stream(), torch.cuda.current_stream()
+    xs = I.make_slot_x(shape.d, steps, batch, seed=14, device="cuda")
+    moved = whole = 0
+    for s in range(steps):
+        x = xs[s]
+        for l, (layer, cache, blob) in enumerate(built):
+            v = layer.views(batch)
+            bits = bits_all[s, l].cuda()
+            moeq.moe_route_topk(x, layer.w_router, layer.bias, shape.k, forced_idx=trace[s, l].contiguous(),
+                                topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"])
+            moeq.moe_permute(v["topk_idx"], shape.E, bits=bits, x=x, out=v, status=v["status"])
+            y_ref = moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, batch, shape.E, shape.d,
+                                            shape.F, shape.group, layer.layout, workspace=v["workspace"],
+                                            status=v["status"]).clone()
+            nw, st = cache.stage(trace[s, l].cpu().reshape(-1), copy, compute, bits_host=bits_all[s, l].reshape(-1))
+            moved += st[2]
+            whole += st[1] * blob
+            y_off = torch.empty_like(y_ref)
+            cache.ffn(v["x_perm"], v["offsets"], batch, shape.d, shape.F, shape.group, layer.layout,
+                      v["workspace"], y_off, v["status"], copy, compute)
+            torch.cuda.synchronize()
+            assert torch.equal(y_off, y_ref), f"step {s} layer {l}"
+            assert int(v["status"].item()) == 0
+            y = torch.empty_like(x)
+            moeq.moe_unpermute_combine(y_off, v["inv_perm"], v["topk_w"], residual=x, y=y)
+            x = y
+    assert 0 < moved < whole
+    for _, cache, _ in built:
+        cache.close()
