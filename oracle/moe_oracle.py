@@ -39,6 +39,8 @@ Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 # ---------------------------------------------------------------------------
@@ -256,8 +258,17 @@ def build_blob(w_gate, w_up, w_down, group: int, layout: str) -> np.ndarray:
 
 
 def router_logits(x: np.ndarray, w_router: np.ndarray, bias=None) -> np.ndarray:
-    """l[t,e] = sum_i x[t,i] * W_r[e,i] (+ bias[e]) in fp64."""
-    l = np.asarray(x, dtype=np.float64) @ np.asarray(w_router, dtype=np.float64).T
+    """l[t,e] = sum_i x[t,i] * W_r[e,i] (+ bias[e]) in fp64.
+
+    Each logit is the same summation of its d exact fp64 products (numpy's
+    reduction along a contiguous row), so experts with identical router rows
+    get identical logits and the tie rule (lower index) applies; a blocked
+    matrix product may round two identical rows differently."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_router, dtype=np.float64)
+    l = np.empty((x.shape[0], w.shape[0]), dtype=np.float64)
+    for t0 in range(0, x.shape[0], 64):
+        l[t0:t0 + 64] = (x[t0:t0 + 64, None, :] * w[None, :, :]).sum(axis=-1)
     if bias is not None:
         l = l + np.asarray(bias, dtype=np.float64)[None, :]
     return l
@@ -315,7 +326,10 @@ def bit_gate(x: np.ndarray, w_bit: np.ndarray, bias_bit, sel: np.ndarray) -> np.
     for t in range(T):
         for j in range(k):
             e = int(sel[t, j])
-            scores = w[e] @ x[t]
+            # each score the correctly rounded sum of its exact fp64 products
+            # (bf16 x fp32 fits fp64), so equal scores are equal here and the
+            # tie rule decides them
+            scores = np.array([math.fsum(w[e, c] * x[t]) for c in range(3)])
             if b is not None:
                 scores = scores + b[e]
             out[t, j] = BIT_WIDTHS[int(np.argmax(scores))]  # first maximum: the narrower width

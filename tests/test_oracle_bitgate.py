@@ -56,3 +56,18 @@ def test_ties_go_to_the_narrower_width():
     w[1, 1] = w[1, 2] = np.array([1.0, 0, 0, 0])   # widths 3 and 4 tie for expert 1
     x = np.array([[2.0, 0, 0, 0]])
     assert O.bit_gate(x, w, None, np.array([[1, 0]], np.int32)).tolist() == [[3, 2]]
+
+
+def test_identical_rows_tie_exactly_at_full_length():
+    # two identical width rows of a realistic length (d = 4096, random
+    # values): the two scores are the same number, so the narrower width wins
+    # every time (a blocked dot product may round identical rows apart)
+    rng = np.random.default_rng(4)
+    d, E, T = 4096, 4, 64
+    w = rng.normal(0, 0.02, (E, 3, d)).astype(np.float32)
+    w[:, 2] = w[:, 1]
+    bias = np.zeros((E, 3), np.float32)
+    bias[:, 0] = -100.0  # width 2 never wins
+    x = rng.normal(size=(T, d)).astype(np.float32)
+    sel = np.stack([rng.permutation(E)[:2] for _ in range(T)]).astype(np.int32)
+    assert (O.bit_gate(x, w, bias, sel) == 3).all()

@@ -179,3 +179,18 @@ def test_forced_selection_and_subset():
     full = O.moe_layer(x, L["w_router"].numpy(), None, shape.k, ex)
     sub = O.moe_layer(x, L["w_router"].numpy(), None, shape.k, ex, token_subset=[0, 5, 11])
     np.testing.assert_allclose(sub["y"][[0, 5, 11]], full["y"][[0, 5, 11]], rtol=1e-12, atol=1e-15)
+
+
+def test_identical_router_rows_give_identical_logits():
+    # duplicated router rows at full length: equal logits, so every token that
+    # picks one of the pair and not the other picks the lower index
+    rng = np.random.default_rng(6)
+    T, E, d, k = 512, 16, 2048, 3
+    w = rng.normal(0, 0.02, (E, d)).astype(np.float32)
+    w[9] = w[4]
+    x = rng.normal(size=(T, d)).astype(np.float32)
+    l = O.router_logits(x, w)
+    assert np.array_equal(l[:, 9], l[:, 4])
+    sel = O.topk_select(l, k)
+    one = [s for s in sel if (4 in s) != (9 in s)]
+    assert one and all(4 in s for s in one)
