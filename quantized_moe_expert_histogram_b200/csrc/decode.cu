@@ -178,50 +178,57 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
   auto mat = [](int f) { return GU ? f : 0; };
   auto frow = [&](int f) { return GU ? n0 : n0 + 16 * f; };
 
+  // Copy sources of this lane, fixed for the item: piece u (0, 1) of
+  // fragment f of stage s starts at src[f][u] + s * step(u) (16 bytes; a
+  // null base: nothing to copy), and its scale/zero piece at
+  // sz_src[f] + s * sz_step (lanes below 4, or 8 for groups of 64).  Per
+  // fragment: INT4 16 rows x 64 B of codes in 64 pieces; planes 16 rows x
+  // (32 B Q2 + 16 B D3 + 16 B D4); then 16 rows x 1 or 2 groups of
+  // (scale, zero) words, contiguous.
+  constexpr int kStep0 = PLANES ? 32 : 64;  // piece 0: codes, or Q2
+  constexpr int kStep1 = PLANES ? 16 : 64;  // piece 1: codes, or D3 / D4
+  const int sz_step = (kStageK / P.group) * 512;
+  const uint8_t* src[FW][2];
+  uint32_t dst[FW][2];
+  const uint8_t* sz_src[FW];
+#pragma unroll
+  for (int f = 0; f < FW; ++f) {
+    const int m = mat(f), r0 = frow(f);
+    if (!PLANES) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int q = lane + 32 * u, rr = q >> 2, cc = q & 3;
+        src[f][u] = blob + P.code_off[m] + static_cast<size_t>(r0 + rr) * (P.K / 2) + cc * 16;
+        dst[f][u] = f * kFragBytes + rr * 64 + cc * 16;
+      }
+    } else {
+      const int rq = lane >> 1, hh = lane & 1;  // Q2: 16 rows x 32 B
+      src[f][0] = blob + P.code_off[m] + static_cast<size_t>(r0 + rq) * (P.K / 4) + hh * 16;
+      dst[f][0] = f * kFragBytes + rq * 32 + hh * 16;
+      const int rr = lane & 15;  // lanes 0-15: D3, 16-31: D4 (16 rows x 16 B each)
+      const bool want = lane < 16 ? bits >= 3 : bits >= 4;
+      src[f][1] = want ? blob + (lane < 16 ? P.d3_off[m] : P.d4_off[m]) + static_cast<size_t>(r0 + rr) * (P.K / 8)
+                       : nullptr;
+      dst[f][1] = f * kFragBytes + (lane < 16 ? 512 : 768) + rr * 16;
+    }
+    const int gi = (lane >> 2) & 1, pc = lane & 3;
+    sz_src[f] = blob + P.sz_off[m] + (static_cast<size_t>(r0 >> 7) * G + gi) * 512 + (r0 & 127) * 4 + pc * 16;
+  }
+  const bool sz_lane = lane < (G64 ? 8 : 4);
+
   // copies of this warp's i-th stage (global stage warp + 8 i) into ring
-  // slot i % kRing: per fragment 64 pieces of 16 B of codes, plus the
-  // fragment's scale/zero words (16 rows x 1 or 2 groups, contiguous)
+  // slot i % kRing
   auto issue = [&](int i) {
     const int s = warp + kWarps * i;
     if (s < n_stages) {
       const uint32_t dst0 = ring_u + (i % kRing) * kSlot;
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
-        const int m = mat(f);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int q = lane + 32 * u;  // piece 0..63 of this fragment
-          const uint8_t* src = nullptr;
-          uint32_t dst = dst0 + f * kFragBytes;
-          if (!PLANES) {
-            const int rr = q >> 2, cc = q & 3;
-            src = blob + P.code_off[m] + static_cast<size_t>(frow(f) + rr) * (P.K / 2) + s * 64 + cc * 16;
-            dst += rr * 64 + cc * 16;
-          } else if (q < 32) {  // Q2: 16 rows x 32 B
-            const int rr = q >> 1, hh = q & 1;
-            src = blob + P.code_off[m] + static_cast<size_t>(frow(f) + rr) * (P.K / 4) + s * 32 + hh * 16;
-            dst += rr * 32 + hh * 16;
-          } else if (q < 48) {  // D3: 16 rows x 16 B
-            const int rr = q - 32;
-            if (bits >= 3) src = blob + P.d3_off[m] + static_cast<size_t>(frow(f) + rr) * (P.K / 8) + s * 16;
-            dst += 512 + rr * 16;
-          } else {  // D4
-            const int rr = q - 48;
-            if (bits >= 4) src = blob + P.d4_off[m] + static_cast<size_t>(frow(f) + rr) * (P.K / 8) + s * 16;
-            dst += 768 + rr * 16;
-          }
-          if (src) cp_async16(dst, src);
-        }
-        // scale/zero: rows frow(f)..+15 of group gi: 64 contiguous bytes
-        const int npieces = G64 ? 8 : 4;
-        if (lane < npieces) {
-          const int gi = lane >> 2, pc = lane & 3;
-          const int row = frow(f);
-          const int grp = s * kStageK / P.group + gi;
-          const uint8_t* src = blob + P.sz_off[m] +
-                               ((static_cast<size_t>(row >> 7) * G + grp) * 128 + (row & 127)) * 4 + pc * 16;
-          cp_async16(dst0 + FW * kFragBytes + f * kSzBytes + gi * 64 + pc * 16, src);
-        }
+        cp_async16(dst0 + dst[f][0], src[f][0] + s * kStep0);
+        if (!PLANES || src[f][1]) cp_async16(dst0 + dst[f][1], src[f][1] + s * kStep1);
+        if (sz_lane)
+          cp_async16(dst0 + FW * kFragBytes + f * kSzBytes + ((lane >> 2) & 1) * 64 + (lane & 3) * 16,
+                     sz_src[f] + s * sz_step);
       }
     }
     cp_async_commit();  // an empty group past the end keeps the count uniform
@@ -247,25 +254,37 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
       pdl_trigger();
       waited = true;
     }
-    // token rows of this lane's B fragments
+    // this lane's run of each token row it feeds (token g of each 8-token
+    // block), advanced by one stage of this warp (8 x 128 K) per iteration
     bool tok_in[NB];
-    const __half* xrow[NB];
+    const __half* xp[NB];
+    int ntok = 0;  // token rows of this pass
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       const int tk = t0 + 8 * nb + g;
       tok_in[nb] = tk < nrows;
-      xrow[nb] = P.act + static_cast<size_t>(row0 + (tok_in[nb] ? tk : 0)) * P.K;
+      xp[nb] = P.act + static_cast<size_t>(row0 + (tok_in[nb] ? tk : 0)) * P.K + warp * kStageK + 32 * c;
+    }
+    ntok = min(8 * NB, nrows - t0);
+    // the pass's activation runs into L1 ahead of their use when they fit
+    // (a stage's 128 K of one token row is two 128-byte lines)
+    if (ntok * P.K * 2 <= (48 << 10) && (c & 1) == 0) {
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+        if (tok_in[nb])
+          for (int i = 0; i < my_stages; ++i)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(xp[nb] + i * kWarps * kStageK));
     }
     for (int i = 0; i < my_stages; ++i) {
-      const int s = warp + kWarps * i;
-      const int kl = s * kStageK + 32 * c;  // this lane's K run
       // activations (4 x 8 elements per token block), loaded before the wait
       uint4 xv[NB][4];
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
+      for (int nb = 0; nb < NB; ++nb) {
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd)
-          xv[nb][wd] = tok_in[nb] ? ldg_act(xrow[nb] + kl + 8 * wd) : make_uint4(0, 0, 0, 0);
+          xv[nb][wd] = tok_in[nb] ? ldg_act(xp[nb] + 8 * wd) : make_uint4(0, 0, 0, 0);
+        xp[nb] += kWarps * kStageK;
+      }
       cp_async_wait<kRing - 1>();
       __syncwarp();
       const uint8_t* sb = ring + (i % kRing) * kSlot;
@@ -275,12 +294,15 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
         const uint32_t* szw = reinterpret_cast<const uint32_t*>(sb + FW * kFragBytes + f * kSzBytes);
         const int gsel = G64 ? (c >> 1) * 16 : 0;  // this lane's group inside the stage
         const uint32_t wlo = szw[gsel + g], whi = szw[gsel + g + 8];
-        const float zlo_f = __uint_as_float(wlo & 0xFFFF0000u), zhi_f = __uint_as_float(whi & 0xFFFF0000u);
         const float slo = __uint_as_float(wlo << 16), shi = __uint_as_float(whi << 16);
-        const __half2 za_lo = __half2half2(__float2half_rn(1024.0f + zlo_f));
-        const __half2 za_hi = __half2half2(__float2half_rn(64.0f + zlo_f));
-        const __half2 zb_lo = __half2half2(__float2half_rn(1024.0f + zhi_f));
-        const __half2 zb_hi = __half2half2(__float2half_rn(64.0f + zhi_f));
+        // zero-points are integers 0..15: 1024 + z and 64 + z as fp16 bit
+        // patterns (units 1 and 1/16 of the mantissa), in both halves
+        const uint32_t zi_lo = static_cast<uint32_t>(__float2int_rz(__uint_as_float(wlo & 0xFFFF0000u)));
+        const uint32_t zi_hi = static_cast<uint32_t>(__float2int_rz(__uint_as_float(whi & 0xFFFF0000u)));
+        const __half2 za_lo = u2h(0x64006400u + zi_lo * 0x10001u);
+        const __half2 za_hi = u2h(0x54005400u + (zi_lo << 4) * 0x10001u);
+        const __half2 zb_lo = u2h(0x64006400u + zi_hi * 0x10001u);
+        const __half2 zb_hi = u2h(0x54005400u + (zi_hi << 4) * 0x10001u);
         // this lane's 32 elements of rows g and g + 8 as four code words each
         uint32_t ca[4], cb[4];
         if (!PLANES) {
@@ -309,11 +331,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
             }
           }
         }
-        float dsum[NB][4];
+        // two accumulation chains per token block (even and odd MMAs of the
+        // stage), so that consecutive MMAs do not wait for each other
+        float dsum[NB][2][4];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) dsum[nb][j] = 0.0f;
+          for (int j = 0; j < 4; ++j) dsum[nb][0][j] = dsum[nb][1][j] = 0.0f;
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd) {
           uint32_t pa[4], pb[4];
@@ -343,17 +367,17 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
               if (G64)
                 mma16816(acc[f][nb], pa[2 * hh], pb[2 * hh], pa[2 * hh + 1], pb[2 * hh + 1], b0, b1);
               else
-                mma16816(dsum[nb], pa[2 * hh], pb[2 * hh], pa[2 * hh + 1], pb[2 * hh + 1], b0, b1);
+                mma16816(dsum[nb][hh], pa[2 * hh], pb[2 * hh], pa[2 * hh + 1], pb[2 * hh + 1], b0, b1);
             }
           }
         }
         if (!G64) {
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb) {
-            acc[f][nb][0] = fmaf(slo, dsum[nb][0], acc[f][nb][0]);
-            acc[f][nb][1] = fmaf(slo, dsum[nb][1], acc[f][nb][1]);
-            acc[f][nb][2] = fmaf(shi, dsum[nb][2], acc[f][nb][2]);
-            acc[f][nb][3] = fmaf(shi, dsum[nb][3], acc[f][nb][3]);
+            acc[f][nb][0] = fmaf(slo, dsum[nb][0][0] + dsum[nb][1][0], acc[f][nb][0]);
+            acc[f][nb][1] = fmaf(slo, dsum[nb][0][1] + dsum[nb][1][1], acc[f][nb][1]);
+            acc[f][nb][2] = fmaf(shi, dsum[nb][0][2] + dsum[nb][1][2], acc[f][nb][2]);
+            acc[f][nb][3] = fmaf(shi, dsum[nb][0][3] + dsum[nb][1][3], acc[f][nb][3]);
           }
         }
       }

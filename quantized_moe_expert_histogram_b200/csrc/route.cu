@@ -464,6 +464,48 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
   select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, blockIdx.x);
 }
 
+// Partial logits of slice `split` (dk wide) for a handful of tokens: a warp
+// per (token, expert) pair, lanes over the slice (four elements per lane per
+// 128, an FMA chain per lane, then a shuffle tree), so that no work is spent
+// on the empty rows of a 64-token tile.  The chain per lane, the tree and the
+// later sum over slices stay within the chunked bound g(32 + d/32) of the
+// tiled path.  The norms of the slice: pairs with e = 0 sum x^2, pairs with
+// t = 0 sum W^2.
+__device__ __forceinline__ void logits_pairs(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr,
+                                             int T, int d, int E, int dk, RouteWs ws, int split) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k0 = split * dk;
+  for (int pr = warp; pr < T * E; pr += kSelWarps) {
+    const int t = pr / E, e = pr - t * E;
+    const __nv_bfloat16* xr = x + static_cast<size_t>(t) * d + k0;
+    const float* w = wr + static_cast<size_t>(e) * d + k0;
+    float acc = 0.f, xq = 0.f, wq = 0.f;
+    for (int i = lane * 4; i < dk; i += 128) {
+      const uint2 xb = *reinterpret_cast<const uint2*>(xr + i);
+      const float4 wv = *reinterpret_cast<const float4*>(w + i);
+      const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb.x));
+      const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb.y));
+      acc = fmaf(x01.x, wv.x, acc);
+      acc = fmaf(x01.y, wv.y, acc);
+      acc = fmaf(x23.x, wv.z, acc);
+      acc = fmaf(x23.y, wv.w, acc);
+      xq = fmaf(x01.x, x01.x, fmaf(x01.y, x01.y, fmaf(x23.x, x23.x, fmaf(x23.y, x23.y, xq))));
+      wq = fmaf(wv.x, wv.x, fmaf(wv.y, wv.y, fmaf(wv.z, wv.z, fmaf(wv.w, wv.w, wq))));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      xq += __shfl_xor_sync(0xffffffffu, xq, o);
+      wq += __shfl_xor_sync(0xffffffffu, wq, o);
+    }
+    if (lane == 0) {
+      ws.partial[(static_cast<size_t>(split) * T + t) * E + e] = acc;
+      if (e == 0) ws.xsq[static_cast<size_t>(split) * T + t] = xq;
+      if (t == 0) ws.wsq[static_cast<size_t>(split) * E + e] = wq;
+    }
+  }
+}
+
 // Both steps in one launch for decode-sized batches (one token tile, one
 // expert tile): the CTAs of one thread-block cluster take one slice of d
 // each (threads 0..kLT-1 write the slice's partial logits and norms to the
@@ -479,7 +521,10 @@ __global__ void __launch_bounds__(kSelThreads) k_route_small(
   pdl_trigger();
   extern __shared__ __align__(16) float sm[];
   const int rank = blockIdx.x;  // the grid is one cluster
-  if (threadIdx.x < kLT) logits_tile<EC>(x, wr, T, d, E, dk, ws, 0, 0, rank, sm);
+  if (T <= kSelWarps)
+    logits_pairs(x, wr, T, d, E, dk, ws, rank);
+  else if (threadIdx.x < kLT)
+    logits_tile<EC>(x, wr, T, d, E, dk, ws, 0, 0, rank, sm);
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   if (rank * kSelWarps < T)
     select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, rank);
