@@ -150,10 +150,9 @@ MOE_API size_t moe_route_workspace_bytes(int T, int d, int E);
 
 /* moe_route_topk_noalloc -- the same router with no workspace argument.
  * (Library plumbing: the pages describe no counterpart.)  For callers that
- * cannot allocate device memory where they route: code running during
- * CUDA graph stream capture (no cudaMalloc allowed), plugins that receive
- * only a stream and no allocator, and serving paths that must not risk an
- * allocation failure or its implicit synchronisation.  The scratch lives in
+ * cannot allocate device memory where they route: plugins and runtimes that
+ * receive only a stream and no allocator, and serving paths that must not
+ * risk an allocation failure or its implicit synchronisation.  The scratch lives in
  * a fixed 8 MiB device array inside the library, which every GPU that loads
  * the library holds until the process exits; the call allocates nothing.
  *   - Arguments and results are those of moe_route_topk (expert ids equal

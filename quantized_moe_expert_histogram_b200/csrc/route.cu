@@ -649,11 +649,9 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
 // Allocation-free router entry point.
 //
 // Some callers cannot allocate device memory at the point where they route:
-// code that runs while a stream is being captured into a CUDA graph (where
-// cudaMalloc is not allowed), plugins and runtimes that hand us only a
-// stream and have no allocator of their own to lend, and latency-critical
-// serving paths that must not risk an allocation failure or an implicit
-// synchronisation.  moe_route_topk_noalloc keeps the router's scratch (the
+// plugins and runtimes that hand us only a stream and have no allocator of
+// their own to lend, and latency-critical serving paths that must not risk
+// an allocation failure or an implicit synchronisation.  moe_route_topk_noalloc keeps the router's scratch (the
 // per-slice fp32 partial logits and squared norms) in a fixed device array
 // owned by this library instead of a caller-provided workspace; the number
 // of d slices is capped so that the scratch fits the array.

@@ -1,9 +1,9 @@
 """The allocation-free router entry point (moe_route_topk_noalloc) against
 the workspace-taking one (moe_route_topk), through the C ABI.
 
-Callers that cannot allocate device memory where they route (graph
-capture, allocator-less plugins, latency-critical serving) use the
-noalloc variant, whose scratch is a fixed array inside the library.  Its
+Callers that cannot allocate device memory where they route (plugins
+handed only a stream, latency-critical serving paths) use the noalloc
+variant, whose scratch is a fixed array inside the library.  Its
 results must equal the regular router's: the same expert ids bit for bit
 and the same gates, on two calls in a row (the second reuses the array).
 This file is collected last so that a failure here never hides another."""
