@@ -548,18 +548,19 @@ def main():
     B.build()
     world, rank, local = dist_setup(args)
     moeq.load()
-    shape = I.SHAPES[args.workload]
+    gate = args.workload == "nested_gate"  # nested layer, widths from the bit gate
+    shape = I.SHAPES["nested" if gate else args.workload]
     T = args.tokens
     peaks = load_peaks()
     stream = torch.cuda.Stream()
     if args.profile:
-        layers = make_instances(shape, T, 1, seed=0, device="cuda")
+        layers = make_instances(shape, T, 1, seed=0, device="cuda", bit_gate=gate)
         for _ in range(args.warmup + args.steps):
             _step_calls(*layers[0], stream, "all")
         torch.cuda.synchronize()
         print(f"profile run done: {shape.name} T={T} steps={args.warmup + args.steps}")
         return
-    layers = make_instances(shape, T, args.instances, seed=rank * 7919, device="cuda")
+    layers = make_instances(shape, T, args.instances, seed=rank * 7919, device="cuda", bit_gate=gate)
     torch.cuda.synchronize()
 
     R = len(layers)

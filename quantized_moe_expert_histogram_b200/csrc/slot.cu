@@ -4,7 +4,9 @@
 //
 // A layer-step's distinct experts are ordered hits first, then the experts
 // that need copies by descending row count (the hottest expert is loaded
-// first), and cut into waves of at most slots/2 experts.  Waves alternate
+// first; in plane mode resident experts that need more planes before the
+// ones that are not resident), and cut into waves of at most slots/2
+// experts.  Waves alternate
 // between slot sets in LRU order and never into a slot of the previous wave,
 // so the copies of wave w+1 overlap the compute of wave w (load E2 while
 // computing E1).  A slot is overwritten only after the compute that last
@@ -371,17 +373,25 @@ moe_status_t moe_slot_stage(moe_slot_cache* c, const int32_t* ids_host, const ui
     ++cnt[e];
     need[e] = std::max(need[e], b);
   }
-  // hits: resident with every plane the step needs; the others need copies
-  // (a fresh load, or in plane mode the missing planes of a resident expert)
-  std::vector<int> hits, copies;
+  // hits: resident with every plane the step needs; upgrades (plane mode):
+  // resident but missing planes; misses: not resident.  Resident experts
+  // come first (hits, then upgrades hottest first), then misses hottest
+  // first, so that every wave after them holds only experts that are not
+  // resident yet -- the slots a later wave pins are then only those of the
+  // wave before it.
+  std::vector<int> hits, upgrades, misses;
   for (int e = 0; e < c->E; ++e) {
     if (!cnt[e]) continue;
     const int s = c->slot_of[e];
-    (s >= 0 && c->width_in[s] >= need[e] ? hits : copies).push_back(e);
+    if (s < 0) misses.push_back(e);
+    else (c->width_in[s] >= need[e] ? hits : upgrades).push_back(e);
   }
-  std::stable_sort(copies.begin(), copies.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
+  auto hotter = [&](int a, int b) { return cnt[a] > cnt[b]; };
+  std::stable_sort(upgrades.begin(), upgrades.end(), hotter);
+  std::stable_sort(misses.begin(), misses.end(), hotter);
   std::vector<int> order(hits);
-  order.insert(order.end(), copies.begin(), copies.end());
+  order.insert(order.end(), upgrades.begin(), upgrades.end());
+  order.insert(order.end(), misses.begin(), misses.end());
   const int W = std::max(1, c->S / 2);
   const int nw = static_cast<int>((order.size() + W - 1) / W);
   c->waves.assign(nw, {});
