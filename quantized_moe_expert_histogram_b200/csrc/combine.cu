@@ -35,17 +35,35 @@ __global__ void __launch_bounds__(256) k_combine(const __half* __restrict__ y_pe
 #pragma unroll
       for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
     }
-    for (int j = 0; j < k; ++j) {
-      const float g = gw[static_cast<size_t>(t) * k + j];
-      // clamped: an inconsistent inv_perm gives wrong rows, never an out-of-range read
-      const int p = min(max(inv_perm[static_cast<size_t>(t) * k + j], 0), T * k - 1);
-      const uint4 raw = *reinterpret_cast<const uint4*>(y_perm + static_cast<size_t>(p) * d + c);
-      const __half2* v2 = reinterpret_cast<const __half2*>(&raw);
+    // up to 8 choices at a time: their gates and rows are loaded before any
+    // is summed (independent loads in flight), the sum stays in ascending j
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      float g[8];
+      int p[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 f = __half22float2(v2[u]);
-        acc[2 * u] = fmaf(g, f.x, acc[2 * u]);
-        acc[2 * u + 1] = fmaf(g, f.y, acc[2 * u + 1]);
+      for (int u = 0; u < 8; ++u) {
+        g[u] = 0.0f;
+        p[u] = 0;
+        if (j0 + u < k) {
+          g[u] = gw[static_cast<size_t>(t) * k + j0 + u];
+          // clamped: an inconsistent inv_perm gives wrong rows, never an out-of-range read
+          p[u] = min(max(inv_perm[static_cast<size_t>(t) * k + j0 + u], 0), T * k - 1);
+        }
+      }
+      uint4 raw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j0 + u < k) raw[u] = *reinterpret_cast<const uint4*>(y_perm + static_cast<size_t>(p[u]) * d + c);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (j0 + u >= k) break;
+        const __half2* v2 = reinterpret_cast<const __half2*>(&raw[u]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __half22float2(v2[q]);
+          acc[2 * q] = fmaf(g[u], f.x, acc[2 * q]);
+          acc[2 * q + 1] = fmaf(g[u], f.y, acc[2 * q + 1]);
+        }
       }
     }
     uint4 o;

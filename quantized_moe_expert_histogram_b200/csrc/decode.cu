@@ -132,26 +132,49 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// D += A B (register-only: the compiler may schedule it freely)
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ldg_act(const __half* p) {
+// D = A B (a fresh accumulator)
+__device__ __forceinline__ void mma16816_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+__device__ __forceinline__ uint4 ldg_act(const __half* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
   uint4 r;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
+  return r;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 r;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a));
+  return r;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t r;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(a));
   return r;
 }
 
 // GU: first GEMM (fragment 0 = gate rows, 1 = up rows of 16 features);
 // else the second GEMM (FW fragments of 16 consecutive W_down rows).  NB
 // token blocks of 8 per pass over K (bins with more rows take more passes).
+// Residency: three CTAs per SM (24 warps, <= 80 registers) with one token
+// block; two with two token blocks, whose B operands need more registers.
 template <bool GU, bool PLANES, bool G64, int FW, int NB>
-__global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
+__global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecParams P) {
   static_assert(!GU || FW == 2, "gate and up fragments");
   constexpr int kSlot = FW * (kFragBytes + kSzBytes);  // one ring stage of a warp
   extern __shared__ __align__(16) uint8_t smem[];
@@ -172,8 +195,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
   const uint8_t* blob = P.blobs + static_cast<size_t>(slot) * P.blob_bytes;
   const int n_stages = P.K / kStageK;
   const int G = P.K / P.group;
-  uint8_t* ring = smem + warp * (kRing * kSlot);
-  const uint32_t ring_u = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
+  const uint32_t ring_u = static_cast<uint32_t>(__cvta_generic_to_shared(smem + warp * (kRing * kSlot)));
   // weight row of fragment f: matrix mat(f), row frow(f) + 0..15
   auto mat = [](int f) { return GU ? f : 0; };
   auto frow = [&](int f) { return GU ? n0 : n0 + 16 * f; };
@@ -216,20 +238,32 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
   }
   const bool sz_lane = lane < (G64 ? 8 : 4);
 
+  const uint32_t sz_dst = FW * kFragBytes + ((lane >> 2) & 1) * 64 + (lane & 3) * 16;
+  // sources of the next stage this warp issues (stage warp, then + 8 each time)
+#pragma unroll
+  for (int f = 0; f < FW; ++f) {
+    src[f][0] += warp * kStep0;
+    if (!PLANES || src[f][1]) src[f][1] += warp * kStep1;
+    sz_src[f] += warp * sz_step;
+  }
+
   // copies of this warp's i-th stage (global stage warp + 8 i) into ring
-  // slot i % kRing
+  // slot i % kRing; called for i = 0, 1, 2, ... in order
   auto issue = [&](int i) {
-    const int s = warp + kWarps * i;
-    if (s < n_stages) {
+    if (warp + kWarps * i < n_stages) {
       const uint32_t dst0 = ring_u + (i % kRing) * kSlot;
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
-        cp_async16(dst0 + dst[f][0], src[f][0] + s * kStep0);
-        if (!PLANES || src[f][1]) cp_async16(dst0 + dst[f][1], src[f][1] + s * kStep1);
-        if (sz_lane)
-          cp_async16(dst0 + FW * kFragBytes + f * kSzBytes + ((lane >> 2) & 1) * 64 + (lane & 3) * 16,
-                     sz_src[f] + s * sz_step);
+        cp_async16(dst0 + dst[f][0], src[f][0]);
+        if (!PLANES || src[f][1]) cp_async16(dst0 + dst[f][1], src[f][1]);
+        if (sz_lane) cp_async16(dst0 + sz_dst + f * kSzBytes, sz_src[f]);
       }
+    }
+#pragma unroll
+    for (int f = 0; f < FW; ++f) {
+      src[f][0] += kWarps * kStep0;
+      if (!PLANES || src[f][1]) src[f][1] += kWarps * kStep1;
+      sz_src[f] += kWarps * sz_step;
     }
     cp_async_commit();  // an empty group past the end keeps the count uniform
   };
@@ -287,13 +321,12 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
       }
       cp_async_wait<kRing - 1>();
       __syncwarp();
-      const uint8_t* sb = ring + (i % kRing) * kSlot;
+      const uint32_t sb = ring_u + (i % kRing) * kSlot;  // this stage's ring slot
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
-        const uint8_t* fb = sb + f * kFragBytes;
-        const uint32_t* szw = reinterpret_cast<const uint32_t*>(sb + FW * kFragBytes + f * kSzBytes);
-        const int gsel = G64 ? (c >> 1) * 16 : 0;  // this lane's group inside the stage
-        const uint32_t wlo = szw[gsel + g], whi = szw[gsel + g + 8];
+        const uint32_t fb = sb + f * kFragBytes;
+        const uint32_t szw = sb + FW * kFragBytes + f * kSzBytes + (G64 ? (c >> 1) * 64 : 0) + g * 4;
+        const uint32_t wlo = lds32(szw), whi = lds32(szw + 32);  // rows g and g + 8
         const float slo = __uint_as_float(wlo << 16), shi = __uint_as_float(whi << 16);
         // zero-points are integers 0..15: 1024 + z and 64 + z as fp16 bit
         // patterns (units 1 and 1/16 of the mantissa), in both halves
@@ -306,8 +339,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
         // this lane's 32 elements of rows g and g + 8 as four code words each
         uint32_t ca[4], cb[4];
         if (!PLANES) {
-          const uint4 va = *reinterpret_cast<const uint4*>(fb + g * 64 + c * 16);
-          const uint4 vb = *reinterpret_cast<const uint4*>(fb + (g + 8) * 64 + c * 16);
+          const uint4 va = lds128(fb + g * 64 + c * 16);
+          const uint4 vb = lds128(fb + (g + 8) * 64 + c * 16);
           ca[0] = va.x; ca[1] = va.y; ca[2] = va.z; ca[3] = va.w;
           cb[0] = vb.x; cb[1] = vb.y; cb[2] = vb.z; cb[3] = vb.w;
         } else {
@@ -316,9 +349,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             const int r = g + 8 * half;
-            const uint2 q2 = *reinterpret_cast<const uint2*>(fb + r * 32 + c * 8);
-            const uint32_t d3 = bits >= 3 ? *reinterpret_cast<const uint32_t*>(fb + 512 + r * 16 + c * 4) : 0u;
-            const uint32_t d4 = bits >= 4 ? *reinterpret_cast<const uint32_t*>(fb + 768 + r * 16 + c * 4) : 0u;
+            const uint2 q2 = lds64(fb + r * 32 + c * 8);
+            const uint32_t d3 = bits >= 3 ? lds32(fb + 512 + r * 16 + c * 4) : 0u;
+            const uint32_t d4 = bits >= 4 ? lds32(fb + 768 + r * 16 + c * 4) : 0u;
             uint32_t* cw = half ? cb : ca;
             const uint32_t qw[2] = {q2.x, q2.y};
 #pragma unroll
@@ -332,12 +365,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
           }
         }
         // two accumulation chains per token block (even and odd MMAs of the
-        // stage), so that consecutive MMAs do not wait for each other
+        // stage), so that consecutive MMAs do not wait for each other; the
+        // first MMA of each chain starts from zero
         float dsum[NB][2][4];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) dsum[nb][0][j] = dsum[nb][1][j] = 0.0f;
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd) {
           uint32_t pa[4], pb[4];
@@ -366,6 +396,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
               }
               if (G64)
                 mma16816(acc[f][nb], pa[2 * hh], pb[2 * hh], pa[2 * hh + 1], pb[2 * hh + 1], b0, b1);
+              else if (wd == 0)
+                mma16816_first(dsum[nb][hh], pa[2 * hh], pb[2 * hh], pa[2 * hh + 1], pb[2 * hh + 1], b0, b1);
               else
                 mma16816(dsum[nb][hh], pa[2 * hh], pb[2 * hh], pa[2 * hh + 1], pb[2 * hh + 1], b0, b1);
             }
@@ -385,6 +417,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_dec(const DecParams P) {
       issue(i + kRing);
     }
     cp_async_wait<0>();
+    // back to this warp's first stage for a further pass over K
+#pragma unroll
+    for (int f = 0; f < FW; ++f) {
+      src[f][0] -= (kRing + my_stages) * kWarps * kStep0;
+      if (!PLANES || src[f][1]) src[f][1] -= (kRing + my_stages) * kWarps * kStep1;
+      sz_src[f] -= (kRing + my_stages) * kWarps * sz_step;
+    }
     __syncthreads();  // every warp's ring is drained: the space becomes the reduction buffer
 #pragma unroll
     for (int f = 0; f < FW; ++f)

@@ -465,9 +465,10 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
 }
 
 // Partial logits of slice `split` (dk wide) for a handful of tokens: a warp
-// per (token, expert) pair, lanes over the slice (four elements per lane per
-// 128, an FMA chain per lane, then a shuffle tree), so that no work is spent
-// on the empty rows of a 64-token tile.  The chain per lane, the tree and the
+// per (token, expert) pair, four pairs per warp at a time with their loads in
+// flight together, lanes over the slice (four elements per lane per 128, an
+// FMA chain per lane, then a shuffle tree), so that no work is spent on the
+// empty rows of a 64-token tile.  The chain per lane, the tree and the
 // later sum over slices stay within the chunked bound g(32 + d/32) of the
 // tiled path.  The norms of the slice: pairs with e = 0 sum x^2, pairs with
 // t = 0 sum W^2.
@@ -475,33 +476,47 @@ __device__ __forceinline__ void logits_pairs(const __nv_bfloat16* __restrict__ x
                                              int T, int d, int E, int dk, RouteWs ws, int split) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k0 = split * dk;
-  for (int pr = warp; pr < T * E; pr += kSelWarps) {
-    const int t = pr / E, e = pr - t * E;
-    const __nv_bfloat16* xr = x + static_cast<size_t>(t) * d + k0;
-    const float* w = wr + static_cast<size_t>(e) * d + k0;
-    float acc = 0.f, xq = 0.f, wq = 0.f;
+  constexpr int kP = 4;  // pairs of a warp whose loads are in flight together
+  for (int p0 = warp * kP; p0 < T * E; p0 += kSelWarps * kP) {
+    float acc[kP], xq[kP], wq[kP];
+#pragma unroll
+    for (int u = 0; u < kP; ++u) acc[u] = xq[u] = wq[u] = 0.f;
     for (int i = lane * 4; i < dk; i += 128) {
-      const uint2 xb = *reinterpret_cast<const uint2*>(xr + i);
-      const float4 wv = *reinterpret_cast<const float4*>(w + i);
-      const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb.x));
-      const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb.y));
-      acc = fmaf(x01.x, wv.x, acc);
-      acc = fmaf(x01.y, wv.y, acc);
-      acc = fmaf(x23.x, wv.z, acc);
-      acc = fmaf(x23.y, wv.w, acc);
-      xq = fmaf(x01.x, x01.x, fmaf(x01.y, x01.y, fmaf(x23.x, x23.x, fmaf(x23.y, x23.y, xq))));
-      wq = fmaf(wv.x, wv.x, fmaf(wv.y, wv.y, fmaf(wv.z, wv.z, fmaf(wv.w, wv.w, wq))));
+      uint2 xb[kP];
+      float4 wv[kP];
+#pragma unroll
+      for (int u = 0; u < kP; ++u) {
+        const int pr = min(p0 + u, T * E - 1), t = pr / E, e = pr - t * E;
+        xb[u] = *reinterpret_cast<const uint2*>(x + static_cast<size_t>(t) * d + k0 + i);
+        wv[u] = *reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * d + k0 + i);
+      }
+#pragma unroll
+      for (int u = 0; u < kP; ++u) {
+        const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb[u].x));
+        const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb[u].y));
+        acc[u] = fmaf(x01.x, wv[u].x, acc[u]);
+        acc[u] = fmaf(x01.y, wv[u].y, acc[u]);
+        acc[u] = fmaf(x23.x, wv[u].z, acc[u]);
+        acc[u] = fmaf(x23.y, wv[u].w, acc[u]);
+        xq[u] = fmaf(x01.x, x01.x, fmaf(x01.y, x01.y, fmaf(x23.x, x23.x, fmaf(x23.y, x23.y, xq[u]))));
+        wq[u] = fmaf(wv[u].x, wv[u].x, fmaf(wv[u].y, wv[u].y, fmaf(wv[u].z, wv[u].z, fmaf(wv[u].w, wv[u].w, wq[u]))));
+      }
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      xq += __shfl_xor_sync(0xffffffffu, xq, o);
-      wq += __shfl_xor_sync(0xffffffffu, wq, o);
-    }
-    if (lane == 0) {
-      ws.partial[(static_cast<size_t>(split) * T + t) * E + e] = acc;
-      if (e == 0) ws.xsq[static_cast<size_t>(split) * T + t] = xq;
-      if (t == 0) ws.wsq[static_cast<size_t>(split) * E + e] = wq;
+    for (int u = 0; u < kP; ++u) {
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+        xq[u] += __shfl_xor_sync(0xffffffffu, xq[u], o);
+        wq[u] += __shfl_xor_sync(0xffffffffu, wq[u], o);
+      }
+      const int pr = p0 + u;
+      if (lane == 0 && pr < T * E) {
+        const int t = pr / E, e = pr - t * E;
+        ws.partial[(static_cast<size_t>(split) * T + t) * E + e] = acc[u];
+        if (e == 0) ws.xsq[static_cast<size_t>(split) * T + t] = xq[u];
+        if (t == 0) ws.wsq[static_cast<size_t>(split) * E + e] = wq[u];
+      }
     }
   }
 }
