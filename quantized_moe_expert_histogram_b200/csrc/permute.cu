@@ -162,7 +162,8 @@ __global__ void __launch_bounds__(1024) k_perm_scan(int32_t* __restrict__ hist, 
 // Scatter of this CTA's assignments once hist_s[w][b] holds the first
 // position of warp w's keys in bin b.
 __device__ __forceinline__ void scatter(const int (&keys)[kSlices], int32_t* hist_s, int nbins,
-                                        int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
+                                        int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+                                        int32_t* perm_s = nullptr) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned lt_mask = (1u << lane) - 1u;
   int32_t* my = hist_s + warp * nbins;
@@ -176,6 +177,7 @@ __device__ __forceinline__ void scatter(const int (&keys)[kSlices], int32_t* his
       const int p = my[key] + __popc(peers & lt_mask);
       perm[p] = a;
       inv_perm[a] = p;
+      if (perm_s) perm_s[p] = a;  // single-CTA path: a copy for the gather
     }
     __syncwarp();
     if (key >= 0 && (peers & lt_mask) == 0) my[key] += __popc(peers);
@@ -309,10 +311,11 @@ __global__ void __launch_bounds__(kWarps * 32) k_perm_one(
   }
   if (tid == 0) offsets[nbins] = n;
   __syncthreads();
-  scatter(keys, hist_s, nbins, perm, inv_perm);
-  if (x_perm) {  // small batches: the gather too (perm is visible to the block after the barrier)
+  __shared__ int32_t perm_s[kCH];  // n <= kCH here
+  scatter(keys, hist_s, nbins, perm, inv_perm, perm_s);
+  if (x_perm) {  // small batches: the gather too, from the block's copy of perm
     __syncthreads();
-    if (gather_rows(x, perm, n, k, d, x_perm, warp, kWarps)) flag_status(status, MOE_DEV_RANGE);
+    if (gather_rows(x, perm_s, n, k, d, x_perm, warp, kWarps)) flag_status(status, MOE_DEV_RANGE);
   }
 }
 
