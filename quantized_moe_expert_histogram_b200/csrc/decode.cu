@@ -11,15 +11,19 @@
 // K run spans two groups, A holds (q - z) * s rounded once to fp16, as in
 // the 128-row kernel).
 //
-// Work split: a CTA (8 warps) owns one item = (bin, block of weight rows):
-// 16 features x {gate, up} in the first GEMM, 16 or 32 rows of W_down in
-// the second, and its warps split K: warp w takes the 128-K stages w, w+8,
-// w+16, ... of every row of the item (so a 14336-long row is eight warps'
-// work, and at any time the CTA reads a contiguous K window of each row).
-// Each warp streams its stages with cp.async into a 4-deep shared-memory
-// ring (the bytes in flight take no registers).  The warps' partial sums
-// are added in shared memory in a fixed order (deterministic), and the
-// epilogue writes h = silu(gate) * up or y_perm (fp16).
+// Work split: a work unit is (bin, block of weight rows, pass over 8 NB of
+// the bin's token rows): 16 features x {gate, up} in the first GEMM, 16 or
+// 32 rows of W_down in the second.  The grid is persistent (as many CTAs as
+// fit on the GPU at once); CTA b takes units b, b + grid, ...  The 8 warps
+// of a CTA split each unit's K: warp w takes the 128-K stages w, w+8, w+16,
+// ... of every row of the unit (so a 14336-long row is eight warps' work,
+// and at any time the CTA reads a contiguous K window of each row).  Each
+// warp streams its stages with cp.async into a shared-memory ring (the bytes
+// in flight take no registers), and the stream runs on across units: the
+// next unit's first stages are in flight while the current unit's partial
+// sums are added (in shared memory, in a fixed order: deterministic) and its
+// epilogue writes h = silu(gate) * up or y_perm (fp16).  The non-empty,
+// resident bins are listed once per CTA in shared memory.
 //
 // Register layout of one MMA, lane = (g, c) = (lane / 4, lane % 4): A rows g
 // and g + 8, K slots {2c, 2c+1, 2c+8, 2c+9}; B token g at the same slots;
@@ -31,7 +35,7 @@
 // words, (2j, 2j + 1) for plane-order words.
 //
 // Both passes are programmatic dependent launches (launch_pdl).  The down
-// pass locates its bin and issues the copies of its first weight stages
+// pass lists its bins and issues the copies of its first weight stages
 // (which do not depend on h) before it waits for the gate/up grid.
 //
 //   gate/up pass:  h[p][f]      = silu(Wg[f] . x_p) * (Wu[f] . x_p)   (fp16)
@@ -48,7 +52,7 @@ constexpr int kWarps = 8;
 constexpr int kStageK = 128;       // K per stage (one group of 128, two of 64)
 constexpr int kFragBytes = 1024;   // one stage of one 16-row fragment: 16 rows x 64 B
 constexpr int kSzBytes = 128;      // its scale/zero words: 16 rows x up to 2 groups
-constexpr int kRing = 4;           // stages in flight per warp
+constexpr int kRing = 3;           // stages in flight per warp
 
 struct DecParams {
   const __half* act;        // x_perm or h: fp16 [rows][K]
@@ -63,44 +67,16 @@ struct DecParams {
   int K, N, nbins, planes_mult;
   int rows;                 // activation rows: bin ranges are clamped into [0, rows]
   int group;
-  int row_blocks;           // items per bin (weight-row blocks)
+  int row_blocks;           // weight-row blocks per bin
+  int max_ent;              // capacity of the bin list (>= non-empty bins)
   __half* out;              // h (gate/up) or y_perm (down): fp16 [rows][N]
   int32_t* status;
 };
 
-// Locate the ordinal-th non-empty, resident bin (ballot over 32 bins at a
-// time).  Returns false when there is none.
-__device__ __forceinline__ bool find_bin(const DecParams& P, int ordinal, int& bin, int& row0, int& nrows,
-                                         int& slot, int& bits) {
-  const int lane = threadIdx.x & 31;
-  int seen = 0;
-  for (int b0 = 0; b0 < P.nbins; b0 += 32) {
-    const int b = b0 + lane;
-    bool ok = false;
-    int sl = 0;
-    if (b < P.nbins) {
-      const int n = min(max(P.offsets[b + 1], 0), P.rows) - min(max(P.offsets[b], 0), P.rows);
-      const int e = b / P.planes_mult;
-      sl = P.slot_of ? P.slot_of[e] : e;
-      ok = n > 0 && sl >= 0;
-    }
-    const unsigned m = __ballot_sync(0xffffffffu, ok);
-    const int cnt = __popc(m);
-    if (ordinal < seen + cnt) {
-      unsigned mm = m;
-      for (int i = 0; i < ordinal - seen; ++i) mm &= mm - 1;
-      const int src = __ffs(mm) - 1;
-      bin = b0 + src;
-      slot = __shfl_sync(0xffffffffu, sl, src);
-      row0 = min(max(P.offsets[bin], 0), P.rows);
-      nrows = max(0, min(max(P.offsets[bin + 1], 0), P.rows) - row0);
-      bits = P.planes_mult == 3 ? 2 + bin % 3 : 4;
-      return true;
-    }
-    seen += cnt;
-  }
-  return false;
-}
+// One listed bin: its rows, blob, width and its first work unit.
+struct BinEnt {
+  int row0, nrows, slot, bits, unit0;
+};
 
 __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t c) {
   uint32_t r;
@@ -168,139 +144,196 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   return r;
 }
 
+// Shared-memory layout of a CTA: the warps' rings, the reduction buffer,
+// the bin list.
+template <int FW, int NB>
+struct Smem {
+  static constexpr int kSlot = FW * (kFragBytes + kSzBytes);  // one ring stage of a warp
+  static constexpr int kVals = FW * NB * 4;                    // partial sums per lane
+  static constexpr int kRing0 = 0;
+  static constexpr int kRed0 = kWarps * kRing * kSlot;
+  static constexpr int kEnt0 = kRed0 + kWarps * kVals * 32 * 4;
+  static constexpr size_t bytes(int max_ent) { return kEnt0 + static_cast<size_t>(max_ent) * sizeof(BinEnt); }
+};
+
 // GU: first GEMM (fragment 0 = gate rows, 1 = up rows of 16 features);
 // else the second GEMM (FW fragments of 16 consecutive W_down rows).  NB
-// token blocks of 8 per pass over K (bins with more rows take more passes).
+// token blocks of 8 per pass over K.
 // Residency: three CTAs per SM (24 warps, <= 80 registers) with one token
 // block; two with two token blocks, whose B operands need more registers.
 template <bool GU, bool PLANES, bool G64, int FW, int NB>
 __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecParams P) {
   static_assert(!GU || FW == 2, "gate and up fragments");
-  constexpr int kSlot = FW * (kFragBytes + kSzBytes);  // one ring stage of a warp
+  using L = Smem<FW, NB>;
+  constexpr int kSlot = L::kSlot;
+  constexpr int kVals = L::kVals;
   extern __shared__ __align__(16) uint8_t smem[];
+  float* red = reinterpret_cast<float*>(smem + L::kRed0);
+  BinEnt* ent = reinterpret_cast<BinEnt*>(smem + L::kEnt0);
+  __shared__ int n_ent_s, n_units_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   if (GU) {  // x_perm comes from the previous launch
     pdl_wait();
     pdl_trigger();
   }
-  int bin, row0, nrows, slot, bits;
-  const int ordinal = blockIdx.x / P.row_blocks;
-  if (!find_bin(P, ordinal, bin, row0, nrows, slot, bits)) {
+  // ---- the non-empty, resident bins and their work units (warp 0): units
+  // of a bin = passes x row blocks, passes = ceil(rows / (8 NB))
+  if (warp == 0) {
+    int n_ent = 0, n_units = 0;
+    for (int b0 = 0; b0 < P.nbins; b0 += 32) {
+      const int b = b0 + lane;
+      int r0 = 0, nr = 0, sl = 0;
+      if (b < P.nbins) {
+        r0 = min(max(P.offsets[b], 0), P.rows);
+        nr = max(0, min(max(P.offsets[b + 1], 0), P.rows) - r0);
+        sl = P.slot_of ? P.slot_of[b / P.planes_mult] : b / P.planes_mult;
+      }
+      const bool ok = nr > 0 && sl >= 0;
+      const unsigned m = __ballot_sync(0xffffffffu, ok);
+      const int units = ok ? ((nr + 8 * NB - 1) / (8 * NB)) * P.row_blocks : 0;
+      int incl = units;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (ok) {
+        const int pos = n_ent + __popc(m & ((1u << lane) - 1u));
+        if (pos < P.max_ent)
+          ent[pos] = BinEnt{r0, nr, sl, P.planes_mult == 3 ? 2 + b % 3 : 4, n_units + incl - units};
+      }
+      n_ent += __popc(m);
+      n_units += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      n_ent_s = min(n_ent, P.max_ent);  // the list holds at most max_ent bins
+      n_units_s = n_ent <= P.max_ent ? n_units : 0;
+      if (n_ent > P.max_ent) flag_status(P.status, MOE_DEV_BAD_INDEX);
+    }
+  }
+  __syncthreads();
+  const int n_ent = n_ent_s, n_units = n_units_s;
+  const int my_units = static_cast<int>(blockIdx.x) < n_units ? (n_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (my_units == 0) {
     if (!GU) pdl_wait();  // CTA-uniform; keeps the wait/trigger order of every CTA
     return;
   }
-  const int rb = blockIdx.x - ordinal * P.row_blocks;
-  const int n0 = rb * (GU ? 16 : 16 * FW);  // first output row (feature) of this item
-  const uint8_t* blob = P.blobs + static_cast<size_t>(slot) * P.blob_bytes;
   const int n_stages = P.K / kStageK;
   const int G = P.K / P.group;
-  const uint32_t ring_u = static_cast<uint32_t>(__cvta_generic_to_shared(smem + warp * (kRing * kSlot)));
-  // weight row of fragment f: matrix mat(f), row frow(f) + 0..15
+  const int my_stages = n_stages > warp ? (n_stages - warp + kWarps - 1) / kWarps : 0;
+  const uint32_t ring_u = static_cast<uint32_t>(__cvta_generic_to_shared(smem + L::kRing0 + warp * (kRing * kSlot)));
+  const int rows_per_unit = GU ? 16 : 16 * FW;
   auto mat = [](int f) { return GU ? f : 0; };
-  auto frow = [&](int f) { return GU ? n0 : n0 + 16 * f; };
 
-  // Copy sources of this lane, fixed for the item: piece u (0, 1) of
-  // fragment f of stage s starts at src[f][u] + s * step(u) (16 bytes; a
-  // null base: nothing to copy), and its scale/zero piece at
-  // sz_src[f] + s * sz_step (lanes below 4, or 8 for groups of 64).  Per
-  // fragment: INT4 16 rows x 64 B of codes in 64 pieces; planes 16 rows x
-  // (32 B Q2 + 16 B D3 + 16 B D4); then 16 rows x 1 or 2 groups of
-  // (scale, zero) words, contiguous.
+  // unit u -> (listed bin, pass, row block)
+  auto locate = [&](int u, int& e, int& pass, int& rb) {
+    int lo = 0, hi = n_ent;  // largest e with ent[e].unit0 <= u
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (ent[mid].unit0 <= u) lo = mid; else hi = mid;
+    }
+    e = lo;
+    const int local = u - ent[lo].unit0;
+    pass = local / P.row_blocks;
+    rb = local - pass * P.row_blocks;
+  };
+
+  // ---- copy side: this warp's stream of stages, unit by unit.  Piece u of
+  // fragment f of the current stage is 16 bytes at src[f][u] (a null base:
+  // nothing to copy), its scale/zero piece at sz_src[f] (lanes below 4, or 8
+  // for groups of 64).  Per fragment: INT4 16 rows x 64 B of codes in 64
+  // pieces; planes 16 rows x (32 B Q2 + 16 B D3 + 16 B D4); then 16 rows x
+  // 1 or 2 groups of (scale, zero) words, contiguous.
   constexpr int kStep0 = PLANES ? 32 : 64;  // piece 0: codes, or Q2
   constexpr int kStep1 = PLANES ? 16 : 64;  // piece 1: codes, or D3 / D4
   const int sz_step = (kStageK / P.group) * 512;
   const uint8_t* src[FW][2];
   uint32_t dst[FW][2];
   const uint8_t* sz_src[FW];
-#pragma unroll
-  for (int f = 0; f < FW; ++f) {
-    const int m = mat(f), r0 = frow(f);
-    if (!PLANES) {
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int q = lane + 32 * u, rr = q >> 2, cc = q & 3;
-        src[f][u] = blob + P.code_off[m] + static_cast<size_t>(r0 + rr) * (P.K / 2) + cc * 16;
-        dst[f][u] = f * kFragBytes + rr * 64 + cc * 16;
-      }
-    } else {
-      const int rq = lane >> 1, hh = lane & 1;  // Q2: 16 rows x 32 B
-      src[f][0] = blob + P.code_off[m] + static_cast<size_t>(r0 + rq) * (P.K / 4) + hh * 16;
-      dst[f][0] = f * kFragBytes + rq * 32 + hh * 16;
-      const int rr = lane & 15;  // lanes 0-15: D3, 16-31: D4 (16 rows x 16 B each)
-      const bool want = lane < 16 ? bits >= 3 : bits >= 4;
-      src[f][1] = want ? blob + (lane < 16 ? P.d3_off[m] : P.d4_off[m]) + static_cast<size_t>(r0 + rr) * (P.K / 8)
-                       : nullptr;
-      dst[f][1] = f * kFragBytes + (lane < 16 ? 512 : 768) + rr * 16;
-    }
-    const int gi = (lane >> 2) & 1, pc = lane & 3;
-    sz_src[f] = blob + P.sz_off[m] + (static_cast<size_t>(r0 >> 7) * G + gi) * 512 + (r0 & 127) * 4 + pc * 16;
-  }
   const bool sz_lane = lane < (G64 ? 8 : 4);
-
   const uint32_t sz_dst = FW * kFragBytes + ((lane >> 2) & 1) * 64 + (lane & 3) * 16;
-  // sources of the next stage this warp issues (stage warp, then + 8 each time)
+  int iq = 0, ii = 0;  // unit (of this CTA) and stage (of this warp) of the next copy
+  // copy bases of this warp's first stage of unit q
+  auto bases = [&](int q) {
+    int e, pass, rb;
+    locate(blockIdx.x + q * gridDim.x, e, pass, rb);
+    const BinEnt be = ent[e];
+    const uint8_t* blob = P.blobs + static_cast<size_t>(be.slot) * P.blob_bytes;
+    const int n0 = rb * rows_per_unit;
 #pragma unroll
-  for (int f = 0; f < FW; ++f) {
-    src[f][0] += warp * kStep0;
-    if (!PLANES || src[f][1]) src[f][1] += warp * kStep1;
-    sz_src[f] += warp * sz_step;
-  }
-
-  // copies of this warp's i-th stage (global stage warp + 8 i) into ring
-  // slot i % kRing; called for i = 0, 1, 2, ... in order
-  auto issue = [&](int i) {
-    if (warp + kWarps * i < n_stages) {
-      const uint32_t dst0 = ring_u + (i % kRing) * kSlot;
+    for (int f = 0; f < FW; ++f) {
+      const int m = mat(f), r0 = GU ? n0 : n0 + 16 * f;
+      if (!PLANES) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int qq = lane + 32 * u, rr = qq >> 2, cc = qq & 3;
+          src[f][u] = blob + P.code_off[m] + static_cast<size_t>(r0 + rr) * (P.K / 2) + cc * 16 + warp * kStep0;
+          dst[f][u] = f * kFragBytes + rr * 64 + cc * 16;
+        }
+      } else {
+        const int rq = lane >> 1, hh = lane & 1;  // Q2: 16 rows x 32 B
+        src[f][0] = blob + P.code_off[m] + static_cast<size_t>(r0 + rq) * (P.K / 4) + hh * 16 + warp * kStep0;
+        dst[f][0] = f * kFragBytes + rq * 32 + hh * 16;
+        const int rr = lane & 15;  // lanes 0-15: D3, 16-31: D4 (16 rows x 16 B each)
+        const bool want = lane < 16 ? be.bits >= 3 : be.bits >= 4;
+        src[f][1] = want ? blob + (lane < 16 ? P.d3_off[m] : P.d4_off[m]) + static_cast<size_t>(r0 + rr) * (P.K / 8) +
+                               warp * kStep1
+                         : nullptr;
+        dst[f][1] = f * kFragBytes + (lane < 16 ? 512 : 768) + rr * 16;
+      }
+      const int gi = (lane >> 2) & 1, pc = lane & 3;
+      sz_src[f] = blob + P.sz_off[m] + (static_cast<size_t>(r0 >> 7) * G + gi) * 512 + (r0 & 127) * 4 + pc * 16 +
+                  warp * sz_step;
+    }
+  };
+  // the next stage of the stream into ring slot j % kRing (j = 0, 1, ... in
+  // order); past the stream's end an empty group keeps the count uniform
+  auto issue = [&](int j) {
+    if (iq < my_units && my_stages > 0) {
+      if (ii == 0) bases(iq);
+      const uint32_t dst0 = ring_u + (j % kRing) * kSlot;
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
         cp_async16(dst0 + dst[f][0], src[f][0]);
         if (!PLANES || src[f][1]) cp_async16(dst0 + dst[f][1], src[f][1]);
         if (sz_lane) cp_async16(dst0 + sz_dst + f * kSzBytes, sz_src[f]);
+        src[f][0] += kWarps * kStep0;
+        if (!PLANES || src[f][1]) src[f][1] += kWarps * kStep1;
+        sz_src[f] += kWarps * sz_step;
+      }
+      if (++ii == my_stages) {
+        ii = 0;
+        ++iq;
       }
     }
-#pragma unroll
-    for (int f = 0; f < FW; ++f) {
-      src[f][0] += kWarps * kStep0;
-      if (!PLANES || src[f][1]) src[f][1] += kWarps * kStep1;
-      sz_src[f] += kWarps * sz_step;
-    }
-    cp_async_commit();  // an empty group past the end keeps the count uniform
+    cp_async_commit();
   };
 
-  const int my_stages = n_stages > warp ? (n_stages - warp + kWarps - 1) / kWarps : 0;
-  bool waited = GU;
-  float acc[FW][NB][4];
-  float* red = reinterpret_cast<float*>(smem);  // reused after the ring drains
-  constexpr int kVals = FW * NB * 4;
+#pragma unroll
+  for (int j = 0; j < kRing; ++j) issue(j);
+  if (!GU) {  // down pass: h is read only from here on
+    pdl_wait();
+    pdl_trigger();
+  }
 
-  for (int t0 = 0; t0 < nrows; t0 += 8 * NB) {  // one pass over K per 8 NB tokens
-#pragma unroll
-    for (int f = 0; f < FW; ++f)
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[f][nb][j] = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kRing; ++i) issue(i);
-    if (!waited) {  // down pass: h is read only from here on
-      pdl_wait();
-      pdl_trigger();
-      waited = true;
-    }
+  int j = 0;  // stream position of the stage being computed
+  for (int q = 0; q < my_units; ++q) {
+    int e, pass, rb;
+    locate(blockIdx.x + q * gridDim.x, e, pass, rb);
+    const BinEnt be = ent[e];
+    const int t0 = pass * 8 * NB, n0 = rb * rows_per_unit;
+    const int ntok = min(8 * NB, be.nrows - t0);  // token rows of this unit
     // this lane's run of each token row it feeds (token g of each 8-token
-    // block), advanced by one stage of this warp (8 x 128 K) per iteration
+    // block), advanced by one stage of this warp (8 x 128 K) per stage
     bool tok_in[NB];
     const __half* xp[NB];
-    int ntok = 0;  // token rows of this pass
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
-      const int tk = t0 + 8 * nb + g;
-      tok_in[nb] = tk < nrows;
-      xp[nb] = P.act + static_cast<size_t>(row0 + (tok_in[nb] ? tk : 0)) * P.K + warp * kStageK + 32 * c;
+      tok_in[nb] = 8 * nb + g < ntok;
+      xp[nb] = P.act + static_cast<size_t>(be.row0 + t0 + (tok_in[nb] ? 8 * nb + g : 0)) * P.K + warp * kStageK + 32 * c;
     }
-    ntok = min(8 * NB, nrows - t0);
-    // the pass's activation runs into L1 ahead of their use when they fit
+    // the unit's activation runs into L1 ahead of their use when they fit
     // (a stage's 128 K of one token row is two 128-byte lines)
     if (ntok * P.K * 2 <= (48 << 10) && (c & 1) == 0) {
 #pragma unroll
@@ -309,7 +342,14 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
           for (int i = 0; i < my_stages; ++i)
             asm volatile("prefetch.global.L1 [%0];" ::"l"(xp[nb] + i * kWarps * kStageK));
     }
-    for (int i = 0; i < my_stages; ++i) {
+    float acc[FW][NB][4];
+#pragma unroll
+    for (int f = 0; f < FW; ++f)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) acc[f][nb][jj] = 0.0f;
+    for (int i = 0; i < my_stages; ++i, ++j) {
       // activations (4 x 8 elements per token block), loaded before the wait
       uint4 xv[NB][4];
 #pragma unroll
@@ -321,7 +361,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
       }
       cp_async_wait<kRing - 1>();
       __syncwarp();
-      const uint32_t sb = ring_u + (i % kRing) * kSlot;  // this stage's ring slot
+      const uint32_t sb = ring_u + (j % kRing) * kSlot;  // this stage's ring slot
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
         const uint32_t fb = sb + f * kFragBytes;
@@ -350,8 +390,8 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
           for (int half = 0; half < 2; ++half) {
             const int r = g + 8 * half;
             const uint2 q2 = lds64(fb + r * 32 + c * 8);
-            const uint32_t d3 = bits >= 3 ? lds32(fb + 512 + r * 16 + c * 4) : 0u;
-            const uint32_t d4 = bits >= 4 ? lds32(fb + 768 + r * 16 + c * 4) : 0u;
+            const uint32_t d3 = be.bits >= 3 ? lds32(fb + 512 + r * 16 + c * 4) : 0u;
+            const uint32_t d4 = be.bits >= 4 ? lds32(fb + 768 + r * 16 + c * 4) : 0u;
             uint32_t* cw = half ? cb : ca;
             const uint32_t qw[2] = {q2.x, q2.y};
 #pragma unroll
@@ -376,9 +416,9 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
           if (G64) {  // groups of 64: the scale goes into A (one fp16 rounding)
             const __half2 sa = __half2half2(__float2half_rn(slo)), sb2 = __half2half2(__float2half_rn(shi));
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              pa[j] = h2u(__hmul2(u2h(pa[j]), sa));
-              pb[j] = h2u(__hmul2(u2h(pb[j]), sb2));
+            for (int jj = 0; jj < 4; ++jj) {
+              pa[jj] = h2u(__hmul2(u2h(pa[jj]), sa));
+              pb[jj] = h2u(__hmul2(u2h(pb[jj]), sb2));
             }
           }
 #pragma unroll
@@ -413,40 +453,31 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
           }
         }
       }
-      __syncwarp();  // every lane is done with ring slot i % kRing
-      issue(i + kRing);
+      __syncwarp();  // every lane is done with ring slot j % kRing
+      issue(j + kRing);
     }
-    cp_async_wait<0>();
-    // back to this warp's first stage for a further pass over K
-#pragma unroll
-    for (int f = 0; f < FW; ++f) {
-      src[f][0] -= (kRing + my_stages) * kWarps * kStep0;
-      if (!PLANES || src[f][1]) src[f][1] -= (kRing + my_stages) * kWarps * kStep1;
-      sz_src[f] -= (kRing + my_stages) * kWarps * sz_step;
-    }
-    __syncthreads();  // every warp's ring is drained: the space becomes the reduction buffer
+    // the unit's partial sums of all warps, added in warp order
 #pragma unroll
     for (int f = 0; f < FW; ++f)
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) red[(warp * kVals + (f * NB + nb) * 4 + j) * 32 + lane] = acc[f][nb][j];
+        for (int jj = 0; jj < 4; ++jj) red[(warp * kVals + (f * NB + nb) * 4 + jj) * 32 + lane] = acc[f][nb][jj];
     __syncthreads();
-    // thread -> (lane', nb, j): sum over warps in order, then the epilogue
     for (int v = threadIdx.x; v < 32 * NB * 4; v += kWarps * 32) {
-      const int ln = v & 31, nb = (v >> 5) / 4, j = (v >> 5) & 3;
+      const int ln = v & 31, nb = (v >> 5) / 4, jj = (v >> 5) & 3;
       const int gg = ln >> 2, cc = ln & 3;
-      const int row = gg + 8 * (j >> 1);           // weight row inside the fragment
-      const int tk = t0 + 8 * nb + 2 * cc + (j & 1);  // token row inside the bin
+      const int row = gg + 8 * (jj >> 1);               // weight row inside the fragment
+      const int tk = t0 + 8 * nb + 2 * cc + (jj & 1);   // token row inside the bin
       float sum[FW];
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
         float a = 0.0f;
-        for (int w = 0; w < kWarps; ++w) a += red[(w * kVals + (f * NB + nb) * 4 + j) * 32 + ln];
+        for (int w = 0; w < kWarps; ++w) a += red[(w * kVals + (f * NB + nb) * 4 + jj) * 32 + ln];
         sum[f] = a;
       }
-      if (tk < nrows) {
-        const size_t p = static_cast<size_t>(row0 + tk);
+      if (tk < be.nrows) {
+        const size_t p = static_cast<size_t>(be.row0 + tk);
         if (GU) {
           P.out[p * P.N + n0 + row] = __float2half_rn(silu_f(sum[0]) * sum[1]);
         } else {
@@ -458,44 +489,61 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
         }
       }
     }
-    __syncthreads();  // the reduction buffer is the next pass's ring
+    __syncthreads();  // the reduction buffer is reused by the next unit
   }
+  cp_async_wait<0>();  // only empty groups remain
 }
 
 template <bool GU, bool PLANES, bool G64, int FW, int NB>
-moe_status_t run_dec(const DecParams& p, int grid, cudaStream_t s, const char* what) {
-  constexpr int smem = kWarps * kRing * FW * (kFragBytes + kSzBytes);
-  static_assert(smem >= kWarps * FW * NB * 4 * 32 * 4, "reduction buffer fits the ring");
+moe_status_t run_dec(const DecParams& p, int units_upper, cudaStream_t s, const char* what) {
+  auto kern = k_dec<GU, PLANES, G64, FW, NB>;
+  const size_t smem = Smem<FW, NB>::bytes(p.max_ent);
+  // the dynamic shared memory depends on max_ent: set the opt-in to the
+  // largest this variant can need (768 bins), once per device; the grid is
+  // the number of CTAs that fit at once (persistent), found per device
   static std::atomic<uint64_t> attr_set{0};
+  static int resident[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_check(e, what);
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  const size_t smem_max = Smem<FW, NB>::bytes(768);
   if (!bit || !(attr_set.load() & bit)) {
-    e = cudaFuncSetAttribute(k_dec<GU, PLANES, G64, FW, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
     if (e != cudaSuccess) return cuda_check(e, what);
+    int per_sm = 0, sms = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarps * 32, Smem<FW, NB>::bytes(256));
+    if (e != cudaSuccess) return cuda_check(e, what);
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_check(e, what);
+    if (dev < 64) resident[dev] = std::max(1, per_sm) * std::max(1, sms);
     attr_set.fetch_or(bit);
   }
-  return cuda_check(launch_pdl(true, k_dec<GU, PLANES, G64, FW, NB>, dim3(grid), dim3(kWarps * 32), smem, s, p),
-                    what);
+  const int fit = dev < 64 && resident[dev] > 0 ? resident[dev] : 148;
+  const int grid = std::max(1, std::min(units_upper, fit));
+  return cuda_check(launch_pdl(true, kern, dim3(grid), dim3(kWarps * 32), smem, s, p), what);
 }
 
 template <bool GU, bool PLANES, bool G64, int FW>
-moe_status_t run_nb(const DecParams& p, int nb, int grid, cudaStream_t s, const char* what) {
-  return nb == 1 ? run_dec<GU, PLANES, G64, FW, 1>(p, grid, s, what) : run_dec<GU, PLANES, G64, FW, 2>(p, grid, s, what);
+moe_status_t run_nb(const DecParams& p, int nb, int units_upper, cudaStream_t s, const char* what) {
+  return nb == 1 ? run_dec<GU, PLANES, G64, FW, 1>(p, units_upper, s, what)
+                 : run_dec<GU, PLANES, G64, FW, 2>(p, units_upper, s, what);
 }
 
+// units_upper: an upper bound of the work units (listed bins x passes x row
+// blocks), which sizes the grid when there are fewer units than CTA slots
 template <bool PLANES, bool G64>
-moe_status_t run_pair(DecParams gu, DecParams dn, int max_bins, int nb, int sms, cudaStream_t s) {
+moe_status_t run_pair(DecParams gu, DecParams dn, int max_bins, int passes, int nb, int sms, cudaStream_t s) {
   gu.row_blocks = gu.N / 16;
-  moe_status_t st = run_nb<true, PLANES, G64, 2>(gu, nb, max_bins * gu.row_blocks, s, "ffn decode gate/up launch");
+  moe_status_t st = run_nb<true, PLANES, G64, 2>(gu, nb, max_bins * passes * gu.row_blocks, s,
+                                                 "ffn decode gate/up launch");
   if (st != MOE_OK) return st;
-  // 32-row items unless that leaves fewer than two CTAs per SM
+  // 32-row units unless that leaves fewer than two units per SM
   const bool wide = static_cast<long>(max_bins) * (dn.N / 32) >= 2L * sms && dn.N % 32 == 0;
   dn.row_blocks = dn.N / (wide ? 32 : 16);
-  const int grid = max_bins * dn.row_blocks;
-  return wide ? run_nb<false, PLANES, G64, 2>(dn, nb, grid, s, "ffn decode down launch")
-              : run_nb<false, PLANES, G64, 1>(dn, nb, grid, s, "ffn decode down launch");
+  const int units = max_bins * passes * dn.row_blocks;
+  return wide ? run_nb<false, PLANES, G64, 2>(dn, nb, units, s, "ffn decode down launch")
+              : run_nb<false, PLANES, G64, 1>(dn, nb, units, s, "ffn decode down launch");
 }
 
 int sm_count_dec() {
@@ -535,6 +583,9 @@ moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t 
     gu.d4_off[m] = a.lay.d4[m];
     gu.sz_off[m] = a.lay.sz[m];
   }
+  const int max_bins = std::min(gu.nbins, a.total_rows);
+  if (max_bins == 0) return MOE_OK;
+  gu.max_ent = max_bins;  // no more bins than rows are non-empty
   DecParams dn = gu;
   dn.act = a.h;
   dn.K = a.F;
@@ -544,13 +595,16 @@ moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t 
   dn.d3_off[0] = a.lay.d3[2];
   dn.d4_off[0] = a.lay.d4[2];
   dn.sz_off[0] = a.lay.sz[2];
-  const int max_bins = std::min(gu.nbins, a.total_rows);
-  if (max_bins == 0) return MOE_OK;
   const int nb = token_blocks <= 1 ? 1 : 2;
+  // passes per bin: a bin never holds more than T rows
+  const int passes = std::max(1, (std::min(a.T, a.total_rows) + 8 * nb - 1) / (8 * nb));
   const int sms = sm_count_dec();
   const bool g64 = a.group == 64;
-  if (planes) return g64 ? run_pair<true, true>(gu, dn, max_bins, nb, sms, s) : run_pair<true, false>(gu, dn, max_bins, nb, sms, s);
-  return g64 ? run_pair<false, true>(gu, dn, max_bins, nb, sms, s) : run_pair<false, false>(gu, dn, max_bins, nb, sms, s);
+  if (planes)
+    return g64 ? run_pair<true, true>(gu, dn, max_bins, passes, nb, sms, s)
+               : run_pair<true, false>(gu, dn, max_bins, passes, nb, sms, s);
+  return g64 ? run_pair<false, true>(gu, dn, max_bins, passes, nb, sms, s)
+             : run_pair<false, false>(gu, dn, max_bins, passes, nb, sms, s);
 }
 
 }  // namespace moeq
