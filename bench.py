@@ -419,6 +419,38 @@ def h2d_peak_gbs(nbytes=256 << 20, reps=5):
     return nbytes * reps / (a.elapsed_time(b) / 1e3) / 1e9
 
 
+def _time_offload(stack, trace, xs, steps, warm, batch, peak):
+    """Time decode steps of an offload stack in its current schedule: wall
+    clock around whole steps, copy and compute busy times from CUDA events
+    that exclude each stream's waits for the other, giving
+        overlap = (copy + compute - wall) / min(copy, compute)
+    (1 = the shorter of the two is hidden entirely, 0 = none of it)."""
+    import torch
+    stack.prefetched = 0
+    for s in range(warm):
+        stack.step(xs[s], trace[s])
+    torch.cuda.synchronize()
+    stack.timing(True)
+    hits = misses = nbytes = 0
+    t0 = time.perf_counter()
+    for s in range(warm, warm + steps):
+        _, st = stack.step(xs[s], trace[s])
+        for h, m, b, _w in st:
+            hits, misses, nbytes = hits + h, misses + m, nbytes + b
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    copy_ms, comp_ms = stack.timing_read()
+    stack.timing(False)
+    wall_ms = wall * 1e3
+    h2d = nbytes / wall / 1e9
+    return {"tokens_per_s": batch * steps / wall, "ms_per_step": wall_ms / steps,
+            "h2d_bytes_per_step": nbytes / steps, "h2d_gbs": h2d, "h2d_frac": h2d / peak,
+            "hit_rate": hits / max(1, hits + misses),
+            "copy_busy_ms_per_step": copy_ms / steps, "compute_busy_ms_per_step": comp_ms / steps,
+            "overlap": (copy_ms + comp_ms - wall_ms) / max(1e-9, min(copy_ms, comp_ms)),
+            "prefetch_copies_per_step": stack.prefetched / (warm + steps)}
+
+
 def run_offload(steps, layers=16, slots=16, batch=8, seed=0, warm=16):
     """The offload workload: stacked OLMoE-shaped layers with experts in pinned
     host memory and a slot cache per layer, decode steps at a fixed batch on a
@@ -426,11 +458,7 @@ def run_offload(steps, layers=16, slots=16, batch=8, seed=0, warm=16):
     stack: a routed-id sync per layer ("sync"), that plus predictive
     prefetching of the next layer's experts ("prefetch"), and lookahead
     (every layer's ids known at the start of the step, one id copy per step,
-    no per-layer sync).  Wall clock around whole steps; busy times of the
-    copies and of the compute from CUDA events that exclude each stream's
-    waits for the other, giving
-        overlap = (copy + compute - wall) / min(copy, compute)
-    (1 = the shorter of the two is hidden entirely, 0 = none of it)."""
+    no per-layer sync).  Timing as in _time_offload."""
     import torch
     from quantized_moe_expert_histogram_b200 import inputs as I
     from quantized_moe_expert_histogram_b200.offload import OffloadStack
@@ -446,29 +474,38 @@ def run_offload(steps, layers=16, slots=16, batch=8, seed=0, warm=16):
            "timing": "host wall clock around whole steps; copy/compute busy time from CUDA events"}
     for mode in ("sync", "prefetch", "lookahead"):
         stack.prefetch, stack.lookahead = mode == "prefetch", mode == "lookahead"
-        stack.prefetched = 0
-        for s in range(warm):
-            stack.step(xs[s], trace[s])
-        torch.cuda.synchronize()
-        stack.timing(True)
-        hits = misses = nbytes = 0
-        t0 = time.perf_counter()
-        for s in range(warm, n):
-            _, st = stack.step(xs[s], trace[s])
-            for h, m, b, _w in st:
-                hits, misses, nbytes = hits + h, misses + m, nbytes + b
-        torch.cuda.synchronize()
-        wall = time.perf_counter() - t0
-        copy_ms, comp_ms = stack.timing_read()
-        stack.timing(False)
-        wall_ms = wall * 1e3
-        h2d = nbytes / wall / 1e9
-        out[mode] = {"tokens_per_s": batch * steps / wall, "ms_per_step": wall_ms / steps,
-                     "h2d_bytes_per_step": nbytes / steps, "h2d_gbs": h2d, "h2d_frac": h2d / peak,
-                     "hit_rate": hits / max(1, hits + misses),
-                     "copy_busy_ms_per_step": copy_ms / steps, "compute_busy_ms_per_step": comp_ms / steps,
-                     "overlap": (copy_ms + comp_ms - wall_ms) / max(1e-9, min(copy_ms, comp_ms)),
-                     "prefetch_copies_per_step": stack.prefetched / n}
+        out[mode] = _time_offload(stack, trace, xs, steps, warm, batch, peak)
+    stack.close()
+    return out
+
+
+def run_offload_nested(steps, layers=8, slots=8, batch=4, seed=0, warm=16):
+    """The nested-plane offload workload: stacked nested 2/3/4-bit layers
+    (d=4096, E=16, top-4, d_ff=1024, g128), each with a bit-width gate that
+    picks every assignment's width, experts in pinned host memory, on the
+    same kind of routing trace.  Each schedule (per-layer sync, lookahead)
+    runs once with plane-mode caches (only the planes up to the widths used
+    are copied, missing planes added on upgrade) and once with whole-blob
+    caches over the same host blobs."""
+    import torch
+    from quantized_moe_expert_histogram_b200 import inputs as I
+    from quantized_moe_expert_histogram_b200.offload import OffloadStack
+    shape = I.SHAPES["nested"]
+    stack = OffloadStack(shape, layers, slots, batch, seed=seed)
+    n = steps + warm
+    trace = I.make_slot_trace(shape.E, shape.k, layers, n, batch, seed=seed + 2).cuda()
+    xs = I.make_slot_x(shape.d, n, batch, seed=seed + 2, device="cuda")
+    peak = h2d_peak_gbs()
+    out = {"workload": f"{layers} nested-plane layers (d=4096, E=16, top-4, d_ff=1024, planes 2+1+1 g128), "
+                       f"widths from a bit-width gate per layer, {slots} GPU slots per layer, batch {batch}, "
+                       f"Zipf routing with 70% successor correlation",
+           "blob_bytes": stack.blob_bytes, "steps": steps, "warmup_steps": warm, "h2d_peak_gbs": peak}
+    for mode in ("sync", "lookahead"):
+        stack.lookahead = mode == "lookahead"
+        for planes in (True, False):
+            stack.set_plane_staging(planes)
+            out[f"{mode}_{'planes' if planes else 'whole'}"] = _time_offload(stack, trace, xs, steps, warm,
+                                                                              batch, peak)
     stack.close()
     return out
 
@@ -629,6 +666,7 @@ def main():
         del layers
         torch.cuda.empty_cache()
         offload = run_offload(args.offload_steps)
+        offload["nested"] = run_offload_nested(max(1, args.offload_steps // 4))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

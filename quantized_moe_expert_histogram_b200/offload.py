@@ -33,6 +33,15 @@ two schedules:
   first copies.  Gates still come from each layer's router logits at the
   given ids (the layer's own input), so the results equal the resident path
   fed the same ids.
+Nested-plane layers (layout "planes"): every layer gets a bit-width gate
+(D2MoE's dual routing) whose widths reach the host with the ids, and the
+caches are plane-mode caches by default (``plane_staging``): an expert
+moves only the planes up to the widest width its assignments use, and a
+resident expert later needed wider receives only the missing planes (D2MoE's
+bit-width-aware I/O).  ``set_plane_staging(False)`` swaps in whole-blob
+caches over the same host blobs, for comparison.  In lookahead mode the
+widths are pre-gated like the ids: each layer's bit gate applied to the
+step's input at the pre-gated ids.
 This module only orchestrates calls of the C ABI; torch supplies device
 memory, pinned host memory and streams.
 """
@@ -47,9 +56,10 @@ from .layer import QuantMoELayer
 
 class OffloadStack:
     def __init__(self, shape, layers: int, slots: int, batch: int, seed: int = 0, device="cuda",
-                 prefetch: bool = False, lookahead: bool = False):
+                 prefetch: bool = False, lookahead: bool = False, plane_staging: bool = True):
         self.shape, self.n_layers, self.slots, self.batch = shape, layers, slots, batch
         self.prefetch, self.lookahead = prefetch, lookahead
+        self.nested = shape.layout == "planes"
         self.predictor = moeq.RoutePredictor(layers, shape.E) if prefetch else None
         self.prefetched = 0
         self.layers, self.host, self.pools, self.caches = [], [], [], []
@@ -59,14 +69,18 @@ class OffloadStack:
             layer = QuantMoELayer.from_weights(shape, r["w_router"], r["bias"], w["w_gate"], w["w_up"],
                                                w["w_down"], max_tokens=batch)
             del w
+            if self.nested:
+                gb = I.make_bit_gate(shape, seed=seed + 101 * l + 2, device=device, bias=True)
+                layer.w_bit, layer.bias_bit = gb["w_bit"], gb["bias_bit"]
             host = layer.blobs.cpu().pin_memory()
             pool = torch.empty(slots, layer.blobs.shape[1], dtype=torch.uint8, device=device)
             layer.blobs = None  # the experts now live in host memory only
             self.layers.append(layer)
             self.host.append(host)
             self.pools.append(pool)
-            self.caches.append(moeq.SlotCache(shape.E, slots, host.shape[1], host, pool))
         self.blob_bytes = self.host[0].shape[1]
+        self.plane_staging = False
+        self.set_plane_staging(plane_staging)
         self.copy = torch.cuda.Stream()
         self.copy2 = torch.cuda.Stream()  # lookahead: odd layers' copies
         self.side = torch.cuda.Stream()   # lookahead: the per-step id copy
@@ -74,7 +88,22 @@ class OffloadStack:
         self.ids_host = [torch.empty(batch, shape.k, dtype=torch.int32).pin_memory() for _ in range(layers)]
         self.ids_all_host = torch.empty(layers, batch, shape.k, dtype=torch.int32).pin_memory()
         self.ids_pregated = torch.empty(layers, batch, shape.k, dtype=torch.int32, device=device)
+        # nested layers: the widths, on the device and on the host
+        self.bits_host = [torch.empty(batch, shape.k, dtype=torch.uint8).pin_memory() for _ in range(layers)]
+        self.bits_all_host = torch.empty(layers, batch, shape.k, dtype=torch.uint8).pin_memory()
+        self.bits_pregated = torch.empty(layers, batch, shape.k, dtype=torch.uint8, device=device)
         self._marks = None  # busy-time events of the compute stream's own segments
+
+    def set_plane_staging(self, enable: bool):
+        """(Re)create every layer's slot cache, empty: plane-mode caches when
+        ``enable`` and the layers are nested-plane layers, whole-blob caches
+        otherwise."""
+        for c in self.caches:
+            c.close()
+        planes = (self.shape.d, self.shape.F, self.shape.group) if enable and self.nested else None
+        self.caches = [moeq.SlotCache(self.shape.E, self.slots, self.blob_bytes, h, p, planes=planes)
+                       for h, p in zip(self.host, self.pools)]
+        self.plane_staging = planes is not None
 
     def timing(self, enable: bool):
         """Record busy time from now on: each cache's copies and FFN waves
@@ -121,12 +150,19 @@ class OffloadStack:
             moeq.moe_route_topk(x, layer.w_router, layer.bias, sh.k,
                                 forced_idx=None if forced_ids is None else forced_ids[l].contiguous(),
                                 topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"])
-            moeq.moe_permute(v["topk_idx"], sh.E, x=x, out=v, status=v["status"])
+            bits = None
+            if self.nested:
+                bits = moeq.moe_bit_gate(x, layer.w_bit, layer.bias_bit, v["topk_idx"], bits=v["bits"],
+                                         status=v["status"])
+            moeq.moe_permute(v["topk_idx"], sh.E, bits=bits, x=x, out=v, status=v["status"])
             self._segment(t0)
-            # the one device -> host crossing per layer: the routed ids
+            # the one device -> host crossing per layer: the routed ids (and widths)
             self.ids_host[l].copy_(v["topk_idx"], non_blocking=True)
+            if bits is not None:
+                self.bits_host[l].copy_(bits, non_blocking=True)
             self.compute.synchronize()
-            n_waves, st = self.caches[l].stage(self.ids_host[l].reshape(-1), self.copy, self.compute)
+            n_waves, st = self.caches[l].stage(self.ids_host[l].reshape(-1), self.copy, self.compute,
+                                               bits_host=self._bits_for(self.bits_host[l]))
             self.caches[l].ffn(v["x_perm"], v["offsets"], self.batch, sh.d, sh.F, sh.group, layer.layout,
                                v["workspace"], v["y_perm"], v["status"], self.copy, self.compute)
             if self.prefetch and self.predictor is not None:
@@ -149,24 +185,39 @@ class OffloadStack:
             x = y
         return x, stats
 
-    def pregate(self, x):
+    def _bits_for(self, bits_host):
+        """Widths for moe_slot_stage: only a plane-mode cache uses them."""
+        return bits_host.reshape(-1) if self.plane_staging else None
+
+    def pregate(self, x, forced_ids=None):
         """Every layer's expert ids for the step from the step's input (each
-        layer's router applied to x): int32 [layers][batch][k] on the device."""
+        layer's router applied to x; or the forced ids) as int32
+        [layers][batch][k] on the device; for nested layers also the widths,
+        each layer's bit gate applied to x at those ids (uint8, same shape;
+        else None)."""
         for l, layer in enumerate(self.layers):
             v = layer.views(self.batch)
-            moeq.moe_route_topk(x, layer.w_router, layer.bias, self.shape.k, topk_idx=self.ids_pregated[l],
-                                topk_w=v["topk_w"], workspace=v["route_ws"])
-        return self.ids_pregated
+            if forced_ids is None:
+                moeq.moe_route_topk(x, layer.w_router, layer.bias, self.shape.k, topk_idx=self.ids_pregated[l],
+                                    topk_w=v["topk_w"], workspace=v["route_ws"])
+            if self.nested:
+                moeq.moe_bit_gate(x, layer.w_bit, layer.bias_bit,
+                                  self.ids_pregated[l] if forced_ids is None else forced_ids[l].contiguous(),
+                                  bits=self.bits_pregated[l], status=v["status"])
+        ids = self.ids_pregated if forced_ids is None else forced_ids
+        return ids, (self.bits_pregated if self.nested else None)
 
     def _step_lookahead(self, x, forced_ids):
         sh, stats = self.shape, []
-        ids = self.pregate(x) if forced_ids is None else forced_ids
-        # the one device -> host crossing per step: all layers' ids
+        ids, bits_all = self.pregate(x, forced_ids)
+        # the one device -> host crossing per step: all layers' ids (and widths)
         ev = torch.cuda.Event()
         ev.record(self.compute)
         self.side.wait_event(ev)
         with torch.cuda.stream(self.side):
             self.ids_all_host.copy_(ids, non_blocking=True)
+            if bits_all is not None:
+                self.bits_all_host.copy_(bits_all, non_blocking=True)
         self.side.synchronize()
         for l, layer in enumerate(self.layers):
             copy = self.copy if l % 2 == 0 else self.copy2
@@ -174,9 +225,11 @@ class OffloadStack:
             t0 = self._mark()
             moeq.moe_route_topk(x, layer.w_router, layer.bias, sh.k, forced_idx=ids[l].contiguous(),
                                 topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"])
-            moeq.moe_permute(v["topk_idx"], sh.E, x=x, out=v, status=v["status"])
+            moeq.moe_permute(v["topk_idx"], sh.E, bits=None if bits_all is None else bits_all[l], x=x, out=v,
+                             status=v["status"])
             self._segment(t0)
-            n_waves, st = self.caches[l].stage(self.ids_all_host[l].reshape(-1), copy, self.compute)
+            n_waves, st = self.caches[l].stage(self.ids_all_host[l].reshape(-1), copy, self.compute,
+                                               bits_host=self._bits_for(self.bits_all_host[l]))
             self.caches[l].ffn(v["x_perm"], v["offsets"], self.batch, sh.d, sh.F, sh.group, layer.layout,
                                v["workspace"], v["y_perm"], v["status"], copy, self.compute)
             y = torch.empty_like(x)

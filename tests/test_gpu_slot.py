@@ -358,3 +358,58 @@ def test_plane_mode_offload_equals_resident_on_mixed_widths():
     assert 0 < moved < whole
     for _, cache, _ in built:
         cache.close()
+
+
+@pytest.mark.parametrize("mode", ["sync", "prefetch", "lookahead"])
+def test_offload_nested_stack_with_bit_gate_equals_resident(mode):
+    """Nested-plane layers, each with a bit-width gate (D2MoE, Dual Routing),
+    through the offload driver: ids from the trace, widths from each layer's
+    bit gate -- on the layer's input, or in lookahead mode on the step's
+    input, pre-gated with the ids.  Every step's output equals the resident
+    layers fed the same ids and widths bit for bit, with plane-mode caches
+    and again with whole-blob caches over the same host blobs; plane-granular
+    staging moves fewer bytes for the same steps."""
+    shape = I.custom_shape(d=256, E=16, k=4, F=256, group=64, layout="planes")
+    n_layers, batch, steps, seed = 3, 8, 5, 21
+    off = OffloadStack(shape, layers=n_layers, slots=8, batch=batch, seed=seed, prefetch=mode == "prefetch",
+                       lookahead=mode == "lookahead")
+    assert off.plane_staging
+    ref = []
+    for l in range(n_layers):
+        w = I.make_expert_weights(shape, seed=seed + 101 * l, device="cuda")
+        r = I.make_router(shape, seed=seed + 101 * l + 1, device="cuda")
+        gb = I.make_bit_gate(shape, seed=seed + 101 * l + 2, device="cuda", bias=True)
+        layer = QuantMoELayer.from_weights(shape, r["w_router"], r["bias"], w["w_gate"], w["w_up"], w["w_down"],
+                                           max_tokens=batch)
+        layer.w_bit, layer.bias_bit = gb["w_bit"], gb["bias_bit"]
+        ref.append(layer)
+    trace = I.make_slot_trace(shape.E, shape.k, n_layers, steps=steps, batch=batch, seed=22).cuda()
+    xs_all = I.make_slot_x(shape.d, steps, batch, seed=22, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moved, widths = {}, set()
+    for planes in (True, False):
+        off.set_plane_staging(planes)
+        nbytes = 0
+        for s in range(steps):
+            x0 = xs_all[s]
+            y_o, stats = off.step(x0, trace[s])
+            nbytes += sum(st[2] for st in stats)
+            xl = x0
+            for l, layer in enumerate(ref):
+                ids = trace[s, l].contiguous()
+                bits = None
+                if mode == "lookahead":
+                    bits = moeq.moe_bit_gate(x0, layer.w_bit, layer.bias_bit, ids, status=status)
+                y = layer.forward(xl, bits=bits, forced_idx=ids, residual=xl).clone()
+                if bits is None:
+                    bits = layer.views(batch)["bits"]
+                widths.update(bits.reshape(-1).tolist())
+                xl = y
+            torch.cuda.synchronize()
+            assert torch.equal(y_o, xl), f"step {s} (plane staging {planes})"
+        moved[planes] = nbytes
+    assert int(status.item()) == 0
+    assert widths <= {2, 3, 4} and len(widths) >= 2
+    if mode != "prefetch":  # prefetches copy whole experts in both modes and are not counted here
+        assert 0 < moved[True] < moved[False]
+    off.close()
