@@ -396,10 +396,15 @@ MOE_API void moe_debug_force_regime(int regime);
  * NULL (the default) disables it. */
 MOE_API void moe_debug_set_trace(void* host_mapped_ints);
 
-/* Test hook: 1 (the default) lets moe_route_topk run decode-sized batches
- * (up to 64 tokens, E <= 64) as one launch of a thread-block cluster; 0
- * forces the two-launch router (same arithmetic).  Process-wide. */
-MOE_API void moe_debug_route_fused(int enable);
+/* Test hook (process-wide), selecting among paths with the same results:
+ * 1 (the default): moe_route_topk takes up to 8 tokens (T*E <= 512,
+ * d % 64 == 0) as fp64 logits in one thread-block-cluster launch and 9 to
+ * 64 tokens (E <= 64) as the fp32-with-bound router in one cluster launch;
+ * moe_bit_gate takes up to 64 assignments (d % 64 == 0) as fp64 scores in
+ * one cluster launch.  2: the fp32-with-bound one-launch router also for up
+ * to 8 tokens, and the fp32-with-bound bit gate for every size.  0: the
+ * two-launch router and the fp32-with-bound bit gate for every size. */
+MOE_API void moe_debug_route_fused(int mode);
 
 /* Test hook of the on-device failure path: while enabled, the tensor-core
  * FFN kernels give every bounded wait a 20 ms limit (instead of 2 s), and in

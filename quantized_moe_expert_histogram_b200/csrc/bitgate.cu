@@ -21,6 +21,11 @@
 // A warp per (token, selected expert): x[t] comes through L1, the expert's
 // three W_bit rows (3 x d fp32) through L2, two 8-element steps of loads in
 // flight per lane.
+//
+// Up to 64 assignments (k_bit_gate_tiny): the 3 T k scores straight in fp64
+// over a thread-block cluster (each CTA one slice of d, partials into CTA
+// 0's shared memory, added in slice order after a cluster barrier), with no
+// bound and no second pass.
 #include <cmath>
 
 #include "common.cuh"
@@ -127,11 +132,62 @@ __global__ void __launch_bounds__(kWarps * 32) k_bit_gate(const __nv_bfloat16* _
   if (lane == 0) bits[a] = static_cast<uint8_t>(2 + best);
 }
 
+constexpr int kTinyAssign = 64;  // assignments of the cluster path (3 x 64 scores)
+
+__global__ void __launch_bounds__(kWarps * 32) k_bit_gate_tiny(const __nv_bfloat16* __restrict__ x,
+                                                              const float* __restrict__ wb,
+                                                              const float* __restrict__ bb,
+                                                              const int32_t* __restrict__ idx, int T, int d,
+                                                              int E, int k, uint8_t* __restrict__ bits,
+                                                              int32_t* status) {
+  __shared__ double part[kClusterSlices * 3 * kTinyAssign];
+  pdl_wait();
+  pdl_trigger();
+  cluster_sync_start();
+  const int rank = blockIdx.x;  // the grid is one cluster
+  const int na = T * k, n = 3 * na, dk = d / kClusterSlices;
+  auto expert = [&](int a) {
+    const int e = idx[a];
+    return e < 0 ? 0 : (e >= E ? E - 1 : e);
+  };
+  cluster_partial_dots(
+      n, rank * dk, dk,
+      [&](int i, const __nv_bfloat16*& xr, const float*& w) {
+        const int a = i / 3;
+        xr = x + static_cast<size_t>(a / k) * d;
+        w = wb + (static_cast<size_t>(expert(a)) * 3 + (i - 3 * a)) * d;
+      },
+      cluster_map_shared(part, 0) + 8u * static_cast<uint32_t>(rank * n));
+  cluster_sync_publish();
+  if (rank != 0) return;
+  for (int a = threadIdx.x; a < na; a += blockDim.x) {
+    const int raw = idx[a];
+    if (raw < 0 || raw >= E) flag_status(status, MOE_DEV_BAD_INDEX);
+    const int e = expert(a);
+    double v[3];
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      double s = part[3 * a + c];
+      for (int r = 1; r < kClusterSlices; ++r) s += part[r * n + 3 * a + c];
+      v[c] = s + (bb ? static_cast<double>(bb[static_cast<size_t>(e) * 3 + c]) : 0.0);
+    }
+    int best = 0;
+    if (v[1] > v[best]) best = 1;
+    if (v[2] > v[best]) best = 2;
+    bits[a] = static_cast<uint8_t>(2 + best);
+  }
+}
+
 }  // namespace
 
 moe_status_t launch_bit_gate(const void* x, const float* w_bit, const float* bias_bit, const int32_t* idx,
                              int T, int d, int E, int k, uint8_t* bits, int32_t* status, cudaStream_t s) {
   if (T == 0) return MOE_OK;
+  if (g_route_fused == 1 && T * k <= kTinyAssign && d % (8 * kClusterSlices) == 0)
+    return cuda_check(launch_cluster_pdl(k_bit_gate_tiny, kClusterSlices, dim3(kWarps * 32), 0, s,
+                                         static_cast<const __nv_bfloat16*>(x), w_bit, bias_bit, idx, T, d, E, k,
+                                         bits, status),
+                      "moe_bit_gate cluster launch");
   const double u = std::ldexp(1.0, -24);
   const double m = ceil_div(d, 256) * 8 + 5;
   const float gamma = static_cast<float>(m * u / (1.0 - m * u));

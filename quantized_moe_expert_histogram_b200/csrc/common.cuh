@@ -100,6 +100,125 @@ __device__ __forceinline__ double dot_bf16_f32_fp64(const __nv_bfloat16* x, cons
 }
 
 
+// ---- fp64 dot products of a thread-block cluster (decode-sized batches) --
+//
+// For a handful of rows the exact-decision dot products (router logits,
+// bit-width scores) are cheapest straight in fp64: every product of a bf16
+// and an fp32 is exact there, and the few thousand FMAs per row spread over
+// a cluster of kClusterSlices CTAs, one slice of d each.  Partial sums go
+// into CTA 0's shared memory (distributed shared memory of the cluster);
+// after a cluster barrier CTA 0 adds them in slice order.
+constexpr int kClusterSlices = 8;
+constexpr int kClusterItems = 512;  // rows pairs of one launch (CTA 0 holds 8 x 512 fp64 partials)
+
+__device__ __forceinline__ uint32_t cluster_map_shared(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_f64(uint32_t addr, double v) {
+  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
+}
+// every CTA of the cluster has started (its shared memory may be written)
+__device__ __forceinline__ void cluster_sync_start() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+// the stores of every CTA before the barrier are visible after it
+__device__ __forceinline__ void cluster_sync_publish() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Slice partials of n dot products by one CTA: item i pairs the bf16 row
+// and the fp32 row that rows(i, xr, wr) names, over elements [k0, k0 + dk)
+// (k0, dk multiples of 8, rows 16-byte aligned).  Warp w takes items w,
+// w + warps, ...; a lane takes the 8-element pieces k0 + 256 c + 8 lane,
+// sums each piece with an fp64 FMA chain from zero and adds the piece sums
+// in piece order; the warp adds the lane sums in a shuffle tree (every lane
+// ends with the same value).  Up to 8 pieces' loads are in flight together.
+// Lane 0 stores item i's partial at shared::cluster address dst + 8 i.
+// The order of operations does not depend on the item, so identical rows
+// give identical partials.
+template <typename RowFn>
+__device__ __forceinline__ void cluster_partial_dots(int n, int k0, int dk, RowFn rows, uint32_t dst) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int nch = (dk + 255) / 256;
+  const int mine = n > warp ? (n - warp + nw - 1) / nw : 0;
+  for (int q0 = 0; q0 < mine; q0 += 8) {
+    const int gi = min(8, mine - q0);
+    const int pieces = gi * nch;
+    double acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+    for (int p0 = 0; p0 < pieces; p0 += 8) {
+      uint4 xb[8];
+      float4 wa[8], wb[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u, qi = p / nch, c = p - qi * nch, off = c * 256 + lane * 8;
+        if (p < pieces && off < dk) {
+          const __nv_bfloat16* xr;
+          const float* wr;
+          rows(warp + nw * (q0 + qi), xr, wr);
+          xb[u] = *reinterpret_cast<const uint4*>(xr + k0 + off);
+          wa[u] = *reinterpret_cast<const float4*>(wr + k0 + off);
+          wb[u] = *reinterpret_cast<const float4*>(wr + k0 + off + 4);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u, qi = p / nch, c = p - qi * nch, off = c * 256 + lane * 8;
+        if (p < pieces && off < dk) {
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb[u]);
+          const float w[8] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w, wb[u].x, wb[u].y, wb[u].z, wb[u].w};
+          double s = 0.0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(b2[j]);
+            s = fma(static_cast<double>(f.x), static_cast<double>(w[2 * j]), s);
+            s = fma(static_cast<double>(f.y), static_cast<double>(w[2 * j + 1]), s);
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j == qi) acc[j] += s;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j < gi) {  // warp-uniform
+        double a = acc[j];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) st_cluster_f64(dst + 8u * static_cast<uint32_t>(warp + nw * (q0 + j)), a);
+      }
+    }
+  }
+}
+
+// A launch of one thread-block cluster of `cluster` CTAs (grid = cluster),
+// as a programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster_pdl(void (*kernel)(KArgs...), int cluster, dim3 block, size_t smem, cudaStream_t s,
+                               Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(cluster);
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Launchers (each returns MOE_OK or an error already recorded).
 moe_status_t launch_pack(const float* w_gate, const float* w_up, const float* w_down, int E, int d,
                          int F, int group, int layout, void* blobs, cudaStream_t s);

@@ -239,18 +239,25 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
     rb = local - pass * P.row_blocks;
   };
 
-  // ---- copy side: this warp's stream of stages, unit by unit.  Piece u of
-  // fragment f of the current stage is 16 bytes at src[f][u] (a null base:
-  // nothing to copy), its scale/zero piece at sz_src[f] (lanes below 4, or 8
-  // for groups of 64).  Per fragment: INT4 16 rows x 64 B of codes in 64
-  // pieces; planes 16 rows x (32 B Q2 + 16 B D3 + 16 B D4); then 16 rows x
-  // 1 or 2 groups of (scale, zero) words, contiguous.
-  constexpr int kStep0 = PLANES ? 32 : 64;  // piece 0: codes, or Q2
-  constexpr int kStep1 = PLANES ? 16 : 64;  // piece 1: codes, or D3 / D4
+  // ---- copy side: this warp's stream of stages, unit by unit.  Per
+  // fragment: INT4 16 rows x 64 B of codes; planes 16 rows x (32 B Q2 + 16 B
+  // D3 + 16 B D4); then 16 rows x 1 or 2 groups of (scale, zero) words,
+  // contiguous.  A lane copies 16 bytes at ring offset lane * 16 (piece 0)
+  // and 512 + lane * 16 (piece 1) of each fragment: the codes of rows
+  // lane / 4 and 8 + lane / 4 (INT4), or Q2 of row lane / 2 and D3 (lanes
+  // below 16) / D4 of row lane % 16 (planes; a null base: plane not needed),
+  // and a scale/zero piece (lanes below 4, or 8 for groups of 64).  Fragment
+  // f's sources are fragment 0's plus f times a fixed stride (the up matrix,
+  // or 16 rows further), so the stream keeps one base per kind of piece.
+  constexpr int kStep0 = PLANES ? 32 : 64;  // piece 0 advance per stage: codes, or Q2
+  constexpr int kStep1 = 16;                // planes' piece 1: D3 / D4
   const int sz_step = (kStageK / P.group) * 512;
-  const uint8_t* src[FW][2];
-  uint32_t dst[FW][2];
-  const uint8_t* sz_src[FW];
+  const size_t fs_c = GU ? P.code_off[1] - P.code_off[0] : static_cast<size_t>(PLANES ? 4 : 8) * P.K;
+  const size_t fs_d = GU ? P.d3_off[1] - P.d3_off[0] : 2 * static_cast<size_t>(P.K);
+  const size_t fs_sz = GU ? P.sz_off[1] - P.sz_off[0] : 64;
+  const uint8_t* cp = nullptr;   // piece 0 of fragment 0 (codes or Q2)
+  const uint8_t* dp = nullptr;   // planes: piece 1 of fragment 0 (D3 / D4), null when not needed
+  const uint8_t* szp = nullptr;  // scale/zero piece of fragment 0
   const bool sz_lane = lane < (G64 ? 8 : 4);
   const uint32_t sz_dst = FW * kFragBytes + ((lane >> 2) & 1) * 64 + (lane & 3) * 16;
   int iq = 0, ii = 0;  // unit (of this CTA) and stage (of this warp) of the next copy
@@ -261,47 +268,35 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
     const BinEnt be = ent[e];
     const uint8_t* blob = P.blobs + static_cast<size_t>(be.slot) * P.blob_bytes;
     const int n0 = rb * rows_per_unit;
-#pragma unroll
-    for (int f = 0; f < FW; ++f) {
-      const int m = mat(f), r0 = GU ? n0 : n0 + 16 * f;
-      if (!PLANES) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int qq = lane + 32 * u, rr = qq >> 2, cc = qq & 3;
-          src[f][u] = blob + P.code_off[m] + static_cast<size_t>(r0 + rr) * (P.K / 2) + cc * 16 + warp * kStep0;
-          dst[f][u] = f * kFragBytes + rr * 64 + cc * 16;
-        }
-      } else {
-        const int rq = lane >> 1, hh = lane & 1;  // Q2: 16 rows x 32 B
-        src[f][0] = blob + P.code_off[m] + static_cast<size_t>(r0 + rq) * (P.K / 4) + hh * 16 + warp * kStep0;
-        dst[f][0] = f * kFragBytes + rq * 32 + hh * 16;
-        const int rr = lane & 15;  // lanes 0-15: D3, 16-31: D4 (16 rows x 16 B each)
-        const bool want = lane < 16 ? be.bits >= 3 : be.bits >= 4;
-        src[f][1] = want ? blob + (lane < 16 ? P.d3_off[m] : P.d4_off[m]) + static_cast<size_t>(r0 + rr) * (P.K / 8) +
-                               warp * kStep1
-                         : nullptr;
-        dst[f][1] = f * kFragBytes + (lane < 16 ? 512 : 768) + rr * 16;
-      }
-      const int gi = (lane >> 2) & 1, pc = lane & 3;
-      sz_src[f] = blob + P.sz_off[m] + (static_cast<size_t>(r0 >> 7) * G + gi) * 512 + (r0 & 127) * 4 + pc * 16 +
-                  warp * sz_step;
+    if (!PLANES) {
+      cp = blob + P.code_off[0] + static_cast<size_t>(n0 + (lane >> 2)) * (P.K / 2) + (lane & 3) * 16 + warp * kStep0;
+    } else {
+      cp = blob + P.code_off[0] + static_cast<size_t>(n0 + (lane >> 1)) * (P.K / 4) + (lane & 1) * 16 + warp * kStep0;
+      const bool want = lane < 16 ? be.bits >= 3 : be.bits >= 4;
+      dp = want ? blob + (lane < 16 ? P.d3_off[0] : P.d4_off[0]) + static_cast<size_t>(n0 + (lane & 15)) * (P.K / 8) +
+                      warp * kStep1
+                : nullptr;
     }
+    szp = blob + P.sz_off[0] + (static_cast<size_t>(n0 >> 7) * G + ((lane >> 2) & 1)) * 512 + (n0 & 127) * 4 +
+          (lane & 3) * 16 + warp * sz_step;
   };
   // the next stage of the stream into ring slot j % kRing (j = 0, 1, ... in
   // order); past the stream's end an empty group keeps the count uniform
   auto issue = [&](int j) {
     if (iq < my_units && my_stages > 0) {
       if (ii == 0) bases(iq);
-      const uint32_t dst0 = ring_u + (j % kRing) * kSlot;
+      const uint32_t slot = ring_u + (j % kRing) * kSlot;
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
-        cp_async16(dst0 + dst[f][0], src[f][0]);
-        if (!PLANES || src[f][1]) cp_async16(dst0 + dst[f][1], src[f][1]);
-        if (sz_lane) cp_async16(dst0 + sz_dst + f * kSzBytes, sz_src[f]);
-        src[f][0] += kWarps * kStep0;
-        if (!PLANES || src[f][1]) src[f][1] += kWarps * kStep1;
-        sz_src[f] += kWarps * sz_step;
+        const uint32_t d0 = slot + f * kFragBytes + lane * 16;
+        cp_async16(d0, cp + f * fs_c);
+        if (!PLANES) cp_async16(d0 + 512, cp + f * fs_c + 4 * static_cast<size_t>(P.K));
+        else if (dp) cp_async16(d0 + 512, dp + f * fs_d);
+        if (sz_lane) cp_async16(slot + sz_dst + f * kSzBytes, szp + f * fs_sz);
       }
+      cp += kWarps * kStep0;
+      if (PLANES && dp) dp += kWarps * kStep1;
+      szp += kWarps * sz_step;
       if (++ii == my_stages) {
         ii = 0;
         ++iq;
@@ -582,6 +577,11 @@ moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t 
     gu.d3_off[m] = a.lay.d3[m];
     gu.d4_off[m] = a.lay.d4[m];
     gu.sz_off[m] = a.lay.sz[m];
+  }
+  if (planes && (a.lay.d3[1] - a.lay.d3[0] != a.lay.q2[1] - a.lay.q2[0] ||
+                 a.lay.d4[1] - a.lay.d4[0] != a.lay.q2[1] - a.lay.q2[0])) {
+    set_error("ffn decode: gate and up plane segments differ in size");
+    return MOE_ERR_INVALID_ARG;
   }
   const int max_bins = std::min(gu.nbins, a.total_rows);
   if (max_bins == 0) return MOE_OK;

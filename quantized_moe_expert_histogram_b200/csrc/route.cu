@@ -26,6 +26,11 @@
 //                   fp64 logits.  Gates are the softmax over the k picked
 //                   logits, in fp64 arithmetic on those values.
 //
+// Up to 8 tokens (k_route_tiny) the T*E dot products are few enough to take
+// straight in fp64, spread over a thread-block cluster: the selection then
+// runs on the fp64 logits with no bound and no second pass.  From 9 to 64
+// tokens both steps above run in one cluster launch (k_route_small).
+//
 // Error bound of the fp32 sum: an FMA chain over m products errs by at most
 // g(m) times the sum of their magnitudes; a chunk (32 products) and then the
 // d/32 chunk sums in any order give g(32) + g(d/32)(1 + g(32)) <= g(32 + d/32).
@@ -545,6 +550,60 @@ __global__ void __launch_bounds__(kSelThreads) k_route_small(
     select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, rank);
 }
 
+// Decode-sized batches (T <= 8, T*E <= kClusterItems, d % 64 == 0): the
+// logits straight in fp64 -- no fp32 stage, no bound, no re-evaluation.
+// One cluster of kClusterSlices CTAs, CTA r takes the slice [r d/8, (r+1)
+// d/8) of every (token, expert) dot product (cluster_partial_dots) and
+// stores the partials into CTA 0's shared memory; after the cluster barrier
+// CTA 0's warp t adds token t's partials in slice order and the bias (in
+// fp64) and selects on those logits (first maximum, ties to the lower index),
+// gates as the fp64 softmax over the picks.
+__global__ void __launch_bounds__(kSelThreads) k_route_tiny(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
+    const int32_t* __restrict__ forced, int T, int d, int E, int k, int32_t* __restrict__ out_idx,
+    float* __restrict__ out_w) {
+  __shared__ double part[kClusterSlices * kClusterItems];
+  pdl_wait();
+  pdl_trigger();
+  cluster_sync_start();
+  const int rank = blockIdx.x;  // the grid is one cluster
+  const int n = T * E, dk = d / kClusterSlices;
+  cluster_partial_dots(
+      n, rank * dk, dk,
+      [&](int i, const __nv_bfloat16*& xr, const float*& w) {
+        const int t = i / E;
+        xr = x + static_cast<size_t>(t) * d;
+        w = wr + static_cast<size_t>(i - t * E) * d;
+      },
+      cluster_map_shared(part, 0) + 8u * static_cast<uint32_t>(rank * n));
+  cluster_sync_publish();
+  if (rank != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = warp; t < T; t += kSelWarps) {
+    double v[kPer];
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) {
+      const int e = lane + 32 * m;
+      v[m] = -INFINITY;
+      if (e < E) {
+        double a = part[t * E + e];
+        for (int r = 1; r < kClusterSlices; ++r) a += part[r * n + t * E + e];
+        v[m] = a + (bias ? static_cast<double>(bias[e]) : 0.0);
+      }
+    }
+    int sel[16];
+    if (forced) {
+      for (int j = 0; j < k; ++j) {
+        const int e = forced[static_cast<size_t>(t) * k + j];
+        sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
+      }
+    } else {
+      warp_topk(v, 0xffu, E, k, lane, sel);
+    }
+    write_gates(v, sel, k, t, lane, out_idx, out_w);
+  }
+}
+
 int route_splits(int T, int d, int E, size_t cap = static_cast<size_t>(-1)) {
   const int ec = E <= 16 ? 16 : 64;
   const int tt = ec == 64 ? Tile<64>::TT : Tile<16>::TT;
@@ -642,6 +701,11 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
   const int splits = route_splits(T, d, E, workspace_bytes);
   const RouteWs ws = route_ws(workspace, splits, T, E);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  // up to 8 tokens: fp64 logits in one cluster launch (no workspace)
+  if (g_route_fused == 1 && T <= kSelWarps && T * E <= kClusterItems && d % (8 * kClusterSlices) == 0)
+    return cuda_check(launch_cluster_pdl(k_route_tiny, kClusterSlices, dim3(kSelThreads), 0, s, xb, w_router, bias,
+                                         forced, T, d, E, k, idx, w),
+                      "moe_route_topk cluster launch");
   // decode-sized batches: one token tile and one expert tile, a cluster of
   // up to 8 CTAs over d, selection in the same launch
   const int fused_splits = std::min(splits, 8);
@@ -708,7 +772,7 @@ moe_status_t route_scratch(void** out) {
 }  // namespace
 }  // namespace moeq
 
-extern "C" void moe_debug_route_fused(int enable) { moeq::g_route_fused = enable ? 1 : 0; }
+extern "C" void moe_debug_route_fused(int mode) { moeq::g_route_fused = (mode >= 0 && mode <= 2) ? mode : 1; }
 
 extern "C" moe_status_t moe_route_topk_noalloc(const void* x, const float* w_router, const float* bias,
                                                 const int32_t* forced_idx, int T, int d, int E, int k,

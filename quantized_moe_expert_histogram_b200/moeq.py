@@ -421,9 +421,11 @@ def moe_debug_force_regime(regime):
     load().moe_debug_force_regime(regime)
 
 
-def moe_debug_route_fused(enable):
-    """Test hook: 0 forces the two-launch router for small batches."""
-    load().moe_debug_route_fused(int(bool(enable)))
+def moe_debug_route_fused(mode):
+    """Test hook: 1 (default) fp64 cluster paths for the smallest batches of
+    the router and the bit gate; 2 the fp32-with-bound one-launch router and
+    fp32 bit gate instead; 0 the two-launch router (see moeq.h)."""
+    load().moe_debug_route_fused(int(mode))
 
 
 def moe_debug_ffn_timeout(enable):

@@ -20,8 +20,9 @@ two schedules:
   With ``prefetch`` (EdgeMoE's expert preloading), once layer l's ids are
   known a host predictor (moe_predictor_*) names layer l+1's likely experts
   and ``moe_slot_prefetch`` copies the confident ones (expected to receive
-  at least one assignment; at most a quarter of a cache) into layer l+1's
-  slots behind layer l's own copies.
+  at least ``prefetch_min_score`` assignments, one by default; at most
+  ``prefetch_max`` copies, a quarter of a cache by default) into layer
+  l+1's slots behind layer l's own copies.
 * lookahead (``lookahead=True``, Read-ME's pre-gating): every layer's
   expert ids for the step are known before the first layer computes -- the
   forced trace, or, without one, each layer's router applied to the step's
@@ -56,9 +57,14 @@ from .layer import QuantMoELayer
 
 class OffloadStack:
     def __init__(self, shape, layers: int, slots: int, batch: int, seed: int = 0, device="cuda",
-                 prefetch: bool = False, lookahead: bool = False, plane_staging: bool = True):
+                 prefetch: bool = False, lookahead: bool = False, plane_staging: bool = True,
+                 prefetch_min_score: float = 1.0, prefetch_max: int | None = None):
         self.shape, self.n_layers, self.slots, self.batch = shape, layers, slots, batch
         self.prefetch, self.lookahead = prefetch, lookahead
+        # prefetch policy: experts whose expected assignment count at the next
+        # layer reaches min_score, at most prefetch_max (default: a quarter of a cache)
+        self.prefetch_min_score = prefetch_min_score
+        self.prefetch_max = slots // 4 if prefetch_max is None else prefetch_max
         self.nested = shape.layout == "planes"
         self.predictor = moeq.RoutePredictor(layers, shape.E) if prefetch else None
         self.prefetched = 0
@@ -173,10 +179,11 @@ class OffloadStack:
                     # confident predictions only: the link is the bottleneck, and a
                     # wrong copy costs a slot and bandwidth; keyed by the experts of
                     # this layer and the one before it (EdgeMoE's profile key)
-                    pred = self.predictor.predict(l + 1, self.ids_host[l], self.slots // 4, min_score=1.0,
+                    pred = self.predictor.predict(l + 1, self.ids_host[l], self.prefetch_max,
+                                                  min_score=self.prefetch_min_score,
                                                   prev2_ids=self.ids_host[l - 1] if l >= 1 else None)
                     if pred.numel():
-                        self.prefetched += self.caches[l + 1].prefetch(pred, self.slots // 4, self.copy)
+                        self.prefetched += self.caches[l + 1].prefetch(pred, self.prefetch_max, self.copy)
             y = torch.empty_like(x)
             t0 = self._mark()
             moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], residual=x, y=y)

@@ -31,9 +31,12 @@ def _oracle_sel(L, shape):
 
 
 @pytest.mark.parametrize("name,T,with_bias", [("nested", 300, False), ("nested", 1, True),
-                                               ("olmoe", 256, True), ("tiny", 64, False),
-                                               ("mixtral", 33, True)])
+                                               ("nested", 16, False), ("olmoe", 8, True),
+                                               ("mixtral", 1, False), ("olmoe", 256, True),
+                                               ("tiny", 64, False), ("mixtral", 33, True)])
 def test_bit_gate_bitexact(name, T, with_bias):
+    """Widths bit for bit against the oracle: up to 64 assignments through the
+    fp64 cluster kernel, beyond through the fp32-with-bound kernel."""
     shape = I.SHAPES[name]
     L = I.make_layer(shape, T, seed=21, weights=False)
     G = I.make_bit_gate(shape, seed=22, bias=with_bias)
@@ -51,15 +54,16 @@ def test_bit_gate_bitexact(name, T, with_bias):
         assert set(np.unique(ref).tolist()) == {2, 3, 4}
 
 
+@pytest.mark.parametrize("T", [200, 8])
 @pytest.mark.parametrize("scale", [0.0, 1e-9, 1e-7, 1e-5])
-def test_bit_gate_near_ties_resolved_exactly(scale):
+def test_bit_gate_near_ties_resolved_exactly(scale, T):
     """Width rows that are copies of each other plus a perturbation of the
     given size: the scores of the pair differ by about scale * |x| (exact ties
     at 0, which go to the narrower width), below what fp32 scores can order,
-    so these assignments take the fp64 re-evaluation and must still match the
+    so these assignments take the fp64 re-evaluation (200 tokens) or the fp64
+    cluster kernel (8 tokens, 32 assignments) and must still match the
     oracle."""
     shape = I.SHAPES["nested"]
-    T = 200
     L = I.make_layer(shape, T, seed=23, weights=False)
     G = I.make_bit_gate(shape, seed=24, bias=True)
     w = G["w_bit"].clone()
@@ -80,7 +84,40 @@ def test_bit_gate_near_ties_resolved_exactly(scale):
         np.testing.assert_array_equal(ref, narrower)
 
 
-def test_bit_gate_flags_bad_ids():
+@pytest.mark.parametrize("mode", [1, 2])
+def test_bit_gate_flags_bad_ids(mode):
+    """Out-of-range ids are flagged and clamped, by the fp64 cluster kernel
+    (mode 1, the default at this size) and the fp32 kernel (mode 2)."""
+    moeq.moe_debug_route_fused(mode)
+    try:
+        _bad_ids_case()
+    finally:
+        moeq.moe_debug_route_fused(1)
+
+
+@pytest.mark.parametrize("name,T", [("nested", 1), ("nested", 16), ("mixtral", 8), ("olmoe", 8)])
+def test_bit_gate_small_paths_agree(name, T):
+    """For up to 64 assignments the fp64 cluster kernel (default) and the
+    fp32-with-bound kernel (test hook mode 2) give the same widths, which are
+    the oracle's."""
+    shape = I.SHAPES[name]
+    L = I.make_layer(shape, T, seed=27, weights=False)
+    G = I.make_bit_gate(shape, seed=28, bias=True)
+    sel = _oracle_sel(L, shape)
+    args = (L["x"].cuda(), G["w_bit"].cuda(), G["bias_bit"].cuda(), torch.from_numpy(sel).cuda())
+    b1 = moeq.moe_bit_gate(*args)
+    moeq.moe_debug_route_fused(2)
+    try:
+        b2 = moeq.moe_bit_gate(*args)
+    finally:
+        moeq.moe_debug_route_fused(1)
+    torch.cuda.synchronize()
+    ref = O.bit_gate(L["x"].float().numpy(), G["w_bit"].numpy(), G["bias_bit"].numpy(), sel)
+    np.testing.assert_array_equal(b1.cpu().numpy(), ref)
+    np.testing.assert_array_equal(b2.cpu().numpy(), ref)
+
+
+def _bad_ids_case():
     shape = I.SHAPES["tiny"]
     L = I.make_layer(shape, 4, seed=1, weights=False)
     G = I.make_bit_gate(shape, seed=2)

@@ -68,35 +68,41 @@ def test_route_bitexact(name, T, dup):
 @pytest.mark.parametrize("name,T", [("olmoe", 1), ("olmoe", 8), ("olmoe", 33), ("olmoe", 64), ("nested", 1),
                                     ("nested", 17), ("mixtral", 1), ("tiny", 64)])
 def test_route_fused_small_batches(name, T):
-    """Decode-sized batches run the router as one cluster launch; its expert
-    ids equal the two-launch router's and the oracle's bit for bit, its gates
-    match the oracle's."""
+    """Decode-sized batches run the router as one cluster launch (fp64 logits
+    up to 8 tokens, fp32 with the bound beyond); its expert ids equal the
+    two-launch router's, the fp32 one-launch router's and the oracle's bit
+    for bit, and all their gates match the oracle's."""
     shape = I.SHAPES[name]
     L = I.make_layer(shape, T, seed=17, weights=False)
     bias = L["bias"].cuda() if L["bias"] is not None else None
     x, wr = L["x"].cuda(), L["w_router"].cuda()
     idx_f, w_f = moeq.moe_route_topk(x, wr, bias, shape.k)
-    moeq.moe_debug_route_fused(0)
-    try:
-        idx_2, _ = moeq.moe_route_topk(x, wr, bias, shape.k)
-    finally:
-        moeq.moe_debug_route_fused(1)
+    others = []
+    for mode in (0, 2):  # the two-launch router; the fp32 one-launch router at any size
+        moeq.moe_debug_route_fused(mode)
+        try:
+            others.append(moeq.moe_route_topk(x, wr, bias, shape.k))
+        finally:
+            moeq.moe_debug_route_fused(1)
     torch.cuda.synchronize()
     sel, gates, _ = O.route(L["x"].float().numpy(), L["w_router"].numpy(),
                             None if L["bias"] is None else L["bias"].numpy(), shape.k)
     np.testing.assert_array_equal(idx_f.cpu().numpy(), sel)
-    np.testing.assert_array_equal(idx_2.cpu().numpy(), sel)
     np.testing.assert_allclose(w_f.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
+    for idx_o, w_o in others:
+        np.testing.assert_array_equal(idx_o.cpu().numpy(), sel)
+        np.testing.assert_allclose(w_o.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
 
 
+@pytest.mark.parametrize("T", [300, 8])
 @pytest.mark.parametrize("scale", [0.0, 1e-9, 1e-7, 1e-5])
-def test_route_near_ties_resolved_exactly(scale):
+def test_route_near_ties_resolved_exactly(scale, T):
     """Router rows that are copies of others plus a perturbation of the given
     size: the logits of the pairs differ by about scale * |x| (exact ties at
     0), below what fp32 logits can order, so these tokens must take the fp64
-    re-evaluation and still match the oracle's choice and order exactly."""
+    re-evaluation (300 tokens) or be decided on fp64 logits (8 tokens) and
+    still match the oracle's choice and order exactly."""
     shape = I.SHAPES["olmoe"]
-    T = 300
     L = I.make_layer(shape, T, seed=9, weights=False)
     w = L["w_router"].clone()
     b = L["bias"].clone()
@@ -111,7 +117,7 @@ def test_route_near_ties_resolved_exactly(scale):
     np.testing.assert_allclose(gw.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
     # the pairs really are near-tied inside many tokens' picks
     both = sum(int((s == 0).any() and (s == 1).any()) for s in sel)
-    assert both > 10
+    assert both > 10 or T < 100
 
 
 def test_route_k_equals_E_and_forced():
@@ -125,6 +131,11 @@ def test_route_k_equals_E_and_forced():
     idx3, w3 = moeq.moe_route_topk(L["x"].cuda(), L["w_router"].cuda(), None, 3, forced_idx=forced.cuda())
     np.testing.assert_array_equal(idx3.cpu().numpy(), forced.numpy())
     np.testing.assert_allclose(w3.cpu().numpy(), O.gates_for(logits, forced.numpy()), rtol=GATE_RTOL, atol=GATE_ATOL)
+    # a decode-sized batch (fp64 cluster path): forced ids and their gates
+    idx4, w4 = moeq.moe_route_topk(L["x"][:4].cuda(), L["w_router"].cuda(), None, 3, forced_idx=forced[:4].cuda())
+    np.testing.assert_array_equal(idx4.cpu().numpy(), forced[:4].numpy())
+    np.testing.assert_allclose(w4.cpu().numpy(), O.gates_for(logits[:4], forced[:4].numpy()), rtol=GATE_RTOL,
+                               atol=GATE_ATOL)
 
 
 # ------------------------------------------------------------- permute ----
