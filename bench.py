@@ -229,10 +229,14 @@ def make_instances(shape, T, R, seed, device, bit_gate=False):
 
 def kernel_launches(shape, T, bit_gate=False):
     """Kernels of this library launched by one layer step, following the
-    library's own choices: router 1 (one cluster launch for decode-sized
-    batches) or 2, bit gate 1 when used, permutation 1 (single CTA, with the
-    gather when it is small) or 1 + gather, or 3 + gather, FFN 2, combine 1."""
+    library's own choices: router, bit gate and permutation as one cluster
+    launch for decode-sized batches (T <= 8, T*k <= 64, T*E <= 512,
+    d % 64 == 0); otherwise router 1 (one cluster launch up to 64 tokens) or
+    2, bit gate 1 when used, permutation 1 (single CTA, with the gather when
+    it is small) or 1 + gather, or 3 + gather; then FFN 2, combine 1."""
     n = T * shape.k
+    if T <= 8 and n <= 64 and T * shape.E <= 512 and shape.d % 64 == 0:
+        return 1 + 2 + 1
     nbins = shape.E * (3 if shape.layout == "planes" else 1)
     d32 = shape.d // 32
     splits = 1
@@ -294,12 +298,10 @@ def _step_calls(layer, x, bits, stream, part):
     T = x.shape[0]
     v = layer.views(T)
     if part == "all":
-        moeq.moe_route_topk(x, layer.w_router, layer.bias, layer.k, topk_idx=v["topk_idx"],
-                            topk_w=v["topk_w"], workspace=v["route_ws"], stream=stream)
-        if bits is None and layer.w_bit is not None:
-            bits = moeq.moe_bit_gate(x, layer.w_bit, layer.bias_bit, v["topk_idx"], bits=v["bits"],
-                                     status=v["status"], stream=stream)
-        moeq.moe_permute(v["topk_idx"], layer.E, bits=bits, x=x, out=v, status=v["status"], stream=stream)
+        gate = bits is None and layer.w_bit is not None
+        moeq.moe_route_permute(x, layer.w_router, layer.bias, layer.k, bits=bits,
+                               w_bit=layer.w_bit if gate else None, bias_bit=layer.bias_bit if gate else None,
+                               out=v, status=v["status"], workspace=v["rp_ws"], stream=stream)
     moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, T, layer.E, layer.d, layer.F,
                             layer.group, layer.layout, workspace=v["workspace"], y_perm=v["y_perm"],
                             status=v["status"], stream=stream)

@@ -91,9 +91,11 @@ MOE_API const char* moe_last_error(void);
  * For hidden size d, expert width F (d_ff) and group size g:
  *   INT4  : gate codes [F][d/8] u32 | up codes [F][d/8] | down codes
  *           [d][F/8] | gate sz | up sz | down sz
- *   PLANES: gate Q2 [F][d/16] | gate D3 [F][d/32] | gate D4 [F][d/32] |
- *           up Q2 | up D3 | up D4 | down Q2 [d][F/16] | down D3 | down D4 |
- *           gate sz | up sz | down sz
+ *   PLANES: gate Q2 [F][d/16] | up Q2 | down Q2 [d][F/16] | gate sz |
+ *           up sz | down sz | gate D3 [F][d/32] | up D3 | down D3 [d][F/32]
+ *           | gate D4 | up D4 | down D4 -- width by width, so that what a
+ *           b-bit read needs (Q2 and the scales; D3 from b = 3; D4 at 4)
+ *           is the blob's first bytes
  * Code word packing: nibble i of an INT4 codes word = element 8w+i (low
  * nibble first).  Planes use the plane order, n(i) = (i >> 1) + 4 (i & 1)
  * for element i of a run of 8 (even elements in nibbles 0..3, odd ones in
@@ -197,6 +199,33 @@ MOE_API moe_status_t moe_permute(const int32_t* topk_idx, const uint8_t* bits, c
  * the (expert, width) bins. */
 MOE_API size_t moe_permute_workspace_bytes(int T, int E, int k, int nested);
 
+/* moe_route_permute -- the front of the layer in one call: moe_route_topk,
+ * then (with a bit gate) moe_bit_gate, then moe_permute, with their results
+ * bit for bit ([ExactMoE] the router decides, every routed expert runs;
+ * [D2MoE] Dual Routing: expert gate and bit gate side by side; [Read-ME]
+ * expert-aware batching).  A decode-sized batch -- T <= 8, T*k <= 64,
+ * T*E <= 512, d % 64 == 0 -- runs as one launch of a thread-block cluster
+ * (fp64 dot products for the logits and the width scores, then the
+ * permutation and the gather in one CTA); other sizes issue the separate
+ * launches on `stream`.
+ *   forced_idx int32 [T][k] or NULL, as in moe_route_topk.
+ *   bits_in    uint8 [T][k] widths given by the caller (nested bins), or NULL.
+ *   w_bit, bias_bit  the bit gate as in moe_bit_gate, or NULL; with w_bit,
+ *              bits_in must be NULL and bits_out (uint8 [T][k]) receives
+ *              the widths, which key the nested bins.
+ *   topk_idx, topk_w, counts, offsets, perm, inv_perm, x_perm: as in
+ *              moe_route_topk and moe_permute (x_perm may be NULL: no gather).
+ *   workspace >= moe_route_permute_workspace_bytes(T, d, E, k, nested)
+ *              bytes, 16-byte aligned (nested != 0 with bits_in or w_bit).
+ * Errors and device flags as in the three calls it stands for. */
+MOE_API moe_status_t moe_route_permute(const void* x, const float* w_router, const float* bias,
+                                       const int32_t* forced_idx, const uint8_t* bits_in, const float* w_bit,
+                                       const float* bias_bit, int T, int d, int E, int k, int32_t* topk_idx,
+                                       float* topk_w, uint8_t* bits_out, int32_t* counts, int32_t* offsets,
+                                       int32_t* perm, int32_t* inv_perm, void* x_perm, int32_t* status,
+                                       void* workspace, size_t workspace_bytes, moe_stream_t stream);
+MOE_API size_t moe_route_permute_workspace_bytes(int T, int d, int E, int k, int nested);
+
 /* Workspace bytes moe_grouped_ffn_wq needs for `total_rows` = T*k rows. */
 MOE_API size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int layout);
 
@@ -215,8 +244,10 @@ MOE_API size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int 
  *            e is blob slot_of[e]; experts with slot_of[e] < 0 are skipped
  *            (their y_perm rows are left untouched).
  *   T        token count (no bin holds more than T rows; selects the
- *            kernel: one-token GEMV for T = 1, the small-batch mma.sync
- *            kernel for T <= 8, the tensor-core grouped GEMM above)
+ *            kernel: up to 16 tokens the decode kernel, which streams the
+ *            weights once per 8 or 16 rows of a bin with mma.sync dot
+ *            products split over warps along K; above, the tensor-core
+ *            grouped GEMM with 128-row tiles)
  *   workspace >= moe_ffn_workspace_bytes() bytes of device scratch
  *   y_perm   fp16 [total_rows][d]
  * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16 and
@@ -287,11 +318,12 @@ MOE_API moe_status_t moe_slot_cache_create(int E, int slots, size_t blob_bytes, 
  * mode ([D2MoE] MWQ: W(2) needs only Q2, W(3) adds D3, W(4) adds D4): a
  * slot holds an expert's planes up to some width, a step copies an expert
  * only up to the widest width its assignments use (the Q2 planes and the
- * scales for width 2, plus D3 for 3, plus D4 for 4), a resident expert that
- * is later needed wider receives only its missing planes, and inside a wave
- * the copies go plane by plane -- every Q2 + scales first, then every D3,
- * then every D4 ([D2MoE] Hottest-Expert-Bit-First: hottest experts first,
- * in bit order). */
+ * scales for width 2, plus D3 for 3, plus D4 for 4), and a resident expert
+ * that is later needed wider receives only its missing planes.  The blob
+ * is laid out width by width, so each of these is one contiguous copy
+ * (the blob's first bytes, or the range between two widths); experts are
+ * staged hottest first and each expert's base planes come first ([D2MoE]
+ * Hottest-Expert-Bit-First). */
 MOE_API moe_status_t moe_slot_cache_create_planes(int E, int slots, int d, int F, int group,
                                                   const void* host_blobs, void* device_pool,
                                                   moe_slot_cache** out);

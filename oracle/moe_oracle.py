@@ -195,9 +195,12 @@ def blob_layout(d: int, F: int, group: int, layout: str) -> dict:
 
     INT4: [gate codes F x d/8 u32 | up codes F x d/8 | down codes d x F/8 |
            gate sz | up sz | down sz]
-    planes: [gate Q2 F x d/16 u32 | gate D3 F x d/32 | gate D4 | up Q2 | up D3
-             | up D4 | down Q2 d x F/16 | down D3 | down D4 | gate sz | up sz
-             | down sz]  (bit order inside the words: split_planes)
+    planes: [gate Q2 F x d/16 u32 | up Q2 | down Q2 d x F/16 | gate sz | up sz
+             | down sz | gate D3 F x d/32 | up D3 | down D3 | gate D4 | up D4
+             | down D4]  (bit order inside the words: split_planes).  Width by
+             width: the planes a b-bit read needs (Q2 and the scales for b = 2,
+             plus D3 for 3, plus D4 for 4) are the blob's first bytes, up to
+             the start of D3 (b = 2), of D4 (b = 3) or the end (b = 4).
     sz of an N x K matrix: (scale, zero) bf16 pairs ordered
       [N/128][K/group][128], i.e. pair index ((n//128)*(K/group) + c)*128 + n%128.
     """
@@ -212,13 +215,14 @@ def blob_layout(d: int, F: int, group: int, layout: str) -> dict:
         for m, N, K in mats:
             off[m + ".q2"] = pos
             pos += N * K // 4
-            off[m + ".d3"] = pos
-            pos += N * K // 8
-            off[m + ".d4"] = pos
-            pos += N * K // 8
     for m, N, K in mats:
         off[m + ".sz"] = pos
         pos += N * (K // group) * 4
+    if layout != "int4":
+        for plane in ("d3", "d4"):
+            for m, N, K in mats:
+                off[m + "." + plane] = pos
+                pos += N * K // 8
     off["bytes"] = pos
     return off
 

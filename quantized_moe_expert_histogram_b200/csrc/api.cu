@@ -63,6 +63,9 @@ BlobLayout blob_layout(int d, int F, int group, int layout) {
   if (layout != MOE_LAYOUT_INT4 && layout != MOE_LAYOUT_PLANES) return L;
   const size_t N[3] = {(size_t)F, (size_t)F, (size_t)d};
   const size_t K[3] = {(size_t)d, (size_t)d, (size_t)F};
+  // INT4: codes of gate, up, down, then their scales.  PLANES, width by
+  // width: Q2 of the three matrices, their scales, then D3 of the three,
+  // then D4 -- the planes of a b-bit read are the blob's first bytes.
   size_t pos = 0;
   for (int m = 0; m < 3; ++m) {
     if (layout == MOE_LAYOUT_INT4) {
@@ -71,15 +74,21 @@ BlobLayout blob_layout(int d, int F, int group, int layout) {
     } else {
       L.q2[m] = pos;
       pos += N[m] * K[m] / 4;
-      L.d3[m] = pos;
-      pos += N[m] * K[m] / 8;
-      L.d4[m] = pos;
-      pos += N[m] * K[m] / 8;
     }
   }
   for (int m = 0; m < 3; ++m) {
     L.sz[m] = pos;
     pos += N[m] * (K[m] / group) * 4;
+  }
+  if (layout == MOE_LAYOUT_PLANES) {
+    for (int m = 0; m < 3; ++m) {
+      L.d3[m] = pos;
+      pos += N[m] * K[m] / 8;
+    }
+    for (int m = 0; m < 3; ++m) {
+      L.d4[m] = pos;
+      pos += N[m] * K[m] / 8;
+    }
   }
   L.bytes = pos;
   L.valid = 1;
@@ -200,6 +209,70 @@ moe_status_t moe_permute(const int32_t* topk_idx, const uint8_t* bits, const voi
   }
   return launch_permute(topk_idx, bits, x, T, d, E, k, counts, offsets, perm, inv_perm, x_perm,
                         status, workspace, S(stream));
+}
+
+size_t moe_route_permute_workspace_bytes(int T, int d, int E, int k, int nested) {
+  if (T <= 0 || d <= 0 || E <= 0 || k <= 0) return 256;
+  const size_t r = (route_workspace_bytes(T, d, E) + 255) / 256 * 256;
+  return r + permute_workspace_bytes(T, k, nested ? 3 * E : E);
+}
+
+moe_status_t moe_route_permute(const void* x, const float* w_router, const float* bias, const int32_t* forced_idx,
+                               const uint8_t* bits_in, const float* w_bit, const float* bias_bit, int T, int d,
+                               int E, int k, int32_t* topk_idx, float* topk_w, uint8_t* bits_out,
+                               int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* x_perm,
+                               int32_t* status, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  moe_status_t st = route_check_args(x, w_router, T, d, E, k, topk_idx, topk_w, "moe_route_permute");
+  if (st != MOE_OK) return st;
+  if (bits_in && w_bit) {
+    set_error("moe_route_permute: give the widths (bits_in) or the bit gate (w_bit), not both");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (w_bit && !bits_out) {
+    set_error("moe_route_permute: the bit gate needs bits_out");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (!counts || !offsets || (T > 0 && (!perm || !inv_perm))) {
+    set_error("moe_route_permute: null pointer");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (w_bit && (d % 8 || !aligned16(w_bit))) {
+    set_error("moe_route_permute: the bit gate needs d %% 8 == 0 and a 16-byte aligned w_bit");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (x_perm && (d % 8 || !aligned16(x_perm))) {
+    set_error("moe_route_permute: gather needs d %% 8 == 0 and a 16-byte aligned x_perm");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (static_cast<long>(T) * k > (1L << 24)) {
+    set_error("moe_route_permute: T*k exceeds 2^24");
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  const bool nested = bits_in || w_bit;
+  const size_t need = moe_route_permute_workspace_bytes(T, d, E, k, nested ? 1 : 0);
+  if (T > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) {
+    set_error("moe_route_permute: workspace %zu < %zu bytes or not 16-byte aligned", workspace_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  if (T == 0) {  // empty batch: the separate calls write the (zero) counts and offsets
+    const uint8_t* nested_flag = bits_in ? bits_in : (w_bit ? bits_out : nullptr);  // selects 3E bins
+    return launch_permute(topk_idx, nested_flag, nullptr, 0, d, E, k, counts, offsets, perm, inv_perm, nullptr,
+                          status, workspace, S(stream));
+  }
+  if (route_permute_fusable(T, d, E, k))
+    return launch_route_permute_tiny(x, w_router, bias, forced_idx, bits_in, w_bit, bias_bit, T, d, E, k, topk_idx,
+                                     topk_w, bits_out, counts, offsets, perm, inv_perm, x_perm, status, S(stream));
+  const size_t rbytes = (route_workspace_bytes(T, d, E) + 255) / 256 * 256;
+  st = launch_route(x, w_router, bias, forced_idx, T, d, E, k, topk_idx, topk_w, workspace, rbytes, S(stream));
+  if (st != MOE_OK) return st;
+  const uint8_t* bits = bits_in;
+  if (w_bit) {
+    st = launch_bit_gate(x, w_bit, bias_bit, topk_idx, T, d, E, k, bits_out, status, S(stream));
+    if (st != MOE_OK) return st;
+    bits = bits_out;
+  }
+  return launch_permute(topk_idx, bits, x_perm ? x : nullptr, T, d, E, k, counts, offsets, perm, inv_perm, x_perm,
+                        status, static_cast<uint8_t*>(workspace) + rbytes, S(stream));
 }
 
 size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int layout) {

@@ -226,7 +226,14 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
                           const int32_t* forced, int T, int d, int E, int k, int32_t* idx,
                           float* w, void* workspace, size_t workspace_bytes, cudaStream_t s);
 size_t route_workspace_bytes(int T, int d, int E);
-extern int g_route_fused;  // test hook: 0 = always the two-launch router
+extern int g_route_fused;  // test hook: 1 default, 2 fp32-bound paths, 0 also the two-launch router
+bool route_permute_fusable(int T, int d, int E, int k);
+moe_status_t launch_route_permute_tiny(const void* x, const float* w_router, const float* bias,
+                                       const int32_t* forced, const uint8_t* bits_in, const float* w_bit,
+                                       const float* bias_bit, int T, int d, int E, int k, int32_t* idx,
+                                       float* w, uint8_t* bits_out, int32_t* counts, int32_t* offsets,
+                                       int32_t* perm, int32_t* inv_perm, void* x_perm, int32_t* status,
+                                       cudaStream_t s);
 size_t route_min_workspace_bytes(int T, int d, int E);
 moe_status_t route_check_args(const void* x, const float* w_router, int T, int d, int E, int k,
                               const int32_t* topk_idx, const float* topk_w, const char* fn);

@@ -578,9 +578,8 @@ moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t 
     gu.d4_off[m] = a.lay.d4[m];
     gu.sz_off[m] = a.lay.sz[m];
   }
-  if (planes && (a.lay.d3[1] - a.lay.d3[0] != a.lay.q2[1] - a.lay.q2[0] ||
-                 a.lay.d4[1] - a.lay.d4[0] != a.lay.q2[1] - a.lay.q2[0])) {
-    set_error("ffn decode: gate and up plane segments differ in size");
+  if (planes && a.lay.d4[1] - a.lay.d4[0] != a.lay.d3[1] - a.lay.d3[0]) {  // one stride for D3 and D4 pieces
+    set_error("ffn decode: gate-to-up offsets of D3 and D4 differ");
     return MOE_ERR_INVALID_ARG;
   }
   const int max_bins = std::min(gu.nbins, a.total_rows);

@@ -604,6 +604,193 @@ __global__ void __launch_bounds__(kSelThreads) k_route_tiny(
   }
 }
 
+// ---- router + bit-width gate + permutation in one launch -------------
+//
+// A decode-sized batch (T <= 8, T*k <= kFusedAssign, T*E <= kClusterItems,
+// d % 64 == 0) through the whole front of the layer in one cluster launch,
+// with the results of k_route_tiny, k_bit_gate_tiny and the permutation
+// kernels (same arithmetic, same order):
+//   1. every CTA: its d-slice of the T*E router dot products (fp64) -> CTA 0
+//   2. CTA 0: logits, selection (or the forced ids), gates; ids to shared
+//   3. with a bit gate: the ids are published to the cluster, every CTA
+//      takes its d-slice of the 3*T*k width scores (fp64) -> CTA 0, which
+//      picks the widths
+//   4. CTA 0: keys (expert, or 3 expert + width - 2), stable ranks by
+//      counting (ties in ascending assignment), counts, offsets, perm,
+//      inv_perm, and the gather of x_perm (fp16) in expert order.
+constexpr int kFusedAssign = 64;
+
+struct RoutePermArgs {
+  const __nv_bfloat16* x;
+  const float* wr;
+  const float* bias;
+  const int32_t* forced;
+  const uint8_t* bits_in;  // widths given by the caller, or null
+  const float* wbit;       // bit gate, or null
+  const float* bbit;
+  int T, d, E, k;
+  int32_t* idx;
+  float* gw;
+  uint8_t* bits_out;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv_perm;
+  __half* x_perm;  // null: no gather
+  int32_t* status;
+};
+
+__global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_constant__ RoutePermArgs A) {
+  __shared__ double part[kClusterSlices * kClusterItems];
+  __shared__ int32_t sel_s[kFusedAssign];
+  __shared__ int32_t key_s[kFusedAssign];
+  __shared__ int32_t perm_s[kFusedAssign];
+  __shared__ uint8_t bits_s[kFusedAssign];
+  pdl_wait();
+  pdl_trigger();
+  cluster_sync_start();
+  const int rank = blockIdx.x;  // the grid is one cluster
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = A.T, d = A.d, E = A.E, k = A.k, n = T * E, na = T * k, dk = d / kClusterSlices;
+  const uint32_t part0 = cluster_map_shared(part, 0);
+  // 1. router partials
+  cluster_partial_dots(
+      n, rank * dk, dk,
+      [&](int i, const __nv_bfloat16*& xr, const float*& w) {
+        const int t = i / E;
+        xr = A.x + static_cast<size_t>(t) * d;
+        w = A.wr + static_cast<size_t>(i - t * E) * d;
+      },
+      part0 + 8u * static_cast<uint32_t>(rank * n));
+  cluster_sync_publish();
+  // 2. selection (CTA 0)
+  if (rank == 0) {
+    for (int t = warp; t < T; t += kSelWarps) {
+      double v[kPer];
+#pragma unroll
+      for (int m = 0; m < kPer; ++m) {
+        const int e = lane + 32 * m;
+        v[m] = -INFINITY;
+        if (e < E) {
+          double a = part[t * E + e];
+          for (int r = 1; r < kClusterSlices; ++r) a += part[r * n + t * E + e];
+          v[m] = a + (A.bias ? static_cast<double>(A.bias[e]) : 0.0);
+        }
+      }
+      int sel[16];
+      if (A.forced) {
+        for (int j = 0; j < k; ++j) {
+          const int e = A.forced[static_cast<size_t>(t) * k + j];
+          sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
+        }
+      } else {
+        warp_topk(v, 0xffu, E, k, lane, sel);
+      }
+      write_gates(v, sel, k, t, lane, A.idx, A.gw);
+      for (int j = 0; j < k; ++j)
+        if (j == lane) sel_s[t * k + j] = sel[j];
+    }
+  }
+  // 3. bit-width gate
+  if (A.wbit) {  // uniform over the cluster
+    cluster_sync_publish();  // CTA 0's ids (sel_s) and its last reads of part are done
+    __shared__ int32_t ids_l[kFusedAssign];
+    const uint32_t sel0 = cluster_map_shared(sel_s, 0);
+    for (int a = threadIdx.x; a < na; a += blockDim.x) {
+      int e;
+      asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(e) : "r"(sel0 + 4u * a) : "memory");
+      ids_l[a] = e;
+    }
+    __syncthreads();
+    cluster_partial_dots(
+        3 * na, rank * dk, dk,
+        [&](int i, const __nv_bfloat16*& xr, const float*& w) {
+          const int a = i / 3;
+          xr = A.x + static_cast<size_t>(a / k) * d;
+          w = A.wbit + (static_cast<size_t>(ids_l[a]) * 3 + (i - 3 * a)) * d;
+        },
+        part0 + 8u * static_cast<uint32_t>(rank * 3 * na));
+    cluster_sync_publish();
+    if (rank == 0) {
+      for (int a = threadIdx.x; a < na; a += blockDim.x) {
+        const int e = sel_s[a];
+        double v[3];
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+          double s = part[3 * a + c];
+          for (int r = 1; r < kClusterSlices; ++r) s += part[r * 3 * na + 3 * a + c];
+          v[c] = s + (A.bbit ? static_cast<double>(A.bbit[static_cast<size_t>(e) * 3 + c]) : 0.0);
+        }
+        int best = 0;
+        if (v[1] > v[best]) best = 1;
+        if (v[2] > v[best]) best = 2;
+        bits_s[a] = static_cast<uint8_t>(2 + best);
+        A.bits_out[a] = static_cast<uint8_t>(2 + best);
+      }
+    }
+  }
+  if (rank != 0) return;
+  __syncthreads();  // sel_s, bits_s complete
+  // 4. permutation of the na assignments
+  const bool nested = A.wbit || A.bits_in;
+  const int nbins = nested ? 3 * E : E;
+  for (int a = threadIdx.x; a < na; a += blockDim.x) {
+    int key = sel_s[a];
+    if (nested) {
+      int b = A.wbit ? bits_s[a] : A.bits_in[a];
+      if (b < 2 || b > 4) {
+        flag_status(A.status, MOE_DEV_BAD_INDEX);
+        b = b < 2 ? 2 : 4;
+      }
+      key = 3 * key + (b - 2);
+    }
+    key_s[a] = key;
+  }
+  __syncthreads();
+  for (int a = threadIdx.x; a < na; a += blockDim.x) {
+    const int key = key_s[a];
+    int pos = 0;
+    for (int o = 0; o < na; ++o) {
+      const int ko = key_s[o];
+      pos += (ko < key || (ko == key && o < a)) ? 1 : 0;
+    }
+    A.perm[pos] = a;
+    A.inv_perm[a] = pos;
+    perm_s[pos] = a;
+  }
+  for (int b = threadIdx.x; b <= nbins; b += blockDim.x) {
+    int below = 0, at = 0;
+    for (int o = 0; o < na; ++o) {
+      below += key_s[o] < b ? 1 : 0;
+      at += key_s[o] == b ? 1 : 0;
+    }
+    A.offsets[b] = below;
+    if (b < nbins) A.counts[b] = at;
+  }
+  if (!A.x_perm) return;
+  __syncthreads();  // perm_s complete
+  // gather: warp per row, 8 elements per lane per step (bf16 -> fp16)
+  bool bad = false;
+  for (int p = warp; p < na; p += kSelWarps) {
+    const uint4* src = reinterpret_cast<const uint4*>(A.x + static_cast<size_t>(perm_s[p] / k) * d);
+    uint4* dst = reinterpret_cast<uint4*>(A.x_perm + static_cast<size_t>(p) * d);
+    for (int c = lane; c < d / 8; c += 32) {
+      const uint4 v = src[c];
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+      uint4 o;
+      __half2* h2 = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(b2[j]);
+        bad |= fabsf(f.x) > 65504.0f || fabsf(f.y) > 65504.0f;
+        h2[j] = __floats2half2_rn(f.x, f.y);
+      }
+      dst[c] = o;
+    }
+  }
+  if (bad) flag_status(A.status, MOE_DEV_RANGE);
+}
+
 int route_splits(int T, int d, int E, size_t cap = static_cast<size_t>(-1)) {
   const int ec = E <= 16 ? 16 : 64;
   const int tt = ec == 64 ? Tile<64>::TT : Tile<16>::TT;
@@ -647,6 +834,24 @@ moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d
 }  // namespace
 
 int g_route_fused = 1;
+
+bool route_permute_fusable(int T, int d, int E, int k) {
+  return g_route_fused == 1 && T >= 1 && T <= kSelWarps && T * k <= kFusedAssign && T * E <= kClusterItems &&
+         d % (8 * kClusterSlices) == 0;
+}
+
+moe_status_t launch_route_permute_tiny(const void* x, const float* w_router, const float* bias,
+                                       const int32_t* forced, const uint8_t* bits_in, const float* w_bit,
+                                       const float* bias_bit, int T, int d, int E, int k, int32_t* idx,
+                                       float* w, uint8_t* bits_out, int32_t* counts, int32_t* offsets,
+                                       int32_t* perm, int32_t* inv_perm, void* x_perm, int32_t* status,
+                                       cudaStream_t s) {
+  RoutePermArgs A{static_cast<const __nv_bfloat16*>(x), w_router, bias, forced, bits_in, w_bit, bias_bit,
+                  T, d, E, k, idx, w, bits_out, counts, offsets, perm, inv_perm, static_cast<__half*>(x_perm),
+                  status};
+  return cuda_check(launch_cluster_pdl(k_route_perm_tiny, kClusterSlices, dim3(kSelThreads), 0, s, A),
+                    "moe_route_permute cluster launch");
+}
 
 size_t route_workspace_bytes(int T, int d, int E) {
   if (T <= 0 || d <= 0 || E <= 0) return 256;

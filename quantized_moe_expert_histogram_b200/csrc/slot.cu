@@ -18,9 +18,11 @@
 // planes it holds.  An expert is copied only up to the widest width its
 // assignments of the step use -- the Q2 planes and the scales for width 2,
 // plus D3 for 3, plus D4 for 4 -- and a resident expert needed wider later
-// receives only the missing planes.  Inside a wave the copies go plane by
-// plane (every Q2 + scales first, then every D3, then every D4): the bit
-// order of D2MoE's Hottest-Expert-Bit-First schedule.
+// receives only the missing planes.  The blob is laid out width by width
+// (Q2 of the three matrices and the scales, then D3, then D4), so either is
+// one contiguous copy -- the range between the ends of two widths -- with
+// an expert's base planes first (the bit order of D2MoE's
+// Hottest-Expert-Bit-First schedule, whose expert order is the wave order).
 #include <algorithm>
 #include <atomic>
 #include <new>
@@ -59,8 +61,7 @@ struct moe_slot_cache {
   uint8_t* pool = nullptr;
   // plane mode: byte ranges of the blob format (gate, up, down)
   bool planes = false;
-  size_t q2_off[3] = {}, q2_len[3] = {}, d3_off[3] = {}, d3_len[3] = {}, d4_off[3] = {}, d4_len[3] = {};
-  size_t sz_off = 0, sz_len = 0;
+  size_t width_end[5] = {};  // plane mode: blob bytes holding the planes up to width b (b = 2, 3, 4)
   std::vector<int> slot_of;        // expert -> slot, -1 when not resident
   std::vector<int> expert_in;      // slot -> expert, -1 when empty
   std::vector<int> width_in;       // slot -> widest width whose planes it holds (4 in blob mode)
@@ -95,14 +96,7 @@ namespace {
 // Bytes a copy of widths (from, to] moves.
 size_t copy_bytes(const moe_slot_cache* c, const SlotCopy& k) {
   if (!c->planes) return c->blob_bytes;
-  size_t n = 0;
-  for (int m = 0; m < 3; ++m) {
-    if (k.from < 2) n += c->q2_len[m];
-    if (k.from < 3 && k.to >= 3) n += c->d3_len[m];
-    if (k.from < 4 && k.to >= 4) n += c->d4_len[m];
-  }
-  if (k.from < 2) n += c->sz_len;
-  return n;
+  return c->width_end[k.to] - c->width_end[k.from];
 }
 
 // After a failed copy: the slots of waves >= w that were to receive copies
@@ -140,9 +134,9 @@ moe_status_t h2d(moe_slot_cache* c, int s, int e, size_t off, size_t len, cudaSt
                     "slot H2D copy");
 }
 
-// Issue the copies `todo` on `copy` after their slots are free: blob mode
-// one copy per expert; plane mode plane by plane (all Q2 + scales, then all
-// D3, then all D4).
+// Issue the copies `todo` on `copy` after their slots are free: one copy
+// per expert (plane mode: the blob range between the ends of widths from
+// and to).
 moe_status_t issue(moe_slot_cache* c, const std::vector<SlotCopy>& todo, cudaStream_t copy) {
   for (const SlotCopy& k : todo) {
     if (c->slot_free_valid[k.s]) {
@@ -152,26 +146,9 @@ moe_status_t issue(moe_slot_cache* c, const std::vector<SlotCopy>& todo, cudaStr
   }
   moe_status_t st = timing_mark(c, 0, copy);
   if (st != MOE_OK) return st;
-  if (!c->planes) {
-    for (const SlotCopy& k : todo)
-      if ((st = h2d(c, k.s, k.e, 0, c->blob_bytes, copy)) != MOE_OK) return st;
-  } else {
-    for (const SlotCopy& k : todo) {
-      if (k.from >= 2) continue;
-      for (int m = 0; m < 3; ++m)
-        if ((st = h2d(c, k.s, k.e, c->q2_off[m], c->q2_len[m], copy)) != MOE_OK) return st;
-      if ((st = h2d(c, k.s, k.e, c->sz_off, c->sz_len, copy)) != MOE_OK) return st;
-    }
-    for (const SlotCopy& k : todo) {
-      if (k.from >= 3 || k.to < 3) continue;
-      for (int m = 0; m < 3; ++m)
-        if ((st = h2d(c, k.s, k.e, c->d3_off[m], c->d3_len[m], copy)) != MOE_OK) return st;
-    }
-    for (const SlotCopy& k : todo) {
-      if (k.to < 4) continue;
-      for (int m = 0; m < 3; ++m)
-        if ((st = h2d(c, k.s, k.e, c->d4_off[m], c->d4_len[m], copy)) != MOE_OK) return st;
-    }
+  for (const SlotCopy& k : todo) {
+    const size_t off = c->planes ? c->width_end[k.from] : 0;
+    if ((st = h2d(c, k.s, k.e, off, copy_bytes(c, k), copy)) != MOE_OK) return st;
   }
   return timing_mark(c, 0, copy);
 }
@@ -211,18 +188,11 @@ moe_status_t create(int E, int slots, size_t blob_bytes, const void* host_blobs,
   c->blob_bytes = blob_bytes;
   c->host = static_cast<const uint8_t*>(host_blobs);
   c->pool = static_cast<uint8_t*>(device_pool);
-  if (planes) {
+  if (planes) {  // width by width: [Q2 x3 | scales x3 | D3 x3 | D4 x3]
     c->planes = true;
-    for (int m = 0; m < 3; ++m) {
-      c->q2_off[m] = planes->q2[m];
-      c->q2_len[m] = planes->d3[m] - planes->q2[m];
-      c->d3_off[m] = planes->d3[m];
-      c->d3_len[m] = planes->d4[m] - planes->d3[m];
-      c->d4_off[m] = planes->d4[m];
-      c->d4_len[m] = (m < 2 ? planes->q2[m + 1] : planes->sz[0]) - planes->d4[m];
-    }
-    c->sz_off = planes->sz[0];
-    c->sz_len = planes->bytes - planes->sz[0];
+    c->width_end[2] = planes->d3[0];
+    c->width_end[3] = planes->d4[0];
+    c->width_end[4] = planes->bytes;
   }
   c->slot_of.assign(E, -1);
   c->expert_in.assign(slots, -1);

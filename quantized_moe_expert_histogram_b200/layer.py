@@ -1,8 +1,9 @@
 """One quantised MoE layer driven through the C ABI.
 
 ``QuantMoELayer`` owns device buffers (plumbing: torch allocates them) and
-runs the path call by call: moe_route_topk -> moe_permute ->
-moe_grouped_ffn_wq -> moe_unpermute_combine.  No arithmetic happens here.
+runs the path call by call: moe_route_permute (router, optional bit gate,
+permutation) -> moe_grouped_ffn_wq -> moe_unpermute_combine.  No arithmetic
+happens here.
 """
 from __future__ import annotations
 
@@ -55,6 +56,9 @@ class QuantMoELayer:
                                  device=dev),
             perm_ws=torch.empty(moeq.moe_permute_workspace_bytes(T, self.E, k, self.layout == moeq.LAYOUT_PLANES),
                                 dtype=torch.uint8, device=dev),
+            rp_ws=torch.empty(moeq.moe_route_permute_workspace_bytes(T, d, self.E, k,
+                                                                     self.layout == moeq.LAYOUT_PLANES),
+                              dtype=torch.uint8, device=dev),
         )
 
     def views(self, T):
@@ -64,7 +68,7 @@ class QuantMoELayer:
                     offsets=b["offsets"], perm=b["perm"][:rows], inv_perm=b["inv_perm"][:rows],
                     x_perm=b["x_perm"][:rows], y_perm=b["y_perm"][:rows], workspace=b["workspace"],
                     y=b["y"][:T], status=b["status"], route_ws=b["route_ws"], perm_ws=b["perm_ws"],
-                    bits=b["bits"][:T])
+                    rp_ws=b["rp_ws"], bits=b["bits"][:T])
 
     def forward(self, x, bits=None, forced_idx=None, residual=None, stream=None):
         """One layer pass.  ``bits`` (uint8 [T,k], nested layout) fixes the
@@ -74,13 +78,10 @@ class QuantMoELayer:
         if T > self.max_tokens:
             raise ValueError(f"T={T} exceeds max_tokens={self.max_tokens}")
         v = self.views(T)
-        moeq.moe_route_topk(x, self.w_router, self.bias, self.k, forced_idx=forced_idx,
-                            topk_idx=v["topk_idx"], topk_w=v["topk_w"], workspace=v["route_ws"],
-                            stream=stream)
-        if bits is None and self.w_bit is not None:
-            bits = moeq.moe_bit_gate(x, self.w_bit, self.bias_bit, v["topk_idx"], bits=v["bits"],
-                                     status=v["status"], stream=stream)
-        moeq.moe_permute(v["topk_idx"], self.E, bits=bits, x=x, out=v, status=v["status"], stream=stream)
+        gate = bits is None and self.w_bit is not None
+        moeq.moe_route_permute(x, self.w_router, self.bias, self.k, forced_idx=forced_idx, bits=bits,
+                               w_bit=self.w_bit if gate else None, bias_bit=self.bias_bit if gate else None,
+                               out=v, status=v["status"], workspace=v["rp_ws"], stream=stream)
         moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], self.blobs, T, self.E, self.d, self.F,
                                 self.group, self.layout, workspace=v["workspace"], y_perm=v["y_perm"],
                                 status=v["status"], stream=stream)

@@ -39,6 +39,9 @@ _SIGS = {
     "moe_permute": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_p,
                            _c_p, _c_p, _c_sz, _c_p]),
     "moe_permute_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
+    "moe_route_permute": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p,
+                                 _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "moe_route_permute_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
     "moe_static_bits": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]),
     "moe_bit_gate": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]),
     "moe_ffn_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
@@ -198,6 +201,53 @@ def moe_permute(topk_idx, E, bits=None, x=None, out=None, status=None, workspace
         _ptr(out["inv_perm"], torch.int32), _ptr(out["x_perm"], torch.float16),
         _ptr(status, torch.int32, "status"), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
+    return out
+
+
+def moe_route_permute_workspace_bytes(T, d, E, k, nested):
+    return int(load().moe_route_permute_workspace_bytes(T, d, E, k, int(bool(nested))))
+
+
+def moe_route_permute(x, w_router, bias, k, forced_idx=None, bits=None, w_bit=None, bias_bit=None, out=None,
+                      status=None, workspace=None, gather=True, stream=None):
+    """Router, optional bit gate (w_bit) or given widths (bits), and the
+    permutation in one call.  Returns dict(topk_idx, topk_w, bits, counts,
+    offsets, perm, inv_perm, x_perm); 'bits' holds the gate's widths (or the
+    given ones, or None)."""
+    lib = load()
+    T, d = x.shape
+    E = w_router.shape[0]
+    dev = x.device
+    nested = bits is not None or w_bit is not None
+    nb = 3 * E if nested else E
+    if out is None:
+        out = {}
+    out = dict(out)
+    for key, shape, dt in (("topk_idx", (T, k), torch.int32), ("topk_w", (T, k), torch.float32),
+                           ("counts", (nb,), torch.int32), ("offsets", (nb + 1,), torch.int32),
+                           ("perm", (T * k,), torch.int32), ("inv_perm", (T * k,), torch.int32)):
+        if out.get(key) is None:
+            out[key] = torch.empty(*shape, dtype=dt, device=dev)
+    if gather and out.get("x_perm") is None:
+        out["x_perm"] = torch.empty(T * k, d, dtype=torch.float16, device=dev)
+    bits_out = None
+    if w_bit is not None:
+        bits_out = out.get("bits")
+        if bits_out is None:
+            bits_out = torch.empty(T, k, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = torch.empty(lib.moe_route_permute_workspace_bytes(T, d, E, k, int(nested)), dtype=torch.uint8,
+                                device=dev)
+    _check("moe_route_permute", lib.moe_route_permute(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_router, torch.float32, "w_router"), _ptr(bias, torch.float32, "bias"),
+        _ptr(forced_idx, torch.int32, "forced_idx"), _ptr(bits, torch.uint8, "bits"),
+        _ptr(w_bit, torch.float32, "w_bit"), _ptr(bias_bit, torch.float32, "bias_bit"), T, d, E, k,
+        _ptr(out["topk_idx"], torch.int32), _ptr(out["topk_w"], torch.float32), _ptr(bits_out, torch.uint8),
+        _ptr(out["counts"], torch.int32), _ptr(out["offsets"], torch.int32), _ptr(out["perm"], torch.int32),
+        _ptr(out["inv_perm"], torch.int32), _ptr(out["x_perm"] if gather else None, torch.float16),
+        _ptr(status, torch.int32, "status"), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    out["bits"] = bits_out if w_bit is not None else bits
     return out
 
 

@@ -183,3 +183,34 @@ def test_blob_layout_sizes_and_roundtrip():
                     word = int(sz[((n // 128) * G + c) * 128 + n % 128])
                     assert O.bf16_bits_to_f32(np.array([word & 0xFFFF]))[0] == s[n, c]
                     assert O.bf16_bits_to_f32(np.array([word >> 16]))[0] == z[n, c]
+
+
+def test_planes_blob_is_laid_out_width_by_width():
+    """Nested-plane blobs: what a b-bit read needs -- Q2 and the scales for
+    b = 2, D3 from b = 3, D4 at b = 4 (MWQ: W(2) = Q2, W(3) = Q2 + D3,
+    W(4) = Q2 + D3 + D4) -- is the blob's first bytes: keeping only the
+    prefix up to the end of width b and zeroing the rest still decodes every
+    matrix's codes truncated to b bits and its scales exactly, for every b."""
+    rng = np.random.default_rng(6)
+    d, F, g = 256, 384, 64
+    wg, wu = rng.normal(0, .02, (2, F, d)).astype(np.float32)
+    wd = rng.normal(0, .02, (d, F)).astype(np.float32)
+    off = O.blob_layout(d, F, g, "planes")
+    blob = O.build_blob(wg, wu, wd, g, "planes")
+    q2_bytes = (2 * F * d + d * F) // 4
+    sz_bytes = (2 * F * (d // g) + d * (F // g)) * 4
+    ends = {2: off["gate.d3"], 3: off["gate.d4"], 4: off["bytes"]}
+    assert ends[2] == q2_bytes + sz_bytes
+    assert ends[3] - ends[2] == ends[4] - ends[3] == (2 * F * d + d * F) // 8
+    for b, end in ends.items():
+        part = blob.copy()
+        part[end:] = 0
+        for m, w in (("gate", wg), ("up", wu), ("down", wd)):
+            N, K = w.shape
+            q, s, z = O.quantize_groups(w, g)
+            Q2 = part[off[m + ".q2"]:off[m + ".q2"] + N * K // 4].view(np.uint32).reshape(N, K // 16)
+            D3 = part[off[m + ".d3"]:off[m + ".d3"] + N * K // 8].view(np.uint32).reshape(N, K // 32)
+            D4 = part[off[m + ".d4"]:off[m + ".d4"] + N * K // 8].view(np.uint32).reshape(N, K // 32)
+            np.testing.assert_array_equal(O.join_planes(Q2, D3, D4, K), (q >> (4 - b)) << (4 - b))
+            o = off[m + ".sz"]
+            np.testing.assert_array_equal(part[o:o + N * (K // g) * 4], blob[o:o + N * (K // g) * 4])
