@@ -230,19 +230,16 @@ def make_instances(shape, T, R, seed, device, bit_gate=False):
 def kernel_launches(shape, T, bit_gate=False):
     """Kernels of this library launched by one layer step, following the
     library's own choices: router, bit gate and permutation as one cluster
-    launch for decode-sized batches (T <= 8, T*k <= 64, T*E <= 512,
-    d % 64 == 0); otherwise router 1 (one cluster launch up to 64 tokens) or
-    2, bit gate 1 when used, permutation 1 (single CTA, with the gather when
-    it is small) or 1 + gather, or 3 + gather; then FFN 2, combine 1."""
+    launch for the smallest batches (T <= 8, T*E <= 128, T*k <= 64, with a
+    bit gate T*k <= 32, d % 64 == 0); otherwise router 1 (fp64 cluster launch
+    for T*E <= 128) or 2, bit gate 1 when used, permutation 1 (single CTA,
+    with the gather when it is small) or 1 + gather, or 3 + gather; then
+    FFN 2, combine 1."""
     n = T * shape.k
-    if T <= 8 and n <= 64 and T * shape.E <= 512 and shape.d % 64 == 0:
+    if T <= 8 and T * shape.E <= 128 and n <= (32 if bit_gate else 64) and shape.d % 64 == 0:
         return 1 + 2 + 1
     nbins = shape.E * (3 if shape.layout == "planes" else 1)
-    d32 = shape.d // 32
-    splits = 1
-    while splits * 2 <= 8 and d32 % (splits * 2) == 0:
-        splits *= 2
-    route = 1 if (T <= 8 * splits and shape.E <= 64 and splits >= 2) else 2
+    route = 1 if (T <= 8 and T * shape.E <= 128 and shape.d % 64 == 0) else 2
     if n <= 1024:
         perm = 1 if n * shape.d <= 64 * 1024 else 2
     else:

@@ -203,8 +203,9 @@ MOE_API size_t moe_permute_workspace_bytes(int T, int E, int k, int nested);
  * then (with a bit gate) moe_bit_gate, then moe_permute, with their results
  * bit for bit ([ExactMoE] the router decides, every routed expert runs;
  * [D2MoE] Dual Routing: expert gate and bit gate side by side; [Read-ME]
- * expert-aware batching).  A decode-sized batch -- T <= 8, T*k <= 64,
- * T*E <= 512, d % 64 == 0 -- runs as one launch of a thread-block cluster
+ * expert-aware batching).  The smallest batches -- T <= 8, T*E <= 128,
+ * T*k <= 64 (with a bit gate T*k <= 32), d % 64 == 0 -- run as one launch
+ * of a thread-block cluster
  * (fp64 dot products for the logits and the width scores, then the
  * permutation and the gather in one CTA); other sizes issue the separate
  * launches on `stream`.
@@ -429,13 +430,12 @@ MOE_API void moe_debug_force_regime(int regime);
 MOE_API void moe_debug_set_trace(void* host_mapped_ints);
 
 /* Test hook (process-wide), selecting among paths with the same results:
- * 1 (the default): moe_route_topk takes up to 8 tokens (T*E <= 512,
- * d % 64 == 0) as fp64 logits in one thread-block-cluster launch and 9 to
- * 64 tokens (E <= 64) as the fp32-with-bound router in one cluster launch;
- * moe_bit_gate takes up to 64 assignments (d % 64 == 0) as fp64 scores in
- * one cluster launch.  2: the fp32-with-bound one-launch router also for up
- * to 8 tokens, and the fp32-with-bound bit gate for every size.  0: the
- * two-launch router and the fp32-with-bound bit gate for every size. */
+ * 1 (the default): moe_route_topk takes the smallest batches (T <= 8,
+ * T*E <= 128, d % 64 == 0) as fp64 logits in one thread-block-cluster
+ * launch, moe_bit_gate up to 32 assignments (d % 64 == 0) as fp64 scores in
+ * one cluster launch, and moe_route_permute fuses all three steps when
+ * both apply.  0: the fp32-with-bound router (two launches) and bit gate,
+ * and separate launches in moe_route_permute, at every size. */
 MOE_API void moe_debug_route_fused(int mode);
 
 /* Test hook of the on-device failure path: while enabled, the tensor-core

@@ -22,7 +22,7 @@
 // three W_bit rows (3 x d fp32) through L2, two 8-element steps of loads in
 // flight per lane.
 //
-// Up to 64 assignments (k_bit_gate_tiny): the 3 T k scores straight in fp64
+// Up to 32 assignments (k_bit_gate_tiny): the 3 T k scores straight in fp64
 // over a thread-block cluster (each CTA one slice of d, partials into CTA
 // 0's shared memory, added in slice order after a cluster barrier), with no
 // bound and no second pass.
@@ -132,7 +132,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_bit_gate(const __nv_bfloat16* _
   if (lane == 0) bits[a] = static_cast<uint8_t>(2 + best);
 }
 
-constexpr int kTinyAssign = 64;  // assignments of the cluster path (3 x 64 scores)
+constexpr int kTinyAssign = 64;  // shared-memory capacity of the cluster path (3 x 64 scores)
+static_assert(kTinyGateAssign <= kTinyAssign, "cluster bit gate capacity");
 
 __global__ void __launch_bounds__(kWarps * 32) k_bit_gate_tiny(const __nv_bfloat16* __restrict__ x,
                                                               const float* __restrict__ wb,
@@ -183,7 +184,10 @@ __global__ void __launch_bounds__(kWarps * 32) k_bit_gate_tiny(const __nv_bfloat
 moe_status_t launch_bit_gate(const void* x, const float* w_bit, const float* bias_bit, const int32_t* idx,
                              int T, int d, int E, int k, uint8_t* bits, int32_t* status, cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  if (g_route_fused == 1 && T * k <= kTinyAssign && d % (8 * kClusterSlices) == 0)
+  // up to kTinyGateAssign assignments (at most two rounds of scores per
+  // warp of the cluster): measured 46.9 -> 36.2 us for the one-token step of
+  // the nested layer with its gate, 82.1 -> 77.1 us at four tokens
+  if (g_route_fused == 1 && T * k <= kTinyGateAssign && d % (8 * kClusterSlices) == 0)
     return cuda_check(launch_cluster_pdl(k_bit_gate_tiny, kClusterSlices, dim3(kWarps * 32), 0, s,
                                          static_cast<const __nv_bfloat16*>(x), w_bit, bias_bit, idx, T, d, E, k,
                                          bits, status),

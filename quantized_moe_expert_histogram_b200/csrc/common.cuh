@@ -226,8 +226,11 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
                           const int32_t* forced, int T, int d, int E, int k, int32_t* idx,
                           float* w, void* workspace, size_t workspace_bytes, cudaStream_t s);
 size_t route_workspace_bytes(int T, int d, int E);
-extern int g_route_fused;  // test hook: 1 default, 2 fp32-bound paths, 0 also the two-launch router
-bool route_permute_fusable(int T, int d, int E, int k);
+extern int g_route_fused;  // test hook: 1 default, 0 no fp64 cluster paths
+constexpr int kTinyRouteItems = 128;  // router dot products of the fp64 cluster path (T*E)
+constexpr int kTinyGateAssign = 32;   // assignments of the fp64 cluster bit gate (T*k)
+bool route_tiny_ok(int T, int d, int E);
+bool route_permute_fusable(int T, int d, int E, int k, bool gate);
 moe_status_t launch_route_permute_tiny(const void* x, const float* w_router, const float* bias,
                                        const int32_t* forced, const uint8_t* bits_in, const float* w_bit,
                                        const float* bias_bit, int T, int d, int E, int k, int32_t* idx,

@@ -26,10 +26,10 @@
 //                   fp64 logits.  Gates are the softmax over the k picked
 //                   logits, in fp64 arithmetic on those values.
 //
-// Up to 8 tokens (k_route_tiny) the T*E dot products are few enough to take
-// straight in fp64, spread over a thread-block cluster: the selection then
-// runs on the fp64 logits with no bound and no second pass.  From 9 to 64
-// tokens both steps above run in one cluster launch (k_route_small).
+// For the smallest batches (k_route_tiny: T <= 8 and T*E <= 128) the T*E
+// dot products are few enough to take straight in fp64, spread over a
+// thread-block cluster: the selection then runs on the fp64 logits with no
+// bound and no second pass.
 //
 // Error bound of the fp32 sum: an FMA chain over m products errs by at most
 // g(m) times the sum of their magnitudes; a chunk (32 products) and then the
@@ -469,88 +469,7 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
   select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, blockIdx.x);
 }
 
-// Partial logits of slice `split` (dk wide) for a handful of tokens: a warp
-// per (token, expert) pair, four pairs per warp at a time with their loads in
-// flight together, lanes over the slice (four elements per lane per 128, an
-// FMA chain per lane, then a shuffle tree), so that no work is spent on the
-// empty rows of a 64-token tile.  The chain per lane, the tree and the
-// later sum over slices stay within the chunked bound g(32 + d/32) of the
-// tiled path.  The norms of the slice: pairs with e = 0 sum x^2, pairs with
-// t = 0 sum W^2.
-__device__ __forceinline__ void logits_pairs(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr,
-                                             int T, int d, int E, int dk, RouteWs ws, int split) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int k0 = split * dk;
-  constexpr int kP = 4;  // pairs of a warp whose loads are in flight together
-  for (int p0 = warp * kP; p0 < T * E; p0 += kSelWarps * kP) {
-    float acc[kP], xq[kP], wq[kP];
-#pragma unroll
-    for (int u = 0; u < kP; ++u) acc[u] = xq[u] = wq[u] = 0.f;
-    for (int i = lane * 4; i < dk; i += 128) {
-      uint2 xb[kP];
-      float4 wv[kP];
-#pragma unroll
-      for (int u = 0; u < kP; ++u) {
-        const int pr = min(p0 + u, T * E - 1), t = pr / E, e = pr - t * E;
-        xb[u] = *reinterpret_cast<const uint2*>(x + static_cast<size_t>(t) * d + k0 + i);
-        wv[u] = *reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * d + k0 + i);
-      }
-#pragma unroll
-      for (int u = 0; u < kP; ++u) {
-        const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb[u].x));
-        const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb[u].y));
-        acc[u] = fmaf(x01.x, wv[u].x, acc[u]);
-        acc[u] = fmaf(x01.y, wv[u].y, acc[u]);
-        acc[u] = fmaf(x23.x, wv[u].z, acc[u]);
-        acc[u] = fmaf(x23.y, wv[u].w, acc[u]);
-        xq[u] = fmaf(x01.x, x01.x, fmaf(x01.y, x01.y, fmaf(x23.x, x23.x, fmaf(x23.y, x23.y, xq[u]))));
-        wq[u] = fmaf(wv[u].x, wv[u].x, fmaf(wv[u].y, wv[u].y, fmaf(wv[u].z, wv[u].z, fmaf(wv[u].w, wv[u].w, wq[u]))));
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kP; ++u) {
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
-        xq[u] += __shfl_xor_sync(0xffffffffu, xq[u], o);
-        wq[u] += __shfl_xor_sync(0xffffffffu, wq[u], o);
-      }
-      const int pr = p0 + u;
-      if (lane == 0 && pr < T * E) {
-        const int t = pr / E, e = pr - t * E;
-        ws.partial[(static_cast<size_t>(split) * T + t) * E + e] = acc[u];
-        if (e == 0) ws.xsq[static_cast<size_t>(split) * T + t] = xq[u];
-        if (t == 0) ws.wsq[static_cast<size_t>(split) * E + e] = wq[u];
-      }
-    }
-  }
-}
-
-// Both steps in one launch for decode-sized batches (one token tile, one
-// expert tile): the CTAs of one thread-block cluster take one slice of d
-// each (threads 0..kLT-1 write the slice's partial logits and norms to the
-// workspace), a cluster barrier with release/acquire semantics makes them
-// visible to the whole cluster, and the first ceil(T / kSelWarps) CTAs run
-// the selection.  Same arithmetic and order as the two-launch path.
-template <int EC>
-__global__ void __launch_bounds__(kSelThreads) k_route_small(
-    const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, RouteWs ws, int splits, int dk,
-    const float* __restrict__ bias, const int32_t* __restrict__ forced, int T, int d, int E, int k,
-    float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w) {
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ __align__(16) float sm[];
-  const int rank = blockIdx.x;  // the grid is one cluster
-  if (T <= kSelWarps)
-    logits_pairs(x, wr, T, d, E, dk, ws, rank);
-  else if (threadIdx.x < kLT)
-    logits_tile<EC>(x, wr, T, d, E, dk, ws, 0, 0, rank, sm);
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-  if (rank * kSelWarps < T)
-    select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, rank);
-}
-
-// Decode-sized batches (T <= 8, T*E <= kClusterItems, d % 64 == 0): the
+// The smallest batches (route_tiny_ok: T <= 8, T*E <= 128, d % 64 == 0): the
 // logits straight in fp64 -- no fp32 stage, no bound, no re-evaluation.
 // One cluster of kClusterSlices CTAs, CTA r takes the slice [r d/8, (r+1)
 // d/8) of every (token, expert) dot product (cluster_partial_dots) and
@@ -606,8 +525,9 @@ __global__ void __launch_bounds__(kSelThreads) k_route_tiny(
 
 // ---- router + bit-width gate + permutation in one launch -------------
 //
-// A decode-sized batch (T <= 8, T*k <= kFusedAssign, T*E <= kClusterItems,
-// d % 64 == 0) through the whole front of the layer in one cluster launch,
+// The smallest batches (route_tiny_ok, T*k <= kFusedAssign, and with a bit
+// gate T*k <= kTinyGateAssign) through the whole front of the layer in one
+// cluster launch,
 // with the results of k_route_tiny, k_bit_gate_tiny and the permutation
 // kernels (same arithmetic, same order):
 //   1. every CTA: its d-slice of the T*E router dot products (fp64) -> CTA 0
@@ -835,9 +755,17 @@ moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d
 
 int g_route_fused = 1;
 
-bool route_permute_fusable(int T, int d, int E, int k) {
-  return g_route_fused == 1 && T >= 1 && T <= kSelWarps && T * k <= kFusedAssign && T * E <= kClusterItems &&
-         d % (8 * kClusterSlices) == 0;
+// The fp64 cluster router pays while each warp of the cluster has at most
+// two rounds of dot products (T*E <= 128 with 8 CTAs of 8 warps): measured
+// on the OLMoE-shaped layer, a one-token step 38.9 -> 32.3 us against the
+// two-launch router, two tokens 46.0 -> 43.0 us; at four and eight tokens
+// (four and eight rounds) the two-launch router was faster.
+bool route_tiny_ok(int T, int d, int E) {
+  return g_route_fused == 1 && T >= 1 && T <= kSelWarps && T * E <= kTinyRouteItems && d % (8 * kClusterSlices) == 0;
+}
+
+bool route_permute_fusable(int T, int d, int E, int k, bool gate) {
+  return route_tiny_ok(T, d, E) && T * k <= kFusedAssign && (!gate || 3 * T * k <= 3 * kTinyGateAssign);
 }
 
 moe_status_t launch_route_permute_tiny(const void* x, const float* w_router, const float* bias,
@@ -863,42 +791,6 @@ size_t route_min_workspace_bytes(int T, int d, int E) {
   return route_ws_for(1, T, E);
 }
 
-// One-launch route for decode-sized batches: a cluster of `splits` CTAs.
-template <int EC>
-moe_status_t launch_small(const __nv_bfloat16* x, const float* wr, const float* bias, const int32_t* forced,
-                          int T, int d, int E, int k, int splits, RouteWs ws, int32_t* idx, float* w,
-                          cudaStream_t s) {
-  using G = Tile<EC>;
-  static std::atomic<uint64_t> attr_set{0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_check(e, "moe_route_topk cudaGetDevice");
-  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
-  if (!bit || !(attr_set.load() & bit)) {
-    e = cudaFuncSetAttribute(k_route_small<EC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(G::SMEM));
-    if (e != cudaSuccess) return cuda_check(e, "moe_route_topk smem attribute");
-    attr_set.fetch_or(bit);
-  }
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(splits);
-  cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = G::SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = splits;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cuda_check(cudaLaunchKernelEx(&cfg, k_route_small<EC>, x, wr, ws, splits, d / splits, bias, forced, T, d, E,
-                                       k, route_gamma(d), idx, w),
-                    "moe_route_topk fused launch");
-}
-
 moe_status_t launch_route(const void* x, const float* w_router, const float* bias,
                           const int32_t* forced, int T, int d, int E, int k, int32_t* idx,
                           float* w, void* workspace, size_t workspace_bytes, cudaStream_t s) {
@@ -906,19 +798,11 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
   const int splits = route_splits(T, d, E, workspace_bytes);
   const RouteWs ws = route_ws(workspace, splits, T, E);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  // up to 8 tokens: fp64 logits in one cluster launch (no workspace)
-  if (g_route_fused == 1 && T <= kSelWarps && T * E <= kClusterItems && d % (8 * kClusterSlices) == 0)
+  // the smallest batches: fp64 logits in one cluster launch (no workspace)
+  if (route_tiny_ok(T, d, E))
     return cuda_check(launch_cluster_pdl(k_route_tiny, kClusterSlices, dim3(kSelThreads), 0, s, xb, w_router, bias,
                                          forced, T, d, E, k, idx, w),
                       "moe_route_topk cluster launch");
-  // decode-sized batches: one token tile and one expert tile, a cluster of
-  // up to 8 CTAs over d, selection in the same launch
-  const int fused_splits = std::min(splits, 8);
-  if (T <= kSelWarps * fused_splits && E <= 64 && fused_splits >= 2 && g_route_fused) {
-    const RouteWs wsf = route_ws(workspace, fused_splits, T, E);
-    return E <= 16 ? launch_small<16>(xb, w_router, bias, forced, T, d, E, k, fused_splits, wsf, idx, w, s)
-                   : launch_small<64>(xb, w_router, bias, forced, T, d, E, k, fused_splits, wsf, idx, w, s);
-  }
   moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, k, splits, ws, s)
                             : launch_logits<64>(xb, w_router, T, d, E, k, splits, ws, s);
   if (st != MOE_OK) return st;
@@ -977,7 +861,7 @@ moe_status_t route_scratch(void** out) {
 }  // namespace
 }  // namespace moeq
 
-extern "C" void moe_debug_route_fused(int mode) { moeq::g_route_fused = (mode >= 0 && mode <= 2) ? mode : 1; }
+extern "C" void moe_debug_route_fused(int mode) { moeq::g_route_fused = mode == 0 ? 0 : 1; }
 
 extern "C" moe_status_t moe_route_topk_noalloc(const void* x, const float* w_router, const float* bias,
                                                 const int32_t* forced_idx, int T, int d, int E, int k,

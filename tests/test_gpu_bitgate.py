@@ -35,7 +35,7 @@ def _oracle_sel(L, shape):
                                                ("mixtral", 1, False), ("olmoe", 256, True),
                                                ("tiny", 64, False), ("mixtral", 33, True)])
 def test_bit_gate_bitexact(name, T, with_bias):
-    """Widths bit for bit against the oracle: up to 64 assignments through the
+    """Widths bit for bit against the oracle: up to 32 assignments through the
     fp64 cluster kernel, beyond through the fp32-with-bound kernel."""
     shape = I.SHAPES[name]
     L = I.make_layer(shape, T, seed=21, weights=False)
@@ -84,10 +84,10 @@ def test_bit_gate_near_ties_resolved_exactly(scale, T):
         np.testing.assert_array_equal(ref, narrower)
 
 
-@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("mode", [1, 0])
 def test_bit_gate_flags_bad_ids(mode):
     """Out-of-range ids are flagged and clamped, by the fp64 cluster kernel
-    (mode 1, the default at this size) and the fp32 kernel (mode 2)."""
+    (mode 1, the default at this size) and the fp32 kernel (mode 0)."""
     moeq.moe_debug_route_fused(mode)
     try:
         _bad_ids_case()
@@ -97,8 +97,8 @@ def test_bit_gate_flags_bad_ids(mode):
 
 @pytest.mark.parametrize("name,T", [("nested", 1), ("nested", 16), ("mixtral", 8), ("olmoe", 8)])
 def test_bit_gate_small_paths_agree(name, T):
-    """For up to 64 assignments the fp64 cluster kernel (default) and the
-    fp32-with-bound kernel (test hook mode 2) give the same widths, which are
+    """The fp64 cluster kernel (default up to 32 assignments) and the
+    fp32-with-bound kernel (test hook mode 0) give the same widths, which are
     the oracle's."""
     shape = I.SHAPES[name]
     L = I.make_layer(shape, T, seed=27, weights=False)
@@ -106,7 +106,7 @@ def test_bit_gate_small_paths_agree(name, T):
     sel = _oracle_sel(L, shape)
     args = (L["x"].cuda(), G["w_bit"].cuda(), G["bias_bit"].cuda(), torch.from_numpy(sel).cuda())
     b1 = moeq.moe_bit_gate(*args)
-    moeq.moe_debug_route_fused(2)
+    moeq.moe_debug_route_fused(0)
     try:
         b2 = moeq.moe_bit_gate(*args)
     finally:

@@ -65,20 +65,21 @@ def test_route_bitexact(name, T, dup):
     np.testing.assert_allclose(w.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
 
 
-@pytest.mark.parametrize("name,T", [("olmoe", 1), ("olmoe", 8), ("olmoe", 33), ("olmoe", 64), ("nested", 1),
-                                    ("nested", 17), ("mixtral", 1), ("tiny", 64)])
+@pytest.mark.parametrize("name,T", [("olmoe", 1), ("olmoe", 2), ("olmoe", 8), ("olmoe", 33), ("nested", 1),
+                                    ("nested", 8), ("nested", 17), ("mixtral", 1), ("mixtral", 8), ("tiny", 16),
+                                    ("tiny", 64)])
 def test_route_fused_small_batches(name, T):
-    """Decode-sized batches run the router as one cluster launch (fp64 logits
-    up to 8 tokens, fp32 with the bound beyond); its expert ids equal the
-    two-launch router's, the fp32 one-launch router's and the oracle's bit
-    for bit, and all their gates match the oracle's."""
+    """The smallest batches run the router as one cluster launch on fp64
+    logits; at every size its expert ids equal the fp32-with-bound two-launch
+    router's and the oracle's bit for bit, and the gates match the
+    oracle's."""
     shape = I.SHAPES[name]
     L = I.make_layer(shape, T, seed=17, weights=False)
     bias = L["bias"].cuda() if L["bias"] is not None else None
     x, wr = L["x"].cuda(), L["w_router"].cuda()
     idx_f, w_f = moeq.moe_route_topk(x, wr, bias, shape.k)
     others = []
-    for mode in (0, 2):  # the two-launch router; the fp32 one-launch router at any size
+    for mode in (0,):  # the fp32-with-bound two-launch router
         moeq.moe_debug_route_fused(mode)
         try:
             others.append(moeq.moe_route_topk(x, wr, bias, shape.k))
@@ -94,14 +95,14 @@ def test_route_fused_small_batches(name, T):
         np.testing.assert_allclose(w_o.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
 
 
-@pytest.mark.parametrize("T", [300, 8])
+@pytest.mark.parametrize("T", [300, 2])
 @pytest.mark.parametrize("scale", [0.0, 1e-9, 1e-7, 1e-5])
 def test_route_near_ties_resolved_exactly(scale, T):
     """Router rows that are copies of others plus a perturbation of the given
     size: the logits of the pairs differ by about scale * |x| (exact ties at
     0), below what fp32 logits can order, so these tokens must take the fp64
-    re-evaluation (300 tokens) or be decided on fp64 logits (8 tokens) and
-    still match the oracle's choice and order exactly."""
+    re-evaluation (300 tokens) or be decided on fp64 logits (2 tokens, the
+    cluster path) and still match the oracle's choice and order exactly."""
     shape = I.SHAPES["olmoe"]
     L = I.make_layer(shape, T, seed=9, weights=False)
     w = L["w_router"].clone()
