@@ -133,55 +133,55 @@ __device__ __forceinline__ void cluster_sync_publish() {
 // Slice partials of n dot products by one CTA: item i pairs the bf16 row
 // and the fp32 row that rows(i, xr, wr) names, over elements [k0, k0 + dk)
 // (k0, dk multiples of 8, rows 16-byte aligned).  Warp w takes items w,
-// w + warps, ...; a lane takes the 8-element pieces k0 + 256 c + 8 lane,
-// sums each piece with an fp64 FMA chain from zero and adds the piece sums
-// in piece order; the warp adds the lane sums in a shuffle tree (every lane
-// ends with the same value).  Up to 8 pieces' loads are in flight together.
-// Lane 0 stores item i's partial at shared::cluster address dst + 8 i.
-// The order of operations does not depend on the item, so identical rows
-// give identical partials.
+// w + warps, ..., eight at a time: their row pointers are resolved once,
+// then chunk by chunk (256 elements) the eight items' pieces are loaded
+// together.  A lane takes the 8-element pieces k0 + 256 c + 8 lane, sums
+// each with an fp64 FMA chain from zero and adds the piece sums in chunk
+// order; the warp adds the lane sums in a shuffle tree (every lane ends
+// with the same value).  Lane 0 stores item i's partial at shared::cluster
+// address dst + 8 i.  The order of operations does not depend on the item,
+// so identical rows give identical partials.
 template <typename RowFn>
 __device__ __forceinline__ void cluster_partial_dots(int n, int k0, int dk, RowFn rows, uint32_t dst) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int nch = (dk + 255) / 256;
   const int mine = n > warp ? (n - warp + nw - 1) / nw : 0;
   for (int q0 = 0; q0 < mine; q0 += 8) {
     const int gi = min(8, mine - q0);
-    const int pieces = gi * nch;
+    const __nv_bfloat16* xr[8];
+    const float* wr[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      xr[j] = nullptr;
+      wr[j] = nullptr;
+      if (j < gi) rows(warp + nw * (q0 + j), xr[j], wr[j]);
+    }
     double acc[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-    for (int p0 = 0; p0 < pieces; p0 += 8) {
+    for (int off = lane * 8; off < dk; off += 256) {
       uint4 xb[8];
       float4 wa[8], wb[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int p = p0 + u, qi = p / nch, c = p - qi * nch, off = c * 256 + lane * 8;
-        if (p < pieces && off < dk) {
-          const __nv_bfloat16* xr;
-          const float* wr;
-          rows(warp + nw * (q0 + qi), xr, wr);
-          xb[u] = *reinterpret_cast<const uint4*>(xr + k0 + off);
-          wa[u] = *reinterpret_cast<const float4*>(wr + k0 + off);
-          wb[u] = *reinterpret_cast<const float4*>(wr + k0 + off + 4);
+      for (int j = 0; j < 8; ++j) {
+        if (j < gi) {
+          xb[j] = *reinterpret_cast<const uint4*>(xr[j] + k0 + off);
+          wa[j] = *reinterpret_cast<const float4*>(wr[j] + k0 + off);
+          wb[j] = *reinterpret_cast<const float4*>(wr[j] + k0 + off + 4);
         }
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int p = p0 + u, qi = p / nch, c = p - qi * nch, off = c * 256 + lane * 8;
-        if (p < pieces && off < dk) {
-          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb[u]);
-          const float w[8] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w, wb[u].x, wb[u].y, wb[u].z, wb[u].w};
+      for (int j = 0; j < 8; ++j) {
+        if (j < gi) {
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb[j]);
+          const float w[8] = {wa[j].x, wa[j].y, wa[j].z, wa[j].w, wb[j].x, wb[j].y, wb[j].z, wb[j].w};
           double s = 0.0;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 f = __bfloat1622float2(b2[j]);
-            s = fma(static_cast<double>(f.x), static_cast<double>(w[2 * j]), s);
-            s = fma(static_cast<double>(f.y), static_cast<double>(w[2 * j + 1]), s);
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(b2[q]);
+            s = fma(static_cast<double>(f.x), static_cast<double>(w[2 * q]), s);
+            s = fma(static_cast<double>(f.y), static_cast<double>(w[2 * q + 1]), s);
           }
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j == qi) acc[j] += s;
+          acc[j] += s;
         }
       }
     }
@@ -195,6 +195,32 @@ __device__ __forceinline__ void cluster_partial_dots(int n, int k0, int dk, RowF
       }
     }
   }
+}
+
+// The k largest of E fp64 values in shared memory, in descending order,
+// ties to the lower index, by one warp: each lane ranks its values
+// e = lane + 32 m against all E (independent compares, no dependent
+// chains) and the value of rank r < k writes its index to sel[r] (shared
+// memory).  NaN values are never picked; if fewer than k values are
+// comparable the remaining picks are expert 0 (the selection order of the
+// warp-shuffle top-k, which takes the first maximum k times).
+__device__ __forceinline__ void warp_topk_rank(const double* vals, int E, int k, int lane, int32_t* sel) {
+  int comparable = 0;
+  for (int e = lane; e < E; e += 32) {
+    const double v = vals[e];
+    comparable += v == v ? 1 : 0;
+    if (v != v) continue;
+    int rank = 0;
+    for (int o = 0; o < E; ++o) {
+      const double u = vals[o];  // NaN: both compares false
+      rank += (u > v || (u == v && o < e)) ? 1 : 0;
+    }
+    if (rank < k) sel[rank] = e;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) comparable += __shfl_xor_sync(0xffffffffu, comparable, o);
+  for (int r = comparable + lane; r < k; r += 32) sel[r] = 0;
+  __syncwarp();
 }
 
 // A launch of one thread-block cluster of `cluster` CTAs (grid = cluster),

@@ -469,19 +469,60 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
   select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, blockIdx.x);
 }
 
+// One token of the fp64 cluster paths, by one warp of CTA 0: its logits
+// (slice partials added in slice order, then the bias) into vals (shared),
+// the selection -- top k by rank counting, or the forced ids clamped into
+// range -- into sel (shared, k entries), then the gates (fp64 softmax over
+// the picks: maximum and sum as shuffle trees over the warp) and the ids to
+// global memory.
+__device__ __forceinline__ void tiny_select(const double* part, int n, int t, const float* bias,
+                                            const int32_t* forced, int E, int k, int lane, double* vals,
+                                            int32_t* sel, int32_t* out_idx, float* out_w) {
+  for (int e = lane; e < E; e += 32) {
+    double a = part[t * E + e];
+    for (int r = 1; r < kClusterSlices; ++r) a += part[r * n + t * E + e];
+    vals[e] = a + (bias ? static_cast<double>(bias[e]) : 0.0);
+  }
+  __syncwarp();
+  if (forced) {
+    for (int j = lane; j < k; j += 32) {
+      const int e = forced[static_cast<size_t>(t) * k + j];
+      sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
+    }
+    __syncwarp();
+  } else {
+    warp_topk_rank(vals, E, k, lane, sel);
+  }
+  const bool mine = lane < k;
+  const int e = mine ? sel[lane] : 0;
+  const double lv = mine ? vals[e] : -INFINITY;
+  double mx = lv;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const double ex = mine ? exp(lv - mx) : 0.0;
+  double sum = ex;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (mine) {
+    out_idx[static_cast<size_t>(t) * k + lane] = e;
+    out_w[static_cast<size_t>(t) * k + lane] = static_cast<float>(ex / sum);
+  }
+}
+
 // The smallest batches (route_tiny_ok: T <= 8, T*E <= 128, d % 64 == 0): the
 // logits straight in fp64 -- no fp32 stage, no bound, no re-evaluation.
 // One cluster of kClusterSlices CTAs, CTA r takes the slice [r d/8, (r+1)
 // d/8) of every (token, expert) dot product (cluster_partial_dots) and
 // stores the partials into CTA 0's shared memory; after the cluster barrier
 // CTA 0's warp t adds token t's partials in slice order and the bias (in
-// fp64) and selects on those logits (first maximum, ties to the lower index),
-// gates as the fp64 softmax over the picks.
+// fp64) and selects on those logits (tiny_select).
 __global__ void __launch_bounds__(kSelThreads) k_route_tiny(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
     const int32_t* __restrict__ forced, int T, int d, int E, int k, int32_t* __restrict__ out_idx,
     float* __restrict__ out_w) {
   __shared__ double part[kClusterSlices * kClusterItems];
+  __shared__ double vals[kTinyRouteItems];
+  __shared__ int32_t sel_s[kSelWarps * 16];
   pdl_wait();
   pdl_trigger();
   cluster_sync_start();
@@ -498,29 +539,8 @@ __global__ void __launch_bounds__(kSelThreads) k_route_tiny(
   cluster_sync_publish();
   if (rank != 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int t = warp; t < T; t += kSelWarps) {
-    double v[kPer];
-#pragma unroll
-    for (int m = 0; m < kPer; ++m) {
-      const int e = lane + 32 * m;
-      v[m] = -INFINITY;
-      if (e < E) {
-        double a = part[t * E + e];
-        for (int r = 1; r < kClusterSlices; ++r) a += part[r * n + t * E + e];
-        v[m] = a + (bias ? static_cast<double>(bias[e]) : 0.0);
-      }
-    }
-    int sel[16];
-    if (forced) {
-      for (int j = 0; j < k; ++j) {
-        const int e = forced[static_cast<size_t>(t) * k + j];
-        sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
-      }
-    } else {
-      warp_topk(v, 0xffu, E, k, lane, sel);
-    }
-    write_gates(v, sel, k, t, lane, out_idx, out_w);
-  }
+  if (warp < T)  // T <= kSelWarps: a warp per token
+    tiny_select(part, n, warp, bias, forced, E, k, lane, vals + warp * E, sel_s + warp * 16, out_idx, out_w);
 }
 
 // ---- router + bit-width gate + permutation in one launch -------------
@@ -562,6 +582,7 @@ struct RoutePermArgs {
 
 __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_constant__ RoutePermArgs A) {
   __shared__ double part[kClusterSlices * kClusterItems];
+  __shared__ double vals[kTinyRouteItems];
   __shared__ int32_t sel_s[kFusedAssign];
   __shared__ int32_t key_s[kFusedAssign];
   __shared__ int32_t perm_s[kFusedAssign];
@@ -583,34 +604,9 @@ __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_co
       },
       part0 + 8u * static_cast<uint32_t>(rank * n));
   cluster_sync_publish();
-  // 2. selection (CTA 0)
-  if (rank == 0) {
-    for (int t = warp; t < T; t += kSelWarps) {
-      double v[kPer];
-#pragma unroll
-      for (int m = 0; m < kPer; ++m) {
-        const int e = lane + 32 * m;
-        v[m] = -INFINITY;
-        if (e < E) {
-          double a = part[t * E + e];
-          for (int r = 1; r < kClusterSlices; ++r) a += part[r * n + t * E + e];
-          v[m] = a + (A.bias ? static_cast<double>(A.bias[e]) : 0.0);
-        }
-      }
-      int sel[16];
-      if (A.forced) {
-        for (int j = 0; j < k; ++j) {
-          const int e = A.forced[static_cast<size_t>(t) * k + j];
-          sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
-        }
-      } else {
-        warp_topk(v, 0xffu, E, k, lane, sel);
-      }
-      write_gates(v, sel, k, t, lane, A.idx, A.gw);
-      for (int j = 0; j < k; ++j)
-        if (j == lane) sel_s[t * k + j] = sel[j];
-    }
-  }
+  // 2. selection (CTA 0): a warp per token (T <= kSelWarps)
+  if (rank == 0 && warp < T)
+    tiny_select(part, n, warp, A.bias, A.forced, E, k, lane, vals + warp * E, sel_s + warp * k, A.idx, A.gw);
   // 3. bit-width gate
   if (A.wbit) {  // uniform over the cluster
     cluster_sync_publish();  // CTA 0's ids (sel_s) and its last reads of part are done
@@ -689,23 +685,31 @@ __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_co
   }
   if (!A.x_perm) return;
   __syncthreads();  // perm_s complete
-  // gather: warp per row, 8 elements per lane per step (bf16 -> fp16)
+  // gather: warp per row, 8 elements per lane per piece and up to 8
+  // pieces' loads in flight (bf16 -> fp16)
   bool bad = false;
   for (int p = warp; p < na; p += kSelWarps) {
     const uint4* src = reinterpret_cast<const uint4*>(A.x + static_cast<size_t>(perm_s[p] / k) * d);
     uint4* dst = reinterpret_cast<uint4*>(A.x_perm + static_cast<size_t>(p) * d);
-    for (int c = lane; c < d / 8; c += 32) {
-      const uint4 v = src[c];
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-      uint4 o;
-      __half2* h2 = reinterpret_cast<__half2*>(&o);
+    for (int c0 = lane; c0 < d / 8; c0 += 8 * 32) {
+      uint4 v[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(b2[j]);
-        bad |= fabsf(f.x) > 65504.0f || fabsf(f.y) > 65504.0f;
-        h2[j] = __floats2half2_rn(f.x, f.y);
+      for (int u = 0; u < 8; ++u)
+        if (c0 + 32 * u < d / 8) v[u] = src[c0 + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (c0 + 32 * u >= d / 8) break;
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+        uint4 o;
+        __half2* h2 = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(b2[j]);
+          bad |= fabsf(f.x) > 65504.0f || fabsf(f.y) > 65504.0f;
+          h2[j] = __floats2half2_rn(f.x, f.y);
+        }
+        dst[c0 + 32 * u] = o;
       }
-      dst[c] = o;
     }
   }
   if (bad) flag_status(A.status, MOE_DEV_RANGE);
