@@ -1,8 +1,10 @@
 """Benchmark: MoE-layer tokens/s of the W4A16 quantised MoE layer on B200.
 
-One step = one pass of the whole hot path over one batch: moe_route_topk ->
-moe_permute (histogram, scan, permutation, gather) -> moe_grouped_ffn_wq
-(dequant-fused gate/up + SwiGLU, then down) -> moe_unpermute_combine.
+One step = one pass of the whole hot path over one batch: moe_route_permute
+(router, optional bit gate, histogram, scan, permutation, gather) ->
+moe_grouped_ffn_combine (dequant-fused gate/up + SwiGLU, then down, then the
+weighted combine).  The FFN-only timing behind the roofline figure runs
+moe_grouped_ffn_wq alone.
 Default workload: the OLMoE-shaped layer (d=2048, E=64, top-8, d_ff=1024,
 INT4 g128, Zipf-skewed router bias) at T=4096 tokens.  Synthetic seeded
 inputs and random weights; R distinct layer instances are rotated so the
@@ -234,10 +236,12 @@ def kernel_launches(shape, T, bit_gate=False):
     bit gate T*k <= 32, d % 64 == 0); otherwise router 1 (fp64 cluster launch
     for T*E <= 128) or 2, bit gate 1 when used, permutation 1 (single CTA,
     with the gather when it is small) or 1 + gather, or 3 + gather; then
-    FFN 2, combine 1."""
+    FFN 2, and the combine 1 unless the decode kernel (T <= 16) sums it in
+    its second GEMM."""
     n = T * shape.k
+    comb = 0 if T <= 16 else 1  # the decode kernel (T <= 16) sums the combine in its second GEMM
     if T <= 8 and T * shape.E <= 128 and n <= (32 if bit_gate else 64) and shape.d % 64 == 0:
-        return 1 + 2 + 1
+        return 1 + 2 + comb
     nbins = shape.E * (3 if shape.layout == "planes" else 1)
     route = 1 if (T <= 8 and T * shape.E <= 128 and shape.d % 64 == 0) else 2
     if n <= 1024:
@@ -245,7 +249,7 @@ def kernel_launches(shape, T, bit_gate=False):
     else:
         perm = 4
     del nbins
-    return route + (1 if bit_gate else 0) + perm + 2 + 1
+    return route + (1 if bit_gate else 0) + perm + 2 + comb
 
 
 def profiled_traffic(workload, T):
@@ -299,11 +303,15 @@ def _step_calls(layer, x, bits, stream, part):
         moeq.moe_route_permute(x, layer.w_router, layer.bias, layer.k, bits=bits,
                                w_bit=layer.w_bit if gate else None, bias_bit=layer.bias_bit if gate else None,
                                out=v, status=v["status"], workspace=v["rp_ws"], stream=stream)
-    moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, T, layer.E, layer.d, layer.F,
-                            layer.group, layer.layout, workspace=v["workspace"], y_perm=v["y_perm"],
-                            status=v["status"], stream=stream)
     if part == "all":
-        moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], y=v["y"], stream=stream)
+        moeq.moe_grouped_ffn_combine(v["x_perm"], v["offsets"], layer.blobs, T, layer.k, layer.E, layer.d,
+                                     layer.F, layer.group, layer.layout, v["perm"], v["inv_perm"], v["topk_w"],
+                                     y=v["y"], y_perm=v["y_perm"], workspace=v["workspace"], status=v["status"],
+                                     stream=stream)
+    else:
+        moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, T, layer.E, layer.d, layer.F,
+                                layer.group, layer.layout, workspace=v["workspace"], y_perm=v["y_perm"],
+                                status=v["status"], stream=stream)
 
 
 def capture(layers, stream, part):

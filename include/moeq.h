@@ -260,6 +260,28 @@ MOE_API moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offse
                                 size_t workspace_bytes, void* y_perm, int32_t* status,
                                 moe_stream_t stream);
 
+/* moe_grouped_ffn_combine -- moe_grouped_ffn_wq (every expert resident,
+ * blob e = expert e) followed by moe_unpermute_combine, with the results of
+ * the two calls bit for bit (y_perm and y; [ExactMoE] every routed expert
+ * runs exactly, weighted by its gate).  With the decode kernel (T <= 16)
+ * the combine runs inside the second GEMM's epilogue: the work unit that
+ * completes the last of a token's k expert rows for a block of output
+ * columns sums that block of y[t] (same fp32 order as the separate
+ * combine), so no combine launch follows; larger batches issue the two
+ * calls.
+ *   perm, inv_perm  int32 [T*k] from moe_permute; topk_w fp32 [T][k];
+ *   residual        bf16 [T][d] or NULL; y bf16 [T][d]; y_perm fp16 [T*k][d]
+ *   workspace >= moe_ffn_combine_workspace_bytes(T, k, E, d, F, layout),
+ *   16-byte aligned (the FFN's intermediate and the combine's counters,
+ *   which the call resets itself).
+ * Requires k <= 16, d % 16 == 0; errors and flags as in the two calls. */
+MOE_API moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets, const void* blobs, int T,
+                                             int k, int E, int d, int F, int group, int layout,
+                                             const int32_t* perm, const int32_t* inv_perm, const float* topk_w,
+                                             const void* residual, void* y, void* y_perm, void* workspace,
+                                             size_t workspace_bytes, int32_t* status, moe_stream_t stream);
+MOE_API size_t moe_ffn_combine_workspace_bytes(int T, int k, int E, int d, int F, int layout);
+
 /* moe_bit_gate -- bit-width router ([D2MoE] Dual Routing: x -> Bit Gate ->
  * b beside x -> Expert Gate -> E; Token-Adaptive Bit-Width Selection): the
  * width at which each selected expert runs for each token.  For the j-th

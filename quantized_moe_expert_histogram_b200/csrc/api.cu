@@ -343,6 +343,90 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   return launch_ffn_decode(a, regime == 1 ? 1 : 2, S(stream));
 }
 
+size_t moe_ffn_combine_workspace_bytes(int T, int k, int E, int d, int F, int layout) {
+  (void)E;
+  (void)layout;
+  if (T <= 0 || k <= 0 || d <= 0 || F <= 0) return 256;
+  return workspace_for(T * k, F) + ((static_cast<size_t>(T) * (d / 16) * sizeof(int32_t) + 255) & ~size_t(255));
+}
+
+moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets, const void* blobs, int T, int k,
+                                     int E, int d, int F, int group, int layout, const int32_t* perm,
+                                     const int32_t* inv_perm, const float* topk_w, const void* residual, void* y,
+                                     void* y_perm, void* workspace, size_t workspace_bytes, int32_t* status,
+                                     moe_stream_t stream) {
+  if (T < 0 || k <= 0 || k > 16 || E <= 0 || d <= 0 || d % 16) {
+    set_error("moe_grouped_ffn_combine: bad sizes T=%d k=%d E=%d d=%d", T, k, E, d);
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (T == 0) return MOE_OK;
+  if (!perm || !inv_perm || !topk_w || !y) {
+    set_error("moe_grouped_ffn_combine: null pointer");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (static_cast<long>(T) * k > (1L << 24)) {
+    set_error("moe_grouped_ffn_combine: T*k exceeds 2^24");
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  const size_t need = moe_ffn_combine_workspace_bytes(T, k, E, d, F, layout);
+  if (!workspace || workspace_bytes < need) {
+    set_error("moe_grouped_ffn_combine: workspace %zu < %zu bytes", workspace_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  const int total_rows = T * k;
+  const size_t hbytes = workspace_for(total_rows, F);
+  int regime = g_force_regime;
+  if (regime == 0) regime = T <= kDecMaxT ? (T <= 8 ? 1 : 3) : 2;
+  if (regime == 1 || regime == 3) {  // decode kernel: the combine rides in the second GEMM's epilogue
+    const BlobLayout L = blob_layout(d, F, group, layout);
+    if (!L.valid) {
+      set_error("moe_grouped_ffn_combine: unsupported shape d=%d F=%d group=%d layout=%d", d, F, group, layout);
+      return MOE_ERR_UNSUPPORTED_SHAPE;
+    }
+    if (!x_perm || !offsets || !blobs || !y_perm) {
+      set_error("moe_grouped_ffn_combine: null pointer");
+      return MOE_ERR_INVALID_ARG;
+    }
+    if (!aligned16(x_perm) || !aligned16(blobs) || !aligned16(workspace) || !aligned16(y_perm)) {
+      set_error("moe_grouped_ffn_combine: buffers must be 16-byte aligned");
+      return MOE_ERR_INVALID_ARG;
+    }
+    if (E * (layout == MOE_LAYOUT_PLANES ? 3 : 1) > 768) {
+      set_error("moe_grouped_ffn_combine: too many bins");
+      return MOE_ERR_UNSUPPORTED_SHAPE;
+    }
+    FfnArgs a{};
+    a.x_perm = static_cast<const __half*>(x_perm);
+    a.offsets = offsets;
+    a.blobs = static_cast<const uint8_t*>(blobs);
+    a.slot_of = nullptr;
+    a.total_rows = total_rows;
+    a.T = T;
+    a.E = E;
+    a.d = d;
+    a.F = F;
+    a.group = group;
+    a.layout = layout;
+    a.blob_bytes = L.bytes;
+    a.lay = L;
+    a.h = static_cast<__half*>(workspace);
+    a.y_perm = static_cast<__half*>(y_perm);
+    a.status = status;
+    a.k = k;
+    a.perm = perm;
+    a.inv_perm = inv_perm;
+    a.topk_w = topk_w;
+    a.residual = static_cast<const __nv_bfloat16*>(residual);
+    a.y = static_cast<__nv_bfloat16*>(y);
+    a.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + hbytes);
+    return launch_ffn_decode(a, regime == 1 ? 1 : 2, S(stream));
+  }
+  moe_status_t st = moe_grouped_ffn_wq(x_perm, offsets, blobs, nullptr, total_rows, T, E, d, F, group, layout,
+                                       workspace, hbytes, y_perm, status, stream);
+  if (st != MOE_OK) return st;
+  return moe_unpermute_combine(y_perm, inv_perm, topk_w, residual, T, k, d, y, stream);
+}
+
 moe_status_t moe_bit_gate(const void* x, const float* w_bit, const float* bias_bit, const int32_t* topk_idx,
                           int T, int d, int E, int k, uint8_t* bits, int32_t* status, moe_stream_t stream) {
   if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E) {

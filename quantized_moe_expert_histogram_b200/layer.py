@@ -2,8 +2,8 @@
 
 ``QuantMoELayer`` owns device buffers (plumbing: torch allocates them) and
 runs the path call by call: moe_route_permute (router, optional bit gate,
-permutation) -> moe_grouped_ffn_wq -> moe_unpermute_combine.  No arithmetic
-happens here.
+permutation) -> moe_grouped_ffn_combine (grouped FFN and weighted
+combine).  No arithmetic happens here.
 """
 from __future__ import annotations
 
@@ -47,7 +47,8 @@ class QuantMoELayer:
             inv_perm=torch.empty(rows, dtype=torch.int32, device=dev),
             x_perm=torch.empty(rows, d, dtype=torch.float16, device=dev),
             y_perm=torch.empty(rows, d, dtype=torch.float16, device=dev),
-            workspace=torch.empty(max(16, moeq.moe_ffn_workspace_bytes(rows, self.E, d, self.F, self.layout)),
+            workspace=torch.empty(max(16, moeq.moe_ffn_workspace_bytes(rows, self.E, d, self.F, self.layout),
+                                      moeq.moe_ffn_combine_workspace_bytes(T, k, self.E, d, self.F, self.layout)),
                                   dtype=torch.uint8, device=dev),
             y=torch.empty(T, d, dtype=torch.bfloat16, device=dev),
             bits=torch.empty(T, k, dtype=torch.uint8, device=dev),
@@ -82,9 +83,8 @@ class QuantMoELayer:
         moeq.moe_route_permute(x, self.w_router, self.bias, self.k, forced_idx=forced_idx, bits=bits,
                                w_bit=self.w_bit if gate else None, bias_bit=self.bias_bit if gate else None,
                                out=v, status=v["status"], workspace=v["rp_ws"], stream=stream)
-        moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], self.blobs, T, self.E, self.d, self.F,
-                                self.group, self.layout, workspace=v["workspace"], y_perm=v["y_perm"],
-                                status=v["status"], stream=stream)
-        moeq.moe_unpermute_combine(v["y_perm"], v["inv_perm"], v["topk_w"], residual=residual,
-                                   y=v["y"], stream=stream)
+        moeq.moe_grouped_ffn_combine(v["x_perm"], v["offsets"], self.blobs, T, self.k, self.E, self.d, self.F,
+                                     self.group, self.layout, v["perm"], v["inv_perm"], v["topk_w"],
+                                     residual=residual, y=v["y"], y_perm=v["y_perm"], workspace=v["workspace"],
+                                     status=v["status"], stream=stream)
         return v["y"]

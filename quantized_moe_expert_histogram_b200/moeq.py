@@ -48,6 +48,9 @@ _SIGS = {
     "moe_grouped_ffn_wq": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                   _c_p, _c_sz, _c_p, _c_p, _c_p]),
     "moe_unpermute_combine": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_p, _c_p]),
+    "moe_grouped_ffn_combine": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p,
+                                       _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p, _c_p]),
+    "moe_ffn_combine_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_i]),
     "moe_slot_cache_create": (_c_i, [_c_i, _c_i, _c_sz, _c_p, _c_p, ctypes.POINTER(_c_p)]),
     "moe_slot_cache_create_planes": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, ctypes.POINTER(_c_p)]),
     "moe_slot_stage": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p]),
@@ -277,6 +280,31 @@ def moe_bit_gate(x, w_bit, bias_bit, topk_idx, bits=None, status=None, stream=No
         _ptr(bias_bit, torch.float32, "bias_bit"), _ptr(topk_idx, torch.int32, "topk_idx"), T, d, E, k,
         _ptr(bits, torch.uint8, "bits"), _ptr(status, torch.int32, "status"), _stream(stream)))
     return bits
+
+
+def moe_ffn_combine_workspace_bytes(T, k, E, d, F, layout):
+    return int(load().moe_ffn_combine_workspace_bytes(T, k, E, d, F, layout))
+
+
+def moe_grouped_ffn_combine(x_perm, offsets, blobs, T, k, E, d, F, group, layout, perm, inv_perm, topk_w,
+                            residual=None, y=None, y_perm=None, workspace=None, status=None, stream=None):
+    """The grouped FFN and the weighted combine in one call; returns (y, y_perm)."""
+    lib = load()
+    dev = x_perm.device
+    if y is None:
+        y = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    if y_perm is None:
+        y_perm = torch.empty(T * k, d, dtype=torch.float16, device=dev)
+    if workspace is None:
+        workspace = torch.empty(lib.moe_ffn_combine_workspace_bytes(T, k, E, d, F, layout), dtype=torch.uint8,
+                                device=dev)
+    _check("moe_grouped_ffn_combine", lib.moe_grouped_ffn_combine(
+        _ptr(x_perm, torch.float16, "x_perm"), _ptr(offsets, torch.int32, "offsets"), _ptr(blobs), T, k, E, d, F,
+        group, layout, _ptr(perm, torch.int32, "perm"), _ptr(inv_perm, torch.int32, "inv_perm"),
+        _ptr(topk_w, torch.float32, "topk_w"), _ptr(residual, torch.bfloat16, "residual"),
+        _ptr(y, torch.bfloat16, "y"), _ptr(y_perm, torch.float16, "y_perm"), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status, torch.int32, "status"), _stream(stream)))
+    return y, y_perm
 
 
 def moe_grouped_ffn_wq(x_perm, offsets, blobs, T, E, d, F, group, layout, slot_of=None,

@@ -1,0 +1,79 @@
+"""The grouped FFN and the weighted combine in one call
+(moe_grouped_ffn_combine; ExactMoE: every routed expert runs exactly,
+weighted by its gate).  With the decode kernel the combine is summed in the
+second GEMM's epilogue by whichever work unit completes a token's rows; y
+and y_perm must equal the separate calls' (moe_grouped_ffn_wq, then
+moe_unpermute_combine) bit for bit, for every batch size, with and without
+a residual, with nested widths, and when a token names one expert twice
+(a bin holding more rows than there are tokens)."""
+import numpy as np
+import pytest
+import torch
+
+from quantized_moe_expert_histogram_b200 import build
+from quantized_moe_expert_histogram_b200 import inputs as I
+from quantized_moe_expert_histogram_b200 import moeq
+from quantized_moe_expert_histogram_b200.layer import QuantMoELayer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+    moeq.load()
+    moeq.moe_debug_force_regime(0)
+
+
+def _run(shape, T, seed, residual=True, forced=None, bits=None):
+    L = I.make_layer(shape, T, seed=seed)
+    layer = QuantMoELayer.from_weights(shape, L["w_router"].cuda(), L["bias"].cuda() if L["bias"] is not None
+                                       else None, L["w_gate"].cuda(), L["w_up"].cuda(), L["w_down"].cuda(),
+                                       max_tokens=T)
+    x = L["x"].cuda()
+    if bits is None and shape.layout == "planes":
+        bits = L["bits"].cuda()
+    v = layer.views(T)
+    moeq.moe_route_permute(x, layer.w_router, layer.bias, shape.k, forced_idx=forced, bits=bits, out=v,
+                           status=v["status"], workspace=v["rp_ws"])
+    res = x if residual else None
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y_f, yp_f = moeq.moe_grouped_ffn_combine(v["x_perm"], v["offsets"], layer.blobs, T, shape.k, shape.E, shape.d,
+                                             shape.F, shape.group, layer.layout, v["perm"], v["inv_perm"],
+                                             v["topk_w"], residual=res, status=status)
+    yp_s = moeq.moe_grouped_ffn_wq(v["x_perm"], v["offsets"], layer.blobs, T, shape.E, shape.d, shape.F,
+                                   shape.group, layer.layout, status=status).clone()
+    y_s = torch.empty_like(y_f)
+    moeq.moe_unpermute_combine(yp_s, v["inv_perm"], v["topk_w"], residual=res, y=y_s)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return y_f, yp_f, y_s, yp_s
+
+
+@pytest.mark.parametrize("name,T", [("olmoe", 1), ("olmoe", 2), ("olmoe", 8), ("olmoe", 9), ("olmoe", 16),
+                                    ("mixtral", 1), ("mixtral", 8), ("nested", 1), ("nested", 4), ("nested", 16),
+                                    ("tiny", 3), ("olmoe", 32)])
+def test_ffn_combine_equals_separate_calls(name, T):
+    shape = I.SHAPES[name]
+    y_f, yp_f, y_s, yp_s = _run(shape, T, seed=61 + T)
+    assert torch.equal(yp_f, yp_s)
+    assert torch.equal(y_f, y_s)
+
+
+def test_ffn_combine_without_residual_and_repeated_experts():
+    """No residual; and forced ids where every token names its first expert
+    twice, so that expert's bin holds up to 2 T rows -- more than the tokens
+    in the batch -- and each token's k rows still complete exactly once."""
+    shape = I.SHAPES["olmoe"]
+    T = 4
+    y_f, yp_f, y_s, yp_s = _run(shape, T, seed=71, residual=False)
+    assert torch.equal(y_f, y_s) and torch.equal(yp_f, yp_s)
+    rng = np.random.default_rng(5)
+    ids = np.stack([rng.permutation(shape.E)[:shape.k] for _ in range(T)]).astype(np.int32)
+    ids[:, 1] = ids[:, 0]
+    ids[:, 0] = 3  # every token: expert 3 twice
+    ids[:, 1] = 3
+    forced = torch.from_numpy(ids).cuda()
+    y_f, yp_f, y_s, yp_s = _run(shape, T, seed=72, forced=forced)
+    assert torch.equal(yp_f, yp_s)
+    assert torch.equal(y_f, y_s)
