@@ -197,6 +197,75 @@ __device__ __forceinline__ void cluster_partial_dots(int n, int k0, int dk, RowF
   }
 }
 
+// fp32 slice partials of n dot products by one CTA, with the sum of the
+// products' magnitudes for the error bound: as cluster_partial_dots, but a
+// lane sums all its products of the slice in one fp32 FMA chain (pieces in
+// chunk order) and the warp adds the lane sums in a 5-level shuffle tree,
+// so |S - s| <= g(m) A with m = (products per lane) + 5 and A the exact sum
+// of magnitudes (the computed A errs by the same relative g(m)).  Lane 0
+// stores (S, A) as a float2 at shared::cluster address dst + 8 i.
+__device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+template <typename RowFn>
+__device__ __forceinline__ void cluster_partial_dots_f32(int n, int k0, int dk, RowFn rows, uint32_t dst) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int mine = n > warp ? (n - warp + nw - 1) / nw : 0;
+  for (int q0 = 0; q0 < mine; q0 += 8) {
+    const int gi = min(8, mine - q0);
+    const __nv_bfloat16* xr[8];
+    const float* wr[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      xr[j] = nullptr;
+      wr[j] = nullptr;
+      if (j < gi) rows(warp + nw * (q0 + j), xr[j], wr[j]);
+    }
+    float acc[8], mag[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = mag[j] = 0.0f;
+    for (int off = lane * 8; off < dk; off += 256) {
+      uint4 xb[8];
+      float4 wa[8], wb[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < gi) {
+          xb[j] = *reinterpret_cast<const uint4*>(xr[j] + k0 + off);
+          wa[j] = *reinterpret_cast<const float4*>(wr[j] + k0 + off);
+          wb[j] = *reinterpret_cast<const float4*>(wr[j] + k0 + off + 4);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < gi) {
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb[j]);
+          const float w[8] = {wa[j].x, wa[j].y, wa[j].z, wa[j].w, wb[j].x, wb[j].y, wb[j].z, wb[j].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(b2[q]);
+            acc[j] = fmaf(f.x, w[2 * q], acc[j]);
+            mag[j] = fmaf(fabsf(f.x), fabsf(w[2 * q]), mag[j]);
+            acc[j] = fmaf(f.y, w[2 * q + 1], acc[j]);
+            mag[j] = fmaf(fabsf(f.y), fabsf(w[2 * q + 1]), mag[j]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j < gi) {  // warp-uniform
+        float a = acc[j], m = mag[j];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          a += __shfl_xor_sync(0xffffffffu, a, o);
+          m += __shfl_xor_sync(0xffffffffu, m, o);
+        }
+        if (lane == 0) st_cluster_f32x2(dst + 8u * static_cast<uint32_t>(warp + nw * (q0 + j)), a, m);
+      }
+    }
+  }
+}
+
 // The k largest of E fp64 values in shared memory, in descending order,
 // ties to the lower index, by one warp: each lane ranks its values
 // e = lane + 32 m against all E (independent compares, no dependent

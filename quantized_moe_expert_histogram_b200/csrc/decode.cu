@@ -11,19 +11,17 @@
 // K run spans two groups, A holds (q - z) * s rounded once to fp16, as in
 // the 128-row kernel).
 //
-// Work split: a work unit is (bin, block of weight rows, pass over xr of the
-// bin's token rows, xr = min(8 NB, T)): 16 features x {gate, up} in the
-// first GEMM, 16 or 32 rows of W_down in the second.  The grid is
-// persistent (as many CTAs as fit on the GPU at once); CTA b takes units b,
-// b + grid, ...  The 8 warps of a CTA split each unit's K: warp w takes the
-// 128-K stages w, w+8, w+16, ... of every row of the unit (so a 14336-long
-// row is eight warps' work, and at any time the CTA reads a contiguous K
-// window of each row).  Each warp streams its stages with cp.async into a
-// shared-memory ring -- the weights and the unit's activation rows of the
-// stage's K range, so neither waits on a global load at use nor holds
-// registers in flight -- and the stream runs on across units: the next
-// unit's first stages are in flight while the current unit's partial sums
-// are added (in shared memory, in a fixed order: deterministic) and its
+// Work split: a work unit is (bin, block of weight rows, pass over 8 NB of
+// the bin's token rows): 16 features x {gate, up} in the first GEMM, 16 or
+// 32 rows of W_down in the second.  The grid is persistent (as many CTAs as
+// fit on the GPU at once); CTA b takes units b, b + grid, ...  The 8 warps
+// of a CTA split each unit's K: warp w takes the 128-K stages w, w+8, w+16,
+// ... of every row of the unit (so a 14336-long row is eight warps' work,
+// and at any time the CTA reads a contiguous K window of each row).  Each
+// warp streams its stages with cp.async into a shared-memory ring (the bytes
+// in flight take no registers), and the stream runs on across units: the
+// next unit's first stages are in flight while the current unit's partial
+// sums are added (in shared memory, in a fixed order: deterministic) and its
 // epilogue writes h = silu(gate) * up or y_perm (fp16).  The non-empty,
 // resident bins are listed once per CTA in shared memory.
 //
@@ -38,8 +36,7 @@
 //
 // Both passes are programmatic dependent launches (launch_pdl).  The down
 // pass lists its bins and issues the copies of its first weight stages
-// (which do not depend on h) before it waits for the gate/up grid, and the
-// activation rows of those stages after it.
+// (which do not depend on h) before it waits for the gate/up grid.
 //
 //   gate/up pass:  h[p][f]      = silu(Wg[f] . x_p) * (Wu[f] . x_p)   (fp16)
 //   down pass:     y_perm[p][n] = Wd[n] . h_p                          (fp16)
@@ -56,7 +53,6 @@ constexpr int kStageK = 128;       // K per stage (one group of 128, two of 64)
 constexpr int kFragBytes = 1024;   // one stage of one 16-row fragment: 16 rows x 64 B
 constexpr int kSzBytes = 128;      // its scale/zero words: 16 rows x up to 2 groups
 constexpr int kRing = 3;           // stages in flight per warp
-constexpr int kXRow = kStageK * 2; // one activation row of a stage (fp16)
 
 struct DecParams {
   const __half* act;        // x_perm or h: fp16 [rows][K]
@@ -73,7 +69,6 @@ struct DecParams {
   int group;
   int row_blocks;           // weight-row blocks per bin
   int max_ent;              // capacity of the bin list (>= non-empty bins)
-  int xr;                   // activation rows staged per ring stage (most token rows of a unit)
   __half* out;              // h (gate/up) or y_perm (down): fp16 [rows][N]
   int32_t* status;
   // fused combine (down pass): y[t][n] = bf16(res[t][n] + sum_j g[t][j] y_perm[inv_perm[t k + j]][n]),
@@ -160,19 +155,15 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
 }
 
 // Shared-memory layout of a CTA: the warps' rings, the reduction buffer,
-// the bin list.  A ring stage holds the weights (FW fragments with their
-// scale/zero words) and xr activation rows of the stage's 128 K (fp16,
-// 256 B each), xr = the most token rows a unit can have.
+// the bin list.
 template <int FW, int NB>
 struct Smem {
-  static constexpr int kW = FW * (kFragBytes + kSzBytes);  // weights of one ring stage of a warp
-  static constexpr int kVals = FW * NB * 4;                // partial sums per lane
-  __host__ __device__ static constexpr int slot(int xr) { return kW + xr * kXRow; }
-  __host__ __device__ static constexpr int red0(int xr) { return kWarps * kRing * slot(xr); }
-  __host__ __device__ static constexpr int ent0(int xr) { return red0(xr) + kWarps * kVals * 32 * 4; }
-  static constexpr size_t bytes(int xr, int max_ent) {
-    return ent0(xr) + static_cast<size_t>(max_ent) * sizeof(BinEnt);
-  }
+  static constexpr int kSlot = FW * (kFragBytes + kSzBytes);  // one ring stage of a warp
+  static constexpr int kVals = FW * NB * 4;                    // partial sums per lane
+  static constexpr int kRing0 = 0;
+  static constexpr int kRed0 = kWarps * kRing * kSlot;
+  static constexpr int kEnt0 = kRed0 + kWarps * kVals * 32 * 4;
+  static constexpr size_t bytes(int max_ent) { return kEnt0 + static_cast<size_t>(max_ent) * sizeof(BinEnt); }
 };
 
 // The fused combine of the down pass: for each token t this unit completed
@@ -205,12 +196,11 @@ template <bool GU, bool PLANES, bool G64, int FW, int NB>
 __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecParams P) {
   static_assert(!GU || FW == 2, "gate and up fragments");
   using L = Smem<FW, NB>;
-  constexpr int kW = L::kW;
+  constexpr int kSlot = L::kSlot;
   constexpr int kVals = L::kVals;
-  const int kSlot = L::slot(P.xr);
   extern __shared__ __align__(16) uint8_t smem[];
-  float* red = reinterpret_cast<float*>(smem + L::red0(P.xr));
-  BinEnt* ent = reinterpret_cast<BinEnt*>(smem + L::ent0(P.xr));
+  float* red = reinterpret_cast<float*>(smem + L::kRed0);
+  BinEnt* ent = reinterpret_cast<BinEnt*>(smem + L::kEnt0);
   __shared__ int n_ent_s, n_units_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -236,7 +226,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
       }
       const bool ok = nr > 0 && sl >= 0;
       const unsigned m = __ballot_sync(0xffffffffu, ok);
-      const int units = ok ? ((nr + P.xr - 1) / P.xr) * P.row_blocks : 0;
+      const int units = ok ? ((nr + 8 * NB - 1) / (8 * NB)) * P.row_blocks : 0;
       int incl = units;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -267,7 +257,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
   const int n_stages = P.K / kStageK;
   const int G = P.K / P.group;
   const int my_stages = n_stages > warp ? (n_stages - warp + kWarps - 1) / kWarps : 0;
-  const uint32_t ring_u = static_cast<uint32_t>(__cvta_generic_to_shared(smem + warp * (kRing * kSlot)));
+  const uint32_t ring_u = static_cast<uint32_t>(__cvta_generic_to_shared(smem + L::kRing0 + warp * (kRing * kSlot)));
   const int rows_per_unit = GU ? 16 : 16 * FW;
   auto mat = [](int f) { return GU ? f : 0; };
 
@@ -325,32 +315,11 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
     szp = blob + P.sz_off[0] + (static_cast<size_t>(n0 >> 7) * G + ((lane >> 2) & 1)) * 512 + (n0 & 127) * 4 +
           (lane & 3) * 16 + warp * sz_step;
   };
-  // activation rows of unit q: the first of this warp's stages, and how many
-  // token rows the unit has
-  auto xbase = [&](int q, const __half*& xs, int& xn) {
-    int e, pass, rb;
-    locate(blockIdx.x + q * gridDim.x, e, pass, rb);
-    const BinEnt be = ent[e];
-    const int t0 = pass * P.xr;
-    xn = min(P.xr, be.nrows - t0);
-    xs = P.act + static_cast<size_t>(be.row0 + t0) * P.K + warp * kStageK;
-  };
-  // a stage's activation rows (xn rows of 128 K) into ring slot `slot`
-  auto issue_x = [&](uint32_t slot, const __half* xs, int xn) {
-    for (int l = lane; l < xn * 16; l += 32)
-      cp_async16(slot + kW + (l >> 4) * kXRow + (l & 15) * 16, xs + static_cast<size_t>(l >> 4) * P.K + (l & 15) * 8);
-  };
-  const __half* xq = nullptr;  // activation rows of the next copy's stage
-  int xqn = 0;
   // the next stage of the stream into ring slot j % kRing (j = 0, 1, ... in
-  // order), with its activation rows when with_x; past the stream's end an
-  // empty group keeps the count uniform
-  auto issue = [&](int j, bool with_x) {
+  // order); past the stream's end an empty group keeps the count uniform
+  auto issue = [&](int j) {
     if (iq < my_units && my_stages > 0) {
-      if (ii == 0) {
-        bases(iq);
-        if (with_x) xbase(iq, xq, xqn);
-      }
+      if (ii == 0) bases(iq);
       const uint32_t slot = ring_u + (j % kRing) * kSlot;
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
@@ -363,10 +332,6 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
       cp += kWarps * kStep0;
       if (PLANES && dp) dp += kWarps * kStep1;
       szp += kWarps * sz_step;
-      if (with_x) {
-        issue_x(slot, xq, xqn);
-        xq += kWarps * kStageK;
-      }
       if (++ii == my_stages) {
         ii = 0;
         ++iq;
@@ -375,30 +340,11 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
     cp_async_commit();
   };
 
-  // the first kRing stages: weights first (the down pass issues them before
-  // waiting for the gate/up grid, whose h it must not read yet), then their
-  // activation rows as one more group
 #pragma unroll
-  for (int j = 0; j < kRing; ++j) issue(j, false);
+  for (int j = 0; j < kRing; ++j) issue(j);
   if (!GU) {  // down pass: h is read only from here on
     pdl_wait();
     pdl_trigger();
-  }
-  {
-    int q = 0, i = 0;
-    const __half* xs = nullptr;
-    int xn = 0;
-    for (int j = 0; j < kRing && q < my_units && my_stages > 0; ++j) {
-      if (i == 0) xbase(q, xs, xn);
-      issue_x(ring_u + j * kSlot, xs, xn);
-      xs += kWarps * kStageK;
-      if (++i == my_stages) {
-        i = 0;
-        ++q;
-      }
-    }
-    cp_async_commit();
-    if (ii > 0) xq = xs, xqn = xn;  // the stream continues inside the unit of stage kRing - 1
   }
 
   int j = 0;  // stream position of the stage being computed
@@ -406,13 +352,26 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
     int e, pass, rb;
     locate(blockIdx.x + q * gridDim.x, e, pass, rb);
     const BinEnt be = ent[e];
-    const int t0 = pass * P.xr, n0 = rb * rows_per_unit;
-    const int ntok = min(P.xr, be.nrows - t0);  // token rows of this unit
-    // this lane feeds token g of each 8-token block (its 32 elements at
-    // 32 c of the stage's activation rows in the ring slot)
+    const int t0 = pass * 8 * NB, n0 = rb * rows_per_unit;
+    const int ntok = min(8 * NB, be.nrows - t0);  // token rows of this unit
+    // this lane's run of each token row it feeds (token g of each 8-token
+    // block), advanced by one stage of this warp (8 x 128 K) per stage
     bool tok_in[NB];
+    const __half* xp[NB];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) tok_in[nb] = 8 * nb + g < ntok;
+    for (int nb = 0; nb < NB; ++nb) {
+      tok_in[nb] = 8 * nb + g < ntok;
+      xp[nb] = P.act + static_cast<size_t>(be.row0 + t0 + (tok_in[nb] ? 8 * nb + g : 0)) * P.K + warp * kStageK + 32 * c;
+    }
+    // the unit's activation runs into L1 ahead of their use when they fit
+    // (a stage's 128 K of one token row is two 128-byte lines)
+    if (ntok * P.K * 2 <= (48 << 10) && (c & 1) == 0) {
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+        if (tok_in[nb])
+          for (int i = 0; i < my_stages; ++i)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(xp[nb] + i * kWarps * kStageK));
+    }
     float acc[FW][NB][4];
 #pragma unroll
     for (int f = 0; f < FW; ++f)
@@ -421,17 +380,18 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) acc[f][nb][jj] = 0.0f;
     for (int i = 0; i < my_stages; ++i, ++j) {
-      // the first stage also waits for the first stages' activation group
-      if (j == 0) cp_async_wait<0>(); else cp_async_wait<kRing - 1>();
-      __syncwarp();
-      const uint32_t sb = ring_u + (j % kRing) * kSlot;  // this stage's ring slot
-      // activations (4 x 8 elements per token block)
+      // activations (4 x 8 elements per token block), loaded before the wait
       uint4 xv[NB][4];
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
+      for (int nb = 0; nb < NB; ++nb) {
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd)
-          xv[nb][wd] = tok_in[nb] ? lds128(sb + kW + (8 * nb + g) * kXRow + c * 64 + wd * 16) : make_uint4(0, 0, 0, 0);
+          xv[nb][wd] = tok_in[nb] ? ldg_act(xp[nb] + 8 * wd) : make_uint4(0, 0, 0, 0);
+        xp[nb] += kWarps * kStageK;
+      }
+      cp_async_wait<kRing - 1>();
+      __syncwarp();
+      const uint32_t sb = ring_u + (j % kRing) * kSlot;  // this stage's ring slot
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
         const uint32_t fb = sb + f * kFragBytes;
@@ -524,7 +484,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
         }
       }
       __syncwarp();  // every lane is done with ring slot j % kRing
-      issue(j + kRing, true);
+      issue(j + kRing);
     }
     // the unit's partial sums of all warps, added in warp order
 #pragma unroll
@@ -538,8 +498,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
       const int ln = v & 31, nb = (v >> 5) / 4, jj = (v >> 5) & 3;
       const int gg = ln >> 2, cc = ln & 3;
       const int row = gg + 8 * (jj >> 1);               // weight row inside the fragment
-      const int tu = 8 * nb + 2 * cc + (jj & 1);        // token row inside the unit
-      const int tk = t0 + tu;                           // token row inside the bin
+      const int tk = t0 + 8 * nb + 2 * cc + (jj & 1);   // token row inside the bin
       float sum[FW];
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
@@ -547,7 +506,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
         for (int w = 0; w < kWarps; ++w) a += red[(w * kVals + (f * NB + nb) * 4 + jj) * 32 + ln];
         sum[f] = a;
       }
-      if (tu < ntok) {
+      if (tk < be.nrows) {
         const size_t p = static_cast<size_t>(be.row0 + tk);
         if (GU) {
           P.out[p * P.N + n0 + row] = __float2half_rn(silu_f(sum[0]) * sum[1]);
@@ -582,33 +541,29 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
 template <bool GU, bool PLANES, bool G64, int FW, int NB>
 moe_status_t run_dec(const DecParams& p, int units_upper, cudaStream_t s, const char* what) {
   auto kern = k_dec<GU, PLANES, G64, FW, NB>;
-  const size_t smem = Smem<FW, NB>::bytes(p.xr, p.max_ent);
-  // the dynamic shared memory depends on the staged activation rows and on
-  // max_ent: set the opt-in to the largest this variant can need (8 NB rows,
-  // 768 bins), once per device; the grid is the number of CTAs that fit at
-  // once (persistent), found per device and row count
+  const size_t smem = Smem<FW, NB>::bytes(p.max_ent);
+  // the dynamic shared memory depends on max_ent: set the opt-in to the
+  // largest this variant can need (768 bins), once per device; the grid is
+  // the number of CTAs that fit at once (persistent), found per device
   static std::atomic<uint64_t> attr_set{0};
-  static std::atomic<int> resident[64][8 * NB + 1] = {};
+  static int resident[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_check(e, what);
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
-  const size_t smem_max = Smem<FW, NB>::bytes(8 * NB, 768);
+  const size_t smem_max = Smem<FW, NB>::bytes(768);
   if (!bit || !(attr_set.load() & bit)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
     if (e != cudaSuccess) return cuda_check(e, what);
-    attr_set.fetch_or(bit);
-  }
-  int fit = dev < 64 ? resident[dev][p.xr].load() : 0;
-  if (fit <= 0) {
     int per_sm = 0, sms = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarps * 32, Smem<FW, NB>::bytes(p.xr, 256));
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarps * 32, Smem<FW, NB>::bytes(256));
     if (e != cudaSuccess) return cuda_check(e, what);
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_check(e, what);
-    fit = std::max(1, per_sm) * std::max(1, sms);
-    if (dev < 64) resident[dev][p.xr].store(fit);
+    if (dev < 64) resident[dev] = std::max(1, per_sm) * std::max(1, sms);
+    attr_set.fetch_or(bit);
   }
+  const int fit = dev < 64 && resident[dev] > 0 ? resident[dev] : 148;
   const int grid = std::max(1, std::min(units_upper, fit));
   return cuda_check(launch_pdl(true, kern, dim3(grid), dim3(kWarps * 32), smem, s, p), what);
 }
@@ -698,13 +653,8 @@ moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t 
   dn.d4_off[0] = a.lay.d4[2];
   dn.sz_off[0] = a.lay.sz[2];
   const int nb = token_blocks <= 1 ? 1 : 2;
-  // activation rows a unit can have: no bin holds more than T rows
-  gu.xr = std::max(1, std::min(8 * nb, std::min(a.T, a.total_rows)));
-  dn.xr = gu.xr;
-  // passes of xr rows per bin, for the grid size (a bin holds at most T rows
-  // when every token's experts are distinct; the kernel counts the passes of
-  // each bin from its rows, so larger bins are still covered)
-  const int passes = std::max(1, (std::min(a.T, a.total_rows) + gu.xr - 1) / gu.xr);
+  // passes per bin: a bin never holds more than T rows
+  const int passes = std::max(1, (std::min(a.T, a.total_rows) + 8 * nb - 1) / (8 * nb));
   const int sms = sm_count_dec();
   const bool g64 = a.group == 64;
   if (planes)

@@ -26,10 +26,10 @@
 //                   fp64 logits.  Gates are the softmax over the k picked
 //                   logits, in fp64 arithmetic on those values.
 //
-// For the smallest batches (k_route_tiny: T <= 8 and T*E <= 128) the T*E
-// dot products are few enough to take straight in fp64, spread over a
-// thread-block cluster: the selection then runs on the fp64 logits with no
-// bound and no second pass.
+// For the smallest batches (k_route_tiny: T <= 8 and T*E <= 128) both steps
+// run in one launch of a thread-block cluster, each CTA one slice of d; the
+// same fp32-plus-bound scheme with a tighter bound (sums of magnitudes, not
+// norms), and fp64 only for the contenders of tokens it leaves open.
 //
 // Error bound of the fp32 sum: an FMA chain over m products errs by at most
 // g(m) times the sum of their magnitudes; a chunk (32 products) and then the
@@ -469,30 +469,43 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
   select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, blockIdx.x);
 }
 
-// One token of the fp64 cluster paths, by one warp of CTA 0: its logits
-// (slice partials added in slice order, then the bias) into vals (shared),
-// the selection -- top k by rank counting, or the forced ids clamped into
-// range -- into sel (shared, k entries), then the gates (fp64 softmax over
-// the picks: maximum and sum as shuffle trees over the warp) and the ids to
-// global memory.
-__device__ __forceinline__ void tiny_select(const double* part, int n, int t, const float* bias,
-                                            const int32_t* forced, int E, int k, int lane, double* vals,
-                                            int32_t* sel, int32_t* out_idx, float* out_w) {
-  for (int e = lane; e < E; e += 32) {
-    double a = part[t * E + e];
-    for (int r = 1; r < kClusterSlices; ++r) a += part[r * n + t * E + e];
-    vals[e] = a + (bias ? static_cast<double>(bias[e]) : 0.0);
-  }
-  __syncwarp();
-  if (forced) {
-    for (int j = lane; j < k; j += 32) {
-      const int e = forced[static_cast<size_t>(t) * k + j];
-      sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
-    }
-    __syncwarp();
-  } else {
-    warp_topk_rank(vals, E, k, lane, sel);
-  }
+// ---- the smallest batches: one cluster launch -------------------------
+//
+// The router of up to 8 tokens with T*E <= kTinyRouteItems over one
+// thread-block cluster of kClusterSlices CTAs, CTA r taking the d-slice
+// [r d/8, (r+1) d/8) of every (token, expert) dot product:
+//   1. fp32 slice partials S and magnitude sums A (cluster_partial_dots_f32)
+//      into CTA 0's shared memory (DSMEM), cluster barrier;
+//   2. CTA 0, a warp per token: L = sum_r S_r + b in fp64 (exact up to
+//      2^-48 of the magnitudes added), bound
+//        |L - l| <= D = 2 (g(m) sum_r A_r (1 + 2^-8) + 2^-48 (sum_r |S_r| + |b|))
+//      (m = products per lane of a slice + 5; factor 2: margin), top k of L by
+//      rank counting, certified when consecutive picks and the cut after the
+//      k-th are separated by more than their bounds; otherwise the token's
+//      contenders (the picks and every expert whose upper bound reaches the
+//      lowest pick's lower bound) are listed;
+//   3. if any token was not certified (the count is read by every CTA after
+//      a barrier, so all take the same branch): every CTA computes its slice
+//      of the listed dot products in fp64 (each bf16 x fp32 product exact),
+//      CTA 0 selects those tokens again on the fp64 logits.
+// Gates: the fp64 softmax over the picked logits.  The fp64 work is only
+// the contenders': scalar fp64 throughput is a small fraction of fp32.
+struct TinyRouteSmem {
+  float2 p32[kClusterSlices * kTinyRouteItems];  // (S, A) per slice and item t*E + e
+  double p64[kClusterSlices * kTinyRouteItems];  // fp64 partials of the listed items (and, in the
+                                                 // fused kernel, of the width scores)
+  double val[kTinyRouteItems];                   // logits of item t*E + e
+  double dev[kTinyRouteItems];                   // their bounds
+  int32_t cand[kTinyRouteItems];                 // listed items
+  int32_t pos[kTinyRouteItems];                  // item -> index in cand, or -1
+  int32_t n_cand;
+  int32_t unsure[kSelWarps];
+};
+
+// Gates of token t from its logits (vals) at its picks (sel, k entries):
+// fp64 softmax, maximum and sum as shuffle trees; ids and gates to global.
+__device__ __forceinline__ void tiny_gates(const double* vals, const int32_t* sel, int k, int t, int lane,
+                                           int32_t* out_idx, float* out_w) {
   const bool mine = lane < k;
   const int e = mine ? sel[lane] : 0;
   const double lv = mine ? vals[e] : -INFINITY;
@@ -509,38 +522,147 @@ __device__ __forceinline__ void tiny_select(const double* part, int n, int t, co
   }
 }
 
-// The smallest batches (route_tiny_ok: T <= 8, T*E <= 128, d % 64 == 0): the
-// logits straight in fp64 -- no fp32 stage, no bound, no re-evaluation.
-// One cluster of kClusterSlices CTAs, CTA r takes the slice [r d/8, (r+1)
-// d/8) of every (token, expert) dot product (cluster_partial_dots) and
-// stores the partials into CTA 0's shared memory; after the cluster barrier
-// CTA 0's warp t adds token t's partials in slice order and the bias (in
-// fp64) and selects on those logits (tiny_select).
+// Every CTA of the cluster calls this (after cluster_sync_start); CTA 0
+// ends with the picks in sel_s ([T][k], shared) and the outputs written.
+__device__ __forceinline__ void tiny_route(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr,
+                                           const float* __restrict__ bias, const int32_t* __restrict__ forced,
+                                           int T, int d, int E, int k, double gamma, int32_t* out_idx,
+                                           float* out_w, TinyRouteSmem& S, int32_t* sel_s) {
+  const int rank = blockIdx.x;  // the grid is one cluster
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = T * E, dk = d / kClusterSlices;
+  auto rows = [&](int i, const __nv_bfloat16*& xr, const float*& w) {
+    const int t = i / E;
+    xr = x + static_cast<size_t>(t) * d;
+    w = wr + static_cast<size_t>(i - t * E) * d;
+  };
+  if (threadIdx.x == 0) S.n_cand = 0;
+  cluster_partial_dots_f32(n, rank * dk, dk, rows, cluster_map_shared(S.p32, 0) + 8u * static_cast<uint32_t>(rank * n));
+  cluster_sync_publish();
+  // 2. fp32-path logits, selection and certification (CTA 0)
+  if (rank == 0 && warp < T) {
+    const int t = warp;
+    double* val = S.val + t * E;
+    double* dev = S.dev + t * E;
+    int32_t* sel = sel_s + t * k;
+    for (int e = lane; e < E; e += 32) {
+      double L = 0.0, mag = 0.0, sabs = 0.0;
+      for (int r = 0; r < kClusterSlices; ++r) {
+        const float2 p = S.p32[r * n + t * E + e];
+        L += p.x;
+        mag += p.y;
+        sabs += fabs(static_cast<double>(p.x));
+      }
+      const double b = bias ? static_cast<double>(bias[e]) : 0.0;
+      val[e] = L + b;
+      dev[e] = 2.0 * (gamma * mag * (1.0 + 0.00390625) + 3.552713678800501e-15 * (sabs + fabs(b))) + 1e-300;
+      S.pos[t * E + e] = -1;
+    }
+    __syncwarp();
+    bool sure = true;
+    if (forced) {
+      for (int j = lane; j < k; j += 32) {
+        const int e = forced[static_cast<size_t>(t) * k + j];
+        sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
+      }
+      __syncwarp();
+    } else {
+      warp_topk_rank(val, E, k, lane, sel);
+      bool ok = true;
+      double lo = INFINITY;
+      if (lane < k) {
+        const int e = sel[lane];
+        lo = val[e] - dev[e];
+        if (lane > 0) ok = val[sel[lane - 1]] - dev[sel[lane - 1]] > val[e] + dev[e];
+        ok = ok && lo == lo && fabs(lo) <= 1e300;
+      }
+      double lo_min = lo;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) lo_min = fmin(lo_min, __shfl_xor_sync(0xffffffffu, lo_min, o));
+      const double lo_k = __shfl_sync(0xffffffffu, lo, k - 1);
+      for (int e = lane; e < E; e += 32) {
+        bool picked = false;
+        for (int j = 0; j < k; ++j) picked = picked || sel[j] == e;
+        if (!picked) ok = ok && val[e] + dev[e] < lo_k;  // NaN: not certified
+      }
+      sure = __all_sync(0xffffffffu, ok);
+      if (!sure) {  // list the contenders for fp64
+        const bool finite = lo_min == lo_min && fabs(lo_min) <= 1e300;
+        for (int e = lane; e < E; e += 32) {
+          bool picked = false;
+          for (int j = 0; j < k; ++j) picked = picked || sel[j] == e;
+          if (!finite || picked || !(val[e] + dev[e] < lo_min)) {
+            const int p = atomicAdd(&S.n_cand, 1);
+            S.cand[p] = t * E + e;
+            S.pos[t * E + e] = p;
+          }
+        }
+      }
+    }
+    if (lane == 0) S.unsure[t] = sure ? 0 : 1;
+    if (sure) tiny_gates(val, sel, k, t, lane, out_idx, out_w);
+  }
+  cluster_sync_publish();  // the contender list is complete
+  int n3;
+  if (rank == 0) {
+    n3 = S.n_cand;
+  } else {
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(n3) : "r"(cluster_map_shared(&S.n_cand, 0)) : "memory");
+  }
+  if (n3 == 0) return;  // cluster-uniform
+  // 3. fp64 for the listed items
+  if (rank != 0) {
+    const uint32_t c0 = cluster_map_shared(S.cand, 0);
+    for (int i = threadIdx.x; i < n3; i += blockDim.x) {
+      int v;
+      asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(c0 + 4u * i) : "memory");
+      S.cand[i] = v;
+    }
+    __syncthreads();
+  }
+  cluster_partial_dots(
+      n3, rank * dk, dk, [&](int i, const __nv_bfloat16*& xr, const float*& w) { rows(S.cand[i], xr, w); },
+      cluster_map_shared(S.p64, 0) + 8u * static_cast<uint32_t>(rank * n3));
+  cluster_sync_publish();
+  if (rank == 0 && warp < T && S.unsure[warp]) {
+    const int t = warp;
+    double* val = S.val + t * E;
+    int32_t* sel = sel_s + t * k;
+    for (int e = lane; e < E; e += 32) {
+      const int p = S.pos[t * E + e];
+      double v = -INFINITY;
+      if (p >= 0) {
+        v = S.p64[p];
+        for (int r = 1; r < kClusterSlices; ++r) v += S.p64[r * n3 + p];
+        v += bias ? static_cast<double>(bias[e]) : 0.0;
+      }
+      val[e] = v;
+    }
+    __syncwarp();
+    warp_topk_rank(val, E, k, lane, sel);
+    tiny_gates(val, sel, k, t, lane, out_idx, out_w);
+  }
+}
+
+// Bound factor of the fp32 cluster path: g(m), m = products per lane of a
+// d-slice + 5 (tree levels).
+double tiny_gamma(int d) {
+  const double u = std::ldexp(1.0, -24);
+  const double m = 8.0 * ceil_div(d / kClusterSlices, 256) + 5.0;
+  return m * u / (1.0 - m * u);
+}
+
+// The smallest batches (route_tiny_ok: T <= 8, T*E <= 128, d % 64 == 0).
 __global__ void __launch_bounds__(kSelThreads) k_route_tiny(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
-    const int32_t* __restrict__ forced, int T, int d, int E, int k, int32_t* __restrict__ out_idx,
+    const int32_t* __restrict__ forced, int T, int d, int E, int k, double gamma, int32_t* __restrict__ out_idx,
     float* __restrict__ out_w) {
-  __shared__ double part[kClusterSlices * kClusterItems];
-  __shared__ double vals[kTinyRouteItems];
-  __shared__ int32_t sel_s[kSelWarps * 16];
+  __shared__ TinyRouteSmem S;
+  __shared__ int32_t sel_s[kTinyRouteItems];
   pdl_wait();
   pdl_trigger();
   cluster_sync_start();
-  const int rank = blockIdx.x;  // the grid is one cluster
-  const int n = T * E, dk = d / kClusterSlices;
-  cluster_partial_dots(
-      n, rank * dk, dk,
-      [&](int i, const __nv_bfloat16*& xr, const float*& w) {
-        const int t = i / E;
-        xr = x + static_cast<size_t>(t) * d;
-        w = wr + static_cast<size_t>(i - t * E) * d;
-      },
-      cluster_map_shared(part, 0) + 8u * static_cast<uint32_t>(rank * n));
-  cluster_sync_publish();
-  if (rank != 0) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp < T)  // T <= kSelWarps: a warp per token
-    tiny_select(part, n, warp, bias, forced, E, k, lane, vals + warp * E, sel_s + warp * 16, out_idx, out_w);
+  tiny_route(x, wr, bias, forced, T, d, E, k, gamma, out_idx, out_w, S, sel_s);
 }
 
 // ---- router + bit-width gate + permutation in one launch -------------
@@ -550,8 +672,7 @@ __global__ void __launch_bounds__(kSelThreads) k_route_tiny(
 // cluster launch,
 // with the results of k_route_tiny, k_bit_gate_tiny and the permutation
 // kernels (same arithmetic, same order):
-//   1. every CTA: its d-slice of the T*E router dot products (fp64) -> CTA 0
-//   2. CTA 0: logits, selection (or the forced ids), gates; ids to shared
+//   1-2. the router of k_route_tiny (tiny_route); CTA 0 holds the ids
 //   3. with a bit gate: the ids are published to the cluster, every CTA
 //      takes its d-slice of the 3*T*k width scores (fp64) -> CTA 0, which
 //      picks the widths
@@ -578,11 +699,11 @@ struct RoutePermArgs {
   int32_t* inv_perm;
   __half* x_perm;  // null: no gather
   int32_t* status;
+  double gamma;  // bound factor of the router's fp32 path
 };
 
 __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_constant__ RoutePermArgs A) {
-  __shared__ double part[kClusterSlices * kClusterItems];
-  __shared__ double vals[kTinyRouteItems];
+  __shared__ TinyRouteSmem S;
   __shared__ int32_t sel_s[kFusedAssign];
   __shared__ int32_t key_s[kFusedAssign];
   __shared__ int32_t perm_s[kFusedAssign];
@@ -592,24 +713,14 @@ __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_co
   cluster_sync_start();
   const int rank = blockIdx.x;  // the grid is one cluster
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = A.T, d = A.d, E = A.E, k = A.k, n = T * E, na = T * k, dk = d / kClusterSlices;
+  const int T = A.T, d = A.d, E = A.E, k = A.k, na = T * k, dk = d / kClusterSlices;
+  double* part = S.p64;
   const uint32_t part0 = cluster_map_shared(part, 0);
-  // 1. router partials
-  cluster_partial_dots(
-      n, rank * dk, dk,
-      [&](int i, const __nv_bfloat16*& xr, const float*& w) {
-        const int t = i / E;
-        xr = A.x + static_cast<size_t>(t) * d;
-        w = A.wr + static_cast<size_t>(i - t * E) * d;
-      },
-      part0 + 8u * static_cast<uint32_t>(rank * n));
-  cluster_sync_publish();
-  // 2. selection (CTA 0): a warp per token (T <= kSelWarps)
-  if (rank == 0 && warp < T)
-    tiny_select(part, n, warp, A.bias, A.forced, E, k, lane, vals + warp * E, sel_s + warp * k, A.idx, A.gw);
+  // 1-2. router
+  tiny_route(A.x, A.wr, A.bias, A.forced, T, d, E, k, A.gamma, A.idx, A.gw, S, sel_s);
   // 3. bit-width gate
   if (A.wbit) {  // uniform over the cluster
-    cluster_sync_publish();  // CTA 0's ids (sel_s) and its last reads of part are done
+    cluster_sync_publish();  // CTA 0's ids (sel_s) and its last reads of S.p64 are done
     __shared__ int32_t ids_l[kFusedAssign];
     const uint32_t sel0 = cluster_map_shared(sel_s, 0);
     for (int a = threadIdx.x; a < na; a += blockDim.x) {
@@ -780,7 +891,7 @@ moe_status_t launch_route_permute_tiny(const void* x, const float* w_router, con
                                        cudaStream_t s) {
   RoutePermArgs A{static_cast<const __nv_bfloat16*>(x), w_router, bias, forced, bits_in, w_bit, bias_bit,
                   T, d, E, k, idx, w, bits_out, counts, offsets, perm, inv_perm, static_cast<__half*>(x_perm),
-                  status};
+                  status, tiny_gamma(d)};
   return cuda_check(launch_cluster_pdl(k_route_perm_tiny, kClusterSlices, dim3(kSelThreads), 0, s, A),
                     "moe_route_permute cluster launch");
 }
@@ -805,7 +916,7 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
   // the smallest batches: fp64 logits in one cluster launch (no workspace)
   if (route_tiny_ok(T, d, E))
     return cuda_check(launch_cluster_pdl(k_route_tiny, kClusterSlices, dim3(kSelThreads), 0, s, xb, w_router, bias,
-                                         forced, T, d, E, k, idx, w),
+                                         forced, T, d, E, k, tiny_gamma(d), idx, w),
                       "moe_route_topk cluster launch");
   moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, k, splits, ws, s)
                             : launch_logits<64>(xb, w_router, T, d, E, k, splits, ws, s);
