@@ -118,6 +118,9 @@ __device__ __forceinline__ uint32_t cluster_map_shared(const void* p, uint32_t r
                : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(rank));
   return r;
 }
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ void st_cluster_f64(uint32_t addr, double v) {
   asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
 }

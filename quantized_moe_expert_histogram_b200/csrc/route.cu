@@ -602,24 +602,21 @@ __device__ __forceinline__ void tiny_route(const __nv_bfloat16* __restrict__ x, 
     if (lane == 0) S.unsure[t] = sure ? 0 : 1;
     if (sure) tiny_gates(val, sel, k, t, lane, out_idx, out_w);
   }
-  cluster_sync_publish();  // the contender list is complete
-  int n3;
+  // CTA 0 writes the contender count and list into every CTA's shared
+  // memory before the barrier, so that after it no CTA reads another's
+  // shared memory (CTA 0 may have exited by then)
   if (rank == 0) {
-    n3 = S.n_cand;
-  } else {
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(n3) : "r"(cluster_map_shared(&S.n_cand, 0)) : "memory");
+    __syncthreads();  // the list is complete
+    const int nc = S.n_cand;
+    for (int r = 1; r < kClusterSlices; ++r) {
+      for (int i = threadIdx.x; i < nc; i += blockDim.x) st_cluster_u32(cluster_map_shared(&S.cand[i], r), S.cand[i]);
+      if (threadIdx.x == 0) st_cluster_u32(cluster_map_shared(&S.n_cand, r), nc);
+    }
   }
+  cluster_sync_publish();  // the contender list is in every CTA
+  const int n3 = S.n_cand;
   if (n3 == 0) return;  // cluster-uniform
   // 3. fp64 for the listed items
-  if (rank != 0) {
-    const uint32_t c0 = cluster_map_shared(S.cand, 0);
-    for (int i = threadIdx.x; i < n3; i += blockDim.x) {
-      int v;
-      asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(c0 + 4u * i) : "memory");
-      S.cand[i] = v;
-    }
-    __syncthreads();
-  }
   cluster_partial_dots(
       n3, rank * dk, dk, [&](int i, const __nv_bfloat16*& xr, const float*& w) { rows(S.cand[i], xr, w); },
       cluster_map_shared(S.p64, 0) + 8u * static_cast<uint32_t>(rank * n3));
@@ -720,15 +717,15 @@ __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_co
   tiny_route(A.x, A.wr, A.bias, A.forced, T, d, E, k, A.gamma, A.idx, A.gw, S, sel_s);
   // 3. bit-width gate
   if (A.wbit) {  // uniform over the cluster
-    cluster_sync_publish();  // CTA 0's ids (sel_s) and its last reads of S.p64 are done
+    // CTA 0 writes the ids into every CTA's shared memory before the barrier
+    // (no CTA reads another's shared memory after a barrier)
     __shared__ int32_t ids_l[kFusedAssign];
-    const uint32_t sel0 = cluster_map_shared(sel_s, 0);
-    for (int a = threadIdx.x; a < na; a += blockDim.x) {
-      int e;
-      asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(e) : "r"(sel0 + 4u * a) : "memory");
-      ids_l[a] = e;
+    if (rank == 0) {
+      __syncthreads();  // sel_s complete
+      for (int r = 0; r < kClusterSlices; ++r)
+        for (int a = threadIdx.x; a < na; a += blockDim.x) st_cluster_u32(cluster_map_shared(&ids_l[a], r), sel_s[a]);
     }
-    __syncthreads();
+    cluster_sync_publish();  // the ids are in every CTA; CTA 0's last reads of S.p64 are done
     cluster_partial_dots(
         3 * na, rank * dk, dk,
         [&](int i, const __nv_bfloat16*& xr, const float*& w) {
