@@ -77,3 +77,44 @@ def test_ffn_combine_without_residual_and_repeated_experts():
     y_f, yp_f, y_s, yp_s = _run(shape, T, seed=72, forced=forced)
     assert torch.equal(yp_f, yp_s)
     assert torch.equal(y_f, y_s)
+
+
+@pytest.mark.parametrize("T,layout", [(1, "int4"), (8, "int4"), (12, "int4"), (2, "planes")])
+def test_long_rows_split_k_against_oracle_and_slot_path(T, layout):
+    """Rows of the second GEMM long enough (d_ff = 8192: 64 stages of 128) for
+    the decode kernel to split K in four (each split's partial reduced in its
+    CTA, the four added in split order by the split that completes the
+    block): the layer matches the oracle within the bar, and the slot path
+    (the FFN wave by wave over a slot pool) gives the resident path's y_perm
+    bit for bit, since the split depends on the shape alone."""
+    from gpu_helpers import oracle_layer, within_tol
+    shape = I.custom_shape(d=256, E=8, k=2, F=8192, group=128, layout=layout)
+    L = I.make_layer(shape, T, seed=81 + T)
+    layer = QuantMoELayer.from_weights(shape, L["w_router"].cuda(), L["bias"].cuda() if L["bias"] is not None
+                                       else None, L["w_gate"].cuda(), L["w_up"].cuda(), L["w_down"].cuda(),
+                                       max_tokens=T)
+    bits = L["bits"].cuda() if layout == "planes" else None
+    layer.buf["status"].zero_()
+    y = layer.forward(L["x"].cuda(), bits=bits, residual=None).float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert int(layer.buf["status"].item()) == 0
+    ref, _ = oracle_layer(shape, L, bits=None if bits is None else bits.cpu())
+    ok, worst = within_tol(y, ref["y"])
+    assert ok, f"worst err/tol = {worst:.3f}"
+    # the slot path: every expert through a pool of 4 slots, in waves
+    v = layer.views(T)
+    y_res = v["y_perm"].clone()
+    blob = layer.blobs.shape[1]
+    host = layer.blobs.cpu().pin_memory()
+    pool = torch.empty(4, blob, dtype=torch.uint8, device="cuda")
+    planes = (shape.d, shape.F, shape.group) if layout == "planes" else None
+    cache = moeq.SlotCache(shape.E, 4, blob, host, pool, planes=planes)
+    copy, compute = torch.cuda.Stream(), torch.cuda.current_stream()
+    cache.stage(v["topk_idx"].cpu().reshape(-1), copy, compute,
+                bits_host=None if bits is None else bits.cpu().reshape(-1))
+    y_off = torch.empty_like(y_res)
+    cache.ffn(v["x_perm"], v["offsets"], T, shape.d, shape.F, shape.group, layer.layout, v["workspace"], y_off,
+              v["status"], copy, compute)
+    torch.cuda.synchronize()
+    assert torch.equal(y_off, y_res)
+    cache.close()
