@@ -22,10 +22,10 @@
 // three W_bit rows (3 x d fp32) through L2, two 8-element steps of loads in
 // flight per lane.
 //
-// Up to 32 assignments (k_bit_gate_tiny): the 3 T k scores straight in fp64
-// over a thread-block cluster (each CTA one slice of d, partials into CTA
-// 0's shared memory, added in slice order after a cluster barrier), with no
-// bound and no second pass.
+// Up to 32 assignments (k_bit_gate_tiny): the 3 T k scores over a
+// thread-block cluster (each CTA one slice of d, fp32 partials with
+// magnitude sums into CTA 0's shared memory, a tighter per-score bound,
+// fp64 only for the assignments it leaves open; tiny_bit_gate).
 #include <cmath>
 
 #include "common.cuh"
@@ -132,51 +132,25 @@ __global__ void __launch_bounds__(kWarps * 32) k_bit_gate(const __nv_bfloat16* _
   if (lane == 0) bits[a] = static_cast<uint8_t>(2 + best);
 }
 
-constexpr int kTinyAssign = 64;  // shared-memory capacity of the cluster path (3 x 64 scores)
-static_assert(kTinyGateAssign <= kTinyAssign, "cluster bit gate capacity");
-
 __global__ void __launch_bounds__(kWarps * 32) k_bit_gate_tiny(const __nv_bfloat16* __restrict__ x,
                                                               const float* __restrict__ wb,
                                                               const float* __restrict__ bb,
                                                               const int32_t* __restrict__ idx, int T, int d,
-                                                              int E, int k, uint8_t* __restrict__ bits,
+                                                              int E, int k, float gamma, uint8_t* __restrict__ bits,
                                                               int32_t* status) {
-  __shared__ double part[kClusterSlices * 3 * kTinyAssign];
+  __shared__ TinyGateSmem S;
+  __shared__ int32_t ids[kTinyGateAssign];
   pdl_wait();
   pdl_trigger();
   cluster_sync_start();
-  const int rank = blockIdx.x;  // the grid is one cluster
-  const int na = T * k, n = 3 * na, dk = d / kClusterSlices;
-  auto expert = [&](int a) {
-    const int e = idx[a];
-    return e < 0 ? 0 : (e >= E ? E - 1 : e);
-  };
-  cluster_partial_dots(
-      n, rank * dk, dk,
-      [&](int i, const __nv_bfloat16*& xr, const float*& w) {
-        const int a = i / 3;
-        xr = x + static_cast<size_t>(a / k) * d;
-        w = wb + (static_cast<size_t>(expert(a)) * 3 + (i - 3 * a)) * d;
-      },
-      cluster_map_shared(part, 0) + 8u * static_cast<uint32_t>(rank * n));
-  cluster_sync_publish();
-  if (rank != 0) return;
+  const int na = T * k;
   for (int a = threadIdx.x; a < na; a += blockDim.x) {
-    const int raw = idx[a];
-    if (raw < 0 || raw >= E) flag_status(status, MOE_DEV_BAD_INDEX);
-    const int e = expert(a);
-    double v[3];
-#pragma unroll
-    for (int c = 0; c < 3; ++c) {
-      double s = part[3 * a + c];
-      for (int r = 1; r < kClusterSlices; ++r) s += part[r * n + 3 * a + c];
-      v[c] = s + (bb ? static_cast<double>(bb[static_cast<size_t>(e) * 3 + c]) : 0.0);
-    }
-    int best = 0;
-    if (v[1] > v[best]) best = 1;
-    if (v[2] > v[best]) best = 2;
-    bits[a] = static_cast<uint8_t>(2 + best);
+    const int e = idx[a];
+    if ((e < 0 || e >= E) && blockIdx.x == 0) flag_status(status, MOE_DEV_BAD_INDEX);
+    ids[a] = e < 0 ? 0 : (e >= E ? E - 1 : e);
   }
+  __syncthreads();
+  tiny_bit_gate(x, wb, bb, ids, T, d, k, gamma, bits, nullptr, S);
 }
 
 }  // namespace
@@ -190,7 +164,7 @@ moe_status_t launch_bit_gate(const void* x, const float* w_bit, const float* bia
   if (g_route_fused == 1 && T * k <= kTinyGateAssign && d % (8 * kClusterSlices) == 0)
     return cuda_check(launch_cluster_pdl(k_bit_gate_tiny, kClusterSlices, dim3(kWarps * 32), 0, s,
                                          static_cast<const __nv_bfloat16*>(x), w_bit, bias_bit, idx, T, d, E, k,
-                                         bits, status),
+                                         cluster_gamma(d), bits, status),
                       "moe_bit_gate cluster launch");
   const double u = std::ldexp(1.0, -24);
   const double m = ceil_div(d, 256) * 8 + 5;

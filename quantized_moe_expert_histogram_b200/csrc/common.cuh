@@ -269,22 +269,23 @@ __device__ __forceinline__ void cluster_partial_dots_f32(int n, int k0, int dk, 
   }
 }
 
-// The k largest of E fp64 values in shared memory, in descending order,
+// The k largest of E values in shared memory, in descending order,
 // ties to the lower index, by one warp: each lane ranks its values
 // e = lane + 32 m against all E (independent compares, no dependent
 // chains) and the value of rank r < k writes its index to sel[r] (shared
 // memory).  NaN values are never picked; if fewer than k values are
 // comparable the remaining picks are expert 0 (the selection order of the
 // warp-shuffle top-k, which takes the first maximum k times).
-__device__ __forceinline__ void warp_topk_rank(const double* vals, int E, int k, int lane, int32_t* sel) {
+template <typename V>
+__device__ __forceinline__ void warp_topk_rank(const V* vals, int E, int k, int lane, int32_t* sel) {
   int comparable = 0;
   for (int e = lane; e < E; e += 32) {
-    const double v = vals[e];
+    const V v = vals[e];
     comparable += v == v ? 1 : 0;
     if (v != v) continue;
     int rank = 0;
     for (int o = 0; o < E; ++o) {
-      const double u = vals[o];  // NaN: both compares false
+      const V u = vals[o];  // NaN: both compares false
       rank += (u > v || (u == v && o < e)) ? 1 : 0;
     }
     if (rank < k) sel[rank] = e;
@@ -293,6 +294,115 @@ __device__ __forceinline__ void warp_topk_rank(const double* vals, int E, int k,
   for (int o = 16; o; o >>= 1) comparable += __shfl_xor_sync(0xffffffffu, comparable, o);
   for (int r = comparable + lane; r < k; r += 32) sel[r] = 0;
   __syncwarp();
+}
+
+// Bound factor of the fp32 cluster paths: g(m + 9), m = products per lane
+// of a d-slice + 5 (tree levels); + 8 for the sum over the slices and 1 for
+// the bias.
+inline float cluster_gamma(int d) {
+  const double u = 1.0 / 16777216.0;
+  const double m = 8.0 * ((d / kClusterSlices + 255) / 256) + 5.0 + 9.0;
+  return static_cast<float>(m * u / (1.0 - m * u));
+}
+
+// The bit-width gate of the smallest batches over one cluster (every CTA
+// calls it after cluster_sync_start): the 3 T k width scores as fp32 slice
+// partials with magnitude sums (cluster_partial_dots_f32) into CTA 0, which
+// picks each assignment's width (first maximum, equal scores to the narrower
+// width) when the winner's lower bound clears the others' upper bounds,
+//   |L[c] - l[c]| <= D[c] = 2 g (A[c] (1 + 2^-8) + |b[c]|),  g = cluster_gamma(d);
+// the assignments it leaves open are listed (CTA 0 writes the list into
+// every CTA before the barrier), their scores recomputed in fp64 over the
+// cluster and decided on those.  ids: the assignments' experts, in range,
+// readable by every CTA.  Widths to bits (global) and, if given, bits_s
+// (CTA 0's shared memory).
+struct TinyGateSmem {
+  float2 p32[kClusterSlices * 3 * 32];
+  double p64[kClusterSlices * 3 * 32];
+  int32_t cand[32];
+  int32_t n_cand;
+};
+__device__ __forceinline__ void tiny_bit_gate(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wb,
+                                              const float* __restrict__ bb, const int32_t* ids, int T, int d,
+                                              int k, float gamma, uint8_t* bits, uint8_t* bits_s,
+                                              TinyGateSmem& S) {
+  const int rank = blockIdx.x;  // the grid is one cluster
+  const int na = T * k, n = 3 * na, dk = d / kClusterSlices;
+  if (threadIdx.x == 0) S.n_cand = 0;
+  cluster_partial_dots_f32(
+      n, rank * dk, dk,
+      [&](int i, const __nv_bfloat16*& xr, const float*& w) {
+        const int a = i / 3;
+        xr = x + static_cast<size_t>(a / k) * d;
+        w = wb + (static_cast<size_t>(ids[a]) * 3 + (i - 3 * a)) * d;
+      },
+      cluster_map_shared(S.p32, 0) + 8u * static_cast<uint32_t>(rank * n));
+  cluster_sync_publish();
+  if (rank == 0) {
+    for (int a = threadIdx.x; a < na; a += blockDim.x) {
+      float L[3], D[3];
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        float s = 0.0f, m = 0.0f;
+        for (int r = 0; r < kClusterSlices; ++r) {
+          const float2 p = S.p32[r * n + 3 * a + c];
+          s += p.x;
+          m += p.y;
+        }
+        const float b = bb ? bb[static_cast<size_t>(ids[a]) * 3 + c] : 0.0f;
+        L[c] = s + b;
+        D[c] = 2.0f * gamma * (m * (1.0f + 0.00390625f) + fabsf(b)) + 1e-30f;
+      }
+      int best = 0;
+      if (L[1] > L[best]) best = 1;
+      if (L[2] > L[best]) best = 2;
+      bool sure = true;  // comparisons with NaN are false: non-finite scores go to fp64
+#pragma unroll
+      for (int c = 0; c < 3; ++c)
+        if (c != best) sure = sure && L[best] - D[best] > L[c] + D[c];
+      if (sure) {
+        bits[a] = static_cast<uint8_t>(2 + best);
+        if (bits_s) bits_s[a] = static_cast<uint8_t>(2 + best);
+      } else {
+        S.cand[atomicAdd(&S.n_cand, 1)] = a;
+      }
+    }
+    __syncthreads();  // the list is complete
+    const int nc = S.n_cand;
+    for (int r = 1; r < kClusterSlices; ++r) {
+      for (int i = threadIdx.x; i < nc; i += blockDim.x) st_cluster_u32(cluster_map_shared(&S.cand[i], r), S.cand[i]);
+      if (threadIdx.x == 0) st_cluster_u32(cluster_map_shared(&S.n_cand, r), nc);
+    }
+  }
+  cluster_sync_publish();  // the list is in every CTA
+  const int n3 = S.n_cand;
+  if (n3 == 0) return;  // cluster-uniform
+  cluster_partial_dots(
+      3 * n3, rank * dk, dk,
+      [&](int i, const __nv_bfloat16*& xr, const float*& w) {
+        const int a = S.cand[i / 3];
+        xr = x + static_cast<size_t>(a / k) * d;
+        w = wb + (static_cast<size_t>(ids[a]) * 3 + (i - 3 * (i / 3))) * d;
+      },
+      cluster_map_shared(S.p64, 0) + 8u * static_cast<uint32_t>(rank * 3 * n3));
+  cluster_sync_publish();
+  if (rank == 0) {
+    for (int j = threadIdx.x; j < n3; j += blockDim.x) {
+      const int a = S.cand[j];
+      double v[3];
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        double s = S.p64[3 * j + c];
+        for (int r = 1; r < kClusterSlices; ++r) s += S.p64[r * 3 * n3 + 3 * j + c];
+        v[c] = s + (bb ? static_cast<double>(bb[static_cast<size_t>(ids[a]) * 3 + c]) : 0.0);
+      }
+      int best = 0;
+      if (v[1] > v[best]) best = 1;
+      if (v[2] > v[best]) best = 2;
+      bits[a] = static_cast<uint8_t>(2 + best);
+      if (bits_s) bits_s[a] = static_cast<uint8_t>(2 + best);
+    }
+  }
 }
 
 // A launch of one thread-block cluster of `cluster` CTAs (grid = cluster),
@@ -325,8 +435,9 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
                           float* w, void* workspace, size_t workspace_bytes, cudaStream_t s);
 size_t route_workspace_bytes(int T, int d, int E);
 extern int g_route_fused;  // test hook: 1 default, 0 no fp64 cluster paths
-constexpr int kTinyRouteItems = 128;  // router dot products of the fp64 cluster path (T*E)
-constexpr int kTinyGateAssign = 32;   // assignments of the fp64 cluster bit gate (T*k)
+constexpr int kTinyRouteItems = 128;  // router dot products of the cluster path (T*E)
+constexpr int kTinyGateAssign = 32;   // assignments of the cluster bit gate (T*k)
+static_assert(kTinyGateAssign <= 32, "TinyGateSmem holds 32 assignments");
 bool route_tiny_ok(int T, int d, int E);
 bool route_permute_fusable(int T, int d, int E, int k, bool gate);
 moe_status_t launch_route_permute_tiny(const void* x, const float* w_router, const float* bias,

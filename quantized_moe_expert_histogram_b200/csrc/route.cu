@@ -476,26 +476,29 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
 // [r d/8, (r+1) d/8) of every (token, expert) dot product:
 //   1. fp32 slice partials S and magnitude sums A (cluster_partial_dots_f32)
 //      into CTA 0's shared memory (DSMEM), cluster barrier;
-//   2. CTA 0, a warp per token: L = sum_r S_r + b in fp64 (exact up to
-//      2^-48 of the magnitudes added), bound
-//        |L - l| <= D = 2 (g(m) sum_r A_r (1 + 2^-8) + 2^-48 (sum_r |S_r| + |b|))
-//      (m = products per lane of a slice + 5; factor 2: margin), top k of L by
-//      rank counting, certified when consecutive picks and the cut after the
-//      k-th are separated by more than their bounds; otherwise the token's
-//      contenders (the picks and every expert whose upper bound reaches the
-//      lowest pick's lower bound) are listed;
+//   2. CTA 0, a warp per token: L = (sum_r S_r) + b and A = sum_r A_r in
+//      fp32 (8 more additions: |L - l| <= g(m) A + g(8) (sum_r |S_r| + |b|)),
+//      bound D = 2 g(m + 9) (A (1 + 2^-8) + |b|) (m = products per lane of a
+//      slice + 5; factor 2: margin), top k of L by rank counting, certified
+//      when consecutive picks and the cut after the k-th are separated by
+//      more than their bounds; otherwise the token's contenders (the picks
+//      and every expert whose upper bound reaches the lowest pick's lower
+//      bound) are listed;
 //   3. if any token was not certified (the count is read by every CTA after
 //      a barrier, so all take the same branch): every CTA computes its slice
 //      of the listed dot products in fp64 (each bf16 x fp32 product exact),
 //      CTA 0 selects those tokens again on the fp64 logits.
-// Gates: the fp64 softmax over the picked logits.  The fp64 work is only
-// the contenders': scalar fp64 throughput is a small fraction of fp32.
+// Gates: the softmax over the picked logits (fp32 for certified tokens,
+// fp64 for re-evaluated ones).  No fp64 arithmetic runs unless a token is
+// left open: measured on B200, scalar fp64 throughput is a small fraction
+// of fp32 and bounded an all-fp64 version of this router.
 struct TinyRouteSmem {
   float2 p32[kClusterSlices * kTinyRouteItems];  // (S, A) per slice and item t*E + e
   double p64[kClusterSlices * kTinyRouteItems];  // fp64 partials of the listed items (and, in the
                                                  // fused kernel, of the width scores)
-  double val[kTinyRouteItems];                   // logits of item t*E + e
-  double dev[kTinyRouteItems];                   // their bounds
+  float val[kTinyRouteItems];                    // fp32-path logits of item t*E + e
+  float dev[kTinyRouteItems];                    // their bounds
+  double val64[kTinyRouteItems];                 // fp64 logits of re-evaluated tokens
   int32_t cand[kTinyRouteItems];                 // listed items
   int32_t pos[kTinyRouteItems];                  // item -> index in cand, or -1
   int32_t n_cand;
@@ -503,17 +506,19 @@ struct TinyRouteSmem {
 };
 
 // Gates of token t from its logits (vals) at its picks (sel, k entries):
-// fp64 softmax, maximum and sum as shuffle trees; ids and gates to global.
-__device__ __forceinline__ void tiny_gates(const double* vals, const int32_t* sel, int k, int t, int lane,
+// softmax in the logits' precision, maximum and sum as shuffle trees; ids
+// and gates to global.
+template <typename V>
+__device__ __forceinline__ void tiny_gates(const V* vals, const int32_t* sel, int k, int t, int lane,
                                            int32_t* out_idx, float* out_w) {
   const bool mine = lane < k;
   const int e = mine ? sel[lane] : 0;
-  const double lv = mine ? vals[e] : -INFINITY;
-  double mx = lv;
+  const V lv = mine ? vals[e] : static_cast<V>(-INFINITY);
+  V mx = lv;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  const double ex = mine ? exp(lv - mx) : 0.0;
-  double sum = ex;
+  for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const V ex = mine ? exp(lv - mx) : static_cast<V>(0);
+  V sum = ex;
 #pragma unroll
   for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (mine) {
@@ -526,7 +531,7 @@ __device__ __forceinline__ void tiny_gates(const double* vals, const int32_t* se
 // ends with the picks in sel_s ([T][k], shared) and the outputs written.
 __device__ __forceinline__ void tiny_route(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr,
                                            const float* __restrict__ bias, const int32_t* __restrict__ forced,
-                                           int T, int d, int E, int k, double gamma, int32_t* out_idx,
+                                           int T, int d, int E, int k, float gamma, int32_t* out_idx,
                                            float* out_w, TinyRouteSmem& S, int32_t* sel_s) {
   const int rank = blockIdx.x;  // the grid is one cluster
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -542,20 +547,19 @@ __device__ __forceinline__ void tiny_route(const __nv_bfloat16* __restrict__ x, 
   // 2. fp32-path logits, selection and certification (CTA 0)
   if (rank == 0 && warp < T) {
     const int t = warp;
-    double* val = S.val + t * E;
-    double* dev = S.dev + t * E;
+    float* val = S.val + t * E;
+    float* dev = S.dev + t * E;
     int32_t* sel = sel_s + t * k;
     for (int e = lane; e < E; e += 32) {
-      double L = 0.0, mag = 0.0, sabs = 0.0;
+      float L = 0.0f, mag = 0.0f;
       for (int r = 0; r < kClusterSlices; ++r) {
         const float2 p = S.p32[r * n + t * E + e];
         L += p.x;
         mag += p.y;
-        sabs += fabs(static_cast<double>(p.x));
       }
-      const double b = bias ? static_cast<double>(bias[e]) : 0.0;
+      const float b = bias ? bias[e] : 0.0f;
       val[e] = L + b;
-      dev[e] = 2.0 * (gamma * mag * (1.0 + 0.00390625) + 3.552713678800501e-15 * (sabs + fabs(b))) + 1e-300;
+      dev[e] = 2.0f * gamma * (mag * (1.0f + 0.00390625f) + fabsf(b)) + 1e-30f;
       S.pos[t * E + e] = -1;
     }
     __syncwarp();
@@ -569,17 +573,17 @@ __device__ __forceinline__ void tiny_route(const __nv_bfloat16* __restrict__ x, 
     } else {
       warp_topk_rank(val, E, k, lane, sel);
       bool ok = true;
-      double lo = INFINITY;
+      float lo = INFINITY;
       if (lane < k) {
         const int e = sel[lane];
         lo = val[e] - dev[e];
         if (lane > 0) ok = val[sel[lane - 1]] - dev[sel[lane - 1]] > val[e] + dev[e];
-        ok = ok && lo == lo && fabs(lo) <= 1e300;
+        ok = ok && lo == lo && fabsf(lo) <= 3.0e38f;
       }
-      double lo_min = lo;
+      float lo_min = lo;
 #pragma unroll
-      for (int o = 16; o; o >>= 1) lo_min = fmin(lo_min, __shfl_xor_sync(0xffffffffu, lo_min, o));
-      const double lo_k = __shfl_sync(0xffffffffu, lo, k - 1);
+      for (int o = 16; o; o >>= 1) lo_min = fminf(lo_min, __shfl_xor_sync(0xffffffffu, lo_min, o));
+      const float lo_k = __shfl_sync(0xffffffffu, lo, k - 1);
       for (int e = lane; e < E; e += 32) {
         bool picked = false;
         for (int j = 0; j < k; ++j) picked = picked || sel[j] == e;
@@ -587,7 +591,7 @@ __device__ __forceinline__ void tiny_route(const __nv_bfloat16* __restrict__ x, 
       }
       sure = __all_sync(0xffffffffu, ok);
       if (!sure) {  // list the contenders for fp64
-        const bool finite = lo_min == lo_min && fabs(lo_min) <= 1e300;
+        const bool finite = lo_min == lo_min && fabsf(lo_min) <= 3.0e38f;
         for (int e = lane; e < E; e += 32) {
           bool picked = false;
           for (int j = 0; j < k; ++j) picked = picked || sel[j] == e;
@@ -623,7 +627,7 @@ __device__ __forceinline__ void tiny_route(const __nv_bfloat16* __restrict__ x, 
   cluster_sync_publish();
   if (rank == 0 && warp < T && S.unsure[warp]) {
     const int t = warp;
-    double* val = S.val + t * E;
+    double* val = S.val64 + t * E;
     int32_t* sel = sel_s + t * k;
     for (int e = lane; e < E; e += 32) {
       const int p = S.pos[t * E + e];
@@ -641,18 +645,10 @@ __device__ __forceinline__ void tiny_route(const __nv_bfloat16* __restrict__ x, 
   }
 }
 
-// Bound factor of the fp32 cluster path: g(m), m = products per lane of a
-// d-slice + 5 (tree levels).
-double tiny_gamma(int d) {
-  const double u = std::ldexp(1.0, -24);
-  const double m = 8.0 * ceil_div(d / kClusterSlices, 256) + 5.0;
-  return m * u / (1.0 - m * u);
-}
-
 // The smallest batches (route_tiny_ok: T <= 8, T*E <= 128, d % 64 == 0).
 __global__ void __launch_bounds__(kSelThreads) k_route_tiny(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
-    const int32_t* __restrict__ forced, int T, int d, int E, int k, double gamma, int32_t* __restrict__ out_idx,
+    const int32_t* __restrict__ forced, int T, int d, int E, int k, float gamma, int32_t* __restrict__ out_idx,
     float* __restrict__ out_w) {
   __shared__ TinyRouteSmem S;
   __shared__ int32_t sel_s[kTinyRouteItems];
@@ -670,9 +666,8 @@ __global__ void __launch_bounds__(kSelThreads) k_route_tiny(
 // with the results of k_route_tiny, k_bit_gate_tiny and the permutation
 // kernels (same arithmetic, same order):
 //   1-2. the router of k_route_tiny (tiny_route); CTA 0 holds the ids
-//   3. with a bit gate: the ids are published to the cluster, every CTA
-//      takes its d-slice of the 3*T*k width scores (fp64) -> CTA 0, which
-//      picks the widths
+//   3. with a bit gate: the ids are published to the cluster, then the bit
+//      gate of k_bit_gate_tiny (tiny_bit_gate)
 //   4. CTA 0: keys (expert, or 3 expert + width - 2), stable ranks by
 //      counting (ties in ascending assignment), counts, offsets, perm,
 //      inv_perm, and the gather of x_perm (fp16) in expert order.
@@ -696,11 +691,12 @@ struct RoutePermArgs {
   int32_t* inv_perm;
   __half* x_perm;  // null: no gather
   int32_t* status;
-  double gamma;  // bound factor of the router's fp32 path
+  float gamma;  // bound factor of the router's fp32 path
 };
 
 __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_constant__ RoutePermArgs A) {
   __shared__ TinyRouteSmem S;
+  __shared__ TinyGateSmem G;
   __shared__ int32_t sel_s[kFusedAssign];
   __shared__ int32_t key_s[kFusedAssign];
   __shared__ int32_t perm_s[kFusedAssign];
@@ -711,8 +707,6 @@ __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_co
   const int rank = blockIdx.x;  // the grid is one cluster
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = A.T, d = A.d, E = A.E, k = A.k, na = T * k, dk = d / kClusterSlices;
-  double* part = S.p64;
-  const uint32_t part0 = cluster_map_shared(part, 0);
   // 1-2. router
   tiny_route(A.x, A.wr, A.bias, A.forced, T, d, E, k, A.gamma, A.idx, A.gw, S, sel_s);
   // 3. bit-width gate
@@ -725,33 +719,8 @@ __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_co
       for (int r = 0; r < kClusterSlices; ++r)
         for (int a = threadIdx.x; a < na; a += blockDim.x) st_cluster_u32(cluster_map_shared(&ids_l[a], r), sel_s[a]);
     }
-    cluster_sync_publish();  // the ids are in every CTA; CTA 0's last reads of S.p64 are done
-    cluster_partial_dots(
-        3 * na, rank * dk, dk,
-        [&](int i, const __nv_bfloat16*& xr, const float*& w) {
-          const int a = i / 3;
-          xr = A.x + static_cast<size_t>(a / k) * d;
-          w = A.wbit + (static_cast<size_t>(ids_l[a]) * 3 + (i - 3 * a)) * d;
-        },
-        part0 + 8u * static_cast<uint32_t>(rank * 3 * na));
-    cluster_sync_publish();
-    if (rank == 0) {
-      for (int a = threadIdx.x; a < na; a += blockDim.x) {
-        const int e = sel_s[a];
-        double v[3];
-#pragma unroll
-        for (int c = 0; c < 3; ++c) {
-          double s = part[3 * a + c];
-          for (int r = 1; r < kClusterSlices; ++r) s += part[r * 3 * na + 3 * a + c];
-          v[c] = s + (A.bbit ? static_cast<double>(A.bbit[static_cast<size_t>(e) * 3 + c]) : 0.0);
-        }
-        int best = 0;
-        if (v[1] > v[best]) best = 1;
-        if (v[2] > v[best]) best = 2;
-        bits_s[a] = static_cast<uint8_t>(2 + best);
-        A.bits_out[a] = static_cast<uint8_t>(2 + best);
-      }
-    }
+    cluster_sync_publish();  // the ids are in every CTA; CTA 0's last reads of S are done
+    tiny_bit_gate(A.x, A.wbit, A.bbit, ids_l, T, d, k, A.gamma, A.bits_out, bits_s, G);
   }
   if (rank != 0) return;
   __syncthreads();  // sel_s, bits_s complete
@@ -888,7 +857,7 @@ moe_status_t launch_route_permute_tiny(const void* x, const float* w_router, con
                                        cudaStream_t s) {
   RoutePermArgs A{static_cast<const __nv_bfloat16*>(x), w_router, bias, forced, bits_in, w_bit, bias_bit,
                   T, d, E, k, idx, w, bits_out, counts, offsets, perm, inv_perm, static_cast<__half*>(x_perm),
-                  status, tiny_gamma(d)};
+                  status, cluster_gamma(d)};
   return cuda_check(launch_cluster_pdl(k_route_perm_tiny, kClusterSlices, dim3(kSelThreads), 0, s, A),
                     "moe_route_permute cluster launch");
 }
@@ -913,7 +882,7 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
   // the smallest batches: fp64 logits in one cluster launch (no workspace)
   if (route_tiny_ok(T, d, E))
     return cuda_check(launch_cluster_pdl(k_route_tiny, kClusterSlices, dim3(kSelThreads), 0, s, xb, w_router, bias,
-                                         forced, T, d, E, k, tiny_gamma(d), idx, w),
+                                         forced, T, d, E, k, cluster_gamma(d), idx, w),
                       "moe_route_topk cluster launch");
   moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, k, splits, ws, s)
                             : launch_logits<64>(xb, w_router, T, d, E, k, splits, ws, s);
