@@ -276,8 +276,11 @@ moe_status_t moe_route_permute(const void* x, const float* w_router, const float
 }
 
 size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int layout) {
+  (void)E;
+  (void)d;
+  (void)layout;
   if (total_rows < 0 || F <= 0) return 0;
-  return workspace_for(total_rows, F) + decode_split_bytes(total_rows, E, d, F, layout);
+  return workspace_for(total_rows, F);
 }
 
 moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, const void* blobs,
@@ -330,9 +333,6 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   a.h = static_cast<__half*>(workspace);
   a.y_perm = static_cast<__half*>(y_perm);
   a.status = status;
-  const size_t hbytes = workspace_for(total_rows, F);
-  a.split_ws = static_cast<uint8_t*>(workspace) + hbytes;
-  a.split_bytes = workspace_bytes - hbytes;
   const bool tc_ok = total_rows >= 16 && tc_supported(a);
   int regime = g_force_regime;
   if (regime == 0) regime = T <= kDecMaxT || !tc_ok ? (T <= 8 ? 1 : 3) : 2;
@@ -347,8 +347,7 @@ size_t moe_ffn_combine_workspace_bytes(int T, int k, int E, int d, int F, int la
   (void)E;
   (void)layout;
   if (T <= 0 || k <= 0 || d <= 0 || F <= 0) return 256;
-  return workspace_for(T * k, F) + ((static_cast<size_t>(T) * (d / 16) * sizeof(int32_t) + 255) & ~size_t(255)) +
-         decode_split_bytes(T * k, E, d, F, layout);
+  return workspace_for(T * k, F) + ((static_cast<size_t>(T) * (d / 16) * sizeof(int32_t) + 255) & ~size_t(255));
 }
 
 moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets, const void* blobs, int T, int k,
@@ -420,9 +419,6 @@ moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets,
     a.residual = static_cast<const __nv_bfloat16*>(residual);
     a.y = static_cast<__nv_bfloat16*>(y);
     a.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + hbytes);
-    const size_t cbytes = (static_cast<size_t>(T) * (d / 16) * sizeof(int32_t) + 255) & ~size_t(255);
-    a.split_ws = static_cast<uint8_t*>(workspace) + hbytes + cbytes;
-    a.split_bytes = workspace_bytes - hbytes - cbytes;
     return launch_ffn_decode(a, regime == 1 ? 1 : 2, S(stream));
   }
   moe_status_t st = moe_grouped_ffn_wq(x_perm, offsets, blobs, nullptr, total_rows, T, E, d, F, group, layout,

@@ -476,14 +476,7 @@ struct FfnArgs {
   const __nv_bfloat16* residual = nullptr;
   __nv_bfloat16* y = nullptr;
   int32_t* counters = nullptr;  // workspace: int32 [T][d/16]
-  // workspace of the decode kernel's split-K down pass (see decode_split_bytes)
-  uint8_t* split_ws = nullptr;
-  size_t split_bytes = 0;
 };
-// Splits of K for the decode kernel's down pass (long rows only), and the
-// workspace they need for total_rows rows (0 when no split applies).
-int decode_split_for(int K);
-size_t decode_split_bytes(int total_rows, int E, int d, int F, int layout);
 moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);
 moe_status_t launch_ffn_gemv_mma(const FfnArgs& a, cudaStream_t s);
 moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t s);

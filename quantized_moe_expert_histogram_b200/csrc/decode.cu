@@ -81,13 +81,6 @@ struct DecParams {
   __nv_bfloat16* y;
   int32_t* counters;
   int n_counters;           // gate/up pass: counters to zero
-  // split K (down pass of long rows): a unit covers 1/ksplit of K; its
-  // CTA-reduced partial goes to kpart, and the split that completes a
-  // (bin, pass, row block) adds the ksplit partials in split order
-  int ksplit;
-  float* kpart;             // [units / ksplit][ksplit][FW * NB * 128]
-  int32_t* kcnt;            // [units / ksplit], zeroed by the gate/up pass
-  int n_kcnt;               // gate/up pass: kcnt entries to zero
 };
 
 // One listed bin: its rows, blob, width and its first work unit.
@@ -218,7 +211,6 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
     // them only after this grid has completed)
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P.n_counters; i += gridDim.x * blockDim.x)
       P.counters[i] = 0;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P.n_kcnt; i += gridDim.x * blockDim.x) P.kcnt[i] = 0;
   }
   // ---- the non-empty, resident bins and their work units (warp 0): units
   // of a bin = passes x row blocks, passes = ceil(rows / (8 NB))
@@ -234,7 +226,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
       }
       const bool ok = nr > 0 && sl >= 0;
       const unsigned m = __ballot_sync(0xffffffffu, ok);
-      const int units = ok ? ((nr + 8 * NB - 1) / (8 * NB)) * P.row_blocks * P.ksplit : 0;
+      const int units = ok ? ((nr + 8 * NB - 1) / (8 * NB)) * P.row_blocks : 0;
       int incl = units;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -262,7 +254,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
     if (!GU) pdl_wait();  // CTA-uniform; keeps the wait/trigger order of every CTA
     return;
   }
-  const int n_stages = P.K / kStageK / P.ksplit;  // stages of one unit (one split of K)
+  const int n_stages = P.K / kStageK;
   const int G = P.K / P.group;
   const int my_stages = n_stages > warp ? (n_stages - warp + kWarps - 1) / kWarps : 0;
   const uint32_t ring_u = static_cast<uint32_t>(__cvta_generic_to_shared(smem + L::kRing0 + warp * (kRing * kSlot)));
@@ -270,7 +262,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
   auto mat = [](int f) { return GU ? f : 0; };
 
   // unit u -> (listed bin, pass, row block)
-  auto locate = [&](int u, int& e, int& pass, int& rb, int& ks) {
+  auto locate = [&](int u, int& e, int& pass, int& rb) {
     int lo = 0, hi = n_ent;  // largest e with ent[e].unit0 <= u
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -278,10 +270,8 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
     }
     e = lo;
     const int local = u - ent[lo].unit0;
-    ks = local % P.ksplit;
-    const int r2 = local / P.ksplit;
-    pass = r2 / P.row_blocks;
-    rb = r2 - pass * P.row_blocks;
+    pass = local / P.row_blocks;
+    rb = local - pass * P.row_blocks;
   };
 
   // ---- copy side: this warp's stream of stages, unit by unit.  Per
@@ -308,23 +298,22 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
   int iq = 0, ii = 0;  // unit (of this CTA) and stage (of this warp) of the next copy
   // copy bases of this warp's first stage of unit q
   auto bases = [&](int q) {
-    int e, pass, rb, ks;
-    locate(blockIdx.x + q * gridDim.x, e, pass, rb, ks);
+    int e, pass, rb;
+    locate(blockIdx.x + q * gridDim.x, e, pass, rb);
     const BinEnt be = ent[e];
     const uint8_t* blob = P.blobs + static_cast<size_t>(be.slot) * P.blob_bytes;
     const int n0 = rb * rows_per_unit;
-    const int s0 = ks * n_stages + warp;  // this warp's first stage of K
     if (!PLANES) {
-      cp = blob + P.code_off[0] + static_cast<size_t>(n0 + (lane >> 2)) * (P.K / 2) + (lane & 3) * 16 + s0 * kStep0;
+      cp = blob + P.code_off[0] + static_cast<size_t>(n0 + (lane >> 2)) * (P.K / 2) + (lane & 3) * 16 + warp * kStep0;
     } else {
-      cp = blob + P.code_off[0] + static_cast<size_t>(n0 + (lane >> 1)) * (P.K / 4) + (lane & 1) * 16 + s0 * kStep0;
+      cp = blob + P.code_off[0] + static_cast<size_t>(n0 + (lane >> 1)) * (P.K / 4) + (lane & 1) * 16 + warp * kStep0;
       const bool want = lane < 16 ? be.bits >= 3 : be.bits >= 4;
       dp = want ? blob + (lane < 16 ? P.d3_off[0] : P.d4_off[0]) + static_cast<size_t>(n0 + (lane & 15)) * (P.K / 8) +
-                      s0 * kStep1
+                      warp * kStep1
                 : nullptr;
     }
     szp = blob + P.sz_off[0] + (static_cast<size_t>(n0 >> 7) * G + ((lane >> 2) & 1)) * 512 + (n0 & 127) * 4 +
-          (lane & 3) * 16 + static_cast<size_t>(s0) * sz_step;
+          (lane & 3) * 16 + warp * sz_step;
   };
   // the next stage of the stream into ring slot j % kRing (j = 0, 1, ... in
   // order); past the stream's end an empty group keeps the count uniform
@@ -360,9 +349,8 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
 
   int j = 0;  // stream position of the stage being computed
   for (int q = 0; q < my_units; ++q) {
-    int e, pass, rb, ks;
-    const int ug = blockIdx.x + q * gridDim.x;  // this unit
-    locate(ug, e, pass, rb, ks);
+    int e, pass, rb;
+    locate(blockIdx.x + q * gridDim.x, e, pass, rb);
     const BinEnt be = ent[e];
     const int t0 = pass * 8 * NB, n0 = rb * rows_per_unit;
     const int ntok = min(8 * NB, be.nrows - t0);  // token rows of this unit
@@ -373,8 +361,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       tok_in[nb] = 8 * nb + g < ntok;
-      xp[nb] = P.act + static_cast<size_t>(be.row0 + t0 + (tok_in[nb] ? 8 * nb + g : 0)) * P.K +
-               static_cast<size_t>(ks * n_stages + warp) * kStageK + 32 * c;
+      xp[nb] = P.act + static_cast<size_t>(be.row0 + t0 + (tok_in[nb] ? 8 * nb + g : 0)) * P.K + warp * kStageK + 32 * c;
     }
     // the unit's activation runs into L1 ahead of their use when they fit
     // (a stage's 128 K of one token row is two 128-byte lines)
@@ -507,31 +494,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) red[(warp * kVals + (f * NB + nb) * 4 + jj) * 32 + lane] = acc[f][nb][jj];
     __syncthreads();
-    constexpr int kPart = FW * 32 * NB * 4;  // values of one unit's partial
-    bool finish = true;                       // this unit writes the outputs
-    if (!GU && P.ksplit > 1) {  // CTA-uniform: the unit's partial, then the last split adds them
-      __shared__ int last_s;
-      float* mine = P.kpart + (static_cast<size_t>(ug / P.ksplit) * P.ksplit + ks) * kPart;
-      for (int v = threadIdx.x; v < 32 * NB * 4; v += kWarps * 32) {
-        const int ln = v & 31, nb = (v >> 5) / 4, jj = (v >> 5) & 3;
-#pragma unroll
-        for (int f = 0; f < FW; ++f) {
-          float a = 0.0f;
-          for (int w = 0; w < kWarps; ++w) a += red[(w * kVals + (f * NB + nb) * 4 + jj) * 32 + ln];
-          mine[f * 32 * NB * 4 + v] = a;
-        }
-      }
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        const int old = atomicAdd(&P.kcnt[ug / P.ksplit], 1);
-        last_s = old == P.ksplit - 1;
-        if (last_s) __threadfence();  // the other splits' partials, read below
-      }
-      __syncthreads();
-      finish = last_s;
-    }
-    for (int v = threadIdx.x; finish && v < 32 * NB * 4; v += kWarps * 32) {
+    for (int v = threadIdx.x; v < 32 * NB * 4; v += kWarps * 32) {
       const int ln = v & 31, nb = (v >> 5) / 4, jj = (v >> 5) & 3;
       const int gg = ln >> 2, cc = ln & 3;
       const int row = gg + 8 * (jj >> 1);               // weight row inside the fragment
@@ -540,12 +503,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
 #pragma unroll
       for (int f = 0; f < FW; ++f) {
         float a = 0.0f;
-        if (!GU && P.ksplit > 1) {  // the splits in order
-          const float* base = P.kpart + static_cast<size_t>(ug / P.ksplit) * P.ksplit * kPart + f * 32 * NB * 4 + v;
-          for (int sp = 0; sp < P.ksplit; ++sp) a += __ldcg(base + static_cast<size_t>(sp) * kPart);
-        } else {
-          for (int w = 0; w < kWarps; ++w) a += red[(w * kVals + (f * NB + nb) * 4 + jj) * 32 + ln];
-        }
+        for (int w = 0; w < kWarps; ++w) a += red[(w * kVals + (f * NB + nb) * 4 + jj) * 32 + ln];
         sum[f] = a;
       }
       if (tk < be.nrows) {
@@ -561,7 +519,7 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
         }
       }
     }
-    if (!GU && P.y && finish) {  // fused combine (CTA-uniform)
+    if (!GU && P.y) {  // fused combine (CTA-uniform)
       __shared__ int done_s[16];  // token completed by this unit, or -1
       __threadfence();            // this unit's y_perm rows before its counts
       __syncthreads();
@@ -627,16 +585,9 @@ moe_status_t run_pair(DecParams gu, DecParams dn, int max_bins, int passes, int 
   // 32-row units unless that leaves fewer than two units per SM
   const bool wide = static_cast<long>(max_bins) * (dn.N / 32) >= 2L * sms && dn.N % 32 == 0;
   dn.row_blocks = dn.N / (wide ? 32 : 16);
-  const int units = max_bins * passes * dn.row_blocks * dn.ksplit;
+  const int units = max_bins * passes * dn.row_blocks;
   return wide ? run_nb<false, PLANES, G64, 2>(dn, nb, units, s, "ffn decode down launch")
               : run_nb<false, PLANES, G64, 1>(dn, nb, units, s, "ffn decode down launch");
-}
-
-// Upper bound of the down pass's (bin, pass, row block) triples for
-// total_rows rows: sum over bins of ceil(rows / 8) <= rows / 8 + bins.
-int64_t split_units_base(int total_rows, int E, int d, int layout) {
-  const int nbins = E * (layout == MOE_LAYOUT_PLANES ? 3 : 1);
-  return (static_cast<int64_t>((total_rows + 7) / 8) + std::min(nbins, total_rows)) * (d / 16);
 }
 
 int sm_count_dec() {
@@ -652,25 +603,6 @@ int sm_count_dec() {
 }
 
 }  // namespace
-
-// K of at least 64 stages (8192) splits in 4 (2 when 4 does not divide the
-// stages): a long-row down pass (d rows x F) then has four times the units,
-// so the last round of units leaves few CTAs idle.  Depends on K only, so
-// every call of a shape sums in the same order.
-int decode_split_for(int K) {
-  const int st = K / kStageK;
-  if (st < 64) return 1;
-  return st % 4 == 0 ? 4 : (st % 2 == 0 ? 2 : 1);
-}
-
-size_t decode_split_bytes(int total_rows, int E, int d, int F, int layout) {
-  if (total_rows <= 0 || total_rows > 256) return 0;  // the decode kernel runs up to 16 tokens x 16 choices
-  const int S = decode_split_for(F);
-  if (S == 1) return 0;
-  const int64_t base = split_units_base(total_rows, E, d, layout);
-  const size_t cnt = (static_cast<size_t>(base) * sizeof(int32_t) + 255) & ~size_t(255);
-  return cnt + static_cast<size_t>(base) * S * 512 * sizeof(float);  // <= 2 x 2 x 128 values per unit
-}
 
 moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t s) {
   const bool planes = a.layout == MOE_LAYOUT_PLANES;
@@ -705,26 +637,8 @@ moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t 
   gu.k = a.k;
   gu.n_counters = a.y ? a.T * (a.d / 16) : 0;
   gu.counters = a.counters;
-  gu.ksplit = 1;
-  gu.n_kcnt = 0;
-  // split K of the down pass when the workspace holds its partials
-  int dn_split = decode_split_for(a.F);
-  if (dn_split > 1) {
-    const size_t need = decode_split_bytes(a.total_rows, a.E, a.d, a.F, a.layout);
-    if (need == 0 || !a.split_ws || a.split_bytes < need) {
-      dn_split = 1;
-    } else {
-      const int64_t base = split_units_base(a.total_rows, a.E, a.d, a.layout);
-      gu.kcnt = reinterpret_cast<int32_t*>(a.split_ws);
-      gu.n_kcnt = static_cast<int>(base);
-      gu.kpart = reinterpret_cast<float*>(a.split_ws + ((static_cast<size_t>(base) * sizeof(int32_t) + 255) &
-                                                        ~size_t(255)));
-    }
-  }
   DecParams dn = gu;
   dn.n_counters = 0;
-  dn.n_kcnt = 0;
-  dn.ksplit = dn_split;
   dn.perm = a.perm;
   dn.inv_perm = a.inv_perm;
   dn.topk_w = a.topk_w;

@@ -80,13 +80,11 @@ def test_ffn_combine_without_residual_and_repeated_experts():
 
 
 @pytest.mark.parametrize("T,layout", [(1, "int4"), (8, "int4"), (12, "int4"), (2, "planes")])
-def test_long_rows_split_k_against_oracle_and_slot_path(T, layout):
-    """Rows of the second GEMM long enough (d_ff = 8192: 64 stages of 128) for
-    the decode kernel to split K in four (each split's partial reduced in its
-    CTA, the four added in split order by the split that completes the
-    block): the layer matches the oracle within the bar, and the slot path
-    (the FFN wave by wave over a slot pool) gives the resident path's y_perm
-    bit for bit, since the split depends on the shape alone."""
+def test_long_rows_against_oracle_and_slot_path(T, layout):
+    """Long rows in the second GEMM (d_ff = 8192: 64 stages of 128 per row,
+    eight per warp): the layer matches the oracle within the bar, and the
+    slot path (the FFN wave by wave over a slot pool) gives the resident
+    path's y_perm bit for bit."""
     from gpu_helpers import oracle_layer, within_tol
     shape = I.custom_shape(d=256, E=8, k=2, F=8192, group=128, layout=layout)
     L = I.make_layer(shape, T, seed=81 + T)
