@@ -706,7 +706,7 @@ __global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_co
   cluster_sync_start();
   const int rank = blockIdx.x;  // the grid is one cluster
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = A.T, d = A.d, E = A.E, k = A.k, na = T * k, dk = d / kClusterSlices;
+  const int T = A.T, d = A.d, E = A.E, k = A.k, na = T * k;
   // 1-2. router
   tiny_route(A.x, A.wr, A.bias, A.forced, T, d, E, k, A.gamma, A.idx, A.gw, S, sel_s);
   // 3. bit-width gate
