@@ -260,8 +260,8 @@ moe_status_t moe_route_permute(const void* x, const float* w_router, const float
                           status, workspace, S(stream));
   }
   if (route_permute_fusable(T, d, E, k, w_bit != nullptr))
-    return launch_route_permute_tiny(x, w_router, bias, forced_idx, bits_in, w_bit, bias_bit, T, d, E, k, topk_idx,
-                                     topk_w, bits_out, counts, offsets, perm, inv_perm, x_perm, status, S(stream));
+    return launch_front_tiny(x, w_router, bias, forced_idx, bits_in, w_bit, bias_bit, T, d, E, k, topk_idx, topk_w,
+                             bits_out, counts, offsets, perm, inv_perm, x_perm, status, S(stream));
   const size_t rbytes = (route_workspace_bytes(T, d, E) + 255) / 256 * 256;
   st = launch_route(x, w_router, bias, forced_idx, T, d, E, k, topk_idx, topk_w, workspace, rbytes, S(stream));
   if (st != MOE_OK) return st;

@@ -440,12 +440,13 @@ constexpr int kTinyGateAssign = 32;   // assignments of the cluster bit gate (T*
 static_assert(kTinyGateAssign <= 32, "TinyGateSmem holds 32 assignments");
 bool route_tiny_ok(int T, int d, int E);
 bool route_permute_fusable(int T, int d, int E, int k, bool gate);
-moe_status_t launch_route_permute_tiny(const void* x, const float* w_router, const float* bias,
-                                       const int32_t* forced, const uint8_t* bits_in, const float* w_bit,
-                                       const float* bias_bit, int T, int d, int E, int k, int32_t* idx,
-                                       float* w, uint8_t* bits_out, int32_t* counts, int32_t* offsets,
-                                       int32_t* perm, int32_t* inv_perm, void* x_perm, int32_t* status,
-                                       cudaStream_t s);
+// Router (+ bit gate) (+ permutation and gather when counts is given) of the
+// smallest batches in one cluster launch (front.cu).
+moe_status_t launch_front_tiny(const void* x, const float* w_router, const float* bias, const int32_t* forced,
+                               const uint8_t* bits_in, const float* w_bit, const float* bias_bit, int T, int d,
+                               int E, int k, int32_t* idx, float* w, uint8_t* bits_out, int32_t* counts,
+                               int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* x_perm, int32_t* status,
+                               cudaStream_t s);
 size_t route_min_workspace_bytes(int T, int d, int E);
 moe_status_t route_check_args(const void* x, const float* w_router, int T, int d, int E, int k,
                               const int32_t* topk_idx, const float* topk_w, const char* fn);

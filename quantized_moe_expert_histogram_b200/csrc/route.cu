@@ -26,10 +26,11 @@
 //                   fp64 logits.  Gates are the softmax over the k picked
 //                   logits, in fp64 arithmetic on those values.
 //
-// For the smallest batches (k_route_tiny: T <= 8 and T*E <= 128) both steps
-// run in one launch of a thread-block cluster, each CTA one slice of d; the
-// same fp32-plus-bound scheme with a tighter bound (sums of magnitudes, not
-// norms), and fp64 only for the contenders of tokens it leaves open.
+// For the smallest batches (T <= 8 and T*E <= 128) both steps run in one
+// launch of a thread-block cluster (k_front, front.cu), each CTA one slice
+// of d; the same fp32-plus-bound scheme with a tighter bound (sums of
+// magnitudes, not norms), and fp64 only for the contenders of tokens it
+// leaves open.
 //
 // Error bound of the fp32 sum: an FMA chain over m products errs by at most
 // g(m) times the sum of their magnitudes; a chunk (32 products) and then the
@@ -469,329 +470,6 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
   select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, blockIdx.x);
 }
 
-// ---- the smallest batches: one cluster launch -------------------------
-//
-// The router of up to 8 tokens with T*E <= kTinyRouteItems over one
-// thread-block cluster of kClusterSlices CTAs, CTA r taking the d-slice
-// [r d/8, (r+1) d/8) of every (token, expert) dot product:
-//   1. fp32 slice partials S and magnitude sums A (cluster_partial_dots_f32)
-//      into CTA 0's shared memory (DSMEM), cluster barrier;
-//   2. CTA 0, a warp per token: L = (sum_r S_r) + b and A = sum_r A_r in
-//      fp32 (8 more additions: |L - l| <= g(m) A + g(8) (sum_r |S_r| + |b|)),
-//      bound D = 2 g(m + 9) (A (1 + 2^-8) + |b|) (m = products per lane of a
-//      slice + 5; factor 2: margin), top k of L by rank counting, certified
-//      when consecutive picks and the cut after the k-th are separated by
-//      more than their bounds; otherwise the token's contenders (the picks
-//      and every expert whose upper bound reaches the lowest pick's lower
-//      bound) are listed;
-//   3. if any token was not certified (the count is read by every CTA after
-//      a barrier, so all take the same branch): every CTA computes its slice
-//      of the listed dot products in fp64 (each bf16 x fp32 product exact),
-//      CTA 0 selects those tokens again on the fp64 logits.
-// Gates: the softmax over the picked logits (fp32 for certified tokens,
-// fp64 for re-evaluated ones).  No fp64 arithmetic runs unless a token is
-// left open: measured on B200, scalar fp64 throughput is a small fraction
-// of fp32 and bounded an all-fp64 version of this router.
-struct TinyRouteSmem {
-  float2 p32[kClusterSlices * kTinyRouteItems];  // (S, A) per slice and item t*E + e
-  double p64[kClusterSlices * kTinyRouteItems];  // fp64 partials of the listed items (and, in the
-                                                 // fused kernel, of the width scores)
-  float val[kTinyRouteItems];                    // fp32-path logits of item t*E + e
-  float dev[kTinyRouteItems];                    // their bounds
-  double val64[kTinyRouteItems];                 // fp64 logits of re-evaluated tokens
-  int32_t cand[kTinyRouteItems];                 // listed items
-  int32_t pos[kTinyRouteItems];                  // item -> index in cand, or -1
-  int32_t n_cand;
-  int32_t unsure[kSelWarps];
-};
-
-// Gates of token t from its logits (vals) at its picks (sel, k entries):
-// softmax in the logits' precision, maximum and sum as shuffle trees; ids
-// and gates to global.
-template <typename V>
-__device__ __forceinline__ void tiny_gates(const V* vals, const int32_t* sel, int k, int t, int lane,
-                                           int32_t* out_idx, float* out_w) {
-  const bool mine = lane < k;
-  const int e = mine ? sel[lane] : 0;
-  const V lv = mine ? vals[e] : static_cast<V>(-INFINITY);
-  V mx = lv;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  const V ex = mine ? exp(lv - mx) : static_cast<V>(0);
-  V sum = ex;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (mine) {
-    out_idx[static_cast<size_t>(t) * k + lane] = e;
-    out_w[static_cast<size_t>(t) * k + lane] = static_cast<float>(ex / sum);
-  }
-}
-
-// Every CTA of the cluster calls this (after cluster_sync_start); CTA 0
-// ends with the picks in sel_s ([T][k], shared) and the outputs written.
-__device__ __forceinline__ void tiny_route(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr,
-                                           const float* __restrict__ bias, const int32_t* __restrict__ forced,
-                                           int T, int d, int E, int k, float gamma, int32_t* out_idx,
-                                           float* out_w, TinyRouteSmem& S, int32_t* sel_s) {
-  const int rank = blockIdx.x;  // the grid is one cluster
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n = T * E, dk = d / kClusterSlices;
-  auto rows = [&](int i, const __nv_bfloat16*& xr, const float*& w) {
-    const int t = i / E;
-    xr = x + static_cast<size_t>(t) * d;
-    w = wr + static_cast<size_t>(i - t * E) * d;
-  };
-  if (threadIdx.x == 0) S.n_cand = 0;
-  cluster_partial_dots_f32(n, rank * dk, dk, rows, cluster_map_shared(S.p32, 0) + 8u * static_cast<uint32_t>(rank * n));
-  cluster_sync_publish();
-  // 2. fp32-path logits, selection and certification (CTA 0)
-  if (rank == 0 && warp < T) {
-    const int t = warp;
-    float* val = S.val + t * E;
-    float* dev = S.dev + t * E;
-    int32_t* sel = sel_s + t * k;
-    for (int e = lane; e < E; e += 32) {
-      float L = 0.0f, mag = 0.0f;
-      for (int r = 0; r < kClusterSlices; ++r) {
-        const float2 p = S.p32[r * n + t * E + e];
-        L += p.x;
-        mag += p.y;
-      }
-      const float b = bias ? bias[e] : 0.0f;
-      val[e] = L + b;
-      dev[e] = 2.0f * gamma * (mag * (1.0f + 0.00390625f) + fabsf(b)) + 1e-30f;
-      S.pos[t * E + e] = -1;
-    }
-    __syncwarp();
-    bool sure = true;
-    if (forced) {
-      for (int j = lane; j < k; j += 32) {
-        const int e = forced[static_cast<size_t>(t) * k + j];
-        sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
-      }
-      __syncwarp();
-    } else {
-      warp_topk_rank(val, E, k, lane, sel);
-      bool ok = true;
-      float lo = INFINITY;
-      if (lane < k) {
-        const int e = sel[lane];
-        lo = val[e] - dev[e];
-        if (lane > 0) ok = val[sel[lane - 1]] - dev[sel[lane - 1]] > val[e] + dev[e];
-        ok = ok && lo == lo && fabsf(lo) <= 3.0e38f;
-      }
-      float lo_min = lo;
-#pragma unroll
-      for (int o = 16; o; o >>= 1) lo_min = fminf(lo_min, __shfl_xor_sync(0xffffffffu, lo_min, o));
-      const float lo_k = __shfl_sync(0xffffffffu, lo, k - 1);
-      for (int e = lane; e < E; e += 32) {
-        bool picked = false;
-        for (int j = 0; j < k; ++j) picked = picked || sel[j] == e;
-        if (!picked) ok = ok && val[e] + dev[e] < lo_k;  // NaN: not certified
-      }
-      sure = __all_sync(0xffffffffu, ok);
-      if (!sure) {  // list the contenders for fp64
-        const bool finite = lo_min == lo_min && fabsf(lo_min) <= 3.0e38f;
-        for (int e = lane; e < E; e += 32) {
-          bool picked = false;
-          for (int j = 0; j < k; ++j) picked = picked || sel[j] == e;
-          if (!finite || picked || !(val[e] + dev[e] < lo_min)) {
-            const int p = atomicAdd(&S.n_cand, 1);
-            S.cand[p] = t * E + e;
-            S.pos[t * E + e] = p;
-          }
-        }
-      }
-    }
-    if (lane == 0) S.unsure[t] = sure ? 0 : 1;
-    if (sure) tiny_gates(val, sel, k, t, lane, out_idx, out_w);
-  }
-  // CTA 0 writes the contender count and list into every CTA's shared
-  // memory before the barrier, so that after it no CTA reads another's
-  // shared memory (CTA 0 may have exited by then)
-  if (rank == 0) {
-    __syncthreads();  // the list is complete
-    const int nc = S.n_cand;
-    for (int r = 1; r < kClusterSlices; ++r) {
-      for (int i = threadIdx.x; i < nc; i += blockDim.x) st_cluster_u32(cluster_map_shared(&S.cand[i], r), S.cand[i]);
-      if (threadIdx.x == 0) st_cluster_u32(cluster_map_shared(&S.n_cand, r), nc);
-    }
-  }
-  cluster_sync_publish();  // the contender list is in every CTA
-  const int n3 = S.n_cand;
-  if (n3 == 0) return;  // cluster-uniform
-  // 3. fp64 for the listed items
-  cluster_partial_dots(
-      n3, rank * dk, dk, [&](int i, const __nv_bfloat16*& xr, const float*& w) { rows(S.cand[i], xr, w); },
-      cluster_map_shared(S.p64, 0) + 8u * static_cast<uint32_t>(rank * n3));
-  cluster_sync_publish();
-  if (rank == 0 && warp < T && S.unsure[warp]) {
-    const int t = warp;
-    double* val = S.val64 + t * E;
-    int32_t* sel = sel_s + t * k;
-    for (int e = lane; e < E; e += 32) {
-      const int p = S.pos[t * E + e];
-      double v = -INFINITY;
-      if (p >= 0) {
-        v = S.p64[p];
-        for (int r = 1; r < kClusterSlices; ++r) v += S.p64[r * n3 + p];
-        v += bias ? static_cast<double>(bias[e]) : 0.0;
-      }
-      val[e] = v;
-    }
-    __syncwarp();
-    warp_topk_rank(val, E, k, lane, sel);
-    tiny_gates(val, sel, k, t, lane, out_idx, out_w);
-  }
-}
-
-// The smallest batches (route_tiny_ok: T <= 8, T*E <= 128, d % 64 == 0).
-__global__ void __launch_bounds__(kSelThreads) k_route_tiny(
-    const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
-    const int32_t* __restrict__ forced, int T, int d, int E, int k, float gamma, int32_t* __restrict__ out_idx,
-    float* __restrict__ out_w) {
-  __shared__ TinyRouteSmem S;
-  __shared__ int32_t sel_s[kTinyRouteItems];
-  pdl_wait();
-  pdl_trigger();
-  cluster_sync_start();
-  tiny_route(x, wr, bias, forced, T, d, E, k, gamma, out_idx, out_w, S, sel_s);
-}
-
-// ---- router + bit-width gate + permutation in one launch -------------
-//
-// The smallest batches (route_tiny_ok, T*k <= kFusedAssign, and with a bit
-// gate T*k <= kTinyGateAssign) through the whole front of the layer in one
-// cluster launch,
-// with the results of k_route_tiny, k_bit_gate_tiny and the permutation
-// kernels (same arithmetic, same order):
-//   1-2. the router of k_route_tiny (tiny_route); CTA 0 holds the ids
-//   3. with a bit gate: the ids are published to the cluster, then the bit
-//      gate of k_bit_gate_tiny (tiny_bit_gate)
-//   4. CTA 0: keys (expert, or 3 expert + width - 2), stable ranks by
-//      counting (ties in ascending assignment), counts, offsets, perm,
-//      inv_perm, and the gather of x_perm (fp16) in expert order.
-constexpr int kFusedAssign = 64;
-
-struct RoutePermArgs {
-  const __nv_bfloat16* x;
-  const float* wr;
-  const float* bias;
-  const int32_t* forced;
-  const uint8_t* bits_in;  // widths given by the caller, or null
-  const float* wbit;       // bit gate, or null
-  const float* bbit;
-  int T, d, E, k;
-  int32_t* idx;
-  float* gw;
-  uint8_t* bits_out;
-  int32_t* counts;
-  int32_t* offsets;
-  int32_t* perm;
-  int32_t* inv_perm;
-  __half* x_perm;  // null: no gather
-  int32_t* status;
-  float gamma;  // bound factor of the router's fp32 path
-};
-
-__global__ void __launch_bounds__(kSelThreads) k_route_perm_tiny(const __grid_constant__ RoutePermArgs A) {
-  __shared__ TinyRouteSmem S;
-  __shared__ TinyGateSmem G;
-  __shared__ int32_t sel_s[kFusedAssign];
-  __shared__ int32_t key_s[kFusedAssign];
-  __shared__ int32_t perm_s[kFusedAssign];
-  __shared__ uint8_t bits_s[kFusedAssign];
-  pdl_wait();
-  pdl_trigger();
-  cluster_sync_start();
-  const int rank = blockIdx.x;  // the grid is one cluster
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = A.T, d = A.d, E = A.E, k = A.k, na = T * k;
-  // 1-2. router
-  tiny_route(A.x, A.wr, A.bias, A.forced, T, d, E, k, A.gamma, A.idx, A.gw, S, sel_s);
-  // 3. bit-width gate
-  if (A.wbit) {  // uniform over the cluster
-    // CTA 0 writes the ids into every CTA's shared memory before the barrier
-    // (no CTA reads another's shared memory after a barrier)
-    __shared__ int32_t ids_l[kFusedAssign];
-    if (rank == 0) {
-      __syncthreads();  // sel_s complete
-      for (int r = 0; r < kClusterSlices; ++r)
-        for (int a = threadIdx.x; a < na; a += blockDim.x) st_cluster_u32(cluster_map_shared(&ids_l[a], r), sel_s[a]);
-    }
-    cluster_sync_publish();  // the ids are in every CTA; CTA 0's last reads of S are done
-    tiny_bit_gate(A.x, A.wbit, A.bbit, ids_l, T, d, k, A.gamma, A.bits_out, bits_s, G);
-  }
-  if (rank != 0) return;
-  __syncthreads();  // sel_s, bits_s complete
-  // 4. permutation of the na assignments
-  const bool nested = A.wbit || A.bits_in;
-  const int nbins = nested ? 3 * E : E;
-  for (int a = threadIdx.x; a < na; a += blockDim.x) {
-    int key = sel_s[a];
-    if (nested) {
-      int b = A.wbit ? bits_s[a] : A.bits_in[a];
-      if (b < 2 || b > 4) {
-        flag_status(A.status, MOE_DEV_BAD_INDEX);
-        b = b < 2 ? 2 : 4;
-      }
-      key = 3 * key + (b - 2);
-    }
-    key_s[a] = key;
-  }
-  __syncthreads();
-  for (int a = threadIdx.x; a < na; a += blockDim.x) {
-    const int key = key_s[a];
-    int pos = 0;
-    for (int o = 0; o < na; ++o) {
-      const int ko = key_s[o];
-      pos += (ko < key || (ko == key && o < a)) ? 1 : 0;
-    }
-    A.perm[pos] = a;
-    A.inv_perm[a] = pos;
-    perm_s[pos] = a;
-  }
-  for (int b = threadIdx.x; b <= nbins; b += blockDim.x) {
-    int below = 0, at = 0;
-    for (int o = 0; o < na; ++o) {
-      below += key_s[o] < b ? 1 : 0;
-      at += key_s[o] == b ? 1 : 0;
-    }
-    A.offsets[b] = below;
-    if (b < nbins) A.counts[b] = at;
-  }
-  if (!A.x_perm) return;
-  __syncthreads();  // perm_s complete
-  // gather: warp per row, 8 elements per lane per piece and up to 8
-  // pieces' loads in flight (bf16 -> fp16)
-  bool bad = false;
-  for (int p = warp; p < na; p += kSelWarps) {
-    const uint4* src = reinterpret_cast<const uint4*>(A.x + static_cast<size_t>(perm_s[p] / k) * d);
-    uint4* dst = reinterpret_cast<uint4*>(A.x_perm + static_cast<size_t>(p) * d);
-    for (int c0 = lane; c0 < d / 8; c0 += 8 * 32) {
-      uint4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (c0 + 32 * u < d / 8) v[u] = src[c0 + 32 * u];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (c0 + 32 * u >= d / 8) break;
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
-        uint4 o;
-        __half2* h2 = reinterpret_cast<__half2*>(&o);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = __bfloat1622float2(b2[j]);
-          bad |= fabsf(f.x) > 65504.0f || fabsf(f.y) > 65504.0f;
-          h2[j] = __floats2half2_rn(f.x, f.y);
-        }
-        dst[c0 + 32 * u] = o;
-      }
-    }
-  }
-  if (bad) flag_status(A.status, MOE_DEV_RANGE);
-}
-
 int route_splits(int T, int d, int E, size_t cap = static_cast<size_t>(-1)) {
   const int ec = E <= 16 ? 16 : 64;
   const int tt = ec == 64 ? Tile<64>::TT : Tile<16>::TT;
@@ -836,32 +514,6 @@ moe_status_t launch_logits(const __nv_bfloat16* x, const float* wr, int T, int d
 
 int g_route_fused = 1;
 
-// The fp64 cluster router pays while each warp of the cluster has at most
-// two rounds of dot products (T*E <= 128 with 8 CTAs of 8 warps): measured
-// on the OLMoE-shaped layer, a one-token step 38.9 -> 32.3 us against the
-// two-launch router, two tokens 46.0 -> 43.0 us; at four and eight tokens
-// (four and eight rounds) the two-launch router was faster.
-bool route_tiny_ok(int T, int d, int E) {
-  return g_route_fused == 1 && T >= 1 && T <= kSelWarps && T * E <= kTinyRouteItems && d % (8 * kClusterSlices) == 0;
-}
-
-bool route_permute_fusable(int T, int d, int E, int k, bool gate) {
-  return route_tiny_ok(T, d, E) && T * k <= kFusedAssign && (!gate || 3 * T * k <= 3 * kTinyGateAssign);
-}
-
-moe_status_t launch_route_permute_tiny(const void* x, const float* w_router, const float* bias,
-                                       const int32_t* forced, const uint8_t* bits_in, const float* w_bit,
-                                       const float* bias_bit, int T, int d, int E, int k, int32_t* idx,
-                                       float* w, uint8_t* bits_out, int32_t* counts, int32_t* offsets,
-                                       int32_t* perm, int32_t* inv_perm, void* x_perm, int32_t* status,
-                                       cudaStream_t s) {
-  RoutePermArgs A{static_cast<const __nv_bfloat16*>(x), w_router, bias, forced, bits_in, w_bit, bias_bit,
-                  T, d, E, k, idx, w, bits_out, counts, offsets, perm, inv_perm, static_cast<__half*>(x_perm),
-                  status, cluster_gamma(d)};
-  return cuda_check(launch_cluster_pdl(k_route_perm_tiny, kClusterSlices, dim3(kSelThreads), 0, s, A),
-                    "moe_route_permute cluster launch");
-}
-
 size_t route_workspace_bytes(int T, int d, int E) {
   if (T <= 0 || d <= 0 || E <= 0) return 256;
   return route_ws_for(static_cast<size_t>(route_splits(T, d, E)), T, E);
@@ -879,11 +531,10 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
   const int splits = route_splits(T, d, E, workspace_bytes);
   const RouteWs ws = route_ws(workspace, splits, T, E);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  // the smallest batches: fp64 logits in one cluster launch (no workspace)
+  // the smallest batches: one cluster launch (no workspace)
   if (route_tiny_ok(T, d, E))
-    return cuda_check(launch_cluster_pdl(k_route_tiny, kClusterSlices, dim3(kSelThreads), 0, s, xb, w_router, bias,
-                                         forced, T, d, E, k, cluster_gamma(d), idx, w),
-                      "moe_route_topk cluster launch");
+    return launch_front_tiny(x, w_router, bias, forced, nullptr, nullptr, nullptr, T, d, E, k, idx, w, nullptr,
+                             nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, s);
   moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, k, splits, ws, s)
                             : launch_logits<64>(xb, w_router, T, d, E, k, splits, ws, s);
   if (st != MOE_OK) return st;

@@ -140,3 +140,36 @@ def test_route_permute_flags_and_argument_errors():
     with pytest.raises(moeq.MoeError) as ei:
         moeq.moe_route_permute(x.cuda(), L["w_router"].cuda(), None, shape.k, bits=bits, w_bit=G["w_bit"].cuda())
     assert ei.value.code == 1
+
+
+@pytest.mark.parametrize("T", [1, 2, 8])
+def test_route_permute_gate_ties_on_open_tokens(T):
+    """Exact ties everywhere the one-launch path has a fallback: router rows
+    of experts 2 and 5 (and 0 and 7) identical, so tokens whose picks or
+    cut involve them are decided on fp64 logits; bit-gate rows of widths 3
+    and 4 identical for every expert (width 2 far below), so every width is
+    a tie that must go to the narrower width, including for the assignments
+    of those tokens.  Ids, widths and the permutation equal the oracle's."""
+    shape = I.SHAPES["nested"]
+    L = I.make_layer(shape, T, seed=47, weights=False)
+    wr = L["w_router"].clone()
+    wr[5] = wr[2]
+    wr[7] = wr[0]
+    G = I.make_bit_gate(shape, seed=48, bias=True)
+    wb, bb = G["w_bit"].clone(), G["bias_bit"].clone()
+    wb[:, 2] = wb[:, 1]
+    bb[:, 2] = bb[:, 1]
+    bb[:, 0] = -10.0
+    x = L["x"].cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moeq.moe_route_permute(x, wr.cuda(), None, shape.k, w_bit=wb.cuda(), bias_bit=bb.cuda(), status=status)
+    sep = _separate(x, wr.cuda(), None, shape.k, w_bit=wb.cuda(), bias_bit=bb.cuda())
+    torch.cuda.synchronize()
+    sel, _, _ = O.route(L["x"].float().numpy(), wr.numpy(), None, shape.k)
+    np.testing.assert_array_equal(out["topk_idx"].cpu().numpy(), sel)
+    b_ref = O.bit_gate(L["x"].float().numpy(), wb.numpy(), bb.numpy(), sel)
+    assert (b_ref == 3).all()
+    np.testing.assert_array_equal(out["bits"].cpu().numpy(), b_ref)
+    for key in KEYS:
+        assert torch.equal(out[key], sep[key]), key
+    assert int(status.item()) == 0
