@@ -232,18 +232,18 @@ def make_instances(shape, T, R, seed, device, bit_gate=False):
 def kernel_launches(shape, T, bit_gate=False):
     """Kernels of this library launched by one layer step, following the
     library's own choices: router, bit gate and permutation as one cluster
-    launch for the smallest batches (T <= 8, T*E <= 128, T*k <= 64, with a
-    bit gate T*k <= 32, d % 64 == 0); otherwise router 1 (fp64 cluster launch
-    for T*E <= 128) or 2, bit gate 1 when used, permutation 1 (single CTA,
+    launch for the smallest batches (T <= 8, T*E <= 512, with a bit gate
+    T*E <= 128, T*k <= 64, d % 256 == 0); otherwise router 1 (one cluster
+    launch under the same rule on T*E) or 2, bit gate 1 when used, permutation 1 (single CTA,
     with the gather when it is small) or 1 + gather, or 3 + gather; then
     FFN 2, and the combine 1 unless the decode kernel (T <= 16) sums it in
     its second GEMM."""
     n = T * shape.k
     comb = 0 if T <= 16 else 1  # the decode kernel (T <= 16) sums the combine in its second GEMM
-    if T <= 8 and T * shape.E <= 128 and n <= (32 if bit_gate else 64) and shape.d % 64 == 0:
+    if T <= 8 and T * shape.E <= (128 if bit_gate else 512) and n <= 64 and shape.d % 256 == 0:
         return 1 + 2 + comb
     nbins = shape.E * (3 if shape.layout == "planes" else 1)
-    route = 1 if (T <= 8 and T * shape.E <= 128 and shape.d % 64 == 0) else 2
+    route = 1 if (T <= 8 and T * shape.E <= 512 and shape.d % 256 == 0) else 2
     if n <= 1024:
         perm = 1 if n * shape.d <= 64 * 1024 else 2
     else:

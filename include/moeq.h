@@ -135,7 +135,7 @@ MOE_API moe_status_t moe_quant_pack(const float* w_gate, const float* w_up, cons
  *   topk_w   fp32 [T][k]: softmax over the k selected logits (the full
  *            softmax renormalised over the selection), from the fp32
  *            logits (fp64 ones for re-evaluated tokens)
- *            The smallest batches (T <= 8, T*E <= 128, d % 64 == 0) run both
+ *            The smallest batches (T <= 8, T*E <= 512, d % 256 == 0) run both
  *            steps as one launch of a thread-block cluster (one d slice per
  *            CTA, a tighter per-logit bound from the sums of the products'
  *            magnitudes, fp64 only for the contenders of unsettled tokens).
@@ -207,11 +207,12 @@ MOE_API size_t moe_permute_workspace_bytes(int T, int E, int k, int nested);
  * then (with a bit gate) moe_bit_gate, then moe_permute, with their results
  * bit for bit ([ExactMoE] the router decides, every routed expert runs;
  * [D2MoE] Dual Routing: expert gate and bit gate side by side; [Read-ME]
- * expert-aware batching).  The smallest batches -- T <= 8, T*E <= 128,
- * T*k <= 64 (with a bit gate T*k <= 32), d % 64 == 0 -- run as one launch
- * of a thread-block cluster (the cluster router of moe_route_topk, fp64
- * width scores, then the permutation and the gather in one CTA); other
- * sizes issue the separate launches on `stream`.
+ * expert-aware batching).  The smallest batches -- T <= 8, T*E <= 512
+ * (with a bit gate T*E <= 128), T*k <= 64, d % 256 == 0 -- run as one
+ * launch of a thread-block cluster (the cluster router of moe_route_topk,
+ * the width scores of every expert computed with the logits and decided
+ * the same way, then the permutation and the gather); other sizes issue
+ * the separate launches on `stream`.
  *   forced_idx int32 [T][k] or NULL, as in moe_route_topk.
  *   bits_in    uint8 [T][k] widths given by the caller (nested bins), or NULL.
  *   w_bit, bias_bit  the bit gate as in moe_bit_gate, or NULL; with w_bit,
@@ -456,9 +457,9 @@ MOE_API void moe_debug_set_trace(void* host_mapped_ints);
 
 /* Test hook (process-wide), selecting among paths with the same results:
  * 1 (the default): moe_route_topk takes the smallest batches (T <= 8,
- * T*E <= 128, d % 64 == 0) in one thread-block-cluster launch, moe_bit_gate
- * up to 32 assignments (d % 64 == 0) as fp64 scores in one cluster launch,
- * and moe_route_permute fuses all three steps when both apply.  0: the
+ * T*E <= 512, d % 256 == 0) in one thread-block-cluster launch,
+ * moe_bit_gate up to 32 assignments (d % 64 == 0) in one cluster launch,
+ * and moe_route_permute fuses all three steps (see there).  0: the
  * two-launch router and the one-kernel bit gate, and separate launches in
  * moe_route_permute, at every size. */
 MOE_API void moe_debug_route_fused(int mode);

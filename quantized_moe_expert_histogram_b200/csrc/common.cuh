@@ -435,7 +435,6 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
                           float* w, void* workspace, size_t workspace_bytes, cudaStream_t s);
 size_t route_workspace_bytes(int T, int d, int E);
 extern int g_route_fused;  // test hook: 1 default, 0 no fp64 cluster paths
-constexpr int kTinyRouteItems = 128;  // router dot products of the cluster path (T*E)
 constexpr int kTinyGateAssign = 32;   // assignments of the cluster bit gate (T*k)
 static_assert(kTinyGateAssign <= 32, "TinyGateSmem holds 32 assignments");
 bool route_tiny_ok(int T, int d, int E);

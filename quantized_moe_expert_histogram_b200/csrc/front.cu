@@ -50,9 +50,10 @@ namespace {
 constexpr int kFC = 8;               // CTAs of the cluster (slices of d)
 constexpr int kFThreads = 256;       // threads of a CTA
 constexpr int kFWarps = kFThreads / 32;
-constexpr int kFMaxTE = kTinyRouteItems;  // T*E
+constexpr int kFMaxTE = 512;              // T*E
+constexpr int kFMaxGateTE = 128;          // T*E with a bit gate (4 T*E dot products)
 constexpr int kFMaxTK = 64;               // T*k
-constexpr int kFMaxItems = 4 * kFMaxTE;   // router + gate dot products
+constexpr int kFMaxItems = kFMaxTE > 4 * kFMaxGateTE ? kFMaxTE : 4 * kFMaxGateTE;  // router + gate dot products
 constexpr int kFMaxList = kFMaxTE + 3 * kFMaxTK;
 
 struct FrontArgs {
@@ -525,15 +526,15 @@ float front_gamma(int d) {
 
 }  // namespace
 
-// The smallest batches (T <= 8, T*E <= 128, d % 256 == 0): one slice of d
-// per CTA is a multiple of 32 elements (4 lanes x 8-element pieces).
+// The smallest batches (T <= 8, T*E <= 512, d % 256 == 0: one slice of d
+// per CTA is a multiple of 32 elements, 4 lanes x 8-element pieces).
 bool route_tiny_ok(int T, int d, int E) {
   return g_route_fused == 1 && T >= 1 && T <= 8 && T * E <= kFMaxTE && d % (32 * kFC) == 0;
 }
 
+// With a bit gate, T*E <= 128 (its 3 T*E scores join the T*E logits).
 bool route_permute_fusable(int T, int d, int E, int k, bool gate) {
-  (void)gate;
-  return route_tiny_ok(T, d, E) && T * k <= kFMaxTK;
+  return route_tiny_ok(T, d, E) && T * k <= kFMaxTK && (!gate || T * E <= kFMaxGateTE);
 }
 
 moe_status_t launch_front_tiny(const void* x, const float* w_router, const float* bias, const int32_t* forced,

@@ -1,7 +1,7 @@
 """The benchmark's count of this library's kernels per layer step
 (`gpu_launches`) follows the library's own launch choices: router, bit gate
 and permutation are one cluster launch for the smallest batches (T <= 8,
-T*E <= 128, T*k <= 64, with a bit gate T*k <= 32); otherwise the router is
+T*E <= 512, with a bit gate T*E <= 128, T*k <= 64); otherwise the router is
 two launches, the bit gate adds one, the
 permutation is one single-CTA launch up to 1024 assignments (gathering the
 rows itself up to 64 K elements, else one gather launch after it) and
@@ -16,8 +16,7 @@ def test_kernel_launches_per_step():
     S = I.SHAPES
     assert bench.kernel_launches(S["olmoe"], 1) == 1 + 2                  # route + permute; combine in the FFN
     assert bench.kernel_launches(S["olmoe"], 2) == 1 + 2                  # T*E = 128
-    assert bench.kernel_launches(S["olmoe"], 8) == 2 + 2 + 2              # T*E = 512: two-launch router;
-    #                                                                       64 x 2048 > 64 K: gather launch
+    assert bench.kernel_launches(S["olmoe"], 8) == 1 + 2                  # T*E = 512, T*k = 64
     assert bench.kernel_launches(S["olmoe"], 16) == 2 + 2 + 2             # decode kernel: combine fused
     assert bench.kernel_launches(S["olmoe"], 17) == 2 + 2 + 2 + 1         # tensor cores: combine launch
     assert bench.kernel_launches(S["olmoe"], 64) == 2 + 2 + 2 + 1

@@ -37,8 +37,8 @@ def _separate(x, wr, bias, k, forced=None, bits=None, w_bit=None, bias_bit=None)
     return out
 
 
-# one cluster launch: olmoe 1-2, mixtral 1-8, tiny 8, nested 1-8 (with the gate 1-8);
-# separate launches: olmoe 8 and 256, nested 16
+# one cluster launch: olmoe 1-8, mixtral 1-8, tiny 8, nested 1-8 (with the gate 1-8);
+# separate launches: olmoe 256, nested 16
 CASES = [("olmoe", 1, "int4"), ("olmoe", 2, "int4"), ("mixtral", 1, "int4"), ("mixtral", 8, "int4"),
          ("tiny", 8, "int4"), ("nested", 1, "bits"), ("nested", 8, "bits"), ("nested", 1, "gate"),
          ("nested", 8, "gate"), ("nested", 16, "gate"), ("olmoe", 8, "int4"), ("olmoe", 256, "int4")]
