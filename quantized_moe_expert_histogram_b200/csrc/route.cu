@@ -24,9 +24,9 @@
 //                   are recomputed by the whole CTA in fp64 (each product of
 //                   a bf16 and an fp32 is exact in fp64) and selected on the
 //                   fp64 logits.  Gates are the softmax over the k picked
-//                   logits, in fp64 arithmetic on those values.
+//                   logits (fp32 for certified tokens, fp64 for the others).
 //
-// For the smallest batches (T <= 8 and T*E <= 128) both steps run in one
+// For the smallest batches (T <= 8 and T*E <= 512) both steps run in one
 // launch of a thread-block cluster (k_front, front.cu), each CTA one slice
 // of d; the same fp32-plus-bound scheme with a tighter bound (sums of
 // magnitudes, not norms), and fp64 only for the contenders of tokens it
@@ -243,23 +243,23 @@ __global__ void __launch_bounds__(kLT, 4) k_route_logits(const __nv_bfloat16* __
   logits_tile<EC>(x, wr, T, d, E, dk, ws, blockIdx.x, blockIdx.y, blockIdx.z, sm);
 }
 
-constexpr int kPer = 8;  // E <= 256: at most 8 experts per lane (e = lane + 32 m)
+constexpr int kMaxPer = 8;  // E <= 256: at most 8 experts per lane (e = lane + 32 m)
 
 // True on every lane of a warp when any lane lists a contender.
 __device__ __forceinline__ bool contender_any(uint32_t c) { return __any_sync(0xffffffffu, c != 0); }
 
 // Top k of the lane-distributed values v[m] (expert lane + 32 m; experts
-// with ok[m] false take no part), ties to the lower index; returns the picks
-// in order and the lane's taken mask.
-template <typename V>
-__device__ __forceinline__ uint32_t warp_topk(const V (&v)[kPer], uint32_t allowed, int E, int k, int lane,
-                                              int (&sel)[16]) {
+// whose bit m of `allowed` is clear take no part), ties to the lower index;
+// lane j < k receives pick j (0 where fewer than k values are comparable).
+template <typename V, int P>
+__device__ __forceinline__ int warp_topk(const V (&v)[P], uint32_t allowed, int E, int k, int lane) {
   uint32_t taken = 0;
+  int mine = 0;
   for (int j = 0; j < k; ++j) {
     V best = -INFINITY;
     int best_e = 0x7fffffff;
 #pragma unroll
-    for (int m = 0; m < kPer; ++m) {
+    for (int m = 0; m < P; ++m) {
       const int e = lane + 32 * m;
       if (e < E && (allowed & (1u << m)) && !(taken & (1u << m)) &&
           (v[m] > best || (v[m] == best && e < best_e))) {
@@ -277,33 +277,24 @@ __device__ __forceinline__ uint32_t warp_topk(const V (&v)[kPer], uint32_t allow
       }
     }
     if (best_e >= E) best_e = 0;  // only when fewer than k values are comparable (NaN)
-    sel[j] = best_e;
+    if (lane == j) mine = best_e;
     if ((best_e & 31) == lane) taken |= 1u << (best_e >> 5);
   }
-  return taken;
+  return mine;
 }
 
-// Value of expert e from the lane-distributed array.
-template <typename V>
-__device__ __forceinline__ V lane_value(const V (&v)[kPer], int e) {
-  V r = 0;
+// Softmax over the k picks (lane j < k holds pick j, in any order) of the
+// lane-distributed values, in fp64; maximum and sum are fixed-order shuffle
+// trees.
+template <typename V, int P>
+__device__ __forceinline__ void write_gates(const V (&v)[P], int mine, int k, int t, int lane, int32_t* out_idx,
+                                            float* out_w) {
+  double lv = 0.0;
 #pragma unroll
-  for (int m = 0; m < kPer; ++m) {
-    const V o = __shfl_sync(0xffffffffu, v[m], e & 31);
-    if ((e >> 5) == m) r = o;
+  for (int m = 0; m < P; ++m) {  // the value of expert `mine`, from the lane that holds it
+    const V o = __shfl_sync(0xffffffffu, v[m], mine & 31);
+    if ((mine >> 5) == m) lv = static_cast<double>(o);
   }
-  return r;
-}
-
-// Softmax over the k picks: lane j < k owns pick j; maximum and sum are
-// fixed-order shuffle trees (picks given by the caller need not be sorted).
-template <typename V>
-__device__ __forceinline__ void write_gates(const V (&v)[kPer], const int (&sel)[16], int k, int t,
-                                            int lane, int32_t* out_idx, float* out_w) {
-  int mine = 0;
-  for (int j = 0; j < k; ++j)
-    if (j == lane) mine = sel[j];
-  const double lv = static_cast<double>(lane_value(v, mine));
   double mx = lane < k ? lv : -INFINITY;
 #pragma unroll
   for (int o = 16; o; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -317,55 +308,69 @@ __device__ __forceinline__ void write_gates(const V (&v)[kPer], const int (&sel)
   }
 }
 
+// Order-preserving unsigned key of an fp32 value (a > b gives key(a) >
+// key(b); -0 sorts below +0); NaN gets 0, below every other key.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return v == v ? ((b & 0x80000000u) ? ~b : (b | 0x80000000u)) : 0u;
+}
+
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 
-// Warp per token.  A token the fp32 bounds do not settle lists its
-// contenders -- every expert whose upper bound reaches the lowest lower
-// bound among the picks (all others are certainly out) -- and the CTA's
-// warps recompute those logits in fp64; the token's warp then selects among
-// them on the fp64 values.
+// Warp per token, P experts per lane (E <= 32 P).  The k largest fp32
+// logits are picked one at a time with warp reductions (redux.sync) over
+// order keys: the largest key, then the lowest expert holding it.  The
+// certificate and the gates are lane-parallel: lane j < k holds pick j.  A
+// token the fp32 bounds do not settle lists its contenders -- every expert
+// whose upper bound reaches the lowest lower bound among the picks (all
+// others are certainly out) -- and the CTA's warps recompute those logits
+// in fp64; the token's warp then selects among them on the fp64 values.
 // Tokens block * kSelWarps .. + kSelWarps - 1, by all kSelThreads threads.
+template <int P>
 __device__ __forceinline__ void select_block(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, RouteWs ws, int splits,
     const float* __restrict__ bias, const int32_t* __restrict__ forced, int T, int d, int E, int k,
     float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w, int block) {
   __shared__ int n_cand[kSelWarps];
-  __shared__ uint8_t cand[kSelWarps][256];
-  __shared__ double l64[kSelWarps][256];
+  __shared__ uint8_t cand[kSelWarps][32 * P];
+  __shared__ double l64[kSelWarps][32 * P];
+  __shared__ float l32[kSelWarps][32 * P], d32[kSelWarps][32 * P];  // fp32 logits and bounds of each warp's token
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = block * kSelWarps + warp;
   if (lane == 0) n_cand[warp] = 0;
   uint32_t contender = 0;  // lane's experts listed for fp64
   if (t < T) {
-    float L[kPer], D[kPer];
-    // split sums in split order, loads of a batch of 16 splits issued together
+    float L[P], D[P];
+    // split sums in split order, loads of a batch of 8 splits issued together
     float xq = 0.f;
-    for (int s0 = 0; s0 < splits; s0 += 16) {
-      float q[16];
+    for (int s0 = 0; s0 < splits; s0 += 8) {
+      float q[8];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) q[u] = s0 + u < splits ? ws.xsq[static_cast<size_t>(s0 + u) * T + t] : 0.f;
+      for (int u = 0; u < 8; ++u) q[u] = s0 + u < splits ? ws.xsq[static_cast<size_t>(s0 + u) * T + t] : 0.f;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) xq += q[u];
+      for (int u = 0; u < 8; ++u) xq += q[u];
     }
     const float xn = sqrtf(xq);
+    float* ls = l32[warp];
+    float* ds = d32[warp];
 #pragma unroll
-    for (int m = 0; m < kPer; ++m) {
+    for (int m = 0; m < P; ++m) {
       const int e = lane + 32 * m;
       L[m] = -INFINITY;
       D[m] = 0.f;
       if (e < E) {
         float v = 0.f, wq = 0.f;
-        for (int s0 = 0; s0 < splits; s0 += 16) {
-          float pv[16], qv[16];
+        for (int s0 = 0; s0 < splits; s0 += 8) {
+          float pv[8], qv[8];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
+          for (int u = 0; u < 8; ++u) {
             const bool in = s0 + u < splits;
             pv[u] = in ? ws.partial[(static_cast<size_t>(s0 + u) * T + t) * E + e] : 0.f;
             qv[u] = in ? ws.wsq[static_cast<size_t>(s0 + u) * E + e] : 0.f;
           }
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
+          for (int u = 0; u < 8; ++u) {
             v += pv[u];
             wq += qv[u];
           }
@@ -375,56 +380,91 @@ __device__ __forceinline__ void select_block(
         L[m] = v;
         D[m] = 2.0f * (gamma * xn * sqrtf(wq) * (1.0f + 0.00390625f) +
                        5.9604645e-8f * (fabsf(v) + fabsf(b))) + 1e-30f;
+        ls[e] = L[m];
+        ds[e] = D[m];
       }
     }
-    int sel[16];
+    __syncwarp();
+    int mine = 0;        // lane j < k: pick j
+    uint32_t taken = 0;  // the lane's picked experts (bit m: expert lane + 32 m)
+    bool sure = true;
     if (forced) {
-      for (int j = 0; j < k; ++j) {
-        const int e = forced[static_cast<size_t>(t) * k + j];
-        sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
+      if (lane < k) {
+        const int e = forced[static_cast<size_t>(t) * k + lane];
+        mine = e < 0 ? 0 : (e >= E ? E - 1 : e);
       }
-      write_gates(L, sel, k, t, lane, out_idx, out_w);
     } else {
-      const uint32_t taken = warp_topk(L, 0xffu, E, k, lane, sel);
+      uint32_t key[P];
+#pragma unroll
+      for (int m = 0; m < P; ++m) key[m] = lane + 32 * m < E ? order_key(L[m]) : 0u;
+      for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int m = 0; m < P; ++m)
+          if (!((taken >> m) & 1u) && key[m] > bk) {  // the lane's lowest expert on equal keys
+            bk = key[m];
+            be = lane + 32 * m;
+          }
+        const uint32_t top = __reduce_max_sync(0xffffffffu, bk);
+        int e = __reduce_min_sync(0xffffffffu, bk == top ? be : 0x7fffffff);
+        if (e >= E) e = 0;  // only when fewer than k values are comparable (NaN)
+        if (top != 0 && (e & 31) == lane) taken |= 1u << (e >> 5);
+        if (lane == j) mine = e;
+      }
+      // Certified when the order of the picks and the cut after the k-th are
+      // both wider than the bounds: pick j beats pick j + 1, and the last
+      // pick beats every other expert (comparisons with NaN are false, so
+      // non-finite values fall through to fp64).
+      float lo = INFINITY, up = -INFINITY;
+      if (lane < k) {
+        lo = ls[mine] - ds[mine];
+        up = ls[mine] + ds[mine];
+      }
+      const float lo_prev = __shfl_up_sync(0xffffffffu, lo, 1);
+      const bool ok = lane >= k || lane == 0 || lo_prev > up;
       float hi = -INFINITY;
 #pragma unroll
-      for (int m = 0; m < kPer; ++m)
+      for (int m = 0; m < P; ++m)
         if (lane + 32 * m < E && !(taken & (1u << m))) hi = fmaxf(hi, L[m] + D[m]);
 #pragma unroll
       for (int o = 16; o; o >>= 1) hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-      // Certified when the order of the picks and the cut after the k-th are
-      // both wider than the bounds: pick j beats pick j+1, and the last pick
-      // beats every other expert (comparisons with NaN are false, so
-      // non-finite values fall through to fp64).
-      bool sure = true;
-      float prev_lo = INFINITY, lo_min = INFINITY;
-      for (int j = 0; j < k; ++j) {
-        const float lj = lane_value(L, sel[j]), dj = lane_value(D, sel[j]);
-        sure = sure && (j == 0 || prev_lo > lj + dj);
-        prev_lo = lj - dj;
-        lo_min = fminf(lo_min, prev_lo);
-      }
-      if (k < E) sure = sure && prev_lo > hi;
-      else sure = sure && prev_lo == prev_lo;
-      if (sure) {
-        write_gates(L, sel, k, t, lane, out_idx, out_w);
-      } else {
+      float lo_min = lo;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) lo_min = fminf(lo_min, __shfl_xor_sync(0xffffffffu, lo_min, o));
+      const float lo_last = __shfl_sync(0xffffffffu, lo, k - 1);
+      sure = __all_sync(0xffffffffu, ok) && (k < E ? lo_last > hi : lo_last == lo_last);
+      if (!sure) {
         // contenders: picks, and every other expert whose upper bound reaches
         // the lowest pick's lower bound (all of them when a value is not finite)
         const bool finite = lo_min == lo_min && fabsf(lo_min) <= 3.0e38f;
 #pragma unroll
-        for (int m = 0; m < kPer; ++m) {
+        for (int m = 0; m < P; ++m) {
           const int e = lane + 32 * m;
           if (e < E && (!finite || (taken & (1u << m)) || !(L[m] + D[m] < lo_min))) contender |= 1u << m;
         }
         int base = 0;
 #pragma unroll
-        for (int m = 0; m < kPer; ++m) {
+        for (int m = 0; m < P; ++m) {
           const unsigned bal = __ballot_sync(0xffffffffu, (contender >> m) & 1u);
           if ((contender >> m) & 1u) cand[warp][base + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * m;
           base += __popc(bal);
         }
         if (lane == 0) n_cand[warp] = base;
+      }
+    }
+    if (sure) {  // gates: the softmax over the picks' fp32 logits, in fp32
+      const float lv = lane < k ? ls[mine] : -INFINITY;
+      float mx = lv;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float ex = lane < k ? expf(lv - mx) : 0.0f;
+      float sum = ex;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane < k) {
+        out_idx[static_cast<size_t>(t) * k + lane] = mine;
+        out_w[static_cast<size_t>(t) * k + lane] = ex / sum;
       }
     }
   }
@@ -442,12 +482,10 @@ __device__ __forceinline__ void select_block(
   }
   __syncthreads();
   if (contender_any(contender)) {
-    double v[kPer];
+    double v[P];
 #pragma unroll
-    for (int m = 0; m < kPer; ++m) v[m] = ((contender >> m) & 1u) ? l64[warp][lane + 32 * m] : -INFINITY;
-    int sel[16];
-    warp_topk(v, contender, E, k, lane, sel);
-    write_gates(v, sel, k, t, lane, out_idx, out_w);
+    for (int m = 0; m < P; ++m) v[m] = ((contender >> m) & 1u) ? l64[warp][lane + 32 * m] : -INFINITY;
+    write_gates(v, warp_topk(v, contender, E, k, lane), k, t, lane, out_idx, out_w);
   }
 }
 
@@ -461,13 +499,14 @@ size_t route_ws_for(size_t S, int T, int E) {
 // of the logits holds for any slicing, since slices are sums of 32-product
 // chunk sums).
 
+template <int P>
 __global__ void __launch_bounds__(kSelThreads, 4) k_route_select(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, RouteWs ws, int splits,
     const float* __restrict__ bias, const int32_t* __restrict__ forced, int T, int d, int E, int k,
     float gamma, int32_t* __restrict__ out_idx, float* __restrict__ out_w) {
   pdl_wait();
   pdl_trigger();
-  select_block(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, blockIdx.x);
+  select_block<P>(x, wr, ws, splits, bias, forced, T, d, E, k, gamma, out_idx, out_w, blockIdx.x);
 }
 
 int route_splits(int T, int d, int E, size_t cap = static_cast<size_t>(-1)) {
@@ -538,8 +577,10 @@ moe_status_t launch_route(const void* x, const float* w_router, const float* bia
   moe_status_t st = E <= 16 ? launch_logits<16>(xb, w_router, T, d, E, k, splits, ws, s)
                             : launch_logits<64>(xb, w_router, T, d, E, k, splits, ws, s);
   if (st != MOE_OK) return st;
-  return cuda_check(launch_pdl(pdl_for(static_cast<long>(T) * k), k_route_select, dim3(ceil_div(T, kSelWarps)), dim3(kSelThreads), 0, s, xb, w_router, ws,
-                               splits, bias, forced, T, d, E, k, route_gamma(d), idx, w),
+  auto sel = E <= 32 ? k_route_select<1> : E <= 64 ? k_route_select<2> : E <= 128 ? k_route_select<4>
+                                                                           : k_route_select<kMaxPer>;
+  return cuda_check(launch_pdl(pdl_for(static_cast<long>(T) * k), sel, dim3(ceil_div(T, kSelWarps)), dim3(kSelThreads),
+                               0, s, xb, w_router, ws, splits, bias, forced, T, d, E, k, route_gamma(d), idx, w),
                     "moe_route_topk select launch");
 }
 

@@ -500,9 +500,10 @@ def moe_debug_force_regime(regime):
 
 
 def moe_debug_route_fused(mode):
-    """Test hook: 1 (default) fp64 cluster paths for the smallest batches of
-    the router, the bit gate and moe_route_permute; 0 the fp32-with-bound
-    kernels and separate launches at every size (see moeq.h)."""
+    """Test hook: 1 (default) one cluster launch for the smallest batches of
+    the router, the bit gate and moe_route_permute; 0 the two-launch router,
+    the one-kernel bit gate and separate launches at every size (see
+    moeq.h)."""
     load().moe_debug_route_fused(int(mode))
 
 
