@@ -14,10 +14,11 @@
 // Work split: a work unit is (bin, block of weight rows, pass over 8 NB of
 // the bin's token rows): 16 features x {gate, up} in the first GEMM, 16 or
 // 32 rows of W_down in the second.  The grid is persistent (as many CTAs as
-// fit on the GPU at once); CTA b takes units b, b + grid, ...  The 8 warps
-// of a CTA split each unit's K: warp w takes the 128-K stages w, w+8, w+16,
-// ... of every row of the unit (so a 14336-long row is eight warps' work,
-// and at any time the CTA reads a contiguous K window of each row).  Each
+// fit on the GPU at once); CTA b takes units b, b + grid, ...  The W warps
+// of a CTA (8, or 12 where that balances the units better) split each
+// unit's K: warp w takes the 128-K stages w, w+W, w+2W, ... of every row of
+// the unit (so a 14336-long row is all the warps' work, and at any time the
+// CTA reads a contiguous K window of each row).  Each
 // warp streams its stages with cp.async into a shared-memory ring (the bytes
 // in flight take no registers), and the stream runs on across units: the
 // next unit's first stages are in flight while the current unit's partial
@@ -48,7 +49,6 @@
 namespace moeq {
 namespace {
 
-constexpr int kWarps = 8;
 constexpr int kStageK = 128;       // K per stage (one group of 128, two of 64)
 constexpr int kFragBytes = 1024;   // one stage of one 16-row fragment: 16 rows x 64 B
 constexpr int kSzBytes = 128;      // its scale/zero words: 16 rows x up to 2 groups
@@ -156,13 +156,13 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
 
 // Shared-memory layout of a CTA: the warps' rings, the reduction buffer,
 // the bin list.
-template <int FW, int NB>
+template <int FW, int NB, int W>
 struct Smem {
   static constexpr int kSlot = FW * (kFragBytes + kSzBytes);  // one ring stage of a warp
   static constexpr int kVals = FW * NB * 4;                    // partial sums per lane
   static constexpr int kRing0 = 0;
-  static constexpr int kRed0 = kWarps * kRing * kSlot;
-  static constexpr int kEnt0 = kRed0 + kWarps * kVals * 32 * 4;
+  static constexpr int kRed0 = W * kRing * kSlot;
+  static constexpr int kEnt0 = kRed0 + W * kVals * 32 * 4;
   static constexpr size_t bytes(int max_ent) { return kEnt0 + static_cast<size_t>(max_ent) * sizeof(BinEnt); }
 };
 
@@ -190,12 +190,15 @@ __device__ __forceinline__ void combine_rows(const DecParams& P, const int* done
 // GU: first GEMM (fragment 0 = gate rows, 1 = up rows of 16 features);
 // else the second GEMM (FW fragments of 16 consecutive W_down rows).  NB
 // token blocks of 8 per pass over K.
-// Residency: three CTAs per SM (24 warps, <= 80 registers) with one token
-// block; two with two token blocks, whose B operands need more registers.
-template <bool GU, bool PLANES, bool G64, int FW, int NB>
-__global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecParams P) {
+// Residency: 24 warps per SM (<= 80 registers) with one token block (three
+// CTAs of 8 warps or two of 12); two CTAs of 8 warps with two token blocks,
+// whose B operands need more registers.
+template <bool GU, bool PLANES, bool G64, int FW, int NB, int W>
+__global__ void __launch_bounds__(W * 32, NB == 1 && W == 8 ? 3 : 2) k_dec(const DecParams P) {
   static_assert(!GU || FW == 2, "gate and up fragments");
-  using L = Smem<FW, NB>;
+  static_assert(W == 8 || W == 12, "warps per CTA");
+  constexpr int kWarps = W;
+  using L = Smem<FW, NB, W>;
   constexpr int kSlot = L::kSlot;
   constexpr int kVals = L::kVals;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -538,40 +541,68 @@ __global__ void __launch_bounds__(kWarps * 32, NB == 1 ? 3 : 2) k_dec(const DecP
   cp_async_wait<0>();  // only empty groups remain
 }
 
-template <bool GU, bool PLANES, bool G64, int FW, int NB>
-moe_status_t run_dec(const DecParams& p, int units_upper, cudaStream_t s, const char* what) {
-  auto kern = k_dec<GU, PLANES, G64, FW, NB>;
-  const size_t smem = Smem<FW, NB>::bytes(p.max_ent);
+// CTAs of a k_dec variant resident on the device at once (found once per device).
+template <bool GU, bool PLANES, bool G64, int FW, int NB, int W>
+int resident_ctas(const char* what, moe_status_t* st) {
+  auto kern = k_dec<GU, PLANES, G64, FW, NB, W>;
   // the dynamic shared memory depends on max_ent: set the opt-in to the
-  // largest this variant can need (768 bins), once per device; the grid is
-  // the number of CTAs that fit at once (persistent), found per device
+  // largest this variant can need (768 bins), once per device
   static std::atomic<uint64_t> attr_set{0};
   static int resident[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_check(e, what);
+  if (e != cudaSuccess) { *st = cuda_check(e, what); return 0; }
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
-  const size_t smem_max = Smem<FW, NB>::bytes(768);
   if (!bit || !(attr_set.load() & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
-    if (e != cudaSuccess) return cuda_check(e, what);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(Smem<FW, NB, W>::bytes(768)));
+    if (e != cudaSuccess) { *st = cuda_check(e, what); return 0; }
     int per_sm = 0, sms = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarps * 32, Smem<FW, NB>::bytes(256));
-    if (e != cudaSuccess) return cuda_check(e, what);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, W * 32, Smem<FW, NB, W>::bytes(256));
+    if (e != cudaSuccess) { *st = cuda_check(e, what); return 0; }
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return cuda_check(e, what);
+    if (e != cudaSuccess) { *st = cuda_check(e, what); return 0; }
     if (dev < 64) resident[dev] = std::max(1, per_sm) * std::max(1, sms);
     attr_set.fetch_or(bit);
   }
-  const int fit = dev < 64 && resident[dev] > 0 ? resident[dev] : 148;
-  const int grid = std::max(1, std::min(units_upper, fit));
-  return cuda_check(launch_pdl(true, kern, dim3(grid), dim3(kWarps * 32), smem, s, p), what);
+  *st = MOE_OK;
+  return dev < 64 && resident[dev] > 0 ? resident[dev] : 148;
 }
 
+// The grid is the number of CTAs that fit at once (persistent), or fewer
+// when there are fewer units.
+template <bool GU, bool PLANES, bool G64, int FW, int NB, int W>
+moe_status_t run_dec(const DecParams& p, int units_upper, int fit, cudaStream_t s, const char* what) {
+  const int grid = std::max(1, std::min(units_upper, fit));
+  return cuda_check(launch_pdl(true, k_dec<GU, PLANES, G64, FW, NB, W>, dim3(grid), dim3(W * 32),
+                               Smem<FW, NB, W>::bytes(p.max_ent), s, p),
+                    what);
+}
+
+// Warps per CTA: a unit's K stages are split over the CTA's warps, and the
+// units over the resident CTAs; the time is about (rounds of units) x
+// (stages of the busiest warp).  With one token block both 8 warps (three
+// CTAs per SM) and 12 (two) are built, and the cheaper is taken: 12 where
+// the units come to just over a whole number of rounds of 8-warp CTAs and
+// rows are long (the Mixtral-shaped down GEMM: 512 units of 112 stages on
+// 444 or 296 CTAs, 2 x 14 against 2 x 10).
 template <bool GU, bool PLANES, bool G64, int FW>
 moe_status_t run_nb(const DecParams& p, int nb, int units_upper, cudaStream_t s, const char* what) {
-  return nb == 1 ? run_dec<GU, PLANES, G64, FW, 1>(p, units_upper, s, what)
-                 : run_dec<GU, PLANES, G64, FW, 2>(p, units_upper, s, what);
+  moe_status_t st = MOE_OK;
+  if (nb != 1) {
+    const int fit = resident_ctas<GU, PLANES, G64, FW, 2, 8>(what, &st);
+    if (st != MOE_OK) return st;
+    return run_dec<GU, PLANES, G64, FW, 2, 8>(p, units_upper, fit, s, what);
+  }
+  const int fit8 = resident_ctas<GU, PLANES, G64, FW, 1, 8>(what, &st);
+  if (st != MOE_OK) return st;
+  const int fit12 = resident_ctas<GU, PLANES, G64, FW, 1, 12>(what, &st);
+  if (st != MOE_OK) return st;
+  const int n_st = p.K / kStageK;
+  const long cost8 = static_cast<long>(ceil_div(units_upper, fit8)) * ceil_div(n_st, 8);
+  const long cost12 = static_cast<long>(ceil_div(units_upper, fit12)) * ceil_div(n_st, 12);
+  return cost12 < cost8 ? run_dec<GU, PLANES, G64, FW, 1, 12>(p, units_upper, fit12, s, what)
+                        : run_dec<GU, PLANES, G64, FW, 1, 8>(p, units_upper, fit8, s, what);
 }
 
 // units_upper: an upper bound of the work units (listed bins x passes x row
