@@ -45,7 +45,8 @@ namespace moeq {
 namespace {
 
 constexpr int kDC = 32;  // d chunk: fp32 accumulation block and shared-memory stage
-constexpr int kMT = 4;   // tokens per thread
+constexpr int kMT = 4;   // tokens per thread (one 16-byte shared-memory load of x per k)
+static_assert(kMT == 4, "x is read as float4");
 constexpr int kLT = 128; // threads of a logits CTA (4 warps)
 
 // EC experts per CTA tile (64, or 16 for E <= 16): ME per thread, TX threads
@@ -56,8 +57,8 @@ struct Tile {
   static constexpr int TX = EC / ME;
   static constexpr int TYW = 32 / TX;
   static constexpr int TT = (kLT / 32) * TYW * kMT;
-  static constexpr int XP = kDC + 1;   // x stage row pitch (floats): conflict-free
-  static constexpr int XS = TT * XP;   // floats per x stage ([token][k])
+  static constexpr int XP = TT + 4;    // x stage row pitch (floats; rows 16-byte aligned)
+  static constexpr int XS = kDC * XP;  // floats per x stage ([k][token]: a thread's kMT tokens in one 16-byte load)
   static constexpr int WS = kDC * EC;  // floats per W stage ([k][expert])
   static constexpr size_t SMEM = 2 * (XS + WS) * sizeof(float);
   static constexpr int XL = TT * 4 / kLT;   // 16-byte x loads per thread per chunk
@@ -87,7 +88,7 @@ __device__ __forceinline__ void logits_tile(const __nv_bfloat16* __restrict__ x,
                                             int T, int d, int E, int dk, RouteWs ws, int bt, int be, int split,
                                             float* sm) {
   using G = Tile<EC>;
-  float* xs = sm;               // [2][TT][XP]
+  float* xs = sm;               // [2][kDC][XP]
   float* wsm = sm + 2 * G::XS;  // [2][kDC][EC]
   const int tid = threadIdx.x, lane = tid & 31;
   const int tx = lane % G::TX;
@@ -129,8 +130,8 @@ __device__ __forceinline__ void logits_tile(const __nv_bfloat16* __restrict__ x,
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 f = __bfloat1622float2(b2[j]);
-        xb[r * G::XP + c + 2 * j] = f.x;
-        xb[r * G::XP + c + 2 * j + 1] = f.y;
+        xb[(c + 2 * j) * G::XP + r] = f.x;
+        xb[(c + 2 * j + 1) * G::XP + r] = f.y;
         if (do_x) xsq[q] = fmaf(f.x, f.x, fmaf(f.y, f.y, xsq[q]));
       }
     }
@@ -159,7 +160,7 @@ __device__ __forceinline__ void logits_tile(const __nv_bfloat16* __restrict__ x,
   for (int c = 0; c < nch; ++c) {
     const int b = c & 1;
     if (c + 1 < nch) fetch(kbeg + (c + 1) * kDC);
-    const float* xb = xs + b * G::XS + ty * kMT * G::XP;
+    const float* xb = xs + b * G::XS + ty * kMT;
     const float* wb = wsm + b * G::WS + tx * 4;
     // chunk sums, two experts per packed fp32 FMA (each lane of the pair is
     // an ordinary round-to-nearest FMA, so the error bound is unchanged)
@@ -177,10 +178,11 @@ __device__ __forceinline__ void logits_tile(const __nv_bfloat16* __restrict__ x,
         wv[j / 2] = make_float2(w4.x, w4.y);
         wv[j / 2 + 1] = make_float2(w4.z, w4.w);
       }
+      const float4 x4 = *reinterpret_cast<const float4*>(xb + kk * G::XP);  // tokens ty kMT .. + 3
+      const float xa[kMT] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
       for (int i = 0; i < kMT; ++i) {
-        const float xv = xb[i * G::XP + kk];
-        const float2 x2 = make_float2(xv, xv);
+        const float2 x2 = make_float2(xa[i], xa[i]);
 #pragma unroll
         for (int j = 0; j < G::ME / 2; ++j) cs[i][j] = __ffma2_rn(x2, wv[j], cs[i][j]);
       }
