@@ -442,10 +442,13 @@ MOE_API void moe_slot_cache_destroy(moe_slot_cache* cache);
  * what = 0 clears it. */
 MOE_API void moe_debug_inject_fault(int what, int count);
 
-/* Test hook: 0 = choose the FFN kernel by T (decode GEMV for T = 1, the
- * small-batch mma.sync kernel for 2 <= T <= 8, tensor-core grouped GEMM
- * above), 1 = always the decode GEMV, 2 = the tensor-core kernel whenever
- * the shape allows it, 3 = always the small-batch kernel.  Process-wide. */
+/* Test hook: 0 = choose the FFN kernel by T (up to 16 tokens the decode
+ * kernel -- one 8-token block per pass, or two where bins average more
+ * than 4 rows -- and the tensor-core grouped GEMM above); 1 = the decode
+ * kernel with one 8-token block per pass; 2 = the tensor-core kernel
+ * whenever the shape allows it; 3 = the decode kernel with two blocks;
+ * 4, 5 = the earlier CUDA-core GEMV and small-batch kernels (comparison
+ * only).  Process-wide. */
 MOE_API void moe_debug_force_regime(int regime);
 
 /* Test hook: when non-NULL, the tensor-core FFN kernels record each warp

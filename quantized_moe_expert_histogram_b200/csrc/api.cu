@@ -109,6 +109,14 @@ inline cudaStream_t S(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 // weight tiles, tcgen05).
 constexpr int kDecMaxT = 16;
 
+// Token blocks of the decode kernel: one 8-token block per pass over the
+// weights (three CTAs per SM) unless bins are likely to hold more than 8
+// rows, where two blocks read each weight stage once for 16 rows.  Bins
+// hold T k / E rows on average; up to 4, a second pass is rare (measured at
+// 16 tokens: OLMoE-shaped 50.9 us with one block against 55.5 with two,
+// nested 110.0 against 130.2).
+inline int decode_regime(int T, int k, int E) { return T <= 8 || static_cast<long>(T) * k <= 4L * E ? 1 : 3; }
+
 // 0: pick by T; 1: the decode kernel with one 8-token block per pass; 2:
 // tensor cores whenever possible; 3: the decode kernel with two 8-token
 // blocks; 4, 5: the earlier CUDA-core GEMV and the earlier small-batch
@@ -335,7 +343,7 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   a.status = status;
   const bool tc_ok = total_rows >= 16 && tc_supported(a);
   int regime = g_force_regime;
-  if (regime == 0) regime = T <= kDecMaxT || !tc_ok ? (T <= 8 ? 1 : 3) : 2;
+  if (regime == 0) regime = T <= kDecMaxT || !tc_ok ? decode_regime(T, std::max(1, total_rows / std::max(1, T)), E) : 2;
   if (regime == 2 && !tc_ok) regime = 3;
   if (regime == 2) return launch_ffn_tc(a, S(stream));
   if (regime == 4) return launch_ffn_gemv(a, S(stream));
@@ -376,7 +384,7 @@ moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets,
   const int total_rows = T * k;
   const size_t hbytes = workspace_for(total_rows, F);
   int regime = g_force_regime;
-  if (regime == 0) regime = T <= kDecMaxT ? (T <= 8 ? 1 : 3) : 2;
+  if (regime == 0) regime = T <= kDecMaxT ? decode_regime(T, k, E) : 2;
   if (regime == 1 || regime == 3) {  // decode kernel: the combine rides in the second GEMM's epilogue
     const BlobLayout L = blob_layout(d, F, group, layout);
     if (!L.valid) {
