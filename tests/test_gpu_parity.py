@@ -65,6 +65,45 @@ def test_route_bitexact(name, T, dup):
     np.testing.assert_allclose(w.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
 
 
+@pytest.mark.parametrize("E,k", [(1, 1), (5, 5), (31, 4), (32, 16), (33, 8), (64, 8), (65, 2), (100, 16),
+                                 (128, 7), (129, 8), (200, 1), (256, 16)])
+def test_route_every_expert_count_per_lane(E, k):
+    """The two-launch router's select kernel is built for 1, 2, 4 and 8
+    experts per lane (E up to 32, 64, 128, 256): ids bit-exact and gates
+    within the bar against the oracle at each, across the boundaries, with
+    k = E, k = 16 (the largest), exact ties (duplicated router rows) and
+    forced ids."""
+    shape = I.custom_shape(d=256, E=E, k=k, F=256, group=64)
+    T = 40  # above the one-launch sizes
+    L = I.make_layer(shape, T, seed=E + 100 * k, weights=False)
+    w = L["w_router"].clone()
+    if E >= 8:
+        w[E - 1] = w[1]
+        w[E // 2] = w[0]
+    b = None  # a bias on every other count (the duplicated rows keep equal biases)
+    if E % 2 == 0:
+        b = torch.randn(E, generator=torch.Generator().manual_seed(E)) * 0.5
+        if E >= 8:
+            b[E - 1] = b[1]
+            b[E // 2] = b[0]
+    bias = b.cuda() if b is not None else None
+    idx, gw = moeq.moe_route_topk(L["x"].cuda(), w.cuda(), bias, k)
+    torch.cuda.synchronize()
+    sel, gates, _ = O.route(L["x"].float().numpy(), w.numpy(), None if b is None else b.numpy(), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), sel)
+    np.testing.assert_allclose(gw.cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
+    rng = np.random.default_rng(E)
+    forced = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    idx2, gw2 = moeq.moe_route_topk(L["x"].cuda(), w.cuda(), bias, k, forced_idx=torch.from_numpy(forced).cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(idx2.cpu().numpy(), forced)
+    logits = L["x"].double().numpy() @ w.double().numpy().T + (0 if b is None else b.double().numpy())
+    lf = np.take_along_axis(logits, forced.astype(np.int64), axis=1)
+    ref = np.exp(lf - lf.max(axis=1, keepdims=True))
+    ref /= ref.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(gw2.cpu().numpy(), ref, rtol=GATE_RTOL, atol=GATE_ATOL)
+
+
 @pytest.mark.parametrize("name,T", [("olmoe", 1), ("olmoe", 2), ("olmoe", 8), ("olmoe", 33), ("nested", 1),
                                     ("nested", 8), ("nested", 17), ("mixtral", 1), ("mixtral", 8), ("tiny", 16),
                                     ("tiny", 64)])
