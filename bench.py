@@ -346,29 +346,49 @@ def time_graph(g, replays, warmup, stream):
 
 def time_e2e(layers, steps, stream):
     """Same steps through the public layer call with pinned host buffers:
-    H2D of x and D2H of y inside the timed region."""
+    every step's H2D of x and D2H of y inside the timed region, pipelined
+    as a serving loop would run them: step i's input copy (copy stream 1)
+    and step i-1's output copy (copy stream 2) overlap step i-1's / i's
+    layer call (the compute stream), with events ordering each buffer's
+    reuse (two device x buffers, two pinned y buffers; a layer instance's y
+    is read out before that instance runs again)."""
     import torch
     R = len(layers)
     T, d = layers[0][1].shape
     hx = [layers[r][1].cpu().pin_memory() for r in range(R)]
-    hy = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
-    dx = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    hy = [torch.empty(T, d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    dx = [torch.empty(T, d, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     hb = [layers[r][2].cpu().pin_memory() if layers[r][2] is not None else None for r in range(R)]
-    db = torch.empty_like(layers[0][2]) if layers[0][2] is not None else None
+    db = [torch.empty_like(layers[0][2]) for _ in range(2)] if layers[0][2] is not None else None
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    ev_in, ev_out, ev_cp = [ev() for _ in range(steps)], [ev() for _ in range(steps)], [ev() for _ in range(steps)]
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     h2d = T * d * 2 + (hb[0].numel() if hb[0] is not None else 0)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for i in range(steps):
-            layer = layers[i % R][0]
-            dx.copy_(hx[i % R], non_blocking=True)
+    start.record(h2d_s)
+    for i in range(steps):
+        s = i % 2
+        with torch.cuda.stream(h2d_s):  # x of step i into slot s, once step i-2 has consumed it
+            if i >= 2:
+                h2d_s.wait_event(ev_out[i - 2])
+            dx[s].copy_(hx[i % R], non_blocking=True)
             if db is not None:
-                db.copy_(hb[i % R], non_blocking=True)
-            y = layer.forward(dx, bits=db, stream=stream)
-            hy.copy_(y, non_blocking=True)
-        end.record(stream)
+                db[s].copy_(hb[i % R], non_blocking=True)
+            ev_in[i].record(h2d_s)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_in[i])
+            if i >= R:  # this instance's y of step i-R has been copied out
+                stream.wait_event(ev_cp[i - R])
+            y = layers[i % R][0].forward(dx[s], bits=None if db is None else db[s], stream=stream)
+            ev_out[i].record(stream)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(ev_out[i])
+            hy[s].copy_(y, non_blocking=True)
+            ev_cp[i].record(d2h_s)
+    d2h_s.wait_event(ev_out[steps - 1])
+    end.record(d2h_s)
     torch.cuda.synchronize()
     return start.elapsed_time(end), h2d, T * d * 2
 
