@@ -236,10 +236,9 @@ def kernel_launches(shape, T, bit_gate=False):
     T*E <= 128, T*k <= 64, d % 256 == 0); otherwise router 1 (one cluster
     launch under the same rule on T*E) or 2, bit gate 1 when used, permutation 1 (single CTA,
     with the gather when it is small) or 1 + gather, or 3 + gather; then
-    FFN 2, and the combine 1 unless the decode kernel (T <= 16) sums it in
-    its second GEMM."""
+    FFN 2 and the combine 1."""
     n = T * shape.k
-    comb = 0 if T <= 16 else 1  # the decode kernel (T <= 16) sums the combine in its second GEMM
+    comb = 1
     if T <= 8 and T * shape.E <= (128 if bit_gate else 512) and n <= 64 and shape.d % 256 == 0:
         return 1 + 2 + comb
     nbins = shape.E * (3 if shape.layout == "planes" else 1)

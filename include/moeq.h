@@ -249,10 +249,12 @@ MOE_API size_t moe_ffn_workspace_bytes(int total_rows, int E, int d, int F, int 
  *            e is blob slot_of[e]; experts with slot_of[e] < 0 are skipped
  *            (their y_perm rows are left untouched).
  *   T        token count (no bin holds more than T rows; selects the
- *            kernel: up to 16 tokens the decode kernel, which streams the
- *            weights once per 8 or 16 rows of a bin with mma.sync dot
- *            products split over warps along K; above, the tensor-core
- *            grouped GEMM with 128-row tiles)
+ *            kernel: up to 16 tokens -- and up to 64 when d >= 4096 and
+ *            bins average at most 12 rows (total_rows <= 12 nbins) -- the
+ *            decode kernel, which streams the weights once per 8 or 16
+ *            rows of a bin with mma.sync dot products split over warps
+ *            along K; otherwise the tensor-core grouped GEMM with 128-row
+ *            tiles)
  *   workspace >= moe_ffn_workspace_bytes() bytes of device scratch
  *   y_perm   fp16 [total_rows][d]
  * Accumulation is fp32; the SwiGLU intermediate h is stored as fp16 and
@@ -265,19 +267,16 @@ MOE_API moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offse
                                 moe_stream_t stream);
 
 /* moe_grouped_ffn_combine -- moe_grouped_ffn_wq (every expert resident,
- * blob e = expert e) followed by moe_unpermute_combine, with the results of
- * the two calls bit for bit (y_perm and y; [ExactMoE] every routed expert
- * runs exactly, weighted by its gate).  With the decode kernel (T <= 16)
- * the combine runs inside the second GEMM's epilogue: the work unit that
- * completes the last of a token's k expert rows for a block of output
- * columns sums that block of y[t] (same fp32 order as the separate
- * combine), so no combine launch follows; larger batches issue the two
- * calls.
+ * blob e = expert e) followed by moe_unpermute_combine on `stream`, with
+ * their results (y_perm and y; [ExactMoE] every routed expert runs exactly,
+ * weighted by its gate): one entry point for the second half of a layer
+ * step.  (Summing the combine inside the decode kernel's second GEMM was
+ * measured slower than the separate launch at every batch size.)
  *   perm, inv_perm  int32 [T*k] from moe_permute; topk_w fp32 [T][k];
- *   residual        bf16 [T][d] or NULL; y bf16 [T][d]; y_perm fp16 [T*k][d]
+ *   residual        bf16 [T][d] or NULL; y bf16 [T][d]; y_perm fp16 [T*k][d],
+ *                   all 16-byte aligned
  *   workspace >= moe_ffn_combine_workspace_bytes(T, k, E, d, F, layout),
- *   16-byte aligned (the FFN's intermediate and the combine's counters,
- *   which the call resets itself).
+ *   16-byte aligned (the FFN's scratch).
  * Requires k <= 16, d % 16 == 0; errors and flags as in the two calls. */
 MOE_API moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets, const void* blobs, int T,
                                              int k, int E, int d, int F, int group, int layout,
@@ -320,7 +319,8 @@ MOE_API moe_status_t moe_static_bits(const int32_t* topk_idx, const uint8_t* wid
  * expert's output is used as the router weighted it).
  *   y[t] = bf16( residual[t] + sum_{j<k} topk_w[t][j] * y_perm[inv_perm[t*k+j]] )
  * summed in fp32 in ascending j; y_perm fp16 [T*k][d]; residual bf16 [T][d]
- * or NULL (0).  y bf16 [T][d]; requires d % 8 == 0 and 16-byte aligned rows. */
+ * or NULL (0).  y bf16 [T][d]; requires d % 8 == 0, and y_perm, y and the
+ * residual 16-byte aligned (MOE_ERR_INVALID_ARG otherwise). */
 MOE_API moe_status_t moe_unpermute_combine(const void* y_perm, const int32_t* inv_perm,
                                    const float* topk_w, const void* residual, int T, int k, int d,
                                    void* y, moe_stream_t stream);

@@ -109,13 +109,27 @@ inline cudaStream_t S(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 // weight tiles, tcgen05).
 constexpr int kDecMaxT = 16;
 
+// Above kDecMaxT tokens the decode kernel still wins on layers with long
+// rows (d >= 4096) while bins stay short: up to 64 tokens with bins of at
+// most 12 rows on average (T k <= 12 E mult; measured FFN, decode against
+// tensor cores: Mixtral-shaped 24 tokens 242 / 340 us, 32 tokens 278 / 340,
+// 48 tokens 327 / 341, 64 tokens 423 / 342; nested 64 tokens 162 / 169).  On
+// the OLMoE-shaped layer (d = 2048: units of two stages per warp) the
+// tensor cores win from 32 tokens (71 against 79 us).
+inline bool decode_fits(int T, int k, int E, int mult, int d) {
+  return T <= kDecMaxT || (T <= 64 && d >= 4096 && static_cast<long>(T) * k <= 12L * E * mult);
+}
+
 // Token blocks of the decode kernel: one 8-token block per pass over the
 // weights (three CTAs per SM) unless bins are likely to hold more than 8
 // rows, where two blocks read each weight stage once for 16 rows.  Bins
-// hold T k / E rows on average; up to 4, a second pass is rare (measured at
-// 16 tokens: OLMoE-shaped 50.9 us with one block against 55.5 with two,
-// nested 110.0 against 130.2).
-inline int decode_regime(int T, int k, int E) { return T <= 8 || static_cast<long>(T) * k <= 4L * E ? 1 : 3; }
+// hold T k / (E mult) rows on average; up to 6, a second pass is rare
+// (measured FFN, one block against two: OLMoE-shaped 16 tokens 50.9 / 55.5
+// us, nested 16 tokens 110.0 / 130.2, Mixtral-shaped 24 tokens 242 / 272;
+// at 32 tokens, 8 rows a bin, two blocks win: 278 against 288).
+inline int decode_regime(int T, int k, int E, int mult) {
+  return T <= 8 || static_cast<long>(T) * k <= 6L * E * mult ? 1 : 3;
+}
 
 // 0: pick by T; 1: the decode kernel with one 8-token block per pass; 2:
 // tensor cores whenever possible; 3: the decode kernel with two 8-token
@@ -343,7 +357,10 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
   a.status = status;
   const bool tc_ok = total_rows >= 16 && tc_supported(a);
   int regime = g_force_regime;
-  if (regime == 0) regime = T <= kDecMaxT || !tc_ok ? decode_regime(T, std::max(1, total_rows / std::max(1, T)), E) : 2;
+  if (regime == 0) {
+    const int k = std::max(1, total_rows / std::max(1, T)), mult = layout == MOE_LAYOUT_PLANES ? 3 : 1;
+    regime = decode_fits(T, k, E, mult, d) || !tc_ok ? decode_regime(T, k, E, mult) : 2;
+  }
   if (regime == 2 && !tc_ok) regime = 3;
   if (regime == 2) return launch_ffn_tc(a, S(stream));
   if (regime == 4) return launch_ffn_gemv(a, S(stream));
@@ -353,11 +370,19 @@ moe_status_t moe_grouped_ffn_wq(const void* x_perm, const int32_t* offsets, cons
 
 size_t moe_ffn_combine_workspace_bytes(int T, int k, int E, int d, int F, int layout) {
   (void)E;
+  (void)d;
   (void)layout;
-  if (T <= 0 || k <= 0 || d <= 0 || F <= 0) return 256;
-  return workspace_for(T * k, F) + ((static_cast<size_t>(T) * (d / 16) * sizeof(int32_t) + 255) & ~size_t(255));
+  if (T <= 0 || k <= 0 || F <= 0) return 256;
+  return workspace_for(T * k, F);
 }
 
+// The FFN call, then the combine launch.  Summing the combine inside the
+// decode kernel's second GEMM (the unit that completes a token's k rows of
+// an output block adds them, after a fence and a count) was built and
+// measured slower at every size (layer step, fused against separate:
+// OLMoE-shaped 1 token 29.5 / 27.9 us, 16 tokens 79.4 / 72.7; nested 64
+// tokens 220.1 / 199.2; Mixtral-shaped 32 tokens 312.6 / 300.6): the fence
+// and barriers each unit pays outweigh the launch.
 moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets, const void* blobs, int T, int k,
                                      int E, int d, int F, int group, int layout, const int32_t* perm,
                                      const int32_t* inv_perm, const float* topk_w, const void* residual, void* y,
@@ -372,6 +397,10 @@ moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets,
     set_error("moe_grouped_ffn_combine: null pointer");
     return MOE_ERR_INVALID_ARG;
   }
+  if (!aligned16(y) || (residual && !aligned16(residual))) {  // the combine's 16-byte loads and stores
+    set_error("moe_grouped_ffn_combine: y and residual must be 16-byte aligned");
+    return MOE_ERR_INVALID_ARG;
+  }
   if (static_cast<long>(T) * k > (1L << 24)) {
     set_error("moe_grouped_ffn_combine: T*k exceeds 2^24");
     return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -381,56 +410,8 @@ moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets,
     set_error("moe_grouped_ffn_combine: workspace %zu < %zu bytes", workspace_bytes, need);
     return MOE_ERR_WORKSPACE;
   }
-  const int total_rows = T * k;
-  const size_t hbytes = workspace_for(total_rows, F);
-  int regime = g_force_regime;
-  if (regime == 0) regime = T <= kDecMaxT ? decode_regime(T, k, E) : 2;
-  if (regime == 1 || regime == 3) {  // decode kernel: the combine rides in the second GEMM's epilogue
-    const BlobLayout L = blob_layout(d, F, group, layout);
-    if (!L.valid) {
-      set_error("moe_grouped_ffn_combine: unsupported shape d=%d F=%d group=%d layout=%d", d, F, group, layout);
-      return MOE_ERR_UNSUPPORTED_SHAPE;
-    }
-    if (!x_perm || !offsets || !blobs || !y_perm) {
-      set_error("moe_grouped_ffn_combine: null pointer");
-      return MOE_ERR_INVALID_ARG;
-    }
-    if (!aligned16(x_perm) || !aligned16(blobs) || !aligned16(workspace) || !aligned16(y_perm)) {
-      set_error("moe_grouped_ffn_combine: buffers must be 16-byte aligned");
-      return MOE_ERR_INVALID_ARG;
-    }
-    if (E * (layout == MOE_LAYOUT_PLANES ? 3 : 1) > 768) {
-      set_error("moe_grouped_ffn_combine: too many bins");
-      return MOE_ERR_UNSUPPORTED_SHAPE;
-    }
-    FfnArgs a{};
-    a.x_perm = static_cast<const __half*>(x_perm);
-    a.offsets = offsets;
-    a.blobs = static_cast<const uint8_t*>(blobs);
-    a.slot_of = nullptr;
-    a.total_rows = total_rows;
-    a.T = T;
-    a.E = E;
-    a.d = d;
-    a.F = F;
-    a.group = group;
-    a.layout = layout;
-    a.blob_bytes = L.bytes;
-    a.lay = L;
-    a.h = static_cast<__half*>(workspace);
-    a.y_perm = static_cast<__half*>(y_perm);
-    a.status = status;
-    a.k = k;
-    a.perm = perm;
-    a.inv_perm = inv_perm;
-    a.topk_w = topk_w;
-    a.residual = static_cast<const __nv_bfloat16*>(residual);
-    a.y = static_cast<__nv_bfloat16*>(y);
-    a.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + hbytes);
-    return launch_ffn_decode(a, regime == 1 ? 1 : 2, S(stream));
-  }
-  moe_status_t st = moe_grouped_ffn_wq(x_perm, offsets, blobs, nullptr, total_rows, T, E, d, F, group, layout,
-                                       workspace, hbytes, y_perm, status, stream);
+  moe_status_t st = moe_grouped_ffn_wq(x_perm, offsets, blobs, nullptr, T * k, T, E, d, F, group, layout,
+                                       workspace, workspace_bytes, y_perm, status, stream);
   if (st != MOE_OK) return st;
   return moe_unpermute_combine(y_perm, inv_perm, topk_w, residual, T, k, d, y, stream);
 }
@@ -488,6 +469,10 @@ moe_status_t moe_unpermute_combine(const void* y_perm, const int32_t* inv_perm,
   }
   if (T > 0 && (!y_perm || !inv_perm || !topk_w || !y)) {
     set_error("moe_unpermute_combine: null pointer");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (!aligned16(y_perm) || !aligned16(y) || (residual && !aligned16(residual))) {  // 16-byte loads and stores
+    set_error("moe_unpermute_combine: y_perm, y and residual must be 16-byte aligned");
     return MOE_ERR_INVALID_ARG;
   }
   return launch_combine(y_perm, inv_perm, topk_w, residual, T, k, d, y, S(stream));

@@ -468,14 +468,6 @@ struct FfnArgs {
   __half* h;          // workspace: fp16 [total_rows][F]
   __half* y_perm;  // [total_rows][d]
   int32_t* status;
-  // weighted combine fused into the second GEMM (decode kernel), or y null
-  int k = 0;
-  const int32_t* perm = nullptr;
-  const int32_t* inv_perm = nullptr;
-  const float* topk_w = nullptr;
-  const __nv_bfloat16* residual = nullptr;
-  __nv_bfloat16* y = nullptr;
-  int32_t* counters = nullptr;  // workspace: int32 [T][d/16]
 };
 moe_status_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t s);
 moe_status_t launch_ffn_gemv_mma(const FfnArgs& a, cudaStream_t s);

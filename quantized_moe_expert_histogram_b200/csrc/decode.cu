@@ -71,16 +71,6 @@ struct DecParams {
   int max_ent;              // capacity of the bin list (>= non-empty bins)
   __half* out;              // h (gate/up) or y_perm (down): fp16 [rows][N]
   int32_t* status;
-  // fused combine (down pass): y[t][n] = bf16(res[t][n] + sum_j g[t][j] y_perm[inv_perm[t k + j]][n]),
-  // taken by the unit that completes token t's row block; counters [T][row_blocks] zeroed by the gate/up pass
-  int k;
-  const int32_t* perm;
-  const int32_t* inv_perm;
-  const float* topk_w;
-  const __nv_bfloat16* residual;
-  __nv_bfloat16* y;
-  int32_t* counters;
-  int n_counters;           // gate/up pass: counters to zero
 };
 
 // One listed bin: its rows, blob, width and its first work unit.
@@ -166,27 +156,6 @@ struct Smem {
   static constexpr size_t bytes(int max_ent) { return kEnt0 + static_cast<size_t>(max_ent) * sizeof(BinEnt); }
 };
 
-// The fused combine of the down pass: for each token t this unit completed
-// (done[i] >= 0), the rows n0 .. n0 + R - 1 of y[t], summed exactly as the
-// separate combine does (fp32: the residual, then g_j * y_perm row of
-// choice j for ascending j; bf16 rounding once).  y_perm rows written by
-// other CTAs are read from L2.
-__device__ __forceinline__ void combine_rows(const DecParams& P, const int* done, int ntok, int n0, int R) {
-  for (int v = threadIdx.x; v < ntok * R; v += blockDim.x) {
-    const int i = v / R, col = n0 + (v - i * R);
-    const int t = done[i];
-    if (t < 0) continue;
-    float acc = P.residual ? __bfloat162float(P.residual[static_cast<size_t>(t) * P.N + col]) : 0.0f;
-    for (int j = 0; j < P.k; ++j) {
-      const float g = P.topk_w[static_cast<size_t>(t) * P.k + j];
-      const int pr = min(max(P.inv_perm[static_cast<size_t>(t) * P.k + j], 0), P.rows - 1);
-      const unsigned short raw = __ldcg(reinterpret_cast<const unsigned short*>(P.out) + static_cast<size_t>(pr) * P.N + col);
-      acc = fmaf(g, __half2float(__ushort_as_half(raw)), acc);
-    }
-    P.y[static_cast<size_t>(t) * P.N + col] = __float2bfloat16_rn(acc);
-  }
-}
-
 // GU: first GEMM (fragment 0 = gate rows, 1 = up rows of 16 features);
 // else the second GEMM (FW fragments of 16 consecutive W_down rows).  NB
 // token blocks of 8 per pass over K.
@@ -210,10 +179,6 @@ __global__ void __launch_bounds__(W * 32, NB == 1 && W == 8 ? 3 : 2) k_dec(const
   if (GU) {  // x_perm comes from the previous launch
     pdl_wait();
     pdl_trigger();
-    // the down pass's combine counters start from zero (the down pass reads
-    // them only after this grid has completed)
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P.n_counters; i += gridDim.x * blockDim.x)
-      P.counters[i] = 0;
   }
   // ---- the non-empty, resident bins and their work units (warp 0): units
   // of a bin = passes x row blocks, passes = ceil(rows / (8 NB))
@@ -522,20 +487,6 @@ __global__ void __launch_bounds__(W * 32, NB == 1 && W == 8 ? 3 : 2) k_dec(const
         }
       }
     }
-    if (!GU && P.y) {  // fused combine (CTA-uniform)
-      __shared__ int done_s[16];  // token completed by this unit, or -1
-      __threadfence();            // this unit's y_perm rows before its counts
-      __syncthreads();
-      if (threadIdx.x < ntok) {
-        const int pr = min(be.row0 + t0 + static_cast<int>(threadIdx.x), P.rows - 1);
-        const int t = min(max(P.perm[pr], 0), P.rows - 1) / P.k;
-        const int old = atomicAdd(&P.counters[t * P.row_blocks + rb], 1);
-        done_s[threadIdx.x] = old == P.k - 1 ? t : -1;
-        if (old == P.k - 1) __threadfence();  // the other units' rows, read below
-      }
-      __syncthreads();
-      combine_rows(P, done_s, ntok, n0, rows_per_unit);
-    }
     __syncthreads();  // the reduction buffer is reused by the next unit
   }
   cp_async_wait<0>();  // only empty groups remain
@@ -665,16 +616,7 @@ moe_status_t launch_ffn_decode(const FfnArgs& a, int token_blocks, cudaStream_t 
   const int max_bins = std::min(gu.nbins, a.total_rows);
   if (max_bins == 0) return MOE_OK;
   gu.max_ent = max_bins;  // no more bins than rows are non-empty
-  gu.k = a.k;
-  gu.n_counters = a.y ? a.T * (a.d / 16) : 0;
-  gu.counters = a.counters;
   DecParams dn = gu;
-  dn.n_counters = 0;
-  dn.perm = a.perm;
-  dn.inv_perm = a.inv_perm;
-  dn.topk_w = a.topk_w;
-  dn.residual = a.residual;
-  dn.y = a.y;
   dn.act = a.h;
   dn.K = a.F;
   dn.N = a.d;

@@ -1,11 +1,11 @@
 """The grouped FFN and the weighted combine in one call
 (moe_grouped_ffn_combine; ExactMoE: every routed expert runs exactly,
-weighted by its gate).  With the decode kernel the combine is summed in the
-second GEMM's epilogue by whichever work unit completes a token's rows; y
-and y_perm must equal the separate calls' (moe_grouped_ffn_wq, then
-moe_unpermute_combine) bit for bit, for every batch size, with and without
-a residual, with nested widths, and when a token names one expert twice
-(a bin holding more rows than there are tokens)."""
+weighted by its gate): y and y_perm must equal the separate calls'
+(moe_grouped_ffn_wq, then moe_unpermute_combine) bit for bit, for every
+batch size and kernel (decode kernel with one or two token blocks, tensor
+cores), with and without a residual, with nested widths, and when a token
+names one expert twice (a bin holding more rows than there are tokens);
+misaligned rows are refused."""
 import numpy as np
 import pytest
 import torch
@@ -52,7 +52,7 @@ def _run(shape, T, seed, residual=True, forced=None, bits=None):
 
 @pytest.mark.parametrize("name,T", [("olmoe", 1), ("olmoe", 2), ("olmoe", 8), ("olmoe", 9), ("olmoe", 16),
                                     ("mixtral", 1), ("mixtral", 8), ("nested", 1), ("nested", 4), ("nested", 16),
-                                    ("tiny", 3), ("olmoe", 32)])
+                                    ("tiny", 3), ("olmoe", 32), ("mixtral", 24), ("mixtral", 48), ("nested", 64)])
 def test_ffn_combine_equals_separate_calls(name, T):
     shape = I.SHAPES[name]
     y_f, yp_f, y_s, yp_s = _run(shape, T, seed=61 + T)
@@ -116,3 +116,29 @@ def test_long_rows_against_oracle_and_slot_path(T, layout):
     torch.cuda.synchronize()
     assert torch.equal(y_off, y_res)
     cache.close()
+
+
+def test_ffn_combine_and_combine_reject_misaligned_rows():
+    """y, the residual and y_perm are read and written 16 bytes at a time:
+    a pointer off a 16-byte boundary is refused on the host (before any
+    launch), by both entry points."""
+    shape = I.SHAPES["tiny"]
+    T = 4
+    L = I.make_layer(shape, T, seed=31)
+    layer = QuantMoELayer.from_weights(shape, L["w_router"].cuda(), None, L["w_gate"].cuda(), L["w_up"].cuda(),
+                                       L["w_down"].cuda(), max_tokens=T)
+    x = L["x"].cuda()
+    v = layer.views(T)
+    moeq.moe_route_permute(x, layer.w_router, None, shape.k, out=v, status=v["status"], workspace=v["rp_ws"])
+    torch.cuda.synchronize()
+    y_off = torch.empty(T * shape.d + 8, dtype=torch.bfloat16, device="cuda")[1:1 + T * shape.d].view(T, shape.d)
+    with pytest.raises(moeq.MoeError) as ei:
+        moeq.moe_grouped_ffn_combine(v["x_perm"], v["offsets"], layer.blobs, T, shape.k, shape.E, shape.d,
+                                     shape.F, shape.group, layer.layout, v["perm"], v["inv_perm"], v["topk_w"],
+                                     residual=x, y=y_off)
+    assert ei.value.code == 1
+    yp = torch.zeros(T * shape.k, shape.d, dtype=torch.float16, device="cuda")
+    with pytest.raises(moeq.MoeError) as ei:
+        moeq.moe_unpermute_combine(yp, v["inv_perm"], v["topk_w"], residual=x, y=y_off)
+    assert ei.value.code == 1
+
