@@ -36,6 +36,12 @@
 // decided after that round: on the fp32 scores when certified, otherwise by
 // CTA 0 alone in fp64 (an open assignment of an open token).
 //
+// Permutation and gather.  When nothing was left open, CTA 0 sends the
+// final picks (and widths) with the empty list; every CTA then ranks the
+// assignments itself (counting, na <= 64) and gathers its eighth of the
+// (row, 8-element piece) items, CTA 0 alone writing perm, inv_perm, counts
+// and offsets.  After an fp64 round CTA 0 does both alone.
+//
 // Shared-memory rule of the cluster: a CTA writes into another CTA's shared
 // memory only before a cluster barrier that the owner also waits at, and no
 // CTA reads another CTA's shared memory.
@@ -196,10 +202,20 @@ __device__ __forceinline__ void front_dots64(const FrontArgs& A, int TE, const i
 }
 
 // CTA 0: every CTA's copy of the list and its length, written before the
-// barrier that follows.
-__device__ __forceinline__ void front_publish_list(FrontSmem& S, int n) {
+// barrier that follows; when the list is empty the picks and, with a bit
+// gate, the widths are final, and every CTA gets them too (the permutation
+// is then computed by each CTA and the gather split over the cluster).
+__device__ __forceinline__ void front_publish_list(FrontSmem& S, int n, int na, bool widths) {
   for (int r = 1; r < kFC; ++r) {
     for (int i = threadIdx.x; i < n; i += blockDim.x) st_cluster_u32(cluster_map_shared(&S.list[i], r), S.list[i]);
+    if (n == 0) {
+      for (int i = threadIdx.x; i < na; i += blockDim.x)
+        st_cluster_u32(cluster_map_shared(&S.sel[i], r), static_cast<uint32_t>(S.sel[i]));
+      const uint32_t* b4 = reinterpret_cast<const uint32_t*>(S.bits);
+      if (widths)
+        for (int i = threadIdx.x; i < (na + 3) / 4; i += blockDim.x)
+          st_cluster_u32(cluster_map_shared(&b4[i], r), b4[i]);
+    }
     if (threadIdx.x == 0) st_cluster_u32(cluster_map_shared(&S.n_list, r), n);
   }
 }
@@ -385,7 +401,7 @@ __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ Fro
       }
     }
     __syncthreads();
-    front_publish_list(S, S.n_list);
+    front_publish_list(S, S.n_list, na, gate);
   }
   cluster_sync_publish();  // the list is in every CTA
   const int nl = S.n_list;
@@ -456,9 +472,14 @@ __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ Fro
       }
     }
   }
-  if (rank != 0 || !A.counts) return;
+  if (!A.counts) return;
+  // with nothing open every CTA holds the final picks (and widths): each
+  // computes the permutation and gathers its share of the rows; otherwise
+  // CTA 0, which decided the open items, does it all
+  const int nct = nl == 0 ? kFC : 1;
+  if (rank >= nct) return;
   __syncthreads();  // picks and widths complete
-  // ---- 4. permutation of the na assignments (CTA 0)
+  // ---- 4. permutation of the na assignments
   const bool nested = gate || A.bits_in;
   const int nbins = nested ? 3 * E : E;
   for (int a = threadIdx.x; a < na; a += blockDim.x) {
@@ -466,7 +487,7 @@ __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ Fro
     if (nested) {
       int b = gate ? S.bits[a] : A.bits_in[a];
       if (b < 2 || b > 4) {
-        flag_status(A.status, MOE_DEV_BAD_INDEX);
+        if (rank == 0) flag_status(A.status, MOE_DEV_BAD_INDEX);
         b = b < 2 ? 2 : 4;
       }
       key = 3 * key + (b - 2);
@@ -481,11 +502,13 @@ __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ Fro
       const int ko = S.key[o];
       pos += (ko < key || (ko == key && o < a)) ? 1 : 0;
     }
-    A.perm[pos] = a;
-    A.inv_perm[a] = pos;
+    if (rank == 0) {
+      A.perm[pos] = a;
+      A.inv_perm[a] = pos;
+    }
     S.perm[pos] = a;
   }
-  for (int b = threadIdx.x; b <= nbins; b += blockDim.x) {
+  for (int b = threadIdx.x; rank == 0 && b <= nbins; b += blockDim.x) {
     int below = 0, at = 0;
     for (int o = 0; o < na; ++o) {
       below += S.key[o] < b ? 1 : 0;
@@ -496,10 +519,11 @@ __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ Fro
   }
   if (!A.x_perm) return;
   __syncthreads();  // S.perm complete
-  // gather: all threads over (row, 8-element piece), bf16 -> fp16
+  // gather: (row, 8-element piece) items split over the nct CTAs and their
+  // threads, bf16 -> fp16
   const int vec = A.d / 8;
   bool bad = false;
-  for (int v = threadIdx.x; v < na * vec; v += blockDim.x) {
+  for (int v = rank * blockDim.x + threadIdx.x; v < na * vec; v += nct * blockDim.x) {
     const int p = v / vec, c = v - p * vec;
     const uint4 in = reinterpret_cast<const uint4*>(A.x + static_cast<size_t>(S.perm[p] / k) * A.d)[c];
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&in);
