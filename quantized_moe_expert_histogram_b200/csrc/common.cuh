@@ -60,6 +60,13 @@ __device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
   return r;
 }
 
+// Order-preserving unsigned key of an fp32 value (a > b gives key(a) >
+// key(b); -0 sorts below +0); NaN gets 0, below every other key.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return v == v ? ((b & 0x80000000u) ? ~b : (b | 0x80000000u)) : 0u;
+}
+
 // SiLU in fp32: v / (1 + exp(-v)).
 __device__ __forceinline__ float silu_f(float v) { return v / (1.0f + __expf(-v)); }
 

@@ -21,9 +21,11 @@
 // the bias in fp32 (kFC more additions), so with g = g(m + kFC + 1)
 //     |L - l| <= D = 2 g (A (1 + 2^-8) + |b|)      (factor 2: margin).
 //
-// Decisions (CTA 0, all its threads).  Router: ranks by counting (top k,
-// ties to the lower index), certified per token when consecutive picks and
-// the cut after the k-th are separated by more than their bounds.  Gate: the
+// Decisions (CTA 0).  Router: a warp per token picks the top k one at a
+// time by warp reductions over order keys of the logits (ties to the lower
+// index), lane j holding pick j, and certifies the token when consecutive
+// picks and the cut after the k-th are separated by more than their
+// bounds.  Gate: the
 // first maximum of the three widths of each chosen expert (ties to the
 // narrower width), certified when the winner's lower bound clears the
 // others' upper bounds.  What is left open -- the contenders of an open
@@ -97,10 +99,7 @@ struct FrontSmem {
   int32_t key[kFMaxTK];
   int32_t perm[kFMaxTK];
   uint8_t bits[kFMaxTK];
-  int32_t comparable[8];          // per token: logits that are not NaN
   int32_t open[8];                // per token: not certified
-  float lo_k[8], lo_min[8];
-  int32_t finite[8];
   int32_t n_list;
   int32_t n_open;
 };
@@ -277,9 +276,17 @@ __device__ __forceinline__ void front_set_width(const FrontArgs& A, FrontSmem& S
 __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ FrontArgs A) {
   extern __shared__ __align__(16) uint8_t front_smem[];
   FrontSmem& S = *reinterpret_cast<FrontSmem*>(front_smem);
+  const int rank = blockIdx.x;  // the grid is one cluster
+  // CTA 0's biases of the logits it sums (items threadIdx.x and + 256; T E
+  // <= 512), read before the wait: no kernel of the path writes them
+  float bias0 = 0.0f, bias1 = 0.0f;
+  if (rank == 0 && A.bias) {
+    const int te = A.T * A.E;
+    if (static_cast<int>(threadIdx.x) < te) bias0 = A.bias[threadIdx.x % A.E];
+    if (static_cast<int>(threadIdx.x) + kFThreads < te) bias1 = A.bias[(threadIdx.x + kFThreads) % A.E];
+  }
   pdl_wait();
   pdl_trigger();
-  const int rank = blockIdx.x;  // the grid is one cluster
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = A.T, E = A.E, k = A.k, TE = T * E, na = T * k, dk = A.d / kFC;
   const bool gate = A.wbit != nullptr;
@@ -292,22 +299,18 @@ __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ Fro
   // ---- 2. decisions on the fp32 values (CTA 0)
   if (rank == 0) {
     for (int i = threadIdx.x; i < TE; i += blockDim.x) {
-      const int t = i / E, e = i - t * E;
       float L = 0.0f, m = 0.0f;
       for (int r = 0; r < kFC; ++r) {
         const float2 p = S.p32[r * nitems + i];
         L += p.x;
         m += p.y;
       }
-      const float b = A.bias ? A.bias[e] : 0.0f;
+      const float b = i < kFThreads ? bias0 : bias1;
       S.val[i] = L + b;
       S.dev[i] = 2.0f * A.gamma * (m * (1.0f + 0.00390625f) + fabsf(b)) + 1e-30f;
     }
     for (int i = threadIdx.x; i < nitems; i += blockDim.x) S.lpos[i] = -1;
-    if (threadIdx.x < T) {
-      S.comparable[threadIdx.x] = 0;
-      S.open[threadIdx.x] = 0;
-    }
+    if (threadIdx.x < T) S.open[threadIdx.x] = 0;
     if (threadIdx.x == 0) S.n_open = 0;
     __syncthreads();
     if (A.forced) {
@@ -315,67 +318,79 @@ __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ Fro
         const int e = A.forced[j];
         S.sel[j] = e < 0 ? 0 : (e >= E ? E - 1 : e);
       }
-    } else {
-      // ranks: thread per (token, expert); NaN logits are never picked
-      for (int i = threadIdx.x; i < TE; i += blockDim.x) {
-        const int t = i / E, e = i - t * E;
-        const float v = S.val[i];
-        if (v != v) continue;
-        atomicAdd(&S.comparable[t], 1);
-        const float* row = S.val + t * E;
-        int r = 0;
-        for (int o = 0; o < E; ++o) {
-          const float u = row[o];
-          r += (u > v || (u == v && o < e)) ? 1 : 0;
-        }
-        if (r < k) S.sel[t * k + r] = e;
-      }
-      __syncthreads();
-      // fewer than k comparable logits: the remaining picks are expert 0
-      for (int j = threadIdx.x; j < na; j += blockDim.x) {
-        const int t = j / k;
-        if (j - t * k >= S.comparable[t]) S.sel[j] = 0;
-      }
-      __syncthreads();
-      // per token: the k-th pick's lower bound and the lowest pick lower bound
-      if (threadIdx.x < T) {
-        const int t = threadIdx.x;
-        float lo_min = INFINITY, lo = INFINITY;
-        int fin = 1;
-        for (int j = 0; j < k; ++j) {
-          const int e = S.sel[t * k + j];
-          lo = S.val[t * E + e] - S.dev[t * E + e];
-          fin = fin && lo == lo && fabsf(lo) <= 3.0e38f;
-          lo_min = fminf(lo_min, lo);
-          if (j > 0) {  // pick j-1 beats pick j by more than both bounds
-            const int ep = S.sel[t * k + j - 1];
-            if (!(S.val[t * E + ep] - S.dev[t * E + ep] > S.val[t * E + e] + S.dev[t * E + e])) S.open[t] = 1;
+    } else if (warp < T) {
+      // warp t decides token t, lane j holding pick j; its experts lane + 32 m
+      const int t = warp, P = (E + 31) >> 5;
+      const float* lv = S.val + t * E;
+      const float* dv = S.dev + t * E;
+      // top k, one pick per round: the largest order key (NaN never picked),
+      // then the lowest expert holding it; expert 0 where fewer than k
+      // logits are comparable
+      uint32_t taken = 0;
+      int mine = 0;
+      for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0;
+        int be = 0x7fffffff;
+        for (int m = 0; m < P; ++m) {
+          const int e = lane + 32 * m;
+          if (e < E && !((taken >> m) & 1u)) {
+            const uint32_t key = order_key(lv[e]);
+            if (key > bk) {
+              bk = key;
+              be = e;
+            }
           }
         }
-        S.lo_k[t] = lo;
-        S.lo_min[t] = lo_min;
-        S.finite[t] = fin;
-        if (!fin) S.open[t] = 1;
+        const uint32_t top = __reduce_max_sync(0xffffffffu, bk);
+        int e = __reduce_min_sync(0xffffffffu, bk == top ? be : 0x7fffffff);
+        if (top == 0) e = 0;
+        else if ((e & 31) == lane) taken |= 1u << (e >> 5);
+        if (lane == j) mine = e;
       }
-      __syncthreads();
-      // the cut: every expert not picked stays below the k-th pick's lower bound
-      for (int i = threadIdx.x; i < TE; i += blockDim.x) {
-        const int t = i / E, e = i - t * E;
-        bool picked = false;
-        for (int j = 0; j < k; ++j) picked = picked || S.sel[t * k + j] == e;
-        if (!picked && !(S.val[i] + S.dev[i] < S.lo_k[t])) S.open[t] = 1;
+      if (lane < k) S.sel[t * k + lane] = mine;
+      // certified when consecutive picks are separated by more than their
+      // bounds, every pick's lower bound is finite, and every expert not
+      // picked stays below the k-th pick's lower bound (NaN: not certified)
+      float lo = INFINITY, up = -INFINITY;
+      if (lane < k) {
+        lo = lv[mine] - dv[mine];
+        up = lv[mine] + dv[mine];
       }
-      __syncthreads();
-      // contenders of the open tokens
-      for (int i = threadIdx.x; i < TE; i += blockDim.x) {
-        const int t = i / E, e = i - t * E;
-        if (!S.open[t]) continue;
-        bool picked = false;
-        for (int j = 0; j < k; ++j) picked = picked || S.sel[t * k + j] == e;
-        if (!S.finite[t] || picked || !(S.val[i] + S.dev[i] < S.lo_min[t])) {
-          const int p = atomicAdd(&S.n_list, 1);
-          S.list[p] = i;
-          S.lpos[i] = p;
+      const float lo_prev = __shfl_up_sync(0xffffffffu, lo, 1);
+      const bool order_bad = lane > 0 && lane < k && !(lo_prev > up);
+      const bool fin = __all_sync(0xffffffffu, lane >= k || (lo == lo && fabsf(lo) <= 3.0e38f));
+      float lo_min = lo;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) lo_min = fminf(lo_min, __shfl_xor_sync(0xffffffffu, lo_min, o));
+      const float lo_k = __shfl_sync(0xffffffffu, lo, k - 1);
+      bool cut_bad = false;
+      for (int m = 0; m < P; ++m) {
+        const int e = lane + 32 * m;
+        if (e < E && !((taken >> m) & 1u) && !(lv[e] + dv[e] < lo_k)) cut_bad = true;
+      }
+      const bool open = __any_sync(0xffffffffu, order_bad || cut_bad) || !fin;
+      if (lane == 0) S.open[t] = open ? 1 : 0;
+      if (open) {
+        // contenders: its picks and every expert whose upper bound reaches the
+        // lowest pick's lower bound (all of them when a bound is not finite)
+        __syncwarp();
+        for (int m = 0; m < P; ++m) {
+          const int e = lane + 32 * m;
+          bool c = false;
+          if (e < E) {
+            bool picked = false;
+            for (int j = 0; j < k; ++j) picked = picked || S.sel[t * k + j] == e;
+            c = !fin || picked || !(lv[e] + dv[e] < lo_min);
+          }
+          const unsigned bal = __ballot_sync(0xffffffffu, c);
+          int base = 0;
+          if (lane == 0 && bal) base = atomicAdd(&S.n_list, __popc(bal));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (c) {
+            const int p = base + __popc(bal & ((1u << lane) - 1u));
+            S.list[p] = t * E + e;
+            S.lpos[t * E + e] = p;
+          }
         }
       }
     }

@@ -310,13 +310,6 @@ __device__ __forceinline__ void write_gates(const V (&v)[P], int mine, int k, in
   }
 }
 
-// Order-preserving unsigned key of an fp32 value (a > b gives key(a) >
-// key(b); -0 sorts below +0); NaN gets 0, below every other key.
-__device__ __forceinline__ uint32_t order_key(float v) {
-  const uint32_t b = __float_as_uint(v);
-  return v == v ? ((b & 0x80000000u) ? ~b : (b | 0x80000000u)) : 0u;
-}
-
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 
