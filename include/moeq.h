@@ -96,6 +96,13 @@ MOE_API const char* moe_last_error(void);
  *           | gate D4 | up D4 | down D4 -- width by width, so that what a
  *           b-bit read needs (Q2 and the scales; D3 from b = 3; D4 at 4)
  *           is the blob's first bytes
+ * Code words are stored in tiles of 16 rows x 128 K: a region of N rows
+ * holds, for each block of 16 rows and each run of 128 K in order, the 16
+ * rows' words of that run one row after another (16 words a row for INT4
+ * codes, 8 for Q2, 4 for D3 and D4); word w of row n is at index
+ * ((n / 16) * (K / 128) + w / per) * 16 per + (n % 16) per + w % per.  A
+ * 16-row stage of 128 K is thus one contiguous 1 KB (INT4), 512 B (Q2) or
+ * 256 B (D3, D4).
  * Code word packing: nibble i of an INT4 codes word = element 8w+i (low
  * nibble first).  Planes use the plane order, n(i) = (i >> 1) + 4 (i & 1)
  * for element i of a run of 8 (even elements in nibbles 0..3, odd ones in

@@ -195,6 +195,9 @@ def blob_layout(d: int, F: int, group: int, layout: str) -> dict:
 
     INT4: [gate codes F x d/8 u32 | up codes F x d/8 | down codes d x F/8 |
            gate sz | up sz | down sz]
+    Code words (INT4 codes, Q2, D3, D4) are stored in tiles of 16 rows x 128
+    elements: a tile's rows one after another (16, 8 or 4 words a row), the
+    tiles of 16-row block r in K order, then block r + 1 (tile_words).
     planes: [gate Q2 F x d/16 u32 | up Q2 | down Q2 d x F/16 | gate sz | up sz
              | down sz | gate D3 F x d/32 | up D3 | down D3 | gate D4 | up D4
              | down D4]  (bit order inside the words: split_planes).  Width by
@@ -227,6 +230,20 @@ def blob_layout(d: int, F: int, group: int, layout: str) -> dict:
     return off
 
 
+def tile_words(words: np.ndarray, per: int) -> np.ndarray:
+    """uint32 [N, W] (N rows of W words, `per` words per 128 elements) ->
+    the blob's order: for each block of 16 rows, for each run of 128
+    elements, the 16 rows' `per` words one row after another."""
+    N, W = words.shape
+    return np.ascontiguousarray(words.reshape(N // 16, 16, W // per, per).transpose(0, 2, 1, 3)).reshape(-1)
+
+
+def untile_words(flat: np.ndarray, N: int, W: int, per: int) -> np.ndarray:
+    """Inverse of tile_words: the blob's words -> uint32 [N, W]."""
+    t = np.asarray(flat, dtype=np.uint32).reshape(N // 16, W // per, 16, per)
+    return np.ascontiguousarray(t.transpose(0, 2, 1, 3)).reshape(N, W)
+
+
 def sz_tiled(s: np.ndarray, z: np.ndarray) -> np.ndarray:
     """(scale, zero) [N, G] -> uint32 words in [N/128][G][128] order, each word
     = bf16(s) | bf16(z) << 16."""
@@ -243,10 +260,10 @@ def build_blob(w_gate, w_up, w_down, group: int, layout: str) -> np.ndarray:
     for m, w in (("gate", w_gate), ("up", w_up), ("down", w_down)):
         q, s, z = quantize_groups(w, group)
         if layout == "int4":
-            parts = {"codes": pack_int4(q)}
+            parts = {"codes": tile_words(pack_int4(q), 16)}
         else:
             Q2, D3, D4 = split_planes(q)
-            parts = {"q2": Q2, "d3": D3, "d4": D4}
+            parts = {"q2": tile_words(Q2, 8), "d3": tile_words(D3, 4), "d4": tile_words(D4, 4)}
         parts["sz"] = sz_tiled(s, z)
         for name, arr in parts.items():
             raw = np.ascontiguousarray(arr, dtype=np.uint32).view(np.uint8).reshape(-1)

@@ -60,6 +60,16 @@ __device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
   return r;
 }
 
+// Byte offset, inside a blob's code region (INT4 codes, Q2, D3 or D4), of
+// byte b of row `row`: the region stores tiles of 16 rows x 128 K, `tb`
+// bytes per tile row (64 INT4, 32 Q2, 16 D3 / D4), row-major inside a tile,
+// the tiles of a 16-row block in K order, then the next block.  A piece of
+// at most 16 bytes starting 16-byte aligned stays inside one tile row.
+__host__ __device__ __forceinline__ size_t code_byte(size_t row, size_t b, int K, int tb) {
+  return ((row >> 4) * static_cast<size_t>(K / 128) + b / tb) * (16 * static_cast<size_t>(tb)) + (row & 15) * tb +
+         b % tb;
+}
+
 // Order-preserving unsigned key of an fp32 value (a > b gives key(a) >
 // key(b); -0 sorts below +0); NaN gets 0, below every other key.
 __device__ __forceinline__ uint32_t order_key(float v) {

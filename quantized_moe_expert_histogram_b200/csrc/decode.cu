@@ -245,15 +245,18 @@ __global__ void __launch_bounds__(W * 32, NB == 1 && W == 8 ? 3 : 2) k_dec(const
   // ---- copy side: this warp's stream of stages, unit by unit.  Per
   // fragment: INT4 16 rows x 64 B of codes; planes 16 rows x (32 B Q2 + 16 B
   // D3 + 16 B D4); then 16 rows x 1 or 2 groups of (scale, zero) words,
-  // contiguous.  A lane copies 16 bytes at ring offset lane * 16 (piece 0)
-  // and 512 + lane * 16 (piece 1) of each fragment: the codes of rows
-  // lane / 4 and 8 + lane / 4 (INT4), or Q2 of row lane / 2 and D3 (lanes
-  // below 16) / D4 of row lane % 16 (planes; a null base: plane not needed),
-  // and a scale/zero piece (lanes below 4, or 8 for groups of 64).  Fragment
-  // f's sources are fragment 0's plus f times a fixed stride (the up matrix,
-  // or 16 rows further), so the stream keeps one base per kind of piece.
-  constexpr int kStep0 = PLANES ? 32 : 64;  // piece 0 advance per stage: codes, or Q2
-  constexpr int kStep1 = 16;                // planes' piece 1: D3 / D4
+  // contiguous.  The blob stores code words in tiles of 16 rows x 128 K, so a
+  // fragment's stage is one contiguous tile of each kind (1 KB of INT4
+  // codes; 512 B of Q2, 256 B of D3, of D4).  A lane copies 16 bytes at ring
+  // offset lane * 16 (piece 0) and 512 + lane * 16 (piece 1) of each
+  // fragment: bytes lane * 16 and 512 + lane * 16 of the INT4 tile, or of the
+  // Q2 tile and of the D3 (lanes below 16) / D4 tile (planes; a null base:
+  // plane not needed), and a scale/zero piece (lanes below 4, or 8 for groups
+  // of 64).  Fragment f's sources are fragment 0's plus f times a fixed
+  // stride (the up matrix, or the next 16-row block), so the stream keeps one
+  // base per kind of piece.
+  constexpr int kStep0 = PLANES ? 512 : 1024;  // piece 0 advance per stage: the next tile of codes, or Q2
+  constexpr int kStep1 = 256;                  // planes' piece 1: D3 / D4
   const int sz_step = (kStageK / P.group) * 512;
   const size_t fs_c = GU ? P.code_off[1] - P.code_off[0] : static_cast<size_t>(PLANES ? 4 : 8) * P.K;
   const size_t fs_d = GU ? P.d3_off[1] - P.d3_off[0] : 2 * static_cast<size_t>(P.K);
@@ -271,14 +274,11 @@ __global__ void __launch_bounds__(W * 32, NB == 1 && W == 8 ? 3 : 2) k_dec(const
     const BinEnt be = ent[e];
     const uint8_t* blob = P.blobs + static_cast<size_t>(be.slot) * P.blob_bytes;
     const int n0 = rb * rows_per_unit;
-    if (!PLANES) {
-      cp = blob + P.code_off[0] + static_cast<size_t>(n0 + (lane >> 2)) * (P.K / 2) + (lane & 3) * 16 + warp * kStep0;
-    } else {
-      cp = blob + P.code_off[0] + static_cast<size_t>(n0 + (lane >> 1)) * (P.K / 4) + (lane & 1) * 16 + warp * kStep0;
+    const size_t tile = static_cast<size_t>(n0 >> 4) * (P.K / kStageK) + warp;  // (16-row block, first stage)
+    cp = blob + P.code_off[0] + tile * kStep0 + lane * 16;
+    if (PLANES) {
       const bool want = lane < 16 ? be.bits >= 3 : be.bits >= 4;
-      dp = want ? blob + (lane < 16 ? P.d3_off[0] : P.d4_off[0]) + static_cast<size_t>(n0 + (lane & 15)) * (P.K / 8) +
-                      warp * kStep1
-                : nullptr;
+      dp = want ? blob + (lane < 16 ? P.d3_off[0] : P.d4_off[0]) + tile * kStep1 + (lane & 15) * 16 : nullptr;
     }
     szp = blob + P.sz_off[0] + (static_cast<size_t>(n0 >> 7) * G + ((lane >> 2) & 1)) * 512 + (n0 & 127) * 4 +
           (lane & 3) * 16 + warp * sz_step;
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(W * 32, NB == 1 && W == 8 ? 3 : 2) k_dec(const
       for (int f = 0; f < FW; ++f) {
         const uint32_t d0 = slot + f * kFragBytes + lane * 16;
         cp_async16(d0, cp + f * fs_c);
-        if (!PLANES) cp_async16(d0 + 512, cp + f * fs_c + 4 * static_cast<size_t>(P.K));
+        if (!PLANES) cp_async16(d0 + 512, cp + f * fs_c + 512);
         else if (dp) cp_async16(d0 + 512, dp + f * fs_d);
         if (sz_lane) cp_async16(slot + sz_dst + f * kSzBytes, szp + f * fs_sz);
       }

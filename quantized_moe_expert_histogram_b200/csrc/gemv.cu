@@ -99,23 +99,19 @@ template <bool PLANES>
 __device__ __forceinline__ uint4 load_codes(const GemvParams& P, const uint8_t* blob, int m,
                                             int row, int k0, int bits) {
   if (!PLANES) {
-    const uint32_t* c = reinterpret_cast<const uint32_t*>(blob + P.code_off[m]) +
-                        static_cast<size_t>(row) * (P.K / 8) + k0 / 8;
+    const uint32_t* c = reinterpret_cast<const uint32_t*>(blob + P.code_off[m] + code_byte(row, k0 / 2, P.K, 64));
     return ldg_nc_v4(c);
   } else {
-    const uint32_t* q2 = reinterpret_cast<const uint32_t*>(blob + P.code_off[m]) +
-                         static_cast<size_t>(row) * (P.K / 16) + k0 / 16;
+    const uint32_t* q2 = reinterpret_cast<const uint32_t*>(blob + P.code_off[m] + code_byte(row, k0 / 4, P.K, 32));
     uint2 base;
     asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
                  : "=r"(base.x), "=r"(base.y)
                  : "l"(q2));
     uint32_t r3 = 0, r4 = 0;
     if (bits >= 3)
-      r3 = ldg_nc_u32(reinterpret_cast<const uint32_t*>(blob + P.d3_off[m]) +
-                      static_cast<size_t>(row) * (P.K / 32) + k0 / 32);
+      r3 = ldg_nc_u32(blob + P.d3_off[m] + code_byte(row, k0 / 8, P.K, 16));
     if (bits >= 4)
-      r4 = ldg_nc_u32(reinterpret_cast<const uint32_t*>(blob + P.d4_off[m]) +
-                      static_cast<size_t>(row) * (P.K / 32) + k0 / 32);
+      r4 = ldg_nc_u32(blob + P.d4_off[m] + code_byte(row, k0 / 8, P.K, 16));
     // plane-order code words (element 2j in nibble j, 2j+1 in nibble 4+j):
     // word wd takes the base from bits 2(wd & 1) of each nibble of Q2 word
     // wd >> 1 and the residuals from bit wd of the D3/D4 word

@@ -154,22 +154,22 @@ __device__ __forceinline__ bool piece_src(const GemvParams& P, const uint8_t* bl
   const int kv = min(kStageK, P.K - k0);  // 256, or 128 at a ragged end
   if (!PLANES) {
     if (32 * p >= kv) return false;
-    src = blob + P.code_off[m] + static_cast<size_t>(row) * (P.K / 2) + k0 / 2 + 16 * p;
+    src = blob + P.code_off[m] + code_byte(row, k0 / 2 + 16 * p, P.K, 64);
     return true;
   }
   if (p < 4) {
     if (64 * p >= kv) return false;
-    src = blob + P.code_off[m] + static_cast<size_t>(row) * (P.K / 4) + k0 / 4 + 16 * p;
+    src = blob + P.code_off[m] + code_byte(row, k0 / 4 + 16 * p, P.K, 32);
     return true;
   }
   const int q = (p - 4) & 1;
   if (128 * q >= kv) return false;
   if (p < 6) {
     if (bits < 3) return false;
-    src = blob + P.d3_off[m] + static_cast<size_t>(row) * (P.K / 8) + k0 / 8 + 16 * q;
+    src = blob + P.d3_off[m] + code_byte(row, k0 / 8 + 16 * q, P.K, 16);
   } else {
     if (bits < 4) return false;
-    src = blob + P.d4_off[m] + static_cast<size_t>(row) * (P.K / 8) + k0 / 8 + 16 * q;
+    src = blob + P.d4_off[m] + code_byte(row, k0 / 8 + 16 * q, P.K, 16);
   }
   return true;
 }

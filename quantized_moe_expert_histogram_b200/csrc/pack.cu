@@ -59,20 +59,25 @@ __global__ void __launch_bounds__(256) k_pack(const float* __restrict__ w, int r
   }
 
   uint8_t* blob = blobs + static_cast<size_t>(e) * blob_bytes;
-  // element index inside the row of this lane's i-th value: c*G + lane + 32 i
+  // element index inside the row of this lane's i-th value: c*G + lane + 32 i.
+  // Code words are stored in tiles of 16 rows x 128 elements (`per` words a
+  // tile row): word w of row n at tile_word(n, w, per).
+  auto tile_word = [&](int w, int per) {
+    return (static_cast<size_t>(n >> 4) * (K / 128) + w / per) * (16 * per) + (n & 15) * per + w % per;
+  };
   if (!planes) {
-    uint32_t* codes = reinterpret_cast<uint32_t*>(blob + off_codes) + static_cast<size_t>(n) * (K / 8);
+    uint32_t* codes = reinterpret_cast<uint32_t*>(blob + off_codes);
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) {
       uint32_t part = q[i] << (4 * (lane & 7));
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1) part |= __shfl_xor_sync(0xffffffffu, part, o);
-      if ((lane & 7) == 0) codes[(c * G + 32 * i + lane) / 8] = part;
+      if ((lane & 7) == 0) codes[tile_word((c * G + 32 * i + lane) / 8, 16)] = part;
     }
   } else {
-    uint32_t* q2 = reinterpret_cast<uint32_t*>(blob + off_q2) + static_cast<size_t>(n) * (K / 16);
-    uint32_t* d3 = reinterpret_cast<uint32_t*>(blob + off_d3) + static_cast<size_t>(n) * (K / 32);
-    uint32_t* d4 = reinterpret_cast<uint32_t*>(blob + off_d4) + static_cast<size_t>(n) * (K / 32);
+    uint32_t* q2 = reinterpret_cast<uint32_t*>(blob + off_q2);
+    uint32_t* d3 = reinterpret_cast<uint32_t*>(blob + off_d3);
+    uint32_t* d4 = reinterpret_cast<uint32_t*>(blob + off_d4);
     // plane order: element i of a run of 8 in nibble (i >> 1) + 4 (i & 1);
     // Q2 shifts the second run of its 16 by 2 bits, D3/D4 run g of 32 by g
     const int nib = 4 * (((lane & 7) >> 1) + 4 * (lane & 1));
@@ -90,10 +95,10 @@ __global__ void __launch_bounds__(256) k_pack(const float* __restrict__ w, int r
         p3 |= __shfl_xor_sync(0xffffffffu, p3, o);
         p4 |= __shfl_xor_sync(0xffffffffu, p4, o);
       }
-      if ((lane & 15) == 0) q2[(c * G + 32 * i + lane) / 16] = part;
+      if ((lane & 15) == 0) q2[tile_word((c * G + 32 * i + lane) / 16, 8)] = part;
       if (lane == 0) {
-        d3[(c * G + 32 * i) / 32] = p3;
-        d4[(c * G + 32 * i) / 32] = p4;
+        d3[tile_word((c * G + 32 * i) / 32, 4)] = p3;
+        d4[tile_word((c * G + 32 * i) / 32, 4)] = p4;
       }
     }
   }

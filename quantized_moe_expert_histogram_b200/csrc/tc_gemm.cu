@@ -180,12 +180,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, uint32_t bar) {
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            int c4, uint32_t bar) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4}], [%5];" ::"r"(dst),
-      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      "cp.async.bulk.tensor.5d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
       : "memory");
 }
 
@@ -545,15 +545,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_tc(const __grid_constant__ 
               const int r0 = row_base(T.mb, m);
               const uint32_t cdst = smem_u32(smem + C::OFF_C + (cs * 2 + m) * C::C_BYTES);
               const CUtensorMap* cm = &P.codes[GATEUP ? m : 0];
-              if (!PLANES) {
-                tma_load_3d(cdst, cm, kc * 16, r0, T.slot, codes_full(cs));
-              } else {
-                tma_load_3d(cdst, cm, kc * 8, r0, T.slot, codes_full(cs));
-                if (T.bits >= 3)
-                  tma_load_3d(cdst + 4096, &P.d3[GATEUP ? m : 0], kc * 4, r0, T.slot, codes_full(cs));
-                if (T.bits >= 4)
-                  tma_load_3d(cdst + 6144, &P.d4[GATEUP ? m : 0], kc * 4, r0, T.slot, codes_full(cs));
-              }
+              // the blob's code tiles (16 rows x 128 K): row blocks r0/16 .. + 7 of K stage kc
+              tma_load_5d(cdst, cm, 0, 0, kc, r0 >> 4, T.slot, codes_full(cs));
+              if (PLANES && T.bits >= 3)
+                tma_load_5d(cdst + 4096, &P.d3[GATEUP ? m : 0], 0, 0, kc, r0 >> 4, T.slot, codes_full(cs));
+              if (PLANES && T.bits >= 4)
+                tma_load_5d(cdst + 6144, &P.d4[GATEUP ? m : 0], 0, 0, kc, r0 >> 4, T.slot, codes_full(cs));
               const uint8_t* src = blob + P.sz_off[GATEUP ? m : 0] +
                                    (static_cast<size_t>(r0 >> 7) * G + kc * gpc) * 512;
               bulk_load(smem_u32(smem + C::OFF_SZ + (cs * 2 + m) * C::SZ_BYTES), src, gpc * 512,
@@ -900,7 +897,7 @@ bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, 
             const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
   auto fn = get_encode();
   if (!fn) return false;
-  cuuint32_t es[3] = {1, 1, 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -939,28 +936,27 @@ moe_status_t make_params(TcParams& P, const FfnArgs& a, const __half* act, int r
   const cuuint32_t br = static_cast<cuuint32_t>(box_rows);
   for (int i = 0; i < nmat; ++i) {
     const int m = mats[i];
+    // code tiles of 16 rows x 128 K: {words of a tile row, 16 rows, K / 128
+    // tiles, N / 16 row blocks, blobs}; a box is one K tile of box_rows rows,
+    // which lands in shared memory row after row as a row-major
+    // [box_rows][words] block
+    const cuuint64_t nk = static_cast<cuuint64_t>(K / 128), nr = static_cast<cuuint64_t>(N / 16);
+    auto tiles = [&](CUtensorMap* map, size_t off, cuuint64_t words, CUtensorMapSwizzle sw) {
+      const cuuint64_t row = words * 4;
+      cuuint64_t dims[5] = {words, 16, nk, nr, static_cast<cuuint64_t>(n_blobs)};
+      cuuint64_t str[4] = {row, 16 * row, nk * 16 * row, static_cast<cuuint64_t>(a.blob_bytes)};
+      cuuint32_t box[5] = {static_cast<cuuint32_t>(words), 16, 1, br / 16, 1};
+      return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 5, a.blobs + off, dims, str, box, sw);
+    };
     if (!planes) {
-      cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 8), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_blobs)};
-      cuuint64_t str[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(a.blob_bytes)};
-      cuuint32_t box[3] = {16, br, 1};
-      if (!encode(&P.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.codes[m], dims, str, box,
-                  CU_TENSOR_MAP_SWIZZLE_64B)) {
+      if (!tiles(&P.codes[i], a.lay.codes[m], 16, CU_TENSOR_MAP_SWIZZLE_64B)) {
         set_error("tensor map (codes) could not be encoded");
         return MOE_ERR_CUDA;
       }
     } else {
-      cuuint64_t dq[3] = {static_cast<cuuint64_t>(K / 16), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_blobs)};
-      cuuint64_t sq[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(a.blob_bytes)};
-      cuuint32_t bq[3] = {8, br, 1};
-      cuuint64_t dr[3] = {static_cast<cuuint64_t>(K / 32), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_blobs)};
-      cuuint64_t sr[2] = {static_cast<cuuint64_t>(K / 8), static_cast<cuuint64_t>(a.blob_bytes)};
-      cuuint32_t bb[3] = {4, br, 1};
-      if (!encode(&P.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.q2[m], dq, sq, bq,
-                  CU_TENSOR_MAP_SWIZZLE_32B) ||
-          !encode(&P.d3[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.d3[m], dr, sr, bb,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
-          !encode(&P.d4[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, a.blobs + a.lay.d4[m], dr, sr, bb,
-                  CU_TENSOR_MAP_SWIZZLE_NONE)) {
+      if (!tiles(&P.codes[i], a.lay.q2[m], 8, CU_TENSOR_MAP_SWIZZLE_32B) ||
+          !tiles(&P.d3[i], a.lay.d3[m], 4, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+          !tiles(&P.d4[i], a.lay.d4[m], 4, CU_TENSOR_MAP_SWIZZLE_NONE)) {
         set_error("tensor map (bit planes) could not be encoded");
         return MOE_ERR_CUDA;
       }

@@ -168,12 +168,12 @@ def test_blob_layout_sizes_and_roundtrip():
             q, s, z = O.quantize_groups(w, g)
             if layout == "int4":
                 o = off[m + ".codes"]
-                words = blob[o:o + N * K // 2].view(np.uint32).reshape(N, K // 8)
+                words = O.untile_words(blob[o:o + N * K // 2].view(np.uint32), N, K // 8, 16)
                 np.testing.assert_array_equal(O.unpack_int4(words, K), q)
             else:
-                Q2 = blob[off[m + ".q2"]:off[m + ".q2"] + N * K // 4].view(np.uint32).reshape(N, K // 16)
-                D3 = blob[off[m + ".d3"]:off[m + ".d3"] + N * K // 8].view(np.uint32).reshape(N, K // 32)
-                D4 = blob[off[m + ".d4"]:off[m + ".d4"] + N * K // 8].view(np.uint32).reshape(N, K // 32)
+                Q2 = O.untile_words(blob[off[m + ".q2"]:off[m + ".q2"] + N * K // 4].view(np.uint32), N, K // 16, 8)
+                D3 = O.untile_words(blob[off[m + ".d3"]:off[m + ".d3"] + N * K // 8].view(np.uint32), N, K // 32, 4)
+                D4 = O.untile_words(blob[off[m + ".d4"]:off[m + ".d4"] + N * K // 8].view(np.uint32), N, K // 32, 4)
                 np.testing.assert_array_equal(O.join_planes(Q2, D3, D4, K), q)
             o = off[m + ".sz"]
             sz = blob[o:o + N * (K // g) * 4].view(np.uint32)
@@ -208,9 +208,33 @@ def test_planes_blob_is_laid_out_width_by_width():
         for m, w in (("gate", wg), ("up", wu), ("down", wd)):
             N, K = w.shape
             q, s, z = O.quantize_groups(w, g)
-            Q2 = part[off[m + ".q2"]:off[m + ".q2"] + N * K // 4].view(np.uint32).reshape(N, K // 16)
-            D3 = part[off[m + ".d3"]:off[m + ".d3"] + N * K // 8].view(np.uint32).reshape(N, K // 32)
-            D4 = part[off[m + ".d4"]:off[m + ".d4"] + N * K // 8].view(np.uint32).reshape(N, K // 32)
+            Q2 = O.untile_words(part[off[m + ".q2"]:off[m + ".q2"] + N * K // 4].view(np.uint32), N, K // 16, 8)
+            D3 = O.untile_words(part[off[m + ".d3"]:off[m + ".d3"] + N * K // 8].view(np.uint32), N, K // 32, 4)
+            D4 = O.untile_words(part[off[m + ".d4"]:off[m + ".d4"] + N * K // 8].view(np.uint32), N, K // 32, 4)
             np.testing.assert_array_equal(O.join_planes(Q2, D3, D4, K), (q >> (4 - b)) << (4 - b))
             o = off[m + ".sz"]
             np.testing.assert_array_equal(part[o:o + N * (K // g) * 4], blob[o:o + N * (K // g) * 4])
+
+
+def test_code_tiles_hand_positions():
+    """The blob's code words come in tiles of 16 rows x 128 elements: word w
+    of row n (K/8 words a row for INT4, 16 per tile row) sits at
+    ((n // 16) * (K / 128) + w // 16) * 256 + (n % 16) * 16 + w % 16.  Hand
+    positions for N = 32, K = 256 (two row blocks, two tiles each), and the
+    round trip."""
+    N, K = 32, 256
+    words = np.arange(N * K // 8, dtype=np.uint32).reshape(N, K // 8)  # value = n * 32 + w
+    flat = O.tile_words(words, 16)
+    assert flat[0] == 0                      # row 0, word 0
+    assert flat[15] == 15                    # row 0, word 15 (end of its first tile row)
+    assert flat[16] == 32                    # row 1, word 0
+    assert flat[255] == 15 * 32 + 15         # row 15, word 15: end of tile (block 0, run 0)
+    assert flat[256] == 16                   # row 0, word 16: tile (block 0, run 1)
+    assert flat[512] == 16 * 32              # row 16, word 0: tile (block 1, run 0)
+    assert flat[788] == 17 * 32 + 20         # row 17, word 20: ((1 * 2 + 1) * 256) + 1 * 16 + 4
+    np.testing.assert_array_equal(O.untile_words(flat, N, K // 8, 16), words)
+    q2 = np.arange(N * K // 16, dtype=np.uint32).reshape(N, K // 16)  # 8 words a tile row
+    f2 = O.tile_words(q2, 8)
+    assert f2[8] == 16 and f2[128] == 8 and f2[256] == 16 * 16
+    np.testing.assert_array_equal(O.untile_words(f2, N, K // 16, 8), q2)
+
