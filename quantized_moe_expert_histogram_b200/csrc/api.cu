@@ -413,7 +413,13 @@ moe_status_t moe_grouped_ffn_combine(const void* x_perm, const int32_t* offsets,
   moe_status_t st = moe_grouped_ffn_wq(x_perm, offsets, blobs, nullptr, T * k, T, E, d, F, group, layout,
                                        workspace, workspace_bytes, y_perm, status, stream);
   if (st != MOE_OK) return st;
-  return moe_unpermute_combine(y_perm, inv_perm, topk_w, residual, T, k, d, y, stream);
+  if (!aligned16(y_perm)) {
+    set_error("moe_grouped_ffn_combine: y_perm must be 16-byte aligned");
+    return MOE_ERR_INVALID_ARG;
+  }
+  // the FFN's second GEMM, the launch just before, writes only y_perm: the
+  // combine may read gates, inv_perm and the residual before its wait
+  return launch_combine(y_perm, inv_perm, topk_w, residual, T, k, d, y, S(stream), true);
 }
 
 moe_status_t moe_bit_gate(const void* x, const float* w_bit, const float* bias_bit, const int32_t* topk_idx,

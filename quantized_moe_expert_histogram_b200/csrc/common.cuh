@@ -471,8 +471,10 @@ moe_status_t launch_permute(const int32_t* idx, const uint8_t* bits, const void*
                             int32_t* inv_perm, void* x_perm, int32_t* status, void* workspace,
                             cudaStream_t s);
 size_t permute_workspace_bytes(int T, int k, int nbins);
+// early: the previous launch on the stream writes none of inv_perm, w and
+// residual (they may be read before the programmatic wait).
 moe_status_t launch_combine(const void* y_perm, const int32_t* inv_perm, const float* w,
-                            const void* residual, int T, int k, int d, void* y, cudaStream_t s);
+                            const void* residual, int T, int k, int d, void* y, cudaStream_t s, bool early = false);
 
 struct FfnArgs {
   const __half* x_perm;
