@@ -449,13 +449,14 @@ MOE_API void moe_slot_cache_destroy(moe_slot_cache* cache);
  * what = 0 clears it. */
 MOE_API void moe_debug_inject_fault(int what, int count);
 
-/* Test hook: 0 = choose the FFN kernel by T (up to 16 tokens the decode
- * kernel -- one 8-token block per pass, or two where bins average more
- * than 4 rows -- and the tensor-core grouped GEMM above); 1 = the decode
- * kernel with one 8-token block per pass; 2 = the tensor-core kernel
- * whenever the shape allows it; 3 = the decode kernel with two blocks;
- * 4, 5 = the earlier CUDA-core GEMV and small-batch kernels (comparison
- * only).  Process-wide. */
+/* Test hook: 0 = the default choice of FFN kernel (the rule stated at
+ * moe_grouped_ffn_wq: the decode kernel for small batches, with one
+ * 8-token block per pass, or two where T > 8 and bins average more than
+ * 6 rows, and the tensor-core grouped GEMM above); 1 = the decode kernel
+ * with one 8-token block per pass; 2 = the tensor-core kernel whenever
+ * the shape allows it; 3 = the decode kernel with two blocks; 4, 5 = the
+ * earlier CUDA-core GEMV and small-batch kernels (comparison only).
+ * Process-wide. */
 MOE_API void moe_debug_force_regime(int regime);
 
 /* Test hook: when non-NULL, the tensor-core FFN kernels record each warp
