@@ -10,10 +10,12 @@
 // logits and, with a bit gate, the 3 T*E (token, expert, width) scores of
 // every expert, so that no second round is needed once the experts are
 // chosen.  Four lanes share an item: each sums its 8-element pieces of the
-// slice (pieces 4 p + lane % 4) with fp32 FMA chains, the value and the sum
-// of the products' magnitudes, and two shuffle levels add the four lanes; a
-// warp takes eight items at a time.  The (value, magnitude) pairs go into
-// CTA 0's shared memory (distributed shared memory of the cluster).
+// slice (pieces 4 p + lane % 4) with an fp32 FMA chain, the value and the
+// sum of the products' magnitudes, and two shuffle levels add the four
+// lanes; a warp holds eight such groups.  Where a group would get four or
+// more tokens of one weight row, it takes the row and those tokens, loading
+// the row's slice once.  The (value, magnitude) pairs go into CTA 0's
+// shared memory (distributed shared memory of the cluster).
 //
 // Error bound.  A slice partial S of an item errs by at most g(m) A (m =
 // products per lane + 2 tree levels, A the exact sum of magnitudes; the
@@ -58,11 +60,23 @@ namespace {
 constexpr int kFC = 8;               // CTAs of the cluster (slices of d)
 constexpr int kFThreads = 256;       // threads of a CTA
 constexpr int kFWarps = kFThreads / 32;
+constexpr int kFMaxT = 8;                 // tokens
 constexpr int kFMaxTE = 512;              // T*E
 constexpr int kFMaxGateTE = 128;          // T*E with a bit gate (4 T*E dot products)
 constexpr int kFMaxTK = 64;               // T*k
 constexpr int kFMaxItems = kFMaxTE > 4 * kFMaxGateTE ? kFMaxTE : 4 * kFMaxGateTE;  // router + gate dot products
 constexpr int kFMaxList = kFMaxTE + 3 * kFMaxTK;
+
+// Groups of four lanes (kFWarps * 8 of them) over the weight rows of the
+// dot products: token chunks and tokens per group (front_dots32_rows).
+__host__ __device__ constexpr int front_token_chunks(int T, int n_rows) {
+  return (8 * kFWarps) / n_rows < 1 ? 1 : ((8 * kFWarps) / n_rows < T ? (8 * kFWarps) / n_rows : T);
+}
+// Row by row where a group gets at least this many tokens (OLMoE-shaped
+// layer step, row by row against item by item: 2 tokens 32.8 / 32.0 us,
+// 4 tokens 39.9 / 40.6, 8 tokens 51.3 / 54.3; nested with the bit gate, 4
+// tokens 60.0 / 60.9, 8 tokens 104.6 / 106.3).
+constexpr int kRowsMinTokens = 4;
 
 struct FrontArgs {
   const __nv_bfloat16* x;
@@ -119,8 +133,11 @@ __device__ __forceinline__ void front_rows(const FrontArgs& A, int TE, int it, c
   }
 }
 
-// fp32 slice partials of items [0, n) into CTA 0's p32 (this CTA's slice).
-__device__ __forceinline__ void front_dots32(const FrontArgs& A, int TE, int n, int k0, int dk, uint32_t dst) {
+// fp32 slice partials of items [0, n) into CTA 0's p32 (this CTA's slice),
+// item by item: a group of four lanes per item, eight items per warp at a
+// time (where every group has one token: the row-major form below would
+// only add work).
+__device__ __forceinline__ void front_dots32_items(const FrontArgs& A, int TE, int n, int k0, int dk, uint32_t dst) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, q = lane >> 2, l4 = lane & 3;
   const int pieces = dk / 32;  // 8-element pieces per lane
   for (int base = warp * 8; base < n; base += kFWarps * 8) {
@@ -164,6 +181,87 @@ __device__ __forceinline__ void front_dots32(const FrontArgs& A, int TE, int n, 
       mag += __shfl_xor_sync(0xffffffffu, mag, o);
     }
     if (live && l4 == 0) st_cluster_f32x2(dst + 8u * static_cast<uint32_t>(it), acc, mag);
+  }
+}
+
+// fp32 slice partials of every item into CTA 0's p32 (this CTA's slice),
+// row by row.  Weight rows: the router's e < E, then (bit gate) E + 3 e +
+// c; the item of (token t, row r) is t E + r for the router and
+// TE + 3 t E + (r - E) for the gate.  A group of four lanes takes one
+// weight row and its tokens t = tc, tc + tch, ... < T <= kFMaxT (tch token
+// chunks split the tokens over groups where there are fewer rows than
+// groups), so each row's slice is loaded once and reused across its
+// tokens.  Lanes of a group sum their
+// 8-element pieces (4 p + lane % 4) with fp32 FMA chains, the value and the
+// sum of the products' magnitudes; two shuffle levels add the four lanes.
+__device__ __forceinline__ void front_dots32_rows(const FrontArgs& A, int TE, int n_rows, int k0, int dk,
+                                                  uint32_t dst) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, l4 = lane & 3;
+  const int T = A.T, E = A.E;
+  const int pieces = dk / 32;  // 8-element pieces per lane
+  constexpr int kGroups = kFWarps * 8;
+  const int g = warp * 8 + (lane >> 2);
+  const int tch = front_token_chunks(T, n_rows);      // token chunks
+  const int rstride = kGroups / tch;                 // rows in flight
+  const int tc = g % tch;
+  const int rounds = (n_rows + rstride - 1) / rstride;  // uniform across the CTA
+  for (int rd = 0; rd < rounds; ++rd) {
+    const int r = g / tch + rd * rstride;
+    const bool live = g < tch * rstride && r < n_rows;
+    const float* w = live ? (r < E ? A.wr + static_cast<size_t>(r) * A.d : A.wbit + static_cast<size_t>(r - E) * A.d)
+                          : A.wr;
+    float acc[kFMaxT], mag[kFMaxT];
+#pragma unroll
+    for (int i = 0; i < kFMaxT; ++i) acc[i] = mag[i] = 0.0f;
+    for (int p0 = 0; p0 < pieces; p0 += 8) {
+      float4 wa[8], wb[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int off = k0 + ((p0 + u) * 4 + l4) * 8;
+        if (live && p0 + u < pieces) {
+          wa[u] = *reinterpret_cast<const float4*>(w + off);
+          wb[u] = *reinterpret_cast<const float4*>(w + off + 4);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kFMaxT; ++i) {
+        const int t = tc + i * tch;
+        if (!live || t >= T) continue;
+        const __nv_bfloat16* xr = A.x + static_cast<size_t>(t) * A.d;
+        uint4 xb[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (p0 + u < pieces) xb[u] = *reinterpret_cast<const uint4*>(xr + k0 + ((p0 + u) * 4 + l4) * 8);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (p0 + u < pieces) {
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb[u]);
+            const float wv[8] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w, wb[u].x, wb[u].y, wb[u].z, wb[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 f = __bfloat1622float2(b2[j]);
+              acc[i] = fmaf(f.x, wv[2 * j], acc[i]);
+              mag[i] = fmaf(fabsf(f.x), fabsf(wv[2 * j]), mag[i]);
+              acc[i] = fmaf(f.y, wv[2 * j + 1], acc[i]);
+              mag[i] = fmaf(fabsf(f.y), fabsf(wv[2 * j + 1]), mag[i]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kFMaxT; ++i) {
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+        mag[i] += __shfl_xor_sync(0xffffffffu, mag[i], o);
+      }
+      const int t = tc + i * tch;
+      if (live && t < T && l4 == 0) {
+        const int it = r < E ? t * E + r : TE + 3 * t * E + (r - E);
+        st_cluster_f32x2(dst + 8u * static_cast<uint32_t>(it), acc[i], mag[i]);
+      }
+    }
   }
 }
 
@@ -273,6 +371,7 @@ __device__ __forceinline__ void front_set_width(const FrontArgs& A, FrontSmem& S
   A.bits_out[a] = static_cast<uint8_t>(b);
 }
 
+template <bool ROWS>
 __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ FrontArgs A) {
   extern __shared__ __align__(16) uint8_t front_smem[];
   FrontSmem& S = *reinterpret_cast<FrontSmem*>(front_smem);
@@ -294,7 +393,12 @@ __global__ void __launch_bounds__(kFThreads) k_front(const __grid_constant__ Fro
   if (threadIdx.x == 0) S.n_list = 0;
   cluster_sync_start();
   // ---- 1. fp32 slice partials of every dot product
-  front_dots32(A, TE, nitems, rank * dk, dk, cluster_map_shared(S.p32, 0) + 8u * static_cast<uint32_t>(rank * nitems));
+  if (ROWS)
+    front_dots32_rows(A, TE, gate ? 4 * E : E, rank * dk, dk,
+                      cluster_map_shared(S.p32, 0) + 8u * static_cast<uint32_t>(rank * nitems));
+  else
+    front_dots32_items(A, TE, nitems, rank * dk, dk,
+                       cluster_map_shared(S.p32, 0) + 8u * static_cast<uint32_t>(rank * nitems));
   cluster_sync_publish();
   // ---- 2. decisions on the fp32 values (CTA 0)
   if (rank == 0) {
@@ -568,7 +672,7 @@ float front_gamma(int d) {
 // The smallest batches (T <= 8, T*E <= 512, d % 256 == 0: one slice of d
 // per CTA is a multiple of 32 elements, 4 lanes x 8-element pieces).
 bool route_tiny_ok(int T, int d, int E) {
-  return g_route_fused == 1 && T >= 1 && T <= 8 && T * E <= kFMaxTE && d % (32 * kFC) == 0;
+  return g_route_fused == 1 && T >= 1 && T <= kFMaxT && T * E <= kFMaxTE && d % (32 * kFC) == 0;
 }
 
 // With a bit gate, T*E <= 128 (its 3 T*E scores join the T*E logits).
@@ -587,15 +691,22 @@ moe_status_t launch_front_tiny(const void* x, const float* w_router, const float
   if (e != cudaSuccess) return cuda_check(e, "front cudaGetDevice");
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
   if (!bit || !(attr_set.load() & bit)) {
-    e = cudaFuncSetAttribute(k_front, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_front<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sizeof(FrontSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_front<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sizeof(FrontSmem)));
     if (e != cudaSuccess) return cuda_check(e, "front smem attribute");
     attr_set.fetch_or(bit);
   }
   FrontArgs A{static_cast<const __nv_bfloat16*>(x), w_router, bias, forced, w_bit, bias_bit, bits_in, T, d, E, k,
               front_gamma(d), idx, w, bits_out, counts, offsets, perm, inv_perm, static_cast<__half*>(x_perm),
               status};
-  return cuda_check(launch_cluster_pdl(k_front, kFC, dim3(kFThreads), sizeof(FrontSmem), s, A), "front cluster launch");
+  const int n_rows = w_bit ? 4 * E : E, tch = front_token_chunks(T, n_rows);
+  const bool rows = (T + tch - 1) / tch >= kRowsMinTokens;
+  return cuda_check(launch_cluster_pdl(rows ? k_front<true> : k_front<false>, kFC, dim3(kFThreads), sizeof(FrontSmem),
+                                       s, A),
+                    "front cluster launch");
 }
 
 }  // namespace moeq
