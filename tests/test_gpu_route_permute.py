@@ -173,3 +173,44 @@ def test_route_permute_gate_ties_on_open_tokens(T):
     for key in KEYS:
         assert torch.equal(out[key], sep[key]), key
     assert int(status.item()) == 0
+
+
+# (E, T, gate): weight rows (E, or 4 E with the gate) against the 64 lane groups
+# of the one-launch kernel's dot products -- one token per group (item by item),
+# several tokens per group in one or more token chunks (row by row), rows that
+# do not divide the groups, more rows than groups
+ROW_CASES = [(32, 8, False), (24, 8, False), (40, 8, False), (64, 5, False), (100, 5, False), (16, 8, False),
+             (8, 8, True), (16, 8, True), (4, 8, True), (12, 6, True)]
+
+
+@pytest.mark.parametrize("E,T,gate", ROW_CASES)
+def test_route_permute_dot_product_forms(E, T, gate):
+    """Every shape of the one-launch kernel's fp32 dot products (item by item,
+    or row by row with token chunks): ids, widths and the permutation equal
+    the separate calls' and the oracle's, gates within the gate tolerance."""
+    shape = I.custom_shape(d=256, E=E, k=2, F=256, group=64, layout="planes" if gate else "int4")
+    L = I.make_layer(shape, T, seed=60 + E + T, weights=False)
+    x, wr = L["x"].cuda(), L["w_router"].cuda()
+    bias = torch.randn(E, generator=torch.Generator().manual_seed(E)).cuda() * 0.5
+    G = I.make_bit_gate(shape, seed=61 + E, bias=True) if gate else None
+    w_bit = None if G is None else G["w_bit"].cuda()
+    bias_bit = None if G is None else G["bias_bit"].cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fused = moeq.moe_route_permute(x, wr, bias, shape.k, w_bit=w_bit, bias_bit=bias_bit, status=status)
+    sep = _separate(x, wr, bias, shape.k, w_bit=w_bit, bias_bit=bias_bit)
+    torch.cuda.synchronize()
+    for key in KEYS:
+        assert torch.equal(fused[key], sep[key]), key
+    assert int(status.item()) == 0
+    sel, gates, _ = O.route(L["x"].float().numpy(), L["w_router"].numpy(), bias.cpu().numpy(), shape.k)
+    np.testing.assert_array_equal(fused["topk_idx"].cpu().numpy(), sel)
+    np.testing.assert_allclose(fused["topk_w"].cpu().numpy(), gates, rtol=GATE_RTOL, atol=GATE_ATOL)
+    b_ref = None
+    if gate:
+        assert torch.equal(fused["bits"], sep["bits"])
+        b_ref = O.bit_gate(L["x"].float().numpy(), G["w_bit"].numpy(), G["bias_bit"].numpy(), sel)
+        np.testing.assert_array_equal(fused["bits"].cpu().numpy(), b_ref)
+    keys, mult = O.assignment_keys(sel, b_ref)
+    _, offsets, perm, _ = O.permute(keys, shape.E * (mult or 1))
+    np.testing.assert_array_equal(fused["offsets"].cpu().numpy(), offsets)
+    np.testing.assert_array_equal(fused["perm"].cpu().numpy(), perm)
