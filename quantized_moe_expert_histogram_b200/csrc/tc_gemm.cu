@@ -400,10 +400,6 @@ __device__ __forceinline__ uint4 dequant8_planes(uint32_t w, __half2 z_lo, __hal
   return make_uint4(v[0], v[1], v[2], v[3]);
 }
 
-// silu(v) = v / (1 + exp(-v)), with the exponential and reciprocal at fp32
-// hardware precision (the result is rounded to fp16 afterwards).
-__device__ __forceinline__ float silu_fast(float v) { return v * __frcp_rn(1.0f + __expf(-v)); }
-
 // GATEUP: matrix 0 = gate rows, matrix 1 = up rows of features
 // [128 mb, 128 mb + 128).  DOWN: matrix 0 = W_down rows [256 mb, +128),
 // matrix 1 = rows [256 mb + 128, +128) when they exist (d % 256 may be 128).
