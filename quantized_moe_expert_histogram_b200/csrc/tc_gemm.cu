@@ -34,9 +34,10 @@
 // 16-byte stores while the next tile's MMAs run.
 //
 // Warp roles (16 warps):
-//   warp 0      codes producer: packed codes (3-D tensor map over the blob
-//               pool, one 128-row box per 128 K per matrix) and their
-//               scale/zero words (1-D bulk copies)
+//   warp 0      codes producer: packed codes (5-D tensor maps over the
+//               blob pool's 16-row x 128-K code tiles, one box of 128 rows
+//               per 128 K per matrix) and their scale/zero words (1-D bulk
+//               copies)
 //   warp 3      activation producer: one 128-row TMA box (128B swizzle)
 //               per 64 K of the tile's fp16 activation rows
 //   warp 1      MMA issuer: the whole warp waits, one elected lane issues
