@@ -1,5 +1,6 @@
-// Decode-regime grouped expert FFN: small bins (up to 16 token rows), where
-// the layer is bound by the bytes of the routed experts' weights.
+// Decode-regime grouped expert FFN: short bins (a few token rows each; a
+// bin longer than a pass takes several passes), where the layer is bound by
+// the bytes of the routed experts' weights.
 //
 // Swap-AB tensor-core dot products (mma.sync m16n8k16, fp32 accumulate):
 // dequantised weight rows are operand A (16 rows x 16 K per instruction)
@@ -17,8 +18,8 @@
 // fit on the GPU at once); CTA b takes units b, b + grid, ...  The W warps
 // of a CTA (8, or 12 where that balances the units better) split each
 // unit's K: warp w takes the 128-K stages w, w+W, w+2W, ... of every row of
-// the unit (so a 14336-long row is all the warps' work, and at any time the
-// CTA reads a contiguous K window of each row).  Each
+// the unit (so a 14336-long row is all the warps' work; a stage of a
+// 16-row fragment is one contiguous 1 KB code tile of the blob).  Each
 // warp streams its stages with cp.async into a shared-memory ring (the bytes
 // in flight take no registers), and the stream runs on across units: the
 // next unit's first stages are in flight while the current unit's partial
