@@ -15,7 +15,8 @@ from oracle import moe_oracle as O
 
 _ORIG = {name: getattr(O, name) for name in (
     "quantize_groups", "dequant", "pack_int4", "join_planes", "router_logits", "topk_select", "gates_for",
-    "permute", "assignment_keys", "silu", "expert_ffn", "combine", "bit_gate", "tile_words")}
+    "permute", "assignment_keys", "silu", "expert_ffn", "combine", "bit_gate", "tile_words", "f32_to_bf16_bits",
+    "sz_tiled")}
 
 
 def _calls(fn):
@@ -123,6 +124,12 @@ MUTANTS = {
         [PR.test_layer_equals_dense_masked_evaluation]),
     "width ties go to the wider width": (
         "bit_gate", _bit_gate_wide_ties, [PB.test_ties_go_to_the_narrower_width]),
+    "bf16 by truncation": (
+        "f32_to_bf16_bits",
+        lambda a: (np.ascontiguousarray(a, dtype=np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16),
+        [PQ.test_bf16_rounding_hand_values]),
+    "scale and zero halves of a word swapped": (
+        "sz_tiled", lambda s, z: _ORIG["sz_tiled"](z, s), [PQ.test_blob_layout_sizes_and_roundtrip]),
     "code tiles of the wrong height": (
         "tile_words", lambda words, per: _ORIG["tile_words"](words, per * 2), [PQ.test_code_tiles_hand_positions]),
 }
